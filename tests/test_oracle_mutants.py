@@ -1,0 +1,60 @@
+"""The pins must catch plausible mistakes: each case below plants one mistake
+in a copy of the oracle's C source (on the CPU), builds it, and runs the pin
+tests against it; at least one pin has to fail."""
+import os
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+SRC = os.path.join(ROOT, "oracle", "ssmq_oracle.c")
+PINS = ["tests/test_oracle_quantizers.py", "tests/test_oracle_scans.py",
+        "tests/test_calibration.py"]
+
+MUTANTS = {
+    "m1_drop_Dx": ("if (p->D) acc += (double)p->D[c] * x;\n    if (p->z) acc *= orc_silu(orc_half_to_double(p->z[idx]));\n    if (o->y) o->y[k * L + t] = acc;",
+                   "if (0) acc += (double)p->D[c] * x;\n    if (p->z) acc *= orc_silu(orc_half_to_double(p->z[idx]));\n    if (o->y) o->y[k * L + t] = acc;"),
+    "m1_decay_sign": ("h[n] = exp(delta * (double)p->A[c * N + n]) * h[n] + delta * Bv * x;\n      acc += Cv * h[n];\n    }\n    if (p->D) acc += (double)p->D[c] * x;\n    if (p->z) acc *= orc_silu(orc_half_to_double(p->z[idx]));\n    if (o->y)",
+                      "h[n] = exp(-delta * (double)p->A[c * N + n]) * h[n] + delta * Bv * x;\n      acc += Cv * h[n];\n    }\n    if (p->D) acc += (double)p->D[c] * x;\n    if (p->z) acc *= orc_silu(orc_half_to_double(p->z[idx]));\n    if (o->y)"),
+    "m1_swap_BC": ("const double Bv = (double)p->B[bi] * (double)p->B_scale[si];\n      const double Cv = (double)p->C[bi] * (double)p->C_scale[si];\n      h[n] = exp(delta * (double)p->A[c * N + n]) * h[n] + delta * Bv * x;\n      acc += Cv * h[n];\n    }\n    if (p->D) acc += (double)p->D[c] * x;\n    if (p->z) acc *= orc_silu(orc_half_to_double(p->z[idx]));\n    if (o->y)",
+                   "const double Cv = (double)p->B[bi] * (double)p->B_scale[si];\n      const double Bv = (double)p->C[bi] * (double)p->C_scale[si];\n      h[n] = exp(delta * (double)p->A[c * N + n]) * h[n] + delta * Bv * x;\n      acc += Cv * h[n];\n    }\n    if (p->D) acc += (double)p->D[c] * x;\n    if (p->z) acc *= orc_silu(orc_half_to_double(p->z[idx]));\n    if (o->y)"),
+    "m1_group_index": ("const int64_t b = u / d, c = u % d, g = c * G / d;\n  const int64_t spg = N / p->state_group_size;\n  double* h = (double*)malloc",
+                       "const int64_t b = u / d, c = u % d, g = c % G;\n  const int64_t spg = N / p->state_group_size;\n  double* h = (double*)malloc"),
+    "quant_round_exact_quotient": ("float r = (float)((double)v / (double)step);\n  double k = nearbyint((double)r);",
+                                   "double r = (double)v / (double)step;\n  double k = nearbyint(r);"),
+    "quant_round_half_away": ("double k = nearbyint((double)r);", "double k = round((double)r);"),
+    "quant_clamp_128": ("if (k < -(double)lim) k = -(double)lim;", "if (k < -(double)lim - 1) k = -(double)lim - 1;"),
+    "softedge_le_threshold": ("if (a < thr_lo)\n      mode = ORC_MODE_SMALL;", "if (a <= thr_lo)\n      mode = ORC_MODE_SMALL;"),
+    "softedge_payload_7bit_small": ("c = (uint8_t)(0x80 | (qv & 0x3F));", "c = (uint8_t)(0x80 | (qv & 0x7F));"),
+    "softedge_ratio_swapped": ("if (mode == ORC_MODE_SMALL) f = ldexp(1.0, -r);", "if (mode == ORC_MODE_SMALL) f = ldexp(1.0, r);"),
+    "ssd_group_index": ("const int64_t b = u / H, hd = u % H, g = hd * G / H;\n  const int64_t spg = N / p->state_group_size;\n  double* h = (double*)malloc((size_t)(P * N) * sizeof(double));\n  double* Bv",
+                        "const int64_t b = u / H, hd = u % H, g = hd % G;\n  const int64_t spg = N / p->state_group_size;\n  double* h = (double*)malloc((size_t)(P * N) * sizeof(double));\n  double* Bv"),
+    "ssd_decay_after_input": ("h[pp * N + n] = dA * h[pp * N + n] + delta * Bv[n] * x;\n        acc += Cv[n] * h[pp * N + n];\n      }\n      if (p->D) acc += (double)p->D[hd] * x;\n      if (p->z) acc *= orc_silu(orc_half_to_double(p->z[xi]));\n      if (o->y) o->y[(k * L + t) * P + pp] = acc;",
+                              "h[pp * N + n] = dA * (h[pp * N + n] + delta * Bv[n] * x);\n        acc += Cv[n] * h[pp * N + n];\n      }\n      if (p->D) acc += (double)p->D[hd] * x;\n      if (p->z) acc *= orc_silu(orc_half_to_double(p->z[xi]));\n      if (o->y) o->y[(k * L + t) * P + pp] = acc;"),
+    "chunked_drop_carry_decay": ("double acc = yd + exp(S[t]) * yo;", "double acc = yd + yo;"),
+    "silu_sign": ("return z / (1.0 + exp(-z));", "return z / (1.0 + exp(z));"),
+    "softplus_dropped_log": ("return v > 0.0 ? v + log1p(exp(-v)) : log1p(exp(v));", "return v > 0.0 ? v : exp(v);"),
+    "cluster_scale_from_min": ("scales[j] = (float)(a[hi - 1].v / 127.0);", "scales[j] = (float)(a[lo].v / 127.0);"),
+    "percentile_no_interp": ("return vk + frac * (vk1 - vk);", "return vk;"),
+    "decode_drop_D": ("if (p->D) acc += (double)p->D[hd] * x;\n    if (p->z) acc *= orc_silu(orc_half_to_double(p->z[xi]));\n    if (o->y) o->y[k * P + pp] = acc;",
+                      "if (0) acc += (double)p->D[hd] * x;\n    if (p->z) acc *= orc_silu(orc_half_to_double(p->z[xi]));\n    if (o->y) o->y[k * P + pp] = acc;"),
+    "half_subnormal": ("v = ldexp((double)m, -24);", "v = ldexp((double)m, -25);"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_catch_mutant(name, tmp_path):
+    old, new = MUTANTS[name]
+    src = open(SRC).read()
+    assert src.count(old) == 1, "mutation anchor not unique / missing: " + name
+    mut = tmp_path / "mut.c"
+    mut.write_text(src.replace(old, new))
+    lib = tmp_path / "libmut.so"
+    subprocess.check_call(["gcc", "-std=c11", "-O1", "-fPIC", "-shared", "-I",
+                           os.path.join(ROOT, "oracle"), "-o", str(lib), str(mut), "-lm",
+                           "-lpthread"])
+    env = dict(os.environ, SSMQ_ORACLE_LIB=str(lib))
+    r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
+                        *PINS], cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode != 0, "pins did not catch mutant " + name
