@@ -1,0 +1,528 @@
+#!/usr/bin/env python
+"""Throughput of the W8A8 selective-scan hot path on B200.
+
+One step = one Mamba-130M-shaped W8A8 layer pass (b 8, L 2048, d 1536, N 16,
+G 1, z gate): group-quantize binary16 x (8 sorted-and-clustered channel
+groups), B and C (one scale per 4 states) with static calibrated scales, then
+the Mamba-1 selective scan.  Metric: Gtokens*ch/s = b L d / step time.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+N > 1 runs under torchrun: every rank scans its own independent layer batch
+(weak scaling, no data-path collective); only the timing is reduced (max over
+ranks).  --impl reference times the CPU oracle (double precision, all host
+cores) on a bounded sample of the same workload.
+"""
+import argparse
+import datetime
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "W8A8 scan Gtokens·ch/s and HBM GB/s (frac of roofline) on 1 B200"
+UNIT = "Gtokens·ch/s"
+WORKLOAD = "m130m"
+SMS = 148
+MUFU_PER_CLK = 16  # ex2 results per clock per SM (SFU)
+
+
+def peaks():
+    p = {"hbm_gbs": 6531.0, "bf16_tflops": 1602.0, "sm_max_mhz": 1965.0, "source": "measured"}
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            m = json.load(f)
+        p.update({k: float(m[k]) for k in ("hbm_gbs", "bf16_tflops", "sm_max_mhz") if k in m})
+        p["bf16_tflops_sustained"] = float(m.get("bf16_tflops_sustained", p["bf16_tflops"]))
+    except (OSError, ValueError, KeyError):
+        p.update({"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"})
+    return p
+
+
+def config_dict(dm):
+    return {"workload": "m130m: Mamba-130M-shaped W8A8 layer (quantize x/B/C + selective scan)",
+            "batch": dm["batch"], "seqlen": dm["seqlen"], "d_inner": dm["dim"],
+            "d_state": dm["dstate"], "ngroups": dm["ngroups"], "x_clusters": dm["x_clusters"],
+            "bc_state_group": dm["state_group_size"], "gate": "silu(z)",
+            "operands": "int8 x/B/C with fp32 scales, f16 dt/z/y, f32 state",
+            "l2": "inputs exceed L2 (f16 x, dt, z, y = 201 MB per step)"}
+
+
+# ---- clocks ------------------------------------------------------------------
+
+_REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+            0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+            0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+            0x100: "display_clock_setting"}
+
+
+class ClockSampler:
+    """Samples the SM clock and clock-event reasons with NVML in a thread."""
+
+    def __init__(self, torch_dev, period=0.01):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self.period = period
+        self.ok = False
+        try:
+            import pynvml as nv
+            nv.nvmlInit()
+            self.nv = nv
+            props = __import__("torch").cuda.get_device_properties(torch_dev)
+            bus = "%08X:%02X:%02X.0" % (getattr(props, "pci_domain_id", 0), props.pci_bus_id,
+                                        props.pci_device_id)
+            try:
+                self.h = nv.nvmlDeviceGetHandleByPciBusId(bus.encode())
+            except Exception:
+                self.h = nv.nvmlDeviceGetHandleByIndex(0)
+            self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(self.h, nv.NVML_CLOCK_SM)
+            self.reason_fn = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                getattr(nv, "nvmlDeviceGetCurrentClocksThrottleReasons")
+            self.ok = True
+        except Exception as e:  # no NVML: report that, do not fail the bench
+            self.err = str(e)
+
+    def _run(self):
+        while not self.stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                r = self.reason_fn(self.h)
+                for bit, name in _REASONS.items():
+                    if r & bit and bit != 0x1:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self.stop = threading.Event()
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self.stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": "NVML unavailable"}
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(self.samples)}
+
+
+# ---- the workload ------------------------------------------------------------
+
+class Layer:
+    """Inputs (resident in HBM), static calibration and outputs of one step."""
+
+    def __init__(self, dev, seed):
+        import torch
+
+        from quantized_state_space_b200 import calibrate, synth
+        self.dm, raw = synth.workload_inputs(WORKLOAD, seed=seed)
+        dm = self.dm
+        self.b, self.L, self.d = dm["batch"], dm["seqlen"], dm["dim"]
+        self.N, self.G, self.gs, self.k = dm["dstate"], dm["ngroups"], dm["state_group_size"], \
+            dm["x_clusters"]
+        # offline calibration (untimed)
+        grp, xs = calibrate.m1_x_clusters(raw["x"], self.k)
+        bs = calibrate.state_group_absmax_scales(raw["B"], self.G, self.N, self.gs, "gnl")
+        cs = calibrate.state_group_absmax_scales(raw["C"], self.G, self.N, self.gs, "gnl")
+        smap = calibrate.state_group_map(self.G, self.N, self.gs)
+        self.raw = raw
+        T = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+        self.host = {k: torch.from_numpy(raw[k]).pin_memory() for k in ("x", "dt", "z", "B", "C")}
+        self.x, self.dt, self.z, self.B, self.C = (T(raw[k]) for k in ("x", "dt", "z", "B", "C"))
+        self.A, self.D = T(raw["A"]), T(raw["D"])
+        self.grp, self.xs, self.bs, self.cs, self.smap = T(grp), T(xs), T(bs), T(cs), T(smap)
+        self.xq = torch.empty(self.x.shape, dtype=torch.int8, device=dev)
+        self.Bq = torch.empty(self.B.shape, dtype=torch.int8, device=dev)
+        self.Cq = torch.empty(self.C.shape, dtype=torch.int8, device=dev)
+        self.y = torch.empty(self.x.shape, dtype=torch.float16, device=dev)
+        self.hf = torch.empty((self.b, self.d, self.N), dtype=torch.float32, device=dev)
+        self.units = self.b * self.L * self.d
+        self.launches_per_step = 4
+
+    def quantize(self):
+        from quantized_state_space_b200 import api
+        b, L, d, G, N, gs = self.b, self.L, self.d, self.G, self.N, self.gs
+        api.quantize_groups(self.x, b, d, L, self.grp, self.k, scales=self.xs, out=self.xq)
+        api.quantize_groups(self.B, b, G * N, L, self.smap, G * N // gs, scales=self.bs, out=self.Bq)
+        api.quantize_groups(self.C, b, G * N, L, self.smap, G * N // gs, scales=self.cs, out=self.Cq)
+
+    def scan(self):
+        from quantized_state_space_b200 import api
+        api.selective_scan(self.xq, self.dt, self.A, self.Bq, self.Cq, self.bs, self.cs, self.gs,
+                           x_group=self.grp, x_scale=self.xs, D=self.D, z=self.z, y=self.y,
+                           h_final=self.hf)
+
+    def scan_bytes(self):
+        """Algorithmic HBM bytes of one scan launch."""
+        b, L, d, N, G = self.b, self.L, self.d, self.N, self.G
+        return (b * d * L * (1 + 2 + 2 + 2)          # x int8, dt, z, y f16
+                + 2 * b * G * N * L                  # B, C int8
+                + d * N * 4 + d * 4 + b * d * N * 4)  # A, D, h_final
+
+    def step_bytes(self):
+        b, L, d, N, G = self.b, self.L, self.d, self.N, self.G
+        return self.scan_bytes() + b * d * L * 3 + 2 * 3 * b * G * N * L
+
+
+def cuda_events(torch):
+    return torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+
+def cpu_baseline(layer, threads=None, max_units=None):
+    """The oracle, as it stands, on the host cores: quantize + scan of a
+    bounded sample of (batch, channel) rows of the same workload."""
+    from oracle import oracle as O
+    raw = layer.raw
+    b, L, d, N, G, gs, k = layer.b, layer.L, layer.d, layer.N, layer.G, layer.gs, layer.k
+    threads = threads or O.default_threads()
+    n_units = max_units or b * d
+    bb = max(1, n_units // d)
+    units = np.arange(min(n_units, b * d))
+    t0 = time.perf_counter()
+    og, oxs = O.cluster_by_absmax(O.absmax_per_mid(raw["x"], b, d, L), k)
+    smap = np.arange(G * N) // gs
+    _, obs, _ = O.quantize_groups(raw["B"], b, G * N, L, smap, G * N // gs, O.SCALE_ABSMAX)
+    _, ocs, _ = O.quantize_groups(raw["C"], b, G * N, L, smap, G * N // gs, O.SCALE_ABSMAX)
+    t_cal = time.perf_counter() - t0
+    t1 = time.perf_counter()
+    xs = raw["x"][:bb]
+    ox, _, _ = O.quantize_groups(xs, bb, d, L, og, k, O.SCALE_STATIC, oxs)
+    oB, _, _ = O.quantize_groups(raw["B"][:bb], bb, G * N, L, smap, G * N // gs, O.SCALE_STATIC, obs)
+    oC, _, _ = O.quantize_groups(raw["C"][:bb], bb, G * N, L, smap, G * N // gs, O.SCALE_STATIC, ocs)
+    O.m1_scan(ox, raw["dt"][:bb], raw["A"], oB, oC, obs, ocs, gs, x_group=og, x_scale=oxs,
+              D=raw["D"], z=raw["z"][:bb], units=units[:bb * d], threads=threads)
+    dt = time.perf_counter() - t1
+    units_done = bb * d * L
+    return {"value": units_done / dt / 1e9, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": "%d of %d batch rows (%d channel rows x L %d): static quantize of "
+                      "x/B/C + double-precision scan; calibration (%.1f s) untimed"
+                      % (bb, b, bb * d, L, t_cal),
+            "seconds": dt}
+
+
+# ---- our arm ----------------------------------------------------------------
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    from quantized_state_space_b200 import build_native
+    if rank == 0:
+        build_native.build()
+    if world > 1:
+        dist.barrier()
+    pk = peaks()
+    layer = Layer(dev, seed=rank)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        layer.quantize()
+        layer.scan()
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    K = args.steps
+    scan_ev = [cuda_events(torch) for _ in range(K)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        e0, e1 = cuda_events(torch)
+        e0.record(stream)
+        for i in range(K):
+            layer.quantize()
+            scan_ev[i][0].record(stream)
+            layer.scan()
+            scan_ev[i][1].record(stream)
+        e1.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ms = e0.elapsed_time(e1)
+    scan_ms = [a.elapsed_time(b) for a, b in scan_ev]
+    if world > 1:
+        t = torch.tensor([ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    ms_step = ms / K
+    value = world * layer.units * K / (ms / 1e3) / 1e9
+
+    # end to end through the public API from pinned host buffers
+    Ke = max(1, min(K, args.e2e_steps))
+    h2d = sum(layer.host[k].numel() * layer.host[k].element_size() for k in layer.host)
+    y_host = torch.empty(layer.y.shape, dtype=torch.float16).pin_memory()
+    d2h = y_host.numel() * 2
+    for _ in range(2):
+        for kname, dst in (("x", layer.x), ("dt", layer.dt), ("z", layer.z), ("B", layer.B),
+                           ("C", layer.C)):
+            dst.copy_(layer.host[kname], non_blocking=True)
+        step()
+        y_host.copy_(layer.y, non_blocking=True)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    a0, a1 = cuda_events(torch)
+    a0.record(stream)
+    for _ in range(Ke):
+        for kname, dst in (("x", layer.x), ("dt", layer.dt), ("z", layer.z), ("B", layer.B),
+                           ("C", layer.C)):
+            dst.copy_(layer.host[kname], non_blocking=True)
+        step()
+        y_host.copy_(layer.y, non_blocking=True)
+    a1.record(stream)
+    torch.cuda.synchronize()
+    ems = a0.elapsed_time(a1)
+    if world > 1:
+        t = torch.tensor([ems], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ems = float(t.item())
+    e2e_value = world * layer.units * Ke / (ems / 1e3) / 1e9
+
+    out = None
+    if rank == 0:
+        scan_avg_s = statistics.mean(scan_ms) / 1e3
+        clocks = clk.summary()
+        mhz_max = float(clocks.get("sm_max_mhz") or pk["sm_max_mhz"])
+        updates = layer.b * layer.L * layer.d * layer.N
+        peak_upd = SMS * MUFU_PER_CLK * mhz_max * 1e6 / 1e9
+        achieved_upd = updates / scan_avg_s / 1e9
+        scan_gbs = layer.scan_bytes() / scan_avg_s / 1e9
+        out = {
+            "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world,
+            "steps": K, "warmup": max(args.warmup, 3), "ms_per_step": round(ms_step, 5),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic (seeded numpy draws shaped like the workload; no dataset)",
+            "config": dict(config_dict(layer.dm), parallelism="dp%d (independent replicas)" % world),
+            "e2e": {"value": round(e2e_value, 3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "steps": Ke},
+            "gpu_launches": layer.launches_per_step * K,
+            "roofline": {"bound": "alu", "kernel": "m1_scan_kernel (selective scan)",
+                         "achieved": round(achieved_upd, 2), "peak": round(peak_upd, 1),
+                         "unit": "Gupdates/s", "frac": round(achieved_upd / peak_upd, 4),
+                         "traffic": None,
+                         "peak_basis": "%d SMs x %d ex2/clk (SFU) x %.0f MHz; one exp per "
+                                       "state update" % (SMS, MUFU_PER_CLK, mhz_max),
+                         "hbm_achieved_gbs": round(scan_gbs, 1), "hbm_peak_gbs": pk["hbm_gbs"],
+                         "hbm_frac": round(scan_gbs / pk["hbm_gbs"], 4),
+                         "algorithmic_bytes_per_launch": layer.scan_bytes(),
+                         "scan_ms_per_launch": round(scan_avg_s * 1e3, 5),
+                         "peaks_source": pk["source"]},
+            "step_hbm_gbs": round(layer.step_bytes() / (ms_step / 1e3) / 1e9, 1),
+            "clocks": clocks,
+        }
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        if world == 1 and not args.no_cpu_baseline:
+            try:
+                out["cpu_baseline"] = cpu_baseline(layer)
+            except Exception as e:  # report, keep the measured line
+                out["cpu_baseline"] = {"error": "%s: %s" % (type(e).__name__, e)}
+        if world == 1 and not args.no_forms:
+            out["forms"] = run_forms(dev, pk, out["clocks"].get("sm_max_mhz") or pk["sm_max_mhz"])
+        print(json.dumps(out), flush=True)
+
+
+# ---- the other forms, device-timed (information beside the headline) -------
+
+def _timed(torch, fn, reps):
+    fn()
+    torch.cuda.synchronize()
+    a, b = cuda_events(torch)
+    a.record()
+    for _ in range(reps):
+        fn()
+    b.record()
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / reps / 1e3
+
+
+def form_decode(torch, dev, pk):
+    """decode8b: 1000 chained single-token state updates (b 64, H 128, P 64,
+    N 128, G 8), int8 inputs quantized ahead of the chain."""
+    from quantized_state_space_b200 import api, calibrate, synth
+    dm, raw = synth.workload_inputs("decode8b")
+    b, H, P, N, G, gs, S, k = (dm["batch"], dm["nheads"], dm["headdim"], dm["dstate"],
+                               dm["ngroups"], dm["state_group_size"], dm["steps"], dm["x_clusters"])
+    T = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+    grp, xs = calibrate.ssd_x_clusters(raw["x"], k)
+    bs = calibrate.state_group_absmax_scales(raw["B"], G, N, gs, "gn")
+    cs = calibrate.state_group_absmax_scales(raw["C"], G, N, gs, "gn")
+    smap = T(calibrate.state_group_map(G, N, gs))
+    xq, _ = api.quantize_groups(T(raw["x"]), S * b, H * P, 1, T(grp), k, scales=T(xs))
+    Bq, _ = api.quantize_groups(T(raw["B"]), S * b, G * N, 1, smap, G * N // gs, scales=T(bs))
+    Cq, _ = api.quantize_groups(T(raw["C"]), S * b, G * N, 1, smap, G * N // gs, scales=T(cs))
+    dt, A, D, grp_t, xs_t, bs_t, cs_t = (T(raw["dt"]), T(raw["A"]), T(raw["D"]), T(grp), T(xs),
+                                        T(bs), T(cs))
+    state = T(raw["state"])
+    y = torch.empty((b, H, P), dtype=torch.float16, device=dev)
+    del raw
+
+    def chain():
+        for t in range(S):
+            api.state_update(state, xq[t], dt[t], A, Bq[t], Cq[t], bs_t, cs_t, gs, x_group=grp_t,
+                             x_scale=xs_t, D=D, y=y)
+
+    sec = _timed(torch, chain, 2) / S
+    byts = 2 * b * H * P * N * 4 + b * H * P * (1 + 2) + b * H * 2 + 2 * b * G * N
+    return {"workload": "decode8b: b 64, H 128, P 64, N 128, G 8, 1000 chained steps",
+            "value": round(b * H * P / sec / 1e9, 3), "unit": "Gtokens·ch/s",
+            "us_per_step": round(sec * 1e6, 2),
+            "roofline": {"bound": "hbm", "achieved": round(byts / sec / 1e9, 1),
+                         "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": round(byts / sec / 1e9 / pk["hbm_gbs"], 4),
+                         "algorithmic_bytes_per_launch": byts, "traffic": None},
+            "l2": "state 268 MB exceeds L2"}
+
+
+def form_softedge(torch, dev, pk, mhz):
+    """softedge: encode binary16 x to soft-edge codes, quantize B/C, scan
+    (b 16, L 8192, d 1536, N 16, z gate)."""
+    from quantized_state_space_b200 import api, calibrate, synth
+    dm, raw = synth.workload_inputs("softedge")
+    b, L, d, N, G, gs = (dm["batch"], dm["seqlen"], dm["dim"], dm["dstate"], dm["ngroups"],
+                         dm["state_group_size"])
+    T = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+    s, lo, hi = calibrate.softedge_params(raw["x"])
+    bs = calibrate.state_group_absmax_scales(raw["B"], G, N, gs, "gnl")
+    cs = calibrate.state_group_absmax_scales(raw["C"], G, N, gs, "gnl")
+    smap = T(calibrate.state_group_map(G, N, gs))
+    x, dt, z, B, C = (T(raw[k]) for k in ("x", "dt", "z", "B", "C"))
+    A, D, bs_t, cs_t = T(raw["A"]), T(raw["D"]), T(bs), T(cs)
+    del raw
+    codes = torch.empty(x.shape, dtype=torch.uint8, device=dev)
+    Bq = torch.empty(B.shape, dtype=torch.int8, device=dev)
+    Cq = torch.empty(C.shape, dtype=torch.int8, device=dev)
+    y = torch.empty(x.shape, dtype=torch.float16, device=dev)
+    hf = torch.empty((b, d, N), dtype=torch.float32, device=dev)
+
+    def enc():
+        api.softedge_encode(x, s, lo, hi, 2, out=codes)
+
+    def quant_bc():
+        api.quantize_groups(B, b, G * N, L, smap, G * N // gs, scales=bs_t, out=Bq)
+        api.quantize_groups(C, b, G * N, L, smap, G * N // gs, scales=cs_t, out=Cq)
+
+    def scan():
+        api.selective_scan(codes, dt, A, Bq, Cq, bs_t, cs_t, gs, se_scale=s, D=D, z=z, y=y,
+                           h_final=hf)
+
+    t_enc = _timed(torch, enc, 5)
+    t_bc = _timed(torch, quant_bc, 5)
+    t_scan = _timed(torch, scan, 3)
+    t = t_enc + t_bc + t_scan
+    n = b * L * d
+    enc_bytes = n * 3
+    upd = n * N
+    peak_upd = SMS * MUFU_PER_CLK * mhz * 1e6 / 1e9
+    return {"workload": "softedge: b 16, L 8192, d 1536, N 16; encode + scan",
+            "value": round(n / t / 1e9, 3), "unit": "Gtokens·ch/s",
+            "ms_per_step": round(t * 1e3, 4),
+            "encode": {"ms": round(t_enc * 1e3, 4), "bound": "hbm",
+                       "achieved": round(enc_bytes / t_enc / 1e9, 1), "peak": pk["hbm_gbs"],
+                       "unit": "GB/s", "frac": round(enc_bytes / t_enc / 1e9 / pk["hbm_gbs"], 4)},
+            "scan": {"ms": round(t_scan * 1e3, 4), "bound": "alu",
+                     "achieved": round(upd / t_scan / 1e9, 1), "peak": round(peak_upd, 1),
+                     "unit": "Gupdates/s", "frac": round(upd / t_scan / 1e9 / peak_upd, 4)}}
+
+
+def run_forms(dev, pk, mhz):
+    import torch
+    out = {}
+    for name, fn in (("decode8b", lambda: form_decode(torch, dev, pk)),
+                     ("softedge", lambda: form_softedge(torch, dev, pk, mhz))):
+        try:
+            out[name] = fn()
+        except Exception as e:  # a failing form is reported, the headline stands
+            out[name] = {"error": "%s: %s" % (type(e).__name__, e)}
+        torch.cuda.empty_cache()
+    return out
+
+
+# ---- reference arm: the CPU oracle ------------------------------------------
+
+def run_reference(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from oracle import oracle as O
+    from quantized_state_space_b200 import calibrate, synth
+
+    class Dummy:
+        pass
+
+    lay = Dummy()
+    lay.dm, lay.raw = synth.workload_inputs(WORKLOAD, seed=0)
+    dm = lay.dm
+    lay.b, lay.L, lay.d, lay.N, lay.G, lay.gs, lay.k = (dm["batch"], dm["seqlen"], dm["dim"],
+                                                       dm["dstate"], dm["ngroups"],
+                                                       dm["state_group_size"], dm["x_clusters"])
+    threads = O.default_threads()
+    # each step: one batch row (d x L channel rows), sized for a few minutes total
+    per = []
+    for i in range(max(args.warmup, 3) + args.steps):
+        r = cpu_baseline(lay, threads=threads, max_units=lay.d)
+        if i >= max(args.warmup, 3):
+            per.append(r["seconds"])
+    s = sum(per)
+    units = lay.d * lay.L * len(per)
+    v = units / s / 1e9
+    out = {"impl": "reference", "metric": METRIC, "value": round(v, 5), "unit": UNIT,
+           "n_gpus": world, "steps": args.steps, "warmup": max(args.warmup, 3),
+           "ms_per_step": round(1e3 * s / len(per), 3), "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+           "data": "synthetic (seeded numpy draws shaped like the workload; no dataset)",
+           "config": dict(config_dict(dm), parallelism="host cores"),
+           "cpu_baseline": {"value": round(v, 5), "unit": UNIT, "cores": threads, "kind": "oracle",
+                            "sample": "per step: 1 of %d batch rows (%d channel rows x L %d), "
+                                      "static quantize + double-precision scan" %
+                                      (lay.b, lay.d, lay.L)},
+           "e2e": {"value": round(v, 5), "unit": UNIT, "h2d_bytes_per_step": 0,
+                   "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--no-forms", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

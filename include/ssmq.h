@@ -1,0 +1,309 @@
+/*
+ * ssmq.h -- C ABI of the B200 (sm_100a) W8A8 selective state-space library.
+ *
+ * The library computes the hot path of quantized selective state-space
+ * models: the Mamba selective-SSM linear recurrence
+ *
+ *     h_t = exp(delta_t * A) (.) h_{t-1} + delta_t * B_t * x_t
+ *     y_t = C_t . h_t + D * x_t          (optionally y_t *= silu(z_t))
+ *     delta_t = softplus(dt_t + dt_bias)  (or dt_t when softplus is off)
+ *
+ * with int8 x (one fp32 scale per sorted-and-clustered channel group) and
+ * int8 B / C (one fp32 scale per block of states), an fp32 state, binary16
+ * dt / z / y.  Sources ("the pages"):
+ *   - "Quamba2: A Robust and Scalable Post-training Quantization Framework
+ *     for Selective State Space Models" (shd-paper.top card), abstract and
+ *     the method section's technical framework (steps 1-4): 8-bit inputs of
+ *     a linear recurrence, sort-and-cluster of x, per-state-group
+ *     quantization of B and C, offline rearrangement for compute invariance;
+ *     Mamba1 and Mamba2 backbones; prefill and generation stages.
+ *   - "SSDi8" (arxivdaily card), abstract: Mamba-2's structured state-space
+ *     duality (SSD) runs a recurrent and an attention mode; a persistent INT8
+ *     path; element-wise products decoupled from the matrix products.
+ *   - Quamba-SE soft-edge quantization write-up (wmrh.cn), sections 1, 2.1,
+ *     2.2, 4.1: one scale maps floats to INT8; three modes scale/4, scale,
+ *     scale*4 chosen by |v| < L, |v| > H; byte codes 0xxxxxxx / 10xxxxxx /
+ *     11xxxxxx; a range check inside a CUDA quantize/dequantize kernel.
+ *
+ * General conventions
+ *   - Every pointer argument named "device" is CUDA device memory owned by
+ *     the caller; the library never allocates, frees or retains memory and
+ *     keeps no state besides a thread-local error message.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *     default stream).  SSMQ_OK means the arguments were valid and every
+ *     kernel was launched; results are ready once the stream reaches them.
+ *   - Argument errors are returned before anything is launched.  No C++
+ *     exception crosses the ABI.  ssmq_last_error() describes the most recent
+ *     non-OK status of the calling thread.
+ *   - Device-side anomalies (non-finite inputs, out-of-range group ids in
+ *     device maps, invalid device scales) are OR-ed into the optional device
+ *     word `status` as SSMQ_DEV_* bits; the caller reads it after a
+ *     synchronisation.  Kernels never trap or assert.
+ *   - binary16 tensors are passed as uint16_t bit patterns.
+ *   - Tensors are dense, row-major, with the layouts stated per call.  Base
+ *     pointers of int8/uint8/binary16 tensors must be 16-byte aligned, fp32
+ *     tensors 16-byte aligned (SSMQ_ERR_ALIGNMENT otherwise).
+ */
+#ifndef SSMQ_H
+#define SSMQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SSMQ_OK = 0,
+  SSMQ_ERR_INVALID_ARG = 1, /* null pointer, bad size, bad enum, L > H ... */
+  SSMQ_ERR_ALIGNMENT = 2,   /* a base pointer violates the alignment rule */
+  SSMQ_ERR_UNSUPPORTED = 3, /* valid, but outside the shapes this build runs */
+  SSMQ_ERR_CUDA = 4,        /* a CUDA launch or runtime call failed */
+  SSMQ_ERR_TIMEOUT = 5,     /* reserved: a bounded device wait gave up */
+  SSMQ_ERR_NONFINITE = 6    /* reserved for host-detected non-finite scalars */
+} ssmq_status;
+
+/* bits OR-ed into the optional device status word */
+#define SSMQ_DEV_NONFINITE 1u /* a non-finite input element was met (coded 0) */
+#define SSMQ_DEV_BAD_GROUP 2u /* a device group id was out of range (coded 0) */
+#define SSMQ_DEV_BAD_SCALE 4u /* a device scale was negative / non-finite */
+
+typedef enum { SSMQ_F32 = 0, SSMQ_F16 = 1 } ssmq_dtype;
+typedef enum { SSMQ_SCALE_STATIC = 0, SSMQ_SCALE_ABSMAX = 1 } ssmq_scale_mode;
+typedef enum { SSMQ_X_INT8_GROUP = 0, SSMQ_X_SOFTEDGE = 1 } ssmq_x_format;
+
+/* ------------------------------------------------------------------------ */
+/* Symmetric int8 group quantizer                                           */
+/* ------------------------------------------------------------------------ */
+/*
+ * Passage: Quamba-SE write-up section 1 (one scale factor maps floats onto the
+ * 8-bit grid); Quamba2 abstract and method step 3 (one scale per cluster of x
+ * channels, one per block of B/C states).
+ *
+ *   q = clamp(round_half_even(fl32(v / s_g)), -127, 127)
+ *
+ * with fl32(v / s_g) the correctly rounded binary32 quotient (formed before
+ * the integer rounding).  `src` is viewed as an (outer, mid, inner) array:
+ * element (o, m, i) sits at (o * mid + m) * inner + i and belongs to group
+ * group_of_mid[m] in [0, n_groups).  This covers every layout of the path:
+ *   Mamba-1 x (b, d, L):       outer = b,     mid = d,     inner = L
+ *   Mamba-1 B/C (b, G, N, L):  outer = b,     mid = G * N, inner = L
+ *   Mamba-2 x (b, L, H, P):    outer = b * L, mid = H * P, inner = 1
+ *   Mamba-2 B/C (b, L, G, N):  outer = b * L, mid = G * N, inner = 1
+ *
+ * src          device, binary16 bits or fp32 (dtype), outer*mid*inner elems
+ * group_of_mid device int32[mid]
+ * mode         SSMQ_SCALE_STATIC: scales[n_groups] (device) are inputs;
+ *              SSMQ_SCALE_ABSMAX: scales[g] = fl32(max |v| in g / 127) are
+ *              computed and written first (the buffer is also used as the
+ *              reduction accumulator)
+ * q_out        device int8, same element count
+ * status       device uint32 word or NULL
+ * Non-finite elements are coded 0 and excluded from the absmax.  A zero scale
+ * codes its group as 0.  Errors: INVALID_ARG for null pointers / negative
+ * sizes / n_groups < 1 / bad enums; ALIGNMENT for unaligned bases.
+ */
+ssmq_status ssmq_quantize_groups(const void* src, ssmq_dtype dtype,
+                                 int64_t outer, int64_t mid, int64_t inner,
+                                 const int32_t* group_of_mid, int32_t n_groups,
+                                 ssmq_scale_mode mode, float* scales,
+                                 int8_t* q_out, uint32_t* status,
+                                 void* stream);
+
+/* ------------------------------------------------------------------------ */
+/* Three-mode soft-edge codec                                                */
+/* ------------------------------------------------------------------------ */
+/*
+ * Passage: Quamba-SE write-up 2.1 (small |v| < L coded at scale / 2^r,
+ * standard at scale, large |v| > H at scale * 2^r; r = 2 is the page's /4 and
+ * x4, r = 1 the shift-only variant of 4.1) and 2.2 (byte codes 0xxxxxxx
+ * standard, 10xxxxxx small, 11xxxxxx large, 6 data bits for small / large).
+ *
+ * Readings: |v| is compared (strict < L, strict > H, equality is standard);
+ * the standard payload is 7-bit two's complement clamped to +-63, the small /
+ * large payload 6-bit two's complement clamped to +-31; the quotient by the
+ * mode's step follows the quantizer's binary32 rule.  Decoding multiplies the
+ * payload by fl32(scale * 2^{-r, 0, +r}).
+ *
+ * encode: src device (binary16 bits or fp32), n elements -> codes device
+ *         uint8[n].  thr_lo <= thr_hi is required (INVALID_ARG otherwise);
+ *         0 <= log2_ratio <= 8.  Non-finite inputs -> code 0x00 and
+ *         SSMQ_DEV_NONFINITE.
+ * decode: codes device uint8[n] -> out device fp32[n].
+ */
+ssmq_status ssmq_softedge_encode(const void* src, ssmq_dtype dtype, int64_t n,
+                                 float scale, float thr_lo, float thr_hi,
+                                 int32_t log2_ratio, uint8_t* codes,
+                                 uint32_t* status, void* stream);
+ssmq_status ssmq_softedge_decode(const uint8_t* codes, int64_t n, float scale,
+                                 int32_t log2_ratio, float* out, void* stream);
+
+/* ------------------------------------------------------------------------ */
+/* Mamba-1 diagonal selective scan                                           */
+/* ------------------------------------------------------------------------ */
+/*
+ * Passage: Quamba2 abstract (W8A8 for the Mamba1 backbone: 8-bit inputs of
+ * the linear recurrence, clustered x, per-state-group B / C) and the
+ * recurrence above with A diagonal per (channel, state).
+ *
+ * Layouts (b = batch, L = seqlen, d = dim, N = dstate, G = ngroups):
+ *   x        (b, d, L)  int8 codes (x_format INT8_GROUP) or soft-edge uint8
+ *                       codes (x_format SOFTEDGE: se_scale, se_log2_ratio)
+ *   x_group  int32[d]   cluster of each channel; x_scale fp32[n_x_groups]
+ *   dt, z    (b, d, L)  binary16; z may be NULL (no gate)
+ *   dt_bias  fp32[d] or NULL;  dt_softplus 0/1
+ *   A        fp32 (d, N);  D fp32[d] or NULL
+ *   B, C     (b, G, N, L) int8; channel c reads group floor(c * G / d)
+ *   B_scale, C_scale fp32[G * N / state_group_size]: state n of group g uses
+ *            index g * (N / state_group_size) + n / state_group_size
+ *   h0       fp32 (b, d, N) or NULL (zero initial state)
+ *   y        (b, d, L) binary16 output
+ *   h_final  fp32 (b, d, N) output or NULL
+ * Supported: N in {4, 8, 16, 32, 64}; d % G == 0; any L >= 0.
+ * status: device word or NULL (SSMQ_DEV_BAD_GROUP for x_group ids out of
+ * range, which then read scale 0).
+ */
+typedef struct {
+  int64_t batch, seqlen, dim, dstate, ngroups;
+  int32_t state_group_size;
+  int32_t x_format; /* ssmq_x_format */
+  const void* x;
+  const int32_t* x_group;
+  const float* x_scale;
+  int32_t n_x_groups;
+  float se_scale;
+  int32_t se_log2_ratio;
+  const uint16_t* dt;
+  const float* dt_bias;
+  int32_t dt_softplus;
+  const float* A;
+  const float* D;
+  const uint16_t* z;
+  const int8_t* B;
+  const int8_t* C;
+  const float* B_scale;
+  const float* C_scale;
+  const float* h0;
+  uint16_t* y;
+  float* h_final;
+  uint32_t* status;
+} ssmq_scan_args;
+
+ssmq_status ssmq_selective_scan_w8(const ssmq_scan_args* args, void* stream);
+
+/* ------------------------------------------------------------------------ */
+/* Mamba-2 SSD chunked scan                                                  */
+/* ------------------------------------------------------------------------ */
+/*
+ * Passage: SSDi8 abstract (SSD combines a recurrent and an attention mode;
+ * element-wise products are kept apart from the matrix products) and Quamba2
+ * abstract (W8A8 for the Mamba2 backbone).  Scalar A per head; the sequence
+ * is processed in chunks of `chunk` steps: inside a chunk the output is the
+ * masked, decay-weighted C B^T "attention" applied to delta * x, plus the
+ * contribution of the state carried in; between chunks the state is passed
+ * on.  The result equals the sequential recurrence up to rounding.
+ *
+ * Layouts (b, L, H = nheads, P = headdim, N = dstate, G = ngroups):
+ *   x        (b, L, H, P) int8 (INT8_GROUP) or soft-edge uint8 (SOFTEDGE)
+ *   x_group  int32[H * P]; x_scale fp32[n_x_groups]
+ *   dt       (b, L, H) binary16;  dt_bias fp32[H] or NULL
+ *   A        fp32[H];  D fp32[H] or NULL
+ *   z        (b, L, H, P) binary16 or NULL
+ *   B, C     (b, L, G, N) int8; head h reads group floor(h * G / H)
+ *   B_scale, C_scale fp32[G * N / state_group_size]
+ *   h0       fp32 (b, H, P, N) or NULL
+ *   y        (b, L, H, P) binary16 output
+ *   h_final  fp32 (b, H, P, N) output or NULL
+ * workspace: device memory of at least ssmq_ssd_workspace_size(args) bytes,
+ *   256-byte aligned, caller-owned, contents need not be initialised.
+ * Supported: P == 64, N == 128, chunk in {64, 128, 256}, H % G == 0.
+ */
+typedef struct {
+  int64_t batch, seqlen, nheads, headdim, dstate, ngroups;
+  int64_t chunk;
+  int32_t state_group_size;
+  int32_t x_format;
+  const void* x;
+  const int32_t* x_group;
+  const float* x_scale;
+  int32_t n_x_groups;
+  float se_scale;
+  int32_t se_log2_ratio;
+  const uint16_t* dt;
+  const float* dt_bias;
+  int32_t dt_softplus;
+  const float* A;
+  const float* D;
+  const uint16_t* z;
+  const int8_t* B;
+  const int8_t* C;
+  const float* B_scale;
+  const float* C_scale;
+  const float* h0;
+  uint16_t* y;
+  float* h_final;
+  uint32_t* status;
+} ssmq_ssd_args;
+
+size_t ssmq_ssd_workspace_size(const ssmq_ssd_args* args);
+ssmq_status ssmq_ssd_chunk_scan_w8(const ssmq_ssd_args* args, void* workspace,
+                                   size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------ */
+/* Single-token decode state update (Mamba-2 form)                           */
+/* ------------------------------------------------------------------------ */
+/*
+ * Passage: Quamba2 abstract (generation stage; W8A8 Mamba2 backbone): one step
+ * of the recurrence on the persistent fp32 state, in place.
+ *
+ * Layouts (b, H, P, N, G):
+ *   state    fp32 (b, H, P, N), read and overwritten
+ *   x        (b, H, P) int8 (INT8_GROUP) or soft-edge uint8 (SOFTEDGE)
+ *   x_group  int32[H * P]; x_scale fp32[n_x_groups]
+ *   dt       (b, H) binary16; dt_bias fp32[H] or NULL
+ *   A fp32[H]; D fp32[H] or NULL; z (b, H, P) binary16 or NULL
+ *   B, C     (b, G, N) int8; head h reads group floor(h * G / H)
+ *   B_scale, C_scale fp32[G * N / state_group_size]
+ *   y        (b, H, P) binary16 output
+ * Supported: N in {16, 32, 64, 128}; H % G == 0.
+ */
+typedef struct {
+  int64_t batch, nheads, headdim, dstate, ngroups;
+  int32_t state_group_size;
+  int32_t x_format;
+  const void* x;
+  const int32_t* x_group;
+  const float* x_scale;
+  int32_t n_x_groups;
+  float se_scale;
+  int32_t se_log2_ratio;
+  const uint16_t* dt;
+  const float* dt_bias;
+  int32_t dt_softplus;
+  const float* A;
+  const float* D;
+  const uint16_t* z;
+  const int8_t* B;
+  const int8_t* C;
+  const float* B_scale;
+  const float* C_scale;
+  float* state;
+  uint16_t* y;
+  uint32_t* status;
+} ssmq_decode_args;
+
+ssmq_status ssmq_state_update_w8(const ssmq_decode_args* args, void* stream);
+
+/* ------------------------------------------------------------------------ */
+/* Diagnostics                                                               */
+/* ------------------------------------------------------------------------ */
+/* Thread-local, NUL-terminated description of the last non-OK status. */
+const char* ssmq_last_error(void);
+/* Library ABI version (major * 10000 + minor * 100 + patch). */
+int32_t ssmq_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SSMQ_H */

@@ -1,0 +1,185 @@
+"""ctypes binding of libssmq.so (include/ssmq.h): argument marshalling only.
+
+Every function here has the name of the C entry point it calls.  Tensor
+arguments may be torch tensors (their device pointer is passed), plain
+integer addresses, or None (NULL).  A non-OK status raises SSMQError with the
+library's message.  There is no fallback: if the shared library is missing
+the import fails.
+"""
+import ctypes as C
+import os
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libssmq.so")
+
+OK, ERR_INVALID_ARG, ERR_ALIGNMENT, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_NONFINITE = range(7)
+STATUS_NAMES = {0: "SSMQ_OK", 1: "SSMQ_ERR_INVALID_ARG", 2: "SSMQ_ERR_ALIGNMENT",
+                3: "SSMQ_ERR_UNSUPPORTED", 4: "SSMQ_ERR_CUDA", 5: "SSMQ_ERR_TIMEOUT",
+                6: "SSMQ_ERR_NONFINITE"}
+DEV_NONFINITE, DEV_BAD_GROUP, DEV_BAD_SCALE = 1, 2, 4
+F32, F16 = 0, 1
+SCALE_STATIC, SCALE_ABSMAX = 0, 1
+X_INT8_GROUP, X_SOFTEDGE = 0, 1
+
+_i64, _i32, _vp, _f32 = C.c_int64, C.c_int32, C.c_void_p, C.c_float
+
+
+class SSMQError(RuntimeError):
+    def __init__(self, status, message):
+        super().__init__("%s: %s" % (STATUS_NAMES.get(status, status), message))
+        self.status = status
+
+
+class ScanArgs(C.Structure):
+    _fields_ = [("batch", _i64), ("seqlen", _i64), ("dim", _i64), ("dstate", _i64),
+                ("ngroups", _i64), ("state_group_size", _i32), ("x_format", _i32),
+                ("x", _vp), ("x_group", _vp), ("x_scale", _vp), ("n_x_groups", _i32),
+                ("se_scale", _f32), ("se_log2_ratio", _i32), ("dt", _vp), ("dt_bias", _vp),
+                ("dt_softplus", _i32), ("A", _vp), ("D", _vp), ("z", _vp), ("B", _vp),
+                ("C", _vp), ("B_scale", _vp), ("C_scale", _vp), ("h0", _vp), ("y", _vp),
+                ("h_final", _vp), ("status", _vp)]
+
+
+class SSDArgs(C.Structure):
+    _fields_ = [("batch", _i64), ("seqlen", _i64), ("nheads", _i64), ("headdim", _i64),
+                ("dstate", _i64), ("ngroups", _i64), ("chunk", _i64),
+                ("state_group_size", _i32), ("x_format", _i32), ("x", _vp), ("x_group", _vp),
+                ("x_scale", _vp), ("n_x_groups", _i32), ("se_scale", _f32),
+                ("se_log2_ratio", _i32), ("dt", _vp), ("dt_bias", _vp), ("dt_softplus", _i32),
+                ("A", _vp), ("D", _vp), ("z", _vp), ("B", _vp), ("C", _vp), ("B_scale", _vp),
+                ("C_scale", _vp), ("h0", _vp), ("y", _vp), ("h_final", _vp), ("status", _vp)]
+
+
+class DecodeArgs(C.Structure):
+    _fields_ = [("batch", _i64), ("nheads", _i64), ("headdim", _i64), ("dstate", _i64),
+                ("ngroups", _i64), ("state_group_size", _i32), ("x_format", _i32),
+                ("x", _vp), ("x_group", _vp), ("x_scale", _vp), ("n_x_groups", _i32),
+                ("se_scale", _f32), ("se_log2_ratio", _i32), ("dt", _vp), ("dt_bias", _vp),
+                ("dt_softplus", _i32), ("A", _vp), ("D", _vp), ("z", _vp), ("B", _vp),
+                ("C", _vp), ("B_scale", _vp), ("C_scale", _vp), ("state", _vp), ("y", _vp),
+                ("status", _vp)]
+
+
+# entry point -> (restype, argtypes); every name declared in include/ssmq.h
+SIGNATURES = {
+    "ssmq_quantize_groups": (_i32, [_vp, _i32, _i64, _i64, _i64, _vp, _i32, _i32, _vp, _vp,
+                                    _vp, _vp]),
+    "ssmq_softedge_encode": (_i32, [_vp, _i32, _i64, _f32, _f32, _f32, _i32, _vp, _vp, _vp]),
+    "ssmq_softedge_decode": (_i32, [_vp, _i64, _f32, _i32, _vp, _vp]),
+    "ssmq_selective_scan_w8": (_i32, [C.POINTER(ScanArgs), _vp]),
+    "ssmq_ssd_workspace_size": (C.c_size_t, [C.POINTER(SSDArgs)]),
+    "ssmq_ssd_chunk_scan_w8": (_i32, [C.POINTER(SSDArgs), _vp, C.c_size_t, _vp]),
+    "ssmq_state_update_w8": (_i32, [C.POINTER(DecodeArgs), _vp]),
+    "ssmq_last_error": (C.c_char_p, []),
+    "ssmq_version": (_i32, []),
+}
+
+_lib = None
+
+
+def lib():
+    """Loads libssmq.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError("libssmq.so is not built; run `python -m "
+                              "quantized_state_space_b200.build_native` (or "
+                              "__graft_entry__.build())")
+        L = C.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+def ptr(t):
+    """Device address of a tensor / int / None."""
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is not None:
+        return stream if isinstance(stream, int) else stream.cuda_stream
+    import torch
+    if torch.cuda.is_available() and torch.cuda.is_initialized():
+        return torch.cuda.current_stream().cuda_stream
+    return None
+
+
+def _dtype_of(t, dtype):
+    if dtype is not None:
+        return dtype
+    import torch
+    if t.dtype == torch.float16:
+        return F16
+    if t.dtype == torch.float32:
+        return F32
+    raise TypeError("source must be float16 or float32")
+
+
+def _check(status):
+    if status != OK:
+        raise SSMQError(status, lib().ssmq_last_error().decode())
+
+
+def ssmq_last_error():
+    return lib().ssmq_last_error().decode()
+
+
+def ssmq_version():
+    return lib().ssmq_version()
+
+
+def ssmq_quantize_groups(src, outer, mid, inner, group_of_mid, n_groups, mode, scales, q_out,
+                         status=None, stream=None, dtype=None):
+    _check(lib().ssmq_quantize_groups(ptr(src), _dtype_of(src, dtype), outer, mid, inner,
+                                      ptr(group_of_mid), n_groups, mode, ptr(scales), ptr(q_out),
+                                      ptr(status), _stream(stream)))
+
+
+def ssmq_softedge_encode(src, n, scale, thr_lo, thr_hi, log2_ratio, codes, status=None,
+                         stream=None, dtype=None):
+    _check(lib().ssmq_softedge_encode(ptr(src), _dtype_of(src, dtype), n, scale, thr_lo, thr_hi,
+                                      log2_ratio, ptr(codes), ptr(status), _stream(stream)))
+
+
+def ssmq_softedge_decode(codes, n, scale, log2_ratio, out, stream=None):
+    _check(lib().ssmq_softedge_decode(ptr(codes), n, scale, log2_ratio, ptr(out),
+                                      _stream(stream)))
+
+
+def _fill(struct_cls, fields):
+    a = struct_cls()
+    names = {f[0] for f in struct_cls._fields_}
+    for k, v in fields.items():
+        if k not in names:
+            raise TypeError("unknown field %r for %s" % (k, struct_cls.__name__))
+        ftype = dict(struct_cls._fields_)[k]
+        setattr(a, k, ptr(v) if ftype is _vp else v)
+    return a
+
+
+def ssmq_selective_scan_w8(stream=None, **fields):
+    """Fields of ssmq_scan_args as keywords (tensors for pointer fields)."""
+    a = _fill(ScanArgs, fields)
+    _check(lib().ssmq_selective_scan_w8(C.byref(a), _stream(stream)))
+
+
+def ssmq_ssd_workspace_size(**fields):
+    return int(lib().ssmq_ssd_workspace_size(C.byref(_fill(SSDArgs, fields))))
+
+
+def ssmq_ssd_chunk_scan_w8(workspace=None, ws_bytes=0, stream=None, **fields):
+    a = _fill(SSDArgs, fields)
+    _check(lib().ssmq_ssd_chunk_scan_w8(C.byref(a), ptr(workspace), ws_bytes, _stream(stream)))
+
+
+def ssmq_state_update_w8(stream=None, **fields):
+    a = _fill(DecodeArgs, fields)
+    _check(lib().ssmq_state_update_w8(C.byref(a), _stream(stream)))

@@ -1,0 +1,124 @@
+"""User-facing calls on torch CUDA tensors.
+
+Each function allocates its outputs with torch (device memory and streams are
+PyTorch's job) and calls one C-ABI entry point through ``_native``; every step
+of the computation runs in the CUDA library.  Layouts and semantics are those
+of include/ssmq.h.
+"""
+import torch
+
+from . import _native as N
+
+
+def _dev_check(*ts):
+    for t in ts:
+        if t is not None and (not t.is_cuda or not t.is_contiguous()):
+            raise ValueError("tensors must be contiguous CUDA tensors")
+
+
+def quantize_groups(src, outer, mid, inner, group_of_mid, n_groups, *, scales=None,
+                    absmax=False, out=None, status=None):
+    """int8 codes of ``src`` (float16/float32) with one scale per group.
+    absmax=True computes the scales (returned); else ``scales`` are used."""
+    _dev_check(src, group_of_mid, scales)
+    q = out if out is not None else torch.empty(src.shape, dtype=torch.int8, device=src.device)
+    if absmax:
+        scales = torch.empty(n_groups, dtype=torch.float32, device=src.device)
+    N.ssmq_quantize_groups(src, outer, mid, inner, group_of_mid, n_groups,
+                           N.SCALE_ABSMAX if absmax else N.SCALE_STATIC, scales, q, status=status)
+    return q, scales
+
+
+def softedge_encode(src, scale, thr_lo, thr_hi, log2_ratio=2, *, out=None, status=None):
+    _dev_check(src)
+    codes = out if out is not None else torch.empty(src.shape, dtype=torch.uint8, device=src.device)
+    N.ssmq_softedge_encode(src, src.numel(), float(scale), float(thr_lo), float(thr_hi),
+                           log2_ratio, codes, status=status)
+    return codes
+
+
+def softedge_decode(codes, scale, log2_ratio=2, *, out=None):
+    _dev_check(codes)
+    o = out if out is not None else torch.empty(codes.shape, dtype=torch.float32,
+                                                device=codes.device)
+    N.ssmq_softedge_decode(codes, codes.numel(), float(scale), log2_ratio, o)
+    return o
+
+
+def _x_fields(x, x_group, x_scale, se_scale, se_log2_ratio):
+    if x.dtype == torch.uint8:
+        return dict(x_format=N.X_SOFTEDGE, x=x, se_scale=float(se_scale),
+                    se_log2_ratio=se_log2_ratio, n_x_groups=0)
+    return dict(x_format=N.X_INT8_GROUP, x=x, x_group=x_group, x_scale=x_scale,
+                n_x_groups=int(x_scale.numel()), se_log2_ratio=se_log2_ratio)
+
+
+def selective_scan(x, dt, A, B, C, B_scale, C_scale, state_group_size, *, x_group=None,
+                   x_scale=None, se_scale=0.0, se_log2_ratio=2, D=None, z=None, dt_bias=None,
+                   dt_softplus=True, h0=None, y=None, h_final=None, return_state=True,
+                   status=None):
+    """Mamba-1 W8A8 selective scan.  x (b, d, L) int8 or soft-edge uint8;
+    dt, z (b, d, L) float16; B, C (b, G, N, L) int8.  Returns (y, h_final)."""
+    b, d, L = x.shape
+    G, Nst = B.shape[1], B.shape[2]
+    _dev_check(x, dt, A, B, C, B_scale, C_scale, x_group, x_scale, D, z, dt_bias, h0)
+    if y is None:
+        y = torch.empty((b, d, L), dtype=torch.float16, device=x.device)
+    if h_final is None and return_state:
+        h_final = torch.empty((b, d, Nst), dtype=torch.float32, device=x.device)
+    N.ssmq_selective_scan_w8(batch=b, seqlen=L, dim=d, dstate=Nst, ngroups=G,
+                             state_group_size=state_group_size,
+                             **_x_fields(x, x_group, x_scale, se_scale, se_log2_ratio),
+                             dt=dt, dt_bias=dt_bias, dt_softplus=int(bool(dt_softplus)), A=A,
+                             D=D, z=z, B=B, C=C, B_scale=B_scale, C_scale=C_scale, h0=h0, y=y,
+                             h_final=h_final, status=status)
+    return y, h_final
+
+
+def ssd_chunk_scan(x, dt, A, B, C, B_scale, C_scale, state_group_size, *, chunk=256,
+                   x_group=None, x_scale=None, se_scale=0.0, se_log2_ratio=2, D=None, z=None,
+                   dt_bias=None, dt_softplus=True, h0=None, y=None, h_final=None,
+                   return_state=True, workspace=None, status=None):
+    """Mamba-2 SSD chunked scan.  x (b, L, H, P) int8 / soft-edge uint8;
+    dt (b, L, H) float16; B, C (b, L, G, N) int8.  Returns (y, h_final)."""
+    b, L, H, P = x.shape
+    G, Nst = B.shape[2], B.shape[3]
+    _dev_check(x, dt, A, B, C, B_scale, C_scale, x_group, x_scale, D, z, dt_bias, h0)
+    if y is None:
+        y = torch.empty((b, L, H, P), dtype=torch.float16, device=x.device)
+    if h_final is None and return_state:
+        h_final = torch.empty((b, H, P, Nst), dtype=torch.float32, device=x.device)
+    fields = dict(batch=b, seqlen=L, nheads=H, headdim=P, dstate=Nst, ngroups=G, chunk=chunk,
+                  state_group_size=state_group_size,
+                  **_x_fields(x, x_group, x_scale, se_scale, se_log2_ratio),
+                  dt=dt, dt_bias=dt_bias, dt_softplus=int(bool(dt_softplus)), A=A, D=D, z=z,
+                  B=B, C=C, B_scale=B_scale, C_scale=C_scale, h0=h0, y=y, h_final=h_final,
+                  status=status)
+    ws = N.ssmq_ssd_workspace_size(**fields)
+    if ws and workspace is None:
+        workspace = torch.empty(ws + 256, dtype=torch.uint8, device=x.device)
+    wptr = None
+    if ws:
+        base = workspace.data_ptr()
+        wptr = (base + 255) // 256 * 256
+    N.ssmq_ssd_chunk_scan_w8(workspace=wptr, ws_bytes=ws, **fields)
+    return y, h_final
+
+
+def state_update(state, x, dt, A, B, C, B_scale, C_scale, state_group_size, *, x_group=None,
+                 x_scale=None, se_scale=0.0, se_log2_ratio=2, D=None, z=None, dt_bias=None,
+                 dt_softplus=True, y=None, status=None):
+    """One decode step in place on ``state`` (b, H, P, N) fp32.  x (b, H, P);
+    dt (b, H); B, C (b, G, N).  Returns y (b, H, P) float16."""
+    b, H, P, Nst = state.shape
+    G = B.shape[1]
+    _dev_check(state, x, dt, A, B, C, B_scale, C_scale, x_group, x_scale, D, z, dt_bias)
+    if y is None:
+        y = torch.empty((b, H, P), dtype=torch.float16, device=state.device)
+    N.ssmq_state_update_w8(batch=b, nheads=H, headdim=P, dstate=Nst, ngroups=G,
+                           state_group_size=state_group_size,
+                           **_x_fields(x, x_group, x_scale, se_scale, se_log2_ratio),
+                           dt=dt, dt_bias=dt_bias, dt_softplus=int(bool(dt_softplus)), A=A, D=D,
+                           z=z, B=B, C=C, B_scale=B_scale, C_scale=C_scale, state=state, y=y,
+                           status=status)
+    return y

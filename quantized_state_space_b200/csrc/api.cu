@@ -1,0 +1,223 @@
+// extern "C" entry points: argument validation, then the launchers.
+// Validation never touches the device, so every error path here can be
+// exercised without a GPU.
+#include <stdarg.h>
+#include <stdio.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include "../../include/ssmq.h"
+#include "internal.h"
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+ssmq_status fail(ssmq_status s, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return s;
+}
+
+bool aligned16(const void* p) { return p == nullptr || (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Host-side fault injection for tests of the error path: when the
+// environment variable SSMQ_FAULT_INJECT names an entry point (or "all"),
+// that entry point reports a launch failure instead of launching.
+bool injected(const char* name) {
+  const char* v = getenv("SSMQ_FAULT_INJECT");
+  if (!v || !*v) return false;
+  return strcmp(v, "all") == 0 || strcmp(v, name) == 0;
+}
+
+ssmq_status finish(cudaError_t e, const char* name) {
+  if (e != cudaSuccess) return fail(SSMQ_ERR_CUDA, "%s: CUDA error %d (%s)", name, (int)e,
+                                    cudaGetErrorString(e));
+  return SSMQ_OK;
+}
+
+#define REQUIRE(cond, code, ...)        \
+  do {                                  \
+    if (!(cond)) return fail(code, __VA_ARGS__); \
+  } while (0)
+
+ssmq_status check_x(int32_t fmt, const void* x, const int32_t* x_group, const float* x_scale,
+                    int32_t n_x_groups, int32_t log2_ratio, const char* fn) {
+  REQUIRE(fmt == SSMQ_X_INT8_GROUP || fmt == SSMQ_X_SOFTEDGE, SSMQ_ERR_INVALID_ARG,
+          "%s: x_format %d is not an ssmq_x_format", fn, fmt);
+  REQUIRE(x != nullptr, SSMQ_ERR_INVALID_ARG, "%s: x is NULL", fn);
+  if (fmt == SSMQ_X_INT8_GROUP) {
+    REQUIRE(x_group && x_scale, SSMQ_ERR_INVALID_ARG, "%s: x_group / x_scale is NULL", fn);
+    REQUIRE(n_x_groups >= 1, SSMQ_ERR_INVALID_ARG, "%s: n_x_groups must be >= 1", fn);
+  } else {
+    REQUIRE(log2_ratio >= 0 && log2_ratio <= 8, SSMQ_ERR_INVALID_ARG,
+            "%s: se_log2_ratio must be in [0, 8]", fn);
+  }
+  return SSMQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* ssmq_last_error(void) { return g_err; }
+
+int32_t ssmq_version(void) { return 100; }
+
+ssmq_status ssmq_quantize_groups(const void* src, ssmq_dtype dtype, int64_t outer, int64_t mid,
+                                 int64_t inner, const int32_t* group_of_mid, int32_t n_groups,
+                                 ssmq_scale_mode mode, float* scales, int8_t* q_out,
+                                 uint32_t* status, void* stream) {
+  const char* fn = "ssmq_quantize_groups";
+  REQUIRE(dtype == SSMQ_F32 || dtype == SSMQ_F16, SSMQ_ERR_INVALID_ARG, "%s: bad dtype %d", fn,
+          (int)dtype);
+  REQUIRE(mode == SSMQ_SCALE_STATIC || mode == SSMQ_SCALE_ABSMAX, SSMQ_ERR_INVALID_ARG,
+          "%s: bad scale mode %d", fn, (int)mode);
+  REQUIRE(outer >= 0 && mid >= 0 && inner >= 0, SSMQ_ERR_INVALID_ARG, "%s: negative size", fn);
+  REQUIRE(n_groups >= 1, SSMQ_ERR_INVALID_ARG, "%s: n_groups must be >= 1", fn);
+  REQUIRE(scales != nullptr, SSMQ_ERR_INVALID_ARG, "%s: scales is NULL", fn);
+  const bool empty = outer == 0 || mid == 0 || inner == 0;
+  if (!empty) {
+    REQUIRE(src && q_out && group_of_mid, SSMQ_ERR_INVALID_ARG, "%s: NULL tensor", fn);
+    REQUIRE(outer <= (INT64_MAX / mid) / inner, SSMQ_ERR_INVALID_ARG, "%s: size overflow", fn);
+  }
+  REQUIRE(aligned16(src) && aligned16(q_out), SSMQ_ERR_ALIGNMENT,
+          "%s: src and q_out must be 16-byte aligned", fn);
+  if (injected(fn)) return fail(SSMQ_ERR_CUDA, "%s: injected launch failure", fn);
+  if (empty && mode == SSMQ_SCALE_STATIC) return SSMQ_OK;
+  return finish(ssmq::launch_quantize(src, dtype == SSMQ_F16, empty ? 0 : outer, mid, inner,
+                                      group_of_mid, n_groups, mode == SSMQ_SCALE_ABSMAX, scales,
+                                      q_out, status, (cudaStream_t)stream),
+                fn);
+}
+
+ssmq_status ssmq_softedge_encode(const void* src, ssmq_dtype dtype, int64_t n, float scale,
+                                 float thr_lo, float thr_hi, int32_t log2_ratio, uint8_t* codes,
+                                 uint32_t* status, void* stream) {
+  const char* fn = "ssmq_softedge_encode";
+  REQUIRE(dtype == SSMQ_F32 || dtype == SSMQ_F16, SSMQ_ERR_INVALID_ARG, "%s: bad dtype", fn);
+  REQUIRE(n >= 0, SSMQ_ERR_INVALID_ARG, "%s: negative size", fn);
+  REQUIRE(thr_lo <= thr_hi, SSMQ_ERR_INVALID_ARG,
+          "%s: thr_lo must not exceed thr_hi (got %g > %g)", fn, (double)thr_lo, (double)thr_hi);
+  REQUIRE(log2_ratio >= 0 && log2_ratio <= 8, SSMQ_ERR_INVALID_ARG,
+          "%s: log2_ratio must be in [0, 8]", fn);
+  if (n > 0) REQUIRE(src && codes, SSMQ_ERR_INVALID_ARG, "%s: NULL tensor", fn);
+  REQUIRE(aligned16(src) && aligned16(codes), SSMQ_ERR_ALIGNMENT, "%s: 16-byte alignment", fn);
+  if (injected(fn)) return fail(SSMQ_ERR_CUDA, "%s: injected launch failure", fn);
+  return finish(ssmq::launch_softedge_encode(src, dtype == SSMQ_F16, n, scale, thr_lo, thr_hi,
+                                             log2_ratio, codes, status, (cudaStream_t)stream),
+                fn);
+}
+
+ssmq_status ssmq_softedge_decode(const uint8_t* codes, int64_t n, float scale, int32_t log2_ratio,
+                                 float* out, void* stream) {
+  const char* fn = "ssmq_softedge_decode";
+  REQUIRE(n >= 0, SSMQ_ERR_INVALID_ARG, "%s: negative size", fn);
+  REQUIRE(log2_ratio >= 0 && log2_ratio <= 8, SSMQ_ERR_INVALID_ARG,
+          "%s: log2_ratio must be in [0, 8]", fn);
+  if (n > 0) REQUIRE(codes && out, SSMQ_ERR_INVALID_ARG, "%s: NULL tensor", fn);
+  REQUIRE(aligned16(codes) && aligned16(out), SSMQ_ERR_ALIGNMENT, "%s: 16-byte alignment", fn);
+  if (injected(fn)) return fail(SSMQ_ERR_CUDA, "%s: injected launch failure", fn);
+  return finish(ssmq::launch_softedge_decode(codes, n, scale, log2_ratio, out,
+                                             (cudaStream_t)stream),
+                fn);
+}
+
+ssmq_status ssmq_selective_scan_w8(const ssmq_scan_args* a, void* stream) {
+  const char* fn = "ssmq_selective_scan_w8";
+  REQUIRE(a != nullptr, SSMQ_ERR_INVALID_ARG, "%s: args is NULL", fn);
+  REQUIRE(a->batch >= 0 && a->seqlen >= 0 && a->dim >= 0, SSMQ_ERR_INVALID_ARG,
+          "%s: negative size", fn);
+  REQUIRE(a->ngroups >= 1 && a->dim % a->ngroups == 0, SSMQ_ERR_INVALID_ARG,
+          "%s: dim must be a multiple of ngroups >= 1", fn);
+  REQUIRE(a->dstate == 4 || a->dstate == 8 || a->dstate == 16 || a->dstate == 32 ||
+              a->dstate == 64,
+          SSMQ_ERR_UNSUPPORTED, "%s: dstate %lld not in {4, 8, 16, 32, 64}", fn,
+          (long long)a->dstate);
+  REQUIRE(a->state_group_size >= 1 && a->dstate % a->state_group_size == 0,
+          SSMQ_ERR_INVALID_ARG, "%s: dstate must be a multiple of state_group_size", fn);
+  if (a->batch == 0 || a->dim == 0) return SSMQ_OK;
+  REQUIRE(aligned16(a->x) && aligned16(a->dt) && aligned16(a->z) && aligned16(a->B) &&
+              aligned16(a->C) && aligned16(a->y) && aligned16(a->h0) && aligned16(a->h_final) &&
+              aligned16(a->A),
+          SSMQ_ERR_ALIGNMENT, "%s: tensors must be 16-byte aligned", fn);
+  REQUIRE(a->batch <= 65535, SSMQ_ERR_UNSUPPORTED, "%s: batch > 65535", fn);
+  if (a->seqlen > 0) {
+    // an empty sequence reads no token tensor (they may be NULL); the final
+    // state is then the initial state
+    const ssmq_status xs = check_x(a->x_format, a->x, a->x_group, a->x_scale, a->n_x_groups,
+                                   a->se_log2_ratio, fn);
+    if (xs != SSMQ_OK) return xs;
+    REQUIRE(a->dt && a->A && a->B && a->C && a->B_scale && a->C_scale && a->y,
+            SSMQ_ERR_INVALID_ARG,
+            "%s: a required tensor (dt, A, B, C, B_scale, C_scale, y) is NULL", fn);
+  }
+  if (injected(fn)) return fail(SSMQ_ERR_CUDA, "%s: injected launch failure", fn);
+  return finish(ssmq::launch_selective_scan(*a, (cudaStream_t)stream), fn);
+}
+
+size_t ssmq_ssd_workspace_size(const ssmq_ssd_args* a) {
+  if (!a) return 0;
+  return ssmq::ssd_workspace_bytes(*a);
+}
+
+ssmq_status ssmq_ssd_chunk_scan_w8(const ssmq_ssd_args* a, void* workspace, size_t ws_bytes,
+                                   void* stream) {
+  const char* fn = "ssmq_ssd_chunk_scan_w8";
+  REQUIRE(a != nullptr, SSMQ_ERR_INVALID_ARG, "%s: args is NULL", fn);
+  REQUIRE(a->batch >= 0 && a->seqlen >= 0 && a->nheads >= 0, SSMQ_ERR_INVALID_ARG,
+          "%s: negative size", fn);
+  REQUIRE(a->ngroups >= 1 && a->nheads % a->ngroups == 0, SSMQ_ERR_INVALID_ARG,
+          "%s: nheads must be a multiple of ngroups >= 1", fn);
+  REQUIRE(a->headdim == 64 && a->dstate == 128, SSMQ_ERR_UNSUPPORTED,
+          "%s: this build runs headdim 64, dstate 128", fn);
+  REQUIRE(a->chunk == 64 || a->chunk == 128 || a->chunk == 256, SSMQ_ERR_UNSUPPORTED,
+          "%s: chunk must be 64, 128 or 256", fn);
+  REQUIRE(a->state_group_size >= 1 && a->dstate % a->state_group_size == 0,
+          SSMQ_ERR_INVALID_ARG, "%s: dstate must be a multiple of state_group_size", fn);
+  if (a->batch == 0 || a->nheads == 0) return SSMQ_OK;
+  const ssmq_status xs = check_x(a->x_format, a->x, a->x_group, a->x_scale, a->n_x_groups,
+                                 a->se_log2_ratio, fn);
+  if (xs != SSMQ_OK) return xs;
+  REQUIRE(a->dt && a->A && a->B && a->C && a->B_scale && a->C_scale && a->y, SSMQ_ERR_INVALID_ARG,
+          "%s: a required tensor (dt, A, B, C, B_scale, C_scale, y) is NULL", fn);
+  REQUIRE(aligned16(a->x) && aligned16(a->dt) && aligned16(a->z) && aligned16(a->B) &&
+              aligned16(a->C) && aligned16(a->y) && aligned16(a->h0) && aligned16(a->h_final),
+          SSMQ_ERR_ALIGNMENT, "%s: tensors must be 16-byte aligned", fn);
+  const size_t need = ssmq::ssd_workspace_bytes(*a);
+  REQUIRE(need == 0 || (workspace && ws_bytes >= need), SSMQ_ERR_INVALID_ARG,
+          "%s: workspace of %zu bytes required (got %zu)", fn, need, ws_bytes);
+  REQUIRE((reinterpret_cast<uintptr_t>(workspace) & 255u) == 0, SSMQ_ERR_ALIGNMENT,
+          "%s: workspace must be 256-byte aligned", fn);
+  if (injected(fn)) return fail(SSMQ_ERR_CUDA, "%s: injected launch failure", fn);
+  return finish(ssmq::launch_ssd(*a, workspace, (cudaStream_t)stream), fn);
+}
+
+ssmq_status ssmq_state_update_w8(const ssmq_decode_args* a, void* stream) {
+  const char* fn = "ssmq_state_update_w8";
+  REQUIRE(a != nullptr, SSMQ_ERR_INVALID_ARG, "%s: args is NULL", fn);
+  REQUIRE(a->batch >= 0 && a->nheads >= 0 && a->headdim >= 0, SSMQ_ERR_INVALID_ARG,
+          "%s: negative size", fn);
+  REQUIRE(a->ngroups >= 1 && a->nheads % a->ngroups == 0, SSMQ_ERR_INVALID_ARG,
+          "%s: nheads must be a multiple of ngroups >= 1", fn);
+  REQUIRE(a->dstate == 16 || a->dstate == 32 || a->dstate == 64 || a->dstate == 128,
+          SSMQ_ERR_UNSUPPORTED, "%s: dstate %lld not in {16, 32, 64, 128}", fn,
+          (long long)a->dstate);
+  REQUIRE(a->state_group_size >= 1 && a->dstate % a->state_group_size == 0,
+          SSMQ_ERR_INVALID_ARG, "%s: dstate must be a multiple of state_group_size", fn);
+  if (a->batch == 0 || a->nheads == 0 || a->headdim == 0) return SSMQ_OK;
+  const ssmq_status xs = check_x(a->x_format, a->x, a->x_group, a->x_scale, a->n_x_groups,
+                                 a->se_log2_ratio, fn);
+  if (xs != SSMQ_OK) return xs;
+  REQUIRE(a->dt && a->A && a->B && a->C && a->B_scale && a->C_scale && a->state && a->y,
+          SSMQ_ERR_INVALID_ARG, "%s: a required tensor is NULL", fn);
+  REQUIRE(aligned16(a->state) && aligned16(a->B) && aligned16(a->C), SSMQ_ERR_ALIGNMENT,
+          "%s: state, B and C must be 16-byte aligned", fn);
+  REQUIRE(a->batch * a->nheads <= 0x7fffffff, SSMQ_ERR_UNSUPPORTED, "%s: too many heads", fn);
+  if (injected(fn)) return fail(SSMQ_ERR_CUDA, "%s: injected launch failure", fn);
+  return finish(ssmq::launch_state_update(*a, (cudaStream_t)stream), fn);
+}
+
+}  // extern "C"

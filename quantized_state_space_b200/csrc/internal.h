@@ -1,0 +1,30 @@
+// Launchers behind the C ABI.  Each returns cudaSuccess or the launch error;
+// arguments were validated by the caller (api.cu).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/ssmq.h"
+
+namespace ssmq {
+
+cudaError_t launch_quantize(const void* src, bool f16, int64_t outer, int64_t mid,
+                            int64_t inner, const int32_t* gmap, int32_t n_groups,
+                            bool absmax, float* scales, int8_t* q, uint32_t* status,
+                            cudaStream_t st);
+
+cudaError_t launch_softedge_encode(const void* src, bool f16, int64_t n, float scale,
+                                   float lo, float hi, int log2_ratio, uint8_t* codes,
+                                   uint32_t* status, cudaStream_t st);
+cudaError_t launch_softedge_decode(const uint8_t* codes, int64_t n, float scale,
+                                   int log2_ratio, float* out, cudaStream_t st);
+
+cudaError_t launch_selective_scan(const ssmq_scan_args& a, cudaStream_t st);
+
+cudaError_t launch_state_update(const ssmq_decode_args& a, cudaStream_t st);
+
+size_t ssd_workspace_bytes(const ssmq_ssd_args& a);
+cudaError_t launch_ssd(const ssmq_ssd_args& a, void* ws, cudaStream_t st);
+
+}  // namespace ssmq

@@ -1,0 +1,368 @@
+// Symmetric int8 group quantizer and the three-mode soft-edge codec.
+//
+// Quamba-SE write-up (wmrh.cn) section 1: one scale factor maps floats onto
+// the INT8 grid; sections 2.1-2.2: three modes (scale/4, scale, scale*4)
+// chosen by comparing |v| with L and H, stored as 0xxxxxxx / 10xxxxxx /
+// 11xxxxxx bytes.  Quamba2 abstract: one scale per cluster of x channels and
+// per block of B/C states.
+//
+// All kernels stream 16 elements per thread per iteration (16-byte stores of
+// codes, 16- or 64-byte loads of binary16 / fp32 inputs) over a grid-stride
+// loop sized to the SM count; they are HBM-bound.
+#include "common.cuh"
+#include "internal.h"
+
+namespace ssmq {
+namespace {
+
+constexpr int kVec = 16;
+constexpr int kThreads = 256;
+constexpr int kMaxBlocks = 148 * 16;
+enum { kPathRow = 0, kPathCol = 1, kPathGen = 2 };
+
+template <bool kF16, typename Idx>
+__device__ __forceinline__ void load16(const void* src, Idx e0, float (&v)[kVec]) {
+  if (kF16) {
+    const uint4* p = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(src) + e0);
+    const uint4 a = __ldg(p), b = __ldg(p + 1);
+    const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[i]));
+      v[2 * i] = f.x;
+      v[2 * i + 1] = f.y;
+    }
+  } else {
+    const float4* p = reinterpret_cast<const float4*>(static_cast<const float*>(src) + e0);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float4 f = __ldg(p + i);
+      v[4 * i] = f.x;
+      v[4 * i + 1] = f.y;
+      v[4 * i + 2] = f.z;
+      v[4 * i + 3] = f.w;
+    }
+  }
+}
+
+template <bool kF16, typename Idx>
+__device__ __forceinline__ float load1(const void* src, Idx e) {
+  if (kF16) return h2f(static_cast<const uint16_t*>(src)[e]);
+  return static_cast<const float*>(src)[e];
+}
+
+// One element of the static quantizer; flags record device-side anomalies.
+__device__ __forceinline__ int quant_elem(float v, float s, bool okg, uint32_t& flags) {
+  if (!okg) {
+    flags |= SSMQ_DEV_BAD_GROUP;
+    return 0;
+  }
+  if (!isfinite(v)) {
+    flags |= SSMQ_DEV_NONFINITE;
+    return 0;
+  }
+  if (!(s > 0.0f) || !isfinite(s)) {
+    if (s != 0.0f) flags |= SSMQ_DEV_BAD_SCALE;
+    return 0;
+  }
+  return quant_rne(v, s, 127);
+}
+
+__device__ __forceinline__ uint32_t pack4(int a, int b, int c, int d) {
+  return (uint32_t)(a & 0xFF) | ((uint32_t)(b & 0xFF) << 8) | ((uint32_t)(c & 0xFF) << 16) |
+         ((uint32_t)(d & 0xFF) << 24);
+}
+
+template <bool kF16, int kPath, typename Idx>
+__global__ void __launch_bounds__(kThreads)
+    quant_static_kernel(const void* __restrict__ src, Idx n, Idx mid, Idx inner,
+                        const int32_t* __restrict__ gmap, int32_t n_groups,
+                        const float* __restrict__ scales, int8_t* __restrict__ q,
+                        uint32_t* status) {
+  uint32_t flags = 0;
+  const Idx nvec = (n + kVec - 1) / kVec;
+  for (Idx v = (Idx)blockIdx.x * kThreads + threadIdx.x; v < nvec; v += (Idx)gridDim.x * kThreads) {
+    const Idx e0 = v * kVec;
+    if (e0 + kVec <= n) {
+      float x[kVec];
+      load16<kF16>(src, e0, x);
+      int r[kVec];
+      if (kPath == kPathRow) {
+        const int g = __ldg(gmap + (e0 / inner) % mid);
+        const bool okg = (unsigned)g < (unsigned)n_groups;
+        const float s = okg ? __ldg(scales + g) : 0.0f;
+#pragma unroll
+        for (int i = 0; i < kVec; ++i) r[i] = quant_elem(x[i], s, okg, flags);
+      } else if (kPath == kPathCol) {
+        const Idx m0 = e0 % mid;
+#pragma unroll
+        for (int i = 0; i < kVec; ++i) {
+          const int g = __ldg(gmap + m0 + i);
+          const bool okg = (unsigned)g < (unsigned)n_groups;
+          r[i] = quant_elem(x[i], okg ? __ldg(scales + g) : 0.0f, okg, flags);
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < kVec; ++i) {
+          const int g = __ldg(gmap + ((e0 + i) / inner) % mid);
+          const bool okg = (unsigned)g < (unsigned)n_groups;
+          r[i] = quant_elem(x[i], okg ? __ldg(scales + g) : 0.0f, okg, flags);
+        }
+      }
+      uint4 o;
+      o.x = pack4(r[0], r[1], r[2], r[3]);
+      o.y = pack4(r[4], r[5], r[6], r[7]);
+      o.z = pack4(r[8], r[9], r[10], r[11]);
+      o.w = pack4(r[12], r[13], r[14], r[15]);
+      *reinterpret_cast<uint4*>(q + e0) = o;
+    } else {
+      for (Idx e = e0; e < n; ++e) {
+        const int g = __ldg(gmap + (e / inner) % mid);
+        const bool okg = (unsigned)g < (unsigned)n_groups;
+        q[e] = (int8_t)quant_elem(load1<kF16>(src, e), okg ? __ldg(scales + g) : 0.0f, okg, flags);
+      }
+    }
+  }
+  flag_status(status, flags);
+}
+
+// Per-group max |v| into `acc` (the scales buffer viewed as uint32 bit
+// patterns: for non-negative floats the unsigned order is the float order).
+template <bool kF16, int kPath, typename Idx>
+__global__ void __launch_bounds__(kThreads)
+    absmax_kernel(const void* __restrict__ src, Idx n, Idx mid, Idx inner,
+                  const int32_t* __restrict__ gmap, int32_t n_groups, unsigned* acc,
+                  uint32_t* status, int use_smem) {
+  extern __shared__ unsigned s_acc[];
+  if (use_smem) {
+    for (int i = threadIdx.x; i < n_groups; i += kThreads) s_acc[i] = 0u;
+    __syncthreads();
+  }
+  unsigned* tgt = use_smem ? s_acc : acc;
+  uint32_t flags = 0;
+  int cur_g = -1;
+  unsigned cur_m = 0u;
+  auto push = [&](int g, float v) {
+    if ((unsigned)g >= (unsigned)n_groups) {
+      flags |= SSMQ_DEV_BAD_GROUP;
+      return;
+    }
+    if (!isfinite(v)) {
+      flags |= SSMQ_DEV_NONFINITE;
+      return;
+    }
+    const unsigned a = __float_as_uint(fabsf(v));
+    if (g != cur_g) {
+      if (cur_g >= 0 && cur_m) atomicMax(tgt + cur_g, cur_m);
+      cur_g = g;
+      cur_m = a;
+    } else {
+      cur_m = max(cur_m, a);
+    }
+  };
+  const Idx nvec = (n + kVec - 1) / kVec;
+  for (Idx v = (Idx)blockIdx.x * kThreads + threadIdx.x; v < nvec; v += (Idx)gridDim.x * kThreads) {
+    const Idx e0 = v * kVec;
+    if (e0 + kVec <= n) {
+      float x[kVec];
+      load16<kF16>(src, e0, x);
+      if (kPath == kPathRow) {
+        const int g = __ldg(gmap + (e0 / inner) % mid);
+#pragma unroll
+        for (int i = 0; i < kVec; ++i) push(g, x[i]);
+      } else if (kPath == kPathCol) {
+        const Idx m0 = e0 % mid;
+#pragma unroll
+        for (int i = 0; i < kVec; ++i) push(__ldg(gmap + m0 + i), x[i]);
+      } else {
+#pragma unroll
+        for (int i = 0; i < kVec; ++i) push(__ldg(gmap + ((e0 + i) / inner) % mid), x[i]);
+      }
+    } else {
+      for (Idx e = e0; e < n; ++e) push(__ldg(gmap + (e / inner) % mid), load1<kF16>(src, e));
+    }
+  }
+  if (cur_g >= 0 && cur_m) atomicMax(tgt + cur_g, cur_m);
+  if (use_smem) {
+    __syncthreads();
+    for (int i = threadIdx.x; i < n_groups; i += kThreads)
+      if (s_acc[i]) atomicMax(acc + i, s_acc[i]);
+  }
+  flag_status(status, flags);
+}
+
+// scale_g = fl32(absmax_g / 127), in place over the accumulator.
+__global__ void absmax_finalize_kernel(float* scales, int32_t n_groups) {
+  const int g = blockIdx.x * blockDim.x + threadIdx.x;
+  if (g < n_groups) {
+    const unsigned bits = reinterpret_cast<unsigned*>(scales)[g];
+    scales[g] = __fdiv_rn(__uint_as_float(bits), 127.0f);
+  }
+}
+
+template <typename Idx>
+unsigned grid_for(Idx n) {
+  const uint64_t nvec = ((uint64_t)n + kVec - 1) / kVec;
+  uint64_t b = (nvec + kThreads - 1) / kThreads;
+  if (b > (uint64_t)kMaxBlocks) b = kMaxBlocks;
+  return (unsigned)(b ? b : 1);
+}
+
+template <bool kF16, int kPath, typename Idx>
+cudaError_t quantize_t(const void* src, Idx n, Idx mid, Idx inner, const int32_t* gmap,
+                       int32_t n_groups, bool absmax, float* scales, int8_t* q,
+                       uint32_t* status, cudaStream_t st) {
+  const unsigned grid = grid_for(n);
+  if (absmax) {
+    cudaError_t e = cudaMemsetAsync(scales, 0, sizeof(float) * (size_t)n_groups, st);
+    if (e != cudaSuccess) return e;
+    const int use_smem = n_groups <= 8192;
+    if (n > 0)
+      absmax_kernel<kF16, kPath, Idx><<<grid, kThreads, use_smem ? n_groups * sizeof(unsigned) : 0,
+                                        st>>>(src, n, mid, inner, gmap, n_groups,
+                                              reinterpret_cast<unsigned*>(scales), status,
+                                              use_smem);
+    absmax_finalize_kernel<<<(n_groups + 255) / 256, 256, 0, st>>>(scales, n_groups);
+  }
+  if (n > 0)
+    quant_static_kernel<kF16, kPath, Idx>
+        <<<grid, kThreads, 0, st>>>(src, n, mid, inner, gmap, n_groups, scales, q, status);
+  return cudaGetLastError();
+}
+
+template <bool kF16, typename Idx>
+cudaError_t quantize_p(const void* src, Idx n, Idx mid, Idx inner, const int32_t* gmap,
+                       int32_t n_groups, bool absmax, float* scales, int8_t* q,
+                       uint32_t* status, cudaStream_t st) {
+  if (inner % kVec == 0)
+    return quantize_t<kF16, kPathRow, Idx>(src, n, mid, inner, gmap, n_groups, absmax, scales, q,
+                                           status, st);
+  if (inner == 1 && mid % kVec == 0)
+    return quantize_t<kF16, kPathCol, Idx>(src, n, mid, inner, gmap, n_groups, absmax, scales, q,
+                                           status, st);
+  return quantize_t<kF16, kPathGen, Idx>(src, n, mid, inner, gmap, n_groups, absmax, scales, q,
+                                         status, st);
+}
+
+// ---- soft-edge ---------------------------------------------------------------
+
+__device__ __forceinline__ uint32_t se_encode1(float v, float lo, float hi, const SeSteps& st,
+                                               uint32_t& flags) {
+  if (!isfinite(v)) {
+    flags |= SSMQ_DEV_NONFINITE;
+    return 0u;
+  }
+  const float a = fabsf(v);
+  const int mode = a < lo ? 1 : (a > hi ? 2 : 0);
+  const float step = st.s[mode];
+  const int lim = mode == 0 ? 63 : 31;
+  const int qv = (step > 0.0f && isfinite(step)) ? quant_rne(v, step, lim) : 0;
+  if (mode == 0) return (uint32_t)(qv & 0x7F);
+  return (mode == 1 ? 0x80u : 0xC0u) | (uint32_t)(qv & 0x3F);
+}
+
+template <bool kF16, typename Idx>
+__global__ void __launch_bounds__(kThreads)
+    se_encode_kernel(const void* __restrict__ src, Idx n, float lo, float hi, SeSteps st,
+                     uint8_t* __restrict__ codes, uint32_t* status) {
+  uint32_t flags = 0;
+  const Idx nvec = (n + kVec - 1) / kVec;
+  for (Idx v = (Idx)blockIdx.x * kThreads + threadIdx.x; v < nvec; v += (Idx)gridDim.x * kThreads) {
+    const Idx e0 = v * kVec;
+    if (e0 + kVec <= n) {
+      float x[kVec];
+      load16<kF16>(src, e0, x);
+      uint32_t w[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        w[k] = se_encode1(x[4 * k], lo, hi, st, flags) |
+               (se_encode1(x[4 * k + 1], lo, hi, st, flags) << 8) |
+               (se_encode1(x[4 * k + 2], lo, hi, st, flags) << 16) |
+               (se_encode1(x[4 * k + 3], lo, hi, st, flags) << 24);
+      *reinterpret_cast<uint4*>(codes + e0) = make_uint4(w[0], w[1], w[2], w[3]);
+    } else {
+      for (Idx e = e0; e < n; ++e) codes[e] = (uint8_t)se_encode1(load1<kF16>(src, e), lo, hi, st, flags);
+    }
+  }
+  flag_status(status, flags);
+}
+
+template <typename Idx>
+__global__ void __launch_bounds__(kThreads)
+    se_decode_kernel(const uint8_t* __restrict__ codes, Idx n, SeSteps st, float* __restrict__ out) {
+  const Idx nvec = (n + kVec - 1) / kVec;
+  for (Idx v = (Idx)blockIdx.x * kThreads + threadIdx.x; v < nvec; v += (Idx)gridDim.x * kThreads) {
+    const Idx e0 = v * kVec;
+    if (e0 + kVec <= n) {
+      const uint4 u = __ldg(reinterpret_cast<const uint4*>(codes + e0));
+      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+      float4* o = reinterpret_cast<float4*>(out + e0);
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        o[k] = make_float4(se_decode(w[k] & 0xFFu, st), se_decode((w[k] >> 8) & 0xFFu, st),
+                           se_decode((w[k] >> 16) & 0xFFu, st), se_decode(w[k] >> 24, st));
+    } else {
+      for (Idx e = e0; e < n; ++e) out[e] = se_decode(codes[e], st);
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_quantize(const void* src, bool f16, int64_t outer, int64_t mid, int64_t inner,
+                            const int32_t* gmap, int32_t n_groups, bool absmax, float* scales,
+                            int8_t* q, uint32_t* status, cudaStream_t st) {
+  const uint64_t n = (uint64_t)outer * (uint64_t)mid * (uint64_t)inner;
+  if (n + 64 < (1ull << 32)) {
+    const uint32_t n32 = (uint32_t)n, m32 = (uint32_t)mid, i32 = (uint32_t)inner;
+    return f16 ? quantize_p<true, uint32_t>(src, n32, m32, i32, gmap, n_groups, absmax, scales, q,
+                                            status, st)
+               : quantize_p<false, uint32_t>(src, n32, m32, i32, gmap, n_groups, absmax, scales, q,
+                                             status, st);
+  }
+  return f16 ? quantize_p<true, uint64_t>(src, n, (uint64_t)mid, (uint64_t)inner, gmap, n_groups,
+                                          absmax, scales, q, status, st)
+             : quantize_p<false, uint64_t>(src, n, (uint64_t)mid, (uint64_t)inner, gmap, n_groups,
+                                           absmax, scales, q, status, st);
+}
+
+cudaError_t launch_softedge_encode(const void* src, bool f16, int64_t n, float scale, float lo,
+                                   float hi, int log2_ratio, uint8_t* codes, uint32_t* status,
+                                   cudaStream_t st) {
+  if (n == 0) return cudaSuccess;
+  const SeSteps steps = se_steps(scale, log2_ratio);
+  if ((uint64_t)n + 64 < (1ull << 32)) {
+    const uint32_t n32 = (uint32_t)n;
+    if (f16)
+      se_encode_kernel<true, uint32_t><<<grid_for(n32), kThreads, 0, st>>>(src, n32, lo, hi, steps,
+                                                                           codes, status);
+    else
+      se_encode_kernel<false, uint32_t><<<grid_for(n32), kThreads, 0, st>>>(src, n32, lo, hi, steps,
+                                                                            codes, status);
+  } else {
+    const uint64_t n64 = (uint64_t)n;
+    if (f16)
+      se_encode_kernel<true, uint64_t><<<grid_for(n64), kThreads, 0, st>>>(src, n64, lo, hi, steps,
+                                                                           codes, status);
+    else
+      se_encode_kernel<false, uint64_t><<<grid_for(n64), kThreads, 0, st>>>(src, n64, lo, hi, steps,
+                                                                            codes, status);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_softedge_decode(const uint8_t* codes, int64_t n, float scale, int log2_ratio,
+                                   float* out, cudaStream_t st) {
+  if (n == 0) return cudaSuccess;
+  const SeSteps steps = se_steps(scale, log2_ratio);
+  if ((uint64_t)n + 64 < (1ull << 32)) {
+    const uint32_t n32 = (uint32_t)n;
+    se_decode_kernel<uint32_t><<<grid_for(n32), kThreads, 0, st>>>(codes, n32, steps, out);
+  } else {
+    const uint64_t n64 = (uint64_t)n;
+    se_decode_kernel<uint64_t><<<grid_for(n64), kThreads, 0, st>>>(codes, n64, steps, out);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace ssmq

@@ -31,3 +31,10 @@ def orc():
     from oracle import oracle as O
     O.lib()
     return O
+
+
+@pytest.fixture(scope="session", autouse=True)
+def _native_built():
+    """Rebuild libssmq.so when a source is newer (a no-op otherwise)."""
+    from quantized_state_space_b200 import build_native
+    build_native.build()

@@ -1,0 +1,175 @@
+"""The C-ABI library on a CPU-only host: it loads, exports every entry point
+declared in include/*.h, its argument structs have the layout the binding
+assumes, and invalid arguments are rejected before any device call."""
+import ctypes as C
+import glob
+import os
+import re
+import subprocess
+
+import pytest
+
+from quantized_state_space_b200 import _native as N
+from quantized_state_space_b200 import build_native
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    build_native.build()
+    return N.lib()
+
+
+def _declared():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        src = re.sub(r"/\*.*?\*/", "", open(h).read(), flags=re.S)
+        names |= set(re.findall(r"\b(ssmq_[a-z0-9_]+)\s*\(", src))
+    return names
+
+
+def test_exports_every_declared_symbol(L):
+    declared = _declared()
+    assert {"ssmq_quantize_groups", "ssmq_selective_scan_w8", "ssmq_ssd_chunk_scan_w8",
+            "ssmq_state_update_w8", "ssmq_softedge_encode", "ssmq_softedge_decode"} <= declared
+    out = subprocess.check_output(["nm", "-D", "--defined-only", N.LIB_PATH], text=True)
+    exported = set(re.findall(r"\bT (ssmq_\w+)", out))
+    assert declared <= exported, declared - exported
+    assert declared <= set(N.SIGNATURES), declared - set(N.SIGNATURES)
+
+
+def test_struct_layout_matches_header(tmp_path):
+    prog = ["#include <stdio.h>", "#include <stddef.h>", '#include "ssmq.h"', "int main(void){"]
+    for cls, cname in ((N.ScanArgs, "ssmq_scan_args"), (N.SSDArgs, "ssmq_ssd_args"),
+                       (N.DecodeArgs, "ssmq_decode_args")):
+        prog.append('printf("%s %%zu\\n", sizeof(%s));' % (cname, cname))
+        for f, _ in cls._fields_:
+            prog.append('printf("%s.%s %%zu\\n", offsetof(%s, %s));' % (cname, f, cname, f))
+    prog.append("return 0;}")
+    src = tmp_path / "layout.c"
+    src.write_text("\n".join(prog))
+    exe = tmp_path / "layout"
+    subprocess.check_call(["gcc", "-I", os.path.join(ROOT, "include"), "-o", str(exe), str(src)])
+    got = dict(line.split() for line in subprocess.check_output([str(exe)], text=True).splitlines())
+    for cls, cname in ((N.ScanArgs, "ssmq_scan_args"), (N.SSDArgs, "ssmq_ssd_args"),
+                       (N.DecodeArgs, "ssmq_decode_args")):
+        assert int(got[cname]) == C.sizeof(cls), cname
+        for f, _ in cls._fields_:
+            assert int(got["%s.%s" % (cname, f)]) == getattr(cls, f).offset, (cname, f)
+
+
+FAKE = 0x10000  # an aligned, never-dereferenced address for validation tests
+
+
+def _status_of(fn, *a):
+    return getattr(N.lib(), fn)(*a)
+
+
+def test_quantize_validation(L):
+    Q = L.ssmq_quantize_groups
+    assert Q(FAKE, 5, 1, 1, 16, FAKE, 1, 0, FAKE, FAKE, None, None) == N.ERR_INVALID_ARG  # dtype
+    assert Q(FAKE, 1, 1, 1, 16, FAKE, 1, 7, FAKE, FAKE, None, None) == N.ERR_INVALID_ARG  # mode
+    assert Q(FAKE, 1, -1, 1, 16, FAKE, 1, 0, FAKE, FAKE, None, None) == N.ERR_INVALID_ARG
+    assert Q(FAKE, 1, 1, 1, 16, FAKE, 0, 0, FAKE, FAKE, None, None) == N.ERR_INVALID_ARG
+    assert Q(None, 1, 1, 1, 16, FAKE, 1, 0, FAKE, FAKE, None, None) == N.ERR_INVALID_ARG
+    assert "NULL" in N.ssmq_last_error()
+    assert Q(FAKE + 2, 1, 1, 1, 16, FAKE, 1, 0, FAKE, FAKE, None, None) == N.ERR_ALIGNMENT
+    # empty static problem: nothing to do, no launch
+    assert Q(None, 1, 0, 5, 16, None, 1, 0, FAKE, None, None, None) == N.OK
+
+
+def test_softedge_validation(L):
+    E = L.ssmq_softedge_encode
+    assert E(FAKE, 1, 16, 1.0, 2.0, 1.0, 2, FAKE, None, None) == N.ERR_INVALID_ARG  # L > H
+    assert "thr_lo" in N.ssmq_last_error()
+    assert E(FAKE, 1, 16, 1.0, 0.5, 1.0, 9, FAKE, None, None) == N.ERR_INVALID_ARG
+    assert E(FAKE, 1, 16, 1.0, 0.5, 1.0, 2, FAKE + 8, None, None) == N.ERR_ALIGNMENT
+    D = L.ssmq_softedge_decode
+    assert D(None, 16, 1.0, 2, FAKE, None) == N.ERR_INVALID_ARG
+    assert D(FAKE, -1, 1.0, 2, FAKE, None) == N.ERR_INVALID_ARG
+
+
+def _scan_args(**kw):
+    f = dict(batch=2, seqlen=64, dim=32, dstate=16, ngroups=1, state_group_size=4,
+             x_format=N.X_INT8_GROUP, x=FAKE, x_group=FAKE, x_scale=FAKE, n_x_groups=4,
+             dt=FAKE, A=FAKE, B=FAKE, C=FAKE, B_scale=FAKE, C_scale=FAKE, y=FAKE,
+             dt_softplus=1)
+    f.update(kw)
+    return N._fill(N.ScanArgs, f)
+
+
+def test_scan_validation(L):
+    S = lambda **kw: L.ssmq_selective_scan_w8(C.byref(_scan_args(**kw)), None)
+    assert S(dstate=12) == N.ERR_UNSUPPORTED
+    assert S(dstate=128) == N.ERR_UNSUPPORTED
+    assert S(ngroups=3) == N.ERR_INVALID_ARG
+    assert S(state_group_size=3) == N.ERR_INVALID_ARG
+    assert S(x_format=5) == N.ERR_INVALID_ARG
+    assert S(x_group=None) == N.ERR_INVALID_ARG
+    assert S(n_x_groups=0) == N.ERR_INVALID_ARG
+    assert S(dt=None) == N.ERR_INVALID_ARG
+    assert S(y=FAKE + 4) == N.ERR_ALIGNMENT
+    assert S(x_format=N.X_SOFTEDGE, x_group=None, x_scale=None, se_log2_ratio=12) == N.ERR_INVALID_ARG
+    assert S(batch=0) == N.OK
+    assert L.ssmq_selective_scan_w8(None, None) == N.ERR_INVALID_ARG
+
+
+def _ssd_args(**kw):
+    f = dict(batch=1, seqlen=512, nheads=8, headdim=64, dstate=128, ngroups=1, chunk=256,
+             state_group_size=8, x_format=N.X_INT8_GROUP, x=FAKE, x_group=FAKE, x_scale=FAKE,
+             n_x_groups=2, dt=FAKE, A=FAKE, B=FAKE, C=FAKE, B_scale=FAKE, C_scale=FAKE, y=FAKE,
+             dt_softplus=1)
+    f.update(kw)
+    return N._fill(N.SSDArgs, f)
+
+
+def test_ssd_validation(L):
+    S = lambda ws=None, nb=0, **kw: L.ssmq_ssd_chunk_scan_w8(C.byref(_ssd_args(**kw)), ws, nb, None)
+    assert S(headdim=32) == N.ERR_UNSUPPORTED
+    assert S(chunk=100) == N.ERR_UNSUPPORTED
+    assert S(ngroups=3) == N.ERR_INVALID_ARG
+    assert S(x=None) == N.ERR_INVALID_ARG
+    need = L.ssmq_ssd_workspace_size(C.byref(_ssd_args()))
+    if need:
+        assert S(ws=None, nb=0) == N.ERR_INVALID_ARG
+        assert S(ws=FAKE + 16, nb=need) == N.ERR_ALIGNMENT
+
+
+def _dec_args(**kw):
+    f = dict(batch=4, nheads=8, headdim=64, dstate=128, ngroups=2, state_group_size=8,
+             x_format=N.X_INT8_GROUP, x=FAKE, x_group=FAKE, x_scale=FAKE, n_x_groups=2, dt=FAKE,
+             A=FAKE, B=FAKE, C=FAKE, B_scale=FAKE, C_scale=FAKE, state=FAKE, y=FAKE,
+             dt_softplus=1)
+    f.update(kw)
+    return N._fill(N.DecodeArgs, f)
+
+
+def test_decode_validation(L):
+    S = lambda **kw: L.ssmq_state_update_w8(C.byref(_dec_args(**kw)), None)
+    assert S(dstate=96) == N.ERR_UNSUPPORTED
+    assert S(ngroups=3) == N.ERR_INVALID_ARG
+    assert S(state=None) == N.ERR_INVALID_ARG
+    assert S(state=FAKE + 4) == N.ERR_ALIGNMENT
+    assert S(batch=0) == N.OK
+
+
+def test_fault_injection_hook(L, monkeypatch):
+    """SSMQ_FAULT_INJECT makes the named entry point report a launch failure
+    after validation, without touching the device."""
+    monkeypatch.setenv("SSMQ_FAULT_INJECT", "ssmq_selective_scan_w8")
+    assert L.ssmq_selective_scan_w8(C.byref(_scan_args()), None) == N.ERR_CUDA
+    assert "injected" in N.ssmq_last_error()
+    with pytest.raises(N.SSMQError) as ei:
+        N.ssmq_selective_scan_w8(stream=0, **{k: getattr(_scan_args(), k)
+                                               for k, _ in N.ScanArgs._fields_})
+    assert ei.value.status == N.ERR_CUDA
+    # validation still runs first
+    assert L.ssmq_selective_scan_w8(C.byref(_scan_args(dt=None)), None) == N.ERR_INVALID_ARG
+    monkeypatch.setenv("SSMQ_FAULT_INJECT", "all")
+    assert L.ssmq_state_update_w8(C.byref(_dec_args()), None) == N.ERR_CUDA
+    assert L.ssmq_quantize_groups(FAKE, 1, 1, 1, 16, FAKE, 1, 0, FAKE, FAKE, None, None) == N.ERR_CUDA
+
+
+def test_version(L):
+    assert N.ssmq_version() >= 100

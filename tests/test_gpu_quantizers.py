@@ -1,0 +1,131 @@
+"""GPU quantizers vs the oracle, bit for bit (Quamba-SE write-up sections 1,
+2.1, 2.2; Quamba2 abstract)."""
+import numpy as np
+import pytest
+import torch
+
+from gpu_util import H, T, dev, status_word
+from quantized_state_space_b200 import _native as N
+from quantized_state_space_b200 import api, calibrate, synth
+
+pytestmark = pytest.mark.gpu
+
+SHAPES = [  # (outer, mid, inner): row path, column path, general path, ragged tails
+    (3, 5, 2048), (2, 37, 1003), (777, 80, 1), (5, 17, 1), (1, 1, 7), (4, 48, 16),
+    (9, 1536, 3), (1, 3, 100_001),
+]
+
+
+@pytest.mark.parametrize("shape", SHAPES)
+@pytest.mark.parametrize("dtype", [np.float16, np.float32])
+def test_quantize_static(orc, shape, dtype):
+    outer, mid, inner = shape
+    rng = np.random.default_rng(sum(shape))
+    k = min(6, mid)
+    gmap = rng.integers(0, k, size=mid).astype(np.int32)
+    x = (rng.standard_normal(shape) * rng.choice([0.1, 1, 20], size=shape)).astype(dtype)
+    sc = synth.random_scales(rng, k, 0.01, 0.2)
+    qg, _ = api.quantize_groups(T(x), outer, mid, inner, T(gmap), k, scales=T(sc))
+    qo, _, _ = orc.quantize_groups(x, outer, mid, inner, gmap, k, orc.SCALE_STATIC, sc)
+    np.testing.assert_array_equal(H(qg), qo)
+
+
+@pytest.mark.parametrize("shape", SHAPES)
+def test_quantize_absmax(orc, shape):
+    outer, mid, inner = shape
+    rng = np.random.default_rng(7 + sum(shape))
+    k = min(5, mid)
+    gmap = rng.integers(0, k, size=mid).astype(np.int32)
+    x = (rng.standard_normal(shape) * 3).astype(np.float16)
+    qg, sg = api.quantize_groups(T(x), outer, mid, inner, T(gmap), k, absmax=True)
+    qo, so, _ = orc.quantize_groups(x, outer, mid, inner, gmap, k, orc.SCALE_ABSMAX)
+    np.testing.assert_array_equal(H(sg), so)
+    np.testing.assert_array_equal(H(qg), qo)
+
+
+def test_quantize_all_f16_patterns(orc):
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    x = bits.view(np.float16).copy()
+    for s in (1.0, 0.0078125, 3.3e-5, 517.0):
+        st = status_word()
+        qg, _ = api.quantize_groups(T(x), 1, 1, x.size, T(np.zeros(1, np.int32)), 1,
+                                    scales=T(np.array([s], np.float32)), status=st)
+        qo, _, nf = orc.quantize_groups(x, 1, 1, x.size, [0], 1, orc.SCALE_STATIC,
+                                        np.array([s], np.float32))
+        np.testing.assert_array_equal(H(qg), qo)
+        assert nf > 0 and int(H(st)[0]) & N.DEV_NONFINITE
+
+
+def test_quantize_status_bits():
+    x = T(np.ones(64, np.float16))
+    st = status_word()
+    api.quantize_groups(x, 1, 64, 1, T(np.full(64, 3, np.int32)), 2, scales=T(np.ones(2, np.float32)),
+                        status=st)
+    torch.cuda.synchronize()
+    assert int(H(st)[0]) & N.DEV_BAD_GROUP
+    st.zero_()
+    q, _ = api.quantize_groups(x, 1, 64, 1, T(np.zeros(64, np.int32)), 1,
+                               scales=T(np.array([-1.0], np.float32)), status=st)
+    assert int(H(st)[0]) & N.DEV_BAD_SCALE and not H(q).any()
+
+
+def test_quantize_m130m_x_full_size(orc):
+    """Full-size Mamba-130M-shaped x with its sort-and-cluster scales."""
+    _, raw = synth.workload_inputs("m130m")
+    x = raw["x"]
+    b, d, L = x.shape
+    grp, sc = calibrate.m1_x_clusters(x, 8)
+    og, osc = orc.cluster_by_absmax(orc.absmax_per_mid(x, b, d, L), 8)
+    np.testing.assert_array_equal(grp, og)
+    np.testing.assert_array_equal(sc, osc)
+    qg, _ = api.quantize_groups(T(x), b, d, L, T(grp), 8, scales=T(sc))
+    qo, _, _ = orc.quantize_groups(x, b, d, L, og, 8, orc.SCALE_STATIC, osc)
+    np.testing.assert_array_equal(H(qg), qo)
+
+
+# ---- soft-edge ---------------------------------------------------------------
+
+@pytest.mark.parametrize("s,lo,hi,r", [(0.05, 0.1, 3.0, 2), (1.0 / 63, 0.02, 1.0, 2),
+                                       (0.2, 0.0, 12.0, 2), (0.05, 0.1, 3.0, 1),
+                                       (1.0, 1.0, 63.0, 2), (3e-6, 1e-5, 2e-4, 2)])
+def test_softedge_encode_all_f16(orc, s, lo, hi, r):
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    x = bits.view(np.float16).copy()
+    s, lo, hi = np.float32(s), np.float32(lo), np.float32(hi)
+    st = status_word()
+    cg = api.softedge_encode(T(x), s, lo, hi, r, status=st)
+    co, nf = orc.softedge_encode(x, s, lo, hi, r)
+    np.testing.assert_array_equal(H(cg), co)
+    assert int(H(st)[0]) & N.DEV_NONFINITE
+
+
+def test_softedge_encode_f32_random(orc):
+    rng = np.random.default_rng(3)
+    x = (rng.standard_t(3, size=1_000_003) * 0.7).astype(np.float32)
+    s, lo, hi = np.float32(0.031), np.float32(0.04), np.float32(2.9)
+    np.testing.assert_array_equal(H(api.softedge_encode(T(x), s, lo, hi, 2)),
+                                  orc.softedge_encode(x, s, lo, hi, 2)[0])
+
+
+@pytest.mark.parametrize("s,r", [(1.0, 2), (0.0173, 2), (0.0173, 1), (2.5e-39, 2)])
+def test_softedge_decode_all_codes(orc, s, r):
+    codes = np.tile(np.arange(256, dtype=np.uint16).astype(np.uint8), 37)[:9001]
+    dg = H(api.softedge_decode(T(codes), s, r))
+    do = orc.softedge_decode(codes, np.float32(s), r)
+    np.testing.assert_array_equal(dg.view(np.uint32), do.view(np.uint32))
+
+
+def test_softedge_full_size_workload(orc):
+    """Full-size soft-edge workload x (16 x 1536 x 8192), thresholds from the
+    5th / 99.9th percentiles of |x|."""
+    _, raw = synth.workload_inputs("softedge")
+    x = raw["x"]
+    s, lo, hi = calibrate.softedge_params(x)
+    assert lo == np.float32(orc.percentile_abs(x, 5.0))
+    assert hi == np.float32(orc.percentile_abs(x, 99.9))
+    cg = H(api.softedge_encode(T(x), s, lo, hi, 2))
+    co, _ = orc.softedge_encode(x, s, lo, hi, 2)
+    np.testing.assert_array_equal(cg, co)
+    # the page's "about 95% standard" holds by construction of L and H
+    frac_std = float(np.mean((co >> 7) == 0))
+    assert 0.93 < frac_std < 0.96

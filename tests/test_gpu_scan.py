@@ -1,0 +1,216 @@
+"""GPU Mamba-1 W8A8 selective scan vs the oracle (Quamba2 abstract: W8A8
+Mamba1 backbone; Quamba-SE write-up 2.2 for soft-edge x).
+
+Tolerances: max |y - y_ref| <= 2e-3 max |y_ref| (y is stored as binary16),
+final state relative L2 <= 1e-4."""
+import numpy as np
+import pytest
+import torch
+
+from gpu_util import H, T, assert_scan_close, dev, status_word
+from problems import m1_problem, oracle_kwargs
+from quantized_state_space_b200 import _native as N
+from quantized_state_space_b200 import api, calibrate, synth
+
+pytestmark = pytest.mark.gpu
+
+
+def gpu_scan(p, **kw):
+    args = dict(D=T(p["D"]), z=T(p["z"]), dt_bias=T(p["dt_bias"]), h0=T(p.get("h0")))
+    if p["x"].dtype == np.uint8:
+        args["se_scale"] = p["se_scale"]
+    else:
+        args["x_group"] = T(p["x_group"])
+        args["x_scale"] = T(p["x_scale"])
+    args.update(kw)
+    y, hf = api.selective_scan(T(p["x"]), T(p["dt"]), T(p["A"]), T(p["B"]), T(p["C"]),
+                               T(p["B_scale"]), T(p["C_scale"]), p["state_group_size"], **args)
+    return H(y).astype(np.float64), H(hf)
+
+
+def oracle_scan(orc, p, **kw):
+    return orc.m1_scan(p["x"], p["dt"], p["A"], p["B"], p["C"], p["B_scale"], p["C_scale"],
+                       p["state_group_size"], **oracle_kwargs(p), **kw)
+
+
+CASES = [
+    # (b, L, d, N, G, gs, gate, h0, bias, fmt)
+    (2, 200, 40, 16, 1, 4, True, False, False, "int8"),      # ragged L, partial channel tile
+    (1, 256, 64, 16, 1, 16, False, False, False, "int8"),    # the tiny workload's shape
+    (3, 129, 48, 16, 2, 4, True, True, True, "int8"),        # G = 2, h0, bias, ragged
+    (2, 64, 64, 4, 1, 2, True, True, False, "int8"),
+    (2, 96, 40, 8, 2, 4, False, True, True, "int8"),
+    (2, 80, 32, 32, 1, 8, True, True, False, "int8"),
+    (1, 70, 24, 64, 1, 16, True, False, True, "int8"),
+    (2, 192, 48, 16, 1, 4, True, True, False, "softedge"),
+    (1, 17, 16, 16, 1, 4, True, False, False, "int8"),       # L < chunk, L % 16 != 0
+    (1, 1, 16, 16, 1, 4, True, True, False, "int8"),         # one step
+    (4, 512, 96, 16, 1, 4, True, False, False, "int8"),      # several chunks and tiles
+]
+
+
+@pytest.mark.parametrize("ci", range(len(CASES)))
+def test_scan_vs_oracle(orc, ci):
+    b, L, d, N_, G, gs, gate, h0, bias, fmt = CASES[ci]
+    p = m1_problem(100 + ci, b, L, d, N_, G=G, gs=gs, gate=gate, h0=h0, bias=bias,
+                   x_format=fmt)
+    y, hf = gpu_scan(p)
+    yo, ho = oracle_scan(orc, p)
+    assert_scan_close(y, yo.reshape(y.shape), hf, ho.reshape(hf.shape))
+
+
+def test_scan_softplus_off_and_delta_zero(orc):
+    p = m1_problem(5, 2, 100, 32, 16, gate=False, h0=True)
+    p["dt"][:] = 0
+    y, hf = gpu_scan(p, dt_softplus=False)
+    yo, ho = oracle_scan(orc, p, dt_softplus=False)
+    assert_scan_close(y, yo.reshape(y.shape), hf, ho.reshape(hf.shape))
+    np.testing.assert_array_equal(hf, p["h0"])  # delta = 0 keeps the state
+
+
+def test_scan_empty_sequence():
+    p = m1_problem(6, 2, 16, 16, 16, h0=True)
+    x = T(np.zeros((2, 16, 0), np.int8))
+    dt = T(np.zeros((2, 16, 0), np.float16))
+    B = T(np.zeros((2, 1, 16, 0), np.int8))
+    y, hf = api.selective_scan(x, dt, T(p["A"]), B, B, T(p["B_scale"]), T(p["C_scale"]), 4,
+                               x_group=T(p["x_group"]), x_scale=T(p["x_scale"]), h0=T(p["h0"]))
+    np.testing.assert_array_equal(H(hf), p["h0"])
+
+
+def test_scan_bad_group_status():
+    p = m1_problem(7, 1, 32, 16, 16)
+    p["x_group"][3] = 99
+    st = status_word()
+    gpu_scan(p, status=st)
+    assert int(H(st)[0]) & N.DEV_BAD_GROUP
+
+
+def test_scan_channel_permutation_bit_exact():
+    """Quamba2 compute invariance: permuting channels with their cluster ids,
+    A, D, dt, z permutes y and the state exactly."""
+    p = m1_problem(8, 2, 300, 64, 16, gate=True, h0=True, bias=True)
+    perm = np.random.default_rng(1).permutation(64)
+    q = dict(p)
+    for k in ("x", "dt", "z"):
+        q[k] = np.ascontiguousarray(p[k][:, perm, :])
+    q["x_group"], q["A"], q["D"] = p["x_group"][perm], p["A"][perm], p["D"][perm]
+    q["dt_bias"], q["h0"] = p["dt_bias"][perm], np.ascontiguousarray(p["h0"][:, perm, :])
+    y, hf = gpu_scan(p)
+    yq, hq = gpu_scan(q)
+    np.testing.assert_array_equal(yq, y[:, perm, :])
+    np.testing.assert_array_equal(hq, hf[:, perm, :])
+
+
+def test_scan_power_of_two_scale_linearity():
+    """Doubling every x scale doubles y and the state exactly (no gate,
+    zero initial state): each product with x is an exact doubling."""
+    p = m1_problem(9, 2, 256, 32, 16, gate=False)
+    y, hf = gpu_scan(p)
+    q = dict(p)
+    q["x_scale"] = (p["x_scale"] * 2).astype(np.float32)
+    y2, h2 = gpu_scan(q)
+    # binary16 subnormals (|y| < 2^-14) round on an absolute grid, so the
+    # doubling is exact only for normal outputs
+    normal = np.abs(2 * y) >= 2.0 ** -14
+    np.testing.assert_array_equal(y2[normal], 2 * y[normal])
+    assert np.all(np.abs(y2[~normal] - 2 * y[~normal]) <= 2.0 ** -24)
+    np.testing.assert_array_equal(h2, 2 * hf)
+
+
+def test_scan_checkpoint_split_bit_exact():
+    """scan(L) equals scan(first 256 steps) then scan(rest, h0 = that state)."""
+    p = m1_problem(10, 2, 512, 32, 16, gate=True)
+    y, hf = gpu_scan(p)
+    a = dict(p)
+    b = dict(p)
+    for k in ("x", "dt", "z"):
+        a[k] = np.ascontiguousarray(p[k][..., :256])
+        b[k] = np.ascontiguousarray(p[k][..., 256:])
+    for k in ("B", "C"):
+        a[k] = np.ascontiguousarray(p[k][..., :256])
+        b[k] = np.ascontiguousarray(p[k][..., 256:])
+    ya, ha = gpu_scan(a)
+    b["h0"] = ha
+    yb, hb = gpu_scan(b)
+    np.testing.assert_array_equal(np.concatenate([ya, yb], axis=-1), y)
+    np.testing.assert_array_equal(hb, hf)
+
+
+# ---- full-size workloads, end to end from raw activations ------------------
+
+def _m1_end_to_end(orc, name, n_units=96):
+    dm, raw = synth.workload_inputs(name)
+    b, L, d, Nst, G, gs = dm["batch"], dm["seqlen"], dm["dim"], dm["dstate"], dm["ngroups"], \
+        dm["state_group_size"]
+    gmap = calibrate.state_group_map(G, Nst, gs)
+    # product: host calibration + GPU quantizers + GPU scan
+    bs = calibrate.state_group_absmax_scales(raw["B"], G, Nst, gs, "gnl")
+    cs = calibrate.state_group_absmax_scales(raw["C"], G, Nst, gs, "gnl")
+    Bq, _ = api.quantize_groups(T(raw["B"]), b, G * Nst, L, T(gmap), G * Nst // gs, scales=T(bs))
+    Cq, _ = api.quantize_groups(T(raw["C"]), b, G * Nst, L, T(gmap), G * Nst // gs, scales=T(cs))
+    if name == "softedge":
+        s, lo, hi = calibrate.softedge_params(raw["x"])
+        xq = api.softedge_encode(T(raw["x"]), s, lo, hi, 2)
+        xkw = dict(se_scale=s)
+    else:
+        k = dm["x_clusters"]
+        if k == 1:
+            xq, xs = api.quantize_groups(T(raw["x"]), b, d, L, T(np.zeros(d, np.int32)), 1,
+                                         absmax=True)
+            xkw = dict(x_group=T(np.zeros(d, np.int32)), x_scale=xs)
+        else:
+            grp, xs = calibrate.m1_x_clusters(raw["x"], k)
+            xq, _ = api.quantize_groups(T(raw["x"]), b, d, L, T(grp), k, scales=T(xs))
+            xkw = dict(x_group=T(grp), x_scale=T(xs))
+    y, hf = api.selective_scan(xq, T(raw["dt"]), T(raw["A"]), Bq, Cq, T(bs), T(cs), gs,
+                               D=T(raw["D"]), z=T(raw["z"]), **xkw)
+    torch.cuda.synchronize()
+    # oracle: its own calibration and quantizers from the same raw arrays; the
+    # B/C scale index of row (g, n) is (g N + n) / gs in the ABI's layout
+    gmap = np.arange(G * Nst) // gs
+    _, obs, _ = orc.quantize_groups(raw["B"], b, G * Nst, L, gmap, G * Nst // gs, orc.SCALE_ABSMAX)
+    _, ocs, _ = orc.quantize_groups(raw["C"], b, G * Nst, L, gmap, G * Nst // gs, orc.SCALE_ABSMAX)
+    oB, _, _ = orc.quantize_groups(raw["B"], b, G * Nst, L, gmap, G * Nst // gs, orc.SCALE_STATIC, obs)
+    oC, _, _ = orc.quantize_groups(raw["C"], b, G * Nst, L, gmap, G * Nst // gs, orc.SCALE_STATIC, ocs)
+    np.testing.assert_array_equal(H(Bq), oB)
+    np.testing.assert_array_equal(H(Cq), oC)
+    if name == "softedge":
+        olo = np.float32(orc.percentile_abs(raw["x"], 5.0))
+        ohi = np.float32(orc.percentile_abs(raw["x"], 99.9))
+        osc = np.float32(np.float64(ohi) / 63.0)
+        ox, _ = orc.softedge_encode(raw["x"], osc, olo, ohi, 2)
+        okw = dict(se_scale=float(osc))
+    else:
+        k = dm["x_clusters"]
+        if k == 1:
+            ox, oxs, _ = orc.quantize_groups(raw["x"], b, d, L, np.zeros(d, np.int32), 1,
+                                             orc.SCALE_ABSMAX)
+            okw = dict(x_group=np.zeros(d, np.int32), x_scale=oxs)
+        else:
+            og, oxs = orc.cluster_by_absmax(orc.absmax_per_mid(raw["x"], b, d, L), k)
+            ox, _, _ = orc.quantize_groups(raw["x"], b, d, L, og, k, orc.SCALE_STATIC, oxs)
+            okw = dict(x_group=og, x_scale=oxs)
+    np.testing.assert_array_equal(H(xq), ox)
+    rng = np.random.default_rng(0)
+    units = rng.choice(b * d, size=min(n_units, b * d), replace=False)
+    if raw.get("outlier_channels") is not None:  # always include the outlier channels
+        units = np.unique(np.concatenate([units, raw["outlier_channels"]]))
+    yo, ho = orc.m1_scan(ox, raw["dt"], raw["A"], oB, oC, obs, ocs, gs, D=raw["D"], z=raw["z"],
+                         units=units, **okw)
+    yg = H(y).reshape(b * d, L)[units].astype(np.float64)
+    hg = H(hf).reshape(b * d, Nst)[units]
+    # the tolerance is relative to max |y_ref| over the sampled channels
+    return assert_scan_close(yg, yo, hg, ho)
+
+
+def test_tiny_workload_end_to_end(orc):
+    _m1_end_to_end(orc, "tiny", n_units=64)
+
+
+def test_m130m_workload_end_to_end(orc):
+    _m1_end_to_end(orc, "m130m")
+
+
+def test_softedge_workload_end_to_end(orc):
+    _m1_end_to_end(orc, "softedge", n_units=64)
