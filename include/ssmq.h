@@ -68,6 +68,7 @@ typedef enum {
 #define SSMQ_DEV_NONFINITE 1u /* a non-finite input element was met (coded 0) */
 #define SSMQ_DEV_BAD_GROUP 2u /* a device group id was out of range (coded 0) */
 #define SSMQ_DEV_BAD_SCALE 4u /* a device scale was negative / non-finite */
+#define SSMQ_DEV_TIMEOUT 8u   /* a bounded wait for the tensor core gave up */
 
 typedef enum { SSMQ_F32 = 0, SSMQ_F16 = 1 } ssmq_dtype;
 typedef enum { SSMQ_SCALE_STATIC = 0, SSMQ_SCALE_ABSMAX = 1 } ssmq_scale_mode;
@@ -217,7 +218,11 @@ ssmq_status ssmq_selective_scan_w8(const ssmq_scan_args* args, void* stream);
  *   h_final  fp32 (b, H, P, N) output or NULL
  * workspace: device memory of at least ssmq_ssd_workspace_size(args) bytes,
  *   256-byte aligned, caller-owned, contents need not be initialised.
- * Supported: P == 64, N == 128, chunk in {64, 128, 256}, H % G == 0.
+ * Supported: P == 64, N == 128, chunk in {64, 128, 256}, H % G == 0.  The
+ * result is the recurrence's for every chunk length (the decomposition is
+ * exact up to rounding); the kernel processes 128-step tiles.
+ * status: SSMQ_DEV_BAD_GROUP as above; SSMQ_DEV_TIMEOUT if a bounded wait for
+ * the tensor core gave up (the call's outputs are then incomplete).
  */
 typedef struct {
   int64_t batch, seqlen, nheads, headdim, dstate, ngroups;

@@ -16,7 +16,7 @@ OK, ERR_INVALID_ARG, ERR_ALIGNMENT, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_
 STATUS_NAMES = {0: "SSMQ_OK", 1: "SSMQ_ERR_INVALID_ARG", 2: "SSMQ_ERR_ALIGNMENT",
                 3: "SSMQ_ERR_UNSUPPORTED", 4: "SSMQ_ERR_CUDA", 5: "SSMQ_ERR_TIMEOUT",
                 6: "SSMQ_ERR_NONFINITE"}
-DEV_NONFINITE, DEV_BAD_GROUP, DEV_BAD_SCALE = 1, 2, 4
+DEV_NONFINITE, DEV_BAD_GROUP, DEV_BAD_SCALE, DEV_TIMEOUT = 1, 2, 4, 8
 F32, F16 = 0, 1
 SCALE_STATIC, SCALE_ABSMAX = 0, 1
 X_INT8_GROUP, X_SOFTEDGE = 0, 1

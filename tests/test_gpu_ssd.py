@@ -1,0 +1,143 @@
+"""GPU Mamba-2 SSD chunked scan (tcgen05) vs the oracle (SSDi8 abstract;
+Quamba2 abstract: W8A8 Mamba2 backbone).
+
+Tolerances: max |y - y_ref| <= 2e-3 max |y_ref|, final state rel-L2 <= 1e-4."""
+import numpy as np
+import pytest
+import torch
+
+from gpu_util import H, T, assert_scan_close, status_word, y_err, state_err
+from problems import oracle_kwargs, ssd_problem
+from quantized_state_space_b200 import _native as N
+from quantized_state_space_b200 import api, calibrate, synth
+
+pytestmark = pytest.mark.gpu
+
+
+def gpu_ssd(p, chunk=256, **kw):
+    args = dict(D=T(p["D"]), z=T(p["z"]), dt_bias=T(p["dt_bias"]), h0=T(p.get("h0")))
+    if p["x"].dtype == np.uint8:
+        args["se_scale"] = p["se_scale"]
+    else:
+        args["x_group"] = T(p["x_group"])
+        args["x_scale"] = T(p["x_scale"])
+    args.update(kw)
+    y, hf = api.ssd_chunk_scan(T(p["x"]), T(p["dt"]), T(p["A"]), T(p["B"]), T(p["C"]),
+                               T(p["B_scale"]), T(p["C_scale"]), p["state_group_size"],
+                               chunk=chunk, **args)
+    return H(y).astype(np.float64), H(hf)
+
+
+def oracle_ssd(orc, p, **kw):
+    return orc.ssd_scan(p["x"], p["dt"], p["A"], p["B"], p["C"], p["B_scale"], p["C_scale"],
+                        p["state_group_size"], **oracle_kwargs(p), **kw)
+
+
+CASES = [
+    # (b, L, H, G, gs, gate, h0, bias, fmt, dt_mean)
+    (1, 128, 2, 1, 8, False, False, False, "int8", -4.0),   # one tile
+    (2, 300, 3, 1, 8, True, True, True, "int8", -4.0),      # ragged last tile, h0, gate
+    (1, 64, 4, 2, 4, False, True, False, "int8", -4.0),     # shorter than a tile, G = 2
+    (1, 1, 2, 1, 8, False, True, False, "int8", -4.0),      # one step
+    (2, 512, 4, 4, 16, True, False, True, "int8", -2.0),    # strong decay, G = 4
+    (1, 384, 2, 1, 8, True, True, False, "softedge", -4.0),
+    (1, 1000, 2, 1, 8, False, False, False, "int8", -5.0),  # weak decay, long
+]
+
+
+@pytest.mark.parametrize("ci", range(len(CASES)))
+def test_ssd_vs_oracle(orc, ci):
+    b, L, Hh, G, gs, gate, h0, bias, fmt, dtm = CASES[ci]
+    p = ssd_problem(400 + ci, b, L, Hh, 64, 128, G=G, gs=gs, gate=gate, h0=h0, bias=bias,
+                    x_format=fmt, dt_mean=dtm)
+    st = status_word()
+    y, hf = gpu_ssd(p, status=st)
+    yo, ho = oracle_ssd(orc, p)
+    assert int(H(st)[0]) == 0
+    assert_scan_close(y.transpose(0, 2, 1, 3).reshape(yo.shape), yo, hf.reshape(ho.shape), ho)
+
+
+@pytest.mark.parametrize("chunk", [64, 128, 256])
+def test_ssd_chunk_lengths_agree(orc, chunk):
+    p = ssd_problem(450, 1, 520, 2, 64, 128, gate=True, h0=True)
+    y, hf = gpu_ssd(p, chunk=chunk)
+    yo, ho = oracle_ssd(orc, p)
+    assert_scan_close(y.transpose(0, 2, 1, 3).reshape(yo.shape), yo, hf.reshape(ho.shape), ho)
+
+
+def test_ssd_split_with_state_bit_exact():
+    """scan(L) equals scan(first 256 steps) then scan(rest, h0 = its state)."""
+    p = ssd_problem(460, 2, 512, 2, 64, 128, gate=True)
+    y, hf = gpu_ssd(p)
+    a, b = dict(p), dict(p)
+    for k in ("x", "dt", "z", "B", "C"):
+        a[k] = np.ascontiguousarray(p[k][:, :256])
+        b[k] = np.ascontiguousarray(p[k][:, 256:])
+    ya, ha = gpu_ssd(a)
+    b["h0"] = ha
+    yb, hb = gpu_ssd(b)
+    np.testing.assert_array_equal(np.concatenate([ya, yb], axis=1), y)
+    np.testing.assert_array_equal(hb, hf)
+
+
+def test_ssd_delta_zero(orc):
+    p = ssd_problem(470, 1, 200, 2, 64, 128, h0=True)
+    p["dt"][:] = 0
+    y, hf = gpu_ssd(p, dt_softplus=False)
+    yo, ho = oracle_ssd(orc, p, dt_softplus=False)
+    assert_scan_close(y.transpose(0, 2, 1, 3).reshape(yo.shape), yo, hf.reshape(ho.shape), ho)
+    np.testing.assert_allclose(hf, p["h0"], rtol=0, atol=0)
+
+
+def test_ssd_bad_group_status():
+    p = ssd_problem(480, 1, 128, 2, 64, 128)
+    p["x_group"][5] = 1000
+    st = status_word()
+    gpu_ssd(p, status=st)
+    assert int(H(st)[0]) & N.DEV_BAD_GROUP
+
+
+def test_ssd27b_workload_end_to_end(orc):
+    """The Mamba-2-2.7B-shaped SSD layer (b 4, L 4096, H 80, P 64, N 128, G 1)
+    from raw activations: host calibration, GPU quantizers, GPU SSD; the
+    oracle repeats every step from the raw arrays on sampled heads."""
+    dm, raw = synth.workload_inputs("ssd27b")
+    b, L, Hh, P, Nst, G, gs, k = (dm["batch"], dm["seqlen"], dm["nheads"], dm["headdim"],
+                                  dm["dstate"], dm["ngroups"], dm["state_group_size"],
+                                  dm["x_clusters"])
+    grp, xs = calibrate.ssd_x_clusters(raw["x"], k)
+    smap = calibrate.state_group_map(G, Nst, gs)
+    bs = calibrate.state_group_absmax_scales(raw["B"], G, Nst, gs, "lgn")
+    cs = calibrate.state_group_absmax_scales(raw["C"], G, Nst, gs, "lgn")
+    xq, _ = api.quantize_groups(T(raw["x"]), b * L, Hh * P, 1, T(grp), k, scales=T(xs))
+    Bq, _ = api.quantize_groups(T(raw["B"]), b * L, G * Nst, 1, T(smap), G * Nst // gs, scales=T(bs))
+    Cq, _ = api.quantize_groups(T(raw["C"]), b * L, G * Nst, 1, T(smap), G * Nst // gs, scales=T(cs))
+    st = status_word()
+    y, hf = api.ssd_chunk_scan(xq, T(raw["dt"]), T(raw["A"]), Bq, Cq, T(bs), T(cs), gs,
+                               chunk=dm["chunk"], x_group=T(grp), x_scale=T(xs), D=T(raw["D"]),
+                               status=st)
+    torch.cuda.synchronize()
+    assert int(H(st)[0]) == 0
+    # oracle chain
+    head_abs = np.abs(raw["x"].astype(np.float32)).max(axis=(0, 1, 3))
+    ohc, oxs = orc.cluster_by_absmax(head_abs.astype(np.float64), k)
+    ogrp = np.repeat(ohc, P).astype(np.int32)
+    omap = np.arange(G * Nst) // gs
+    _, obs, _ = orc.quantize_groups(raw["B"], b * L, G * Nst, 1, omap, G * Nst // gs, orc.SCALE_ABSMAX)
+    _, ocs, _ = orc.quantize_groups(raw["C"], b * L, G * Nst, 1, omap, G * Nst // gs, orc.SCALE_ABSMAX)
+    ox, _, _ = orc.quantize_groups(raw["x"], b * L, Hh * P, 1, ogrp, k, orc.SCALE_STATIC, oxs)
+    oB, _, _ = orc.quantize_groups(raw["B"], b * L, G * Nst, 1, omap, G * Nst // gs, orc.SCALE_STATIC, obs)
+    oC, _, _ = orc.quantize_groups(raw["C"], b * L, G * Nst, 1, omap, G * Nst // gs, orc.SCALE_STATIC, ocs)
+    np.testing.assert_array_equal(H(xq), ox)
+    np.testing.assert_array_equal(H(Bq), oB)
+    # sampled heads, including the fastest- and slowest-decaying ones
+    rng = np.random.default_rng(2)
+    units = set(rng.choice(b * Hh, size=6, replace=False).tolist())
+    units |= {int(np.argmin(raw["A"])), int(np.argmax(raw["A"])) + Hh}
+    units = np.array(sorted(units))
+    yo, ho = orc.ssd_scan(ox, raw["dt"], raw["A"], oB, oC, obs, ocs, gs, x_group=ogrp,
+                          x_scale=oxs, D=raw["D"], units=units)
+    yg = H(y).astype(np.float64)  # (b, L, H, P)
+    yg = np.stack([yg[u // Hh, :, u % Hh, :] for u in units])
+    hg = H(hf).reshape(b * Hh, P, Nst)[units]
+    assert_scan_close(yg, yo, hg, ho)
