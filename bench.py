@@ -215,15 +215,45 @@ def cpu_baseline(layer, threads=None, max_units=None):
             "seconds": dt}
 
 
+# ---- ranks -----------------------------------------------------------------
+# One process per GPU; every rank scans its own independent layer batch (the
+# path has no exchange step), so the only cross-rank traffic is the reduction
+# of the measured time.
+
+def rank_env():
+    """(world, rank, local_rank) from the torchrun environment."""
+    return (int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def rank_seed(rank):
+    """Each rank draws an independent batch of the workload."""
+    return rank
+
+
+def max_over_ranks(value, dist=None, device=None):
+    """The slowest rank's time (max over the process group)."""
+    if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
+        return float(value)
+    import torch
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_scaling_value(world, units_per_rank, steps, ms_max):
+    """Whole-job throughput: units of all ranks over the slowest rank's time,
+    in giga-units per second."""
+    return world * units_per_rank * steps / (ms_max / 1e3) / 1e9
+
+
 # ---- our arm ----------------------------------------------------------------
 
 def run_ours(args):
     import torch
     import torch.distributed as dist
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    world, rank, local = rank_env()
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     if world > 1:
@@ -235,7 +265,7 @@ def run_ours(args):
     if world > 1:
         dist.barrier()
     pk = peaks()
-    layer = Layer(dev, seed=rank)
+    layer = Layer(dev, seed=rank_seed(rank))
     stream = torch.cuda.current_stream()
 
     def step():
@@ -262,14 +292,10 @@ def run_ours(args):
         torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    ms = e0.elapsed_time(e1)
+    ms = max_over_ranks(e0.elapsed_time(e1), dist if world > 1 else None, dev)
     scan_ms = [a.elapsed_time(b) for a, b in scan_ev]
-    if world > 1:
-        t = torch.tensor([ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
     ms_step = ms / K
-    value = world * layer.units * K / (ms / 1e3) / 1e9
+    value = weak_scaling_value(world, layer.units, K, ms)
 
     # end to end through the public API from pinned host buffers
     Ke = max(1, min(K, args.e2e_steps))
@@ -295,12 +321,8 @@ def run_ours(args):
         y_host.copy_(layer.y, non_blocking=True)
     a1.record(stream)
     torch.cuda.synchronize()
-    ems = a0.elapsed_time(a1)
-    if world > 1:
-        t = torch.tensor([ems], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ems = float(t.item())
-    e2e_value = world * layer.units * Ke / (ems / 1e3) / 1e9
+    ems = max_over_ranks(a0.elapsed_time(a1), dist if world > 1 else None, dev)
+    e2e_value = weak_scaling_value(world, layer.units, Ke, ems)
 
     out = None
     if rank == 0:
@@ -344,7 +366,8 @@ def run_ours(args):
             except Exception as e:  # report, keep the measured line
                 out["cpu_baseline"] = {"error": "%s: %s" % (type(e).__name__, e)}
         if world == 1 and not args.no_forms:
-            out["forms"] = run_forms(dev, pk, out["clocks"].get("sm_max_mhz") or pk["sm_max_mhz"])
+            out["forms"] = run_forms(dev, pk, out["clocks"].get("sm_max_mhz") or pk["sm_max_mhz"],
+                                     only=args.forms.split(",") if args.forms else None)
         print(json.dumps(out), flush=True)
 
 
@@ -451,11 +474,68 @@ def form_softedge(torch, dev, pk, mhz):
                      "unit": "Gupdates/s", "frac": round(upd / t_scan / 1e9 / peak_upd, 4)}}
 
 
-def run_forms(dev, pk, mhz):
+def form_ssd(torch, dev, pk):
+    """ssd27b: quantize x / B / C and run the SSD chunked scan (b 4, L 4096,
+    H 80, P 64, N 128, G 1, chunk 256) on tcgen05."""
+    from quantized_state_space_b200 import api, calibrate, synth
+    dm, raw = synth.workload_inputs("ssd27b")
+    b, L, H, P, N, G, gs, k = (dm["batch"], dm["seqlen"], dm["nheads"], dm["headdim"],
+                               dm["dstate"], dm["ngroups"], dm["state_group_size"],
+                               dm["x_clusters"])
+    T = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+    grp, xs = calibrate.ssd_x_clusters(raw["x"], k)
+    smap = T(calibrate.state_group_map(G, N, gs))
+    bs = calibrate.state_group_absmax_scales(raw["B"], G, N, gs, "lgn")
+    cs = calibrate.state_group_absmax_scales(raw["C"], G, N, gs, "lgn")
+    x, dt, B, C = T(raw["x"]), T(raw["dt"]), T(raw["B"]), T(raw["C"])
+    A, D, grp_t, xs_t, bs_t, cs_t = T(raw["A"]), T(raw["D"]), T(grp), T(xs), T(bs), T(cs)
+    del raw
+    xq = torch.empty(x.shape, dtype=torch.int8, device=dev)
+    Bq = torch.empty(B.shape, dtype=torch.int8, device=dev)
+    Cq = torch.empty(C.shape, dtype=torch.int8, device=dev)
+    y = torch.empty(x.shape, dtype=torch.float16, device=dev)
+    hf = torch.empty((b, H, P, N), dtype=torch.float32, device=dev)
+
+    def quant():
+        api.quantize_groups(x, b * L, H * P, 1, grp_t, k, scales=xs_t, out=xq)
+        api.quantize_groups(B, b * L, G * N, 1, smap, G * N // gs, scales=bs_t, out=Bq)
+        api.quantize_groups(C, b * L, G * N, 1, smap, G * N // gs, scales=cs_t, out=Cq)
+
+    def ssd():
+        api.ssd_chunk_scan(xq, dt, A, Bq, Cq, bs_t, cs_t, gs, chunk=dm["chunk"], x_group=grp_t,
+                           x_scale=xs_t, D=D, y=y, h_final=hf)
+
+    t_q = _timed(torch, quant, 5)
+    t_s = _timed(torch, ssd, 5)
+    q = 256  # the chunk length the algorithmic count refers to
+    nch = L // q
+    useful = (2 * q * (q + 1) // 2 * N * b * nch * G          # C B^T, causal half
+              + 2 * q * (q + 1) // 2 * P * b * nch * H        # diagonal blocks
+              + 2 * 2 * q * N * P * b * nch * H)              # carried state in and out
+    executed = 2 * b * H * (L // 128) * (128 ** 3 + 128 * 128 * 64 * 5)
+    byts = b * L * H * P * (1 + 2) + b * L * H * 2 + 2 * b * L * G * N + b * H * P * N * 4
+    tf = useful / t_s / 1e12
+    return {"workload": "ssd27b: b 4, L 4096, H 80, P 64, N 128, G 1, chunk 256; quantize + SSD",
+            "value": round(b * L * H * P / (t_q + t_s) / 1e9, 3), "unit": "Gtokens·ch/s",
+            "ms_per_step": round((t_q + t_s) * 1e3, 4), "ssd_ms": round(t_s * 1e3, 4),
+            "quantize_ms": round(t_q * 1e3, 4),
+            "roofline": {"bound": "tensor", "achieved": round(tf, 1), "peak": pk["bf16_tflops"],
+                         "unit": "TFLOP/s", "frac": round(tf / pk["bf16_tflops"], 4),
+                         "algorithmic_flops_per_launch": useful,
+                         "executed_mma_flops_per_launch": executed,
+                         "hbm_achieved_gbs": round(byts / t_s / 1e9, 1),
+                         "hbm_frac": round(byts / t_s / 1e9 / pk["hbm_gbs"], 4),
+                         "traffic": None}}
+
+
+def run_forms(dev, pk, mhz, only=None):
     import torch
     out = {}
-    for name, fn in (("decode8b", lambda: form_decode(torch, dev, pk)),
+    for name, fn in (("ssd27b", lambda: form_ssd(torch, dev, pk)),
+                     ("decode8b", lambda: form_decode(torch, dev, pk)),
                      ("softedge", lambda: form_softedge(torch, dev, pk, mhz))):
+        if only and name not in only:
+            continue
         try:
             out[name] = fn()
         except Exception as e:  # a failing form is reported, the headline stands
@@ -467,8 +547,7 @@ def run_forms(dev, pk, mhz):
 # ---- reference arm: the CPU oracle ------------------------------------------
 
 def run_reference(args):
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
+    world, rank, _ = rank_env()
     if rank != 0:
         return
     from oracle import oracle as O
@@ -516,6 +595,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-forms", action="store_true")
+    ap.add_argument("--forms", default="", help="comma list of ssd27b,decode8b,softedge")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.impl == "reference":

@@ -301,6 +301,52 @@ typedef struct {
 ssmq_status ssmq_state_update_w8(const ssmq_decode_args* args, void* stream);
 
 /* ------------------------------------------------------------------------ */
+/* Single-token decode state update (Mamba-1 form)                           */
+/* ------------------------------------------------------------------------ */
+/*
+ * Passage: Quamba2 abstract (generation stage; W8A8 Mamba1 backbone): one
+ * step of the diagonal recurrence on the persistent fp32 state, in place,
+ * with A per (channel, state).
+ *
+ * Layouts (b, d, N, G):
+ *   state    fp32 (b, d, N), read and overwritten
+ *   x        (b, d) int8 (INT8_GROUP) or soft-edge uint8 (SOFTEDGE)
+ *   x_group  int32[d]; x_scale fp32[n_x_groups]
+ *   dt       (b, d) binary16; dt_bias fp32[d] or NULL
+ *   A fp32 (d, N); D fp32[d] or NULL; z (b, d) binary16 or NULL
+ *   B, C     (b, G, N) int8; channel c reads group floor(c * G / d)
+ *   B_scale, C_scale fp32[G * N / state_group_size]
+ *   y        (b, d) binary16 output
+ * Supported: N in {4, 8, 16, 32, 64, 128}; d % G == 0.
+ */
+typedef struct {
+  int64_t batch, dim, dstate, ngroups;
+  int32_t state_group_size;
+  int32_t x_format;
+  const void* x;
+  const int32_t* x_group;
+  const float* x_scale;
+  int32_t n_x_groups;
+  float se_scale;
+  int32_t se_log2_ratio;
+  const uint16_t* dt;
+  const float* dt_bias;
+  int32_t dt_softplus;
+  const float* A;
+  const float* D;
+  const uint16_t* z;
+  const int8_t* B;
+  const int8_t* C;
+  const float* B_scale;
+  const float* C_scale;
+  float* state;
+  uint16_t* y;
+  uint32_t* status;
+} ssmq_m1_decode_args;
+
+ssmq_status ssmq_selective_state_update_w8(const ssmq_m1_decode_args* args, void* stream);
+
+/* ------------------------------------------------------------------------ */
 /* Diagnostics                                                               */
 /* ------------------------------------------------------------------------ */
 /* Thread-local, NUL-terminated description of the last non-OK status. */

@@ -60,6 +60,15 @@ class DecodeArgs(C.Structure):
                 ("status", _vp)]
 
 
+class M1DecodeArgs(C.Structure):
+    _fields_ = [("batch", _i64), ("dim", _i64), ("dstate", _i64), ("ngroups", _i64),
+                ("state_group_size", _i32), ("x_format", _i32), ("x", _vp), ("x_group", _vp),
+                ("x_scale", _vp), ("n_x_groups", _i32), ("se_scale", _f32),
+                ("se_log2_ratio", _i32), ("dt", _vp), ("dt_bias", _vp), ("dt_softplus", _i32),
+                ("A", _vp), ("D", _vp), ("z", _vp), ("B", _vp), ("C", _vp), ("B_scale", _vp),
+                ("C_scale", _vp), ("state", _vp), ("y", _vp), ("status", _vp)]
+
+
 # entry point -> (restype, argtypes); every name declared in include/ssmq.h
 SIGNATURES = {
     "ssmq_quantize_groups": (_i32, [_vp, _i32, _i64, _i64, _i64, _vp, _i32, _i32, _vp, _vp,
@@ -70,6 +79,7 @@ SIGNATURES = {
     "ssmq_ssd_workspace_size": (C.c_size_t, [C.POINTER(SSDArgs)]),
     "ssmq_ssd_chunk_scan_w8": (_i32, [C.POINTER(SSDArgs), _vp, C.c_size_t, _vp]),
     "ssmq_state_update_w8": (_i32, [C.POINTER(DecodeArgs), _vp]),
+    "ssmq_selective_state_update_w8": (_i32, [C.POINTER(M1DecodeArgs), _vp]),
     "ssmq_last_error": (C.c_char_p, []),
     "ssmq_version": (_i32, []),
 }
@@ -183,3 +193,8 @@ def ssmq_ssd_chunk_scan_w8(workspace=None, ws_bytes=0, stream=None, **fields):
 def ssmq_state_update_w8(stream=None, **fields):
     a = _fill(DecodeArgs, fields)
     _check(lib().ssmq_state_update_w8(C.byref(a), _stream(stream)))
+
+
+def ssmq_selective_state_update_w8(stream=None, **fields):
+    a = _fill(M1DecodeArgs, fields)
+    _check(lib().ssmq_selective_state_update_w8(C.byref(a), _stream(stream)))

@@ -122,3 +122,22 @@ def state_update(state, x, dt, A, B, C, B_scale, C_scale, state_group_size, *, x
                            z=z, B=B, C=C, B_scale=B_scale, C_scale=C_scale, state=state, y=y,
                            status=status)
     return y
+
+
+def selective_state_update(state, x, dt, A, B, C, B_scale, C_scale, state_group_size, *,
+                           x_group=None, x_scale=None, se_scale=0.0, se_log2_ratio=2, D=None,
+                           z=None, dt_bias=None, dt_softplus=True, y=None, status=None):
+    """One Mamba-1 decode step in place on ``state`` (b, d, N) fp32.  x, dt, z
+    (b, d); B, C (b, G, N); A (d, N).  Returns y (b, d) float16."""
+    b, d, Nst = state.shape
+    G = B.shape[1]
+    _dev_check(state, x, dt, A, B, C, B_scale, C_scale, x_group, x_scale, D, z, dt_bias)
+    if y is None:
+        y = torch.empty((b, d), dtype=torch.float16, device=state.device)
+    N.ssmq_selective_state_update_w8(batch=b, dim=d, dstate=Nst, ngroups=G,
+                                     state_group_size=state_group_size,
+                                     **_x_fields(x, x_group, x_scale, se_scale, se_log2_ratio),
+                                     dt=dt, dt_bias=dt_bias, dt_softplus=int(bool(dt_softplus)),
+                                     A=A, D=D, z=z, B=B, C=C, B_scale=B_scale, C_scale=C_scale,
+                                     state=state, y=y, status=status)
+    return y

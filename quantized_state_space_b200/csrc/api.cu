@@ -220,4 +220,30 @@ ssmq_status ssmq_state_update_w8(const ssmq_decode_args* a, void* stream) {
   return finish(ssmq::launch_state_update(*a, (cudaStream_t)stream), fn);
 }
 
+ssmq_status ssmq_selective_state_update_w8(const ssmq_m1_decode_args* a, void* stream) {
+  const char* fn = "ssmq_selective_state_update_w8";
+  REQUIRE(a != nullptr, SSMQ_ERR_INVALID_ARG, "%s: args is NULL", fn);
+  REQUIRE(a->batch >= 0 && a->dim >= 0, SSMQ_ERR_INVALID_ARG, "%s: negative size", fn);
+  REQUIRE(a->ngroups >= 1 && a->dim % a->ngroups == 0, SSMQ_ERR_INVALID_ARG,
+          "%s: dim must be a multiple of ngroups >= 1", fn);
+  REQUIRE(a->dstate == 4 || a->dstate == 8 || a->dstate == 16 || a->dstate == 32 ||
+              a->dstate == 64 || a->dstate == 128,
+          SSMQ_ERR_UNSUPPORTED, "%s: dstate %lld not in {4, 8, 16, 32, 64, 128}", fn,
+          (long long)a->dstate);
+  REQUIRE(a->state_group_size >= 1 && a->dstate % a->state_group_size == 0,
+          SSMQ_ERR_INVALID_ARG, "%s: dstate must be a multiple of state_group_size", fn);
+  if (a->batch == 0 || a->dim == 0) return SSMQ_OK;
+  const ssmq_status xs = check_x(a->x_format, a->x, a->x_group, a->x_scale, a->n_x_groups,
+                                 a->se_log2_ratio, fn);
+  if (xs != SSMQ_OK) return xs;
+  REQUIRE(a->dt && a->A && a->B && a->C && a->B_scale && a->C_scale && a->state && a->y,
+          SSMQ_ERR_INVALID_ARG, "%s: a required tensor is NULL", fn);
+  REQUIRE(aligned16(a->state) && aligned16(a->A) && aligned16(a->B) && aligned16(a->C),
+          SSMQ_ERR_ALIGNMENT, "%s: state, A, B and C must be 16-byte aligned", fn);
+  REQUIRE(a->batch * a->dim * (a->dstate / 4) <= 0x7fffffffLL * 256, SSMQ_ERR_UNSUPPORTED,
+          "%s: too many channels", fn);
+  if (injected(fn)) return fail(SSMQ_ERR_CUDA, "%s: injected launch failure", fn);
+  return finish(ssmq::launch_m1_state_update(*a, (cudaStream_t)stream), fn);
+}
+
 }  // extern "C"

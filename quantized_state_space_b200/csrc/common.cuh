@@ -12,6 +12,24 @@ constexpr float kLog2e = 1.4426950408889634f;
 __device__ __forceinline__ float h2f(uint16_t b) { return __half2float(__ushort_as_half(b)); }
 __device__ __forceinline__ uint16_t f2h(float v) { return __half_as_ushort(__float2half_rn(v)); }
 
+// int8 byte i of w as an exact fp32 value without a conversion instruction:
+// (q + 128) placed in the low mantissa of 2^23, then 2^23 + 128 subtracted.
+// xw must be w ^ 0x80808080.
+__device__ __forceinline__ float s8_to_f32(uint32_t xw, int i) {
+  return __int_as_float((int)__byte_perm(xw, 0x4B000000u, 0x7650u + (uint32_t)i)) - 8388736.0f;
+}
+// int8 bytes i and j of w as an exact binary16 pair: (q + 128) in the low
+// mantissa of 1024.0, then 1152 subtracted in half precision.  xw = w ^ 0x80808080.
+__device__ __forceinline__ __half2 s8x2_to_h2(uint32_t xw, int i, int j) {
+  const uint32_t bits = __byte_perm(xw, 0x64646464u, (uint32_t)(i | (4 << 4) | (j << 8) | (4 << 12)));
+  return __hsub2(*reinterpret_cast<const __half2*>(&bits), __float2half2_rn(1152.0f));
+}
+__device__ __forceinline__ uint32_t h2_bits(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
+// two fp32 values rounded to a packed binary16 pair (one instruction)
+__device__ __forceinline__ uint32_t pack_half2(float a, float b) {
+  return h2_bits(__floats2half2_rn(a, b));
+}
+
 // 2^x on the special-function unit (MUFU.EX2); ~2 ulp, subnormal results
 // flushed to zero.
 __device__ __forceinline__ float ex2_sfu(float x) {
@@ -64,6 +82,23 @@ __device__ __forceinline__ int quant_rne(float v, float step, int lim) {
   return max(-lim, min(lim, k));
 }
 
+// The same integer by a faster route.  rs is the correctly rounded binary32
+// reciprocal of step (step normal, rs finite).  y = fl32(v * rs) differs from
+// v / step by at most 2^-23 relative, i.e. by less than 2^-15 for |v / step|
+// <= 128, and fl32(v / step) lies within 2^-18 of v / step there.  So unless
+// y is within 2^-14 of a half-integer, y and fl32(v / step) round to the same
+// integer, and clamping before rounding commutes with the rule (every value
+// beyond +-lim rounds to at least lim).  Near a tie the exact division
+// decides.  v must be finite.
+__device__ __forceinline__ int quant_rne_fast(float v, float step, float rs, int lim) {
+  const float flim = (float)lim;
+  const float yc = fminf(fmaxf(v * rs, -flim), flim);
+  const float m = yc + 12582912.0f;  // 1.5 * 2^23: the sum rounds yc to an integer, ties to even
+  const float k = m - 12582912.0f;
+  if (fabsf(fabsf(yc - k) - 0.5f) < (1.0f / 16384.0f)) return quant_rne(v, step, lim);
+  return __float_as_int(m) - 0x4B400000;
+}
+
 // Soft-edge byte -> (payload, mode) with mode 0 standard, 1 small, 2 large.
 __device__ __forceinline__ void se_split(uint32_t c, int& q, int& mode) {
   if ((c & 0x80u) == 0u) {
@@ -79,15 +114,25 @@ __device__ __forceinline__ void se_split(uint32_t c, int& q, int& mode) {
 
 // Step sizes of the three soft-edge modes: {scale, scale / 2^r, scale * 2^r},
 // each one binary32 product.
+// rs[] are the correctly rounded reciprocals of s[] when s[] is a normal
+// number with a finite reciprocal, else 0 (which selects the exact division).
 struct SeSteps {
   float s[3];
+  float rs[3];
 };
-__host__ __device__ inline SeSteps se_steps(float scale, int log2_ratio) {
+__host__ __device__ inline bool usable_recip(float s, float r) {
+  return s >= 1.17549435e-38f && r > 0.0f && r <= 3.40282347e+38f && r >= 1.17549435e-38f;
+}
+__host__ inline SeSteps se_steps(float scale, int log2_ratio) {
   SeSteps st;
   const float f = (float)(1u << log2_ratio);
   st.s[0] = scale;
   st.s[1] = scale * (1.0f / f);
   st.s[2] = scale * f;
+  for (int i = 0; i < 3; ++i) {
+    const float r = 1.0f / st.s[i];
+    st.rs[i] = usable_recip(st.s[i], r) ? r : 0.0f;
+  }
   return st;
 }
 

@@ -165,3 +165,137 @@ cudaError_t launch_state_update(const ssmq_decode_args& a, cudaStream_t st) {
 }
 
 }  // namespace ssmq
+
+// ---------------------------------------------------------------------------
+// Mamba-1 form: A per (channel, state).  One thread per 4 states of a
+// (batch, channel); the N / 4 threads of a channel reduce C . h with
+// shuffles.  The state (b, d, N) is read and written once with 16-byte
+// accesses.
+namespace ssmq {
+namespace {
+
+struct M1DecParams {
+  int64_t units;  // b * d
+  int64_t d, G;
+  int gs;
+  int xfmt;
+  const void* x;
+  const int32_t* x_group;
+  const float* x_scale;
+  int n_x_groups;
+  SeSteps se;
+  const uint16_t* dt;
+  const float* dt_bias;
+  int softplus;
+  const float* A;
+  const float* D;
+  const uint16_t* z;
+  const int8_t* B;
+  const int8_t* C;
+  const float* B_scale;
+  const float* C_scale;
+  float* state;
+  uint16_t* y;
+  uint32_t* status;
+};
+
+template <int kN>
+__global__ void __launch_bounds__(256) m1_decode_kernel(const M1DecParams p) {
+  constexpr int LPC = kN / 4;
+  const int64_t gt = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int64_t u = gt / LPC;  // b * d + c
+  const int j = (int)(gt % LPC);
+  const bool ok = u < p.units;
+  uint32_t flags = 0;
+  float part = 0.0f, xv = 0.0f;
+  int64_t c = 0;
+  if (ok) {
+    const int64_t bb = u / p.d;
+    c = u % p.d;
+    const int64_t g = c * p.G / p.d;
+    const int spg = kN / p.gs;
+    if (p.xfmt == SSMQ_X_SOFTEDGE) {
+      xv = se_decode(static_cast<const uint8_t*>(p.x)[u], p.se);
+    } else {
+      const int xg = __ldg(p.x_group + c);
+      if ((unsigned)xg < (unsigned)p.n_x_groups)
+        xv = (float)static_cast<const int8_t*>(p.x)[u] * __ldg(p.x_scale + xg);
+      else
+        flags |= SSMQ_DEV_BAD_GROUP;
+    }
+    const float dv = h2f(p.dt[u]) + (p.dt_bias ? __ldg(p.dt_bias + c) : 0.0f);
+    const float delta = p.softplus ? softplus_f(dv) : dv;
+    const float dx = delta * xv;
+    const float4 a = __ldg(reinterpret_cast<const float4*>(p.A + c * kN) + j);
+    float4 h = *(reinterpret_cast<const float4*>(p.state + u * kN) + j);
+    const int64_t bo = (bb * p.G + g) * kN + 4 * j;
+    const char4 bq = *reinterpret_cast<const char4*>(p.B + bo);
+    const char4 cq = *reinterpret_cast<const char4*>(p.C + bo);
+    const float av[4] = {a.x, a.y, a.z, a.w};
+    const int8_t bqa[4] = {bq.x, bq.y, bq.z, bq.w};
+    const int8_t cqa[4] = {cq.x, cq.y, cq.z, cq.w};
+    float hv[4] = {h.x, h.y, h.z, h.w};
+#pragma unroll
+    for (int s = 0; s < 4; ++s) {
+      const int si = (int)g * spg + (4 * j + s) / p.gs;
+      const float bvv = (float)bqa[s] * __ldg(p.B_scale + si);
+      const float cvv = (float)cqa[s] * __ldg(p.C_scale + si);
+      hv[s] = fmaf(ex2_sfu(delta * av[s] * kLog2e), hv[s], dx * bvv);
+      part = fmaf(cvv, hv[s], part);
+    }
+    *(reinterpret_cast<float4*>(p.state + u * kN) + j) = make_float4(hv[0], hv[1], hv[2], hv[3]);
+  }
+#pragma unroll
+  for (int off = LPC / 2; off >= 1; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
+  if (ok && j == 0) {
+    float yv = part + (p.D ? __ldg(p.D + c) : 0.0f) * xv;
+    if (p.z) yv *= silu_f(h2f(p.z[u]));
+    p.y[u] = f2h(yv);
+  }
+  flag_status(p.status, flags);
+}
+
+}  // namespace
+
+cudaError_t launch_m1_state_update(const ssmq_m1_decode_args& a, cudaStream_t st) {
+  const int64_t units = a.batch * a.dim;
+  if (units == 0) return cudaSuccess;
+  M1DecParams p{};
+  p.units = units;
+  p.d = a.dim;
+  p.G = a.ngroups;
+  p.gs = a.state_group_size;
+  p.xfmt = a.x_format;
+  p.x = a.x;
+  p.x_group = a.x_group;
+  p.x_scale = a.x_scale;
+  p.n_x_groups = a.n_x_groups;
+  p.se = se_steps(a.se_scale, a.se_log2_ratio);
+  p.dt = a.dt;
+  p.dt_bias = a.dt_bias;
+  p.softplus = a.dt_softplus;
+  p.A = a.A;
+  p.D = a.D;
+  p.z = a.z;
+  p.B = a.B;
+  p.C = a.C;
+  p.B_scale = a.B_scale;
+  p.C_scale = a.C_scale;
+  p.state = a.state;
+  p.y = a.y;
+  p.status = a.status;
+  const int64_t threads = units * (a.dstate / 4);
+  const unsigned grid = (unsigned)((threads + 255) / 256);
+  switch (a.dstate) {
+    case 4: m1_decode_kernel<4><<<grid, 256, 0, st>>>(p); break;
+    case 8: m1_decode_kernel<8><<<grid, 256, 0, st>>>(p); break;
+    case 16: m1_decode_kernel<16><<<grid, 256, 0, st>>>(p); break;
+    case 32: m1_decode_kernel<32><<<grid, 256, 0, st>>>(p); break;
+    case 64: m1_decode_kernel<64><<<grid, 256, 0, st>>>(p); break;
+    case 128: m1_decode_kernel<128><<<grid, 256, 0, st>>>(p); break;
+    default: return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace ssmq

@@ -23,6 +23,7 @@ cudaError_t launch_softedge_decode(const uint8_t* codes, int64_t n, float scale,
 cudaError_t launch_selective_scan(const ssmq_scan_args& a, cudaStream_t st);
 
 cudaError_t launch_state_update(const ssmq_decode_args& a, cudaStream_t st);
+cudaError_t launch_m1_state_update(const ssmq_m1_decode_args& a, cudaStream_t st);
 
 size_t ssd_workspace_bytes(const ssmq_ssd_args& a);
 cudaError_t launch_ssd(const ssmq_ssd_args& a, void* ws, cudaStream_t st);

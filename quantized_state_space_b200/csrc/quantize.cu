@@ -52,7 +52,8 @@ __device__ __forceinline__ float load1(const void* src, Idx e) {
 }
 
 // One element of the static quantizer; flags record device-side anomalies.
-__device__ __forceinline__ int quant_elem(float v, float s, bool okg, uint32_t& flags) {
+// rs: reciprocal of s for the fast route, 0 to force the exact division.
+__device__ __forceinline__ int quant_elem(float v, float s, float rs, bool okg, uint32_t& flags) {
   if (!okg) {
     flags |= SSMQ_DEV_BAD_GROUP;
     return 0;
@@ -65,12 +66,106 @@ __device__ __forceinline__ int quant_elem(float v, float s, bool okg, uint32_t& 
     if (s != 0.0f) flags |= SSMQ_DEV_BAD_SCALE;
     return 0;
   }
-  return quant_rne(v, s, 127);
+  return rs != 0.0f ? quant_rne_fast(v, s, rs, 127) : quant_rne(v, s, 127);
+}
+
+// Per-CTA table of (scale, reciprocal) for small group counts.
+constexpr int kMaxTab = 256;
+__device__ __forceinline__ void fill_tab(const float* scales, int32_t n_groups, float2* tab) {
+  for (int g = threadIdx.x; g < n_groups && g < kMaxTab; g += blockDim.x) {
+    const float s = scales[g];
+    const float r = __frcp_rn(s);
+    tab[g] = make_float2(s, usable_recip(s, r) ? r : 0.0f);
+  }
+  __syncthreads();
+}
+__device__ __forceinline__ float2 tab_get(const float2* tab, const float* scales, int g,
+                                          int32_t n_groups) {
+  return n_groups <= kMaxTab ? tab[g] : make_float2(__ldg(scales + g), 0.0f);
 }
 
 __device__ __forceinline__ uint32_t pack4(int a, int b, int c, int d) {
   return (uint32_t)(a & 0xFF) | ((uint32_t)(b & 0xFF) << 8) | ((uint32_t)(c & 0xFF) << 16) |
          ((uint32_t)(d & 0xFF) << 24);
+}
+
+// Branch-free fast route for 16 elements sharing one valid (s, rs): the code
+// byte of each element is the low byte of fl32(clamp(v rs) + 1.5 2^23) (that
+// sum holds 0x4B400000 + k for the integer k = rne(clamp(v rs))).  Returns
+// false when an element is non-finite or lies within 2^-14 of a tie, in which
+// case the caller redoes the vector element by element.
+__device__ __forceinline__ bool quant16_fast(const float (&x)[kVec], float rs, uint4& out) {
+  uint32_t mb[kVec];
+  bool bad = false;
+#pragma unroll
+  for (int i = 0; i < kVec; ++i) {
+    bad |= !(fabsf(x[i]) <= 3.402823466e38f);
+    const float yc = fminf(fmaxf(x[i] * rs, -127.0f), 127.0f);
+    const float m = yc + 12582912.0f;
+    bad |= fabsf(fabsf(yc - (m - 12582912.0f)) - 0.5f) < (1.0f / 16384.0f);
+    mb[i] = __float_as_uint(m);
+  }
+  out.x = __byte_perm(__byte_perm(mb[0], mb[1], 0x0040), __byte_perm(mb[2], mb[3], 0x0040), 0x5410);
+  out.y = __byte_perm(__byte_perm(mb[4], mb[5], 0x0040), __byte_perm(mb[6], mb[7], 0x0040), 0x5410);
+  out.z = __byte_perm(__byte_perm(mb[8], mb[9], 0x0040), __byte_perm(mb[10], mb[11], 0x0040), 0x5410);
+  out.w = __byte_perm(__byte_perm(mb[12], mb[13], 0x0040), __byte_perm(mb[14], mb[15], 0x0040), 0x5410);
+  return !bad;
+}
+
+// One full 16-element vector of the static quantizer.
+template <bool kF16, int kPath, typename Idx>
+__device__ __forceinline__ void quant_vec(const float (&x)[kVec], Idx e0, Idx mid, Idx inner,
+                                          const int32_t* __restrict__ gmap, int32_t n_groups,
+                                          const float* __restrict__ scales, const float2* tab,
+                                          const int* ugrp, int8_t* __restrict__ q,
+                                          uint32_t& flags) {
+  int gu = -1;  // one group for the whole vector, if known
+  if (kPath == kPathRow) {
+    gu = __ldg(gmap + (e0 / inner) % mid);
+  } else if (kPath == kPathCol && ugrp) {
+    gu = ugrp[(e0 % mid) >> 4];
+  }
+  if ((unsigned)gu < (unsigned)n_groups) {
+    const float2 sr = tab_get(tab, scales, gu, n_groups);
+    uint4 o;
+    if (sr.y != 0.0f && quant16_fast(x, sr.y, o)) {
+      *reinterpret_cast<uint4*>(q + e0) = o;
+      return;
+    }
+  }
+  int r[kVec];
+#pragma unroll
+  for (int i = 0; i < kVec; ++i) {
+    const int g = gu >= 0 || kPath == kPathRow
+                      ? gu
+                      : (kPath == kPathCol ? __ldg(gmap + e0 % mid + i)
+                                           : __ldg(gmap + ((e0 + i) / inner) % mid));
+    const bool okg = (unsigned)g < (unsigned)n_groups;
+    const float2 sr = okg ? tab_get(tab, scales, g, n_groups) : make_float2(0.0f, 0.0f);
+    r[i] = quant_elem(x[i], sr.x, sr.y, okg, flags);
+  }
+  uint4 o;
+  o.x = pack4(r[0], r[1], r[2], r[3]);
+  o.y = pack4(r[4], r[5], r[6], r[7]);
+  o.z = pack4(r[8], r[9], r[10], r[11]);
+  o.w = pack4(r[12], r[13], r[14], r[15]);
+  *reinterpret_cast<uint4*>(q + e0) = o;
+}
+
+// Column path (inner == 1, mid % 16 == 0): groups of 16 consecutive columns
+// that share one group id are marked in a per-CTA table (-1 otherwise).
+constexpr int kMaxU = 1024;
+__device__ __forceinline__ const int* fill_ugrp(const int32_t* gmap, uint64_t mid, int* ug) {
+  const uint64_t nu = mid / kVec;
+  if (nu > (uint64_t)kMaxU) return nullptr;
+  for (uint64_t u = threadIdx.x; u < nu; u += blockDim.x) {
+    const int g0 = __ldg(gmap + u * kVec);
+    bool same = true;
+    for (int i = 1; i < kVec; ++i) same &= __ldg(gmap + u * kVec + i) == g0;
+    ug[u] = same ? g0 : -1;
+  }
+  __syncthreads();
+  return ug;
 }
 
 template <bool kF16, int kPath, typename Idx>
@@ -79,47 +174,37 @@ __global__ void __launch_bounds__(kThreads)
                         const int32_t* __restrict__ gmap, int32_t n_groups,
                         const float* __restrict__ scales, int8_t* __restrict__ q,
                         uint32_t* status) {
+  __shared__ float2 tab[kMaxTab];
+  __shared__ int ug_s[kPath == kPathCol ? kMaxU : 1];
+  fill_tab(scales, n_groups, tab);
+  const int* ugrp = kPath == kPathCol ? fill_ugrp(gmap, (uint64_t)mid, ug_s) : nullptr;
   uint32_t flags = 0;
   const Idx nvec = (n + kVec - 1) / kVec;
-  for (Idx v = (Idx)blockIdx.x * kThreads + threadIdx.x; v < nvec; v += (Idx)gridDim.x * kThreads) {
-    const Idx e0 = v * kVec;
-    if (e0 + kVec <= n) {
-      float x[kVec];
-      load16<kF16>(src, e0, x);
-      int r[kVec];
-      if (kPath == kPathRow) {
-        const int g = __ldg(gmap + (e0 / inner) % mid);
-        const bool okg = (unsigned)g < (unsigned)n_groups;
-        const float s = okg ? __ldg(scales + g) : 0.0f;
+  const Idx stride = (Idx)gridDim.x * kThreads;
+  // two vectors in flight per thread
+  for (Idx v0 = (Idx)blockIdx.x * kThreads + threadIdx.x; v0 < nvec; v0 += 2 * stride) {
+    const Idx v1 = v0 + stride;
+    const bool f0 = v0 * kVec + kVec <= n;
+    const bool h1 = v1 < nvec;
+    const bool f1 = h1 && v1 * kVec + kVec <= n;
+    float x0[kVec], x1[kVec];
+    if (f0) load16<kF16>(src, v0 * kVec, x0);
+    if (f1) load16<kF16>(src, v1 * kVec, x1);
 #pragma unroll
-        for (int i = 0; i < kVec; ++i) r[i] = quant_elem(x[i], s, okg, flags);
-      } else if (kPath == kPathCol) {
-        const Idx m0 = e0 % mid;
-#pragma unroll
-        for (int i = 0; i < kVec; ++i) {
-          const int g = __ldg(gmap + m0 + i);
-          const bool okg = (unsigned)g < (unsigned)n_groups;
-          r[i] = quant_elem(x[i], okg ? __ldg(scales + g) : 0.0f, okg, flags);
-        }
+    for (int w = 0; w < 2; ++w) {
+      const Idx v = w ? v1 : v0;
+      if (w && !h1) break;
+      const Idx e0 = v * kVec;
+      if (w ? f1 : f0) {
+        quant_vec<kF16, kPath, Idx>(w ? x1 : x0, e0, mid, inner, gmap, n_groups, scales, tab,
+                                    ugrp, q, flags);
       } else {
-#pragma unroll
-        for (int i = 0; i < kVec; ++i) {
-          const int g = __ldg(gmap + ((e0 + i) / inner) % mid);
+        for (Idx e = e0; e < n; ++e) {
+          const int g = __ldg(gmap + (e / inner) % mid);
           const bool okg = (unsigned)g < (unsigned)n_groups;
-          r[i] = quant_elem(x[i], okg ? __ldg(scales + g) : 0.0f, okg, flags);
+          q[e] = (int8_t)quant_elem(load1<kF16>(src, e), okg ? __ldg(scales + g) : 0.0f, 0.0f,
+                                    okg, flags);
         }
-      }
-      uint4 o;
-      o.x = pack4(r[0], r[1], r[2], r[3]);
-      o.y = pack4(r[4], r[5], r[6], r[7]);
-      o.z = pack4(r[8], r[9], r[10], r[11]);
-      o.w = pack4(r[12], r[13], r[14], r[15]);
-      *reinterpret_cast<uint4*>(q + e0) = o;
-    } else {
-      for (Idx e = e0; e < n; ++e) {
-        const int g = __ldg(gmap + (e / inner) % mid);
-        const bool okg = (unsigned)g < (unsigned)n_groups;
-        q[e] = (int8_t)quant_elem(load1<kF16>(src, e), okg ? __ldg(scales + g) : 0.0f, okg, flags);
       }
     }
   }
@@ -256,9 +341,43 @@ __device__ __forceinline__ uint32_t se_encode1(float v, float lo, float hi, cons
   const int mode = a < lo ? 1 : (a > hi ? 2 : 0);
   const float step = st.s[mode];
   const int lim = mode == 0 ? 63 : 31;
-  const int qv = (step > 0.0f && isfinite(step)) ? quant_rne(v, step, lim) : 0;
+  const float rs = st.rs[mode];
+  const int qv = (step > 0.0f && isfinite(step))
+                     ? (rs != 0.0f ? quant_rne_fast(v, step, rs, lim) : quant_rne(v, step, lim))
+                     : 0;
   if (mode == 0) return (uint32_t)(qv & 0x7F);
   return (mode == 1 ? 0x80u : 0xC0u) | (uint32_t)(qv & 0x3F);
+}
+
+// Branch-free fast route for 16 soft-edge codes: mode by compares, then the
+// quantizer's reciprocal + magic-number rounding with the mode's step and
+// clamp; the payload bits are the low bits of the rounding sum, masked to the
+// mode's width and or-ed with its prefix.  Returns false when an element is
+// non-finite, a mode's reciprocal is unusable, or an element lies within
+// 2^-14 of a rounding tie; the caller then encodes the vector element-wise.
+__device__ __forceinline__ bool se16_fast(const float (&x)[kVec], float lo, float hi,
+                                          const SeSteps& st, uint4& out) {
+  uint32_t cb[kVec];
+  bool bad = !(st.rs[0] != 0.0f && st.rs[1] != 0.0f && st.rs[2] != 0.0f);
+#pragma unroll
+  for (int i = 0; i < kVec; ++i) {
+    const float a = fabsf(x[i]);
+    bad |= !(a <= 3.402823466e38f);
+    const bool sm = a < lo, lg = a > hi;
+    const float rs = sm ? st.rs[1] : (lg ? st.rs[2] : st.rs[0]);
+    const float lim = (sm || lg) ? 31.0f : 63.0f;
+    const float yc = fminf(fmaxf(x[i] * rs, -lim), lim);
+    const float m = yc + 12582912.0f;
+    bad |= fabsf(fabsf(yc - (m - 12582912.0f)) - 0.5f) < (1.0f / 16384.0f);
+    const uint32_t mask = (sm || lg) ? 0x3Fu : 0x7Fu;
+    const uint32_t prefix = sm ? 0x80u : (lg ? 0xC0u : 0x00u);
+    cb[i] = (__float_as_uint(m) & mask) | prefix;
+  }
+  out.x = __byte_perm(__byte_perm(cb[0], cb[1], 0x0040), __byte_perm(cb[2], cb[3], 0x0040), 0x5410);
+  out.y = __byte_perm(__byte_perm(cb[4], cb[5], 0x0040), __byte_perm(cb[6], cb[7], 0x0040), 0x5410);
+  out.z = __byte_perm(__byte_perm(cb[8], cb[9], 0x0040), __byte_perm(cb[10], cb[11], 0x0040), 0x5410);
+  out.w = __byte_perm(__byte_perm(cb[12], cb[13], 0x0040), __byte_perm(cb[14], cb[15], 0x0040), 0x5410);
+  return !bad;
 }
 
 template <bool kF16, typename Idx>
@@ -267,21 +386,38 @@ __global__ void __launch_bounds__(kThreads)
                      uint8_t* __restrict__ codes, uint32_t* status) {
   uint32_t flags = 0;
   const Idx nvec = (n + kVec - 1) / kVec;
-  for (Idx v = (Idx)blockIdx.x * kThreads + threadIdx.x; v < nvec; v += (Idx)gridDim.x * kThreads) {
-    const Idx e0 = v * kVec;
-    if (e0 + kVec <= n) {
-      float x[kVec];
-      load16<kF16>(src, e0, x);
-      uint32_t w[4];
+  const Idx stride = (Idx)gridDim.x * kThreads;
+  for (Idx v0 = (Idx)blockIdx.x * kThreads + threadIdx.x; v0 < nvec; v0 += 2 * stride) {
+    const Idx v1 = v0 + stride;
+    const bool f0 = v0 * kVec + kVec <= n;
+    const bool h1 = v1 < nvec;
+    const bool f1 = h1 && v1 * kVec + kVec <= n;
+    float x0[kVec], x1[kVec];
+    if (f0) load16<kF16>(src, v0 * kVec, x0);
+    if (f1) load16<kF16>(src, v1 * kVec, x1);
 #pragma unroll
-      for (int k = 0; k < 4; ++k)
-        w[k] = se_encode1(x[4 * k], lo, hi, st, flags) |
-               (se_encode1(x[4 * k + 1], lo, hi, st, flags) << 8) |
-               (se_encode1(x[4 * k + 2], lo, hi, st, flags) << 16) |
-               (se_encode1(x[4 * k + 3], lo, hi, st, flags) << 24);
-      *reinterpret_cast<uint4*>(codes + e0) = make_uint4(w[0], w[1], w[2], w[3]);
-    } else {
-      for (Idx e = e0; e < n; ++e) codes[e] = (uint8_t)se_encode1(load1<kF16>(src, e), lo, hi, st, flags);
+    for (int w = 0; w < 2; ++w) {
+      if (w && !h1) break;
+      const Idx e0 = (w ? v1 : v0) * kVec;
+      if (w ? f1 : f0) {
+        const float(&x)[kVec] = w ? x1 : x0;
+        uint4 fast;
+        if (se16_fast(x, lo, hi, st, fast)) {
+          *reinterpret_cast<uint4*>(codes + e0) = fast;
+          continue;
+        }
+        uint32_t wd[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          wd[k] = se_encode1(x[4 * k], lo, hi, st, flags) |
+                  (se_encode1(x[4 * k + 1], lo, hi, st, flags) << 8) |
+                  (se_encode1(x[4 * k + 2], lo, hi, st, flags) << 16) |
+                  (se_encode1(x[4 * k + 3], lo, hi, st, flags) << 24);
+        *reinterpret_cast<uint4*>(codes + e0) = make_uint4(wd[0], wd[1], wd[2], wd[3]);
+      } else {
+        for (Idx e = e0; e < n; ++e)
+          codes[e] = (uint8_t)se_encode1(load1<kF16>(src, e), lo, hi, st, flags);
+      }
     }
   }
   flag_status(status, flags);

@@ -13,19 +13,20 @@
 // Work decomposition.  Every (b, c, n) recurrence is owned by one thread from
 // t = 0 to L - 1, so each decay exp(delta A) is evaluated exactly once and no
 // carry pass is needed.  A CTA owns kCH channels of one batch row and one B/C
-// group and walks L in chunks of kT = 64 steps:
-//   phase A  all threads stage the chunk: 16-byte loads of x codes and of
-//            binary16 dt / z, dequantisation, softplus, silu, D x; B and C
-//            rows are loaded as int8, dequantised once per (t, n) and
-//            transposed into shared memory as [t][n] fp32 (shared by all
-//            channels of the CTA);
-//   phase B  thread (c, j) advances states 4j..4j+3 of channel c through the
-//            chunk: one MUFU.EX2 per state update, the rest FMA; the
-//            per-thread partial sums of C . h are combined across the
+// group and walks L in chunks of kT = 64 steps.  The raw bytes of chunk k + 1
+// (x codes, binary16 dt / z, int8 B / C rows) are fetched with cp.async into
+// a second shared-memory buffer while chunk k is scanned, so the recurrence
+// never waits on global memory.  Per chunk:
+//   stage    all threads turn the raw bytes of the chunk into (delta, delta x)
+//            per (c, t) and dequantised B, C rows laid out [t][n] (shared by
+//            every channel of the CTA);
+//   scan     thread (c, j) advances states 4j..4j+3 of channel c: one
+//            MUFU.EX2 per state update and packed fp32x2 FMA for the rest;
+//            the per-thread partial sums of C . h are combined across the
 //            N / 4 threads of a channel by a shuffle reduce-scatter, so each
 //            thread ends up owning the full y of one time step;
-//   phase C  all threads apply (y + D x) * silu(z) and store binary16 y with
-//            16-byte stores.
+//   store    all threads apply (y + D x) * silu(z) from the raw bytes and
+//            store binary16 y with 16-byte stores.
 // The state stays in registers across chunks; the final state is written once.
 #include "common.cuh"
 #include "internal.h"
@@ -34,8 +35,7 @@ namespace ssmq {
 namespace {
 
 constexpr int kT = 64;    // time steps per chunk
-constexpr int kSeg = 16;  // time steps per staging work item
-constexpr int kSPL = 4;   // states per thread
+constexpr int kSeg = 16;  // time steps per staging work item (16 bytes of codes)
 
 struct M1Params {
   int64_t b, L, d, G;
@@ -63,30 +63,27 @@ struct M1Params {
   int vec_ok;
 };
 
-__device__ __forceinline__ void load_u8x16(const uint8_t* p, int cnt, bool vec, uint8_t (&o)[16]) {
-  if (vec && cnt == 16) {
-    const uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-    for (int i = 0; i < 16; ++i) o[i] = (uint8_t)(w[i >> 2] >> (8 * (i & 3)));
-  } else {
-#pragma unroll
-    for (int i = 0; i < 16; ++i) o[i] = i < cnt ? p[i] : (uint8_t)0;
-  }
+// ---- packed fp32x2 arithmetic (sm_100) ------------------------------------
+__device__ __forceinline__ uint64_t pk(float2 v) { return *reinterpret_cast<uint64_t*>(&v); }
+__device__ __forceinline__ float2 upk(uint64_t v) { return *reinterpret_cast<float2*>(&v); }
+__device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(pk(a)), "l"(pk(b)));
+  return upk(d);
+}
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(pk(a)), "l"(pk(b)), "l"(pk(c)));
+  return upk(d);
 }
 
-__device__ __forceinline__ void load_h16(const uint16_t* p, int cnt, bool vec, uint16_t (&o)[16]) {
-  if (vec && cnt == 16) {
-    const uint4 a = __ldg(reinterpret_cast<const uint4*>(p));
-    const uint4 b = __ldg(reinterpret_cast<const uint4*>(p) + 1);
-    const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-#pragma unroll
-    for (int i = 0; i < 16; ++i) o[i] = (uint16_t)(w[i >> 1] >> (16 * (i & 1)));
-  } else {
-#pragma unroll
-    for (int i = 0; i < 16; ++i) o[i] = i < cnt ? p[i] : (uint16_t)0;
-  }
+// ---- cp.async (16-byte, L2-only) -------------------------------------------
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc) {
+  const uint32_t s = (uint32_t)__cvta_generic_to_shared(smem_dst);
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(s), "l"(gsrc) : "memory");
 }
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 
 // Reduce-scatter over the LPC consecutive lanes of a channel: on entry each
 // lane holds LPC partial sums (one per time step of the group); on exit lane
@@ -106,19 +103,88 @@ __device__ __forceinline__ float reduce_scatter(float (&p)[LPC], int j) {
   return p[0];
 }
 
-template <int kN, int kCH, int kXFmt>
+// Raw bytes of one chunk, as fetched from global memory.
+template <int kN, int kCH>
+struct Raw {
+  uint8_t x[kCH][kT];
+  uint16_t dt[kCH][kT];
+  uint16_t z[kCH][kT];
+  int8_t B[kN][kT];
+  int8_t C[kN][kT];
+};
+
+template <int kN, int kCH>
+struct M1Smem {
+  Raw<kN, kCH> raw[2];                  // double-buffered raw bytes
+  __align__(16) float2 dd[kCH][kT + 2]; // (delta, delta x); 16-byte rows
+  __align__(16) float b[kT][kN];        // dequantised B, [t][n]
+  __align__(16) float c[kT][kN];        // dequantised C, [t][n]
+  float y[kCH][kT + 4];                 // C . h per (c, t)
+};
+
+template <int kN, int kCH>
+__device__ __forceinline__ void fetch_chunk(const M1Params& p, Raw<kN, kCH>& r, int64_t bb, int g,
+                                            int c0, int nc, int64_t t0, int tl, int tid, int NT) {
+  constexpr int SEGS = kT / kSeg;
+  const int64_t d = p.d, L = p.L;
+  if (p.vec_ok) {
+    // every row starts 16-byte aligned (L % 16 == 0): 16-byte cp.async pieces
+    for (int w = tid; w < kCH * SEGS; w += NT) {
+      const int c = w / SEGS, tb = (w % SEGS) * kSeg;
+      if (c >= nc || tb >= tl) continue;
+      const int64_t row = (bb * d + c0 + c) * L + t0 + tb;
+      cp_async16(&r.x[c][tb], static_cast<const uint8_t*>(p.x) + row);
+      cp_async16(&r.dt[c][tb], p.dt + row);
+      cp_async16(&r.dt[c][tb + 8], p.dt + row + 8);
+      if (p.z) {
+        cp_async16(&r.z[c][tb], p.z + row);
+        cp_async16(&r.z[c][tb + 8], p.z + row + 8);
+      }
+    }
+    for (int w = tid; w < 2 * kN * SEGS; w += NT) {
+      const int which = w / (kN * SEGS), rem = w % (kN * SEGS);
+      const int n = rem % kN, tb = (rem / kN) * kSeg;
+      if (tb >= tl) continue;
+      const int64_t row = ((bb * p.G + g) * kN + n) * L + t0 + tb;
+      cp_async16(which ? &r.C[n][tb] : &r.B[n][tb], (which ? p.C : p.B) + row);
+    }
+  } else {
+    // rows not 16-byte aligned: plain element loads, bounded by the row end
+    for (int w = tid; w < kCH * kT; w += NT) {
+      const int c = w / kT, t = w % kT;
+      if (c >= nc || t >= tl) continue;
+      const int64_t row = (bb * d + c0 + c) * L + t0 + t;
+      r.x[c][t] = static_cast<const uint8_t*>(p.x)[row];
+      r.dt[c][t] = p.dt[row];
+      if (p.z) r.z[c][t] = p.z[row];
+    }
+    for (int w = tid; w < 2 * kN * kT; w += NT) {
+      const int which = w / (kN * kT), rem = w % (kN * kT);
+      const int n = rem / kT, t = rem % kT;
+      if (t >= tl) continue;
+      const int64_t row = ((bb * p.G + g) * kN + n) * L + t0 + t;
+      (which ? r.C : r.B)[n][t] = (which ? p.C : p.B)[row];
+    }
+  }
+}
+
+template <int kN, int kCH, int kSPL, int kXFmt>
 __global__ void __launch_bounds__(kCH * (kN / kSPL))
     m1_scan_kernel(const M1Params p) {
+  static_assert(kSPL == 2 || kSPL == 4, "2 or 4 states per thread");
+  constexpr int NP = kSPL / 2;  // fp32x2 pairs per thread
   constexpr int LPC = kN / kSPL;
   constexpr int NT = kCH * LPC;
-  constexpr int RW = kT + 1;   // float2 row: conflict-free column reads in phase B
+  constexpr int RW = kT + 2;   // float2 row: 16-byte aligned, conflict-free column reads
   constexpr int RY = kT + 4;   // float row of the reduced sums
   constexpr int SEGS = kT / kSeg;
-  __shared__ float2 sDD[kCH][RW];  // (delta, delta * x)
-  __shared__ float2 sEP[kCH][RW];  // (D * x, silu(z) or 1)
-  __shared__ __align__(16) float sB[kT][kN];
-  __shared__ __align__(16) float sC[kT][kN];
-  __shared__ float sY[kCH][RY];
+  extern __shared__ __align__(16) uint8_t smem_bytes[];
+  M1Smem<kN, kCH>& S = *reinterpret_cast<M1Smem<kN, kCH>*>(smem_bytes);
+  Raw<kN, kCH>* raw = S.raw;
+  float2 (*sDD)[RW] = S.dd;  // (delta, delta * x)
+  float (*sB)[kN] = S.b;
+  float (*sC)[kN] = S.c;
+  float (*sY)[RY] = S.y;
 
   const int tid = threadIdx.x;
   const int64_t bb = blockIdx.y;
@@ -128,38 +194,96 @@ __global__ void __launch_bounds__(kCH * (kN / kSPL))
   const int c0 = g * dg + (blockIdx.x % p.n_ctile) * kCH;
   const int nc = min(kCH, g * dg + dg - c0);
   const int spg = kN / p.gs;
-  const bool vec = p.vec_ok != 0;
   uint32_t flags = 0;
 
-  // scan role
+  // scan role: channel lc, states 4 lj .. 4 lj + 3
   const int lc = tid / LPC, lj = tid % LPC;
   const bool lvalid = lc < nc;
   const int64_t lch = c0 + lc;
-  float h[kSPL], a2[kSPL];
+  float2 hp[NP], ap[NP];  // states 2i, 2i+1 of this thread's block of kSPL
 #pragma unroll
-  for (int s = 0; s < kSPL; ++s) {
-    const int n = lj * kSPL + s;
-    a2[s] = lvalid ? __ldg(p.A + lch * kN + n) * kLog2e : 0.0f;
-    h[s] = (lvalid && p.h0) ? __ldg(p.h0 + (bb * d + lch) * kN + n) : 0.0f;
+  for (int i = 0; i < NP; ++i) {
+    const int n = lj * kSPL + 2 * i;
+    ap[i] = lvalid ? make_float2(__ldg(p.A + lch * kN + n) * kLog2e, __ldg(p.A + lch * kN + n + 1) * kLog2e)
+                   : make_float2(0.0f, 0.0f);
+    hp[i] = (lvalid && p.h0) ? make_float2(__ldg(p.h0 + (bb * d + lch) * kN + n),
+                                           __ldg(p.h0 + (bb * d + lch) * kN + n + 1))
+                             : make_float2(0.0f, 0.0f);
   }
 
-  for (int64_t t0 = 0; t0 < L; t0 += kT) {
-    const int tl = (int)min((int64_t)kT, L - t0);
+  // per-channel constants of the staging role (item c = w / SEGS is fixed
+  // across chunks when NT is a multiple of kCH * SEGS or larger)
+  const int nchunks = (int)((L + kT - 1) / kT);
+  fetch_chunk<kN, kCH>(p, raw[0], bb, g, c0, nc, 0, (int)min((int64_t)kT, L), tid, NT);
+  cp_async_commit();
 
-    // ---- phase A: x, dt, z -> (delta, delta x) and (D x, gate)
+  // y = (C . h + D x) * silu(z) of chunk kk, binary16, from its raw bytes
+  auto store_chunk = [&](int kk) {
+    const int64_t t0 = (int64_t)kk * kT;
+    const int tl = (int)min((int64_t)kT, L - t0);
+    Raw<kN, kCH>& r = raw[kk & 1];
     for (int w = tid; w < kCH * SEGS; w += NT) {
       const int c = w / SEGS, tb = (w % SEGS) * kSeg;
-      float2 dd[kSeg], ep[kSeg];
-      if (c < nc && tb < tl) {
+      if (c >= nc || tb >= tl) continue;
+      const int64_t ch = c0 + c;
+      float xs = 1.0f;
+      if (kXFmt == SSMQ_X_INT8_GROUP) {
+        const int xg = __ldg(p.x_group + ch);
+        xs = (unsigned)xg < (unsigned)p.n_x_groups ? __ldg(p.x_scale + xg) : 0.0f;
+      }
+      const float Dc = p.D ? __ldg(p.D + ch) : 0.0f;
+      const int cnt = min(kSeg, tl - tb);
+      const uint4 xw = *reinterpret_cast<const uint4*>(&r.x[c][tb]);
+      const uint32_t xb[4] = {xw.x, xw.y, xw.z, xw.w};
+      uint32_t zw[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+      if (p.z) {
+        const uint4 z0 = *reinterpret_cast<const uint4*>(&r.z[c][tb]);
+        const uint4 z1 = *reinterpret_cast<const uint4*>(&r.z[c][tb + 8]);
+        zw[0] = z0.x; zw[1] = z0.y; zw[2] = z0.z; zw[3] = z0.w;
+        zw[4] = z1.x; zw[5] = z1.y; zw[6] = z1.z; zw[7] = z1.w;
+      }
+      uint32_t wv[kSeg / 2];
+#pragma unroll
+      for (int i = 0; i < kSeg; i += 2) {
+        float yv[2];
+        const float2 zf = __half22float2(*reinterpret_cast<const __half2*>(&zw[i >> 1]));
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int t = i + e;
+          const uint32_t code = (xb[t >> 2] >> (8 * (t & 3))) & 0xFFu;
+          const float xv = kXFmt == SSMQ_X_INT8_GROUP ? s8_to_f32(xb[t >> 2] ^ 0x80808080u, t & 3) * xs
+                                                      : se_decode(code, p.se);
+          float v = fmaf(Dc, xv, sY[c][tb + t]);
+          if (p.z) v *= silu_f(e ? zf.y : zf.x);
+          yv[e] = v;
+        }
+        wv[i / 2] = pack_half2(yv[0], yv[1]);
+      }
+      uint16_t* dst = p.y + (bb * d + ch) * L + t0 + tb;
+      if (p.vec_ok && cnt == kSeg) {
+        uint4* o = reinterpret_cast<uint4*>(dst);
+        o[0] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+        o[1] = make_uint4(wv[4], wv[5], wv[6], wv[7]);
+      } else {
+        for (int i = 0; i < cnt; ++i) dst[i] = (uint16_t)(wv[i / 2] >> (16 * (i & 1)));
+      }
+    }
+    };
+
+  for (int k = 0; k < nchunks; ++k) {
+    const int64_t t0 = (int64_t)k * kT;
+    const int tl = (int)min((int64_t)kT, L - t0);
+    Raw<kN, kCH>& r = raw[k & 1];
+    cp_async_wait_all();
+    __syncthreads();  // raw bytes of chunk k landed; the scan of chunk k - 1 is complete
+    if (k > 0) store_chunk(k - 1);  // reads sY and the raw bytes of chunk k - 1 only
+
+    // ---- stage: (delta, delta x) per (c, t); B, C dequantised to [t][n]
+    for (int w = tid; w < kCH * SEGS; w += NT) {
+      const int c = w / SEGS, tb = (w % SEGS) * kSeg;
+      float xs = 1.0f, bias = 0.0f;
+      if (c < nc) {
         const int64_t ch = c0 + c;
-        const int64_t row = (bb * d + ch) * L + t0 + tb;
-        const int cnt = min(kSeg, tl - tb);
-        uint8_t xq[kSeg];
-        uint16_t dtb[kSeg], zb[kSeg];
-        load_u8x16(static_cast<const uint8_t*>(p.x) + row, cnt, vec, xq);
-        load_h16(p.dt + row, cnt, vec, dtb);
-        if (p.z) load_h16(p.z + row, cnt, vec, zb);
-        float xs = 1.0f;
         if (kXFmt == SSMQ_X_INT8_GROUP) {
           const int xg = __ldg(p.x_group + ch);
           if ((unsigned)xg < (unsigned)p.n_x_groups) {
@@ -169,122 +293,116 @@ __global__ void __launch_bounds__(kCH * (kN / kSPL))
             flags |= SSMQ_DEV_BAD_GROUP;
           }
         }
-        const float bias = p.dt_bias ? __ldg(p.dt_bias + ch) : 0.0f;
-        const float Dc = p.D ? __ldg(p.D + ch) : 0.0f;
+        bias = p.dt_bias ? __ldg(p.dt_bias + ch) : 0.0f;
+      }
+      const uint4 xw = *reinterpret_cast<const uint4*>(&r.x[c][tb]);
+      const uint32_t xb[4] = {xw.x, xw.y, xw.z, xw.w};
+      const uint4 d0 = *reinterpret_cast<const uint4*>(&r.dt[c][tb]);
+      const uint4 d1 = *reinterpret_cast<const uint4*>(&r.dt[c][tb + 8]);
+      const uint32_t dw[8] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w};
+      float4 out[kSeg / 2];
 #pragma unroll
-        for (int i = 0; i < kSeg; ++i) {
-          float xv;
-          if (kXFmt == SSMQ_X_INT8_GROUP)
-            xv = (float)(int8_t)xq[i] * xs;
-          else
-            xv = se_decode(xq[i], p.se);
-          const float dv = h2f(dtb[i]) + bias;
+      for (int i = 0; i < kSeg; i += 2) {
+        float dd[2], dx[2];
+        const float2 dtf = __half22float2(*reinterpret_cast<const __half2*>(&dw[i >> 1]));
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int t = i + e;
+          const uint32_t code = (xb[t >> 2] >> (8 * (t & 3))) & 0xFFu;
+          const float xv = kXFmt == SSMQ_X_INT8_GROUP ? s8_to_f32(xb[t >> 2] ^ 0x80808080u, t & 3) * xs
+                                                      : se_decode(code, p.se);
+          const float dv = (e ? dtf.y : dtf.x) + bias;
           float delta = p.softplus ? softplus_f(dv) : dv;
-          if (i >= cnt) delta = 0.0f;
-          dd[i] = make_float2(delta, delta * xv);
-          ep[i] = make_float2(Dc * xv, p.z ? silu_f(h2f(zb[i])) : 1.0f);
+          if (c >= nc || tb + t >= tl) delta = 0.0f;
+          dd[e] = delta;
+          dx[e] = delta * xv;
         }
-      } else {
-#pragma unroll
-        for (int i = 0; i < kSeg; ++i) {
-          dd[i] = make_float2(0.0f, 0.0f);
-          ep[i] = make_float2(0.0f, 0.0f);
-        }
+        out[i / 2] = make_float4(dd[0], dx[0], dd[1], dx[1]);
       }
+      float4* dst = reinterpret_cast<float4*>(&sDD[c][tb]);
 #pragma unroll
-      for (int i = 0; i < kSeg; ++i) {
-        sDD[c][tb + i] = dd[i];
-        sEP[c][tb + i] = ep[i];
-      }
+      for (int i = 0; i < kSeg / 2; ++i) dst[i] = out[i];
     }
-    // ---- phase A: B and C rows of group g -> [t][n] fp32
     for (int w = tid; w < 2 * kN * SEGS; w += NT) {
-      const int which = w / (kN * SEGS);
-      const int rem = w % (kN * SEGS);
-      const int n = rem / SEGS, tb = (rem % SEGS) * kSeg;
-      const int cnt = max(0, min(kSeg, tl - tb));
-      const int8_t* base = which ? p.C : p.B;
+      const int which = w / (kN * SEGS), rem = w % (kN * SEGS);
+      const int n = rem % kN, tb = (rem / kN) * kSeg;
       const float sc = __ldg((which ? p.C_scale : p.B_scale) + g * spg + n / p.gs);
-      uint8_t q[kSeg];
-      if (cnt > 0)
-        load_u8x16(reinterpret_cast<const uint8_t*>(base) + ((bb * p.G + g) * kN + n) * L + t0 + tb,
-                   cnt, vec, q);
-      else
-#pragma unroll
-        for (int i = 0; i < kSeg; ++i) q[i] = 0;
+      const uint4 qw = *reinterpret_cast<const uint4*>(which ? &r.C[n][tb] : &r.B[n][tb]);
+      const uint32_t qb[4] = {qw.x ^ 0x80808080u, qw.y ^ 0x80808080u, qw.z ^ 0x80808080u,
+                              qw.w ^ 0x80808080u};
       float* dst = which ? &sC[0][0] : &sB[0][0];
 #pragma unroll
-      for (int i = 0; i < kSeg; ++i) dst[(tb + i) * kN + n] = (float)(int8_t)q[i] * sc;
+      for (int i = 0; i < kSeg; ++i) {
+        const float v = s8_to_f32(qb[i >> 2], i & 3) * sc;
+        dst[(tb + i) * kN + n] = tb + i < tl ? v : 0.0f;
+      }
     }
     __syncthreads();
 
-    // ---- phase B: the recurrence, one thread per 4 states of a channel
-#pragma unroll 1
+    // ---- prefetch the next chunk (into the buffer chunk k - 1 used) while
+    // this one is scanned
+    if (k + 1 < nchunks)
+      fetch_chunk<kN, kCH>(p, raw[(k + 1) & 1], bb, g, c0, nc, t0 + kT,
+                           (int)min((int64_t)kT, L - t0 - kT), tid, NT);
+    cp_async_commit();
+
+    // ---- scan
+#pragma unroll 2
     for (int tg = 0; tg < kT / LPC; ++tg) {
       float part[LPC];
 #pragma unroll
-      for (int k = 0; k < LPC; ++k) {
-        const int t = tg * LPC + k;
+      for (int kk = 0; kk < LPC; ++kk) {
+        const int t = tg * LPC + kk;
         const float2 dd = sDD[lc][t];
-        const float4 b4 = *reinterpret_cast<const float4*>(&sB[t][lj * kSPL]);
-        const float4 c4 = *reinterpret_cast<const float4*>(&sC[t][lj * kSPL]);
-        const float e0 = ex2_sfu(dd.x * a2[0]);
-        const float e1 = ex2_sfu(dd.x * a2[1]);
-        const float e2 = ex2_sfu(dd.x * a2[2]);
-        const float e3 = ex2_sfu(dd.x * a2[3]);
-        h[0] = fmaf(e0, h[0], dd.y * b4.x);
-        h[1] = fmaf(e1, h[1], dd.y * b4.y);
-        h[2] = fmaf(e2, h[2], dd.y * b4.z);
-        h[3] = fmaf(e3, h[3], dd.y * b4.w);
-        part[k] = fmaf(c4.x, h[0], fmaf(c4.y, h[1], fmaf(c4.z, h[2], c4.w * h[3])));
+        float2 bq[NP], cq[NP];
+        if (kSPL == 4) {
+          const float4 b4 = *reinterpret_cast<const float4*>(&sB[t][lj * kSPL]);
+          const float4 c4 = *reinterpret_cast<const float4*>(&sC[t][lj * kSPL]);
+          bq[0] = make_float2(b4.x, b4.y);
+          bq[NP - 1] = make_float2(b4.z, b4.w);
+          cq[0] = make_float2(c4.x, c4.y);
+          cq[NP - 1] = make_float2(c4.z, c4.w);
+        } else {
+          bq[0] = *reinterpret_cast<const float2*>(&sB[t][lj * kSPL]);
+          cq[0] = *reinterpret_cast<const float2*>(&sC[t][lj * kSPL]);
+        }
+        const float2 dl = make_float2(dd.x, dd.x), dxv = make_float2(dd.y, dd.y);
+        float2 q = make_float2(0.0f, 0.0f);
+#pragma unroll
+        for (int i = 0; i < NP; ++i) {
+          const float2 r = fmul2(dl, ap[i]);
+          const float2 e = make_float2(ex2_sfu(r.x), ex2_sfu(r.y));
+          hp[i] = ffma2(e, hp[i], fmul2(dxv, bq[i]));
+          q = i == 0 ? fmul2(cq[i], hp[i]) : ffma2(cq[i], hp[i], q);
+        }
+        part[kk] = q.x + q.y;
       }
       sY[lc][tg * LPC + lj] = reduce_scatter<LPC>(part, lj);
     }
-    __syncthreads();
-
-    // ---- phase C: epilogue and binary16 stores
-    for (int w = tid; w < kCH * SEGS; w += NT) {
-      const int c = w / SEGS, tb = (w % SEGS) * kSeg;
-      if (c < nc && tb < tl) {
-        const int cnt = min(kSeg, tl - tb);
-        uint16_t* dst = p.y + (bb * d + c0 + c) * L + t0 + tb;
-        uint32_t wv[kSeg / 2];
-#pragma unroll
-        for (int i = 0; i < kSeg; i += 2) {
-          const float2 e0 = sEP[c][tb + i], e1 = sEP[c][tb + i + 1];
-          const float y0 = (sY[c][tb + i] + e0.x) * e0.y;
-          const float y1 = (sY[c][tb + i + 1] + e1.x) * e1.y;
-          wv[i / 2] = (uint32_t)f2h(y0) | ((uint32_t)f2h(y1) << 16);
-        }
-        if (vec && cnt == kSeg) {
-          uint4* o = reinterpret_cast<uint4*>(dst);
-          o[0] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
-          o[1] = make_uint4(wv[4], wv[5], wv[6], wv[7]);
-        } else {
-          for (int i = 0; i < cnt; ++i) dst[i] = (uint16_t)(wv[i / 2] >> (16 * (i & 1)));
-        }
-      }
-    }
-    __syncthreads();
   }
+  __syncthreads();
+  store_chunk(nchunks - 1);
 
   if (lvalid && p.h_final)
-    *reinterpret_cast<float4*>(p.h_final + (bb * d + lch) * kN + lj * kSPL) =
-        make_float4(h[0], h[1], h[2], h[3]);
+#pragma unroll
+    for (int i = 0; i < NP; ++i)
+      *reinterpret_cast<float2*>(p.h_final + (bb * d + lch) * kN + lj * kSPL + 2 * i) = hp[i];
   flag_status(p.status, flags);
 }
 
-template <int kN, int kCH>
+template <int kN, int kCH, int kSPL>
 cudaError_t launch_m1(const M1Params& prm, int xfmt, int64_t batch, cudaStream_t st) {
   M1Params p = prm;
   const int dg = (int)(p.d / p.G);
   p.n_ctile = (dg + kCH - 1) / kCH;
   const dim3 grid((unsigned)(p.n_ctile * p.G), (unsigned)batch);
   const dim3 block(kCH * (kN / kSPL));
-  if (xfmt == SSMQ_X_SOFTEDGE)
-    m1_scan_kernel<kN, kCH, SSMQ_X_SOFTEDGE><<<grid, block, 0, st>>>(p);
-  else
-    m1_scan_kernel<kN, kCH, SSMQ_X_INT8_GROUP><<<grid, block, 0, st>>>(p);
+  const size_t smem = sizeof(M1Smem<kN, kCH>);
+  auto kern = xfmt == SSMQ_X_SOFTEDGE ? m1_scan_kernel<kN, kCH, kSPL, SSMQ_X_SOFTEDGE>
+                                      : m1_scan_kernel<kN, kCH, kSPL, SSMQ_X_INT8_GROUP>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  kern<<<grid, block, smem, st>>>(p);
   return cudaGetLastError();
 }
 
@@ -328,11 +446,11 @@ cudaError_t launch_selective_scan(const ssmq_scan_args& a, cudaStream_t st) {
     return cudaSuccess;
   }
   switch (a.dstate) {
-    case 4: return launch_m1<4, 32>(p, a.x_format, a.batch, st);
-    case 8: return launch_m1<8, 32>(p, a.x_format, a.batch, st);
-    case 16: return launch_m1<16, 16>(p, a.x_format, a.batch, st);
-    case 32: return launch_m1<32, 16>(p, a.x_format, a.batch, st);
-    case 64: return launch_m1<64, 8>(p, a.x_format, a.batch, st);
+    case 4: return launch_m1<4, 32, 4>(p, a.x_format, a.batch, st);
+    case 8: return launch_m1<8, 16, 4>(p, a.x_format, a.batch, st);
+    case 16: return launch_m1<16, 16, 4>(p, a.x_format, a.batch, st);
+    case 32: return launch_m1<32, 16, 4>(p, a.x_format, a.batch, st);
+    case 64: return launch_m1<64, 8, 4>(p, a.x_format, a.batch, st);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -22,9 +22,11 @@
 //   - the state operand of MMA2 and the w X operand of MMA3 are split into a
 //     binary16 high part and a binary16 residual (two MMAs each), with a
 //     tile-wide power-of-two normalisation: the state then carries ~22 bits.
-// One CTA (8 warps) owns one (batch, head) and walks the sequence in tiles;
-// the fp32 state lives in registers (row n, 32 of the 64 p per thread),
-// accumulators in TMEM (256 columns), operands in shared memory (176 KB).
+// One CTA (16 warps) owns one (batch, head) and walks the sequence in tiles;
+// the fp32 state lives in registers (row n, 16 of the 64 p per thread: warp w
+// reads TMEM lanes 32 (w % 4).. and columns 16 (w / 4)..), accumulators in
+// TMEM (512 columns), operands in shared memory (222 KB, including the raw
+// int8 rows of the next tile, prefetched with cp.async during this one).
 // The chunk length of the interface only fixes where the decomposition
 // restarts; the result is the recurrence's for any length, so the kernel uses
 // 128-step tiles for every accepted chunk length.
@@ -38,9 +40,9 @@ namespace {
 constexpr int kQ = 128;  // tile length
 constexpr int kP = 64;   // head dim
 constexpr int kN = 128;  // state dim
-constexpr int kThreads = 256;
-constexpr uint32_t kWaitLimit = 1u << 22;  // mbarrier polls before giving up
-constexpr uint32_t kTmemCols = 256;
+constexpr int kThreads = 512;
+constexpr uint32_t kWaitLimit = 1u << 20;  // mbarrier probes (~1 us each) before giving up
+constexpr uint32_t kTmemCols = 512;
 
 // shared-memory map (bytes)
 constexpr int OFF_C = 0;                        // C codes * w'     [t][n]  K-major   32 KB
@@ -58,13 +60,19 @@ constexpr int F_DW = F_S2 + kQ;    // delta_s                  [128]
 constexpr int F_WX = F_DW + kQ;    // w_s = exp(S_last-S_s) d_s [128]
 constexpr int F_ES = F_WX + kQ;    // exp(S_t)                 [128]
 constexpr int F_RS = F_ES + kQ;    // 2^e_t row scale of M     [128]
-constexpr int F_RM = F_RS + kQ;    // row max halves           [2][128]
-constexpr int F_WN = F_RM + 2 * kQ;  // w'_n                   [128]
+constexpr int F_RM = F_RS + kQ;    // row max quarters         [4][128]
+constexpr int F_WN = F_RM + 4 * kQ;  // w'_n                   [128]
 constexpr int F_SB = F_WN + kN;    // sB_n                     [128]
 constexpr int F_SX = F_SB + kN;    // x scale per p            [64]
-constexpr int F_RED = F_SX + kP;   // reductions               [32]
+constexpr int F_CW = F_SX + kP;    // exp(S_p(s) - S_s) d_s w_max, p(s) = s | 31  [128]
+constexpr int F_RED = F_CW + kQ;   // reductions               [32]
 constexpr int F_END = F_RED + 32;
-constexpr int kSmemBytes = OFF_F + F_END * 4;
+// raw int8 rows of the next tile, fetched with cp.async during this tile
+constexpr int OFF_RAW = (OFF_F + F_END * 4 + 127) / 128 * 128;
+constexpr int OFF_RC = OFF_RAW;                 // C codes [t][n]  16 KB
+constexpr int OFF_RB = OFF_RC + kQ * kN;        // B codes [t][n]  16 KB
+constexpr int OFF_RX = OFF_RB + kQ * kN;        // x codes [t][p]   8 KB
+constexpr int kSmemBytes = OFF_RX + kQ * kP;
 
 struct SsdParams {
   int64_t L, H, G;
@@ -104,9 +112,14 @@ __device__ __forceinline__ int norm_exp(float a) {
   return max(-100, min(100, E - 15));
 }
 
-__device__ __forceinline__ uint32_t pack_h2(float a, float b) {
-  return (uint32_t)__half_as_ushort(__float2half_rn(a)) |
-         ((uint32_t)__half_as_ushort(__float2half_rn(b)) << 16);
+__device__ __forceinline__ uint32_t pack_h2(float a, float b) { return pack_half2(a, b); }
+
+// v = hi + lo with hi, lo binary16 (two packed pairs)
+__device__ __forceinline__ void split_h2(float v0, float v1, uint32_t& hi, uint32_t& lo) {
+  const __half2 h = __floats2half2_rn(v0, v1);
+  const float2 hf = __half22float2(h);
+  hi = h2_bits(h);
+  lo = pack_half2(v0 - hf.x, v1 - hf.y);
 }
 
 // value of one x element as an exactly representable binary16 number, the
@@ -132,10 +145,32 @@ __device__ __forceinline__ float block_max(float v, float* red, int tid) {
   return r;
 }
 
+// cp.async the int8 rows (C, B: N bytes; x: P bytes) of the tile starting
+// at t0 into the raw buffer; rows at or beyond ql are left as they are (the
+// staging masks them).
+__device__ __forceinline__ void fetch_tile(const SsdParams& p, uint8_t* smem, int64_t bb,
+                                           int64_t hd, int64_t g, int64_t t0, int ql, int tid) {
+  for (int w = tid; w < kQ * (kN / 16); w += kThreads) {
+    const int r = w / (kN / 16), c = w % (kN / 16);
+    if (r >= ql) continue;
+    const int64_t ro = ((bb * p.L + t0 + r) * p.G + g) * kN + 16 * c;
+    const int slot = c ^ (r & 7);  // swizzle: conflict-free column reads of 8 rows
+    tc::cp_async16(smem + OFF_RC + r * kN + 16 * slot, p.C + ro);
+    tc::cp_async16(smem + OFF_RB + r * kN + 16 * slot, p.B + ro);
+  }
+  for (int w = tid; w < kQ * (kP / 16); w += kThreads) {
+    const int r = w / (kP / 16), c = w % (kP / 16);
+    if (r >= ql) continue;
+    const int64_t xo = ((bb * p.L + t0 + r) * p.H + hd) * kP + 16 * c;
+    tc::cp_async16(smem + OFF_RX + r * kP + 16 * (c ^ (r & 3)), static_cast<const uint8_t*>(p.x) + xo);
+  }
+  tc::cp_async_commit();
+}
+
 __global__ void __launch_bounds__(kThreads, 1) ssd_kernel(const SsdParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ uint32_t tmem_slot;
-  __shared__ __align__(8) uint64_t bars[2];
+  __shared__ __align__(8) uint64_t bars[3];
   __shared__ int abort_flag;
   float* F = reinterpret_cast<float*>(smem + OFF_F);
 
@@ -144,8 +179,8 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_kernel(const SsdParams p) {
   const int64_t H = p.H, L = p.L;
   const int64_t bb = u / H, hd = u % H;
   const int64_t g = hd * p.G / H;
-  const int row = 32 * (warp & 3) + lane;  // TMEM lane owned by this thread
-  const int half = warp >> 2;              // column half
+  const int row = 32 * (warp & 3) + lane;  // TMEM lane (row t or n) owned by this thread
+  const int q4 = warp >> 2;                // column quarter
   const uint32_t s_base = tc::smem_u32(smem);
   uint32_t flags = 0;
 
@@ -174,6 +209,7 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_kernel(const SsdParams p) {
   if (tid == 0) {
     tc::mbar_init(&bars[0], 1);
     tc::mbar_init(&bars[1], 1);
+    tc::mbar_init(&bars[2], 1);
   }
   __syncthreads();
   const float wmax = block_max(tid < kN ? F[F_WN + tid] : 0.0f, F + F_RED, tid);
@@ -181,9 +217,12 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_kernel(const SsdParams p) {
   const float A2 = __ldg(p.A + hd) * kLog2e;
   const float bias = p.dt_bias ? __ldg(p.dt_bias + hd) : 0.0f;
   const float Dh = p.D ? __ldg(p.D + hd) : 0.0f;
+  // per-thread constants of the rows it owns
+  const float hfac = F[F_SB + row] > 0.0f ? wmax / F[F_SB + row] : 0.0f;  // state -> MMA2 operand
+  const float sbr = F[F_SB + row];
 
-  // ---- initial state: thread (row = n, half) holds p in [32 half, 32 half + 32)
-  float hs[32];
+  // ---- initial state: thread (row = n, quarter) holds p in [16 q4, 16 q4 + 16)
+  float hs[16];
   {
     float* stage = reinterpret_cast<float*>(smem + OFF_M);  // P x N fp32 = 32 KB
     if (p.h0) {
@@ -192,7 +231,7 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_kernel(const SsdParams p) {
     }
     __syncthreads();
 #pragma unroll
-    for (int j = 0; j < 32; ++j) hs[j] = p.h0 ? stage[(32 * half + j) * kN + row] : 0.0f;
+    for (int j = 0; j < 16; ++j) hs[j] = p.h0 ? stage[(16 * q4 + j) * kN + row] : 0.0f;
     __syncthreads();
   }
   tc::fence_before();
@@ -200,74 +239,117 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_kernel(const SsdParams p) {
   tc::fence_after();
   const uint32_t tmem = tmem_slot;
   const uint32_t t_lane = (uint32_t)(32 * (warp & 3)) << 16;
-  const uint32_t T_CB = 0, T_ACC = 0, T_YD = 128, T_YO = 192;
+  const uint32_t T_CB = 0, T_YD = 128, T_YO = 192, T_ACC = 256;
+
+  // raw rows of tile 0, and its dt (warp 0: 4 steps per lane)
+  fetch_tile(p, smem, bb, hd, g, 0, (int)min((int64_t)kQ, L), tid);
+  float dtv[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+  if (warp == 0) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      if (4 * lane + i < L) dtv[i] = h2f(p.dt[(bb * L + 4 * lane + i) * H + hd]);
+  }
 
   uint32_t phase = 0;
   for (int64_t t0 = 0; t0 < L; t0 += kQ, phase ^= 1u) {
     const int ql = (int)min((int64_t)kQ, L - t0);
-    // ---- delta, S = cumsum(delta A) (threads 0..127, one step each)
-    if (tid < kQ) {
-      float dl = 0.0f;
-      if (tid < ql) {
-        const float v = h2f(p.dt[(bb * L + t0 + tid) * H + hd]) + bias;
-        dl = p.softplus ? softplus_f(v) : v;
+    tc::cp_async_wait_all();
+
+    // ---- warp 0: delta, S = cumsum(delta A) (log2 units), w_s, exp(S_t)
+    if (warp == 0) {
+      float dl[4], sc[4];
+      float run = 0.0f;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int t = 4 * lane + i;
+        float d = 0.0f;
+        if (t < ql) {
+          const float v = dtv[i] + bias;
+          d = p.softplus ? softplus_f(v) : v;
+        }
+        dl[i] = d;
+        run += d * A2;
+        sc[i] = run;
       }
-      float s = dl * A2;  // log2 units
+      float ex = run;  // inclusive scan of the lane totals
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
-        const float n = __shfl_up_sync(0xffffffffu, s, o);
-        if (lane >= o) s += n;
+        const float n = __shfl_up_sync(0xffffffffu, ex, o);
+        if (lane >= o) ex += n;
       }
-      if (lane == 31) F[F_RED + warp] = s;  // warp totals (warps 0..3)
-      F[F_DW + tid] = dl;
-      F[F_S2 + tid] = s;
+      const float off = ex - run;
+      const float s_last = __shfl_sync(0xffffffffu, ex, 31);
+      float wmx = 0.0f;
+      // S at the end of this lane's 32-step column block (lane 8 b + 7 holds it)
+      const float s_blk = __shfl_sync(0xffffffffu, sc[3] + off, lane | 7);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int t = 4 * lane + i;
+        const float s2 = sc[i] + off;
+        const float w = ex2_sfu(s_last - s2) * dl[i];
+        F[F_S2 + t] = s2;
+        F[F_DW + t] = dl[i];
+        F[F_WX + t] = w;
+        F[F_ES + t] = ex2_sfu(s2);
+        F[F_CW + t] = ex2_sfu(s_blk - s2) * dl[i] * wmax;
+        wmx = fmaxf(wmx, w);
+      }
+#pragma unroll
+      for (int o = 16; o >= 1; o >>= 1) wmx = fmaxf(wmx, __shfl_xor_sync(0xffffffffu, wmx, o));
+      if (lane == 0) {
+        F[F_RED] = wmx;
+        F[F_RED + 1] = s_last;
+      }
     }
-    __syncthreads();
-    if (tid < kQ) {
-      float off = 0.0f;
-      for (int w = 0; w < (tid >> 5); ++w) off += F[F_RED + w];
-      F[F_S2 + tid] += off;
-    }
-    __syncthreads();
-    const float s_last = F[F_S2 + kQ - 1];
-    float wx = 0.0f;
-    if (tid < kQ) {
-      const float s2 = F[F_S2 + tid];
-      wx = ex2_sfu(s_last - s2) * F[F_DW + tid];
-      F[F_WX + tid] = wx;
-      F[F_ES + tid] = ex2_sfu(s2);
-    }
-    const float wx_max = block_max(wx, F + F_RED, tid);
-    const int ex = norm_exp(wx_max * p.x_bound);  // x_bound >= max |x_exact|
-    const float xsc = pow2i(-ex);
-
-    // ---- stage C (codes * w'_n) and B (codes) rows: thread -> (row, 64 states)
+    // every warp: max |state operand| partial
     {
-      const int r = tid >> 1, part = tid & 1;
-      const bool ok = r < ql;
-      const int64_t ro = ((bb * L + t0 + r) * p.G + g) * kN + 64 * part;
-      uint4 cq[4], bq[4];
+      float hm = 0.0f;
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        cq[i] = ok ? __ldg(reinterpret_cast<const uint4*>(p.C + ro) + i) : make_uint4(0, 0, 0, 0);
-        bq[i] = ok ? __ldg(reinterpret_cast<const uint4*>(p.B + ro) + i) : make_uint4(0, 0, 0, 0);
+      for (int j = 0; j < 16; ++j) hm = fmaxf(hm, fabsf(hs[j] * hfac));
+#pragma unroll
+      for (int o = 16; o >= 1; o >>= 1) hm = fmaxf(hm, __shfl_xor_sync(0xffffffffu, hm, o));
+      if (lane == 0) F[F_RED + 2 + warp] = hm;
+    }
+    __syncthreads();  // (A): raw tile landed for everyone, S and maxima published
+    const float s_last = F[F_RED + 1];
+    const int ex = norm_exp(F[F_RED] * p.x_bound);  // x_bound >= max |x_exact|
+    const float xsc = pow2i(-ex);
+    float hmax_all = 0.0f;
+#pragma unroll
+    for (int w = 0; w < kThreads / 32; ++w) hmax_all = fmaxf(hmax_all, F[F_RED + 2 + w]);
+    const int eh = norm_exp(hmax_all);
+
+    // ---- stage C (codes * w'_n) and B (codes): thread -> (row, 32 states);
+    // the states are warp-uniform so the w'_n reads are broadcasts
+    {
+      const int r = 32 * (warp >> 2) + lane, part = warp & 3;
+      const bool ok = r < ql;
+      uint4 cq[2], bq[2];
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const int slot = (2 * part + i) ^ (r & 7);
+        cq[i] = ok ? *reinterpret_cast<const uint4*>(smem + OFF_RC + r * kN + 16 * slot)
+                   : make_uint4(0, 0, 0, 0);
+        bq[i] = ok ? *reinterpret_cast<const uint4*>(smem + OFF_RB + r * kN + 16 * slot)
+                   : make_uint4(0, 0, 0, 0);
       }
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const uint32_t cw[4] = {cq[i].x, cq[i].y, cq[i].z, cq[i].w};
-        const uint32_t bw[4] = {bq[i].x, bq[i].y, bq[i].z, bq[i].w};
+      for (int i = 0; i < 2; ++i) {
+        const uint32_t cw[4] = {cq[i].x ^ 0x80808080u, cq[i].y ^ 0x80808080u,
+                                cq[i].z ^ 0x80808080u, cq[i].w ^ 0x80808080u};
+        const uint32_t bw[4] = {bq[i].x ^ 0x80808080u, bq[i].y ^ 0x80808080u,
+                                bq[i].z ^ 0x80808080u, bq[i].w ^ 0x80808080u};
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {  // 8 states per 16-byte core-matrix row
-          const int n0 = 64 * part + 16 * i + 8 * hh;
+          const int n0 = 32 * part + 16 * i + 8 * hh;
           uint32_t oc[4], ob[4];
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
             const uint32_t wc = cw[2 * hh + k / 2], wb = bw[2 * hh + k / 2];
-            const int sh = 16 * (k & 1);
-            const float c0 = (float)(int8_t)(wc >> sh), c1 = (float)(int8_t)(wc >> (sh + 8));
-            const float b0 = (float)(int8_t)(wb >> sh), b1 = (float)(int8_t)(wb >> (sh + 8));
+            const int b0i = 2 * (k & 1);
+            const float c0 = s8_to_f32(wc, b0i), c1 = s8_to_f32(wc, b0i + 1);
             oc[k] = pack_h2(c0 * F[F_WN + n0 + 2 * k], c1 * F[F_WN + n0 + 2 * k + 1]);
-            ob[k] = pack_h2(b0, b1);
+            ob[k] = h2_bits(s8x2_to_h2(wb, b0i, b0i + 1));
           }
           *reinterpret_cast<uint4*>(smem + OFF_C + tc::kmaj_off(r, n0, kN)) =
               make_uint4(oc[0], oc[1], oc[2], oc[3]);
@@ -276,73 +358,80 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_kernel(const SsdParams p) {
         }
       }
     }
-    // ---- stage x (exact) and w x (hi / lo) rows: thread -> (row s, 32 p)
+    // ---- stage x (exact) and w x (hi / lo): thread -> (row s, 16 p)
     {
-      const int s = tid >> 1, part = tid & 1;
+      const int s = 32 * (warp >> 2) + lane, part = warp & 3;
       const bool ok = s < ql;
-      const int64_t xo = ((bb * L + t0 + s) * H + hd) * kP + 32 * part;
-      uint4 xq[2];
-#pragma unroll
-      for (int i = 0; i < 2; ++i)
-        xq[i] = ok ? __ldg(reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(p.x) + xo) + i)
-                   : make_uint4(0, 0, 0, 0);
+      const uint4 xq = ok ? *reinterpret_cast<const uint4*>(smem + OFF_RX + s * kP +
+                                                            16 * (part ^ (s & 3)))
+                          : make_uint4(0, 0, 0, 0);
       const float ws = F[F_WX + s] * xsc;
 #pragma unroll
-      for (int grp = 0; grp < 4; ++grp) {  // 8 p per group
-        const uint4 q = xq[grp / 2];
-        const uint32_t w0 = (grp & 1) ? q.z : q.x, w1 = (grp & 1) ? q.w : q.y;
+      for (int grp = 0; grp < 2; ++grp) {  // 8 p per group
+        const uint32_t w0 = grp ? xq.z : xq.x, w1 = grp ? xq.w : xq.y;
         float xv[8];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          xv[k] = x_exact((w0 >> (8 * k)) & 0xFFu, p.xfmt, p.se_shift);
-          xv[4 + k] = x_exact((w1 >> (8 * k)) & 0xFFu, p.xfmt, p.se_shift);
-        }
         uint32_t ox[4], oh[4], ol[4];
+        if (p.xfmt == SSMQ_X_INT8_GROUP) {
+          const uint32_t x0 = w0 ^ 0x80808080u, x1 = w1 ^ 0x80808080u;
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          ox[k] = pack_h2(xv[2 * k], xv[2 * k + 1]);
-          const float v0 = ws * xv[2 * k], v1 = ws * xv[2 * k + 1];
-          const __half h0v = __float2half_rn(v0), h1v = __float2half_rn(v1);
-          oh[k] = (uint32_t)__half_as_ushort(h0v) | ((uint32_t)__half_as_ushort(h1v) << 16);
-          ol[k] = pack_h2(v0 - __half2float(h0v), v1 - __half2float(h1v));
+          for (int k = 0; k < 4; ++k) {
+            xv[k] = s8_to_f32(x0, k);
+            xv[4 + k] = s8_to_f32(x1, k);
+          }
+          ox[0] = h2_bits(s8x2_to_h2(x0, 0, 1));
+          ox[1] = h2_bits(s8x2_to_h2(x0, 2, 3));
+          ox[2] = h2_bits(s8x2_to_h2(x1, 0, 1));
+          ox[3] = h2_bits(s8x2_to_h2(x1, 2, 3));
+        } else {
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            xv[k] = x_exact((w0 >> (8 * k)) & 0xFFu, p.xfmt, p.se_shift);
+            xv[4 + k] = x_exact((w1 >> (8 * k)) & 0xFFu, p.xfmt, p.se_shift);
+          }
+#pragma unroll
+          for (int k = 0; k < 4; ++k) ox[k] = pack_h2(xv[2 * k], xv[2 * k + 1]);
         }
-        const uint32_t off = tc::mnmaj_off(32 * part + 8 * grp, s, kP);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) split_h2(ws * xv[2 * k], ws * xv[2 * k + 1], oh[k], ol[k]);
+        const uint32_t off = tc::mnmaj_off(16 * part + 8 * grp, s, kP);
         *reinterpret_cast<uint4*>(smem + OFF_X + off) = make_uint4(ox[0], ox[1], ox[2], ox[3]);
         *reinterpret_cast<uint4*>(smem + OFF_XH + off) = make_uint4(oh[0], oh[1], oh[2], oh[3]);
         *reinterpret_cast<uint4*>(smem + OFF_XL + off) = make_uint4(ol[0], ol[1], ol[2], ol[3]);
       }
     }
     // ---- stage the state (hi / lo) for Y_off: h'' = h w_max / sB_n, normalised
-    float hmax = 0.0f;
     {
-      const float f = F[F_SB + row] > 0.0f ? wmax / F[F_SB + row] : 0.0f;
+      const float f = hfac * pow2i(-eh);
 #pragma unroll
-      for (int j = 0; j < 32; ++j) hmax = fmaxf(hmax, fabsf(hs[j] * f));
-    }
-    const float hmax_all = block_max(hmax, F + F_RED, tid);
-    const int eh = norm_exp(hmax_all);
-    {
-      const float f = (F[F_SB + row] > 0.0f ? wmax / F[F_SB + row] : 0.0f) * pow2i(-eh);
-#pragma unroll
-      for (int grp = 0; grp < 4; ++grp) {
+      for (int grp = 0; grp < 2; ++grp) {
         uint32_t oh[4], ol[4];
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const float v0 = hs[8 * grp + 2 * k] * f, v1 = hs[8 * grp + 2 * k + 1] * f;
-          const __half h0v = __float2half_rn(v0), h1v = __float2half_rn(v1);
-          oh[k] = (uint32_t)__half_as_ushort(h0v) | ((uint32_t)__half_as_ushort(h1v) << 16);
-          ol[k] = pack_h2(v0 - __half2float(h0v), v1 - __half2float(h1v));
-        }
-        const uint32_t off = tc::mnmaj_off(32 * half + 8 * grp, row, kP);
+        for (int k = 0; k < 4; ++k)
+          split_h2(hs[8 * grp + 2 * k] * f, hs[8 * grp + 2 * k + 1] * f, oh[k], ol[k]);
+        const uint32_t off = tc::mnmaj_off(16 * q4 + 8 * grp, row, kP);
         *reinterpret_cast<uint4*>(smem + OFF_HH + off) = make_uint4(oh[0], oh[1], oh[2], oh[3]);
         *reinterpret_cast<uint4*>(smem + OFF_HL + off) = make_uint4(ol[0], ol[1], ol[2], ol[3]);
       }
     }
     tc::fence_async_smem();
     tc::fence_before();
-    __syncthreads();
+    __syncthreads();  // (B): operands staged, raw buffer consumed
 
-    // ---- MMA0: CB = C' B^T  (M = t, N = s, K = n)
+    // ---- fetch the next tile while this one runs
+    if (t0 + kQ < L) {
+      fetch_tile(p, smem, bb, hd, g, t0 + kQ, (int)min((int64_t)kQ, L - t0 - kQ), tid);
+      if (warp == 0) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int64_t t = t0 + kQ + 4 * lane + i;
+          dtv[i] = t < L ? h2f(p.dt[(bb * L + t) * H + hd]) : 0.0f;
+        }
+      }
+    }
+
+    // ---- MMA0: CB = C' B^T  (M = t, N = s, K = n); then, independent of
+    // M, MMA2 (Y_off, hi + lo) and MMA3 (state, hi + lo) run while the CUDA
+    // cores form M
     if (tid == 0) {
       tc::fence_after();
       const uint32_t id = tc::idesc_f16(kQ, kQ, false, false);
@@ -351,66 +440,8 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_kernel(const SsdParams p) {
         tc::mma_f16(tmem + T_CB, tc::kmaj_desc(s_base + OFF_C, k0, kN),
                     tc::kmaj_desc(s_base + OFF_B, k0, kN), id, k0 > 0);
       tc::mma_commit(&bars[0]);
-    }
-    __syncwarp();
-    if (!tc::mbar_wait(&bars[0], phase, kWaitLimit)) {
-      flags |= SSMQ_DEV_TIMEOUT;
-      atomicExch(&abort_flag, 1);
-    }
-    if (__syncthreads_or(abort_flag)) break;
-    tc::fence_after();
-
-    // ---- M = CB * exp(S_t - S_s) * delta_s * w_max, row-normalised, s <= t
-    {
-      const int t = row;
-      const float st = F[F_S2 + t];
-      float mv[64];
-      float rmax = 0.0f;
-      const bool any = (64 * half) <= t;  // columns of this half reach the diagonal
-      if (any) {
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          float v[32];
-          tc::tmem_ld32(tmem + t_lane + T_CB + 64 * half + 32 * c, v);
-#pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const int s = 64 * half + 32 * c + j;
-            const float m = s <= t ? v[j] * ex2_sfu(st - F[F_S2 + s]) * F[F_DW + s] * wmax : 0.0f;
-            mv[32 * c + j] = m;
-            rmax = fmaxf(rmax, fabsf(m));
-          }
-        }
-      } else {
-#pragma unroll
-        for (int j = 0; j < 64; ++j) mv[j] = 0.0f;
-      }
-      F[F_RM + half * kQ + t] = rmax;
-      __syncthreads();
-      const int et = norm_exp(fmaxf(F[F_RM + t], F[F_RM + kQ + t]));
-      const float sc = pow2i(-et);
-      if (half == 0) F[F_RS + t] = pow2i(et);
-#pragma unroll
-      for (int grp = 0; grp < 8; ++grp) {
-        uint32_t o[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) o[k] = pack_h2(mv[8 * grp + 2 * k] * sc, mv[8 * grp + 2 * k + 1] * sc);
-        *reinterpret_cast<uint4*>(smem + OFF_M + tc::kmaj_off(t, 64 * half + 8 * grp, kQ)) =
-            make_uint4(o[0], o[1], o[2], o[3]);
-      }
-    }
-    tc::fence_async_smem();
-    tc::fence_before();
-    __syncthreads();
-
-    // ---- MMA1 (Y_diag), MMA2 (Y_off, hi + lo), MMA3 (state, hi + lo)
-    if (tid == 0) {
-      tc::fence_after();
       const uint32_t id_y = tc::idesc_f16(kQ, kP, false, true);
       const uint32_t id_s = tc::idesc_f16(kN, kP, true, true);
-#pragma unroll
-      for (int k0 = 0; k0 < kQ; k0 += 16)
-        tc::mma_f16(tmem + T_YD, tc::kmaj_desc(s_base + OFF_M, k0, kQ),
-                    tc::mnmaj_desc(s_base + OFF_X, k0, kP), id_y, k0 > 0);
 #pragma unroll
       for (int k0 = 0; k0 < kN; k0 += 16)
         tc::mma_f16(tmem + T_YO, tc::kmaj_desc(s_base + OFF_C, k0, kN),
@@ -427,33 +458,116 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_kernel(const SsdParams p) {
       for (int k0 = 0; k0 < kQ; k0 += 16)
         tc::mma_f16(tmem + T_ACC, tc::mnmaj_desc(s_base + OFF_B, k0, kN),
                     tc::mnmaj_desc(s_base + OFF_XL, k0, kP), id_s, 1u);
+      tc::mma_commit(&bars[2]);
+    }
+    __syncwarp();
+    if (!tc::mbar_wait(&bars[0], phase, kWaitLimit)) {
+      flags |= SSMQ_DEV_TIMEOUT;
+      abort_flag = 1;
+    }
+    tc::fence_after();
+
+    // ---- M = CB * exp(S_t - S_s) * delta_s * w_max, row-normalised, s <= t
+    // (thread: row t, columns s in [32 q4, 32 q4 + 32))
+    // Column block q4 against row block (warp & 3), both warp-uniform: above
+    // the diagonal M is zero; strictly below it exp(S_t - S_s) =
+    // exp(S_t - S_p) exp(S_p - S_s) with p the block's last step, both
+    // factors <= 1 (no overflow, underflow only of negligible terms); on the
+    // diagonal block each element takes its own exponential.
+    float mv[32];
+    {
+      const int t = row, s0 = 32 * q4, rb = warp & 3;
+      float rmax = 0.0f;
+      if (q4 <= rb) {
+        float v[32];
+        tc::tmem_ld32(tmem + t_lane + T_CB + s0, v);
+        const float st = F[F_S2 + t];
+        if (q4 < rb) {
+          const float rt = ex2_sfu(st - F[F_S2 + s0 + 31]);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const float m = v[j] * (rt * F[F_CW + s0 + j]);
+            mv[j] = m;
+            rmax = fmaxf(rmax, fabsf(m));
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int s = s0 + j;
+            const float m = s <= t ? v[j] * ex2_sfu(st - F[F_S2 + s]) * F[F_DW + s] * wmax : 0.0f;
+            mv[j] = m;
+            rmax = fmaxf(rmax, fabsf(m));
+          }
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) mv[j] = 0.0f;
+      }
+      F[F_RM + q4 * kQ + t] = rmax;
+    }
+    if (__syncthreads_or(abort_flag)) break;  // (C): row maxima published
+    {
+      const int t = row;
+      const float rm = fmaxf(fmaxf(F[F_RM + t], F[F_RM + kQ + t]),
+                             fmaxf(F[F_RM + 2 * kQ + t], F[F_RM + 3 * kQ + t]));
+      const int et = norm_exp(rm);
+      const float sc = pow2i(-et);
+      if (q4 == 0) F[F_RS + t] = pow2i(et);
+#pragma unroll
+      for (int grp = 0; grp < 4; ++grp) {
+        uint32_t o[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) o[k] = pack_h2(mv[8 * grp + 2 * k] * sc, mv[8 * grp + 2 * k + 1] * sc);
+        *reinterpret_cast<uint4*>(smem + OFF_M + tc::kmaj_off(t, 32 * q4 + 8 * grp, kQ)) =
+            make_uint4(o[0], o[1], o[2], o[3]);
+      }
+    }
+    tc::fence_async_smem();
+    tc::fence_before();
+    __syncthreads();  // (D): M staged
+
+    // ---- MMA1 (Y_diag = M X)
+    if (tid == 0) {
+      tc::fence_after();
+      const uint32_t id_y = tc::idesc_f16(kQ, kP, false, true);
+#pragma unroll
+      for (int k0 = 0; k0 < kQ; k0 += 16)
+        tc::mma_f16(tmem + T_YD, tc::kmaj_desc(s_base + OFF_M, k0, kQ),
+                    tc::mnmaj_desc(s_base + OFF_X, k0, kP), id_y, k0 > 0);
       tc::mma_commit(&bars[1]);
     }
     __syncwarp();
-    if (!tc::mbar_wait(&bars[1], phase, kWaitLimit)) {
+    if (!tc::mbar_wait(&bars[1], phase, kWaitLimit) || !tc::mbar_wait(&bars[2], phase, kWaitLimit)) {
       flags |= SSMQ_DEV_TIMEOUT;
-      atomicExch(&abort_flag, 1);
+      abort_flag = 1;
     }
-    if (__syncthreads_or(abort_flag)) break;
     tc::fence_after();
 
-    // ---- y = Y_diag 2^e_t sx + exp(S_t) 2^e_h Y_off + D x  (thread: row t, 32 p)
+    // ---- y = Y_diag 2^e_t sx + exp(S_t) 2^e_h Y_off + D x  (thread: row t, 16 p)
     {
       const int t = row;
-      float yd[32], yo[32];
-      tc::tmem_ld32(tmem + t_lane + T_YD + 32 * half, yd);
-      tc::tmem_ld32(tmem + t_lane + T_YO + 32 * half, yo);
+      float yd[16], yo[16];
+      tc::tmem_ld16(tmem + t_lane + T_YD + 16 * q4, yd);
+      tc::tmem_ld16(tmem + t_lane + T_YO + 16 * q4, yo);
       if (t < ql) {
         const float rs = F[F_RS + t], es = F[F_ES + t] * pow2i(eh);
-        const int64_t yo_off = ((bb * L + t0 + t) * H + hd) * kP + 32 * half;
-        const uint4* xr = reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(p.x) + yo_off);
-        const uint4 xa = __ldg(xr), xb = __ldg(xr + 1);
-        const uint32_t xw[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
-        uint32_t zw[16];
+        const int64_t yo_off = ((bb * L + t0 + t) * H + hd) * kP + 16 * q4;
+        // x of this row as exact binary16 values from the staged MMA operand
+        uint32_t xw[8];
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          const uint4 v = *reinterpret_cast<const uint4*>(smem + OFF_X +
+                                                          tc::mnmaj_off(16 * q4 + 8 * i, t, kP));
+          xw[4 * i] = v.x;
+          xw[4 * i + 1] = v.y;
+          xw[4 * i + 2] = v.z;
+          xw[4 * i + 3] = v.w;
+        }
+        uint32_t zw[8];
         if (p.z) {
           const uint4* zr = reinterpret_cast<const uint4*>(p.z + yo_off);
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
+          for (int i = 0; i < 2; ++i) {
             const uint4 zz = __ldg(zr + i);
             zw[4 * i] = zz.x;
             zw[4 * i + 1] = zz.y;
@@ -461,37 +575,40 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_kernel(const SsdParams p) {
             zw[4 * i + 3] = zz.w;
           }
         }
-        uint32_t out[16];
+        uint32_t out[8];
 #pragma unroll
-        for (int j = 0; j < 32; j += 2) {
+        for (int j = 0; j < 16; j += 2) {
+          const float2 xp = __half22float2(*reinterpret_cast<const __half2*>(&xw[j >> 1]));
+          float2 zf = make_float2(0.0f, 0.0f);
+          if (p.z) zf = __half22float2(*reinterpret_cast<const __half2*>(&zw[j >> 1]));
           float r2[2];
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
             const int pj = j + e;
-            const float sx = F[F_SX + 32 * half + pj];
-            const float xv = x_exact((xw[pj >> 2] >> (8 * (pj & 3))) & 0xFFu, p.xfmt, p.se_shift) * sx;
+            const float sx = F[F_SX + 16 * q4 + pj];
+            const float xv = (e ? xp.y : xp.x) * sx;
             float yv = yd[pj] * rs * sx + es * yo[pj] + Dh * xv;
-            if (p.z) yv *= silu_f(h2f((uint16_t)(zw[pj >> 1] >> (16 * (pj & 1)))));
+            if (p.z) yv *= silu_f(e ? zf.y : zf.x);
             r2[e] = yv;
           }
-          out[j / 2] = (uint32_t)f2h(r2[0]) | ((uint32_t)f2h(r2[1]) << 16);
+          out[j / 2] = pack_half2(r2[0], r2[1]);
         }
         uint4* yr = reinterpret_cast<uint4*>(p.y + yo_off);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) yr[i] = make_uint4(out[4 * i], out[4 * i + 1], out[4 * i + 2], out[4 * i + 3]);
+        yr[0] = make_uint4(out[0], out[1], out[2], out[3]);
+        yr[1] = make_uint4(out[4], out[5], out[6], out[7]);
       }
     }
-    // ---- state: h = exp(S_last) h + sB_n sx_p 2^-e_x acc  (thread: row n, 32 p)
+    // ---- state: h = exp(S_last) h + sB_n sx_p 2^e_x acc  (thread: row n, 16 p)
     {
-      float acc[32];
-      tc::tmem_ld32(tmem + t_lane + T_ACC + 32 * half, acc);
+      float acc[16];
+      tc::tmem_ld16(tmem + t_lane + T_ACC + 16 * q4, acc);
       const float decay = ex2_sfu(s_last);
-      const float f = F[F_SB + row] * pow2i(ex);
+      const float f = sbr * pow2i(ex);
 #pragma unroll
-      for (int j = 0; j < 32; ++j) hs[j] = fmaf(decay, hs[j], f * F[F_SX + 32 * half + j] * acc[j]);
+      for (int j = 0; j < 16; ++j) hs[j] = fmaf(decay, hs[j], f * F[F_SX + 16 * q4 + j] * acc[j]);
     }
     tc::fence_before();
-    __syncthreads();
+    if (__syncthreads_or(abort_flag)) break;  // (E): tile done
   }
 
   // ---- final state (P, N) through shared memory for coalesced stores
@@ -499,7 +616,7 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_kernel(const SsdParams p) {
     float* stage = reinterpret_cast<float*>(smem + OFF_M);
     __syncthreads();
 #pragma unroll
-    for (int j = 0; j < 32; ++j) stage[(32 * half + j) * kN + row] = hs[j];
+    for (int j = 0; j < 16; ++j) stage[(16 * q4 + j) * kN + row] = hs[j];
     __syncthreads();
     float4* dst = reinterpret_cast<float4*>(p.h_final + u * kP * kN);
     for (int i = tid; i < kP * kN / 4; i += kThreads) dst[i] = reinterpret_cast<float4*>(stage)[i];

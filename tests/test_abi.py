@@ -39,10 +39,13 @@ def test_exports_every_declared_symbol(L):
     assert declared <= set(N.SIGNATURES), declared - set(N.SIGNATURES)
 
 
+STRUCTS = ((N.ScanArgs, "ssmq_scan_args"), (N.SSDArgs, "ssmq_ssd_args"),
+           (N.DecodeArgs, "ssmq_decode_args"), (N.M1DecodeArgs, "ssmq_m1_decode_args"))
+
+
 def test_struct_layout_matches_header(tmp_path):
     prog = ["#include <stdio.h>", "#include <stddef.h>", '#include "ssmq.h"', "int main(void){"]
-    for cls, cname in ((N.ScanArgs, "ssmq_scan_args"), (N.SSDArgs, "ssmq_ssd_args"),
-                       (N.DecodeArgs, "ssmq_decode_args")):
+    for cls, cname in STRUCTS:
         prog.append('printf("%s %%zu\\n", sizeof(%s));' % (cname, cname))
         for f, _ in cls._fields_:
             prog.append('printf("%s.%s %%zu\\n", offsetof(%s, %s));' % (cname, f, cname, f))
@@ -52,8 +55,7 @@ def test_struct_layout_matches_header(tmp_path):
     exe = tmp_path / "layout"
     subprocess.check_call(["gcc", "-I", os.path.join(ROOT, "include"), "-o", str(exe), str(src)])
     got = dict(line.split() for line in subprocess.check_output([str(exe)], text=True).splitlines())
-    for cls, cname in ((N.ScanArgs, "ssmq_scan_args"), (N.SSDArgs, "ssmq_ssd_args"),
-                       (N.DecodeArgs, "ssmq_decode_args")):
+    for cls, cname in STRUCTS:
         assert int(got[cname]) == C.sizeof(cls), cname
         for f, _ in cls._fields_:
             assert int(got["%s.%s" % (cname, f)]) == getattr(cls, f).offset, (cname, f)
@@ -173,3 +175,19 @@ def test_fault_injection_hook(L, monkeypatch):
 
 def test_version(L):
     assert N.ssmq_version() >= 100
+
+
+def test_m1_decode_validation(L):
+    f = dict(batch=4, dim=32, dstate=16, ngroups=1, state_group_size=4, x_format=N.X_INT8_GROUP,
+             x=FAKE, x_group=FAKE, x_scale=FAKE, n_x_groups=2, dt=FAKE, A=FAKE, B=FAKE, C=FAKE,
+             B_scale=FAKE, C_scale=FAKE, state=FAKE, y=FAKE, dt_softplus=1)
+
+    def S(**kw):
+        g = dict(f)
+        g.update(kw)
+        return L.ssmq_selective_state_update_w8(C.byref(N._fill(N.M1DecodeArgs, g)), None)
+    assert S(dstate=12) == N.ERR_UNSUPPORTED
+    assert S(ngroups=3) == N.ERR_INVALID_ARG
+    assert S(A=None) == N.ERR_INVALID_ARG
+    assert S(A=FAKE + 4) == N.ERR_ALIGNMENT
+    assert S(batch=0) == N.OK

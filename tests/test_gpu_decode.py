@@ -129,3 +129,65 @@ def test_decode_checkpoint_resume_bit_exact():
     s3 = T(host)
     run(s3, 500, 1000)
     np.testing.assert_array_equal(H(s3), H(s1))
+
+
+# ---- Mamba-1 form (A per channel and state) ---------------------------------
+
+from problems import m1_problem  # noqa: E402
+
+M1_CASES = [
+    # (b, d, N, G, gs, gate, bias, fmt)
+    (3, 64, 16, 1, 4, True, False, "int8"),
+    (2, 40, 4, 2, 2, False, True, "int8"),
+    (2, 24, 8, 1, 8, True, True, "softedge"),
+    (1, 16, 32, 4, 8, False, False, "int8"),
+    (2, 8, 64, 1, 16, True, False, "int8"),
+    (2, 8, 128, 2, 16, True, True, "int8"),
+]
+
+
+@pytest.mark.parametrize("ci", range(len(M1_CASES)))
+def test_m1_decode_chain_vs_oracle(orc, ci):
+    b, d, N_, G, gs, gate, bias, fmt = M1_CASES[ci]
+    steps = 20
+    p = m1_problem(500 + ci, b, steps, d, N_, G=G, gs=gs, gate=gate, h0=True, bias=bias,
+                   x_format=fmt)
+    state = T(p["h0"])
+    ref = p["h0"].astype(np.float64).reshape(b * d, N_).copy()
+    kw = dict(D=T(p["D"]), dt_bias=T(p["dt_bias"]))
+    okw = dict(D=p["D"], dt_bias=p["dt_bias"])
+    if fmt == "softedge":
+        kw["se_scale"] = okw["se_scale"] = p["se_scale"]
+    else:
+        kw.update(x_group=T(p["x_group"]), x_scale=T(p["x_scale"]))
+        okw.update(x_group=p["x_group"], x_scale=p["x_scale"])
+    for t in range(steps):
+        xt = np.ascontiguousarray(p["x"][:, :, t])
+        zt = None if p["z"] is None else np.ascontiguousarray(p["z"][:, :, t])
+        Bt = np.ascontiguousarray(p["B"][:, :, :, t])
+        Ct = np.ascontiguousarray(p["C"][:, :, :, t])
+        dtt = np.ascontiguousarray(p["dt"][:, :, t])
+        y = api.selective_state_update(state, T(xt), T(dtt), T(p["A"]), T(Bt), T(Ct),
+                                       T(p["B_scale"]), T(p["C_scale"]), gs, z=T(zt), **kw)
+        yo = orc.m1_decode_step(ref, xt, dtt, p["A"], Bt, Ct, p["B_scale"], p["C_scale"], gs,
+                                z=zt, **okw)
+        assert y_err(H(y).reshape(yo.shape), yo) <= Y_TOL
+    assert state_err(H(state).reshape(ref.shape), ref) <= STATE_TOL
+
+
+def test_m1_decode_equals_scan_steps():
+    """L single-token Mamba-1 steps reproduce the GPU scan's final state."""
+    p = m1_problem(520, 2, 64, 32, 16, gate=True, h0=True)
+    kw = dict(x_group=T(p["x_group"]), x_scale=T(p["x_scale"]), D=T(p["D"]))
+    _, hf = api.selective_scan(T(p["x"]), T(p["dt"]), T(p["A"]), T(p["B"]), T(p["C"]),
+                               T(p["B_scale"]), T(p["C_scale"]), 4, z=T(p["z"]), h0=T(p["h0"]),
+                               **kw)
+    state = T(p["h0"])
+    for t in range(64):
+        api.selective_state_update(state, T(np.ascontiguousarray(p["x"][:, :, t])),
+                                   T(np.ascontiguousarray(p["dt"][:, :, t])), T(p["A"]),
+                                   T(np.ascontiguousarray(p["B"][:, :, :, t])),
+                                   T(np.ascontiguousarray(p["C"][:, :, :, t])), T(p["B_scale"]),
+                                   T(p["C_scale"]), 4, z=T(np.ascontiguousarray(p["z"][:, :, t])),
+                                   **kw)
+    assert state_err(H(state), H(hf)) <= 1e-5
