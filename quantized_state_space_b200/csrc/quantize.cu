@@ -6,11 +6,14 @@
 // 11xxxxxx bytes.  Quamba2 abstract: one scale per cluster of x channels and
 // per block of B/C states.
 //
-// All kernels stream 16 elements per thread per iteration (16-byte stores of
-// codes, 16- or 64-byte loads of binary16 / fp32 inputs) over a grid-stride
-// loop sized to the SM count; they are HBM-bound.
+// The quantizer, the absmax pass and the encoder are HBM-bound streams: their
+// input flows through the bulk-copy pipeline of stream.cuh (64 KB in flight
+// per CTA, two CTAs per SM) and each consumer thread turns 16 elements into 16
+// code bytes stored with one 16-byte store.  The decoder (1 byte in, 4 out)
+// is store-bound and streams with plain 16-byte loads.
 #include "common.cuh"
 #include "internal.h"
+#include "stream.cuh"
 
 namespace ssmq {
 namespace {
@@ -152,6 +155,13 @@ __device__ __forceinline__ void quant_vec(const float (&x)[kVec], Idx e0, Idx mi
   *reinterpret_cast<uint4*>(q + e0) = o;
 }
 
+// Dynamic shared memory: the pipeline's stages and barriers, then (absmax
+// only) the per-CTA group accumulators.
+template <bool kF16>
+__host__ __device__ constexpr int acc_smem_offset() {
+  return (stream::smem_bytes<kF16 ? 2 : 4>() + 15) / 16 * 16;
+}
+
 // Column path (inner == 1, mid % 16 == 0): groups of 16 consecutive columns
 // that share one group id are marked in a per-CTA table (-1 otherwise).
 constexpr int kMaxU = 1024;
@@ -169,60 +179,44 @@ __device__ __forceinline__ const int* fill_ugrp(const int32_t* gmap, uint64_t mi
 }
 
 template <bool kF16, int kPath, typename Idx>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(stream::kThreads)
     quant_static_kernel(const void* __restrict__ src, Idx n, Idx mid, Idx inner,
                         const int32_t* __restrict__ gmap, int32_t n_groups,
                         const float* __restrict__ scales, int8_t* __restrict__ q,
                         uint32_t* status) {
+  extern __shared__ __align__(128) uint8_t smem[];
   __shared__ float2 tab[kMaxTab];
   __shared__ int ug_s[kPath == kPathCol ? kMaxU : 1];
   fill_tab(scales, n_groups, tab);
   const int* ugrp = kPath == kPathCol ? fill_ugrp(gmap, (uint64_t)mid, ug_s) : nullptr;
   uint32_t flags = 0;
-  const Idx nvec = (n + kVec - 1) / kVec;
-  const Idx stride = (Idx)gridDim.x * kThreads;
-  // two vectors in flight per thread
-  for (Idx v0 = (Idx)blockIdx.x * kThreads + threadIdx.x; v0 < nvec; v0 += 2 * stride) {
-    const Idx v1 = v0 + stride;
-    const bool f0 = v0 * kVec + kVec <= n;
-    const bool h1 = v1 < nvec;
-    const bool f1 = h1 && v1 * kVec + kVec <= n;
-    float x0[kVec], x1[kVec];
-    if (f0) load16<kF16>(src, v0 * kVec, x0);
-    if (f1) load16<kF16>(src, v1 * kVec, x1);
-#pragma unroll
-    for (int w = 0; w < 2; ++w) {
-      const Idx v = w ? v1 : v0;
-      if (w && !h1) break;
-      const Idx e0 = v * kVec;
-      if (w ? f1 : f0) {
-        quant_vec<kF16, kPath, Idx>(w ? x1 : x0, e0, mid, inner, gmap, n_groups, scales, tab,
-                                    ugrp, q, flags);
-      } else {
-        for (Idx e = e0; e < n; ++e) {
-          const int g = __ldg(gmap + (e / inner) % mid);
-          const bool okg = (unsigned)g < (unsigned)n_groups;
-          q[e] = (int8_t)quant_elem(load1<kF16>(src, e), okg ? __ldg(scales + g) : 0.0f, 0.0f,
-                                    okg, flags);
-        }
-      }
-    }
-  }
+  stream::run<kF16, Idx>(
+      src, n, smem,
+      [&](const float(&x)[kVec], Idx e0) {
+        quant_vec<kF16, kPath, Idx>(x, e0, mid, inner, gmap, n_groups, scales, tab, ugrp, q,
+                                    flags);
+      },
+      [&](float v, Idx e) {
+        const int g = __ldg(gmap + (e / inner) % mid);
+        const bool okg = (unsigned)g < (unsigned)n_groups;
+        q[e] = (int8_t)quant_elem(v, okg ? __ldg(scales + g) : 0.0f, 0.0f, okg, flags);
+      },
+      flags);
   flag_status(status, flags);
 }
 
 // Per-group max |v| into `acc` (the scales buffer viewed as uint32 bit
 // patterns: for non-negative floats the unsigned order is the float order).
 template <bool kF16, int kPath, typename Idx>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(stream::kThreads)
     absmax_kernel(const void* __restrict__ src, Idx n, Idx mid, Idx inner,
                   const int32_t* __restrict__ gmap, int32_t n_groups, unsigned* acc,
                   uint32_t* status, int use_smem) {
-  extern __shared__ unsigned s_acc[];
-  if (use_smem) {
-    for (int i = threadIdx.x; i < n_groups; i += kThreads) s_acc[i] = 0u;
-    __syncthreads();
-  }
+  extern __shared__ __align__(128) uint8_t smem[];
+  unsigned* s_acc = reinterpret_cast<unsigned*>(smem + acc_smem_offset<kF16>());
+  if (use_smem)
+    for (int i = threadIdx.x; i < n_groups; i += blockDim.x) s_acc[i] = 0u;
+  // (stream::run begins with a block barrier)
   unsigned* tgt = use_smem ? s_acc : acc;
   uint32_t flags = 0;
   int cur_g = -1;
@@ -245,32 +239,27 @@ __global__ void __launch_bounds__(kThreads)
       cur_m = max(cur_m, a);
     }
   };
-  const Idx nvec = (n + kVec - 1) / kVec;
-  for (Idx v = (Idx)blockIdx.x * kThreads + threadIdx.x; v < nvec; v += (Idx)gridDim.x * kThreads) {
-    const Idx e0 = v * kVec;
-    if (e0 + kVec <= n) {
-      float x[kVec];
-      load16<kF16>(src, e0, x);
-      if (kPath == kPathRow) {
-        const int g = __ldg(gmap + (e0 / inner) % mid);
+  stream::run<kF16, Idx>(
+      src, n, smem,
+      [&](const float(&x)[kVec], Idx e0) {
+        if (kPath == kPathRow) {
+          const int g = __ldg(gmap + (e0 / inner) % mid);
 #pragma unroll
-        for (int i = 0; i < kVec; ++i) push(g, x[i]);
-      } else if (kPath == kPathCol) {
-        const Idx m0 = e0 % mid;
+          for (int i = 0; i < kVec; ++i) push(g, x[i]);
+        } else if (kPath == kPathCol) {
+          const Idx m0 = e0 % mid;
 #pragma unroll
-        for (int i = 0; i < kVec; ++i) push(__ldg(gmap + m0 + i), x[i]);
-      } else {
+          for (int i = 0; i < kVec; ++i) push(__ldg(gmap + m0 + i), x[i]);
+        } else {
 #pragma unroll
-        for (int i = 0; i < kVec; ++i) push(__ldg(gmap + ((e0 + i) / inner) % mid), x[i]);
-      }
-    } else {
-      for (Idx e = e0; e < n; ++e) push(__ldg(gmap + (e / inner) % mid), load1<kF16>(src, e));
-    }
-  }
+          for (int i = 0; i < kVec; ++i) push(__ldg(gmap + ((e0 + i) / inner) % mid), x[i]);
+        }
+      },
+      [&](float v, Idx e) { push(__ldg(gmap + (e / inner) % mid), v); }, flags);
   if (cur_g >= 0 && cur_m) atomicMax(tgt + cur_g, cur_m);
   if (use_smem) {
     __syncthreads();
-    for (int i = threadIdx.x; i < n_groups; i += kThreads)
+    for (int i = threadIdx.x; i < n_groups; i += blockDim.x)
       if (s_acc[i]) atomicMax(acc + i, s_acc[i]);
   }
   flag_status(status, flags);
@@ -293,25 +282,47 @@ unsigned grid_for(Idx n) {
   return (unsigned)(b ? b : 1);
 }
 
+int sm_count() {
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  return sms > 0 ? sms : 148;
+}
+
+// Launches a pipeline kernel with `smem` bytes of dynamic shared memory.
+template <class... P, class... A>
+cudaError_t launch_stream(void (*kern)(P...), uint64_t n, size_t smem, cudaStream_t st,
+                          A... args) {
+  cudaError_t e =
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  kern<<<stream::grid_for(n, sm_count()), stream::kThreads, smem, st>>>(args...);
+  return cudaGetLastError();
+}
+
 template <bool kF16, int kPath, typename Idx>
 cudaError_t quantize_t(const void* src, Idx n, Idx mid, Idx inner, const int32_t* gmap,
                        int32_t n_groups, bool absmax, float* scales, int8_t* q,
                        uint32_t* status, cudaStream_t st) {
-  const unsigned grid = grid_for(n);
+  constexpr size_t pipe = (size_t)acc_smem_offset<kF16>();
+  cudaError_t e = cudaSuccess;
   if (absmax) {
-    cudaError_t e = cudaMemsetAsync(scales, 0, sizeof(float) * (size_t)n_groups, st);
+    e = cudaMemsetAsync(scales, 0, sizeof(float) * (size_t)n_groups, st);
     if (e != cudaSuccess) return e;
     const int use_smem = n_groups <= 8192;
-    if (n > 0)
-      absmax_kernel<kF16, kPath, Idx><<<grid, kThreads, use_smem ? n_groups * sizeof(unsigned) : 0,
-                                        st>>>(src, n, mid, inner, gmap, n_groups,
-                                              reinterpret_cast<unsigned*>(scales), status,
-                                              use_smem);
+    if (n > 0) {
+      e = launch_stream(absmax_kernel<kF16, kPath, Idx>, (uint64_t)n,
+                        pipe + (use_smem ? n_groups * sizeof(unsigned) : 0), st, src, n, mid,
+                        inner, gmap, n_groups, reinterpret_cast<unsigned*>(scales), status,
+                        use_smem);
+      if (e != cudaSuccess) return e;
+    }
     absmax_finalize_kernel<<<(n_groups + 255) / 256, 256, 0, st>>>(scales, n_groups);
   }
   if (n > 0)
-    quant_static_kernel<kF16, kPath, Idx>
-        <<<grid, kThreads, 0, st>>>(src, n, mid, inner, gmap, n_groups, scales, q, status);
+    e = launch_stream(quant_static_kernel<kF16, kPath, Idx>, (uint64_t)n, pipe, st, src, n, mid,
+                      inner, gmap, n_groups, (const float*)scales, q, status);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
@@ -381,30 +392,18 @@ __device__ __forceinline__ bool se16_fast(const float (&x)[kVec], float lo, floa
 }
 
 template <bool kF16, typename Idx>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(stream::kThreads)
     se_encode_kernel(const void* __restrict__ src, Idx n, float lo, float hi, SeSteps st,
                      uint8_t* __restrict__ codes, uint32_t* status) {
+  extern __shared__ __align__(128) uint8_t smem[];
   uint32_t flags = 0;
-  const Idx nvec = (n + kVec - 1) / kVec;
-  const Idx stride = (Idx)gridDim.x * kThreads;
-  for (Idx v0 = (Idx)blockIdx.x * kThreads + threadIdx.x; v0 < nvec; v0 += 2 * stride) {
-    const Idx v1 = v0 + stride;
-    const bool f0 = v0 * kVec + kVec <= n;
-    const bool h1 = v1 < nvec;
-    const bool f1 = h1 && v1 * kVec + kVec <= n;
-    float x0[kVec], x1[kVec];
-    if (f0) load16<kF16>(src, v0 * kVec, x0);
-    if (f1) load16<kF16>(src, v1 * kVec, x1);
-#pragma unroll
-    for (int w = 0; w < 2; ++w) {
-      if (w && !h1) break;
-      const Idx e0 = (w ? v1 : v0) * kVec;
-      if (w ? f1 : f0) {
-        const float(&x)[kVec] = w ? x1 : x0;
+  stream::run<kF16, Idx>(
+      src, n, smem,
+      [&](const float(&x)[kVec], Idx e0) {
         uint4 fast;
         if (se16_fast(x, lo, hi, st, fast)) {
           *reinterpret_cast<uint4*>(codes + e0) = fast;
-          continue;
+          return;
         }
         uint32_t wd[4];
 #pragma unroll
@@ -414,12 +413,8 @@ __global__ void __launch_bounds__(kThreads)
                   (se_encode1(x[4 * k + 2], lo, hi, st, flags) << 16) |
                   (se_encode1(x[4 * k + 3], lo, hi, st, flags) << 24);
         *reinterpret_cast<uint4*>(codes + e0) = make_uint4(wd[0], wd[1], wd[2], wd[3]);
-      } else {
-        for (Idx e = e0; e < n; ++e)
-          codes[e] = (uint8_t)se_encode1(load1<kF16>(src, e), lo, hi, st, flags);
-      }
-    }
-  }
+      },
+      [&](float v, Idx e) { codes[e] = (uint8_t)se_encode1(v, lo, hi, st, flags); }, flags);
   flag_status(status, flags);
 }
 
@@ -467,24 +462,19 @@ cudaError_t launch_softedge_encode(const void* src, bool f16, int64_t n, float s
                                    cudaStream_t st) {
   if (n == 0) return cudaSuccess;
   const SeSteps steps = se_steps(scale, log2_ratio);
+  const size_t smem = (size_t)acc_smem_offset<true>(), smem32 = (size_t)acc_smem_offset<false>();
   if ((uint64_t)n + 64 < (1ull << 32)) {
     const uint32_t n32 = (uint32_t)n;
-    if (f16)
-      se_encode_kernel<true, uint32_t><<<grid_for(n32), kThreads, 0, st>>>(src, n32, lo, hi, steps,
-                                                                           codes, status);
-    else
-      se_encode_kernel<false, uint32_t><<<grid_for(n32), kThreads, 0, st>>>(src, n32, lo, hi, steps,
-                                                                            codes, status);
-  } else {
-    const uint64_t n64 = (uint64_t)n;
-    if (f16)
-      se_encode_kernel<true, uint64_t><<<grid_for(n64), kThreads, 0, st>>>(src, n64, lo, hi, steps,
-                                                                           codes, status);
-    else
-      se_encode_kernel<false, uint64_t><<<grid_for(n64), kThreads, 0, st>>>(src, n64, lo, hi, steps,
-                                                                            codes, status);
+    return f16 ? launch_stream(se_encode_kernel<true, uint32_t>, (uint64_t)n, smem, st, src, n32,
+                               lo, hi, steps, codes, status)
+               : launch_stream(se_encode_kernel<false, uint32_t>, (uint64_t)n, smem32, st, src,
+                               n32, lo, hi, steps, codes, status);
   }
-  return cudaGetLastError();
+  const uint64_t n64 = (uint64_t)n;
+  return f16 ? launch_stream(se_encode_kernel<true, uint64_t>, n64, smem, st, src, n64, lo, hi,
+                             steps, codes, status)
+             : launch_stream(se_encode_kernel<false, uint64_t>, n64, smem32, st, src, n64, lo, hi,
+                             steps, codes, status);
 }
 
 cudaError_t launch_softedge_decode(const uint8_t* codes, int64_t n, float scale, int log2_ratio,
