@@ -9,6 +9,30 @@ namespace ssmq {
 
 constexpr float kLog2e = 1.4426950408889634f;
 
+// ---- packed fp32x2 arithmetic (sm_100: one instruction, two lanes) ---------
+__device__ __forceinline__ uint64_t pk(float2 v) { return *reinterpret_cast<uint64_t*>(&v); }
+__device__ __forceinline__ float2 upk(uint64_t v) { return *reinterpret_cast<float2*>(&v); }
+__device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(pk(a)), "l"(pk(b)));
+  return upk(d);
+}
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(pk(a)), "l"(pk(b)));
+  return upk(d);
+}
+__device__ __forceinline__ float2 fsub2(float2 a, float2 b) {
+  uint64_t d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(pk(a)), "l"(pk(b)));
+  return upk(d);
+}
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(pk(a)), "l"(pk(b)), "l"(pk(c)));
+  return upk(d);
+}
+
 __device__ __forceinline__ float h2f(uint16_t b) { return __half2float(__ushort_as_half(b)); }
 __device__ __forceinline__ uint16_t f2h(float v) { return __half_as_ushort(__float2half_rn(v)); }
 
@@ -139,7 +163,8 @@ __host__ inline SeSteps se_steps(float scale, int log2_ratio) {
 __device__ __forceinline__ float se_decode(uint32_t c, const SeSteps& st) {
   int q, mode;
   se_split(c, q, mode);
-  return (float)q * st.s[mode];
+  // selects, not an indexed load: keeps the steps in registers
+  return (float)q * (mode == 0 ? st.s[0] : (mode == 1 ? st.s[1] : st.s[2]));
 }
 
 __device__ __forceinline__ void flag_status(uint32_t* status, uint32_t bits) {

@@ -7,13 +7,14 @@
 // per block of B/C states.
 //
 // The quantizer, the absmax pass and the encoder are HBM-bound streams: their
-// input flows through the bulk-copy pipeline of stream.cuh (64 KB in flight
-// per CTA, two CTAs per SM) and each consumer thread turns 16 elements into 16
+// input flows through the bulk-copy pipeline of stream.cuh (48 KB in flight
+// per CTA, three CTAs per SM) and each consumer thread turns 16 elements into 16
 // code bytes stored with one 16-byte store.  The decoder (1 byte in, 4 out)
 // is store-bound and streams with plain 16-byte loads.
 #include "common.cuh"
 #include "internal.h"
 #include "stream.cuh"
+#include "fastdiv.h"
 
 namespace ssmq {
 namespace {
@@ -54,6 +55,28 @@ __device__ __forceinline__ float load1(const void* src, Idx e) {
   return static_cast<const float*>(src)[e];
 }
 
+// Index geometry of a (outer, mid, inner) tensor: mid_of(e) = (e / inner) %
+// mid is the group-map index of element e, col_of(e) = e % mid.  32-bit
+// indices divide by multiply-shift (fastdiv.h), 64-bit ones by division.
+template <typename Idx>
+struct Geo;
+template <>
+struct Geo<uint32_t> {
+  FastDiv inner, mid;
+  __device__ __forceinline__ uint32_t mid_of(uint32_t e) const { return fmod_(fdiv(e, inner), mid); }
+  __device__ __forceinline__ uint32_t col_of(uint32_t e) const { return fmod_(e, mid); }
+};
+template <>
+struct Geo<uint64_t> {
+  uint64_t inner, mid;
+  __device__ __forceinline__ uint64_t mid_of(uint64_t e) const { return (e / inner) % mid; }
+  __device__ __forceinline__ uint64_t col_of(uint64_t e) const { return e % mid; }
+};
+inline Geo<uint32_t> make_geo(uint32_t mid, uint32_t inner) {
+  return Geo<uint32_t>{make_fastdiv(inner), make_fastdiv(mid)};
+}
+inline Geo<uint64_t> make_geo(uint64_t mid, uint64_t inner) { return Geo<uint64_t>{inner, mid}; }
+
 // One element of the static quantizer; flags record device-side anomalies.
 // rs: reciprocal of s for the fast route, 0 to force the exact division.
 __device__ __forceinline__ int quant_elem(float v, float s, float rs, bool okg, uint32_t& flags) {
@@ -92,41 +115,52 @@ __device__ __forceinline__ uint32_t pack4(int a, int b, int c, int d) {
          ((uint32_t)(d & 0xFF) << 24);
 }
 
-// Branch-free fast route for 16 elements sharing one valid (s, rs): the code
-// byte of each element is the low byte of fl32(clamp(v rs) + 1.5 2^23) (that
-// sum holds 0x4B400000 + k for the integer k = rne(clamp(v rs))).  Returns
-// false when an element is non-finite or lies within 2^-14 of a tie, in which
-// case the caller redoes the vector element by element.
+// Branch-free fast route for 16 elements sharing one valid (s, rs) (the
+// argument of quant_rne_fast, in packed fp32x2 arithmetic): the code byte of
+// each element is the low byte of m = fl32(clamp(v rs) + 1.5 2^23), which
+// holds 0x4B400000 + k for the integer k = rne(clamp(v rs)).  Two running
+// reductions replace per-element tests: the largest |y - (m - 1.5 2^23)|
+// (at least 0.5 - 2^-14 only when some element lies within 2^-14 of a tie)
+// and the sum of v * 0 (NaN exactly when some v is not finite).  Returns false
+// in either case; the caller then redoes the vector element by element.
 __device__ __forceinline__ bool quant16_fast(const float (&x)[kVec], float rs, uint4& out) {
+  const float2 r2 = make_float2(rs, rs), mg = make_float2(12582912.0f, 12582912.0f);
+  const float2 zero = make_float2(0.0f, 0.0f);
+  float2 nf = zero;
+  float dmax = 0.0f;
   uint32_t mb[kVec];
-  bool bad = false;
 #pragma unroll
-  for (int i = 0; i < kVec; ++i) {
-    bad |= !(fabsf(x[i]) <= 3.402823466e38f);
-    const float yc = fminf(fmaxf(x[i] * rs, -127.0f), 127.0f);
-    const float m = yc + 12582912.0f;
-    bad |= fabsf(fabsf(yc - (m - 12582912.0f)) - 0.5f) < (1.0f / 16384.0f);
-    mb[i] = __float_as_uint(m);
+  for (int i = 0; i < kVec; i += 2) {
+    const float2 xv = make_float2(x[i], x[i + 1]);
+    float2 y = fmul2(xv, r2);
+    y.x = fminf(fmaxf(y.x, -127.0f), 127.0f);
+    y.y = fminf(fmaxf(y.y, -127.0f), 127.0f);
+    const float2 m = fadd2(y, mg);
+    const float2 d = fsub2(y, fsub2(m, mg));
+    dmax = fmaxf(dmax, fmaxf(fabsf(d.x), fabsf(d.y)));
+    nf = ffma2(xv, zero, nf);
+    mb[i] = __float_as_uint(m.x);
+    mb[i + 1] = __float_as_uint(m.y);
   }
   out.x = __byte_perm(__byte_perm(mb[0], mb[1], 0x0040), __byte_perm(mb[2], mb[3], 0x0040), 0x5410);
   out.y = __byte_perm(__byte_perm(mb[4], mb[5], 0x0040), __byte_perm(mb[6], mb[7], 0x0040), 0x5410);
   out.z = __byte_perm(__byte_perm(mb[8], mb[9], 0x0040), __byte_perm(mb[10], mb[11], 0x0040), 0x5410);
   out.w = __byte_perm(__byte_perm(mb[12], mb[13], 0x0040), __byte_perm(mb[14], mb[15], 0x0040), 0x5410);
-  return !bad;
+  return dmax < 0.5f - 1.0f / 16384.0f && nf.x == 0.0f && nf.y == 0.0f;
 }
 
 // One full 16-element vector of the static quantizer.
 template <bool kF16, int kPath, typename Idx>
-__device__ __forceinline__ void quant_vec(const float (&x)[kVec], Idx e0, Idx mid, Idx inner,
+__device__ __forceinline__ void quant_vec(const float (&x)[kVec], Idx e0, const Geo<Idx>& geo,
                                           const int32_t* __restrict__ gmap, int32_t n_groups,
                                           const float* __restrict__ scales, const float2* tab,
                                           const int* ugrp, int8_t* __restrict__ q,
                                           uint32_t& flags) {
   int gu = -1;  // one group for the whole vector, if known
   if (kPath == kPathRow) {
-    gu = __ldg(gmap + (e0 / inner) % mid);
+    gu = __ldg(gmap + geo.mid_of(e0));
   } else if (kPath == kPathCol && ugrp) {
-    gu = ugrp[(e0 % mid) >> 4];
+    gu = ugrp[geo.col_of(e0) >> 4];
   }
   if ((unsigned)gu < (unsigned)n_groups) {
     const float2 sr = tab_get(tab, scales, gu, n_groups);
@@ -141,8 +175,8 @@ __device__ __forceinline__ void quant_vec(const float (&x)[kVec], Idx e0, Idx mi
   for (int i = 0; i < kVec; ++i) {
     const int g = gu >= 0 || kPath == kPathRow
                       ? gu
-                      : (kPath == kPathCol ? __ldg(gmap + e0 % mid + i)
-                                           : __ldg(gmap + ((e0 + i) / inner) % mid));
+                      : (kPath == kPathCol ? __ldg(gmap + geo.col_of(e0) + i)
+                                           : __ldg(gmap + geo.mid_of(e0 + i)));
     const bool okg = (unsigned)g < (unsigned)n_groups;
     const float2 sr = okg ? tab_get(tab, scales, g, n_groups) : make_float2(0.0f, 0.0f);
     r[i] = quant_elem(x[i], sr.x, sr.y, okg, flags);
@@ -180,7 +214,7 @@ __device__ __forceinline__ const int* fill_ugrp(const int32_t* gmap, uint64_t mi
 
 template <bool kF16, int kPath, typename Idx>
 __global__ void __launch_bounds__(stream::kThreads)
-    quant_static_kernel(const void* __restrict__ src, Idx n, Idx mid, Idx inner,
+    quant_static_kernel(const void* __restrict__ src, Idx n, Idx mid, const Geo<Idx> geo,
                         const int32_t* __restrict__ gmap, int32_t n_groups,
                         const float* __restrict__ scales, int8_t* __restrict__ q,
                         uint32_t* status) {
@@ -193,11 +227,10 @@ __global__ void __launch_bounds__(stream::kThreads)
   stream::run<kF16, Idx>(
       src, n, smem,
       [&](const float(&x)[kVec], Idx e0) {
-        quant_vec<kF16, kPath, Idx>(x, e0, mid, inner, gmap, n_groups, scales, tab, ugrp, q,
-                                    flags);
+        quant_vec<kF16, kPath, Idx>(x, e0, geo, gmap, n_groups, scales, tab, ugrp, q, flags);
       },
       [&](float v, Idx e) {
-        const int g = __ldg(gmap + (e / inner) % mid);
+        const int g = __ldg(gmap + geo.mid_of(e));
         const bool okg = (unsigned)g < (unsigned)n_groups;
         q[e] = (int8_t)quant_elem(v, okg ? __ldg(scales + g) : 0.0f, 0.0f, okg, flags);
       },
@@ -209,7 +242,7 @@ __global__ void __launch_bounds__(stream::kThreads)
 // patterns: for non-negative floats the unsigned order is the float order).
 template <bool kF16, int kPath, typename Idx>
 __global__ void __launch_bounds__(stream::kThreads)
-    absmax_kernel(const void* __restrict__ src, Idx n, Idx mid, Idx inner,
+    absmax_kernel(const void* __restrict__ src, Idx n, const Geo<Idx> geo,
                   const int32_t* __restrict__ gmap, int32_t n_groups, unsigned* acc,
                   uint32_t* status, int use_smem) {
   extern __shared__ __align__(128) uint8_t smem[];
@@ -243,19 +276,19 @@ __global__ void __launch_bounds__(stream::kThreads)
       src, n, smem,
       [&](const float(&x)[kVec], Idx e0) {
         if (kPath == kPathRow) {
-          const int g = __ldg(gmap + (e0 / inner) % mid);
+          const int g = __ldg(gmap + geo.mid_of(e0));
 #pragma unroll
           for (int i = 0; i < kVec; ++i) push(g, x[i]);
         } else if (kPath == kPathCol) {
-          const Idx m0 = e0 % mid;
+          const Idx m0 = geo.col_of(e0);
 #pragma unroll
           for (int i = 0; i < kVec; ++i) push(__ldg(gmap + m0 + i), x[i]);
         } else {
 #pragma unroll
-          for (int i = 0; i < kVec; ++i) push(__ldg(gmap + ((e0 + i) / inner) % mid), x[i]);
+          for (int i = 0; i < kVec; ++i) push(__ldg(gmap + geo.mid_of(e0 + i)), x[i]);
         }
       },
-      [&](float v, Idx e) { push(__ldg(gmap + (e / inner) % mid), v); }, flags);
+      [&](float v, Idx e) { push(__ldg(gmap + geo.mid_of(e)), v); }, flags);
   if (cur_g >= 0 && cur_m) atomicMax(tgt + cur_g, cur_m);
   if (use_smem) {
     __syncthreads();
@@ -305,6 +338,7 @@ cudaError_t quantize_t(const void* src, Idx n, Idx mid, Idx inner, const int32_t
                        int32_t n_groups, bool absmax, float* scales, int8_t* q,
                        uint32_t* status, cudaStream_t st) {
   constexpr size_t pipe = (size_t)acc_smem_offset<kF16>();
+  const Geo<Idx> geo = make_geo(mid, inner);
   cudaError_t e = cudaSuccess;
   if (absmax) {
     e = cudaMemsetAsync(scales, 0, sizeof(float) * (size_t)n_groups, st);
@@ -312,16 +346,15 @@ cudaError_t quantize_t(const void* src, Idx n, Idx mid, Idx inner, const int32_t
     const int use_smem = n_groups <= 8192;
     if (n > 0) {
       e = launch_stream(absmax_kernel<kF16, kPath, Idx>, (uint64_t)n,
-                        pipe + (use_smem ? n_groups * sizeof(unsigned) : 0), st, src, n, mid,
-                        inner, gmap, n_groups, reinterpret_cast<unsigned*>(scales), status,
-                        use_smem);
+                        pipe + (use_smem ? n_groups * sizeof(unsigned) : 0), st, src, n, geo,
+                        gmap, n_groups, reinterpret_cast<unsigned*>(scales), status, use_smem);
       if (e != cudaSuccess) return e;
     }
     absmax_finalize_kernel<<<(n_groups + 255) / 256, 256, 0, st>>>(scales, n_groups);
   }
   if (n > 0)
     e = launch_stream(quant_static_kernel<kF16, kPath, Idx>, (uint64_t)n, pipe, st, src, n, mid,
-                      inner, gmap, n_groups, (const float*)scales, q, status);
+                      geo, gmap, n_groups, (const float*)scales, q, status);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
@@ -350,9 +383,9 @@ __device__ __forceinline__ uint32_t se_encode1(float v, float lo, float hi, cons
   }
   const float a = fabsf(v);
   const int mode = a < lo ? 1 : (a > hi ? 2 : 0);
-  const float step = st.s[mode];
+  const float step = mode == 0 ? st.s[0] : (mode == 1 ? st.s[1] : st.s[2]);
   const int lim = mode == 0 ? 63 : 31;
-  const float rs = st.rs[mode];
+  const float rs = mode == 0 ? st.rs[0] : (mode == 1 ? st.rs[1] : st.rs[2]);
   const int qv = (step > 0.0f && isfinite(step))
                      ? (rs != 0.0f ? quant_rne_fast(v, step, rs, lim) : quant_rne(v, step, lim))
                      : 0;
@@ -360,35 +393,41 @@ __device__ __forceinline__ uint32_t se_encode1(float v, float lo, float hi, cons
   return (mode == 1 ? 0x80u : 0xC0u) | (uint32_t)(qv & 0x3F);
 }
 
-// Branch-free fast route for 16 soft-edge codes: mode by compares, then the
-// quantizer's reciprocal + magic-number rounding with the mode's step and
-// clamp; the payload bits are the low bits of the rounding sum, masked to the
-// mode's width and or-ed with its prefix.  Returns false when an element is
-// non-finite, a mode's reciprocal is unusable, or an element lies within
-// 2^-14 of a rounding tie; the caller then encodes the vector element-wise.
+// Branch-free fast route for 16 soft-edge codes (every st.rs[] usable):
+// the mode by two compares, then quant16_fast's rounding with the mode's
+// reciprocal and clamp.  From the low byte b of the rounding sum (two's
+// complement k) the code is b & 0x7F (standard), (b & 0x3F) | 0x80 (small)
+// or b | 0xC0 (large, |k| <= 31).  Same fallback conditions as quant16_fast.
 __device__ __forceinline__ bool se16_fast(const float (&x)[kVec], float lo, float hi,
                                           const SeSteps& st, uint4& out) {
+  const float2 mg = make_float2(12582912.0f, 12582912.0f), zero = make_float2(0.0f, 0.0f);
+  float2 nf = zero;
+  float dmax = 0.0f;
   uint32_t cb[kVec];
-  bool bad = !(st.rs[0] != 0.0f && st.rs[1] != 0.0f && st.rs[2] != 0.0f);
 #pragma unroll
-  for (int i = 0; i < kVec; ++i) {
-    const float a = fabsf(x[i]);
-    bad |= !(a <= 3.402823466e38f);
-    const bool sm = a < lo, lg = a > hi;
-    const float rs = sm ? st.rs[1] : (lg ? st.rs[2] : st.rs[0]);
-    const float lim = (sm || lg) ? 31.0f : 63.0f;
-    const float yc = fminf(fmaxf(x[i] * rs, -lim), lim);
-    const float m = yc + 12582912.0f;
-    bad |= fabsf(fabsf(yc - (m - 12582912.0f)) - 0.5f) < (1.0f / 16384.0f);
-    const uint32_t mask = (sm || lg) ? 0x3Fu : 0x7Fu;
-    const uint32_t prefix = sm ? 0x80u : (lg ? 0xC0u : 0x00u);
-    cb[i] = (__float_as_uint(m) & mask) | prefix;
+  for (int i = 0; i < kVec; i += 2) {
+    const float2 xv = make_float2(x[i], x[i + 1]);
+    const bool s0 = fabsf(xv.x) < lo, l0 = fabsf(xv.x) > hi;
+    const bool s1 = fabsf(xv.y) < lo, l1 = fabsf(xv.y) > hi;
+    const float2 rs = make_float2(s0 ? st.rs[1] : (l0 ? st.rs[2] : st.rs[0]),
+                                  s1 ? st.rs[1] : (l1 ? st.rs[2] : st.rs[0]));
+    const float lim0 = (s0 || l0) ? 31.0f : 63.0f, lim1 = (s1 || l1) ? 31.0f : 63.0f;
+    float2 y = fmul2(xv, rs);
+    y.x = fminf(fmaxf(y.x, -lim0), lim0);
+    y.y = fminf(fmaxf(y.y, -lim1), lim1);
+    const float2 m = fadd2(y, mg);
+    const float2 d = fsub2(y, fsub2(m, mg));
+    dmax = fmaxf(dmax, fmaxf(fabsf(d.x), fabsf(d.y)));
+    nf = ffma2(xv, zero, nf);
+    const uint32_t b0 = __float_as_uint(m.x), b1 = __float_as_uint(m.y);
+    cb[i] = s0 ? ((b0 & 0x3Fu) | 0x80u) : (l0 ? (b0 | 0xC0u) : (b0 & 0x7Fu));
+    cb[i + 1] = s1 ? ((b1 & 0x3Fu) | 0x80u) : (l1 ? (b1 | 0xC0u) : (b1 & 0x7Fu));
   }
   out.x = __byte_perm(__byte_perm(cb[0], cb[1], 0x0040), __byte_perm(cb[2], cb[3], 0x0040), 0x5410);
   out.y = __byte_perm(__byte_perm(cb[4], cb[5], 0x0040), __byte_perm(cb[6], cb[7], 0x0040), 0x5410);
   out.z = __byte_perm(__byte_perm(cb[8], cb[9], 0x0040), __byte_perm(cb[10], cb[11], 0x0040), 0x5410);
   out.w = __byte_perm(__byte_perm(cb[12], cb[13], 0x0040), __byte_perm(cb[14], cb[15], 0x0040), 0x5410);
-  return !bad;
+  return dmax < 0.5f - 1.0f / 16384.0f && nf.x == 0.0f && nf.y == 0.0f;
 }
 
 template <bool kF16, typename Idx>
@@ -397,11 +436,12 @@ __global__ void __launch_bounds__(stream::kThreads)
                      uint8_t* __restrict__ codes, uint32_t* status) {
   extern __shared__ __align__(128) uint8_t smem[];
   uint32_t flags = 0;
+  const bool fast_ok = st.rs[0] != 0.0f && st.rs[1] != 0.0f && st.rs[2] != 0.0f;
   stream::run<kF16, Idx>(
       src, n, smem,
       [&](const float(&x)[kVec], Idx e0) {
         uint4 fast;
-        if (se16_fast(x, lo, hi, st, fast)) {
+        if (fast_ok && se16_fast(x, lo, hi, st, fast)) {
           *reinterpret_cast<uint4*>(codes + e0) = fast;
           return;
         }

@@ -63,20 +63,6 @@ struct M1Params {
   int vec_ok;
 };
 
-// ---- packed fp32x2 arithmetic (sm_100) ------------------------------------
-__device__ __forceinline__ uint64_t pk(float2 v) { return *reinterpret_cast<uint64_t*>(&v); }
-__device__ __forceinline__ float2 upk(uint64_t v) { return *reinterpret_cast<float2*>(&v); }
-__device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
-  uint64_t d;
-  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(pk(a)), "l"(pk(b)));
-  return upk(d);
-}
-__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
-  uint64_t d;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(pk(a)), "l"(pk(b)), "l"(pk(c)));
-  return upk(d);
-}
-
 // ---- cp.async (16-byte, L2-only) -------------------------------------------
 __device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc) {
   const uint32_t s = (uint32_t)__cvta_generic_to_shared(smem_dst);

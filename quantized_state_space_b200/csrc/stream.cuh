@@ -23,8 +23,8 @@ constexpr int kVec = 16;                       // elements per consumer thread p
 constexpr int kConsumers = 256;                // 8 consumer warps
 constexpr int kThreads = kConsumers + 32;      // + 1 producer warp
 constexpr int kTileElems = kConsumers * kVec;  // 4096
-constexpr int kInFlightBytes = 64 * 1024;      // per CTA
-constexpr int kCtasPerSm = 2;
+constexpr int kInFlightBytes = 48 * 1024;      // per CTA
+constexpr int kCtasPerSm = 3;
 constexpr uint32_t kWaitLimit = 1u << 20;      // mbarrier probes (~1 us each)
 
 template <int kEsz>
