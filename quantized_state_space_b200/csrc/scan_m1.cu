@@ -12,30 +12,36 @@
 //
 // Work decomposition.  Every (b, c, n) recurrence is owned by one thread from
 // t = 0 to L - 1, so each decay exp(delta A) is evaluated exactly once and no
-// carry pass is needed.  A CTA owns kCH channels of one batch row and one B/C
-// group and walks L in chunks of kT = 64 steps.  The raw bytes of chunk k + 1
-// (x codes, binary16 dt / z, int8 B / C rows) are fetched with cp.async into
-// a second shared-memory buffer while chunk k is scanned, so the recurrence
-// never waits on global memory.  Per chunk:
-//   stage    all threads turn the raw bytes of the chunk into (delta, delta x)
-//            per (c, t) and dequantised B, C rows laid out [t][n] (shared by
-//            every channel of the CTA);
-//   scan     thread (c, j) advances states 4j..4j+3 of channel c: one
-//            MUFU.EX2 per state update and packed fp32x2 FMA for the rest;
-//            the per-thread partial sums of C . h are combined across the
-//            N / 4 threads of a channel by a shuffle reduce-scatter, so each
-//            thread ends up owning the full y of one time step;
-//   store    all threads apply (y + D x) * silu(z) from the raw bytes and
-//            store binary16 y with 16-byte stores.
-// The state stays in registers across chunks; the final state is written once.
+// carry pass is needed: thread (c, j) of a CTA advances states 4j..4j+3 of
+// channel c (one MUFU.EX2 per state update, packed fp32x2 FMA for the rest)
+// and the N / 4 lanes of a channel, which share a warp, combine their partial
+// sums of C . h with a shuffle reduce-scatter.  A CTA owns kCH channels of
+// one batch row and one B/C group and walks L in chunks of kT steps, each cut
+// into segments of kSeg steps.  After scanning segment s of chunk k a warp,
+// in the same instruction stream,
+//   stores   y of segment s of chunk k for its own channels: (C.h + D x) *
+//            silu(z) from the raw bytes, binary16;
+//   stages   segment s of chunk k + 1 for its own channels: (delta, delta x)
+//            with delta = softplus(dt + bias), written in place over the
+//            values it has just consumed; and its share of the dequantised
+//            B, C rows of chunk k + 1 ([t][n], shared by the whole CTA,
+//            double-buffered);
+// so the special-function and FMA work of staging overlaps the recurrence.
+// Raw bytes (x codes, binary16 dt / z, int8 B / C rows) rotate through three
+// shared-memory buffers: chunk k (stores), k + 1 (staging) and k + 2, fetched
+// with cp.async one chunk ahead.  One block barrier per chunk.  The state
+// stays in registers; the final state is written once.
 #include "common.cuh"
 #include "internal.h"
 
 namespace ssmq {
 namespace {
 
-constexpr int kT = 64;    // time steps per chunk
-constexpr int kSeg = 16;  // time steps per staging work item (16 bytes of codes)
+constexpr int kT = 32;              // steps per chunk (one block barrier each)
+constexpr int kSeg = 16;            // steps per segment (scan / store / stage granule)
+constexpr int kSegs = kT / kSeg;
+constexpr int kSPL = 4;             // states per thread
+constexpr int kRawBufs = 3;         // stores of k, staging of k + 1, prefetch of k + 2
 
 struct M1Params {
   int64_t b, L, d, G;
@@ -101,38 +107,60 @@ struct Raw {
 
 template <int kN, int kCH>
 struct M1Smem {
-  Raw<kN, kCH> raw[2];                  // double-buffered raw bytes
-  __align__(16) float2 dd[kCH][kT + 2]; // (delta, delta x); 16-byte rows
-  __align__(16) float b[kT][kN];        // dequantised B, [t][n]
-  __align__(16) float c[kT][kN];        // dequantised C, [t][n]
-  float y[kCH][kT + 4];                 // C . h per (c, t)
+  Raw<kN, kCH> raw[kRawBufs];
+  __align__(16) float2 dd[kCH][kT + 2];   // (delta, delta x) of the chunk being scanned
+  __align__(16) float bc[2][2][kT][kN];   // [buffer][B, C][t][n], dequantised
+  __align__(16) float y[kCH][kSeg + 4];   // C . h of the current segment
+  float scale[2][kN];                     // B, C scale of each state
 };
+
+// kBytes (1, 2, 4, 8, 16 or 32) contiguous bytes of shared memory as words
+template <int kBytes>
+__device__ __forceinline__ void lds_words(const void* p, uint32_t (&w)[(kBytes + 3) / 4]) {
+  if constexpr (kBytes >= 16) {
+#pragma unroll
+    for (int i = 0; i < kBytes / 16; ++i) {
+      const uint4 v = reinterpret_cast<const uint4*>(p)[i];
+      w[4 * i] = v.x;
+      w[4 * i + 1] = v.y;
+      w[4 * i + 2] = v.z;
+      w[4 * i + 3] = v.w;
+    }
+  } else if constexpr (kBytes == 8) {
+    const uint2 v = *reinterpret_cast<const uint2*>(p);
+    w[0] = v.x;
+    w[1] = v.y;
+  } else if constexpr (kBytes == 4) {
+    w[0] = *reinterpret_cast<const uint32_t*>(p);
+  } else if constexpr (kBytes == 2) {
+    w[0] = *reinterpret_cast<const uint16_t*>(p);
+  } else {
+    w[0] = *reinterpret_cast<const uint8_t*>(p);
+  }
+}
 
 template <int kN, int kCH>
 __device__ __forceinline__ void fetch_chunk(const M1Params& p, Raw<kN, kCH>& r, int64_t bb, int g,
                                             int c0, int nc, int64_t t0, int tl, int tid, int NT) {
-  constexpr int SEGS = kT / kSeg;
   const int64_t d = p.d, L = p.L;
   if (p.vec_ok) {
-    // every row starts 16-byte aligned (L % 16 == 0): 16-byte cp.async pieces
-    for (int w = tid; w < kCH * SEGS; w += NT) {
-      const int c = w / SEGS, tb = (w % SEGS) * kSeg;
-      if (c >= nc || tb >= tl) continue;
-      const int64_t row = (bb * d + c0 + c) * L + t0 + tb;
-      cp_async16(&r.x[c][tb], static_cast<const uint8_t*>(p.x) + row);
-      cp_async16(&r.dt[c][tb], p.dt + row);
-      cp_async16(&r.dt[c][tb + 8], p.dt + row + 8);
-      if (p.z) {
-        cp_async16(&r.z[c][tb], p.z + row);
-        cp_async16(&r.z[c][tb + 8], p.z + row + 8);
-      }
+    // every row starts 16-byte aligned (L % 16 == 0) and tl % 16 == 0
+    constexpr int XP = kT / 16, DP = kT / 8;  // 16-byte pieces per row
+    for (int w = tid; w < kCH * DP; w += NT) {
+      const int c = w / DP, q = w % DP;
+      if (c >= nc || q * 8 >= tl) continue;
+      const int64_t row = (bb * d + c0 + c) * L + t0;
+      cp_async16(&r.dt[c][8 * q], p.dt + row + 8 * q);
+      if (p.z) cp_async16(&r.z[c][8 * q], p.z + row + 8 * q);
+      if (q < XP && q * 16 < tl)
+        cp_async16(&r.x[c][16 * q], static_cast<const uint8_t*>(p.x) + row + 16 * q);
     }
-    for (int w = tid; w < 2 * kN * SEGS; w += NT) {
-      const int which = w / (kN * SEGS), rem = w % (kN * SEGS);
-      const int n = rem % kN, tb = (rem / kN) * kSeg;
-      if (tb >= tl) continue;
-      const int64_t row = ((bb * p.G + g) * kN + n) * L + t0 + tb;
-      cp_async16(which ? &r.C[n][tb] : &r.B[n][tb], (which ? p.C : p.B) + row);
+    for (int w = tid; w < 2 * kN * XP; w += NT) {
+      const int which = w / (kN * XP), rem = w % (kN * XP);
+      const int n = rem / XP, q = rem % XP;
+      if (q * 16 >= tl) continue;
+      const int64_t row = ((bb * p.G + g) * kN + n) * L + t0 + 16 * q;
+      cp_async16(which ? &r.C[n][16 * q] : &r.B[n][16 * q], (which ? p.C : p.B) + row);
     }
   } else {
     // rows not 16-byte aligned: plain element loads, bounded by the row end
@@ -154,23 +182,15 @@ __device__ __forceinline__ void fetch_chunk(const M1Params& p, Raw<kN, kCH>& r, 
   }
 }
 
-template <int kN, int kCH, int kSPL, int kXFmt>
-__global__ void __launch_bounds__(kCH * (kN / kSPL))
-    m1_scan_kernel(const M1Params p) {
-  static_assert(kSPL == 2 || kSPL == 4, "2 or 4 states per thread");
-  constexpr int NP = kSPL / 2;  // fp32x2 pairs per thread
-  constexpr int LPC = kN / kSPL;
+template <int kN, int kCH, int kXFmt>
+__global__ void __launch_bounds__(kCH*(kN / kSPL)) m1_scan_kernel(const M1Params p) {
+  constexpr int NP = kSPL / 2;      // fp32x2 pairs per thread
+  constexpr int LPC = kN / kSPL;    // lanes per channel
   constexpr int NT = kCH * LPC;
-  constexpr int RW = kT + 2;   // float2 row: 16-byte aligned, conflict-free column reads
-  constexpr int RY = kT + 4;   // float row of the reduced sums
-  constexpr int SEGS = kT / kSeg;
+  constexpr int SPS = kSeg / LPC;   // steps per lane per segment (stores, staging)
+  static_assert(LPC >= 1 && LPC <= 16 && kSeg % LPC == 0, "lanes per channel");
   extern __shared__ __align__(16) uint8_t smem_bytes[];
   M1Smem<kN, kCH>& S = *reinterpret_cast<M1Smem<kN, kCH>*>(smem_bytes);
-  Raw<kN, kCH>* raw = S.raw;
-  float2 (*sDD)[RW] = S.dd;  // (delta, delta * x)
-  float (*sB)[kN] = S.b;
-  float (*sC)[kN] = S.c;
-  float (*sY)[RY] = S.y;
 
   const int tid = threadIdx.x;
   const int64_t bb = blockIdx.y;
@@ -182,11 +202,12 @@ __global__ void __launch_bounds__(kCH * (kN / kSPL))
   const int spg = kN / p.gs;
   uint32_t flags = 0;
 
-  // scan role: channel lc, states 4 lj .. 4 lj + 3
+  // this lane: channel lc, states 4 lj .. 4 lj + 3; staging / store steps
+  // lj * SPS .. + SPS of every segment of its channel
   const int lc = tid / LPC, lj = tid % LPC;
   const bool lvalid = lc < nc;
   const int64_t lch = c0 + lc;
-  float2 hp[NP], ap[NP];  // states 2i, 2i+1 of this thread's block of kSPL
+  float2 hp[NP], ap[NP];
 #pragma unroll
   for (int i = 0; i < NP; ++i) {
     const int n = lj * kSPL + 2 * i;
@@ -196,178 +217,175 @@ __global__ void __launch_bounds__(kCH * (kN / kSPL))
                                            __ldg(p.h0 + (bb * d + lch) * kN + n + 1))
                              : make_float2(0.0f, 0.0f);
   }
-
-  // per-channel constants of the staging role (item c = w / SEGS is fixed
-  // across chunks when NT is a multiple of kCH * SEGS or larger)
-  const int nchunks = (int)((L + kT - 1) / kT);
-  fetch_chunk<kN, kCH>(p, raw[0], bb, g, c0, nc, 0, (int)min((int64_t)kT, L), tid, NT);
-  cp_async_commit();
-
-  // y = (C . h + D x) * silu(z) of chunk kk, binary16, from its raw bytes
-  auto store_chunk = [&](int kk) {
-    const int64_t t0 = (int64_t)kk * kT;
-    const int tl = (int)min((int64_t)kT, L - t0);
-    Raw<kN, kCH>& r = raw[kk & 1];
-    for (int w = tid; w < kCH * SEGS; w += NT) {
-      const int c = w / SEGS, tb = (w % SEGS) * kSeg;
-      if (c >= nc || tb >= tl) continue;
-      const int64_t ch = c0 + c;
-      float xs = 1.0f;
-      if (kXFmt == SSMQ_X_INT8_GROUP) {
-        const int xg = __ldg(p.x_group + ch);
-        xs = (unsigned)xg < (unsigned)p.n_x_groups ? __ldg(p.x_scale + xg) : 0.0f;
-      }
-      const float Dc = p.D ? __ldg(p.D + ch) : 0.0f;
-      const int cnt = min(kSeg, tl - tb);
-      const uint4 xw = *reinterpret_cast<const uint4*>(&r.x[c][tb]);
-      const uint32_t xb[4] = {xw.x, xw.y, xw.z, xw.w};
-      uint32_t zw[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-      if (p.z) {
-        const uint4 z0 = *reinterpret_cast<const uint4*>(&r.z[c][tb]);
-        const uint4 z1 = *reinterpret_cast<const uint4*>(&r.z[c][tb + 8]);
-        zw[0] = z0.x; zw[1] = z0.y; zw[2] = z0.z; zw[3] = z0.w;
-        zw[4] = z1.x; zw[5] = z1.y; zw[6] = z1.z; zw[7] = z1.w;
-      }
-      uint32_t wv[kSeg / 2];
-#pragma unroll
-      for (int i = 0; i < kSeg; i += 2) {
-        float yv[2];
-        const float2 zf = __half22float2(*reinterpret_cast<const __half2*>(&zw[i >> 1]));
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int t = i + e;
-          const uint32_t code = (xb[t >> 2] >> (8 * (t & 3))) & 0xFFu;
-          const float xv = kXFmt == SSMQ_X_INT8_GROUP ? s8_to_f32(xb[t >> 2] ^ 0x80808080u, t & 3) * xs
-                                                      : se_decode(code, p.se);
-          float v = fmaf(Dc, xv, sY[c][tb + t]);
-          if (p.z) v *= silu_f(e ? zf.y : zf.x);
-          yv[e] = v;
-        }
-        wv[i / 2] = pack_half2(yv[0], yv[1]);
-      }
-      uint16_t* dst = p.y + (bb * d + ch) * L + t0 + tb;
-      if (p.vec_ok && cnt == kSeg) {
-        uint4* o = reinterpret_cast<uint4*>(dst);
-        o[0] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
-        o[1] = make_uint4(wv[4], wv[5], wv[6], wv[7]);
+  float xs = 1.0f, bias = 0.0f, Dc = 0.0f;
+  if (lvalid) {
+    if (kXFmt == SSMQ_X_INT8_GROUP) {
+      const int xg = __ldg(p.x_group + lch);
+      if ((unsigned)xg < (unsigned)p.n_x_groups) {
+        xs = __ldg(p.x_scale + xg);
       } else {
-        for (int i = 0; i < cnt; ++i) dst[i] = (uint16_t)(wv[i / 2] >> (16 * (i & 1)));
+        xs = 0.0f;
+        if (lj == 0) flags |= SSMQ_DEV_BAD_GROUP;
       }
     }
-    };
+    bias = p.dt_bias ? __ldg(p.dt_bias + lch) : 0.0f;
+    Dc = p.D ? __ldg(p.D + lch) : 0.0f;
+  }
+  for (int i = tid; i < 2 * kN; i += NT) {
+    const int which = i / kN, n = i % kN;
+    S.scale[which][n] = __ldg((which ? p.C_scale : p.B_scale) + g * spg + n / p.gs);
+  }
 
-  for (int k = 0; k < nchunks; ++k) {
-    const int64_t t0 = (int64_t)k * kT;
-    const int tl = (int)min((int64_t)kT, L - t0);
-    Raw<kN, kCH>& r = raw[k & 1];
-    cp_async_wait_all();
-    __syncthreads();  // raw bytes of chunk k landed; the scan of chunk k - 1 is complete
-    if (k > 0) store_chunk(k - 1);  // reads sY and the raw bytes of chunk k - 1 only
+  auto x_value = [&](uint32_t word, int e) -> float {
+    if (kXFmt == SSMQ_X_INT8_GROUP) return s8_to_f32(word ^ 0x80808080u, e) * xs;
+    return se_decode((word >> (8 * e)) & 0xFFu, p.se);
+  };
 
-    // ---- stage: (delta, delta x) per (c, t); B, C dequantised to [t][n]
-    for (int w = tid; w < kCH * SEGS; w += NT) {
-      const int c = w / SEGS, tb = (w % SEGS) * kSeg;
-      float xs = 1.0f, bias = 0.0f;
-      if (c < nc) {
-        const int64_t ch = c0 + c;
-        if (kXFmt == SSMQ_X_INT8_GROUP) {
-          const int xg = __ldg(p.x_group + ch);
-          if ((unsigned)xg < (unsigned)p.n_x_groups) {
-            xs = __ldg(p.x_scale + xg);
-          } else {
-            xs = 0.0f;
-            flags |= SSMQ_DEV_BAD_GROUP;
-          }
-        }
-        bias = p.dt_bias ? __ldg(p.dt_bias + ch) : 0.0f;
-      }
-      const uint4 xw = *reinterpret_cast<const uint4*>(&r.x[c][tb]);
-      const uint32_t xb[4] = {xw.x, xw.y, xw.z, xw.w};
-      const uint4 d0 = *reinterpret_cast<const uint4*>(&r.dt[c][tb]);
-      const uint4 d1 = *reinterpret_cast<const uint4*>(&r.dt[c][tb + 8]);
-      const uint32_t dw[8] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w};
-      float4 out[kSeg / 2];
+  // (delta, delta x) of steps s kSeg + lj SPS .. + SPS of this lane's channel,
+  // chunk with tl valid steps, from raw bytes r
+  auto stage_dd = [&](const Raw<kN, kCH>& r, int s, int tl) {
+    const int tb = s * kSeg + lj * SPS;
+    uint32_t xw[(SPS + 3) / 4], dw[(2 * SPS + 3) / 4];
+    lds_words<SPS>(&r.x[lc][tb], xw);
+    lds_words<2 * SPS>(&r.dt[lc][tb], dw);
 #pragma unroll
-      for (int i = 0; i < kSeg; i += 2) {
-        float dd[2], dx[2];
-        const float2 dtf = __half22float2(*reinterpret_cast<const __half2*>(&dw[i >> 1]));
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int t = i + e;
-          const uint32_t code = (xb[t >> 2] >> (8 * (t & 3))) & 0xFFu;
-          const float xv = kXFmt == SSMQ_X_INT8_GROUP ? s8_to_f32(xb[t >> 2] ^ 0x80808080u, t & 3) * xs
-                                                      : se_decode(code, p.se);
-          const float dv = (e ? dtf.y : dtf.x) + bias;
-          float delta = p.softplus ? softplus_f(dv) : dv;
-          if (c >= nc || tb + t >= tl) delta = 0.0f;
-          dd[e] = delta;
-          dx[e] = delta * xv;
-        }
-        out[i / 2] = make_float4(dd[0], dx[0], dd[1], dx[1]);
-      }
-      float4* dst = reinterpret_cast<float4*>(&sDD[c][tb]);
-#pragma unroll
-      for (int i = 0; i < kSeg / 2; ++i) dst[i] = out[i];
+    for (int i = 0; i < SPS; ++i) {
+      const float dv = h2f((uint16_t)(dw[i >> 1] >> (16 * (i & 1)))) + bias;
+      float delta = p.softplus ? softplus_f(dv) : dv;
+      if (!lvalid || tb + i >= tl) delta = 0.0f;
+      S.dd[lc][tb + i] = make_float2(delta, delta * x_value(xw[i >> 2], i & 3));
     }
-    for (int w = tid; w < 2 * kN * SEGS; w += NT) {
-      const int which = w / (kN * SEGS), rem = w % (kN * SEGS);
-      const int n = rem % kN, tb = (rem / kN) * kSeg;
-      const float sc = __ldg((which ? p.C_scale : p.B_scale) + g * spg + n / p.gs);
-      const uint4 qw = *reinterpret_cast<const uint4*>(which ? &r.C[n][tb] : &r.B[n][tb]);
-      const uint32_t qb[4] = {qw.x ^ 0x80808080u, qw.y ^ 0x80808080u, qw.z ^ 0x80808080u,
-                              qw.w ^ 0x80808080u};
-      float* dst = which ? &sC[0][0] : &sB[0][0];
+  };
+  // this thread's share of the dequantised B, C rows of segment s (8 steps of
+  // one row per item)
+  auto stage_bc = [&](const Raw<kN, kCH>& r, int s, int buf, int tl) {
+    for (int w = tid; w < 4 * kN; w += NT) {
+      const int which = w / (2 * kN), n = (w / 2) % kN, tb = s * kSeg + 8 * (w & 1);
+      const float sc = S.scale[which][n];
+      const uint2 qw = *reinterpret_cast<const uint2*>(which ? &r.C[n][tb] : &r.B[n][tb]);
+      const uint32_t q0 = qw.x ^ 0x80808080u, q1 = qw.y ^ 0x80808080u;
+      float* dst = &S.bc[buf][which][0][0];
 #pragma unroll
-      for (int i = 0; i < kSeg; ++i) {
-        const float v = s8_to_f32(qb[i >> 2], i & 3) * sc;
+      for (int i = 0; i < 8; ++i) {
+        const float v = s8_to_f32(i < 4 ? q0 : q1, i & 3) * sc;
         dst[(tb + i) * kN + n] = tb + i < tl ? v : 0.0f;
       }
     }
-    __syncthreads();
+  };
+  // y = (C.h + D x) silu(z) of steps s kSeg + lj SPS .. + SPS of this lane's
+  // channel, chunk starting at t0 with tl valid steps
+  auto store_seg = [&](const Raw<kN, kCH>& r, int s, int64_t t0, int tl) {
+    const int tb = s * kSeg + lj * SPS;
+    if (!lvalid || tb >= tl) return;
+    uint32_t xw[(SPS + 3) / 4], zw[(2 * SPS + 3) / 4];
+    lds_words<SPS>(&r.x[lc][tb], xw);
+    if (p.z) lds_words<2 * SPS>(&r.z[lc][tb], zw);
+    float yv[SPS];
+#pragma unroll
+    for (int i = 0; i < SPS; ++i) {
+      float v = fmaf(Dc, x_value(xw[i >> 2], i & 3), S.y[lc][lj * SPS + i]);
+      if (p.z) v *= silu_f(h2f((uint16_t)(zw[i >> 1] >> (16 * (i & 1)))));
+      yv[i] = v;
+    }
+    uint16_t* dst = p.y + (bb * d + lch) * L + t0 + tb;
+    if (p.vec_ok && SPS >= 2) {
+      // tl % 16 == 0: the whole run is valid
+      uint32_t wv[(SPS + 1) / 2];
+#pragma unroll
+      for (int i = 0; i < SPS; i += 2) wv[i / 2] = pack_half2(yv[i], yv[i + 1]);
+      if constexpr (SPS >= 8) {
+#pragma unroll
+        for (int i = 0; i < SPS / 8; ++i)
+          reinterpret_cast<uint4*>(dst)[i] =
+              make_uint4(wv[4 * i], wv[4 * i + 1], wv[4 * i + 2], wv[4 * i + 3]);
+      } else if constexpr (SPS == 4) {
+        *reinterpret_cast<uint2*>(dst) = make_uint2(wv[0], wv[1]);
+      } else {
+        *reinterpret_cast<uint32_t*>(dst) = wv[0];
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < SPS; ++i)
+        if (tb + i < tl) dst[i] = f2h(yv[i]);
+    }
+  };
 
-    // ---- prefetch the next chunk (into the buffer chunk k - 1 used) while
-    // this one is scanned
-    if (k + 1 < nchunks)
-      fetch_chunk<kN, kCH>(p, raw[(k + 1) & 1], bb, g, c0, nc, t0 + kT,
-                           (int)min((int64_t)kT, L - t0 - kT), tid, NT);
+  const int nchunks = (int)((L + kT - 1) / kT);
+  auto chunk_len = [&](int k) { return (int)min((int64_t)kT, L - (int64_t)k * kT); };
+
+  // prologue: raw bytes of chunks 0 and 1, chunk 0 staged
+  fetch_chunk<kN, kCH>(p, S.raw[0], bb, g, c0, nc, 0, chunk_len(0), tid, NT);
+  cp_async_commit();
+  cp_async_wait_all();
+  __syncthreads();
+  if (nchunks > 1) fetch_chunk<kN, kCH>(p, S.raw[1], bb, g, c0, nc, kT, chunk_len(1), tid, NT);
+  cp_async_commit();
+#pragma unroll
+  for (int s = 0; s < kSegs; ++s) {
+    stage_dd(S.raw[0], s, chunk_len(0));
+    stage_bc(S.raw[0], s, 0, chunk_len(0));
+  }
+
+  for (int k = 0; k < nchunks; ++k) {
+    const int64_t t0 = (int64_t)k * kT;
+    const int tl = chunk_len(k);
+    const bool has_next = k + 1 < nchunks;
+    const int tl_next = has_next ? chunk_len(k + 1) : 0;
+    const Raw<kN, kCH>& rcur = S.raw[k % kRawBufs];
+    const Raw<kN, kCH>& rnext = S.raw[(k + 1) % kRawBufs];
+    const float(*sB)[kN] = S.bc[k & 1][0];
+    const float(*sC)[kN] = S.bc[k & 1][1];
+    // chunk k staged and raw bytes of chunk k + 1 landed (every thread's
+    // copies); every warp is done with chunk k - 1, whose raw buffer and B/C
+    // buffer are free again
+    cp_async_wait_all();
+    __syncthreads();
+    if (k + 2 < nchunks)
+      fetch_chunk<kN, kCH>(p, S.raw[(k + 2) % kRawBufs], bb, g, c0, nc, t0 + 2 * kT,
+                           chunk_len(k + 2), tid, NT);
     cp_async_commit();
 
-    // ---- scan
-#pragma unroll 2
-    for (int tg = 0; tg < kT / LPC; ++tg) {
-      float part[LPC];
 #pragma unroll
-      for (int kk = 0; kk < LPC; ++kk) {
-        const int t = tg * LPC + kk;
-        const float2 dd = sDD[lc][t];
-        float2 bq[NP], cq[NP];
-        if (kSPL == 4) {
+    for (int s = 0; s < kSegs; ++s) {
+      // ---- scan segment s: kSeg / LPC groups of LPC steps; after each group
+      // lane lj holds y of step (group start + lj)
+#pragma unroll
+      for (int tg = 0; tg < kSeg / LPC; ++tg) {
+        float part[LPC];
+#pragma unroll
+        for (int kk = 0; kk < LPC; ++kk) {
+          const int t = s * kSeg + tg * LPC + kk;
+          const float2 dd = S.dd[lc][t];
+          float2 bq[NP], cq[NP];
           const float4 b4 = *reinterpret_cast<const float4*>(&sB[t][lj * kSPL]);
           const float4 c4 = *reinterpret_cast<const float4*>(&sC[t][lj * kSPL]);
           bq[0] = make_float2(b4.x, b4.y);
-          bq[NP - 1] = make_float2(b4.z, b4.w);
+          bq[1] = make_float2(b4.z, b4.w);
           cq[0] = make_float2(c4.x, c4.y);
-          cq[NP - 1] = make_float2(c4.z, c4.w);
-        } else {
-          bq[0] = *reinterpret_cast<const float2*>(&sB[t][lj * kSPL]);
-          cq[0] = *reinterpret_cast<const float2*>(&sC[t][lj * kSPL]);
-        }
-        const float2 dl = make_float2(dd.x, dd.x), dxv = make_float2(dd.y, dd.y);
-        float2 q = make_float2(0.0f, 0.0f);
+          cq[1] = make_float2(c4.z, c4.w);
+          const float2 dl = make_float2(dd.x, dd.x), dxv = make_float2(dd.y, dd.y);
+          float2 q = make_float2(0.0f, 0.0f);
 #pragma unroll
-        for (int i = 0; i < NP; ++i) {
-          const float2 r = fmul2(dl, ap[i]);
-          const float2 e = make_float2(ex2_sfu(r.x), ex2_sfu(r.y));
-          hp[i] = ffma2(e, hp[i], fmul2(dxv, bq[i]));
-          q = i == 0 ? fmul2(cq[i], hp[i]) : ffma2(cq[i], hp[i], q);
+          for (int i = 0; i < NP; ++i) {
+            const float2 r = fmul2(dl, ap[i]);
+            const float2 e = make_float2(ex2_sfu(r.x), ex2_sfu(r.y));
+            hp[i] = ffma2(e, hp[i], fmul2(dxv, bq[i]));
+            q = i == 0 ? fmul2(cq[i], hp[i]) : ffma2(cq[i], hp[i], q);
+          }
+          part[kk] = q.x + q.y;
         }
-        part[kk] = q.x + q.y;
+        S.y[lc][tg * LPC + lj] = reduce_scatter<LPC>(part, lj);
       }
-      sY[lc][tg * LPC + lj] = reduce_scatter<LPC>(part, lj);
+      __syncwarp();
+      store_seg(rcur, s, t0, tl);
+      if (has_next) {
+        // the warp has consumed these (delta, delta x) of its channels
+        stage_dd(rnext, s, tl_next);
+        stage_bc(rnext, s, (k + 1) & 1, tl_next);
+      }
+      __syncwarp();
     }
   }
-  __syncthreads();
-  store_chunk(nchunks - 1);
 
   if (lvalid && p.h_final)
 #pragma unroll
@@ -376,7 +394,7 @@ __global__ void __launch_bounds__(kCH * (kN / kSPL))
   flag_status(p.status, flags);
 }
 
-template <int kN, int kCH, int kSPL>
+template <int kN, int kCH>
 cudaError_t launch_m1(const M1Params& prm, int xfmt, int64_t batch, cudaStream_t st) {
   M1Params p = prm;
   const int dg = (int)(p.d / p.G);
@@ -384,8 +402,8 @@ cudaError_t launch_m1(const M1Params& prm, int xfmt, int64_t batch, cudaStream_t
   const dim3 grid((unsigned)(p.n_ctile * p.G), (unsigned)batch);
   const dim3 block(kCH * (kN / kSPL));
   const size_t smem = sizeof(M1Smem<kN, kCH>);
-  auto kern = xfmt == SSMQ_X_SOFTEDGE ? m1_scan_kernel<kN, kCH, kSPL, SSMQ_X_SOFTEDGE>
-                                      : m1_scan_kernel<kN, kCH, kSPL, SSMQ_X_INT8_GROUP>;
+  auto kern = xfmt == SSMQ_X_SOFTEDGE ? m1_scan_kernel<kN, kCH, SSMQ_X_SOFTEDGE>
+                                      : m1_scan_kernel<kN, kCH, SSMQ_X_INT8_GROUP>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   kern<<<grid, block, smem, st>>>(p);
@@ -432,11 +450,11 @@ cudaError_t launch_selective_scan(const ssmq_scan_args& a, cudaStream_t st) {
     return cudaSuccess;
   }
   switch (a.dstate) {
-    case 4: return launch_m1<4, 32, 4>(p, a.x_format, a.batch, st);
-    case 8: return launch_m1<8, 16, 4>(p, a.x_format, a.batch, st);
-    case 16: return launch_m1<16, 16, 4>(p, a.x_format, a.batch, st);
-    case 32: return launch_m1<32, 16, 4>(p, a.x_format, a.batch, st);
-    case 64: return launch_m1<64, 8, 4>(p, a.x_format, a.batch, st);
+    case 4: return launch_m1<4, 32>(p, a.x_format, a.batch, st);
+    case 8: return launch_m1<8, 16>(p, a.x_format, a.batch, st);
+    case 16: return launch_m1<16, 16>(p, a.x_format, a.batch, st);
+    case 32: return launch_m1<32, 16>(p, a.x_format, a.batch, st);
+    case 64: return launch_m1<64, 8>(p, a.x_format, a.batch, st);
     default: return cudaErrorInvalidValue;
   }
 }
