@@ -385,11 +385,12 @@ def _timed(torch, fn, reps):
     return a.elapsed_time(b) / reps / 1e3
 
 
-def form_decode(torch, dev, pk):
-    """decode8b: 1000 chained single-token state updates (b 64, H 128, P 64,
-    N 128, G 8), int8 inputs quantized ahead of the chain."""
+def setup_decode(torch, dev, steps=None):
+    """decode8b inputs for `steps` chained single-token updates (b 64, H 128,
+    P 64, N 128, G 8), int8 inputs quantized ahead of the chain; returns the
+    dims and step(t)."""
     from quantized_state_space_b200 import api, calibrate, synth
-    dm, raw = synth.workload_inputs("decode8b")
+    dm, raw = synth.workload_inputs("decode8b", **({"steps": steps} if steps else {}))
     b, H, P, N, G, gs, S, k = (dm["batch"], dm["nheads"], dm["headdim"], dm["dstate"],
                                dm["ngroups"], dm["state_group_size"], dm["steps"], dm["x_clusters"])
     T = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev)
@@ -406,10 +407,21 @@ def form_decode(torch, dev, pk):
     y = torch.empty((b, H, P), dtype=torch.float16, device=dev)
     del raw
 
+    def step(t):
+        api.state_update(state, xq[t], dt[t], A, Bq[t], Cq[t], bs_t, cs_t, gs, x_group=grp_t,
+                         x_scale=xs_t, D=D, y=y)
+
+    return dict(b=b, H=H, P=P, N=N, G=G, S=S, step=step)
+
+
+def form_decode(torch, dev, pk):
+    """decode8b: 1000 chained single-token state updates."""
+    c = setup_decode(torch, dev)
+    b, H, P, N, G, S = c["b"], c["H"], c["P"], c["N"], c["G"], c["S"]
+
     def chain():
         for t in range(S):
-            api.state_update(state, xq[t], dt[t], A, Bq[t], Cq[t], bs_t, cs_t, gs, x_group=grp_t,
-                             x_scale=xs_t, D=D, y=y)
+            c["step"](t)
 
     sec = _timed(torch, chain, 2) / S
     byts = 2 * b * H * P * N * 4 + b * H * P * (1 + 2) + b * H * 2 + 2 * b * G * N
@@ -423,9 +435,9 @@ def form_decode(torch, dev, pk):
             "l2": "state 268 MB exceeds L2"}
 
 
-def form_softedge(torch, dev, pk, mhz):
-    """softedge: encode binary16 x to soft-edge codes, quantize B/C, scan
-    (b 16, L 8192, d 1536, N 16, z gate)."""
+def setup_softedge(torch, dev):
+    """softedge inputs (b 16, L 8192, d 1536, N 16, z gate); returns the dims
+    and enc (binary16 x -> soft-edge codes), quant_bc, scan."""
     from quantized_state_space_b200 import api, calibrate, synth
     dm, raw = synth.workload_inputs("softedge")
     b, L, d, N, G, gs = (dm["batch"], dm["seqlen"], dm["dim"], dm["dstate"], dm["ngroups"],
@@ -455,6 +467,14 @@ def form_softedge(torch, dev, pk, mhz):
         api.selective_scan(codes, dt, A, Bq, Cq, bs_t, cs_t, gs, se_scale=s, D=D, z=z, y=y,
                            h_final=hf)
 
+    return dict(b=b, L=L, d=d, N=N, enc=enc, quant_bc=quant_bc, scan=scan)
+
+
+def form_softedge(torch, dev, pk, mhz):
+    """softedge: encode binary16 x to soft-edge codes, quantize B/C, scan."""
+    c = setup_softedge(torch, dev)
+    b, L, d, N = c["b"], c["L"], c["d"], c["N"]
+    enc, quant_bc, scan = c["enc"], c["quant_bc"], c["scan"]
     t_enc = _timed(torch, enc, 5)
     t_bc = _timed(torch, quant_bc, 5)
     t_scan = _timed(torch, scan, 3)
@@ -474,9 +494,9 @@ def form_softedge(torch, dev, pk, mhz):
                      "unit": "Gupdates/s", "frac": round(upd / t_scan / 1e9 / peak_upd, 4)}}
 
 
-def form_ssd(torch, dev, pk):
-    """ssd27b: quantize x / B / C and run the SSD chunked scan (b 4, L 4096,
-    H 80, P 64, N 128, G 1, chunk 256) on tcgen05."""
+def setup_ssd(torch, dev):
+    """ssd27b inputs (b 4, L 4096, H 80, P 64, N 128, G 1, chunk 256); returns
+    the dims and quant (x / B / C), ssd."""
     from quantized_state_space_b200 import api, calibrate, synth
     dm, raw = synth.workload_inputs("ssd27b")
     b, L, H, P, N, G, gs, k = (dm["batch"], dm["seqlen"], dm["nheads"], dm["headdim"],
@@ -505,6 +525,14 @@ def form_ssd(torch, dev, pk):
         api.ssd_chunk_scan(xq, dt, A, Bq, Cq, bs_t, cs_t, gs, chunk=dm["chunk"], x_group=grp_t,
                            x_scale=xs_t, D=D, y=y, h_final=hf)
 
+    return dict(b=b, L=L, H=H, P=P, N=N, G=G, quant=quant, ssd=ssd)
+
+
+def form_ssd(torch, dev, pk):
+    """ssd27b: quantize x / B / C and run the SSD chunked scan on tcgen05."""
+    c = setup_ssd(torch, dev)
+    b, L, H, P, N, G = c["b"], c["L"], c["H"], c["P"], c["N"], c["G"]
+    quant, ssd = c["quant"], c["ssd"]
     t_q = _timed(torch, quant, 5)
     t_s = _timed(torch, ssd, 5)
     q = 256  # the chunk length the algorithmic count refers to
@@ -587,6 +615,48 @@ def run_reference(args):
     print(json.dumps(out), flush=True)
 
 
+def run_kernel(args):
+    """Profiling aid: one kernel on its workload, `--warmup` untimed then
+    `--steps` timed launches (no benchmark line)."""
+    import torch
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    from quantized_state_space_b200 import api
+    name = args.kernel
+    if name in ("scan", "quantize"):
+        lay = Layer(dev, 0)
+        lay.quantize()
+        fn = lay.scan if name == "scan" else (
+            lambda: api.quantize_groups(lay.x, lay.b, lay.d, lay.L, lay.grp, lay.k,
+                                        scales=lay.xs, out=lay.xq))
+        label = "m130m " + ("selective scan" if name == "scan" else "x quantize (static scales)")
+    elif name == "ssd":
+        c = setup_ssd(torch, dev)
+        c["quant"]()
+        fn, label = c["ssd"], "ssd27b SSD chunk scan"
+    elif name in ("encode", "softedge-scan"):
+        c = setup_softedge(torch, dev)
+        c["enc"]()
+        c["quant_bc"]()
+        fn = c["enc"] if name == "encode" else c["scan"]
+        label = "softedge " + ("encode" if name == "encode" else "scan of soft-edge codes")
+    else:  # decode
+        c = setup_decode(torch, dev, steps=args.warmup + args.steps + 1)
+        it = iter(range(args.warmup + args.steps + 1))
+        fn, label = (lambda: c["step"](next(it))), "decode8b single-token update"
+    for _ in range(args.warmup):
+        fn()
+    torch.cuda.synchronize()
+    if args.steps > 1:
+        ms = _timed(torch, fn, args.steps - 1) * 1e3  # first timed-region launch included
+    else:
+        fn()
+        torch.cuda.synchronize()
+        ms = None
+    print(json.dumps({"kernel": label, "ms_per_launch": ms, "launches": args.warmup + args.steps}),
+          flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -597,8 +667,13 @@ def main():
     ap.add_argument("--no-forms", action="store_true")
     ap.add_argument("--forms", default="", help="comma list of ssd27b,decode8b,softedge")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--kernel", choices=["scan", "quantize", "ssd", "encode", "softedge-scan",
+                                         "decode"],
+                    help="profiling aid: run only this kernel on its workload")
     args = ap.parse_args()
-    if args.impl == "reference":
+    if args.kernel:
+        run_kernel(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_ours(args)

@@ -40,7 +40,6 @@ namespace {
 constexpr int kT = 32;              // steps per chunk (one block barrier each)
 constexpr int kSeg = 16;            // steps per segment (scan / store / stage granule)
 constexpr int kSegs = kT / kSeg;
-constexpr int kSPL = 4;             // states per thread
 constexpr int kRawBufs = 3;         // stores of k, staging of k + 1, prefetch of k + 2
 
 struct M1Params {
@@ -182,8 +181,9 @@ __device__ __forceinline__ void fetch_chunk(const M1Params& p, Raw<kN, kCH>& r, 
   }
 }
 
-template <int kN, int kCH, int kXFmt>
+template <int kN, int kCH, int kSPL, int kXFmt>
 __global__ void __launch_bounds__(kCH*(kN / kSPL)) m1_scan_kernel(const M1Params p) {
+  static_assert(kSPL == 2 || kSPL == 4, "2 or 4 states per thread");
   constexpr int NP = kSPL / 2;      // fp32x2 pairs per thread
   constexpr int LPC = kN / kSPL;    // lanes per channel
   constexpr int NT = kCH * LPC;
@@ -259,8 +259,9 @@ __global__ void __launch_bounds__(kCH*(kN / kSPL)) m1_scan_kernel(const M1Params
   // this thread's share of the dequantised B, C rows of segment s (8 steps of
   // one row per item)
   auto stage_bc = [&](const Raw<kN, kCH>& r, int s, int buf, int tl) {
-    for (int w = tid; w < 4 * kN; w += NT) {
-      const int which = w / (2 * kN), n = (w / 2) % kN, tb = s * kSeg + 8 * (w & 1);
+    constexpr int H = kSeg / 8;  // items per row and segment
+    for (int w = tid; w < 2 * kN * H; w += NT) {
+      const int which = w / (kN * H), n = (w / H) % kN, tb = s * kSeg + 8 * (w % H);
       const float sc = S.scale[which][n];
       const uint2 qw = *reinterpret_cast<const uint2*>(which ? &r.C[n][tb] : &r.B[n][tb]);
       const uint32_t q0 = qw.x ^ 0x80808080u, q1 = qw.y ^ 0x80808080u;
@@ -357,12 +358,17 @@ __global__ void __launch_bounds__(kCH*(kN / kSPL)) m1_scan_kernel(const M1Params
           const int t = s * kSeg + tg * LPC + kk;
           const float2 dd = S.dd[lc][t];
           float2 bq[NP], cq[NP];
-          const float4 b4 = *reinterpret_cast<const float4*>(&sB[t][lj * kSPL]);
-          const float4 c4 = *reinterpret_cast<const float4*>(&sC[t][lj * kSPL]);
-          bq[0] = make_float2(b4.x, b4.y);
-          bq[1] = make_float2(b4.z, b4.w);
-          cq[0] = make_float2(c4.x, c4.y);
-          cq[1] = make_float2(c4.z, c4.w);
+          if constexpr (kSPL == 4) {
+            const float4 b4 = *reinterpret_cast<const float4*>(&sB[t][lj * kSPL]);
+            const float4 c4 = *reinterpret_cast<const float4*>(&sC[t][lj * kSPL]);
+            bq[0] = make_float2(b4.x, b4.y);
+            bq[NP - 1] = make_float2(b4.z, b4.w);
+            cq[0] = make_float2(c4.x, c4.y);
+            cq[NP - 1] = make_float2(c4.z, c4.w);
+          } else {
+            bq[0] = *reinterpret_cast<const float2*>(&sB[t][lj * kSPL]);
+            cq[0] = *reinterpret_cast<const float2*>(&sC[t][lj * kSPL]);
+          }
           const float2 dl = make_float2(dd.x, dd.x), dxv = make_float2(dd.y, dd.y);
           float2 q = make_float2(0.0f, 0.0f);
 #pragma unroll
@@ -394,7 +400,7 @@ __global__ void __launch_bounds__(kCH*(kN / kSPL)) m1_scan_kernel(const M1Params
   flag_status(p.status, flags);
 }
 
-template <int kN, int kCH>
+template <int kN, int kCH, int kSPL>
 cudaError_t launch_m1(const M1Params& prm, int xfmt, int64_t batch, cudaStream_t st) {
   M1Params p = prm;
   const int dg = (int)(p.d / p.G);
@@ -402,8 +408,8 @@ cudaError_t launch_m1(const M1Params& prm, int xfmt, int64_t batch, cudaStream_t
   const dim3 grid((unsigned)(p.n_ctile * p.G), (unsigned)batch);
   const dim3 block(kCH * (kN / kSPL));
   const size_t smem = sizeof(M1Smem<kN, kCH>);
-  auto kern = xfmt == SSMQ_X_SOFTEDGE ? m1_scan_kernel<kN, kCH, SSMQ_X_SOFTEDGE>
-                                      : m1_scan_kernel<kN, kCH, SSMQ_X_INT8_GROUP>;
+  auto kern = xfmt == SSMQ_X_SOFTEDGE ? m1_scan_kernel<kN, kCH, kSPL, SSMQ_X_SOFTEDGE>
+                                      : m1_scan_kernel<kN, kCH, kSPL, SSMQ_X_INT8_GROUP>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   kern<<<grid, block, smem, st>>>(p);
@@ -450,11 +456,11 @@ cudaError_t launch_selective_scan(const ssmq_scan_args& a, cudaStream_t st) {
     return cudaSuccess;
   }
   switch (a.dstate) {
-    case 4: return launch_m1<4, 32>(p, a.x_format, a.batch, st);
-    case 8: return launch_m1<8, 16>(p, a.x_format, a.batch, st);
-    case 16: return launch_m1<16, 16>(p, a.x_format, a.batch, st);
-    case 32: return launch_m1<32, 16>(p, a.x_format, a.batch, st);
-    case 64: return launch_m1<64, 8>(p, a.x_format, a.batch, st);
+    case 4: return launch_m1<4, 32, 4>(p, a.x_format, a.batch, st);
+    case 8: return launch_m1<8, 16, 4>(p, a.x_format, a.batch, st);
+    case 16: return launch_m1<16, 16, 4>(p, a.x_format, a.batch, st);
+    case 32: return launch_m1<32, 16, 4>(p, a.x_format, a.batch, st);
+    case 64: return launch_m1<64, 8, 4>(p, a.x_format, a.batch, st);
     default: return cudaErrorInvalidValue;
   }
 }
