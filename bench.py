@@ -15,6 +15,7 @@ cores) on a bounded sample of the same workload.
 """
 import argparse
 import datetime
+import hashlib
 import json
 import os
 import statistics
@@ -32,6 +33,22 @@ UNIT = "Gtokens·ch/s"
 WORKLOAD = "m130m"
 SMS = 148
 MUFU_PER_CLK = 16  # ex2 results per clock per SM (SFU)
+
+
+def measured_traffic(kernel):
+    """DRAM bytes per launch of `kernel` from one ncu capture
+    (profiles/traffic.json: dram__bytes_read.sum + dram__bytes_write.sum),
+    or None once any of its source files has changed since that capture."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            e = json.load(f)["kernels"][kernel]
+        h = hashlib.sha256()
+        for rel in e["sources"]:
+            with open(os.path.join(ROOT, rel), "rb") as f:
+                h.update(f.read())
+        return e["bytes_per_launch"] if h.hexdigest() == e["sha256"] else None
+    except (OSError, KeyError, ValueError):
+        return None
 
 
 def peaks():
@@ -345,7 +362,7 @@ def run_ours(args):
             "roofline": {"bound": "alu", "kernel": "m1_scan_kernel (selective scan)",
                          "achieved": round(achieved_upd, 2), "peak": round(peak_upd, 1),
                          "unit": "Gupdates/s", "frac": round(achieved_upd / peak_upd, 4),
-                         "traffic": None,
+                         "traffic": measured_traffic("m1_scan_kernel"),
                          "peak_basis": "%d SMs x %d ex2/clk (SFU) x %.0f MHz; one exp per "
                                        "state update" % (SMS, MUFU_PER_CLK, mhz_max),
                          "hbm_achieved_gbs": round(scan_gbs, 1), "hbm_peak_gbs": pk["hbm_gbs"],
@@ -431,7 +448,8 @@ def form_decode(torch, dev, pk):
             "roofline": {"bound": "hbm", "achieved": round(byts / sec / 1e9, 1),
                          "peak": pk["hbm_gbs"], "unit": "GB/s",
                          "frac": round(byts / sec / 1e9 / pk["hbm_gbs"], 4),
-                         "algorithmic_bytes_per_launch": byts, "traffic": None},
+                         "algorithmic_bytes_per_launch": byts,
+                         "traffic": measured_traffic("decode_kernel")},
             "l2": "state 268 MB exceeds L2"}
 
 
@@ -553,7 +571,7 @@ def form_ssd(torch, dev, pk):
                          "executed_mma_flops_per_launch": executed,
                          "hbm_achieved_gbs": round(byts / t_s / 1e9, 1),
                          "hbm_frac": round(byts / t_s / 1e9 / pk["hbm_gbs"], 4),
-                         "traffic": None}}
+                         "traffic": measured_traffic("ssd_kernel")}}
 
 
 def run_forms(dev, pk, mhz, only=None):
