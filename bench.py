@@ -558,7 +558,7 @@ def form_ssd(torch, dev, pk):
     useful = (2 * q * (q + 1) // 2 * N * b * nch * G          # C B^T, causal half
               + 2 * q * (q + 1) // 2 * P * b * nch * H        # diagonal blocks
               + 2 * 2 * q * N * P * b * nch * H)              # carried state in and out
-    executed = 2 * b * H * (L // 128) * (128 ** 3 + 128 * 128 * 64 * 5)
+    executed = 2 * b * H * (L // 128) * (128 ** 3 + 128 * 128 * 64 * 4)  # CB, Y_diag, Y_off, 2 x state
     byts = b * L * H * P * (1 + 2) + b * L * H * 2 + 2 * b * L * G * N + b * H * P * N * 4
     tf = useful / t_s / 1e12
     return {"workload": "ssd27b: b 4, L 4096, H 80, P 64, N 128, G 1, chunk 256; quantize + SSD",

@@ -16,16 +16,21 @@
 // cores only see exact int8 values (as binary16) or power-of-two-normalised
 // binary16 operands:
 //   - C and B are int8 codes (exact); the per-state-group scales enter as
-//     w'_n = sC_n sB_n / max_n(sC sB) on C (one rounding, range <= 127);
+//     w'_n = fl16(sC_n sB_n / max_n(sC sB)) on C (C' = fl16(c w'_n), one
+//     packed half2 multiply); the state operand of MMA2 carries sC_n / w'_n
+//     so the rounding of w' cancels there;
 //   - each row of M is scaled by a power of two so its largest entry lies in
 //     [2^14, 2^15) (undone in fp32 after the MMA);
-//   - the state operand of MMA2 and the w X operand of MMA3 are split into a
-//     binary16 high part and a binary16 residual (two MMAs each), with a
-//     tile-wide power-of-two normalisation: the state then carries ~22 bits.
+//   - the w X operand of MMA3 is split into a binary16 high part and a
+//     binary16 residual (two MMAs), with a tile-wide power-of-two
+//     normalisation, so the state increments carry ~22 bits; the state
+//     operand of MMA2 (which only feeds y) is one normalised binary16 value.
 // One CTA (16 warps) owns one (batch, head) and walks the sequence in tiles;
+// warp 0 prepares the next tile's decay factors while the others finish the
+// current tile's outputs;
 // the fp32 state lives in registers (row n, 16 of the 64 p per thread: warp w
 // reads TMEM lanes 32 (w % 4).. and columns 16 (w / 4)..), accumulators in
-// TMEM (512 columns), operands in shared memory (222 KB, including the raw
+// TMEM (512 columns), operands in shared memory (209 KB, including the raw
 // int8 rows of the next tile, prefetched with cp.async during this one).
 // The chunk length of the interface only fixes where the decomposition
 // restarts; the result is the recurrence's for any length, so the kernel uses
@@ -50,22 +55,24 @@ constexpr int OFF_B = OFF_C + kQ * kN * 2;      // B codes          [s][n]      
 constexpr int OFF_X = OFF_B + kQ * kN * 2;      // x (exact)        [s][p]  MN-major  16 KB
 constexpr int OFF_XH = OFF_X + kQ * kP * 2;     // w x hi           [s][p]            16 KB
 constexpr int OFF_XL = OFF_XH + kQ * kP * 2;    // w x lo                             16 KB
-constexpr int OFF_HH = OFF_XL + kQ * kP * 2;    // state hi         [n][p]  MN-major  16 KB
-constexpr int OFF_HL = OFF_HH + kN * kP * 2;    // state lo                           16 KB
-constexpr int OFF_M = OFF_HL + kN * kP * 2;     // M                [t][s]  K-major   32 KB
+constexpr int OFF_HH = OFF_XL + kQ * kP * 2;    // state            [n][p]  MN-major  16 KB
+constexpr int OFF_M = OFF_HH + kN * kP * 2;     // M                [t][s]  K-major   32 KB
 constexpr int OFF_F = OFF_M + kQ * kQ * 2;      // fp32 scalars
-// fp32 scalar arrays (in floats, from OFF_F)
-constexpr int F_S2 = 0;            // S_t * log2(e)            [128]
-constexpr int F_DW = F_S2 + kQ;    // delta_s                  [128]
-constexpr int F_WX = F_DW + kQ;    // w_s = exp(S_last-S_s) d_s [128]
-constexpr int F_ES = F_WX + kQ;    // exp(S_t)                 [128]
-constexpr int F_RS = F_ES + kQ;    // 2^e_t row scale of M     [128]
-constexpr int F_RM = F_RS + kQ;    // row max quarters         [4][128]
-constexpr int F_WN = F_RM + 4 * kQ;  // w'_n                   [128]
-constexpr int F_SB = F_WN + kN;    // sB_n                     [128]
-constexpr int F_SX = F_SB + kN;    // x scale per p            [64]
-constexpr int F_CW = F_SX + kP;    // exp(S_p(s) - S_s) d_s w_max, p(s) = s | 31  [128]
-constexpr int F_RED = F_CW + kQ;   // reductions               [32]
+// fp32 scalar arrays (in floats, from OFF_F).  The per-step arrays of a tile
+// are double-buffered: warp 0 fills the next tile's while the others finish
+// this one.
+constexpr int F_S2 = 0;                 // S_t * log2(e)                       [2][128]
+constexpr int F_DW = F_S2 + 2 * kQ;     // delta_s                             [2][128]
+constexpr int F_WX = F_DW + 2 * kQ;     // w_s = exp(S_last - S_s) delta_s      [2][128]
+constexpr int F_ES = F_WX + 2 * kQ;     // exp(S_t)                            [2][128]
+constexpr int F_CW = F_ES + 2 * kQ;     // exp(S_p(s) - S_s) d_s w_max, p(s) = s | 31  [2][128]
+constexpr int F_RS = F_CW + 2 * kQ;     // 2^e_t row scale of M                [128]
+constexpr int F_RM = F_RS + kQ;         // row max quarters                    [4][128]
+constexpr int F_WH = F_RM + 4 * kQ;     // w'_n as binary16 pairs              [64]
+constexpr int F_HF = F_WH + kN / 2;     // sC_n / w'_n (state operand factor)  [128]
+constexpr int F_SB = F_HF + kN;         // sB_n                                [128]
+constexpr int F_SX = F_SB + kN;         // x scale per p                       [64]
+constexpr int F_RED = F_SX + kP;        // reductions: w max, S_last, per-warp state max  [32]
 constexpr int F_END = F_RED + 32;
 // raw int8 rows of the next tile, fetched with cp.async during this tile
 constexpr int OFF_RAW = (OFF_F + F_END * 4 + 127) / 128 * 128;
@@ -167,6 +174,64 @@ __device__ __forceinline__ void fetch_tile(const SsdParams& p, uint8_t* smem, in
   tc::cp_async_commit();
 }
 
+// Warp 0: delta, S = cumsum(delta A) (log2 units) and the per-step factors of
+// the tile of ql steps whose dt values the lanes hold (4 steps per lane),
+// into buffer fb; the tile's w max and S_last go to F_RED[0], F_RED[1].
+__device__ __forceinline__ void tile_factors(float* F, int fb, int ql, const float (&dtv)[4],
+                                             float bias, int softplus, float A2, float wmax,
+                                             int lane) {
+  float dl[4], sc[4];
+  float run = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int t = 4 * lane + i;
+    float d = 0.0f;
+    if (t < ql) {
+      const float v = dtv[i] + bias;
+      d = softplus ? softplus_f(v) : v;
+    }
+    dl[i] = d;
+    run += d * A2;
+    sc[i] = run;
+  }
+  float ex = run;  // inclusive scan of the lane totals
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const float n = __shfl_up_sync(0xffffffffu, ex, o);
+    if (lane >= o) ex += n;
+  }
+  const float off = ex - run;
+  const float s_last = __shfl_sync(0xffffffffu, ex, 31);
+  float wmx = 0.0f;
+  // S at the end of this lane's 32-step column block (lane 8 b + 7 holds it)
+  const float s_blk = __shfl_sync(0xffffffffu, sc[3] + off, lane | 7);
+  float4 s2v, dwv, wxv, esv, cwv;
+  float* o4[5] = {&s2v.x, &dwv.x, &wxv.x, &esv.x, &cwv.x};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float s2 = sc[i] + off;
+    const float w = ex2_sfu(s_last - s2) * dl[i];
+    o4[0][i] = s2;
+    o4[1][i] = dl[i];
+    o4[2][i] = w;
+    o4[3][i] = ex2_sfu(s2);
+    o4[4][i] = ex2_sfu(s_blk - s2) * dl[i] * wmax;
+    wmx = fmaxf(wmx, w);
+  }
+  const int t0 = fb * kQ + 4 * lane;
+  *reinterpret_cast<float4*>(F + F_S2 + t0) = s2v;
+  *reinterpret_cast<float4*>(F + F_DW + t0) = dwv;
+  *reinterpret_cast<float4*>(F + F_WX + t0) = wxv;
+  *reinterpret_cast<float4*>(F + F_ES + t0) = esv;
+  *reinterpret_cast<float4*>(F + F_CW + t0) = cwv;
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) wmx = fmaxf(wmx, __shfl_xor_sync(0xffffffffu, wmx, o));
+  if (lane == 0) {
+    F[F_RED] = wmx;
+    F[F_RED + 1] = s_last;
+  }
+}
+
 __global__ void __launch_bounds__(kThreads, 1) ssd_kernel(const SsdParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ uint32_t tmem_slot;
@@ -185,11 +250,12 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_kernel(const SsdParams p) {
   uint32_t flags = 0;
 
   // ---- per-CTA constants
+  float sc_n = 0.0f, sb_n = 0.0f;
   if (tid < kN) {
     const int si = (int)g * (kN / p.gs) + tid / p.gs;
-    const float sc = __ldg(p.C_scale + si), sb = __ldg(p.B_scale + si);
-    F[F_WN + tid] = sc * sb;
-    F[F_SB + tid] = sb;
+    sc_n = __ldg(p.C_scale + si);
+    sb_n = __ldg(p.B_scale + si);
+    F[F_SB + tid] = sb_n;
   }
   if (tid < kP) {
     float sx = p.se.s[0];
@@ -212,14 +278,17 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_kernel(const SsdParams p) {
     tc::mbar_init(&bars[2], 1);
   }
   __syncthreads();
-  const float wmax = block_max(tid < kN ? F[F_WN + tid] : 0.0f, F + F_RED, tid);
-  if (tid < kN) F[F_WN + tid] = wmax > 0.0f ? F[F_WN + tid] / wmax : 0.0f;
+  const float wmax = block_max(sc_n * sb_n, F + F_RED, tid);
+  if (tid < kN) {
+    // w'_n rounded to binary16 once; the state operand factor undoes the rounding
+    const __half wh = __float2half_rn(wmax > 0.0f ? sc_n * sb_n / wmax : 0.0f);
+    reinterpret_cast<__half*>(F + F_WH)[tid] = wh;
+    const float whf = __half2float(wh);
+    F[F_HF + tid] = whf > 0.0f ? sc_n / whf : 0.0f;
+  }
   const float A2 = __ldg(p.A + hd) * kLog2e;
   const float bias = p.dt_bias ? __ldg(p.dt_bias + hd) : 0.0f;
   const float Dh = p.D ? __ldg(p.D + hd) : 0.0f;
-  // per-thread constants of the rows it owns
-  const float hfac = F[F_SB + row] > 0.0f ? wmax / F[F_SB + row] : 0.0f;  // state -> MMA2 operand
-  const float sbr = F[F_SB + row];
 
   // ---- initial state: thread (row = n, quarter) holds p in [16 q4, 16 q4 + 16)
   float hs[16];
@@ -232,85 +301,45 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_kernel(const SsdParams p) {
     __syncthreads();
 #pragma unroll
     for (int j = 0; j < 16; ++j) hs[j] = p.h0 ? stage[(16 * q4 + j) * kN + row] : 0.0f;
-    __syncthreads();
   }
-  tc::fence_before();
-  __syncthreads();
-  tc::fence_after();
+  const float hfac = F[F_HF + row];  // state -> MMA2 operand
+  const float sbr = F[F_SB + row];
   const uint32_t tmem = tmem_slot;
   const uint32_t t_lane = (uint32_t)(32 * (warp & 3)) << 16;
   const uint32_t T_CB = 0, T_YD = 128, T_YO = 192, T_ACC = 256;
 
-  // raw rows of tile 0, and its dt (warp 0: 4 steps per lane)
+  // ---- tile 0: raw rows, per-step factors, state maximum
   fetch_tile(p, smem, bb, hd, g, 0, (int)min((int64_t)kQ, L), tid);
   float dtv[4] = {0.0f, 0.0f, 0.0f, 0.0f};
   if (warp == 0) {
 #pragma unroll
     for (int i = 0; i < 4; ++i)
       if (4 * lane + i < L) dtv[i] = h2f(p.dt[(bb * L + 4 * lane + i) * H + hd]);
+    tile_factors(F, 0, (int)min((int64_t)kQ, L), dtv, bias, p.softplus, A2, wmax, lane);
   }
+  auto state_max = [&]() {
+    float hm = 0.0f;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) hm = fmaxf(hm, fabsf(hs[j] * hfac));
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) hm = fmaxf(hm, __shfl_xor_sync(0xffffffffu, hm, o));
+    if (lane == 0) F[F_RED + 2 + warp] = hm;
+  };
+  state_max();
+  tc::cp_async_wait_all();
+  tc::fence_before();
+  __syncthreads();
+  tc::fence_after();
 
   uint32_t phase = 0;
-  for (int64_t t0 = 0; t0 < L; t0 += kQ, phase ^= 1u) {
+  int fb = 0;  // buffer of this tile's per-step factors
+  for (int64_t t0 = 0; t0 < L; t0 += kQ, phase ^= 1u, fb ^= 1) {
     const int ql = (int)min((int64_t)kQ, L - t0);
-    tc::cp_async_wait_all();
-
-    // ---- warp 0: delta, S = cumsum(delta A) (log2 units), w_s, exp(S_t)
-    if (warp == 0) {
-      float dl[4], sc[4];
-      float run = 0.0f;
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int t = 4 * lane + i;
-        float d = 0.0f;
-        if (t < ql) {
-          const float v = dtv[i] + bias;
-          d = p.softplus ? softplus_f(v) : v;
-        }
-        dl[i] = d;
-        run += d * A2;
-        sc[i] = run;
-      }
-      float ex = run;  // inclusive scan of the lane totals
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const float n = __shfl_up_sync(0xffffffffu, ex, o);
-        if (lane >= o) ex += n;
-      }
-      const float off = ex - run;
-      const float s_last = __shfl_sync(0xffffffffu, ex, 31);
-      float wmx = 0.0f;
-      // S at the end of this lane's 32-step column block (lane 8 b + 7 holds it)
-      const float s_blk = __shfl_sync(0xffffffffu, sc[3] + off, lane | 7);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int t = 4 * lane + i;
-        const float s2 = sc[i] + off;
-        const float w = ex2_sfu(s_last - s2) * dl[i];
-        F[F_S2 + t] = s2;
-        F[F_DW + t] = dl[i];
-        F[F_WX + t] = w;
-        F[F_ES + t] = ex2_sfu(s2);
-        F[F_CW + t] = ex2_sfu(s_blk - s2) * dl[i] * wmax;
-        wmx = fmaxf(wmx, w);
-      }
-#pragma unroll
-      for (int o = 16; o >= 1; o >>= 1) wmx = fmaxf(wmx, __shfl_xor_sync(0xffffffffu, wmx, o));
-      if (lane == 0) {
-        F[F_RED] = wmx;
-        F[F_RED + 1] = s_last;
-      }
-    }
-    // every warp: max |state operand| partial
-    {
-      float hm = 0.0f;
-#pragma unroll
-      for (int j = 0; j < 16; ++j) hm = fmaxf(hm, fabsf(hs[j] * hfac));
-#pragma unroll
-      for (int o = 16; o >= 1; o >>= 1) hm = fmaxf(hm, __shfl_xor_sync(0xffffffffu, hm, o));
-      if (lane == 0) F[F_RED + 2 + warp] = hm;
-    }
-    __syncthreads();  // (A): raw tile landed for everyone, S and maxima published
+    const float* S2 = F + F_S2 + fb * kQ;
+    const float* DW = F + F_DW + fb * kQ;
+    const float* WX = F + F_WX + fb * kQ;
+    const float* ES = F + F_ES + fb * kQ;
+    const float* CW = F + F_CW + fb * kQ;
     const float s_last = F[F_RED + 1];
     const int ex = norm_exp(F[F_RED] * p.x_bound);  // x_bound >= max |x_exact|
     const float xsc = pow2i(-ex);
@@ -319,8 +348,8 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_kernel(const SsdParams p) {
     for (int w = 0; w < kThreads / 32; ++w) hmax_all = fmaxf(hmax_all, F[F_RED + 2 + w]);
     const int eh = norm_exp(hmax_all);
 
-    // ---- stage C (codes * w'_n) and B (codes): thread -> (row, 32 states);
-    // the states are warp-uniform so the w'_n reads are broadcasts
+    // ---- stage C' = fl16(codes * w'_n) and B (codes): thread -> (row, 32
+    // states); the states are warp-uniform so the w' reads are broadcasts
     {
       const int r = 32 * (warp >> 2) + lane, part = warp & 3;
       const bool ok = r < ql;
@@ -342,13 +371,15 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_kernel(const SsdParams p) {
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {  // 8 states per 16-byte core-matrix row
           const int n0 = 32 * part + 16 * i + 8 * hh;
+          const uint4 wq = *reinterpret_cast<const uint4*>(F + F_WH + n0 / 2);
+          const uint32_t wv[4] = {wq.x, wq.y, wq.z, wq.w};
           uint32_t oc[4], ob[4];
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
             const uint32_t wc = cw[2 * hh + k / 2], wb = bw[2 * hh + k / 2];
             const int b0i = 2 * (k & 1);
-            const float c0 = s8_to_f32(wc, b0i), c1 = s8_to_f32(wc, b0i + 1);
-            oc[k] = pack_h2(c0 * F[F_WN + n0 + 2 * k], c1 * F[F_WN + n0 + 2 * k + 1]);
+            oc[k] = h2_bits(__hmul2(s8x2_to_h2(wc, b0i, b0i + 1),
+                                    *reinterpret_cast<const __half2*>(&wv[k])));
             ob[k] = h2_bits(s8x2_to_h2(wb, b0i, b0i + 1));
           }
           *reinterpret_cast<uint4*>(smem + OFF_C + tc::kmaj_off(r, n0, kN)) =
@@ -365,7 +396,7 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_kernel(const SsdParams p) {
       const uint4 xq = ok ? *reinterpret_cast<const uint4*>(smem + OFF_RX + s * kP +
                                                             16 * (part ^ (s & 3)))
                           : make_uint4(0, 0, 0, 0);
-      const float ws = F[F_WX + s] * xsc;
+      const float ws = WX[s] * xsc;
 #pragma unroll
       for (int grp = 0; grp < 2; ++grp) {  // 8 p per group
         const uint32_t w0 = grp ? xq.z : xq.x, w1 = grp ? xq.w : xq.y;
@@ -399,18 +430,16 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_kernel(const SsdParams p) {
         *reinterpret_cast<uint4*>(smem + OFF_XL + off) = make_uint4(ol[0], ol[1], ol[2], ol[3]);
       }
     }
-    // ---- stage the state (hi / lo) for Y_off: h'' = h w_max / sB_n, normalised
+    // ---- stage the state for Y_off: h'' = h sC_n / w'_n, normalised, binary16
     {
       const float f = hfac * pow2i(-eh);
 #pragma unroll
       for (int grp = 0; grp < 2; ++grp) {
-        uint32_t oh[4], ol[4];
+        uint32_t oh[4];
 #pragma unroll
-        for (int k = 0; k < 4; ++k)
-          split_h2(hs[8 * grp + 2 * k] * f, hs[8 * grp + 2 * k + 1] * f, oh[k], ol[k]);
+        for (int k = 0; k < 4; ++k) oh[k] = pack_h2(hs[8 * grp + 2 * k] * f, hs[8 * grp + 2 * k + 1] * f);
         const uint32_t off = tc::mnmaj_off(16 * q4 + 8 * grp, row, kP);
         *reinterpret_cast<uint4*>(smem + OFF_HH + off) = make_uint4(oh[0], oh[1], oh[2], oh[3]);
-        *reinterpret_cast<uint4*>(smem + OFF_HL + off) = make_uint4(ol[0], ol[1], ol[2], ol[3]);
       }
     }
     tc::fence_async_smem();
@@ -418,7 +447,8 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_kernel(const SsdParams p) {
     __syncthreads();  // (B): operands staged, raw buffer consumed
 
     // ---- fetch the next tile while this one runs
-    if (t0 + kQ < L) {
+    const bool has_next = t0 + kQ < L;
+    if (has_next) {
       fetch_tile(p, smem, bb, hd, g, t0 + kQ, (int)min((int64_t)kQ, L - t0 - kQ), tid);
       if (warp == 0) {
 #pragma unroll
@@ -430,8 +460,7 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_kernel(const SsdParams p) {
     }
 
     // ---- MMA0: CB = C' B^T  (M = t, N = s, K = n); then, independent of
-    // M, MMA2 (Y_off, hi + lo) and MMA3 (state, hi + lo) run while the CUDA
-    // cores form M
+    // M, MMA2 (Y_off) and MMA3 (state, hi + lo) run while the CUDA cores form M
     if (tid == 0) {
       tc::fence_after();
       const uint32_t id = tc::idesc_f16(kQ, kQ, false, false);
@@ -446,10 +475,6 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_kernel(const SsdParams p) {
       for (int k0 = 0; k0 < kN; k0 += 16)
         tc::mma_f16(tmem + T_YO, tc::kmaj_desc(s_base + OFF_C, k0, kN),
                     tc::mnmaj_desc(s_base + OFF_HH, k0, kP), id_y, k0 > 0);
-#pragma unroll
-      for (int k0 = 0; k0 < kN; k0 += 16)
-        tc::mma_f16(tmem + T_YO, tc::kmaj_desc(s_base + OFF_C, k0, kN),
-                    tc::mnmaj_desc(s_base + OFF_HL, k0, kP), id_y, 1u);
 #pragma unroll
       for (int k0 = 0; k0 < kQ; k0 += 16)
         tc::mma_f16(tmem + T_ACC, tc::mnmaj_desc(s_base + OFF_B, k0, kN),
@@ -472,29 +497,37 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_kernel(const SsdParams p) {
     // Column block q4 against row block (warp & 3), both warp-uniform: above
     // the diagonal M is zero; strictly below it exp(S_t - S_s) =
     // exp(S_t - S_p) exp(S_p - S_s) with p the block's last step, both
-    // factors <= 1 (no overflow, underflow only of negligible terms); on the
-    // diagonal block each element takes its own exponential.
+    // factors <= 1 (no overflow, underflow only of negligible terms), and the
+    // row factor is applied with the normalisation; on the diagonal block
+    // each element takes its own exponential.
     float mv[32];
+    float rt = 1.0f;  // row factor still to apply to mv
     {
       const int t = row, s0 = 32 * q4, rb = warp & 3;
       float rmax = 0.0f;
       if (q4 <= rb) {
         float v[32];
         tc::tmem_ld32(tmem + t_lane + T_CB + s0, v);
-        const float st = F[F_S2 + t];
+        const float st = S2[t];
         if (q4 < rb) {
-          const float rt = ex2_sfu(st - F[F_S2 + s0 + 31]);
+          rt = ex2_sfu(st - S2[s0 + 31]);
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const float m = v[j] * (rt * F[F_CW + s0 + j]);
-            mv[j] = m;
-            rmax = fmaxf(rmax, fabsf(m));
+          for (int j4 = 0; j4 < 8; ++j4) {
+            const float4 c4 = *reinterpret_cast<const float4*>(CW + s0 + 4 * j4);
+            const float cw[4] = {c4.x, c4.y, c4.z, c4.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float m = v[4 * j4 + e] * cw[e];
+              mv[4 * j4 + e] = m;
+              rmax = fmaxf(rmax, fabsf(m));
+            }
           }
+          rmax *= rt;
         } else {
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
             const int s = s0 + j;
-            const float m = s <= t ? v[j] * ex2_sfu(st - F[F_S2 + s]) * F[F_DW + s] * wmax : 0.0f;
+            const float m = s <= t ? v[j] * ex2_sfu(st - S2[s]) * DW[s] * wmax : 0.0f;
             mv[j] = m;
             rmax = fmaxf(rmax, fabsf(m));
           }
@@ -511,7 +544,7 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_kernel(const SsdParams p) {
       const float rm = fmaxf(fmaxf(F[F_RM + t], F[F_RM + kQ + t]),
                              fmaxf(F[F_RM + 2 * kQ + t], F[F_RM + 3 * kQ + t]));
       const int et = norm_exp(rm);
-      const float sc = pow2i(-et);
+      const float sc = pow2i(-et) * rt;
       if (q4 == 0) F[F_RS + t] = pow2i(et);
 #pragma unroll
       for (int grp = 0; grp < 4; ++grp) {
@@ -543,14 +576,24 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_kernel(const SsdParams p) {
     }
     tc::fence_after();
 
-    // ---- y = Y_diag 2^e_t sx + exp(S_t) 2^e_h Y_off + D x  (thread: row t, 16 p)
+    // x scales of this thread's 16 columns
+    float sxv[16];
+#pragma unroll
+    for (int j4 = 0; j4 < 4; ++j4) {
+      const float4 v = *reinterpret_cast<const float4*>(F + F_SX + 16 * q4 + 4 * j4);
+      sxv[4 * j4] = v.x;
+      sxv[4 * j4 + 1] = v.y;
+      sxv[4 * j4 + 2] = v.z;
+      sxv[4 * j4 + 3] = v.w;
+    }
+    // ---- y = sx_p (Y_diag 2^e_t + D x_code) + exp(S_t) 2^e_h Y_off  (thread: row t, 16 p)
     {
       const int t = row;
       float yd[16], yo[16];
       tc::tmem_ld16(tmem + t_lane + T_YD + 16 * q4, yd);
       tc::tmem_ld16(tmem + t_lane + T_YO + 16 * q4, yo);
       if (t < ql) {
-        const float rs = F[F_RS + t], es = F[F_ES + t] * pow2i(eh);
+        const float rs = F[F_RS + t], es = ES[t] * pow2i(eh);
         const int64_t yo_off = ((bb * L + t0 + t) * H + hd) * kP + 16 * q4;
         // x of this row as exact binary16 values from the staged MMA operand
         uint32_t xw[8];
@@ -585,9 +628,7 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_kernel(const SsdParams p) {
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
             const int pj = j + e;
-            const float sx = F[F_SX + 16 * q4 + pj];
-            const float xv = (e ? xp.y : xp.x) * sx;
-            float yv = yd[pj] * rs * sx + es * yo[pj] + Dh * xv;
+            float yv = fmaf(sxv[pj], fmaf(Dh, e ? xp.y : xp.x, yd[pj] * rs), es * yo[pj]);
             if (p.z) yv *= silu_f(e ? zf.y : zf.x);
             r2[e] = yv;
           }
@@ -605,11 +646,21 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_kernel(const SsdParams p) {
       const float decay = ex2_sfu(s_last);
       const float f = sbr * pow2i(ex);
 #pragma unroll
-      for (int j = 0; j < 16; ++j) hs[j] = fmaf(decay, hs[j], f * F[F_SX + 16 * q4 + j] * acc[j]);
+      for (int j = 0; j < 16; ++j) hs[j] = fmaf(decay, hs[j], f * sxv[j] * acc[j]);
     }
+    // ---- next tile: per-step factors (warp 0, other buffer), state maximum,
+    // raw rows landed
+    if (has_next && warp == 0)
+      tile_factors(F, fb ^ 1, (int)min((int64_t)kQ, L - t0 - kQ), dtv, bias, p.softplus, A2,
+                   wmax, lane);
+    state_max();
+    tc::cp_async_wait_all();
     tc::fence_before();
     if (__syncthreads_or(abort_flag)) break;  // (E): tile done
+    tc::fence_after();
   }
+
+  tc::cp_async_wait_all();  // no copy may land after the CTA has exited (abort path)
 
   // ---- final state (P, N) through shared memory for coalesced stores
   if (p.h_final) {
