@@ -143,7 +143,7 @@ class ClockSampler:
 class Layer:
     """Inputs (resident in HBM), static calibration and outputs of one step."""
 
-    def __init__(self, dev, seed):
+    def __init__(self, dev, seed, fused=False):
         import torch
 
         from quantized_state_space_b200 import calibrate, synth
@@ -169,31 +169,38 @@ class Layer:
         self.y = torch.empty(self.x.shape, dtype=torch.float16, device=dev)
         self.hf = torch.empty((self.b, self.d, self.N), dtype=torch.float32, device=dev)
         self.units = self.b * self.L * self.d
-        self.launches_per_step = 4
+        # fused: the scan reads binary16 x and quantizes it itself (the result
+        # is byte-identical to quantizing x first); else x is quantized by
+        # its own launch and the scan reads the int8 codes
+        self.fused = fused
+        self.launches_per_step = 3 if fused else 4
 
     def quantize(self):
         from quantized_state_space_b200 import api
         b, L, d, G, N, gs = self.b, self.L, self.d, self.G, self.N, self.gs
-        api.quantize_groups(self.x, b, d, L, self.grp, self.k, scales=self.xs, out=self.xq)
+        if not self.fused:
+            api.quantize_groups(self.x, b, d, L, self.grp, self.k, scales=self.xs, out=self.xq)
         api.quantize_groups(self.B, b, G * N, L, self.smap, G * N // gs, scales=self.bs, out=self.Bq)
         api.quantize_groups(self.C, b, G * N, L, self.smap, G * N // gs, scales=self.cs, out=self.Cq)
 
     def scan(self):
         from quantized_state_space_b200 import api
-        api.selective_scan(self.xq, self.dt, self.A, self.Bq, self.Cq, self.bs, self.cs, self.gs,
-                           x_group=self.grp, x_scale=self.xs, D=self.D, z=self.z, y=self.y,
-                           h_final=self.hf)
+        api.selective_scan(self.x if self.fused else self.xq, self.dt, self.A, self.Bq, self.Cq,
+                           self.bs, self.cs, self.gs, x_group=self.grp, x_scale=self.xs, D=self.D,
+                           z=self.z, y=self.y, h_final=self.hf)
 
     def scan_bytes(self):
         """Algorithmic HBM bytes of one scan launch."""
         b, L, d, N, G = self.b, self.L, self.d, self.N, self.G
-        return (b * d * L * (1 + 2 + 2 + 2)          # x int8, dt, z, y f16
-                + 2 * b * G * N * L                  # B, C int8
+        xb = 2 if self.fused else 1                   # binary16 x or int8 codes
+        return (b * d * L * (xb + 2 + 2 + 2)          # x, dt, z, y f16
+                + 2 * b * G * N * L                   # B, C int8
                 + d * N * 4 + d * 4 + b * d * N * 4)  # A, D, h_final
 
     def step_bytes(self):
         b, L, d, N, G = self.b, self.L, self.d, self.N, self.G
-        return self.scan_bytes() + b * d * L * 3 + 2 * 3 * b * G * N * L
+        xq = 0 if self.fused else b * d * L * 3
+        return self.scan_bytes() + xq + 2 * 3 * b * G * N * L
 
 
 def cuda_events(torch):
@@ -282,7 +289,7 @@ def run_ours(args):
     if world > 1:
         dist.barrier()
     pk = peaks()
-    layer = Layer(dev, seed=rank_seed(rank))
+    layer = Layer(dev, seed=rank_seed(rank), fused=args.fused)
     stream = torch.cuda.current_stream()
 
     def step():
@@ -359,10 +366,14 @@ def run_ours(args):
             "e2e": {"value": round(e2e_value, 3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "steps": Ke},
             "gpu_launches": layer.launches_per_step * K,
+            "x_path": ("binary16 x quantized inside the scan (byte-identical to a separate "
+                       "quantize launch followed by the int8 scan)" if layer.fused else
+                       "x quantized by its own launch; the scan reads int8 codes"),
             "roofline": {"bound": "alu", "kernel": "m1_scan_kernel (selective scan)",
                          "achieved": round(achieved_upd, 2), "peak": round(peak_upd, 1),
                          "unit": "Gupdates/s", "frac": round(achieved_upd / peak_upd, 4),
-                         "traffic": measured_traffic("m1_scan_kernel"),
+                         "traffic": measured_traffic("m1_scan_kernel" if not layer.fused
+                                                     else "m1_scan_kernel_f16x"),
                          "peak_basis": "%d SMs x %d ex2/clk (SFU) x %.0f MHz; one exp per "
                                        "state update" % (SMS, MUFU_PER_CLK, mhz_max),
                          "hbm_achieved_gbs": round(scan_gbs, 1), "hbm_peak_gbs": pk["hbm_gbs"],
@@ -383,8 +394,12 @@ def run_ours(args):
             except Exception as e:  # report, keep the measured line
                 out["cpu_baseline"] = {"error": "%s: %s" % (type(e).__name__, e)}
         if world == 1 and not args.no_forms:
-            out["forms"] = run_forms(dev, pk, out["clocks"].get("sm_max_mhz") or pk["sm_max_mhz"],
-                                     only=args.forms.split(",") if args.forms else None)
+            only = args.forms.split(",") if args.forms else None
+            out["forms"] = {}
+            if not only or "m130m_other_x_path" in only:
+                out["forms"]["m130m_other_x_path"] = form_other_x_path(torch, layer)
+            out["forms"].update(run_forms(dev, pk, out["clocks"].get("sm_max_mhz") or
+                                          pk["sm_max_mhz"], only=only))
         print(json.dumps(out), flush=True)
 
 
@@ -429,6 +444,26 @@ def setup_decode(torch, dev, steps=None):
                          x_scale=xs_t, D=D, y=y)
 
     return dict(b=b, H=H, P=P, N=N, G=G, S=S, step=step)
+
+
+def form_other_x_path(torch, layer):
+    """The headline step with the other x path on the same inputs: binary16 x
+    encoded inside the scan vs x quantized by its own launch (byte-identical
+    results; the GPU parity tests check that)."""
+    layer.fused = not layer.fused
+    try:
+        def step():
+            layer.quantize()
+            layer.scan()
+        t = _timed(torch, step, 50)
+        t_scan = _timed(torch, layer.scan, 20)
+        return {"workload": "m130m step, " + ("binary16 x encoded inside the scan" if layer.fused
+                                               else "x quantized by its own launch"),
+                "value": round(layer.units / t / 1e9, 3), "unit": UNIT,
+                "ms_per_step": round(t * 1e3, 4), "scan_ms": round(t_scan * 1e3, 4),
+                "launches_per_step": layer.launches_per_step}
+    finally:
+        layer.fused = not layer.fused
 
 
 def form_decode(torch, dev, pk):
@@ -485,7 +520,11 @@ def setup_softedge(torch, dev):
         api.selective_scan(codes, dt, A, Bq, Cq, bs_t, cs_t, gs, se_scale=s, D=D, z=z, y=y,
                            h_final=hf)
 
-    return dict(b=b, L=L, d=d, N=N, enc=enc, quant_bc=quant_bc, scan=scan)
+    def scan_fused():  # binary16 x encoded inside the scan
+        api.selective_scan(x, dt, A, Bq, Cq, bs_t, cs_t, gs, se_scale=s, se_lo=lo, se_hi=hi, D=D,
+                           z=z, y=y, h_final=hf)
+
+    return dict(b=b, L=L, d=d, N=N, enc=enc, quant_bc=quant_bc, scan=scan, scan_fused=scan_fused)
 
 
 def form_softedge(torch, dev, pk, mhz):
@@ -496,7 +535,9 @@ def form_softedge(torch, dev, pk, mhz):
     t_enc = _timed(torch, enc, 5)
     t_bc = _timed(torch, quant_bc, 5)
     t_scan = _timed(torch, scan, 3)
+    t_fused = _timed(torch, c["scan_fused"], 3)
     t = t_enc + t_bc + t_scan
+    t_f = t_bc + t_fused
     n = b * L * d
     enc_bytes = n * 3
     upd = n * N
@@ -504,6 +545,11 @@ def form_softedge(torch, dev, pk, mhz):
     return {"workload": "softedge: b 16, L 8192, d 1536, N 16; encode + scan",
             "value": round(n / t / 1e9, 3), "unit": "Gtokens·ch/s",
             "ms_per_step": round(t * 1e3, 4),
+            "x_path": "encode launch, then the scan reads the codes",
+            "fused_path": {"x_path": "binary16 x soft-edge encoded inside the scan "
+                                     "(byte-identical result)",
+                           "value": round(n / t_f / 1e9, 3), "ms_per_step": round(t_f * 1e3, 4),
+                           "scan_ms": round(t_fused * 1e3, 4)},
             "encode": {"ms": round(t_enc * 1e3, 4), "bound": "hbm",
                        "achieved": round(enc_bytes / t_enc / 1e9, 1), "peak": pk["hbm_gbs"],
                        "unit": "GB/s", "frac": round(enc_bytes / t_enc / 1e9 / pk["hbm_gbs"], 4)},
@@ -641,13 +687,15 @@ def run_kernel(args):
     torch.cuda.set_device(dev)
     from quantized_state_space_b200 import api
     name = args.kernel
-    if name in ("scan", "quantize"):
-        lay = Layer(dev, 0)
+    if name in ("scan", "scan-int8", "quantize"):
+        lay = Layer(dev, 0, fused=name == "scan")
         lay.quantize()
-        fn = lay.scan if name == "scan" else (
+        fn = lay.scan if name != "quantize" else (
             lambda: api.quantize_groups(lay.x, lay.b, lay.d, lay.L, lay.grp, lay.k,
                                         scales=lay.xs, out=lay.xq))
-        label = "m130m " + ("selective scan" if name == "scan" else "x quantize (static scales)")
+        label = "m130m " + {"scan": "selective scan, binary16 x encoded in the scan",
+                            "scan-int8": "selective scan of int8 x codes",
+                            "quantize": "x quantize (static scales)"}[name]
     elif name == "ssd":
         c = setup_ssd(torch, dev)
         c["quant"]()
@@ -683,10 +731,13 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-forms", action="store_true")
-    ap.add_argument("--forms", default="", help="comma list of ssd27b,decode8b,softedge")
+    ap.add_argument("--forms", default="", help="comma list of m130m_other_x_path,ssd27b,decode8b,softedge")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--kernel", choices=["scan", "quantize", "ssd", "encode", "softedge-scan",
-                                         "decode"],
+    ap.add_argument("--fused", action="store_true",
+                    help="headline step with binary16 x encoded inside the scan (byte-identical "
+                         "result; default: x quantized by its own launch, the faster path here)")
+    ap.add_argument("--kernel", choices=["scan", "scan-int8", "quantize", "ssd", "encode",
+                                         "softedge-scan", "decode"],
                     help="profiling aid: run only this kernel on its workload")
     args = ap.parse_args()
     if args.kernel:

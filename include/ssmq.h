@@ -72,7 +72,12 @@ typedef enum {
 
 typedef enum { SSMQ_F32 = 0, SSMQ_F16 = 1 } ssmq_dtype;
 typedef enum { SSMQ_SCALE_STATIC = 0, SSMQ_SCALE_ABSMAX = 1 } ssmq_scale_mode;
-typedef enum { SSMQ_X_INT8_GROUP = 0, SSMQ_X_SOFTEDGE = 1 } ssmq_x_format;
+typedef enum {
+  SSMQ_X_INT8_GROUP = 0,   /* int8 codes, one fp32 scale per channel cluster */
+  SSMQ_X_SOFTEDGE = 1,     /* soft-edge uint8 codes (se_scale, se_log2_ratio) */
+  SSMQ_X_F16_GROUP = 2,    /* binary16 x quantized inside the kernel (Mamba-1 scan only) */
+  SSMQ_X_F16_SOFTEDGE = 3  /* binary16 x soft-edge encoded inside the kernel (Mamba-1 scan only) */
+} ssmq_x_format;
 
 /* ------------------------------------------------------------------------ */
 /* Symmetric int8 group quantizer                                           */
@@ -150,7 +155,20 @@ ssmq_status ssmq_softedge_decode(const uint8_t* codes, int64_t n, float scale,
  *
  * Layouts (b = batch, L = seqlen, d = dim, N = dstate, G = ngroups):
  *   x        (b, d, L)  int8 codes (x_format INT8_GROUP) or soft-edge uint8
- *                       codes (x_format SOFTEDGE: se_scale, se_log2_ratio)
+ *                       codes (x_format SOFTEDGE: se_scale, se_log2_ratio);
+ *                       or binary16 activations encoded on the fly ("encode
+ *                       then scan"):
+ *                       F16_GROUP: each element becomes the int8 code that
+ *                         ssmq_quantize_groups (SCALE_STATIC, group x_group[c],
+ *                         scale x_scale) gives it, and the recurrence reads
+ *                         code * scale;
+ *                       F16_SOFTEDGE: each element becomes the code that
+ *                         ssmq_softedge_encode(se_scale, se_lo, se_hi,
+ *                         se_log2_ratio) gives it, read back as the decoded value;
+ *                       either way y and h_final equal, byte for byte, the
+ *                       separate encode followed by INT8_GROUP / SOFTEDGE, and
+ *                       the status word gets the encoder's bits (NONFINITE,
+ *                       BAD_SCALE)
  *   x_group  int32[d]   cluster of each channel; x_scale fp32[n_x_groups]
  *   dt, z    (b, d, L)  binary16; z may be NULL (no gate)
  *   dt_bias  fp32[d] or NULL;  dt_softplus 0/1
@@ -189,6 +207,8 @@ typedef struct {
   uint16_t* y;
   float* h_final;
   uint32_t* status;
+  float se_lo, se_hi; /* soft-edge thresholds of x_format F16_SOFTEDGE (|v| < se_lo small,
+                         |v| > se_hi large); ignored otherwise */
 } ssmq_scan_args;
 
 ssmq_status ssmq_selective_scan_w8(const ssmq_scan_args* args, void* stream);

@@ -19,7 +19,7 @@ STATUS_NAMES = {0: "SSMQ_OK", 1: "SSMQ_ERR_INVALID_ARG", 2: "SSMQ_ERR_ALIGNMENT"
 DEV_NONFINITE, DEV_BAD_GROUP, DEV_BAD_SCALE, DEV_TIMEOUT = 1, 2, 4, 8
 F32, F16 = 0, 1
 SCALE_STATIC, SCALE_ABSMAX = 0, 1
-X_INT8_GROUP, X_SOFTEDGE = 0, 1
+X_INT8_GROUP, X_SOFTEDGE, X_F16_GROUP, X_F16_SOFTEDGE = 0, 1, 2, 3
 
 _i64, _i32, _vp, _f32 = C.c_int64, C.c_int32, C.c_void_p, C.c_float
 
@@ -37,7 +37,7 @@ class ScanArgs(C.Structure):
                 ("se_scale", _f32), ("se_log2_ratio", _i32), ("dt", _vp), ("dt_bias", _vp),
                 ("dt_softplus", _i32), ("A", _vp), ("D", _vp), ("z", _vp), ("B", _vp),
                 ("C", _vp), ("B_scale", _vp), ("C_scale", _vp), ("h0", _vp), ("y", _vp),
-                ("h_final", _vp), ("status", _vp)]
+                ("h_final", _vp), ("status", _vp), ("se_lo", _f32), ("se_hi", _f32)]
 
 
 class SSDArgs(C.Structure):

@@ -45,20 +45,30 @@ def softedge_decode(codes, scale, log2_ratio=2, *, out=None):
     return o
 
 
-def _x_fields(x, x_group, x_scale, se_scale, se_log2_ratio):
+def _x_fields(x, x_group, x_scale, se_scale, se_log2_ratio, se_lo=None, se_hi=None):
+    """x format from the tensor: uint8 soft-edge codes, int8 codes, or
+    binary16 activations encoded inside the kernel (soft-edge when thresholds
+    are given, else the static group quantizer)."""
     if x.dtype == torch.uint8:
         return dict(x_format=N.X_SOFTEDGE, x=x, se_scale=float(se_scale),
                     se_log2_ratio=se_log2_ratio, n_x_groups=0)
-    return dict(x_format=N.X_INT8_GROUP, x=x, x_group=x_group, x_scale=x_scale,
+    if x.dtype == torch.float16 and se_lo is not None:
+        return dict(x_format=N.X_F16_SOFTEDGE, x=x, se_scale=float(se_scale),
+                    se_log2_ratio=se_log2_ratio, n_x_groups=0, se_lo=float(se_lo),
+                    se_hi=float(se_hi))
+    fmt = N.X_F16_GROUP if x.dtype == torch.float16 else N.X_INT8_GROUP
+    return dict(x_format=fmt, x=x, x_group=x_group, x_scale=x_scale,
                 n_x_groups=int(x_scale.numel()), se_log2_ratio=se_log2_ratio)
 
 
 def selective_scan(x, dt, A, B, C, B_scale, C_scale, state_group_size, *, x_group=None,
-                   x_scale=None, se_scale=0.0, se_log2_ratio=2, D=None, z=None, dt_bias=None,
-                   dt_softplus=True, h0=None, y=None, h_final=None, return_state=True,
-                   status=None):
-    """Mamba-1 W8A8 selective scan.  x (b, d, L) int8 or soft-edge uint8;
-    dt, z (b, d, L) float16; B, C (b, G, N, L) int8.  Returns (y, h_final)."""
+                   x_scale=None, se_scale=0.0, se_log2_ratio=2, se_lo=None, se_hi=None, D=None,
+                   z=None, dt_bias=None, dt_softplus=True, h0=None, y=None, h_final=None,
+                   return_state=True, status=None):
+    """Mamba-1 W8A8 selective scan.  x (b, d, L) int8 codes, soft-edge uint8
+    codes, or float16 activations that the kernel encodes itself (with
+    x_group / x_scale, or with se_scale / se_lo / se_hi); dt, z (b, d, L)
+    float16; B, C (b, G, N, L) int8.  Returns (y, h_final)."""
     b, d, L = x.shape
     G, Nst = B.shape[1], B.shape[2]
     _dev_check(x, dt, A, B, C, B_scale, C_scale, x_group, x_scale, D, z, dt_bias, h0)
@@ -68,7 +78,8 @@ def selective_scan(x, dt, A, B, C, B_scale, C_scale, state_group_size, *, x_grou
         h_final = torch.empty((b, d, Nst), dtype=torch.float32, device=x.device)
     N.ssmq_selective_scan_w8(batch=b, seqlen=L, dim=d, dstate=Nst, ngroups=G,
                              state_group_size=state_group_size,
-                             **_x_fields(x, x_group, x_scale, se_scale, se_log2_ratio),
+                             **_x_fields(x, x_group, x_scale, se_scale, se_log2_ratio, se_lo,
+                                         se_hi),
                              dt=dt, dt_bias=dt_bias, dt_softplus=int(bool(dt_softplus)), A=A,
                              D=D, z=z, B=B, C=C, B_scale=B_scale, C_scale=C_scale, h0=h0, y=y,
                              h_final=h_final, status=status)

@@ -44,11 +44,14 @@ ssmq_status finish(cudaError_t e, const char* name) {
   } while (0)
 
 ssmq_status check_x(int32_t fmt, const void* x, const int32_t* x_group, const float* x_scale,
-                    int32_t n_x_groups, int32_t log2_ratio, const char* fn) {
-  REQUIRE(fmt == SSMQ_X_INT8_GROUP || fmt == SSMQ_X_SOFTEDGE, SSMQ_ERR_INVALID_ARG,
+                    int32_t n_x_groups, int32_t log2_ratio, const char* fn,
+                    bool allow_f16 = false) {
+  REQUIRE(fmt >= SSMQ_X_INT8_GROUP && fmt <= SSMQ_X_F16_SOFTEDGE, SSMQ_ERR_INVALID_ARG,
           "%s: x_format %d is not an ssmq_x_format", fn, fmt);
+  REQUIRE(allow_f16 || fmt == SSMQ_X_INT8_GROUP || fmt == SSMQ_X_SOFTEDGE, SSMQ_ERR_UNSUPPORTED,
+          "%s: binary16 x (x_format %d) is accepted by the Mamba-1 scan only", fn, fmt);
   REQUIRE(x != nullptr, SSMQ_ERR_INVALID_ARG, "%s: x is NULL", fn);
-  if (fmt == SSMQ_X_INT8_GROUP) {
+  if (fmt == SSMQ_X_INT8_GROUP || fmt == SSMQ_X_F16_GROUP) {
     REQUIRE(x_group && x_scale, SSMQ_ERR_INVALID_ARG, "%s: x_group / x_scale is NULL", fn);
     REQUIRE(n_x_groups >= 1, SSMQ_ERR_INVALID_ARG, "%s: n_x_groups must be >= 1", fn);
   } else {
@@ -148,8 +151,10 @@ ssmq_status ssmq_selective_scan_w8(const ssmq_scan_args* a, void* stream) {
     // an empty sequence reads no token tensor (they may be NULL); the final
     // state is then the initial state
     const ssmq_status xs = check_x(a->x_format, a->x, a->x_group, a->x_scale, a->n_x_groups,
-                                   a->se_log2_ratio, fn);
+                                   a->se_log2_ratio, fn, true);
     if (xs != SSMQ_OK) return xs;
+    REQUIRE(a->x_format != SSMQ_X_F16_SOFTEDGE || a->se_lo <= a->se_hi, SSMQ_ERR_INVALID_ARG,
+            "%s: se_lo must not exceed se_hi (as ssmq_softedge_encode)", fn);
     REQUIRE(a->dt && a->A && a->B && a->C && a->B_scale && a->C_scale && a->y,
             SSMQ_ERR_INVALID_ARG,
             "%s: a required tensor (dt, A, B, C, B_scale, C_scale, y) is NULL", fn);

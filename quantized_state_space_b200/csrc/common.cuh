@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "../../include/ssmq.h"
+
 namespace ssmq {
 
 constexpr float kLog2e = 1.4426950408889634f;
@@ -165,6 +167,44 @@ __device__ __forceinline__ float se_decode(uint32_t c, const SeSteps& st) {
   se_split(c, q, mode);
   // selects, not an indexed load: keeps the steps in registers
   return (float)q * (mode == 0 ? st.s[0] : (mode == 1 ? st.s[1] : st.s[2]));
+}
+
+// One element of the static quantizer; flags record device-side anomalies.
+// rs: reciprocal of s for the fast route, 0 to force the exact division.
+__device__ __forceinline__ int quant_elem(float v, float s, float rs, bool okg, uint32_t& flags) {
+  if (!okg) {
+    flags |= SSMQ_DEV_BAD_GROUP;
+    return 0;
+  }
+  if (!isfinite(v)) {
+    flags |= SSMQ_DEV_NONFINITE;
+    return 0;
+  }
+  if (!(s > 0.0f) || !isfinite(s)) {
+    if (s != 0.0f) flags |= SSMQ_DEV_BAD_SCALE;
+    return 0;
+  }
+  return rs != 0.0f ? quant_rne_fast(v, s, rs, 127) : quant_rne(v, s, 127);
+}
+
+// One soft-edge code (Quamba-SE write-up 2.1-2.2): mode by |v| against the
+// thresholds, payload by the quantizer at the mode's step and clamp.
+__device__ __forceinline__ uint32_t se_encode1(float v, float lo, float hi, const SeSteps& st,
+                                               uint32_t& flags) {
+  if (!isfinite(v)) {
+    flags |= SSMQ_DEV_NONFINITE;
+    return 0u;
+  }
+  const float a = fabsf(v);
+  const int mode = a < lo ? 1 : (a > hi ? 2 : 0);
+  const float step = mode == 0 ? st.s[0] : (mode == 1 ? st.s[1] : st.s[2]);
+  const int lim = mode == 0 ? 63 : 31;
+  const float rs = mode == 0 ? st.rs[0] : (mode == 1 ? st.rs[1] : st.rs[2]);
+  const int qv = (step > 0.0f && isfinite(step))
+                     ? (rs != 0.0f ? quant_rne_fast(v, step, rs, lim) : quant_rne(v, step, lim))
+                     : 0;
+  if (mode == 0) return (uint32_t)(qv & 0x7F);
+  return (mode == 1 ? 0x80u : 0xC0u) | (uint32_t)(qv & 0x3F);
 }
 
 __device__ __forceinline__ void flag_status(uint32_t* status, uint32_t bits) {

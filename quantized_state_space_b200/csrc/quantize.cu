@@ -77,24 +77,6 @@ inline Geo<uint32_t> make_geo(uint32_t mid, uint32_t inner) {
 }
 inline Geo<uint64_t> make_geo(uint64_t mid, uint64_t inner) { return Geo<uint64_t>{inner, mid}; }
 
-// One element of the static quantizer; flags record device-side anomalies.
-// rs: reciprocal of s for the fast route, 0 to force the exact division.
-__device__ __forceinline__ int quant_elem(float v, float s, float rs, bool okg, uint32_t& flags) {
-  if (!okg) {
-    flags |= SSMQ_DEV_BAD_GROUP;
-    return 0;
-  }
-  if (!isfinite(v)) {
-    flags |= SSMQ_DEV_NONFINITE;
-    return 0;
-  }
-  if (!(s > 0.0f) || !isfinite(s)) {
-    if (s != 0.0f) flags |= SSMQ_DEV_BAD_SCALE;
-    return 0;
-  }
-  return rs != 0.0f ? quant_rne_fast(v, s, rs, 127) : quant_rne(v, s, 127);
-}
-
 // Per-CTA table of (scale, reciprocal) for small group counts.
 constexpr int kMaxTab = 256;
 __device__ __forceinline__ void fill_tab(const float* scales, int32_t n_groups, float2* tab) {
@@ -374,24 +356,6 @@ cudaError_t quantize_p(const void* src, Idx n, Idx mid, Idx inner, const int32_t
 }
 
 // ---- soft-edge ---------------------------------------------------------------
-
-__device__ __forceinline__ uint32_t se_encode1(float v, float lo, float hi, const SeSteps& st,
-                                               uint32_t& flags) {
-  if (!isfinite(v)) {
-    flags |= SSMQ_DEV_NONFINITE;
-    return 0u;
-  }
-  const float a = fabsf(v);
-  const int mode = a < lo ? 1 : (a > hi ? 2 : 0);
-  const float step = mode == 0 ? st.s[0] : (mode == 1 ? st.s[1] : st.s[2]);
-  const int lim = mode == 0 ? 63 : 31;
-  const float rs = mode == 0 ? st.rs[0] : (mode == 1 ? st.rs[1] : st.rs[2]);
-  const int qv = (step > 0.0f && isfinite(step))
-                     ? (rs != 0.0f ? quant_rne_fast(v, step, rs, lim) : quant_rne(v, step, lim))
-                     : 0;
-  if (mode == 0) return (uint32_t)(qv & 0x7F);
-  return (mode == 1 ? 0x80u : 0xC0u) | (uint32_t)(qv & 0x3F);
-}
 
 // Branch-free fast route for 16 soft-edge codes (every st.rs[] usable):
 // the mode by two compares, then quant16_fast's rounding with the mode's

@@ -31,6 +31,8 @@
 // shared-memory buffers: chunk k (stores), k + 1 (staging) and k + 2, fetched
 // with cp.async one chunk ahead.  One block barrier per chunk.  The state
 // stays in registers; the final state is written once.
+#include <type_traits>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -50,6 +52,7 @@ struct M1Params {
   const float* x_scale;
   int n_x_groups;
   SeSteps se;
+  float se_lo, se_hi;  // soft-edge thresholds (binary16 x encoded in the kernel)
   const uint16_t* dt;
   const float* dt_bias;
   int softplus;
@@ -94,19 +97,20 @@ __device__ __forceinline__ float reduce_scatter(float (&p)[LPC], int j) {
   return p[0];
 }
 
-// Raw bytes of one chunk, as fetched from global memory.
-template <int kN, int kCH>
+// Raw bytes of one chunk, as fetched from global memory (x: 8-bit codes, or
+// binary16 activations that the kernel encodes itself).
+template <int kN, int kCH, typename XT>
 struct Raw {
-  uint8_t x[kCH][kT];
+  XT x[kCH][kT];
   uint16_t dt[kCH][kT];
   uint16_t z[kCH][kT];
   int8_t B[kN][kT];
   int8_t C[kN][kT];
 };
 
-template <int kN, int kCH>
+template <int kN, int kCH, typename XT>
 struct M1Smem {
-  Raw<kN, kCH> raw[kRawBufs];
+  Raw<kN, kCH, XT> raw[kRawBufs];
   __align__(16) float2 dd[kCH][kT + 2];   // (delta, delta x) of the chunk being scanned
   __align__(16) float bc[2][2][kT][kN];   // [buffer][B, C][t][n], dequantised
   __align__(16) float y[kCH][kSeg + 4];   // C . h of the current segment
@@ -138,21 +142,23 @@ __device__ __forceinline__ void lds_words(const void* p, uint32_t (&w)[(kBytes +
   }
 }
 
-template <int kN, int kCH>
-__device__ __forceinline__ void fetch_chunk(const M1Params& p, Raw<kN, kCH>& r, int64_t bb, int g,
-                                            int c0, int nc, int64_t t0, int tl, int tid, int NT) {
+template <int kN, int kCH, typename XT>
+__device__ __forceinline__ void fetch_chunk(const M1Params& p, Raw<kN, kCH, XT>& r, int64_t bb,
+                                            int g, int c0, int nc, int64_t t0, int tl, int tid,
+                                            int NT) {
   const int64_t d = p.d, L = p.L;
+  const XT* xs = static_cast<const XT*>(p.x);
   if (p.vec_ok) {
     // every row starts 16-byte aligned (L % 16 == 0) and tl % 16 == 0
     constexpr int XP = kT / 16, DP = kT / 8;  // 16-byte pieces per row
+    constexpr int XS = 16 / (int)sizeof(XT);   // x steps per piece
     for (int w = tid; w < kCH * DP; w += NT) {
       const int c = w / DP, q = w % DP;
       if (c >= nc || q * 8 >= tl) continue;
       const int64_t row = (bb * d + c0 + c) * L + t0;
       cp_async16(&r.dt[c][8 * q], p.dt + row + 8 * q);
       if (p.z) cp_async16(&r.z[c][8 * q], p.z + row + 8 * q);
-      if (q < XP && q * 16 < tl)
-        cp_async16(&r.x[c][16 * q], static_cast<const uint8_t*>(p.x) + row + 16 * q);
+      if (q < kT / XS && q * XS < tl) cp_async16(&r.x[c][XS * q], xs + row + XS * q);
     }
     for (int w = tid; w < 2 * kN * XP; w += NT) {
       const int which = w / (kN * XP), rem = w % (kN * XP);
@@ -167,7 +173,7 @@ __device__ __forceinline__ void fetch_chunk(const M1Params& p, Raw<kN, kCH>& r, 
       const int c = w / kT, t = w % kT;
       if (c >= nc || t >= tl) continue;
       const int64_t row = (bb * d + c0 + c) * L + t0 + t;
-      r.x[c][t] = static_cast<const uint8_t*>(p.x)[row];
+      r.x[c][t] = xs[row];
       r.dt[c][t] = p.dt[row];
       if (p.z) r.z[c][t] = p.z[row];
     }
@@ -184,13 +190,16 @@ __device__ __forceinline__ void fetch_chunk(const M1Params& p, Raw<kN, kCH>& r, 
 template <int kN, int kCH, int kSPL, int kXFmt>
 __global__ void __launch_bounds__(kCH*(kN / kSPL)) m1_scan_kernel(const M1Params p) {
   static_assert(kSPL == 2 || kSPL == 4, "2 or 4 states per thread");
+  constexpr bool kXF16 = kXFmt == SSMQ_X_F16_GROUP || kXFmt == SSMQ_X_F16_SOFTEDGE;
+  using XT = typename std::conditional<kXF16, uint16_t, uint8_t>::type;
+  using RawT = Raw<kN, kCH, XT>;
   constexpr int NP = kSPL / 2;      // fp32x2 pairs per thread
   constexpr int LPC = kN / kSPL;    // lanes per channel
   constexpr int NT = kCH * LPC;
   constexpr int SPS = kSeg / LPC;   // steps per lane per segment (stores, staging)
   static_assert(LPC >= 1 && LPC <= 16 && kSeg % LPC == 0, "lanes per channel");
   extern __shared__ __align__(16) uint8_t smem_bytes[];
-  M1Smem<kN, kCH>& S = *reinterpret_cast<M1Smem<kN, kCH>*>(smem_bytes);
+  M1Smem<kN, kCH, XT>& S = *reinterpret_cast<M1Smem<kN, kCH, XT>*>(smem_bytes);
 
   const int tid = threadIdx.x;
   const int64_t bb = blockIdx.y;
@@ -217,16 +226,21 @@ __global__ void __launch_bounds__(kCH*(kN / kSPL)) m1_scan_kernel(const M1Params
                                            __ldg(p.h0 + (bb * d + lch) * kN + n + 1))
                              : make_float2(0.0f, 0.0f);
   }
-  float xs = 1.0f, bias = 0.0f, Dc = 0.0f;
+  float xs = 1.0f, xrs = 0.0f, bias = 0.0f, Dc = 0.0f;
+  bool xok = true;  // x_group id valid
   if (lvalid) {
-    if (kXFmt == SSMQ_X_INT8_GROUP) {
+    if (kXFmt == SSMQ_X_INT8_GROUP || kXFmt == SSMQ_X_F16_GROUP) {
       const int xg = __ldg(p.x_group + lch);
       if ((unsigned)xg < (unsigned)p.n_x_groups) {
         xs = __ldg(p.x_scale + xg);
       } else {
         xs = 0.0f;
+        xok = false;
         if (lj == 0) flags |= SSMQ_DEV_BAD_GROUP;
       }
+      // reciprocal for the quantizer's fast route (0: exact division only)
+      const float r = __frcp_rn(xs);
+      xrs = usable_recip(xs, r) ? r : 0.0f;
     }
     bias = p.dt_bias ? __ldg(p.dt_bias + lch) : 0.0f;
     Dc = p.D ? __ldg(p.D + lch) : 0.0f;
@@ -236,29 +250,79 @@ __global__ void __launch_bounds__(kCH*(kN / kSPL)) m1_scan_kernel(const M1Params
     S.scale[which][n] = __ldg((which ? p.C_scale : p.B_scale) + g * spg + n / p.gs);
   }
 
-  auto x_value = [&](uint32_t word, int e) -> float {
-    if (kXFmt == SSMQ_X_INT8_GROUP) return s8_to_f32(word ^ 0x80808080u, e) * xs;
-    return se_decode((word >> (8 * e)) & 0xFFu, p.se);
+  // Value the recurrence reads for element e of the packed words w: a code
+  // times its scale or a decoded soft-edge code.  With binary16 x, staging
+  // has already replaced each element by its code (low byte of the slot).
+  auto x_value = [&](const uint32_t* w, int e) -> float {
+    if constexpr (kXFmt == SSMQ_X_INT8_GROUP) {
+      return s8_to_f32(w[e >> 2] ^ 0x80808080u, e & 3) * xs;
+    } else if constexpr (kXFmt == SSMQ_X_SOFTEDGE) {
+      return se_decode((w[e >> 2] >> (8 * (e & 3))) & 0xFFu, p.se);
+    } else if constexpr (kXFmt == SSMQ_X_F16_GROUP) {
+      return s8_to_f32(w[e >> 1] ^ 0x80808080u, 2 * (e & 1)) * xs;
+    } else {
+      return se_decode((w[e >> 1] >> (16 * (e & 1))) & 0xFFu, p.se);
+    }
+  };
+  // binary16 x: the code the quantizer / encoder kernels give element v, by
+  // the same reciprocal + magic-number route (exact division near a tie or
+  // for a non-finite v, with the same status bits)
+  const bool qfast = xok && xrs != 0.0f;
+  const bool sfast = p.se.rs[0] != 0.0f && p.se.rs[1] != 0.0f && p.se.rs[2] != 0.0f;
+  auto x_encode = [&](float v) -> uint32_t {
+    if constexpr (kXFmt == SSMQ_X_F16_GROUP) {
+      if (qfast) {
+        const float yc = fminf(fmaxf(v * xrs, -127.0f), 127.0f);
+        const float m = yc + 12582912.0f;
+        if (fabsf(yc - (m - 12582912.0f)) < 0.5f - 1.0f / 16384.0f && fabsf(v) <= 3.402823466e38f)
+          return __float_as_uint(m) & 0xFFu;
+      }
+      return (uint32_t)quant_elem(v, xs, xrs, xok, flags) & 0xFFu;
+    } else {
+      if (sfast) {
+        const float a = fabsf(v);
+        const bool sm = a < p.se_lo, lg = a > p.se_hi;
+        const float rs = sm ? p.se.rs[1] : (lg ? p.se.rs[2] : p.se.rs[0]);
+        const float lim = (sm || lg) ? 31.0f : 63.0f;
+        const float yc = fminf(fmaxf(v * rs, -lim), lim);
+        const float m = yc + 12582912.0f;
+        if (fabsf(yc - (m - 12582912.0f)) < 0.5f - 1.0f / 16384.0f && a <= 3.402823466e38f) {
+          const uint32_t b = __float_as_uint(m);
+          return sm ? ((b & 0x3Fu) | 0x80u) : (lg ? ((b | 0xC0u) & 0xFFu) : (b & 0x7Fu));
+        }
+      }
+      return se_encode1(v, p.se_lo, p.se_hi, p.se, flags);
+    }
   };
 
-  // (delta, delta x) of steps s kSeg + lj SPS .. + SPS of this lane's channel,
-  // chunk with tl valid steps, from raw bytes r
-  auto stage_dd = [&](const Raw<kN, kCH>& r, int s, int tl) {
+  constexpr int XB = SPS * (int)sizeof(XT);  // x bytes of a lane's run
+  auto stage_dd = [&](RawT& r, int s, int tl) {
     const int tb = s * kSeg + lj * SPS;
-    uint32_t xw[(SPS + 3) / 4], dw[(2 * SPS + 3) / 4];
-    lds_words<SPS>(&r.x[lc][tb], xw);
+    uint32_t xw[(XB + 3) / 4], dw[(2 * SPS + 3) / 4];
+    lds_words<XB>(&r.x[lc][tb], xw);
     lds_words<2 * SPS>(&r.dt[lc][tb], dw);
+    if constexpr (kXF16) {
+      // encode in place: each slot's low byte becomes the element's code
+      // (this lane reads the same slots again when it stores y)
+#pragma unroll
+      for (int i = 0; i < SPS; ++i) {
+        const uint32_t sh = 16 * (i & 1);
+        const uint32_t c = (lvalid && tb + i < tl) ? x_encode(h2f((uint16_t)(xw[i >> 1] >> sh))) : 0u;
+        xw[i >> 1] = (xw[i >> 1] & ~(0xFFFFu << sh)) | (c << sh);
+        r.x[lc][tb + i] = (uint16_t)c;
+      }
+    }
 #pragma unroll
     for (int i = 0; i < SPS; ++i) {
       const float dv = h2f((uint16_t)(dw[i >> 1] >> (16 * (i & 1)))) + bias;
       float delta = p.softplus ? softplus_f(dv) : dv;
       if (!lvalid || tb + i >= tl) delta = 0.0f;
-      S.dd[lc][tb + i] = make_float2(delta, delta * x_value(xw[i >> 2], i & 3));
+      S.dd[lc][tb + i] = make_float2(delta, delta * x_value(xw, i));
     }
   };
   // this thread's share of the dequantised B, C rows of segment s (8 steps of
   // one row per item)
-  auto stage_bc = [&](const Raw<kN, kCH>& r, int s, int buf, int tl) {
+  auto stage_bc = [&](const RawT& r, int s, int buf, int tl) {
     constexpr int H = kSeg / 8;  // items per row and segment
     for (int w = tid; w < 2 * kN * H; w += NT) {
       const int which = w / (kN * H), n = (w / H) % kN, tb = s * kSeg + 8 * (w % H);
@@ -275,16 +339,16 @@ __global__ void __launch_bounds__(kCH*(kN / kSPL)) m1_scan_kernel(const M1Params
   };
   // y = (C.h + D x) silu(z) of steps s kSeg + lj SPS .. + SPS of this lane's
   // channel, chunk starting at t0 with tl valid steps
-  auto store_seg = [&](const Raw<kN, kCH>& r, int s, int64_t t0, int tl) {
+  auto store_seg = [&](const RawT& r, int s, int64_t t0, int tl) {
     const int tb = s * kSeg + lj * SPS;
     if (!lvalid || tb >= tl) return;
-    uint32_t xw[(SPS + 3) / 4], zw[(2 * SPS + 3) / 4];
-    lds_words<SPS>(&r.x[lc][tb], xw);
+    uint32_t xw[(XB + 3) / 4], zw[(2 * SPS + 3) / 4];
+    lds_words<XB>(&r.x[lc][tb], xw);
     if (p.z) lds_words<2 * SPS>(&r.z[lc][tb], zw);
     float yv[SPS];
 #pragma unroll
     for (int i = 0; i < SPS; ++i) {
-      float v = fmaf(Dc, x_value(xw[i >> 2], i & 3), S.y[lc][lj * SPS + i]);
+      float v = fmaf(Dc, x_value(xw, i), S.y[lc][lj * SPS + i]);
       if (p.z) v *= silu_f(h2f((uint16_t)(zw[i >> 1] >> (16 * (i & 1)))));
       yv[i] = v;
     }
@@ -315,11 +379,11 @@ __global__ void __launch_bounds__(kCH*(kN / kSPL)) m1_scan_kernel(const M1Params
   auto chunk_len = [&](int k) { return (int)min((int64_t)kT, L - (int64_t)k * kT); };
 
   // prologue: raw bytes of chunks 0 and 1, chunk 0 staged
-  fetch_chunk<kN, kCH>(p, S.raw[0], bb, g, c0, nc, 0, chunk_len(0), tid, NT);
+  fetch_chunk<kN, kCH, XT>(p, S.raw[0], bb, g, c0, nc, 0, chunk_len(0), tid, NT);
   cp_async_commit();
   cp_async_wait_all();
   __syncthreads();
-  if (nchunks > 1) fetch_chunk<kN, kCH>(p, S.raw[1], bb, g, c0, nc, kT, chunk_len(1), tid, NT);
+  if (nchunks > 1) fetch_chunk<kN, kCH, XT>(p, S.raw[1], bb, g, c0, nc, kT, chunk_len(1), tid, NT);
   cp_async_commit();
 #pragma unroll
   for (int s = 0; s < kSegs; ++s) {
@@ -332,8 +396,8 @@ __global__ void __launch_bounds__(kCH*(kN / kSPL)) m1_scan_kernel(const M1Params
     const int tl = chunk_len(k);
     const bool has_next = k + 1 < nchunks;
     const int tl_next = has_next ? chunk_len(k + 1) : 0;
-    const Raw<kN, kCH>& rcur = S.raw[k % kRawBufs];
-    const Raw<kN, kCH>& rnext = S.raw[(k + 1) % kRawBufs];
+    const RawT& rcur = S.raw[k % kRawBufs];
+    RawT& rnext = S.raw[(k + 1) % kRawBufs];
     const float(*sB)[kN] = S.bc[k & 1][0];
     const float(*sC)[kN] = S.bc[k & 1][1];
     // chunk k staged and raw bytes of chunk k + 1 landed (every thread's
@@ -342,7 +406,7 @@ __global__ void __launch_bounds__(kCH*(kN / kSPL)) m1_scan_kernel(const M1Params
     cp_async_wait_all();
     __syncthreads();
     if (k + 2 < nchunks)
-      fetch_chunk<kN, kCH>(p, S.raw[(k + 2) % kRawBufs], bb, g, c0, nc, t0 + 2 * kT,
+      fetch_chunk<kN, kCH, XT>(p, S.raw[(k + 2) % kRawBufs], bb, g, c0, nc, t0 + 2 * kT,
                            chunk_len(k + 2), tid, NT);
     cp_async_commit();
 
@@ -407,9 +471,12 @@ cudaError_t launch_m1(const M1Params& prm, int xfmt, int64_t batch, cudaStream_t
   p.n_ctile = (dg + kCH - 1) / kCH;
   const dim3 grid((unsigned)(p.n_ctile * p.G), (unsigned)batch);
   const dim3 block(kCH * (kN / kSPL));
-  const size_t smem = sizeof(M1Smem<kN, kCH>);
-  auto kern = xfmt == SSMQ_X_SOFTEDGE ? m1_scan_kernel<kN, kCH, kSPL, SSMQ_X_SOFTEDGE>
-                                      : m1_scan_kernel<kN, kCH, kSPL, SSMQ_X_INT8_GROUP>;
+  const bool f16 = xfmt == SSMQ_X_F16_GROUP || xfmt == SSMQ_X_F16_SOFTEDGE;
+  const size_t smem = f16 ? sizeof(M1Smem<kN, kCH, uint16_t>) : sizeof(M1Smem<kN, kCH, uint8_t>);
+  auto kern = xfmt == SSMQ_X_SOFTEDGE       ? m1_scan_kernel<kN, kCH, kSPL, SSMQ_X_SOFTEDGE>
+              : xfmt == SSMQ_X_F16_GROUP    ? m1_scan_kernel<kN, kCH, kSPL, SSMQ_X_F16_GROUP>
+              : xfmt == SSMQ_X_F16_SOFTEDGE ? m1_scan_kernel<kN, kCH, kSPL, SSMQ_X_F16_SOFTEDGE>
+                                            : m1_scan_kernel<kN, kCH, kSPL, SSMQ_X_INT8_GROUP>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   kern<<<grid, block, smem, st>>>(p);
@@ -431,6 +498,8 @@ cudaError_t launch_selective_scan(const ssmq_scan_args& a, cudaStream_t st) {
   p.x_scale = a.x_scale;
   p.n_x_groups = a.n_x_groups;
   p.se = se_steps(a.se_scale, a.se_log2_ratio);
+  p.se_lo = a.se_lo;
+  p.se_hi = a.se_hi;
   p.dt = a.dt;
   p.dt_bias = a.dt_bias;
   p.softplus = a.dt_softplus;

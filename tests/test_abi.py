@@ -113,6 +113,14 @@ def test_scan_validation(L):
     assert S(dt=None) == N.ERR_INVALID_ARG
     assert S(y=FAKE + 4) == N.ERR_ALIGNMENT
     assert S(x_format=N.X_SOFTEDGE, x_group=None, x_scale=None, se_log2_ratio=12) == N.ERR_INVALID_ARG
+    # binary16 x encoded in the kernel: group form needs the cluster map, the
+    # soft-edge form ordered thresholds (as ssmq_softedge_encode)
+    assert S(x_format=N.X_F16_GROUP, x_group=None) == N.ERR_INVALID_ARG
+    assert S(x_format=N.X_F16_SOFTEDGE, x_group=None, x_scale=None, se_lo=2.0,
+             se_hi=1.0) == N.ERR_INVALID_ARG
+    assert S(x_format=N.X_F16_SOFTEDGE, x_group=None, x_scale=None, se_lo=float("nan"),
+             se_hi=1.0) == N.ERR_INVALID_ARG
+    assert S(x_format=4) == N.ERR_INVALID_ARG
     assert S(batch=0) == N.OK
     assert L.ssmq_selective_scan_w8(None, None) == N.ERR_INVALID_ARG
 
@@ -132,6 +140,7 @@ def test_ssd_validation(L):
     assert S(chunk=100) == N.ERR_UNSUPPORTED
     assert S(ngroups=3) == N.ERR_INVALID_ARG
     assert S(x=None) == N.ERR_INVALID_ARG
+    assert S(x_format=N.X_F16_GROUP) == N.ERR_UNSUPPORTED  # Mamba-1 scan only
     need = L.ssmq_ssd_workspace_size(C.byref(_ssd_args()))
     if need:
         assert S(ws=None, nb=0) == N.ERR_INVALID_ARG
@@ -153,6 +162,7 @@ def test_decode_validation(L):
     assert S(ngroups=3) == N.ERR_INVALID_ARG
     assert S(state=None) == N.ERR_INVALID_ARG
     assert S(state=FAKE + 4) == N.ERR_ALIGNMENT
+    assert S(x_format=N.X_F16_SOFTEDGE) == N.ERR_UNSUPPORTED  # Mamba-1 scan only
     assert S(batch=0) == N.OK
 
 

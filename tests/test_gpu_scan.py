@@ -214,3 +214,75 @@ def test_m130m_workload_end_to_end(orc):
 
 def test_softedge_workload_end_to_end(orc):
     _m1_end_to_end(orc, "softedge", n_units=64)
+
+
+# ---- encode then scan: binary16 x encoded inside the scan (SURVEY-next
+# producer-side fusion; Quamba-SE write-up 4.1: the range check inside
+# quantisation).  The fused call must equal the separate encoder followed by
+# the code-reading scan, byte for byte, status word included.
+
+FUSED_CASES = [
+    # (b, L, d, N, G, gs, gate, h0, fmt)
+    (2, 200, 40, 16, 1, 4, True, False, "group"),     # ragged L (no 16-byte rows), partial tile
+    (2, 256, 64, 16, 2, 4, True, True, "group"),
+    (2, 96, 64, 4, 1, 2, False, True, "group"),
+    (1, 64, 16, 64, 1, 16, True, False, "group"),
+    (2, 160, 48, 16, 1, 4, True, True, "softedge"),
+    (1, 70, 32, 8, 1, 4, False, False, "softedge"),
+]
+
+
+def _f16_activations(rng, shape, outliers=True):
+    x = rng.standard_normal(shape).astype(np.float32)
+    if outliers:
+        idx = rng.choice(x.size, size=max(1, x.size // 2000), replace=False)
+        x.reshape(-1)[idx] *= rng.uniform(20, 200, size=idx.size)
+    return x.astype(np.float16)
+
+
+@pytest.mark.parametrize("ci", range(len(FUSED_CASES)))
+def test_fused_encode_scan_bit_exact(ci):
+    b, L, d, N_, G, gs, gate, h0, fmt = FUSED_CASES[ci]
+    p = m1_problem(700 + ci, b, L, d, N_, G=G, gs=gs, gate=gate, h0=h0)
+    rng = np.random.default_rng(750 + ci)
+    xf = _f16_activations(rng, (b, d, L))
+    xf.reshape(-1)[rng.choice(xf.size, size=3, replace=False)] = [np.inf, -np.inf, np.nan]
+    xt = T(xf)
+    common = dict(D=T(p["D"]), z=T(p["z"]), h0=T(p.get("h0")))
+    args = (T(p["dt"]), T(p["A"]), T(p["B"]), T(p["C"]), T(p["B_scale"]), T(p["C_scale"]), gs)
+    s_sep, s_fused = status_word(), status_word()
+    if fmt == "group":
+        grp = T(p["x_group"])
+        xs = T(p["x_scale"])
+        codes, _ = api.quantize_groups(xt, b, d, L, grp, int(xs.numel()), scales=xs, status=s_sep)
+        y1, h1 = api.selective_scan(codes, *args, x_group=grp, x_scale=xs, status=s_sep, **common)
+        y2, h2 = api.selective_scan(xt, *args, x_group=grp, x_scale=xs, status=s_fused, **common)
+    else:
+        finite = np.abs(xf[np.isfinite(xf)].astype(np.float64))
+        lo, hi = float(np.percentile(finite, 5)), float(np.percentile(finite, 99.9))
+        s = float(np.float32(hi / 63))
+        codes = api.softedge_encode(xt, s, lo, hi, 2, status=s_sep)
+        y1, h1 = api.selective_scan(codes, *args, se_scale=s, status=s_sep, **common)
+        y2, h2 = api.selective_scan(xt, *args, se_scale=s, se_lo=lo, se_hi=hi, status=s_fused,
+                                    **common)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(H(y2).view(np.uint16), H(y1).view(np.uint16))
+    np.testing.assert_array_equal(H(h2).view(np.uint32), H(h1).view(np.uint32))
+    assert int(H(s_fused)[0]) == int(H(s_sep)[0]) and int(H(s_fused)[0]) & 1  # NONFINITE seen
+
+
+def test_fused_encode_scan_vs_oracle(orc):
+    """The fused path against the oracle's quantizer followed by its scan."""
+    b, L, d, N_, gs = 2, 300, 48, 16, 4
+    p = m1_problem(790, b, L, d, N_, gs=gs, gate=True, h0=True, bias=True)
+    rng = np.random.default_rng(791)
+    xf = _f16_activations(rng, (b, d, L))
+    y, hf = api.selective_scan(T(xf), T(p["dt"]), T(p["A"]), T(p["B"]), T(p["C"]),
+                               T(p["B_scale"]), T(p["C_scale"]), gs, x_group=T(p["x_group"]),
+                               x_scale=T(p["x_scale"]), D=T(p["D"]), z=T(p["z"]),
+                               dt_bias=T(p["dt_bias"]), h0=T(p["h0"]))
+    k = int(p["x_scale"].size)
+    q, _, _ = orc.quantize_groups(xf, b, d, L, p["x_group"], k, orc.SCALE_STATIC, p["x_scale"])
+    po = dict(p, x=q.reshape(b, d, L))
+    yo, ho = oracle_scan(orc, po)
+    assert_scan_close(H(y).astype(np.float64), yo.reshape(y.shape), H(hf), ho.reshape(hf.shape))
