@@ -398,6 +398,8 @@ def run_ours(args):
             out["forms"] = {}
             if not only or "m130m_other_x_path" in only:
                 out["forms"]["m130m_other_x_path"] = form_other_x_path(torch, layer)
+            if not only or "m130m_int8_y" in only:
+                out["forms"]["m130m_int8_y"] = form_int8_y(torch, layer)
             out["forms"].update(run_forms(dev, pk, out["clocks"].get("sm_max_mhz") or
                                           pk["sm_max_mhz"], only=only))
         print(json.dumps(out), flush=True)
@@ -464,6 +466,42 @@ def form_other_x_path(torch, layer):
                 "launches_per_step": layer.launches_per_step}
     finally:
         layer.fused = not layer.fused
+
+
+def form_int8_y(torch, layer):
+    """The headline step with the persistent-INT8 epilogue: the scan writes int8
+    y (static per-cluster output scales calibrated on this layer's binary16 y)
+    instead of binary16 y; beside it the binary16 step followed by a separate
+    quantize of y, which produces the same bytes."""
+    from quantized_state_space_b200 import api, calibrate
+    b, d, L, k = layer.b, layer.d, layer.L, layer.k
+    layer.quantize()
+    layer.scan()
+    torch.cuda.synchronize()
+    ygrp, ysc = calibrate.m1_x_clusters(layer.y.cpu().numpy(), k)
+    yg = torch.from_numpy(ygrp).to(layer.y.device)
+    ys = torch.from_numpy(ysc).to(layer.y.device)
+    yq = torch.empty(layer.y.shape, dtype=torch.int8, device=layer.y.device)
+
+    def step_q():
+        layer.quantize()
+        api.selective_scan(layer.x if layer.fused else layer.xq, layer.dt, layer.A, layer.Bq,
+                           layer.Cq, layer.bs, layer.cs, layer.gs, x_group=layer.grp,
+                           x_scale=layer.xs, D=layer.D, z=layer.z, h_final=layer.hf, y_group=yg,
+                           y_scale=ys, y_q=yq, want_y=False)
+
+    def step_sep():
+        layer.quantize()
+        layer.scan()
+        api.quantize_groups(layer.y, b, d, L, yg, k, scales=ys, out=yq)
+
+    t_q = _timed(torch, step_q, 50)
+    t_s = _timed(torch, step_sep, 50)
+    return {"workload": "m130m step with int8 y (persistent-INT8 epilogue, no binary16 y)",
+            "value": round(layer.units / t_q / 1e9, 3), "unit": UNIT,
+            "ms_per_step": round(t_q * 1e3, 4),
+            "separate_quantize_of_y": {"value": round(layer.units / t_s / 1e9, 3),
+                                       "ms_per_step": round(t_s * 1e3, 4)}}
 
 
 def form_decode(torch, dev, pk):
@@ -731,7 +769,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-forms", action="store_true")
-    ap.add_argument("--forms", default="", help="comma list of m130m_other_x_path,ssd27b,decode8b,softedge")
+    ap.add_argument("--forms", default="", help="comma list of m130m_other_x_path,m130m_int8_y,ssd27b,decode8b,softedge")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--fused", action="store_true",
                     help="headline step with binary16 x encoded inside the scan (byte-identical "

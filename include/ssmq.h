@@ -177,11 +177,16 @@ ssmq_status ssmq_softedge_decode(const uint8_t* codes, int64_t n, float scale,
  *   B_scale, C_scale fp32[G * N / state_group_size]: state n of group g uses
  *            index g * (N / state_group_size) + n / state_group_size
  *   h0       fp32 (b, d, N) or NULL (zero initial state)
- *   y        (b, d, L) binary16 output
+ *   y        (b, d, L) binary16 output, or NULL when y_q is given
  *   h_final  fp32 (b, d, N) output or NULL
+ *   y_q      (b, d, L) int8 output or NULL: the persistent-INT8 epilogue
+ *            (SSDi8 abstract: an INT8 path through the block).  Each y is
+ *            rounded to binary16 and quantized with its channel's static
+ *            scale, y_group int32[d] -> y_scale fp32[n_y_groups]: the bytes
+ *            equal ssmq_quantize_groups (SCALE_STATIC) of the binary16 y.
  * Supported: N in {4, 8, 16, 32, 64}; d % G == 0; any L >= 0.
- * status: device word or NULL (SSMQ_DEV_BAD_GROUP for x_group ids out of
- * range, which then read scale 0).
+ * status: device word or NULL (SSMQ_DEV_BAD_GROUP for x_group / y_group ids
+ * out of range, which then read scale 0; the quantizer's bits for y_q).
  */
 typedef struct {
   int64_t batch, seqlen, dim, dstate, ngroups;
@@ -209,6 +214,10 @@ typedef struct {
   uint32_t* status;
   float se_lo, se_hi; /* soft-edge thresholds of x_format F16_SOFTEDGE (|v| < se_lo small,
                          |v| > se_hi large); ignored otherwise */
+  int8_t* y_q;              /* int8 y (see above) or NULL */
+  const int32_t* y_group;   /* [d] output cluster of each channel (with y_q) */
+  const float* y_scale;     /* [n_y_groups] static output scales (with y_q) */
+  int32_t n_y_groups;
 } ssmq_scan_args;
 
 ssmq_status ssmq_selective_scan_w8(const ssmq_scan_args* args, void* stream);
@@ -234,8 +243,12 @@ ssmq_status ssmq_selective_scan_w8(const ssmq_scan_args* args, void* stream);
  *   B, C     (b, L, G, N) int8; head h reads group floor(h * G / H)
  *   B_scale, C_scale fp32[G * N / state_group_size]
  *   h0       fp32 (b, H, P, N) or NULL
- *   y        (b, L, H, P) binary16 output
+ *   y        (b, L, H, P) binary16 output, or NULL when y_q is given
  *   h_final  fp32 (b, H, P, N) output or NULL
+ *   y_q      (b, L, H, P) int8 output or NULL: the persistent-INT8 epilogue,
+ *            channel h * P + p quantized with y_scale[y_group[h * P + p]]
+ *            after rounding to binary16 (the bytes of ssmq_quantize_groups
+ *            of the binary16 y)
  * workspace: device memory of at least ssmq_ssd_workspace_size(args) bytes,
  *   256-byte aligned, caller-owned, contents need not be initialised.
  * Supported: P == 64, N == 128, chunk in {64, 128, 256}, H % G == 0.  The
@@ -269,6 +282,10 @@ typedef struct {
   uint16_t* y;
   float* h_final;
   uint32_t* status;
+  int8_t* y_q;              /* int8 y (see above) or NULL */
+  const int32_t* y_group;   /* [H * P] output cluster of each channel (with y_q) */
+  const float* y_scale;     /* [n_y_groups] static output scales (with y_q) */
+  int32_t n_y_groups;
 } ssmq_ssd_args;
 
 size_t ssmq_ssd_workspace_size(const ssmq_ssd_args* args);

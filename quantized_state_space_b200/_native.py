@@ -37,7 +37,8 @@ class ScanArgs(C.Structure):
                 ("se_scale", _f32), ("se_log2_ratio", _i32), ("dt", _vp), ("dt_bias", _vp),
                 ("dt_softplus", _i32), ("A", _vp), ("D", _vp), ("z", _vp), ("B", _vp),
                 ("C", _vp), ("B_scale", _vp), ("C_scale", _vp), ("h0", _vp), ("y", _vp),
-                ("h_final", _vp), ("status", _vp), ("se_lo", _f32), ("se_hi", _f32)]
+                ("h_final", _vp), ("status", _vp), ("se_lo", _f32), ("se_hi", _f32),
+                ("y_q", _vp), ("y_group", _vp), ("y_scale", _vp), ("n_y_groups", _i32)]
 
 
 class SSDArgs(C.Structure):
@@ -47,7 +48,8 @@ class SSDArgs(C.Structure):
                 ("x_scale", _vp), ("n_x_groups", _i32), ("se_scale", _f32),
                 ("se_log2_ratio", _i32), ("dt", _vp), ("dt_bias", _vp), ("dt_softplus", _i32),
                 ("A", _vp), ("D", _vp), ("z", _vp), ("B", _vp), ("C", _vp), ("B_scale", _vp),
-                ("C_scale", _vp), ("h0", _vp), ("y", _vp), ("h_final", _vp), ("status", _vp)]
+                ("C_scale", _vp), ("h0", _vp), ("y", _vp), ("h_final", _vp), ("status", _vp), ("y_q", _vp),
+                ("y_group", _vp), ("y_scale", _vp), ("n_y_groups", _i32)]
 
 
 class DecodeArgs(C.Structure):

@@ -61,19 +61,34 @@ def _x_fields(x, x_group, x_scale, se_scale, se_log2_ratio, se_lo=None, se_hi=No
                 n_x_groups=int(x_scale.numel()), se_log2_ratio=se_log2_ratio)
 
 
+def _y_fields(shape, device, y_group, y_scale, y_q, want_y, y):
+    """Optional int8 output (static per-cluster scales) and the binary16 y."""
+    f = {}
+    if y_group is not None:
+        _dev_check(y_group, y_scale)
+        if y_q is None:
+            y_q = torch.empty(shape, dtype=torch.int8, device=device)
+        f = dict(y_q=y_q, y_group=y_group, y_scale=y_scale, n_y_groups=int(y_scale.numel()))
+    if want_y and y is None:
+        y = torch.empty(shape, dtype=torch.float16, device=device)
+    return (y if want_y else None), y_q, f
+
+
 def selective_scan(x, dt, A, B, C, B_scale, C_scale, state_group_size, *, x_group=None,
                    x_scale=None, se_scale=0.0, se_log2_ratio=2, se_lo=None, se_hi=None, D=None,
                    z=None, dt_bias=None, dt_softplus=True, h0=None, y=None, h_final=None,
-                   return_state=True, status=None):
+                   return_state=True, y_group=None, y_scale=None, y_q=None, want_y=True,
+                   status=None):
     """Mamba-1 W8A8 selective scan.  x (b, d, L) int8 codes, soft-edge uint8
     codes, or float16 activations that the kernel encodes itself (with
     x_group / x_scale, or with se_scale / se_lo / se_hi); dt, z (b, d, L)
-    float16; B, C (b, G, N, L) int8.  Returns (y, h_final)."""
+    float16; B, C (b, G, N, L) int8.  Returns (y, h_final), or (y, h_final,
+    y_q) when y_group / y_scale ask for the int8 output (y is None when
+    want_y is False)."""
     b, d, L = x.shape
     G, Nst = B.shape[1], B.shape[2]
     _dev_check(x, dt, A, B, C, B_scale, C_scale, x_group, x_scale, D, z, dt_bias, h0)
-    if y is None:
-        y = torch.empty((b, d, L), dtype=torch.float16, device=x.device)
+    y, y_q, yf = _y_fields((b, d, L), x.device, y_group, y_scale, y_q, want_y, y)
     if h_final is None and return_state:
         h_final = torch.empty((b, d, Nst), dtype=torch.float32, device=x.device)
     N.ssmq_selective_scan_w8(batch=b, seqlen=L, dim=d, dstate=Nst, ngroups=G,
@@ -82,21 +97,22 @@ def selective_scan(x, dt, A, B, C, B_scale, C_scale, state_group_size, *, x_grou
                                          se_hi),
                              dt=dt, dt_bias=dt_bias, dt_softplus=int(bool(dt_softplus)), A=A,
                              D=D, z=z, B=B, C=C, B_scale=B_scale, C_scale=C_scale, h0=h0, y=y,
-                             h_final=h_final, status=status)
-    return y, h_final
+                             h_final=h_final, status=status, **yf)
+    return (y, h_final, y_q) if yf else (y, h_final)
 
 
 def ssd_chunk_scan(x, dt, A, B, C, B_scale, C_scale, state_group_size, *, chunk=256,
                    x_group=None, x_scale=None, se_scale=0.0, se_log2_ratio=2, D=None, z=None,
                    dt_bias=None, dt_softplus=True, h0=None, y=None, h_final=None,
-                   return_state=True, workspace=None, status=None):
+                   return_state=True, y_group=None, y_scale=None, y_q=None, want_y=True,
+                   workspace=None, status=None):
     """Mamba-2 SSD chunked scan.  x (b, L, H, P) int8 / soft-edge uint8;
-    dt (b, L, H) float16; B, C (b, L, G, N) int8.  Returns (y, h_final)."""
+    dt (b, L, H) float16; B, C (b, L, G, N) int8.  Returns (y, h_final), or
+    (y, h_final, y_q) with the int8 output (y_group over the H * P channels)."""
     b, L, H, P = x.shape
     G, Nst = B.shape[2], B.shape[3]
     _dev_check(x, dt, A, B, C, B_scale, C_scale, x_group, x_scale, D, z, dt_bias, h0)
-    if y is None:
-        y = torch.empty((b, L, H, P), dtype=torch.float16, device=x.device)
+    y, y_q, yf = _y_fields((b, L, H, P), x.device, y_group, y_scale, y_q, want_y, y)
     if h_final is None and return_state:
         h_final = torch.empty((b, H, P, Nst), dtype=torch.float32, device=x.device)
     fields = dict(batch=b, seqlen=L, nheads=H, headdim=P, dstate=Nst, ngroups=G, chunk=chunk,
@@ -104,7 +120,7 @@ def ssd_chunk_scan(x, dt, A, B, C, B_scale, C_scale, state_group_size, *, chunk=
                   **_x_fields(x, x_group, x_scale, se_scale, se_log2_ratio),
                   dt=dt, dt_bias=dt_bias, dt_softplus=int(bool(dt_softplus)), A=A, D=D, z=z,
                   B=B, C=C, B_scale=B_scale, C_scale=C_scale, h0=h0, y=y, h_final=h_final,
-                  status=status)
+                  status=status, **yf)
     ws = N.ssmq_ssd_workspace_size(**fields)
     if ws and workspace is None:
         workspace = torch.empty(ws + 256, dtype=torch.uint8, device=x.device)
@@ -113,7 +129,7 @@ def ssd_chunk_scan(x, dt, A, B, C, B_scale, C_scale, state_group_size, *, chunk=
         base = workspace.data_ptr()
         wptr = (base + 255) // 256 * 256
     N.ssmq_ssd_chunk_scan_w8(workspace=wptr, ws_bytes=ws, **fields)
-    return y, h_final
+    return (y, h_final, y_q) if yf else (y, h_final)
 
 
 def state_update(state, x, dt, A, B, C, B_scale, C_scale, state_group_size, *, x_group=None,

@@ -61,6 +61,16 @@ ssmq_status check_x(int32_t fmt, const void* x, const int32_t* x_group, const fl
   return SSMQ_OK;
 }
 
+// optional int8 output: the cluster map and scales come with it
+ssmq_status check_yq(const int8_t* y_q, const int32_t* y_group, const float* y_scale,
+                     int32_t n_y_groups, const char* fn) {
+  if (!y_q) return SSMQ_OK;
+  REQUIRE(aligned16(y_q), SSMQ_ERR_ALIGNMENT, "%s: y_q must be 16-byte aligned", fn);
+  REQUIRE(y_group && y_scale && n_y_groups >= 1, SSMQ_ERR_INVALID_ARG,
+          "%s: y_q needs y_group, y_scale and n_y_groups >= 1", fn);
+  return SSMQ_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -155,9 +165,11 @@ ssmq_status ssmq_selective_scan_w8(const ssmq_scan_args* a, void* stream) {
     if (xs != SSMQ_OK) return xs;
     REQUIRE(a->x_format != SSMQ_X_F16_SOFTEDGE || a->se_lo <= a->se_hi, SSMQ_ERR_INVALID_ARG,
             "%s: se_lo must not exceed se_hi (as ssmq_softedge_encode)", fn);
-    REQUIRE(a->dt && a->A && a->B && a->C && a->B_scale && a->C_scale && a->y,
+    REQUIRE(a->dt && a->A && a->B && a->C && a->B_scale && a->C_scale && (a->y || a->y_q),
             SSMQ_ERR_INVALID_ARG,
-            "%s: a required tensor (dt, A, B, C, B_scale, C_scale, y) is NULL", fn);
+            "%s: a required tensor (dt, A, B, C, B_scale, C_scale, y or y_q) is NULL", fn);
+    const ssmq_status ys = check_yq(a->y_q, a->y_group, a->y_scale, a->n_y_groups, fn);
+    if (ys != SSMQ_OK) return ys;
   }
   if (injected(fn)) return fail(SSMQ_ERR_CUDA, "%s: injected launch failure", fn);
   return finish(ssmq::launch_selective_scan(*a, (cudaStream_t)stream), fn);
@@ -186,11 +198,14 @@ ssmq_status ssmq_ssd_chunk_scan_w8(const ssmq_ssd_args* a, void* workspace, size
   const ssmq_status xs = check_x(a->x_format, a->x, a->x_group, a->x_scale, a->n_x_groups,
                                  a->se_log2_ratio, fn);
   if (xs != SSMQ_OK) return xs;
-  REQUIRE(a->dt && a->A && a->B && a->C && a->B_scale && a->C_scale && a->y, SSMQ_ERR_INVALID_ARG,
-          "%s: a required tensor (dt, A, B, C, B_scale, C_scale, y) is NULL", fn);
+  REQUIRE(a->dt && a->A && a->B && a->C && a->B_scale && a->C_scale && (a->y || a->y_q),
+          SSMQ_ERR_INVALID_ARG,
+          "%s: a required tensor (dt, A, B, C, B_scale, C_scale, y or y_q) is NULL", fn);
   REQUIRE(aligned16(a->x) && aligned16(a->dt) && aligned16(a->z) && aligned16(a->B) &&
               aligned16(a->C) && aligned16(a->y) && aligned16(a->h0) && aligned16(a->h_final),
           SSMQ_ERR_ALIGNMENT, "%s: tensors must be 16-byte aligned", fn);
+  const ssmq_status ys = check_yq(a->y_q, a->y_group, a->y_scale, a->n_y_groups, fn);
+  if (ys != SSMQ_OK) return ys;
   const size_t need = ssmq::ssd_workspace_bytes(*a);
   REQUIRE(need == 0 || (workspace && ws_bytes >= need), SSMQ_ERR_INVALID_ARG,
           "%s: workspace of %zu bytes required (got %zu)", fn, need, ws_bytes);

@@ -65,6 +65,10 @@ struct M1Params {
   const float* C_scale;
   const float* h0;
   uint16_t* y;
+  int8_t* y_q;
+  const int32_t* y_group;
+  const float* y_scale;
+  int n_y_groups;
   float* h_final;
   uint32_t* status;
   int n_ctile;
@@ -187,7 +191,7 @@ __device__ __forceinline__ void fetch_chunk(const M1Params& p, Raw<kN, kCH, XT>&
   }
 }
 
-template <int kN, int kCH, int kSPL, int kXFmt>
+template <int kN, int kCH, int kSPL, int kXFmt, bool kYQ>
 __global__ void __launch_bounds__(kCH*(kN / kSPL)) m1_scan_kernel(const M1Params p) {
   static_assert(kSPL == 2 || kSPL == 4, "2 or 4 states per thread");
   constexpr bool kXF16 = kXFmt == SSMQ_X_F16_GROUP || kXFmt == SSMQ_X_F16_SOFTEDGE;
@@ -244,6 +248,19 @@ __global__ void __launch_bounds__(kCH*(kN / kSPL)) m1_scan_kernel(const M1Params
     }
     bias = p.dt_bias ? __ldg(p.dt_bias + lch) : 0.0f;
     Dc = p.D ? __ldg(p.D + lch) : 0.0f;
+  }
+  // int8 output: this channel's static scale and its reciprocal
+  float ys = 0.0f, yrs = 0.0f;
+  bool yok = true;
+  if (kYQ && lvalid) {
+    const int yg = __ldg(p.y_group + lch);
+    if ((unsigned)yg < (unsigned)p.n_y_groups) {
+      ys = __ldg(p.y_scale + yg);
+      const float r = __frcp_rn(ys);
+      yrs = usable_recip(ys, r) ? r : 0.0f;
+    } else {
+      yok = false;
+    }
   }
   for (int i = tid; i < 2 * kN; i += NT) {
     const int which = i / kN, n = i % kN;
@@ -352,6 +369,42 @@ __global__ void __launch_bounds__(kCH*(kN / kSPL)) m1_scan_kernel(const M1Params
       if (p.z) v *= silu_f(h2f((uint16_t)(zw[i >> 1] >> (16 * (i & 1)))));
       yv[i] = v;
     }
+    if constexpr (kYQ) {
+      // persistent-INT8 epilogue: the quantizer applied to the binary16 y, by
+      // its reciprocal + magic-number route (exact division near a tie)
+      const bool yfast = yok && yrs != 0.0f;
+      uint32_t qw[(SPS + 3) / 4] = {};
+#pragma unroll
+      for (int i = 0; i < SPS; ++i) {
+        const float v = h2f(f2h(yv[i]));
+        const float yc = fminf(fmaxf(v * yrs, -127.0f), 127.0f);
+        const float m = yc + 12582912.0f;
+        const uint32_t c =
+            (yfast && fabsf(yc - (m - 12582912.0f)) < 0.5f - 1.0f / 16384.0f && fabsf(v) <= 3.402823466e38f)
+                ? __float_as_uint(m) & 0xFFu
+                : (uint32_t)quant_elem(v, ys, yrs, yok, flags) & 0xFFu;
+        qw[i >> 2] |= c << (8 * (i & 3));
+      }
+      int8_t* qd = p.y_q + (bb * d + lch) * L + t0 + tb;
+      if (p.vec_ok) {
+        if constexpr (SPS == 16) {
+          *reinterpret_cast<uint4*>(qd) = make_uint4(qw[0], qw[1], qw[2], qw[3]);
+        } else if constexpr (SPS == 8) {
+          *reinterpret_cast<uint2*>(qd) = make_uint2(qw[0], qw[1]);
+        } else if constexpr (SPS == 4) {
+          *reinterpret_cast<uint32_t*>(qd) = qw[0];
+        } else if constexpr (SPS == 2) {
+          *reinterpret_cast<uint16_t*>(qd) = (uint16_t)qw[0];
+        } else {
+          qd[0] = (int8_t)qw[0];
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < SPS; ++i)
+          if (tb + i < tl) qd[i] = (int8_t)(qw[i >> 2] >> (8 * (i & 3)));
+      }
+    }
+    if (kYQ && !p.y) return;
     uint16_t* dst = p.y + (bb * d + lch) * L + t0 + tb;
     if (p.vec_ok && SPS >= 2) {
       // tl % 16 == 0: the whole run is valid
@@ -473,10 +526,14 @@ cudaError_t launch_m1(const M1Params& prm, int xfmt, int64_t batch, cudaStream_t
   const dim3 block(kCH * (kN / kSPL));
   const bool f16 = xfmt == SSMQ_X_F16_GROUP || xfmt == SSMQ_X_F16_SOFTEDGE;
   const size_t smem = f16 ? sizeof(M1Smem<kN, kCH, uint16_t>) : sizeof(M1Smem<kN, kCH, uint8_t>);
-  auto kern = xfmt == SSMQ_X_SOFTEDGE       ? m1_scan_kernel<kN, kCH, kSPL, SSMQ_X_SOFTEDGE>
-              : xfmt == SSMQ_X_F16_GROUP    ? m1_scan_kernel<kN, kCH, kSPL, SSMQ_X_F16_GROUP>
-              : xfmt == SSMQ_X_F16_SOFTEDGE ? m1_scan_kernel<kN, kCH, kSPL, SSMQ_X_F16_SOFTEDGE>
-                                            : m1_scan_kernel<kN, kCH, kSPL, SSMQ_X_INT8_GROUP>;
+  auto pick = [&](auto yq) {
+    constexpr bool Q = decltype(yq)::value;
+    return xfmt == SSMQ_X_SOFTEDGE       ? m1_scan_kernel<kN, kCH, kSPL, SSMQ_X_SOFTEDGE, Q>
+           : xfmt == SSMQ_X_F16_GROUP    ? m1_scan_kernel<kN, kCH, kSPL, SSMQ_X_F16_GROUP, Q>
+           : xfmt == SSMQ_X_F16_SOFTEDGE ? m1_scan_kernel<kN, kCH, kSPL, SSMQ_X_F16_SOFTEDGE, Q>
+                                         : m1_scan_kernel<kN, kCH, kSPL, SSMQ_X_INT8_GROUP, Q>;
+  };
+  auto kern = p.y_q ? pick(std::true_type{}) : pick(std::false_type{});
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   kern<<<grid, block, smem, st>>>(p);
@@ -512,6 +569,10 @@ cudaError_t launch_selective_scan(const ssmq_scan_args& a, cudaStream_t st) {
   p.C_scale = a.C_scale;
   p.h0 = a.h0;
   p.y = a.y;
+  p.y_q = a.y_q;
+  p.y_group = a.y_group;
+  p.y_scale = a.y_scale;
+  p.n_y_groups = a.n_y_groups;
   p.h_final = a.h_final;
   p.status = a.status;
   p.vec_ok = (a.seqlen % 16 == 0) ? 1 : 0;

@@ -72,7 +72,10 @@ constexpr int F_WH = F_RM + 4 * kQ;     // w'_n as binary16 pairs              [
 constexpr int F_HF = F_WH + kN / 2;     // sC_n / w'_n (state operand factor)  [128]
 constexpr int F_SB = F_HF + kN;         // sB_n                                [128]
 constexpr int F_SX = F_SB + kN;         // x scale per p                       [64]
-constexpr int F_RED = F_SX + kP;        // reductions: w max, S_last, per-warp state max  [32]
+constexpr int F_YS = F_SX + kP;         // int8-y scale per p                  [64]
+constexpr int F_YR = F_YS + kP;         // its reciprocal (0: exact division)  [64]
+constexpr int F_YOK = F_YR + kP;        // 1 if the p's output cluster id is valid  [64]
+constexpr int F_RED = F_YOK + kP;       // reductions: w max, S_last, per-warp state max  [32]
 constexpr int F_END = F_RED + 32;
 // raw int8 rows of the next tile, fetched with cp.async during this tile
 constexpr int OFF_RAW = (OFF_F + F_END * 4 + 127) / 128 * 128;
@@ -104,6 +107,10 @@ struct SsdParams {
   const float* C_scale;
   const float* h0;
   uint16_t* y;
+  int8_t* y_q;
+  const int32_t* y_group;
+  const float* y_scale;
+  int n_y_groups;
   float* h_final;
   uint32_t* status;
 };
@@ -232,6 +239,7 @@ __device__ __forceinline__ void tile_factors(float* F, int fb, int ql, const flo
   }
 }
 
+template <bool kYQ>
 __global__ void __launch_bounds__(kThreads, 1) ssd_kernel(const SsdParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ uint32_t tmem_slot;
@@ -269,6 +277,19 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_kernel(const SsdParams p) {
       }
     }
     F[F_SX + tid] = sx;
+    float ysc = 0.0f, yok = 1.0f;
+    if (kYQ) {
+      const int yg = __ldg(p.y_group + hd * kP + tid);
+      if ((unsigned)yg < (unsigned)p.n_y_groups) {
+        ysc = __ldg(p.y_scale + yg);
+      } else {
+        yok = 0.0f;
+      }
+    }
+    const float yr = __frcp_rn(ysc);
+    F[F_YS + tid] = ysc;
+    F[F_YR + tid] = usable_recip(ysc, yr) ? yr : 0.0f;
+    F[F_YOK + tid] = yok;
   }
   if (tid == 0) abort_flag = 0;
   if (warp == 0) tc::tmem_alloc(&tmem_slot, kTmemCols);
@@ -618,7 +639,7 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_kernel(const SsdParams p) {
             zw[4 * i + 3] = zz.w;
           }
         }
-        uint32_t out[8];
+        uint32_t out[8], qo[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
         for (int j = 0; j < 16; j += 2) {
           const float2 xp = __half22float2(*reinterpret_cast<const __half2*>(&xw[j >> 1]));
@@ -631,12 +652,30 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_kernel(const SsdParams p) {
             float yv = fmaf(sxv[pj], fmaf(Dh, e ? xp.y : xp.x, yd[pj] * rs), es * yo[pj]);
             if (p.z) yv *= silu_f(e ? zf.y : zf.x);
             r2[e] = yv;
+            if constexpr (kYQ) {
+              // persistent-INT8 epilogue: the quantizer applied to the binary16 y,
+              // by its reciprocal + magic-number route (exact division near a tie)
+              const int pc = 16 * q4 + pj;
+              const float v = h2f(f2h(yv)), ysc = F[F_YS + pc], yrs = F[F_YR + pc];
+              const bool yok = F[F_YOK + pc] != 0.0f;
+              const float yc = fminf(fmaxf(v * yrs, -127.0f), 127.0f);
+              const float m = yc + 12582912.0f;
+              const uint32_t c = (yok && yrs != 0.0f &&
+                                  fabsf(yc - (m - 12582912.0f)) < 0.5f - 1.0f / 16384.0f &&
+                                  fabsf(v) <= 3.402823466e38f)
+                                     ? __float_as_uint(m) & 0xFFu
+                                     : (uint32_t)quant_elem(v, ysc, yrs, yok, flags) & 0xFFu;
+              qo[pj >> 2] |= c << (8 * (pj & 3));
+            }
           }
           out[j / 2] = pack_half2(r2[0], r2[1]);
         }
-        uint4* yr = reinterpret_cast<uint4*>(p.y + yo_off);
-        yr[0] = make_uint4(out[0], out[1], out[2], out[3]);
-        yr[1] = make_uint4(out[4], out[5], out[6], out[7]);
+        if (kYQ) *reinterpret_cast<uint4*>(p.y_q + yo_off) = make_uint4(qo[0], qo[1], qo[2], qo[3]);
+        if (!kYQ || p.y) {
+          uint4* yr = reinterpret_cast<uint4*>(p.y + yo_off);
+          yr[0] = make_uint4(out[0], out[1], out[2], out[3]);
+          yr[1] = make_uint4(out[4], out[5], out[6], out[7]);
+        }
       }
     }
     // ---- state: h = exp(S_last) h + sB_n sx_p 2^e_x acc  (thread: row n, 16 p)
@@ -717,12 +756,17 @@ cudaError_t launch_ssd(const ssmq_ssd_args& a, void*, cudaStream_t st) {
   p.C_scale = a.C_scale;
   p.h0 = a.h0;
   p.y = a.y;
+  p.y_q = a.y_q;
+  p.y_group = a.y_group;
+  p.y_scale = a.y_scale;
+  p.n_y_groups = a.n_y_groups;
   p.h_final = a.h_final;
   p.status = a.status;
-  cudaError_t e = cudaFuncSetAttribute(ssd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  auto kern = p.y_q ? ssd_kernel<true> : ssd_kernel<false>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        kSmemBytes);
   if (e != cudaSuccess) return e;
-  ssd_kernel<<<(unsigned)units, kThreads, kSmemBytes, st>>>(p);
+  kern<<<(unsigned)units, kThreads, kSmemBytes, st>>>(p);
   return cudaGetLastError();
 }
 

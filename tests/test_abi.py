@@ -121,6 +121,11 @@ def test_scan_validation(L):
     assert S(x_format=N.X_F16_SOFTEDGE, x_group=None, x_scale=None, se_lo=float("nan"),
              se_hi=1.0) == N.ERR_INVALID_ARG
     assert S(x_format=4) == N.ERR_INVALID_ARG
+    # int8 y: needs its cluster map; y may be dropped only when y_q is given
+    assert S(y_q=FAKE, y_group=None, y_scale=FAKE, n_y_groups=2) == N.ERR_INVALID_ARG
+    assert S(y_q=FAKE, y_group=FAKE, y_scale=FAKE, n_y_groups=0) == N.ERR_INVALID_ARG
+    assert S(y_q=FAKE + 8, y_group=FAKE, y_scale=FAKE, n_y_groups=2) == N.ERR_ALIGNMENT
+    assert S(y=None) == N.ERR_INVALID_ARG
     assert S(batch=0) == N.OK
     assert L.ssmq_selective_scan_w8(None, None) == N.ERR_INVALID_ARG
 
@@ -141,6 +146,8 @@ def test_ssd_validation(L):
     assert S(ngroups=3) == N.ERR_INVALID_ARG
     assert S(x=None) == N.ERR_INVALID_ARG
     assert S(x_format=N.X_F16_GROUP) == N.ERR_UNSUPPORTED  # Mamba-1 scan only
+    assert S(y=None) == N.ERR_INVALID_ARG
+    assert S(y_q=FAKE, y_group=None, y_scale=FAKE, n_y_groups=2) == N.ERR_INVALID_ARG
     need = L.ssmq_ssd_workspace_size(C.byref(_ssd_args()))
     if need:
         assert S(ws=None, nb=0) == N.ERR_INVALID_ARG

@@ -286,3 +286,56 @@ def test_fused_encode_scan_vs_oracle(orc):
     po = dict(p, x=q.reshape(b, d, L))
     yo, ho = oracle_scan(orc, po)
     assert_scan_close(H(y).astype(np.float64), yo.reshape(y.shape), H(hf), ho.reshape(hf.shape))
+
+
+# ---- persistent-INT8 epilogue (SSDi8 abstract): int8 y with static per-cluster
+# output scales; the bytes must equal the quantizer applied to the binary16 y.
+
+YQ_CASES = [
+    # (b, L, d, N, gs, fmt)
+    (2, 256, 64, 16, 4, "int8"),
+    (2, 200, 40, 16, 4, "int8"),      # ragged L: scalar stores
+    (1, 96, 64, 4, 2, "int8"),
+    (1, 64, 16, 64, 16, "softedge"),
+]
+
+
+@pytest.mark.parametrize("ci", range(len(YQ_CASES)))
+def test_scan_int8_y_bit_exact(orc, ci):
+    b, L, d, N_, gs, fmt = YQ_CASES[ci]
+    p = m1_problem(800 + ci, b, L, d, N_, gs=gs, gate=True, h0=True, x_format=fmt)
+    rng = np.random.default_rng(820 + ci)
+    ky = 4
+    ygrp = rng.integers(0, ky, size=d).astype(np.int32)
+    ygrp[3] = ky + 5                                   # one channel with a bad cluster id
+    ysc = synth.random_scales(rng, ky, 0.002, 0.02)
+    st = status_word()
+    y, hf, yq = (None, None, None)
+    y_t, hf_t, yq_t = api.selective_scan(
+        T(p["x"]), T(p["dt"]), T(p["A"]), T(p["B"]), T(p["C"]), T(p["B_scale"]), T(p["C_scale"]),
+        gs, y_group=T(ygrp), y_scale=T(ysc), status=st,
+        **({"se_scale": p["se_scale"]} if fmt == "softedge" else
+           {"x_group": T(p["x_group"]), "x_scale": T(p["x_scale"])}),
+        D=T(p["D"]), z=T(p["z"]), h0=T(p["h0"]))
+    ref, _ = api.quantize_groups(y_t, b, d, L, T(ygrp), ky, scales=T(ysc))
+    np.testing.assert_array_equal(H(yq_t), H(ref))
+    assert int(H(st)[0]) & 2                           # SSMQ_DEV_BAD_GROUP seen
+    assert not H(yq_t)[:, 3].any()
+    # without the binary16 y: same codes, same state
+    y2, hf2, yq2 = api.selective_scan(
+        T(p["x"]), T(p["dt"]), T(p["A"]), T(p["B"]), T(p["C"]), T(p["B_scale"]), T(p["C_scale"]),
+        gs, y_group=T(ygrp), y_scale=T(ysc), want_y=False,
+        **({"se_scale": p["se_scale"]} if fmt == "softedge" else
+           {"x_group": T(p["x_group"]), "x_scale": T(p["x_scale"])}),
+        D=T(p["D"]), z=T(p["z"]), h0=T(p["h0"]))
+    assert y2 is None
+    np.testing.assert_array_equal(H(yq2), H(yq_t))
+    np.testing.assert_array_equal(H(hf2).view(np.uint32), H(hf_t).view(np.uint32))
+    # the dequantized codes against the oracle's y: within the y tolerance plus half a step
+    yo, _ = oracle_scan(orc, p)
+    yo = yo.reshape(b, d, L)
+    deq = H(yq_t).astype(np.float64) * ysc[np.clip(ygrp, 0, ky - 1)][None, :, None]
+    ok = ygrp < ky
+    lim = 2e-3 * np.abs(yo).max() + 0.5 * ysc[np.clip(ygrp, 0, ky - 1)][None, :, None]
+    inside = np.abs(yo) <= 127 * ysc[np.clip(ygrp, 0, ky - 1)][None, :, None]
+    assert np.all((np.abs(deq - yo) <= lim)[:, ok][inside[:, ok]])

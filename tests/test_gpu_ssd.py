@@ -141,3 +141,26 @@ def test_ssd27b_workload_end_to_end(orc):
     yg = np.stack([yg[u // Hh, :, u % Hh, :] for u in units])
     hg = H(hf).reshape(b * Hh, P, Nst)[units]
     assert_scan_close(yg, yo, hg, ho)
+
+
+def test_ssd_int8_y_bit_exact():
+    """Persistent-INT8 epilogue (SSDi8 abstract): int8 y whose bytes equal the
+    quantizer applied to the binary16 y; with the binary16 y dropped the codes
+    and the state are unchanged."""
+    b, L, Hh, P, N_ = 2, 384, 4, 64, 128
+    p = ssd_problem(860, b, L, Hh, P, N_, G=1, gs=8, gate=True, h0=True)
+    rng = np.random.default_rng(861)
+    ky = 6
+    ygrp = rng.integers(0, ky, size=Hh * P).astype(np.int32)
+    ysc = synth.random_scales(rng, ky, 0.002, 0.02)
+    kw = dict(x_group=T(p["x_group"]), x_scale=T(p["x_scale"]), D=T(p["D"]), z=T(p["z"]),
+              h0=T(p["h0"]), y_group=T(ygrp), y_scale=T(ysc))
+    args = (T(p["x"]), T(p["dt"]), T(p["A"]), T(p["B"]), T(p["C"]), T(p["B_scale"]),
+            T(p["C_scale"]), 8)
+    y, hf, yq = api.ssd_chunk_scan(*args, **kw)
+    ref, _ = api.quantize_groups(y, b * L, Hh * P, 1, T(ygrp), ky, scales=T(ysc))
+    np.testing.assert_array_equal(H(yq), H(ref))
+    y2, hf2, yq2 = api.ssd_chunk_scan(*args, want_y=False, **kw)
+    assert y2 is None
+    np.testing.assert_array_equal(H(yq2), H(yq))
+    np.testing.assert_array_equal(H(hf2).view(np.uint32), H(hf).view(np.uint32))
