@@ -146,6 +146,59 @@ ssmq_status ssmq_softedge_decode(const uint8_t* codes, int64_t n, float scale,
                                  int32_t log2_ratio, float* out, void* stream);
 
 /* ------------------------------------------------------------------------ */
+/* Calibration on the device                                                 */
+/* ------------------------------------------------------------------------ */
+/*
+ * Passages: Quamba2 method steps 1-2 (activation statistics; channels sorted
+ * by magnitude and cut into clusters sharing one scale) and the Quamba-SE
+ * write-up 4.1 (thresholds L = 5th, H = 99.9th percentile of the activation
+ * magnitudes, refreshed as alpha * new + (1 - alpha) * running, alpha 0.1).
+ *
+ * ssmq_group_absmax: absmax[g] = largest |v| over the finite elements of
+ *   group g (same tensor / group-map conventions as ssmq_quantize_groups);
+ *   0 for a group without finite elements.  Exact (no rounding).  Status:
+ *   NONFINITE / BAD_GROUP as the quantizer.  absmax is device fp32[n_groups].
+ *
+ * ssmq_cluster_by_absmax: channels sorted by (absmax, index) ascending; the
+ *   sorted order is cut into k clusters, cluster j holding sorted positions
+ *   [floor(n j / k), floor(n (j + 1) / k)); cluster_of[c] (device int32[n])
+ *   gets the cluster of channel c, scales[j] (device fp32[k]) the binary32
+ *   quotient fl32(max member absmax / 127).  1 <= k <= n <= 65536
+ *   (SSMQ_ERR_UNSUPPORTED above).  Negative or non-finite absmax values set
+ *   SSMQ_DEV_NONFINITE and sort last.
+ *
+ * ssmq_percentile_abs: out[i] (device fp32[nq]) = the q[i]-th percentile
+ *   (host doubles in [0, 100], 1 <= nq <= 4) of |v| over the m finite
+ *   elements of src: with pos = (m - 1) q / 100, k = floor(pos) (clamped to
+ *   [0, m - 1]), the k-th and (k+1)-th smallest (0-based) values a, b give
+ *   fl32(a + (pos - k) (b - a)) evaluated in double; 0 when m == 0.  Exact
+ *   order statistics (radix selection on the magnitude bits).
+ *
+ * ssmq_softedge_calibrate: thresholds (device fp32[3] = {scale, lo, hi},
+ *   in/out): lo' = fl32(P(q_lo)), hi' = fl32(P(q_hi)) as above; then, for
+ *   alpha < 1, lo = fl32(alpha lo' + (1 - alpha) lo), hi likewise (in double),
+ *   else lo = lo', hi = hi'; finally scale = fl32(hi / 63) -- the parameters of
+ *   ssmq_softedge_encode.  0 <= q_lo <= q_hi <= 100, 0 < alpha <= 1.
+ *
+ * The two percentile calls need a caller-owned device workspace of
+ * ssmq_percentile_workspace_size() bytes, 256-byte aligned (contents need
+ * not be initialised; one call at a time per workspace).
+ */
+ssmq_status ssmq_group_absmax(const void* src, ssmq_dtype dtype, int64_t outer, int64_t mid,
+                              int64_t inner, const int32_t* group_of_mid, int32_t n_groups,
+                              float* absmax, uint32_t* status, void* stream);
+ssmq_status ssmq_cluster_by_absmax(const float* absmax, int64_t n, int32_t k,
+                                   int32_t* cluster_of, float* scales, uint32_t* status,
+                                   void* stream);
+size_t ssmq_percentile_workspace_size(void);
+ssmq_status ssmq_percentile_abs(const void* src, ssmq_dtype dtype, int64_t n, const double* q,
+                                int32_t nq, float* out, void* workspace, size_t ws_bytes,
+                                void* stream);
+ssmq_status ssmq_softedge_calibrate(const void* src, ssmq_dtype dtype, int64_t n, double q_lo,
+                                    double q_hi, float alpha, float* thresholds,
+                                    void* workspace, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------ */
 /* Mamba-1 diagonal selective scan                                           */
 /* ------------------------------------------------------------------------ */
 /*

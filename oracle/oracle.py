@@ -91,6 +91,9 @@ def lib():
         L.orc_cluster_by_absmax.argtypes = [_vp, _i64, _i32, _vp, _vp]
         L.orc_percentile_abs.restype = C.c_double
         L.orc_percentile_abs.argtypes = [_vp, _i32, _i64, C.c_double]
+        L.orc_softedge_thresholds.restype = None
+        L.orc_softedge_thresholds.argtypes = [_vp, _i32, _i64, C.c_double, C.c_double,
+                                              C.c_double, _vp]
         _lib = L
     return _lib
 
@@ -373,3 +376,11 @@ def cluster_by_absmax(absmax, k):
 def percentile_abs(src, q):
     s, is16 = _src(src)
     return float(lib().orc_percentile_abs(_p(s), is16, s.size, q))
+
+
+def softedge_thresholds(src, q_lo, q_hi, alpha, previous=(0.0, 0.0, 0.0)):
+    """{scale, lo, hi} float32[3] after one threshold update."""
+    s, is16 = _src(src)
+    thr = np.asarray(previous, dtype=np.float32).copy()
+    lib().orc_softedge_thresholds(_p(s), is16, s.size, q_lo, q_hi, alpha, _p(thr))
+    return thr

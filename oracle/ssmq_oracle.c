@@ -718,3 +718,20 @@ double orc_percentile_abs(const void* src, int32_t src_is_f16, int64_t n,
   free(v);
   return vk + frac * (vk1 - vk);
 }
+
+/* [SE] 4.1: L at the 5th and H at the 99.9th percentile of the activation
+ * magnitudes, refreshed from a new batch by alpha * new + (1 - alpha) *
+ * running (alpha = 0.1 there); the base scale puts H at the top of the
+ * standard mode (reading: s = H / 63). */
+void orc_softedge_thresholds(const void* src, int32_t src_is_f16, int64_t n, double q_lo,
+                             double q_hi, double alpha, float* thr) {
+  float lo = (float)orc_percentile_abs(src, src_is_f16, n, q_lo);
+  float hi = (float)orc_percentile_abs(src, src_is_f16, n, q_hi);
+  if (alpha != 1.0) {
+    lo = (float)(alpha * (double)lo + (1.0 - alpha) * (double)thr[1]);
+    hi = (float)(alpha * (double)hi + (1.0 - alpha) * (double)thr[2]);
+  }
+  thr[1] = lo;
+  thr[2] = hi;
+  thr[0] = (float)((double)hi / 63.0);
+}

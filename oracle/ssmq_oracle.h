@@ -166,6 +166,11 @@ int32_t orc_cluster_by_absmax(const double* absmax, int64_t n, int32_t k,
 /* q-th percentile (linear interpolation between order statistics) of |v| */
 double orc_percentile_abs(const void* src, int32_t src_is_f16, int64_t n,
                           double q);
+/* soft-edge parameters thr = {scale, lo, hi}: lo, hi from the q_lo / q_hi
+ * percentiles of |v| (rounded to binary32), blended as alpha new +
+ * (1 - alpha) previous when alpha != 1, then scale = fl32(hi / 63). */
+void orc_softedge_thresholds(const void* src, int32_t src_is_f16, int64_t n, double q_lo,
+                             double q_hi, double alpha, float* thr);
 
 #ifdef __cplusplus
 }

@@ -82,6 +82,13 @@ SIGNATURES = {
     "ssmq_ssd_chunk_scan_w8": (_i32, [C.POINTER(SSDArgs), _vp, C.c_size_t, _vp]),
     "ssmq_state_update_w8": (_i32, [C.POINTER(DecodeArgs), _vp]),
     "ssmq_selective_state_update_w8": (_i32, [C.POINTER(M1DecodeArgs), _vp]),
+    "ssmq_group_absmax": (_i32, [_vp, _i32, _i64, _i64, _i64, _vp, _i32, _vp, _vp, _vp]),
+    "ssmq_cluster_by_absmax": (_i32, [_vp, _i64, _i32, _vp, _vp, _vp, _vp]),
+    "ssmq_percentile_workspace_size": (C.c_size_t, []),
+    "ssmq_percentile_abs": (_i32, [_vp, _i32, _i64, C.POINTER(C.c_double), _i32, _vp, _vp,
+                                   C.c_size_t, _vp]),
+    "ssmq_softedge_calibrate": (_i32, [_vp, _i32, _i64, C.c_double, C.c_double, _f32, _vp, _vp,
+                                       C.c_size_t, _vp]),
     "ssmq_last_error": (C.c_char_p, []),
     "ssmq_version": (_i32, []),
 }
@@ -200,3 +207,32 @@ def ssmq_state_update_w8(stream=None, **fields):
 def ssmq_selective_state_update_w8(stream=None, **fields):
     a = _fill(M1DecodeArgs, fields)
     _check(lib().ssmq_selective_state_update_w8(C.byref(a), _stream(stream)))
+
+
+def ssmq_group_absmax(src, outer, mid, inner, group_of_mid, n_groups, absmax, status=None,
+                      stream=None, dtype=None):
+    _check(lib().ssmq_group_absmax(ptr(src), _dtype_of(src, dtype), outer, mid, inner,
+                                   ptr(group_of_mid), n_groups, ptr(absmax), ptr(status),
+                                   _stream(stream)))
+
+
+def ssmq_cluster_by_absmax(absmax, n, k, cluster_of, scales, status=None, stream=None):
+    _check(lib().ssmq_cluster_by_absmax(ptr(absmax), n, k, ptr(cluster_of), ptr(scales),
+                                        ptr(status), _stream(stream)))
+
+
+def ssmq_percentile_workspace_size():
+    return int(lib().ssmq_percentile_workspace_size())
+
+
+def ssmq_percentile_abs(src, n, q, out, workspace, ws_bytes, stream=None, dtype=None):
+    qa = (C.c_double * len(q))(*[float(v) for v in q])
+    _check(lib().ssmq_percentile_abs(ptr(src), _dtype_of(src, dtype), n, qa, len(q), ptr(out),
+                                     ptr(workspace), ws_bytes, _stream(stream)))
+
+
+def ssmq_softedge_calibrate(src, n, q_lo, q_hi, alpha, thresholds, workspace, ws_bytes,
+                            stream=None, dtype=None):
+    _check(lib().ssmq_softedge_calibrate(ptr(src), _dtype_of(src, dtype), n, float(q_lo),
+                                         float(q_hi), float(alpha), ptr(thresholds),
+                                         ptr(workspace), ws_bytes, _stream(stream)))

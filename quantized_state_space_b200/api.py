@@ -168,3 +168,52 @@ def selective_state_update(state, x, dt, A, B, C, B_scale, C_scale, state_group_
                                      A=A, D=D, z=z, B=B, C=C, B_scale=B_scale, C_scale=C_scale,
                                      state=state, y=y, status=status)
     return y
+
+
+# ---- calibration on the device ----------------------------------------------
+
+def group_absmax(src, outer, mid, inner, group_of_mid, n_groups, *, out=None, status=None):
+    """Exact max |v| per group over the finite elements (float32[n_groups])."""
+    _dev_check(src, group_of_mid)
+    a = out if out is not None else torch.empty(n_groups, dtype=torch.float32, device=src.device)
+    N.ssmq_group_absmax(src, outer, mid, inner, group_of_mid, n_groups, a, status=status)
+    return a
+
+
+def cluster_by_absmax(absmax, k, *, status=None):
+    """Sort-and-cluster on the device: (cluster id per channel int32, scales float32[k])."""
+    _dev_check(absmax)
+    n = absmax.numel()
+    cl = torch.empty(n, dtype=torch.int32, device=absmax.device)
+    sc = torch.empty(k, dtype=torch.float32, device=absmax.device)
+    N.ssmq_cluster_by_absmax(absmax, n, k, cl, sc, status=status)
+    return cl, sc
+
+
+def _pct_workspace(device, workspace):
+    nb = N.ssmq_percentile_workspace_size()
+    if workspace is None:
+        workspace = torch.empty(nb + 256, dtype=torch.uint8, device=device)
+    base = workspace.data_ptr()
+    return (base + 255) // 256 * 256, nb
+
+
+def percentile_abs(src, q, *, out=None, workspace=None):
+    """Percentiles (linear interpolation) of |src| over its finite elements."""
+    _dev_check(src)
+    q = [float(v) for v in (q if hasattr(q, "__len__") else [q])]
+    o = out if out is not None else torch.empty(len(q), dtype=torch.float32, device=src.device)
+    wptr, nb = _pct_workspace(src.device, workspace)
+    N.ssmq_percentile_abs(src, src.numel(), q, o, wptr, nb)
+    return o
+
+
+def softedge_calibrate(src, thresholds=None, *, q_lo=5.0, q_hi=99.9, alpha=1.0, workspace=None):
+    """Soft-edge parameters {scale, lo, hi} (float32[3], updated in place):
+    percentiles of |src|, blended into the running values when alpha < 1."""
+    _dev_check(src)
+    thr = thresholds if thresholds is not None else torch.zeros(3, dtype=torch.float32,
+                                                                  device=src.device)
+    wptr, nb = _pct_workspace(src.device, workspace)
+    N.ssmq_softedge_calibrate(src, src.numel(), q_lo, q_hi, alpha, thr, wptr, nb)
+    return thr

@@ -71,6 +71,19 @@ ssmq_status check_yq(const int8_t* y_q, const int32_t* y_group, const float* y_s
   return SSMQ_OK;
 }
 
+ssmq_status check_pct(const void* src, ssmq_dtype dtype, int64_t n, void* workspace,
+                      size_t ws_bytes, const char* fn) {
+  REQUIRE(dtype == SSMQ_F32 || dtype == SSMQ_F16, SSMQ_ERR_INVALID_ARG, "%s: bad dtype", fn);
+  REQUIRE(n >= 0, SSMQ_ERR_INVALID_ARG, "%s: negative size", fn);
+  if (n > 0) REQUIRE(src != nullptr, SSMQ_ERR_INVALID_ARG, "%s: src is NULL", fn);
+  REQUIRE(workspace && ws_bytes >= ssmq::percentile_workspace_bytes(), SSMQ_ERR_INVALID_ARG,
+          "%s: workspace of %zu bytes required (got %zu)", fn,
+          ssmq::percentile_workspace_bytes(), ws_bytes);
+  REQUIRE((reinterpret_cast<uintptr_t>(workspace) & 255u) == 0, SSMQ_ERR_ALIGNMENT,
+          "%s: workspace must be 256-byte aligned", fn);
+  return SSMQ_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -121,6 +134,74 @@ ssmq_status ssmq_softedge_encode(const void* src, ssmq_dtype dtype, int64_t n, f
   if (injected(fn)) return fail(SSMQ_ERR_CUDA, "%s: injected launch failure", fn);
   return finish(ssmq::launch_softedge_encode(src, dtype == SSMQ_F16, n, scale, thr_lo, thr_hi,
                                              log2_ratio, codes, status, (cudaStream_t)stream),
+                fn);
+}
+
+ssmq_status ssmq_group_absmax(const void* src, ssmq_dtype dtype, int64_t outer, int64_t mid,
+                              int64_t inner, const int32_t* group_of_mid, int32_t n_groups,
+                              float* absmax, uint32_t* status, void* stream) {
+  const char* fn = "ssmq_group_absmax";
+  REQUIRE(dtype == SSMQ_F32 || dtype == SSMQ_F16, SSMQ_ERR_INVALID_ARG, "%s: bad dtype %d", fn,
+          (int)dtype);
+  REQUIRE(outer >= 0 && mid >= 0 && inner >= 0, SSMQ_ERR_INVALID_ARG, "%s: negative size", fn);
+  REQUIRE(n_groups >= 1 && absmax, SSMQ_ERR_INVALID_ARG, "%s: need n_groups >= 1 and absmax", fn);
+  const int64_t n = outer * mid * inner;
+  if (n > 0) REQUIRE(src && group_of_mid, SSMQ_ERR_INVALID_ARG, "%s: NULL tensor", fn);
+  REQUIRE(aligned16(src), SSMQ_ERR_ALIGNMENT, "%s: src must be 16-byte aligned", fn);
+  if (injected(fn)) return fail(SSMQ_ERR_CUDA, "%s: injected launch failure", fn);
+  return finish(ssmq::launch_group_absmax(src, dtype == SSMQ_F16, outer, mid, inner,
+                                          group_of_mid, n_groups, absmax, status,
+                                          (cudaStream_t)stream),
+                fn);
+}
+
+ssmq_status ssmq_cluster_by_absmax(const float* absmax, int64_t n, int32_t k, int32_t* cluster_of,
+                                   float* scales, uint32_t* status, void* stream) {
+  const char* fn = "ssmq_cluster_by_absmax";
+  REQUIRE(n >= 1 && k >= 1 && k <= n, SSMQ_ERR_INVALID_ARG, "%s: need 1 <= k <= n", fn);
+  REQUIRE(n <= 65536, SSMQ_ERR_UNSUPPORTED, "%s: n > 65536 channels", fn);
+  REQUIRE(absmax && cluster_of && scales, SSMQ_ERR_INVALID_ARG, "%s: NULL tensor", fn);
+  if (injected(fn)) return fail(SSMQ_ERR_CUDA, "%s: injected launch failure", fn);
+  return finish(ssmq::launch_cluster_by_absmax(absmax, (int)n, k, cluster_of, scales, status,
+                                               (cudaStream_t)stream),
+                fn);
+}
+
+size_t ssmq_percentile_workspace_size(void) { return ssmq::percentile_workspace_bytes(); }
+
+
+ssmq_status ssmq_percentile_abs(const void* src, ssmq_dtype dtype, int64_t n, const double* q,
+                                int32_t nq, float* out, void* workspace, size_t ws_bytes,
+                                void* stream) {
+  const char* fn = "ssmq_percentile_abs";
+  const ssmq_status c = check_pct(src, dtype, n, workspace, ws_bytes, fn);
+  if (c != SSMQ_OK) return c;
+  REQUIRE(q && out && nq >= 1 && nq <= ssmq::percentile_max_q(), SSMQ_ERR_INVALID_ARG,
+          "%s: need 1 <= nq <= %d percentiles and out", fn, ssmq::percentile_max_q());
+  for (int i = 0; i < nq; ++i)
+    REQUIRE(q[i] >= 0.0 && q[i] <= 100.0, SSMQ_ERR_INVALID_ARG,
+            "%s: percentile %d outside [0, 100]", fn, i);
+  if (injected(fn)) return fail(SSMQ_ERR_CUDA, "%s: injected launch failure", fn);
+  return finish(ssmq::launch_percentile_abs(src, dtype == SSMQ_F16, n, q, nq, out, nullptr, 1.0f,
+                                            workspace, (cudaStream_t)stream),
+                fn);
+}
+
+ssmq_status ssmq_softedge_calibrate(const void* src, ssmq_dtype dtype, int64_t n, double q_lo,
+                                    double q_hi, float alpha, float* thresholds, void* workspace,
+                                    size_t ws_bytes, void* stream) {
+  const char* fn = "ssmq_softedge_calibrate";
+  const ssmq_status c = check_pct(src, dtype, n, workspace, ws_bytes, fn);
+  if (c != SSMQ_OK) return c;
+  REQUIRE(thresholds != nullptr, SSMQ_ERR_INVALID_ARG, "%s: thresholds is NULL", fn);
+  REQUIRE(q_lo >= 0.0 && q_lo <= q_hi && q_hi <= 100.0, SSMQ_ERR_INVALID_ARG,
+          "%s: need 0 <= q_lo <= q_hi <= 100", fn);
+  REQUIRE(alpha > 0.0f && alpha <= 1.0f, SSMQ_ERR_INVALID_ARG, "%s: alpha must be in (0, 1]", fn);
+  if (injected(fn)) return fail(SSMQ_ERR_CUDA, "%s: injected launch failure", fn);
+  const double q[2] = {q_lo, q_hi};
+  return finish(ssmq::launch_percentile_abs(src, dtype == SSMQ_F16, n, q, 2,
+                                            ssmq::percentile_scratch_out(workspace), thresholds,
+                                            alpha, workspace, (cudaStream_t)stream),
                 fn);
 }
 

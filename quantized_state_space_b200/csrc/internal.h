@@ -25,6 +25,18 @@ cudaError_t launch_selective_scan(const ssmq_scan_args& a, cudaStream_t st);
 cudaError_t launch_state_update(const ssmq_decode_args& a, cudaStream_t st);
 cudaError_t launch_m1_state_update(const ssmq_m1_decode_args& a, cudaStream_t st);
 
+cudaError_t launch_group_absmax(const void* src, bool f16, int64_t outer, int64_t mid,
+                                int64_t inner, const int32_t* gmap, int32_t n_groups,
+                                float* absmax, uint32_t* status, cudaStream_t st);
+cudaError_t launch_cluster_by_absmax(const float* absmax, int n, int k, int32_t* cluster_of,
+                                     float* scales, uint32_t* status, cudaStream_t st);
+size_t percentile_workspace_bytes();
+float* percentile_scratch_out(void* ws);
+int percentile_max_q();
+cudaError_t launch_percentile_abs(const void* src, bool f16, int64_t n, const double* q, int nq,
+                                  float* out, float* thr, float alpha, void* workspace,
+                                  cudaStream_t st);
+
 size_t ssd_workspace_bytes(const ssmq_ssd_args& a);
 cudaError_t launch_ssd(const ssmq_ssd_args& a, void* ws, cudaStream_t st);
 

@@ -341,6 +341,30 @@ cudaError_t quantize_t(const void* src, Idx n, Idx mid, Idx inner, const int32_t
   return cudaGetLastError();
 }
 
+// exact max |v| of every group (finite elements), no scale division
+template <bool kF16, int kPath, typename Idx>
+cudaError_t group_absmax_t(const void* src, Idx n, Idx mid, Idx inner, const int32_t* gmap,
+                           int32_t n_groups, float* absmax, uint32_t* status, cudaStream_t st) {
+  constexpr size_t pipe = (size_t)acc_smem_offset<kF16>();
+  const Geo<Idx> geo = make_geo(mid, inner);
+  cudaError_t e = cudaMemsetAsync(absmax, 0, sizeof(float) * (size_t)n_groups, st);
+  if (e != cudaSuccess || n == 0) return e;
+  const int use_smem = n_groups <= 8192;
+  return launch_stream(absmax_kernel<kF16, kPath, Idx>, (uint64_t)n,
+                       pipe + (use_smem ? n_groups * sizeof(unsigned) : 0), st, src, n, geo, gmap,
+                       n_groups, reinterpret_cast<unsigned*>(absmax), status, use_smem);
+}
+
+template <bool kF16, typename Idx>
+cudaError_t group_absmax_p(const void* src, Idx n, Idx mid, Idx inner, const int32_t* gmap,
+                           int32_t n_groups, float* absmax, uint32_t* status, cudaStream_t st) {
+  if (inner % kVec == 0)
+    return group_absmax_t<kF16, kPathRow, Idx>(src, n, mid, inner, gmap, n_groups, absmax, status, st);
+  if (inner == 1 && mid % kVec == 0)
+    return group_absmax_t<kF16, kPathCol, Idx>(src, n, mid, inner, gmap, n_groups, absmax, status, st);
+  return group_absmax_t<kF16, kPathGen, Idx>(src, n, mid, inner, gmap, n_groups, absmax, status, st);
+}
+
 template <bool kF16, typename Idx>
 cudaError_t quantize_p(const void* src, Idx n, Idx mid, Idx inner, const int32_t* gmap,
                        int32_t n_groups, bool absmax, float* scales, int8_t* q,
@@ -459,6 +483,21 @@ cudaError_t launch_quantize(const void* src, bool f16, int64_t outer, int64_t mi
                                           absmax, scales, q, status, st)
              : quantize_p<false, uint64_t>(src, n, (uint64_t)mid, (uint64_t)inner, gmap, n_groups,
                                            absmax, scales, q, status, st);
+}
+
+cudaError_t launch_group_absmax(const void* src, bool f16, int64_t outer, int64_t mid,
+                                int64_t inner, const int32_t* gmap, int32_t n_groups,
+                                float* absmax, uint32_t* status, cudaStream_t st) {
+  const uint64_t n = (uint64_t)outer * (uint64_t)mid * (uint64_t)inner;
+  if (n + 64 < (1ull << 32)) {
+    const uint32_t n32 = (uint32_t)n, m32 = (uint32_t)mid, i32 = (uint32_t)inner;
+    return f16 ? group_absmax_p<true, uint32_t>(src, n32, m32, i32, gmap, n_groups, absmax, status, st)
+               : group_absmax_p<false, uint32_t>(src, n32, m32, i32, gmap, n_groups, absmax, status, st);
+  }
+  return f16 ? group_absmax_p<true, uint64_t>(src, n, (uint64_t)mid, (uint64_t)inner, gmap, n_groups,
+                                              absmax, status, st)
+             : group_absmax_p<false, uint64_t>(src, n, (uint64_t)mid, (uint64_t)inner, gmap,
+                                               n_groups, absmax, status, st);
 }
 
 cudaError_t launch_softedge_encode(const void* src, bool f16, int64_t n, float scale, float lo,

@@ -94,3 +94,34 @@ def test_ssd_head_clusters():
     assert grp.shape == (64,)
     # every channel of a head shares its cluster
     assert np.all(grp.reshape(16, 4) == grp.reshape(16, 4)[:, :1])
+
+
+# ---- threshold update (Quamba-SE write-up 4.1), oracle pins ------------------
+
+def test_oracle_softedge_thresholds_alpha_one_equals_host_params(orc):
+    """alpha = 1: the thresholds are the percentiles, as the host calibration
+    (numpy-pinned percentiles) computes them."""
+    rng = np.random.default_rng(41)
+    x = (rng.standard_t(3, size=50000)).astype(np.float16)
+    s, lo, hi = calibrate.softedge_params(x)
+    thr = orc.softedge_thresholds(x, 5.0, 99.9, 1.0, previous=(7.0, 7.0, 7.0))
+    assert thr.tolist() == [float(s), float(lo), float(hi)]
+
+
+def test_oracle_softedge_thresholds_worked_blend(orc):
+    """A worked example: every |v| equals 2, so both percentiles are 2; with
+    alpha 1/2 and previous (lo, hi) = (4, 6) the blend gives exactly (3, 4) and
+    the scale fl32(4 / 63)."""
+    x = np.array([2.0, -2.0, 2.0, -2.0], dtype=np.float32)
+    thr = orc.softedge_thresholds(x, 5.0, 99.9, 0.5, previous=(0.0, 4.0, 6.0))
+    assert thr[1] == 3.0 and thr[2] == 4.0
+    assert thr[0] == np.float32(4.0 / 63.0)
+    # alpha = 0.1 of the page, previous 0: 0.1 * 2 rounded once to binary32
+    thr = orc.softedge_thresholds(x, 5.0, 99.9, float(np.float32(0.1)), previous=(0, 0, 0))
+    assert thr[1] == np.float32(float(np.float32(0.1)) * 2.0)
+
+
+def test_oracle_softedge_thresholds_ignores_nonfinite(orc):
+    x = np.array([1.0, np.nan, 3.0, np.inf, -2.0], dtype=np.float32)
+    thr = orc.softedge_thresholds(x, 0.0, 100.0, 1.0)
+    assert thr[1] == 1.0 and thr[2] == 3.0
