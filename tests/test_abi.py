@@ -208,3 +208,29 @@ def test_m1_decode_validation(L):
     assert S(A=None) == N.ERR_INVALID_ARG
     assert S(A=FAKE + 4) == N.ERR_ALIGNMENT
     assert S(batch=0) == N.OK
+
+
+def test_calibration_validation(L):
+    """Device calibration calls reject bad arguments before any launch."""
+    F = N.F16
+    assert L.ssmq_group_absmax(FAKE, 7, 2, 3, 4, FAKE, 3, FAKE, None, None) == N.ERR_INVALID_ARG
+    assert L.ssmq_group_absmax(FAKE, F, 2, 3, 4, FAKE, 0, FAKE, None, None) == N.ERR_INVALID_ARG
+    assert L.ssmq_group_absmax(FAKE + 2, F, 2, 3, 4, FAKE, 3, FAKE, None, None) == N.ERR_ALIGNMENT
+    assert L.ssmq_cluster_by_absmax(FAKE, 10, 11, FAKE, FAKE, None, None) == N.ERR_INVALID_ARG
+    assert L.ssmq_cluster_by_absmax(FAKE, 10, 0, FAKE, FAKE, None, None) == N.ERR_INVALID_ARG
+    assert L.ssmq_cluster_by_absmax(FAKE, 70000, 8, FAKE, FAKE, None, None) == N.ERR_UNSUPPORTED
+    nb = L.ssmq_percentile_workspace_size()
+    assert nb >= 32768 * 4
+    q = (C.c_double * 2)(5.0, 99.9)
+    P = lambda **kw: L.ssmq_percentile_abs(kw.get("src", FAKE), F, 100, kw.get("q", q),
+                                           kw.get("nq", 2), FAKE, kw.get("ws", FAKE),
+                                           kw.get("nb", nb), None)
+    assert P(nb=nb - 1) == N.ERR_INVALID_ARG
+    assert P(ws=FAKE + 16) == N.ERR_ALIGNMENT
+    assert P(nq=0) == N.ERR_INVALID_ARG
+    assert P(q=(C.c_double * 2)(5.0, 100.5)) == N.ERR_INVALID_ARG
+    assert P(src=None) == N.ERR_INVALID_ARG
+    S = lambda lo, hi, a: L.ssmq_softedge_calibrate(FAKE, F, 100, lo, hi, a, FAKE, FAKE, nb, None)
+    assert S(5.0, 99.9, 0.0) == N.ERR_INVALID_ARG
+    assert S(5.0, 99.9, 1.5) == N.ERR_INVALID_ARG
+    assert S(99.9, 5.0, 0.1) == N.ERR_INVALID_ARG
