@@ -198,6 +198,22 @@ ssmq_status ssmq_softedge_calibrate(const void* src, ssmq_dtype dtype, int64_t n
                                     double q_hi, float alpha, float* thresholds,
                                     void* workspace, size_t ws_bytes, void* stream);
 
+/*
+ * Allocation-free variants of the two percentile calls: the same computation
+ * and results, with the library's own scratch instead of a caller workspace --
+ * a static device array (one per device, found with cudaGetSymbolAddress for
+ * the current device).  Nothing is allocated or freed.  Calls that use the
+ * scratch of one device must not overlap (issue them on one stream, or
+ * synchronise between them).  SSMQ_ERR_UNSUPPORTED if the scratch a call
+ * needs exceeds the static array.  The pages have no counterpart: this is a
+ * deployment convenience of this library, not part of the method.
+ */
+ssmq_status ssmq_percentile_abs_noalloc(const void* src, ssmq_dtype dtype, int64_t n,
+                                        const double* q, int32_t nq, float* out, void* stream);
+ssmq_status ssmq_softedge_calibrate_noalloc(const void* src, ssmq_dtype dtype, int64_t n,
+                                            double q_lo, double q_hi, float alpha,
+                                            float* thresholds, void* stream);
+
 /* ------------------------------------------------------------------------ */
 /* Mamba-1 diagonal selective scan                                           */
 /* ------------------------------------------------------------------------ */

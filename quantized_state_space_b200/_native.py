@@ -89,6 +89,10 @@ SIGNATURES = {
                                    C.c_size_t, _vp]),
     "ssmq_softedge_calibrate": (_i32, [_vp, _i32, _i64, C.c_double, C.c_double, _f32, _vp, _vp,
                                        C.c_size_t, _vp]),
+    "ssmq_percentile_abs_noalloc": (_i32, [_vp, _i32, _i64, C.POINTER(C.c_double), _i32, _vp,
+                                           _vp]),
+    "ssmq_softedge_calibrate_noalloc": (_i32, [_vp, _i32, _i64, C.c_double, C.c_double, _f32,
+                                               _vp, _vp]),
     "ssmq_last_error": (C.c_char_p, []),
     "ssmq_version": (_i32, []),
 }
@@ -236,3 +240,16 @@ def ssmq_softedge_calibrate(src, n, q_lo, q_hi, alpha, thresholds, workspace, ws
     _check(lib().ssmq_softedge_calibrate(ptr(src), _dtype_of(src, dtype), n, float(q_lo),
                                          float(q_hi), float(alpha), ptr(thresholds),
                                          ptr(workspace), ws_bytes, _stream(stream)))
+
+
+def ssmq_percentile_abs_noalloc(src, n, q, out, stream=None, dtype=None):
+    qa = (C.c_double * len(q))(*[float(v) for v in q])
+    _check(lib().ssmq_percentile_abs_noalloc(ptr(src), _dtype_of(src, dtype), n, qa, len(q),
+                                             ptr(out), _stream(stream)))
+
+
+def ssmq_softedge_calibrate_noalloc(src, n, q_lo, q_hi, alpha, thresholds, stream=None,
+                                    dtype=None):
+    _check(lib().ssmq_softedge_calibrate_noalloc(ptr(src), _dtype_of(src, dtype), n, float(q_lo),
+                                                 float(q_hi), float(alpha), ptr(thresholds),
+                                                 _stream(stream)))

@@ -71,11 +71,14 @@ ssmq_status check_yq(const int8_t* y_q, const int32_t* y_group, const float* y_s
   return SSMQ_OK;
 }
 
-ssmq_status check_pct(const void* src, ssmq_dtype dtype, int64_t n, void* workspace,
-                      size_t ws_bytes, const char* fn) {
+ssmq_status check_src(const void* src, ssmq_dtype dtype, int64_t n, const char* fn) {
   REQUIRE(dtype == SSMQ_F32 || dtype == SSMQ_F16, SSMQ_ERR_INVALID_ARG, "%s: bad dtype", fn);
   REQUIRE(n >= 0, SSMQ_ERR_INVALID_ARG, "%s: negative size", fn);
   if (n > 0) REQUIRE(src != nullptr, SSMQ_ERR_INVALID_ARG, "%s: src is NULL", fn);
+  return SSMQ_OK;
+}
+
+ssmq_status check_ws(void* workspace, size_t ws_bytes, const char* fn) {
   REQUIRE(workspace && ws_bytes >= ssmq::percentile_workspace_bytes(), SSMQ_ERR_INVALID_ARG,
           "%s: workspace of %zu bytes required (got %zu)", fn,
           ssmq::percentile_workspace_bytes(), ws_bytes);
@@ -83,6 +86,30 @@ ssmq_status check_pct(const void* src, ssmq_dtype dtype, int64_t n, void* worksp
           "%s: workspace must be 256-byte aligned", fn);
   return SSMQ_OK;
 }
+
+ssmq_status check_pct_q(const double* q, int32_t nq, const float* out, const char* fn) {
+  REQUIRE(q && out && nq >= 1 && nq <= ssmq::percentile_max_q(), SSMQ_ERR_INVALID_ARG,
+          "%s: need 1 <= nq <= %d percentiles and out", fn, ssmq::percentile_max_q());
+  for (int i = 0; i < nq; ++i)
+    REQUIRE(q[i] >= 0.0 && q[i] <= 100.0, SSMQ_ERR_INVALID_ARG,
+            "%s: percentile %d outside [0, 100]", fn, i);
+  return SSMQ_OK;
+}
+
+ssmq_status check_se_cal(double q_lo, double q_hi, float alpha, const float* thresholds,
+                         const char* fn) {
+  REQUIRE(thresholds != nullptr, SSMQ_ERR_INVALID_ARG, "%s: thresholds is NULL", fn);
+  REQUIRE(q_lo >= 0.0 && q_lo <= q_hi && q_hi <= 100.0, SSMQ_ERR_INVALID_ARG,
+          "%s: need 0 <= q_lo <= q_hi <= 100", fn);
+  REQUIRE(alpha > 0.0f && alpha <= 1.0f, SSMQ_ERR_INVALID_ARG, "%s: alpha must be in (0, 1]", fn);
+  return SSMQ_OK;
+}
+
+#define CHECK(call)                     \
+  do {                                  \
+    const ssmq_status s_ = (call);      \
+    if (s_ != SSMQ_OK) return s_;       \
+  } while (0)
 
 }  // namespace
 
@@ -174,13 +201,9 @@ ssmq_status ssmq_percentile_abs(const void* src, ssmq_dtype dtype, int64_t n, co
                                 int32_t nq, float* out, void* workspace, size_t ws_bytes,
                                 void* stream) {
   const char* fn = "ssmq_percentile_abs";
-  const ssmq_status c = check_pct(src, dtype, n, workspace, ws_bytes, fn);
-  if (c != SSMQ_OK) return c;
-  REQUIRE(q && out && nq >= 1 && nq <= ssmq::percentile_max_q(), SSMQ_ERR_INVALID_ARG,
-          "%s: need 1 <= nq <= %d percentiles and out", fn, ssmq::percentile_max_q());
-  for (int i = 0; i < nq; ++i)
-    REQUIRE(q[i] >= 0.0 && q[i] <= 100.0, SSMQ_ERR_INVALID_ARG,
-            "%s: percentile %d outside [0, 100]", fn, i);
+  CHECK(check_src(src, dtype, n, fn));
+  CHECK(check_pct_q(q, nq, out, fn));
+  CHECK(check_ws(workspace, ws_bytes, fn));
   if (injected(fn)) return fail(SSMQ_ERR_CUDA, "%s: injected launch failure", fn);
   return finish(ssmq::launch_percentile_abs(src, dtype == SSMQ_F16, n, q, nq, out, nullptr, 1.0f,
                                             workspace, (cudaStream_t)stream),
@@ -191,18 +214,51 @@ ssmq_status ssmq_softedge_calibrate(const void* src, ssmq_dtype dtype, int64_t n
                                     double q_hi, float alpha, float* thresholds, void* workspace,
                                     size_t ws_bytes, void* stream) {
   const char* fn = "ssmq_softedge_calibrate";
-  const ssmq_status c = check_pct(src, dtype, n, workspace, ws_bytes, fn);
-  if (c != SSMQ_OK) return c;
-  REQUIRE(thresholds != nullptr, SSMQ_ERR_INVALID_ARG, "%s: thresholds is NULL", fn);
-  REQUIRE(q_lo >= 0.0 && q_lo <= q_hi && q_hi <= 100.0, SSMQ_ERR_INVALID_ARG,
-          "%s: need 0 <= q_lo <= q_hi <= 100", fn);
-  REQUIRE(alpha > 0.0f && alpha <= 1.0f, SSMQ_ERR_INVALID_ARG, "%s: alpha must be in (0, 1]", fn);
+  CHECK(check_src(src, dtype, n, fn));
+  CHECK(check_se_cal(q_lo, q_hi, alpha, thresholds, fn));
+  CHECK(check_ws(workspace, ws_bytes, fn));
   if (injected(fn)) return fail(SSMQ_ERR_CUDA, "%s: injected launch failure", fn);
   const double q[2] = {q_lo, q_hi};
   return finish(ssmq::launch_percentile_abs(src, dtype == SSMQ_F16, n, q, 2,
                                             ssmq::percentile_scratch_out(workspace), thresholds,
                                             alpha, workspace, (cudaStream_t)stream),
                 fn);
+}
+
+namespace {
+// the library's static scratch of the current device, or an error status
+ssmq_status static_scratch(void** ws, const char* fn) {
+  cudaError_t e;
+  const size_t need = ssmq::percentile_workspace_bytes();
+  *ws = ssmq::percentile_static_scratch(need, &e);
+  REQUIRE(e == cudaSuccess, SSMQ_ERR_CUDA, "%s: %s", fn, cudaGetErrorString(e));
+  REQUIRE(*ws != nullptr, SSMQ_ERR_UNSUPPORTED, "%s: %zu bytes of scratch exceed the static array",
+          fn, need);
+  return SSMQ_OK;
+}
+}  // namespace
+
+ssmq_status ssmq_percentile_abs_noalloc(const void* src, ssmq_dtype dtype, int64_t n,
+                                        const double* q, int32_t nq, float* out, void* stream) {
+  const char* fn = "ssmq_percentile_abs_noalloc";
+  CHECK(check_src(src, dtype, n, fn));  // argument errors before any device call
+  CHECK(check_pct_q(q, nq, out, fn));
+  void* ws = nullptr;
+  CHECK(static_scratch(&ws, fn));
+  return ssmq_percentile_abs(src, dtype, n, q, nq, out, ws, ssmq::percentile_workspace_bytes(),
+                             stream);
+}
+
+ssmq_status ssmq_softedge_calibrate_noalloc(const void* src, ssmq_dtype dtype, int64_t n,
+                                            double q_lo, double q_hi, float alpha,
+                                            float* thresholds, void* stream) {
+  const char* fn = "ssmq_softedge_calibrate_noalloc";
+  CHECK(check_src(src, dtype, n, fn));
+  CHECK(check_se_cal(q_lo, q_hi, alpha, thresholds, fn));
+  void* ws = nullptr;
+  CHECK(static_scratch(&ws, fn));
+  return ssmq_softedge_calibrate(src, dtype, n, q_lo, q_hi, alpha, thresholds, ws,
+                                 ssmq::percentile_workspace_bytes(), stream);
 }
 
 ssmq_status ssmq_softedge_decode(const uint8_t* codes, int64_t n, float scale, int32_t log2_ratio,

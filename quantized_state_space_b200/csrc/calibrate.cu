@@ -291,7 +291,20 @@ cudaError_t percentile_t(const void* src, int64_t n, const double* q, int nq, fl
   return cudaGetLastError();
 }
 
+// Scratch of the allocation-free entry points: a static device array (module
+// globals exist once per device context), sized exactly for one call.
+constexpr size_t kPctWsBytes = (sizeof(PctWs) + 255) / 256 * 256 + 256;
+__device__ __align__(256) uint8_t g_pct_scratch[kPctWsBytes];
+
 }  // namespace
+
+void* percentile_static_scratch(size_t need, cudaError_t* err) {
+  *err = cudaSuccess;
+  if (need > kPctWsBytes) return nullptr;  // caller reports the size mismatch
+  void* p = nullptr;
+  *err = cudaGetSymbolAddress(&p, g_pct_scratch);  // the current device's copy
+  return *err == cudaSuccess ? p : nullptr;
+}
 
 // workspace: the histograms and control block, then 256 bytes for the
 // percentile values of the soft-edge update

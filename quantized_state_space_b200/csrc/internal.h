@@ -32,6 +32,7 @@ cudaError_t launch_cluster_by_absmax(const float* absmax, int n, int k, int32_t*
                                      float* scales, uint32_t* status, cudaStream_t st);
 size_t percentile_workspace_bytes();
 float* percentile_scratch_out(void* ws);
+void* percentile_static_scratch(size_t need, cudaError_t* err);
 int percentile_max_q();
 cudaError_t launch_percentile_abs(const void* src, bool f16, int64_t n, const double* q, int nq,
                                   float* out, float* thr, float alpha, void* workspace,
