@@ -401,7 +401,7 @@ def run_ours(args):
             if not only or "m130m_int8_y" in only:
                 out["forms"]["m130m_int8_y"] = form_int8_y(torch, layer)
             out["forms"].update(run_forms(dev, pk, out["clocks"].get("sm_max_mhz") or
-                                          pk["sm_max_mhz"], only=only))
+                                          pk["sm_max_mhz"], only=only, layer=layer))
         print(json.dumps(out), flush=True)
 
 
@@ -658,9 +658,45 @@ def form_ssd(torch, dev, pk):
                          "traffic": measured_traffic("ssd_kernel")}}
 
 
-def run_forms(dev, pk, mhz, only=None):
+def form_calibrate(torch, dev, pk, layer):
+    """Device calibration: per-channel maxima of the m130m x and their
+    sort-and-cluster (the offline step, on the GPU), and the soft-edge
+    thresholds (5th / 99.9th percentiles of |x|) of the softedge x."""
+    from quantized_state_space_b200 import api, synth
+    b, d, L, k = layer.b, layer.d, layer.L, layer.k
+    ident = torch.arange(d, dtype=torch.int32, device=dev)
+    amax = torch.empty(d, dtype=torch.float32, device=dev)
+    t_max = _timed(torch, lambda: api.group_absmax(layer.x, b, d, L, ident, d, out=amax), 10)
+    t_cl = _timed(torch, lambda: api.cluster_by_absmax(amax, k), 10)
+    dm, raw = synth.workload_inputs("softedge")
+    x = torch.from_numpy(raw["x"]).to(dev)
+    del raw
+    nb = api.N.ssmq_percentile_workspace_size()
+    ws = torch.empty(nb + 256, dtype=torch.uint8, device=dev)
+    thr = torch.zeros(3, dtype=torch.float32, device=dev)
+    t_pct = _timed(torch, lambda: api.softedge_calibrate(x, thr, workspace=ws), 5)
+    bx = layer.x.numel() * 2
+    bs = x.numel() * 2
+    return {"workload": "m130m x channel maxima + sort-and-cluster (k %d); softedge x "
+                        "thresholds (%d M binary16 elements)" % (k, x.numel() // 10**6),
+            "absmax_ms": round(t_max * 1e3, 4),
+            "absmax_hbm": {"achieved": round(bx / t_max / 1e9, 1), "peak": pk["hbm_gbs"],
+                           "unit": "GB/s", "frac": round(bx / t_max / 1e9 / pk["hbm_gbs"], 4)},
+            "cluster_ms": round(t_cl * 1e3, 4),
+            "thresholds_ms": round(t_pct * 1e3, 4),
+            "thresholds_hbm": {"achieved": round(bs / t_pct / 1e9, 1), "peak": pk["hbm_gbs"],
+                               "unit": "GB/s", "frac": round(bs / t_pct / 1e9 / pk["hbm_gbs"], 4)}}
+
+
+def run_forms(dev, pk, mhz, only=None, layer=None):
     import torch
     out = {}
+    if layer is not None and (not only or "calibrate" in only):
+        try:
+            out["calibrate"] = form_calibrate(torch, dev, pk, layer)
+        except Exception as e:
+            out["calibrate"] = {"error": "%s: %s" % (type(e).__name__, e)}
+        torch.cuda.empty_cache()
     for name, fn in (("ssd27b", lambda: form_ssd(torch, dev, pk)),
                      ("decode8b", lambda: form_decode(torch, dev, pk)),
                      ("softedge", lambda: form_softedge(torch, dev, pk, mhz))):
@@ -769,7 +805,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-forms", action="store_true")
-    ap.add_argument("--forms", default="", help="comma list of m130m_other_x_path,m130m_int8_y,ssd27b,decode8b,softedge")
+    ap.add_argument("--forms", default="", help="comma list of m130m_other_x_path,m130m_int8_y,calibrate,ssd27b,decode8b,"
+                         "softedge")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--fused", action="store_true",
                     help="headline step with binary16 x encoded inside the scan (byte-identical "

@@ -1,0 +1,81 @@
+"""The operand-rounding plan of the SSD tensor-core kernel, emulated in numpy
+against the exact recurrence (SSDi8 abstract: element-wise products kept
+apart from the matrix products).  binary16 MMA operands: C' = fl16(c fl16(w'))
+with w' = sC sB / max; M row-normalised by a power of two and rounded to
+binary16; the Y_off state operand one normalised binary16 value carrying
+sC / w'; the w X operand of the state update split into binary16 high part
+and residual; fp32 accumulation (emulated in double).  The y error and the
+final-state error must sit inside the GPU tolerances (2e-3 of max |y| and
+1e-4 relative L2) with margin, and a plain bf16 operand plan must not."""
+import numpy as np
+
+
+def f16(a):
+    return np.asarray(a, np.float64).astype(np.float16).astype(np.float64)
+
+
+def bf16(a):
+    u = np.asarray(a, np.float32).view(np.uint32).astype(np.uint64)
+    r = ((u + 0x7FFF + ((u >> 16) & 1)) >> 16) << 16
+    return r.astype(np.uint32).view(np.float32).astype(np.float64)
+
+
+def p2(m):
+    """power of two putting max |m| into [2^14, 2^15)"""
+    m = np.max(np.abs(m))
+    return 1.0 if m == 0 else 2.0 ** -(int(np.floor(np.log2(m))) - 14)
+
+
+def run(plan, seed, L=768, P=32, N=64, Q=128):
+    rng = np.random.default_rng(seed)
+    A = -np.exp(rng.uniform(0, np.log(16)))
+    delta = np.logaddexp(0, rng.standard_normal(L) * 0.5 - 4)
+    sx = 5 / 127
+    sB = rng.uniform(0.5, 1.5, N) * 5 / 127
+    sC = rng.uniform(0.5, 1.5, N) * 5 / 127
+    Xq = np.clip(np.rint(rng.standard_normal((L, P)) / sx), -127, 127)
+    Bq = np.clip(np.rint(rng.standard_normal((L, N)) / sB), -127, 127)
+    Cq = np.clip(np.rint(rng.standard_normal((L, N)) / sC), -127, 127)
+    x, Bv, Cv = Xq * sx, Bq * sB, Cq * sC
+    h = np.zeros((P, N))
+    y = np.zeros((L, P))
+    for t in range(L):
+        h = np.exp(delta[t] * A) * h + delta[t] * np.outer(x[t], Bv[t])
+        y[t] = h @ Cv[t]
+    rnd = f16 if plan == "f16" else bf16
+    w = sC * sB
+    wmax = w.max()
+    wh = rnd(w / wmax)
+    Cp = rnd(Cq * wh[None, :])
+    hk = np.zeros((N, P))
+    yk = np.zeros((L, P))
+    for c0 in range(0, L, Q):
+        sl = slice(c0, c0 + Q)
+        S = np.cumsum(delta[sl] * A)
+        CB = Cp[sl] @ Bq[sl].T
+        M = np.tril(CB * np.exp(S[:, None] - S[None, :]) * delta[sl][None, :]) * wmax
+        rs = np.array([p2(r) for r in M])
+        Yd = (rnd(M * rs[:, None]) @ Xq[sl]) / rs[:, None]
+        op = hk * (sC / wh)[:, None]
+        sc = p2(op)
+        Yo = (Cp[sl] @ rnd(op * sc)) / sc
+        yk[sl] = Yd * sx + np.exp(S)[:, None] * Yo
+        wS = np.exp(S[-1] - S) * delta[sl]
+        v = wS[:, None] * Xq[sl]
+        hi = rnd(v)
+        lo = rnd(v - hi)
+        hk = np.exp(S[-1]) * hk + (sB[:, None] * sx) * (Bq[sl].T @ (hi + lo))
+    ey = np.max(np.abs(f16(yk) - y)) / np.max(np.abs(y))
+    es = np.linalg.norm(hk.T - h) / np.linalg.norm(h)
+    return ey, es
+
+
+def test_f16_plan_inside_tolerances():
+    for seed in range(3):
+        ey, es = run("f16", seed)
+        assert ey < 1.0e-3 and es < 1e-6, (seed, ey, es)
+
+
+def test_bf16_plan_fails_y_tolerance():
+    worst = max(run("bf16", seed)[0] for seed in range(3))
+    assert worst > 2e-3
