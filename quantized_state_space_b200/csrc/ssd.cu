@@ -66,7 +66,9 @@ constexpr int F_DW = F_S2 + 2 * kQ;     // delta_s                             [
 constexpr int F_WX = F_DW + 2 * kQ;     // w_s = exp(S_last - S_s) delta_s      [2][128]
 constexpr int F_ES = F_WX + 2 * kQ;     // exp(S_t)                            [2][128]
 constexpr int F_CW = F_ES + 2 * kQ;     // exp(S_p(s) - S_s) d_s w_max, p(s) = s | 31  [2][128]
-constexpr int F_RS = F_CW + 2 * kQ;     // 2^e_t row scale of M                [128]
+constexpr int F_CD = F_CW + 2 * kQ;     // exp(S_m(s) - S_s) d_s w_max, m(s) = s & ~31  [2][128]
+constexpr int F_BS = F_CD + 2 * kQ;     // spread max - min of S (log2) per 32-step block  [2][4]
+constexpr int F_RS = F_BS + 8;          // 2^e_t row scale of M                [128]
 constexpr int F_RM = F_RS + kQ;         // row max quarters                    [4][128]
 constexpr int F_WH = F_RM + 4 * kQ;     // w'_n as binary16 pairs              [64]
 constexpr int F_HF = F_WH + kN / 2;     // sC_n / w'_n (state operand factor)  [128]
@@ -210,10 +212,20 @@ __device__ __forceinline__ void tile_factors(float* F, int fb, int ql, const flo
   const float off = ex - run;
   const float s_last = __shfl_sync(0xffffffffu, ex, 31);
   float wmx = 0.0f;
-  // S at the end of this lane's 32-step column block (lane 8 b + 7 holds it)
+  // S at the end and at the start of this lane's 32-step block (lanes 8 b + 7
+  // and 8 b hold them), and the spread of S over the block
   const float s_blk = __shfl_sync(0xffffffffu, sc[3] + off, lane | 7);
-  float4 s2v, dwv, wxv, esv, cwv;
-  float* o4[5] = {&s2v.x, &dwv.x, &wxv.x, &esv.x, &cwv.x};
+  const float s_beg = __shfl_sync(0xffffffffu, sc[0] + off, lane & ~7);
+  float smax = fmaxf(fmaxf(sc[0], sc[1]), fmaxf(sc[2], sc[3])) + off;
+  float smin = fminf(fminf(sc[0], sc[1]), fminf(sc[2], sc[3])) + off;
+#pragma unroll
+  for (int o = 4; o >= 1; o >>= 1) {
+    smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, o));
+    smin = fminf(smin, __shfl_xor_sync(0xffffffffu, smin, o));
+  }
+  if ((lane & 7) == 0) F[F_BS + fb * 4 + (lane >> 3)] = smax - smin;
+  float4 s2v, dwv, wxv, esv, cwv, cdv;
+  float* o4[6] = {&s2v.x, &dwv.x, &wxv.x, &esv.x, &cwv.x, &cdv.x};
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const float s2 = sc[i] + off;
@@ -223,6 +235,7 @@ __device__ __forceinline__ void tile_factors(float* F, int fb, int ql, const flo
     o4[2][i] = w;
     o4[3][i] = ex2_sfu(s2);
     o4[4][i] = ex2_sfu(s_blk - s2) * dl[i] * wmax;
+    o4[5][i] = ex2_sfu(s_beg - s2) * dl[i] * wmax;
     wmx = fmaxf(wmx, w);
   }
   const int t0 = fb * kQ + 4 * lane;
@@ -231,6 +244,7 @@ __device__ __forceinline__ void tile_factors(float* F, int fb, int ql, const flo
   *reinterpret_cast<float4*>(F + F_WX + t0) = wxv;
   *reinterpret_cast<float4*>(F + F_ES + t0) = esv;
   *reinterpret_cast<float4*>(F + F_CW + t0) = cwv;
+  *reinterpret_cast<float4*>(F + F_CD + t0) = cdv;
 #pragma unroll
   for (int o = 16; o >= 1; o >>= 1) wmx = fmaxf(wmx, __shfl_xor_sync(0xffffffffu, wmx, o));
   if (lane == 0) {
@@ -361,6 +375,7 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_kernel(const SsdParams p) {
     const float* WX = F + F_WX + fb * kQ;
     const float* ES = F + F_ES + fb * kQ;
     const float* CW = F + F_CW + fb * kQ;
+    const float* CD = F + F_CD + fb * kQ;
     const float s_last = F[F_RED + 1];
     const int ex = norm_exp(F[F_RED] * p.x_bound);  // x_bound >= max |x_exact|
     const float xsc = pow2i(-ex);
@@ -539,6 +554,24 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_kernel(const SsdParams p) {
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               const float m = v[4 * j4 + e] * cw[e];
+              mv[4 * j4 + e] = m;
+              rmax = fmaxf(rmax, fabsf(m));
+            }
+          }
+          rmax *= rt;
+        } else if (F[F_BS + fb * 4 + q4] < 90.0f) {
+          // diagonal block, S spread below 2^90: exp(S_t - S_s) =
+          // exp(S_t - S_m) exp(S_m - S_s) with m the block's first step (both
+          // factors within 2^+-90, the products far from fp32 overflow)
+          const float sm = S2[s0];
+          rt = ex2_sfu(st - sm);
+#pragma unroll
+          for (int j4 = 0; j4 < 8; ++j4) {
+            const float4 c4 = *reinterpret_cast<const float4*>(CD + s0 + 4 * j4);
+            const float cd[4] = {c4.x, c4.y, c4.z, c4.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float m = s0 + 4 * j4 + e <= t ? v[4 * j4 + e] * cd[e] : 0.0f;
               mv[4 * j4 + e] = m;
               rmax = fmaxf(rmax, fabsf(m));
             }
