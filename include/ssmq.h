@@ -319,7 +319,10 @@ ssmq_status ssmq_selective_scan_w8(const ssmq_scan_args* args, void* stream);
  *            after rounding to binary16 (the bytes of ssmq_quantize_groups
  *            of the binary16 y)
  * workspace: device memory of at least ssmq_ssd_workspace_size(args) bytes,
- *   256-byte aligned, caller-owned, contents need not be initialised.
+ *   256-byte aligned, caller-owned, contents need not be initialised; it
+ *   receives the head-independent binary16 MMA operands (C scaled per state
+ *   group, B), 64 KB per (batch, group, 128-step tile), written once for all
+ *   heads of a group.
  * Supported: P == 64, N == 128, chunk in {64, 128, 256}, H % G == 0.  The
  * result is the recurrence's for every chunk length (the decomposition is
  * exact up to rounding); the kernel processes 128-step tiles.

@@ -25,18 +25,22 @@
 //     binary16 residual (two MMAs), with a tile-wide power-of-two
 //     normalisation, so the state increments carry ~22 bits; the state
 //     operand of MMA2 (which only feeds y) is one normalised binary16 value.
+// The head-independent operands (C' and B of a tile) are written once per
+// (batch, group) by ssd_operand_kernel into the workspace, in the layouts the
+// MMAs read, and bulk-copied into shared memory by each head's CTA.
 // One CTA (16 warps) owns one (batch, head) and walks the sequence in tiles;
 // warp 0 prepares the next tile's decay factors while the others finish the
 // current tile's outputs;
 // the fp32 state lives in registers (row n, 16 of the 64 p per thread: warp w
 // reads TMEM lanes 32 (w % 4).. and columns 16 (w / 4)..), accumulators in
-// TMEM (512 columns), operands in shared memory (209 KB, including the raw
-// int8 rows of the next tile, prefetched with cp.async during this one).
+// TMEM (512 columns), operands in shared memory (183 KB, including the raw
+// int8 x rows of the next tile, prefetched with cp.async during this one).
 // The chunk length of the interface only fixes where the decomposition
 // restarts; the result is the recurrence's for any length, so the kernel uses
 // 128-step tiles for every accepted chunk length.
 #include "common.cuh"
 #include "internal.h"
+#include "stream.cuh"
 #include "tc.cuh"
 
 namespace ssmq {
@@ -81,10 +85,12 @@ constexpr int F_RED = F_YOK + kP;       // reductions: w max, S_last, per-warp s
 constexpr int F_END = F_RED + 32;
 // raw int8 rows of the next tile, fetched with cp.async during this tile
 constexpr int OFF_RAW = (OFF_F + F_END * 4 + 127) / 128 * 128;
-constexpr int OFF_RC = OFF_RAW;                 // C codes [t][n]  16 KB
-constexpr int OFF_RB = OFF_RC + kQ * kN;        // B codes [t][n]  16 KB
-constexpr int OFF_RX = OFF_RB + kQ * kN;        // x codes [t][p]   8 KB
+constexpr int OFF_RX = OFF_RAW;                 // x codes [t][p]   8 KB
 constexpr int kSmemBytes = OFF_RX + kQ * kP;
+// operand blocks written by ssd_operand_kernel, per (batch, group, tile):
+// C' then B, each in the K-major canonical layout of OFF_C / OFF_B
+constexpr int kOpBlock = kQ * kN * 2;           // 32 KB
+constexpr int kOpTile = 2 * kOpBlock;           // 64 KB
 
 struct SsdParams {
   int64_t L, H, G;
@@ -115,6 +121,8 @@ struct SsdParams {
   int n_y_groups;
   float* h_final;
   uint32_t* status;
+  const uint8_t* ops;  // operand blocks (workspace)
+  int64_t ntiles;
 };
 
 // 2^e as an exact float for |e| < 126
@@ -161,19 +169,11 @@ __device__ __forceinline__ float block_max(float v, float* red, int tid) {
   return r;
 }
 
-// cp.async the int8 rows (C, B: N bytes; x: P bytes) of the tile starting
-// at t0 into the raw buffer; rows at or beyond ql are left as they are (the
-// staging masks them).
+// cp.async the x codes (P bytes per step) of the tile starting at t0 into the
+// raw buffer; rows at or beyond ql are left as they are (the staging masks
+// them).
 __device__ __forceinline__ void fetch_tile(const SsdParams& p, uint8_t* smem, int64_t bb,
-                                           int64_t hd, int64_t g, int64_t t0, int ql, int tid) {
-  for (int w = tid; w < kQ * (kN / 16); w += kThreads) {
-    const int r = w / (kN / 16), c = w % (kN / 16);
-    if (r >= ql) continue;
-    const int64_t ro = ((bb * p.L + t0 + r) * p.G + g) * kN + 16 * c;
-    const int slot = c ^ (r & 7);  // swizzle: conflict-free column reads of 8 rows
-    tc::cp_async16(smem + OFF_RC + r * kN + 16 * slot, p.C + ro);
-    tc::cp_async16(smem + OFF_RB + r * kN + 16 * slot, p.B + ro);
-  }
+                                           int64_t hd, int64_t t0, int ql, int tid) {
   for (int w = tid; w < kQ * (kP / 16); w += kThreads) {
     const int r = w / (kP / 16), c = w % (kP / 16);
     if (r >= ql) continue;
@@ -181,6 +181,73 @@ __device__ __forceinline__ void fetch_tile(const SsdParams& p, uint8_t* smem, in
     tc::cp_async16(smem + OFF_RX + r * kP + 16 * (c ^ (r & 3)), static_cast<const uint8_t*>(p.x) + xo);
   }
   tc::cp_async_commit();
+}
+
+// w'_n = fl16(sC_n sB_n / max_n(sC sB)) of group g (every thread calls it;
+// threads n < N return their w'_n, the others 0); wmax is returned too.
+__device__ __forceinline__ __half group_wprime(const SsdParams& p, int64_t g, int tid, float* red,
+                                               float& wmax, float& sc_n, float& sb_n) {
+  sc_n = 0.0f;
+  sb_n = 0.0f;
+  if (tid < kN) {
+    const int si = (int)g * (kN / p.gs) + tid / p.gs;
+    sc_n = __ldg(p.C_scale + si);
+    sb_n = __ldg(p.B_scale + si);
+  }
+  wmax = block_max(sc_n * sb_n, red, tid);
+  return __float2half_rn(wmax > 0.0f ? sc_n * sb_n / wmax : 0.0f);
+}
+
+// The head-independent MMA operands of one (batch, group, tile): C' =
+// fl16(codes * w'_n) and B (codes, exact) in the canonical K-major layouts the
+// SSD kernel's MMAs read, written once for all heads of the group.  Rows at
+// or beyond the sequence end are zero.
+__global__ void __launch_bounds__(kThreads) ssd_operand_kernel(const SsdParams p, uint8_t* ops) {
+  __shared__ float red[kThreads / 32];
+  __shared__ __align__(16) __half wh[kN];
+  const int tid = threadIdx.x;
+  const int64_t tile = blockIdx.x, bg = blockIdx.y;
+  const int64_t bb = bg / p.G, g = bg % p.G;
+  float wmax, sc_n, sb_n;
+  const __half w = group_wprime(p, g, tid, red, wmax, sc_n, sb_n);
+  if (tid < kN) wh[tid] = w;
+  __syncthreads();
+  const int64_t t0 = tile * kQ;
+  const int ql = (int)min((int64_t)kQ, p.L - t0);
+  uint8_t* dst = ops + (bg * p.ntiles + tile) * kOpTile;
+  // item (r, c): row r, states 16 c .. 16 c + 15; 8 consecutive items write
+  // one 128-byte core matrix
+  for (int it = tid; it < kQ * (kN / 16); it += kThreads) {
+    const int c = it / kQ, r = it % kQ;
+    uint4 cq = make_uint4(0, 0, 0, 0), bq = make_uint4(0, 0, 0, 0);
+    if (r < ql) {
+      const int64_t ro = ((bb * p.L + t0 + r) * p.G + g) * kN + 16 * c;
+      cq = __ldg(reinterpret_cast<const uint4*>(p.C + ro));
+      bq = __ldg(reinterpret_cast<const uint4*>(p.B + ro));
+    }
+    const uint32_t cw[4] = {cq.x ^ 0x80808080u, cq.y ^ 0x80808080u, cq.z ^ 0x80808080u,
+                            cq.w ^ 0x80808080u};
+    const uint32_t bw[4] = {bq.x ^ 0x80808080u, bq.y ^ 0x80808080u, bq.z ^ 0x80808080u,
+                            bq.w ^ 0x80808080u};
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {  // 8 states per 16-byte core-matrix row
+      const int n0 = 16 * c + 8 * hh;
+      const uint4 wq = *reinterpret_cast<const uint4*>(wh + n0);
+      const uint32_t wv[4] = {wq.x, wq.y, wq.z, wq.w};
+      uint32_t oc[4], ob[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const uint32_t wc = cw[2 * hh + k / 2], wb = bw[2 * hh + k / 2];
+        const int b0i = 2 * (k & 1);
+        oc[k] = h2_bits(__hmul2(s8x2_to_h2(wc, b0i, b0i + 1),
+                                *reinterpret_cast<const __half2*>(&wv[k])));
+        ob[k] = h2_bits(s8x2_to_h2(wb, b0i, b0i + 1));
+      }
+      const uint32_t off = tc::kmaj_off(r, n0, kN);
+      *reinterpret_cast<uint4*>(dst + off) = make_uint4(oc[0], oc[1], oc[2], oc[3]);
+      *reinterpret_cast<uint4*>(dst + kOpBlock + off) = make_uint4(ob[0], ob[1], ob[2], ob[3]);
+    }
+  }
 }
 
 // Warp 0: delta, S = cumsum(delta A) (log2 units) and the per-step factors of
@@ -257,7 +324,7 @@ template <bool kYQ>
 __global__ void __launch_bounds__(kThreads, 1) ssd_kernel(const SsdParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ uint32_t tmem_slot;
-  __shared__ __align__(8) uint64_t bars[3];
+  __shared__ __align__(8) uint64_t bars[4];  // MMA0, MMA1, MMA2+3, operand copies
   __shared__ int abort_flag;
   float* F = reinterpret_cast<float*>(smem + OFF_F);
 
@@ -311,8 +378,21 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_kernel(const SsdParams p) {
     tc::mbar_init(&bars[0], 1);
     tc::mbar_init(&bars[1], 1);
     tc::mbar_init(&bars[2], 1);
+    tc::mbar_init(&bars[3], 1);
   }
   __syncthreads();
+  // the group's operand blocks of a tile (C' then B) -> OFF_C / OFF_B, one
+  // bulk copy each, completion counted in bytes on bars[3]
+  const uint8_t* ops_bg = p.ops + (bb * p.G + g) * p.ntiles * (int64_t)kOpTile;
+  bool ops_pending = false;  // thread 0: a copy issued and not yet waited for
+  auto issue_ops = [&](int64_t tile) {
+    const uint8_t* src = ops_bg + tile * kOpTile;
+    stream::expect_tx(&bars[3], (uint32_t)kOpTile);
+    stream::bulk_g2s(smem + OFF_C, src, (uint32_t)kOpBlock, &bars[3]);
+    stream::bulk_g2s(smem + OFF_B, src + kOpBlock, (uint32_t)kOpBlock, &bars[3]);
+    ops_pending = true;
+  };
+  if (tid == 0) issue_ops(0);
   const float wmax = block_max(sc_n * sb_n, F + F_RED, tid);
   if (tid < kN) {
     // w'_n rounded to binary16 once; the state operand factor undoes the rounding
@@ -344,7 +424,7 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_kernel(const SsdParams p) {
   const uint32_t T_CB = 0, T_YD = 128, T_YO = 192, T_ACC = 256;
 
   // ---- tile 0: raw rows, per-step factors, state maximum
-  fetch_tile(p, smem, bb, hd, g, 0, (int)min((int64_t)kQ, L), tid);
+  fetch_tile(p, smem, bb, hd, 0, (int)min((int64_t)kQ, L), tid);
   float dtv[4] = {0.0f, 0.0f, 0.0f, 0.0f};
   if (warp == 0) {
 #pragma unroll
@@ -384,47 +464,6 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_kernel(const SsdParams p) {
     for (int w = 0; w < kThreads / 32; ++w) hmax_all = fmaxf(hmax_all, F[F_RED + 2 + w]);
     const int eh = norm_exp(hmax_all);
 
-    // ---- stage C' = fl16(codes * w'_n) and B (codes): thread -> (row, 32
-    // states); the states are warp-uniform so the w' reads are broadcasts
-    {
-      const int r = 32 * (warp >> 2) + lane, part = warp & 3;
-      const bool ok = r < ql;
-      uint4 cq[2], bq[2];
-#pragma unroll
-      for (int i = 0; i < 2; ++i) {
-        const int slot = (2 * part + i) ^ (r & 7);
-        cq[i] = ok ? *reinterpret_cast<const uint4*>(smem + OFF_RC + r * kN + 16 * slot)
-                   : make_uint4(0, 0, 0, 0);
-        bq[i] = ok ? *reinterpret_cast<const uint4*>(smem + OFF_RB + r * kN + 16 * slot)
-                   : make_uint4(0, 0, 0, 0);
-      }
-#pragma unroll
-      for (int i = 0; i < 2; ++i) {
-        const uint32_t cw[4] = {cq[i].x ^ 0x80808080u, cq[i].y ^ 0x80808080u,
-                                cq[i].z ^ 0x80808080u, cq[i].w ^ 0x80808080u};
-        const uint32_t bw[4] = {bq[i].x ^ 0x80808080u, bq[i].y ^ 0x80808080u,
-                                bq[i].z ^ 0x80808080u, bq[i].w ^ 0x80808080u};
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {  // 8 states per 16-byte core-matrix row
-          const int n0 = 32 * part + 16 * i + 8 * hh;
-          const uint4 wq = *reinterpret_cast<const uint4*>(F + F_WH + n0 / 2);
-          const uint32_t wv[4] = {wq.x, wq.y, wq.z, wq.w};
-          uint32_t oc[4], ob[4];
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const uint32_t wc = cw[2 * hh + k / 2], wb = bw[2 * hh + k / 2];
-            const int b0i = 2 * (k & 1);
-            oc[k] = h2_bits(__hmul2(s8x2_to_h2(wc, b0i, b0i + 1),
-                                    *reinterpret_cast<const __half2*>(&wv[k])));
-            ob[k] = h2_bits(s8x2_to_h2(wb, b0i, b0i + 1));
-          }
-          *reinterpret_cast<uint4*>(smem + OFF_C + tc::kmaj_off(r, n0, kN)) =
-              make_uint4(oc[0], oc[1], oc[2], oc[3]);
-          *reinterpret_cast<uint4*>(smem + OFF_B + tc::kmaj_off(r, n0, kN)) =
-              make_uint4(ob[0], ob[1], ob[2], ob[3]);
-        }
-      }
-    }
     // ---- stage x (exact) and w x (hi / lo): thread -> (row s, 16 p)
     {
       const int s = 32 * (warp >> 2) + lane, part = warp & 3;
@@ -485,7 +524,7 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_kernel(const SsdParams p) {
     // ---- fetch the next tile while this one runs
     const bool has_next = t0 + kQ < L;
     if (has_next) {
-      fetch_tile(p, smem, bb, hd, g, t0 + kQ, (int)min((int64_t)kQ, L - t0 - kQ), tid);
+      fetch_tile(p, smem, bb, hd, t0 + kQ, (int)min((int64_t)kQ, L - t0 - kQ), tid);
       if (warp == 0) {
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -499,6 +538,12 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_kernel(const SsdParams p) {
     // M, MMA2 (Y_off) and MMA3 (state, hi + lo) run while the CUDA cores form M
     if (tid == 0) {
       tc::fence_after();
+      // this tile's operand blocks have landed
+      if (!tc::mbar_wait(&bars[3], phase, kWaitLimit)) {
+        flags |= SSMQ_DEV_TIMEOUT;
+        abort_flag = 1;
+      }
+      ops_pending = false;
       const uint32_t id = tc::idesc_f16(kQ, kQ, false, false);
 #pragma unroll
       for (int k0 = 0; k0 < kN; k0 += 16)
@@ -629,6 +674,8 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_kernel(const SsdParams p) {
       abort_flag = 1;
     }
     tc::fence_after();
+    // every MMA reading OFF_C / OFF_B is complete: bring in the next tile's
+    if (tid == 0 && has_next && !abort_flag) issue_ops(t0 / kQ + 1);
 
     // x scales of this thread's 16 columns
     float sxv[16];
@@ -733,6 +780,9 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_kernel(const SsdParams p) {
   }
 
   tc::cp_async_wait_all();  // no copy may land after the CTA has exited (abort path)
+  // a copy still pending belongs to the tile after the one the loop left in
+  if (tid == 0 && ops_pending && !tc::mbar_wait(&bars[3], phase ^ 1u, kWaitLimit))
+    flags |= SSMQ_DEV_TIMEOUT;
 
   // ---- final state (P, N) through shared memory for coalesced stores
   if (p.h_final) {
@@ -752,9 +802,13 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_kernel(const SsdParams p) {
 
 }  // namespace
 
-size_t ssd_workspace_bytes(const ssmq_ssd_args&) { return 0; }
+size_t ssd_workspace_bytes(const ssmq_ssd_args& a) {
+  if (a.seqlen <= 0 || a.batch <= 0 || a.nheads <= 0) return 0;
+  const int64_t ntiles = (a.seqlen + kQ - 1) / kQ;
+  return (size_t)(a.batch * a.ngroups * ntiles) * (size_t)kOpTile;
+}
 
-cudaError_t launch_ssd(const ssmq_ssd_args& a, void*, cudaStream_t st) {
+cudaError_t launch_ssd(const ssmq_ssd_args& a, void* ws, cudaStream_t st) {
   const int64_t units = a.batch * a.nheads;
   if (units == 0) return cudaSuccess;
   if (a.seqlen == 0) {
@@ -795,6 +849,10 @@ cudaError_t launch_ssd(const ssmq_ssd_args& a, void*, cudaStream_t st) {
   p.n_y_groups = a.n_y_groups;
   p.h_final = a.h_final;
   p.status = a.status;
+  p.ntiles = (a.seqlen + kQ - 1) / kQ;
+  p.ops = static_cast<const uint8_t*>(ws);
+  ssd_operand_kernel<<<dim3((unsigned)p.ntiles, (unsigned)(a.batch * a.ngroups)), kThreads, 0, st>>>(
+      p, static_cast<uint8_t*>(ws));
   auto kern = p.y_q ? ssd_kernel<true> : ssd_kernel<false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        kSmemBytes);
