@@ -687,12 +687,14 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_kernel(const SsdParams p) {
       sxv[4 * j4 + 2] = v.z;
       sxv[4 * j4 + 3] = v.w;
     }
+    // the three accumulators this thread reads (Y_diag, Y_off: row t; the
+    // state increments: row n), one round trip to tensor memory
+    float yd[16], yo[16], acc[16];
+    tc::tmem_ld16x3(tmem + t_lane + T_YD + 16 * q4, tmem + t_lane + T_YO + 16 * q4,
+                    tmem + t_lane + T_ACC + 16 * q4, yd, yo, acc);
     // ---- y = sx_p (Y_diag 2^e_t + D x_code) + exp(S_t) 2^e_h Y_off  (thread: row t, 16 p)
     {
       const int t = row;
-      float yd[16], yo[16];
-      tc::tmem_ld16(tmem + t_lane + T_YD + 16 * q4, yd);
-      tc::tmem_ld16(tmem + t_lane + T_YO + 16 * q4, yo);
       if (t < ql) {
         const float rs = F[F_RS + t], es = ES[t] * pow2i(eh);
         const int64_t yo_off = ((bb * L + t0 + t) * H + hd) * kP + 16 * q4;
@@ -760,8 +762,6 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_kernel(const SsdParams p) {
     }
     // ---- state: h = exp(S_last) h + sB_n sx_p 2^e_x acc  (thread: row n, 16 p)
     {
-      float acc[16];
-      tc::tmem_ld16(tmem + t_lane + T_ACC + 16 * q4, acc);
       const float decay = ex2_sfu(s_last);
       const float f = sbr * pow2i(ex);
 #pragma unroll
