@@ -326,6 +326,14 @@ ssmq_status ssmq_selective_scan_w8(const ssmq_scan_args* args, void* stream);
  * Supported: P == 64, N == 128, chunk in {64, 128, 256}, H % G == 0.  The
  * result is the recurrence's for every chunk length (the decomposition is
  * exact up to rounding); the kernel processes 128-step tiles.
+ * Segments: when the (batch, head) sequences do not fill the last round of
+ * SMs evenly, the remaining sequences are cut into segments run in parallel
+ * from a zero state, and a second kernel adds each later segment's carried
+ * state term (exp(S_t) C_t h_start, gated like y) and forms h_final; y of
+ * those sequences is then rounded to binary16 twice.  max_segments = 1 turns
+ * this off (one pass per sequence: a call on steps [0, L) equals, byte for
+ * byte, a call on [0, L1) followed by one on [L1, L) with h0 = its h_final,
+ * L1 a multiple of 128); so do y_q and a NULL y.
  * status: SSMQ_DEV_BAD_GROUP as above; SSMQ_DEV_TIMEOUT if a bounded wait for
  * the tensor core gave up (the call's outputs are then incomplete).
  */
@@ -358,6 +366,10 @@ typedef struct {
   const int32_t* y_group;   /* [H * P] output cluster of each channel (with y_q) */
   const float* y_scale;     /* [n_y_groups] static output scales (with y_q) */
   int32_t n_y_groups;
+  int32_t max_segments;     /* 0: the library may cut some sequences into up
+                               to 32 segments (see above); n > 1: up to n;
+                               1: one pass per sequence.  The workspace size
+                               depends on it, on y and on y_q. */
 } ssmq_ssd_args;
 
 size_t ssmq_ssd_workspace_size(const ssmq_ssd_args* args);

@@ -49,7 +49,8 @@ class SSDArgs(C.Structure):
                 ("se_log2_ratio", _i32), ("dt", _vp), ("dt_bias", _vp), ("dt_softplus", _i32),
                 ("A", _vp), ("D", _vp), ("z", _vp), ("B", _vp), ("C", _vp), ("B_scale", _vp),
                 ("C_scale", _vp), ("h0", _vp), ("y", _vp), ("h_final", _vp), ("status", _vp), ("y_q", _vp),
-                ("y_group", _vp), ("y_scale", _vp), ("n_y_groups", _i32)]
+                ("y_group", _vp), ("y_scale", _vp), ("n_y_groups", _i32),
+                ("max_segments", _i32)]
 
 
 class DecodeArgs(C.Structure):

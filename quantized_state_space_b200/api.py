@@ -105,10 +105,11 @@ def ssd_chunk_scan(x, dt, A, B, C, B_scale, C_scale, state_group_size, *, chunk=
                    x_group=None, x_scale=None, se_scale=0.0, se_log2_ratio=2, D=None, z=None,
                    dt_bias=None, dt_softplus=True, h0=None, y=None, h_final=None,
                    return_state=True, y_group=None, y_scale=None, y_q=None, want_y=True,
-                   workspace=None, status=None):
+                   max_segments=0, workspace=None, status=None):
     """Mamba-2 SSD chunked scan.  x (b, L, H, P) int8 / soft-edge uint8;
     dt (b, L, H) float16; B, C (b, L, G, N) int8.  Returns (y, h_final), or
-    (y, h_final, y_q) with the int8 output (y_group over the H * P channels)."""
+    (y, h_final, y_q) with the int8 output (y_group over the H * P channels).
+    max_segments = 1: one pass per sequence (byte-exact checkpoint / resume)."""
     b, L, H, P = x.shape
     G, Nst = B.shape[2], B.shape[3]
     _dev_check(x, dt, A, B, C, B_scale, C_scale, x_group, x_scale, D, z, dt_bias, h0)
@@ -120,7 +121,7 @@ def ssd_chunk_scan(x, dt, A, B, C, B_scale, C_scale, state_group_size, *, chunk=
                   **_x_fields(x, x_group, x_scale, se_scale, se_log2_ratio),
                   dt=dt, dt_bias=dt_bias, dt_softplus=int(bool(dt_softplus)), A=A, D=D, z=z,
                   B=B, C=C, B_scale=B_scale, C_scale=C_scale, h0=h0, y=y, h_final=h_final,
-                  status=status, **yf)
+                  status=status, max_segments=max_segments, **yf)
     ws = N.ssmq_ssd_workspace_size(**fields)
     if ws and workspace is None:
         workspace = torch.empty(ws + 256, dtype=torch.uint8, device=x.device)

@@ -331,6 +331,7 @@ ssmq_status ssmq_ssd_chunk_scan_w8(const ssmq_ssd_args* a, void* workspace, size
           "%s: chunk must be 64, 128 or 256", fn);
   REQUIRE(a->state_group_size >= 1 && a->dstate % a->state_group_size == 0,
           SSMQ_ERR_INVALID_ARG, "%s: dstate must be a multiple of state_group_size", fn);
+  REQUIRE(a->max_segments >= 0, SSMQ_ERR_INVALID_ARG, "%s: max_segments must be >= 0", fn);
   if (a->batch == 0 || a->nheads == 0) return SSMQ_OK;
   const ssmq_status xs = check_x(a->x_format, a->x, a->x_group, a->x_scale, a->n_x_groups,
                                  a->se_log2_ratio, fn);

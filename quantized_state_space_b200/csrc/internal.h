@@ -38,6 +38,9 @@ cudaError_t launch_percentile_abs(const void* src, bool f16, int64_t n, const do
                                   float* out, float* thr, float alpha, void* workspace,
                                   cudaStream_t st);
 
+// streaming multiprocessors of the current device
+int sm_count();
+
 size_t ssd_workspace_bytes(const ssmq_ssd_args& a);
 cudaError_t launch_ssd(const ssmq_ssd_args& a, void* ws, cudaStream_t st);
 

@@ -17,6 +17,14 @@
 #include "fastdiv.h"
 
 namespace ssmq {
+
+int sm_count() {
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  return sms > 0 ? sms : 148;
+}
+
 namespace {
 
 constexpr int kVec = 16;
@@ -295,13 +303,6 @@ unsigned grid_for(Idx n) {
   uint64_t b = (nvec + kThreads - 1) / kThreads;
   if (b > (uint64_t)kMaxBlocks) b = kMaxBlocks;
   return (unsigned)(b ? b : 1);
-}
-
-int sm_count() {
-  int dev = 0, sms = 148;
-  if (cudaGetDevice(&dev) == cudaSuccess)
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  return sms > 0 ? sms : 148;
 }
 
 // Launches a pipeline kernel with `smem` bytes of dynamic shared memory.

@@ -123,6 +123,13 @@ struct SsdParams {
   uint32_t* status;
   const uint8_t* ops;  // operand blocks (workspace)
   int64_t ntiles;
+  // work items: units [0, full) are whole sequences; each later unit is cut
+  // into kseg segments of seg_tiles tiles whose local final states and total
+  // log2-decays go to seg_state / seg_dec (index (unit - full) * kseg + seg)
+  int64_t full;
+  int kseg, seg_tiles;
+  float* seg_state;
+  float* seg_dec;
 };
 
 // 2^e as an exact float for |e| < 126
@@ -253,10 +260,12 @@ __global__ void __launch_bounds__(kThreads) ssd_operand_kernel(const SsdParams p
 // Warp 0: delta, S = cumsum(delta A) (log2 units) and the per-step factors of
 // the tile of ql steps whose dt values the lanes hold (4 steps per lane),
 // into buffer fb; the tile's w max and S_last go to F_RED[0], F_RED[1].
-__device__ __forceinline__ void tile_factors(float* F, int fb, int ql, const float (&dtv)[4],
-                                             float bias, int softplus, float A2, float wmax,
-                                             int lane) {
-  float dl[4], sc[4];
+// Warp 0: delta_t of the tile's steps 4 lane .. 4 lane + 3 (0 at or beyond
+// ql) into dl, and S within the lane's steps (log2 units) into sc; off is the
+// lane's offset (S = sc + off) and s_last S at the tile's last step.
+__device__ __forceinline__ void tile_decay(int ql, const float (&dtv)[4], float bias,
+                                           int softplus, float A2, int lane, float (&dl)[4],
+                                           float (&sc)[4], float& off, float& s_last) {
   float run = 0.0f;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
@@ -276,8 +285,15 @@ __device__ __forceinline__ void tile_factors(float* F, int fb, int ql, const flo
     const float n = __shfl_up_sync(0xffffffffu, ex, o);
     if (lane >= o) ex += n;
   }
-  const float off = ex - run;
-  const float s_last = __shfl_sync(0xffffffffu, ex, 31);
+  off = ex - run;
+  s_last = __shfl_sync(0xffffffffu, ex, 31);
+}
+
+__device__ __forceinline__ void tile_factors(float* F, int fb, int ql, const float (&dtv)[4],
+                                             float bias, int softplus, float A2, float wmax,
+                                             int lane) {
+  float dl[4], sc[4], off, s_last;
+  tile_decay(ql, dtv, bias, softplus, A2, lane, dl, sc, off, s_last);
   float wmx = 0.0f;
   // S at the end and at the start of this lane's 32-step block (lanes 8 b + 7
   // and 8 b hold them), and the spread of S over the block
@@ -329,7 +345,19 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_kernel(const SsdParams p) {
   float* F = reinterpret_cast<float*>(smem + OFF_F);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int64_t u = blockIdx.x;  // b * H + h
+  // work item: a whole (batch, head) sequence, or segment seg of one
+  int64_t u, t_beg = 0, t_end = p.L;
+  int seg = 0, slot = -1;
+  if ((int64_t)blockIdx.x < p.full) {
+    u = blockIdx.x;  // b * H + h
+  } else {
+    const int64_t idx = (int64_t)blockIdx.x - p.full;
+    u = p.full + idx / p.kseg;
+    seg = (int)(idx % p.kseg);
+    slot = (int)idx;
+    t_beg = (int64_t)seg * p.seg_tiles * kQ;
+    t_end = min(p.L, t_beg + (int64_t)p.seg_tiles * kQ);
+  }
   const int64_t H = p.H, L = p.L;
   const int64_t bb = u / H, hd = u % H;
   const int64_t g = hd * p.G / H;
@@ -385,14 +413,16 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_kernel(const SsdParams p) {
   // bulk copy each, completion counted in bytes on bars[3]
   const uint8_t* ops_bg = p.ops + (bb * p.G + g) * p.ntiles * (int64_t)kOpTile;
   bool ops_pending = false;  // thread 0: a copy issued and not yet waited for
+  uint32_t ops_issued = 0;   // copies issued: copy i completes bars[3] phase i & 1
   auto issue_ops = [&](int64_t tile) {
     const uint8_t* src = ops_bg + tile * kOpTile;
     stream::expect_tx(&bars[3], (uint32_t)kOpTile);
     stream::bulk_g2s(smem + OFF_C, src, (uint32_t)kOpBlock, &bars[3]);
     stream::bulk_g2s(smem + OFF_B, src + kOpBlock, (uint32_t)kOpBlock, &bars[3]);
     ops_pending = true;
+    ++ops_issued;
   };
-  if (tid == 0) issue_ops(0);
+  if (tid == 0 && t_beg < t_end) issue_ops(t_beg / kQ);
   const float wmax = block_max(sc_n * sb_n, F + F_RED, tid);
   if (tid < kN) {
     // w'_n rounded to binary16 once; the state operand factor undoes the rounding
@@ -409,13 +439,13 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_kernel(const SsdParams p) {
   float hs[16];
   {
     float* stage = reinterpret_cast<float*>(smem + OFF_M);  // P x N fp32 = 32 KB
-    if (p.h0) {
+    if (p.h0 && seg == 0) {
       const float4* src = reinterpret_cast<const float4*>(p.h0 + u * kP * kN);
       for (int i = tid; i < kP * kN / 4; i += kThreads) reinterpret_cast<float4*>(stage)[i] = src[i];
     }
     __syncthreads();
 #pragma unroll
-    for (int j = 0; j < 16; ++j) hs[j] = p.h0 ? stage[(16 * q4 + j) * kN + row] : 0.0f;
+    for (int j = 0; j < 16; ++j) hs[j] = (p.h0 && seg == 0) ? stage[(16 * q4 + j) * kN + row] : 0.0f;
   }
   const float hfac = F[F_HF + row];  // state -> MMA2 operand
   const float sbr = F[F_SB + row];
@@ -424,13 +454,14 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_kernel(const SsdParams p) {
   const uint32_t T_CB = 0, T_YD = 128, T_YO = 192, T_ACC = 256;
 
   // ---- tile 0: raw rows, per-step factors, state maximum
-  fetch_tile(p, smem, bb, hd, 0, (int)min((int64_t)kQ, L), tid);
+  fetch_tile(p, smem, bb, hd, t_beg, (int)min((int64_t)kQ, t_end - t_beg), tid);
   float dtv[4] = {0.0f, 0.0f, 0.0f, 0.0f};
   if (warp == 0) {
 #pragma unroll
     for (int i = 0; i < 4; ++i)
-      if (4 * lane + i < L) dtv[i] = h2f(p.dt[(bb * L + 4 * lane + i) * H + hd]);
-    tile_factors(F, 0, (int)min((int64_t)kQ, L), dtv, bias, p.softplus, A2, wmax, lane);
+      if (t_beg + 4 * lane + i < t_end) dtv[i] = h2f(p.dt[(bb * L + t_beg + 4 * lane + i) * H + hd]);
+    tile_factors(F, 0, (int)min((int64_t)kQ, t_end - t_beg), dtv, bias, p.softplus, A2, wmax,
+                 lane);
   }
   auto state_max = [&]() {
     float hm = 0.0f;
@@ -448,8 +479,9 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_kernel(const SsdParams p) {
 
   uint32_t phase = 0;
   int fb = 0;  // buffer of this tile's per-step factors
-  for (int64_t t0 = 0; t0 < L; t0 += kQ, phase ^= 1u, fb ^= 1) {
-    const int ql = (int)min((int64_t)kQ, L - t0);
+  float s_tot = 0.0f;  // log2 decay over the work item (thread 0)
+  for (int64_t t0 = t_beg; t0 < t_end; t0 += kQ, phase ^= 1u, fb ^= 1) {
+    const int ql = (int)min((int64_t)kQ, t_end - t0);
     const float* S2 = F + F_S2 + fb * kQ;
     const float* DW = F + F_DW + fb * kQ;
     const float* WX = F + F_WX + fb * kQ;
@@ -522,14 +554,15 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_kernel(const SsdParams p) {
     __syncthreads();  // (B): operands staged, raw buffer consumed
 
     // ---- fetch the next tile while this one runs
-    const bool has_next = t0 + kQ < L;
+    const bool has_next = t0 + kQ < t_end;
+    if (tid == 0) s_tot += s_last;
     if (has_next) {
-      fetch_tile(p, smem, bb, hd, t0 + kQ, (int)min((int64_t)kQ, L - t0 - kQ), tid);
+      fetch_tile(p, smem, bb, hd, t0 + kQ, (int)min((int64_t)kQ, t_end - t0 - kQ), tid);
       if (warp == 0) {
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const int64_t t = t0 + kQ + 4 * lane + i;
-          dtv[i] = t < L ? h2f(p.dt[(bb * L + t) * H + hd]) : 0.0f;
+          dtv[i] = t < t_end ? h2f(p.dt[(bb * L + t) * H + hd]) : 0.0f;
         }
       }
     }
@@ -770,7 +803,7 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_kernel(const SsdParams p) {
     // ---- next tile: per-step factors (warp 0, other buffer), state maximum,
     // raw rows landed
     if (has_next && warp == 0)
-      tile_factors(F, fb ^ 1, (int)min((int64_t)kQ, L - t0 - kQ), dtv, bias, p.softplus, A2,
+      tile_factors(F, fb ^ 1, (int)min((int64_t)kQ, t_end - t0 - kQ), dtv, bias, p.softplus, A2,
                    wmax, lane);
     state_max();
     tc::cp_async_wait_all();
@@ -780,18 +813,23 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_kernel(const SsdParams p) {
   }
 
   tc::cp_async_wait_all();  // no copy may land after the CTA has exited (abort path)
-  // a copy still pending belongs to the tile after the one the loop left in
-  if (tid == 0 && ops_pending && !tc::mbar_wait(&bars[3], phase ^ 1u, kWaitLimit))
+  // a copy issued but not waited for (the loop was left early) lands first
+  if (tid == 0 && ops_pending &&
+      !tc::mbar_wait(&bars[3], (ops_issued - 1u) & 1u, kWaitLimit))
     flags |= SSMQ_DEV_TIMEOUT;
 
-  // ---- final state (P, N) through shared memory for coalesced stores
-  if (p.h_final) {
+  // ---- final state (P, N) through shared memory for coalesced stores: the
+  // sequence's h_final, or a segment's local state for the second kernel
+  float* fin = slot < 0 ? (p.h_final ? p.h_final + u * kP * kN : nullptr)
+                        : p.seg_state + (int64_t)slot * kP * kN;
+  if (slot >= 0 && tid == 0) p.seg_dec[slot] = s_tot;
+  if (fin) {
     float* stage = reinterpret_cast<float*>(smem + OFF_M);
     __syncthreads();
 #pragma unroll
     for (int j = 0; j < 16; ++j) stage[(16 * q4 + j) * kN + row] = hs[j];
     __syncthreads();
-    float4* dst = reinterpret_cast<float4*>(p.h_final + u * kP * kN);
+    float4* dst = reinterpret_cast<float4*>(fin);
     for (int i = tid; i < kP * kN / 4; i += kThreads) dst[i] = reinterpret_cast<float4*>(stage)[i];
   }
   tc::fence_before();
@@ -800,12 +838,257 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_kernel(const SsdParams p) {
   flag_status(p.status, flags);
 }
 
+// ---- segments of one sequence
+// A sequence of the last SM round may be cut into kseg segments of seg_tiles
+// tiles, each run by ssd_kernel from a zero state (segment 0 from h0).  The
+// recurrence is linear in the state, so segment j's true state entering step
+// t is its local one plus exp(S_t - S_j) h_start(j), S_j the cumulative decay
+// at its first step, with h_start(j) = exp(dec_{j-1}) h_start(j-1) + loc_{j-1}
+// from its predecessors' local final states loc and total decays dec
+// (h_start(1) = loc_0, segment 0 having started from h0).  The
+// missing output is the Y_off term of the segment's start state,
+// exp(S_t - S_j) C_t h_start(j) (times silu(z_t) when gated): the second
+// kernel adds it to y, rounding to binary16 once more, and forms h_final from
+// the last segment.
+constexpr int FX_C = 0;                       // C' block, K-major        32 KB
+constexpr int FX_HH = FX_C + kOpBlock;        // start state operand      16 KB
+constexpr int FX_ST = FX_HH + kN * kP * 2;    // start state fp32 (P, N)  32 KB
+constexpr int FX_S2 = FX_ST + kP * kN * 4;    // S of the tile (log2)     [128]
+constexpr int FX_HF = FX_S2 + kQ * 4;         // sC_n / w'_n              [128]
+constexpr int FX_RED = FX_HF + kN * 4;        // reductions               [32]
+constexpr int kFixSmem = FX_RED + 32 * 4;
+constexpr uint32_t kFixCols = 64;
+
+__global__ void __launch_bounds__(kThreads) ssd_fixup_kernel(const SsdParams p) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  __shared__ uint32_t tmem_slot;
+  __shared__ __align__(8) uint64_t bars[2];  // C' copy, MMA
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int seg = 1 + (int)blockIdx.x;
+  const int64_t slot0 = (int64_t)blockIdx.y * p.kseg;  // first segment slot of the unit
+  const int64_t u = p.full + blockIdx.y;
+  const int64_t H = p.H, L = p.L;
+  const int64_t bb = u / H, hd = u % H;
+  const int64_t g = hd * p.G / H;
+  const int row = 32 * (warp & 3) + lane;
+  const int q4 = warp >> 2;
+  const uint32_t s_base = tc::smem_u32(smem);
+  float* red = reinterpret_cast<float*>(smem + FX_RED);
+  float* S2 = reinterpret_cast<float*>(smem + FX_S2);
+  uint32_t flags = 0;
+
+  if (warp == 0) tc::tmem_alloc(&tmem_slot, kFixCols);
+  if (tid == 0) {
+    tc::mbar_init(&bars[0], 1);
+    tc::mbar_init(&bars[1], 1);
+  }
+  // state operand factor of the group (as in ssd_kernel)
+  {
+    float wmax, sc_n, sb_n;
+    const __half wh = group_wprime(p, g, tid, red, wmax, sc_n, sb_n);
+    if (tid < kN) {
+      const float whf = __half2float(wh);
+      reinterpret_cast<float*>(smem + FX_HF)[tid] = whf > 0.0f ? sc_n / whf : 0.0f;
+    }
+  }
+  // h_start(seg) by the chain, elementwise; the last segment also forms h_final
+  {
+    const float4* loc = reinterpret_cast<const float4*>(p.seg_state + slot0 * kP * kN);
+    const float* dec = p.seg_dec + slot0;
+    const bool last = seg == p.kseg - 1;
+    float4* st = reinterpret_cast<float4*>(smem + FX_ST);
+    for (int e = tid; e < kP * kN / 4; e += kThreads) {
+      // segment 0 ran from h0: its local state is already the true one
+      float4 h = loc[e];
+      for (int m = 1; m < seg; ++m) {
+        const float d = ex2_sfu(dec[m]);
+        const float4 l = loc[(int64_t)m * (kP * kN / 4) + e];
+        h = make_float4(fmaf(d, h.x, l.x), fmaf(d, h.y, l.y), fmaf(d, h.z, l.z),
+                        fmaf(d, h.w, l.w));
+      }
+      st[e] = h;
+      if (last && p.h_final) {
+        const float d = ex2_sfu(dec[seg]);
+        const float4 l = loc[(int64_t)seg * (kP * kN / 4) + e];
+        reinterpret_cast<float4*>(p.h_final + u * kP * kN)[e] =
+            make_float4(fmaf(d, h.x, l.x), fmaf(d, h.y, l.y), fmaf(d, h.z, l.z),
+                        fmaf(d, h.w, l.w));
+      }
+    }
+  }
+  __syncthreads();
+  // operand h'' = h sC_n / w'_n 2^-e_h in binary16 (thread: row n, 16 p)
+  int eh;
+  {
+    const float hfac = reinterpret_cast<const float*>(smem + FX_HF)[row];
+    const float* st = reinterpret_cast<const float*>(smem + FX_ST);
+    float hs[16];
+    float hm = 0.0f;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      hs[j] = st[(16 * q4 + j) * kN + row] * hfac;
+      hm = fmaxf(hm, fabsf(hs[j]));
+    }
+    eh = norm_exp(block_max(hm, red, tid));
+    const float f = pow2i(-eh);
+#pragma unroll
+    for (int grp = 0; grp < 2; ++grp) {
+      uint32_t oh[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        oh[k] = pack_h2(hs[8 * grp + 2 * k] * f, hs[8 * grp + 2 * k + 1] * f);
+      *reinterpret_cast<uint4*>(smem + FX_HH + tc::mnmaj_off(16 * q4 + 8 * grp, row, kP)) =
+          make_uint4(oh[0], oh[1], oh[2], oh[3]);
+    }
+  }
+  tc::fence_async_smem();
+  tc::fence_before();
+  __syncthreads();
+  tc::fence_after();
+
+  const uint32_t tmem = tmem_slot;
+  const uint32_t t_lane = (uint32_t)(32 * (warp & 3)) << 16;
+  const float A2 = __ldg(p.A + hd) * kLog2e;
+  const float bias = p.dt_bias ? __ldg(p.dt_bias + hd) : 0.0f;
+  const uint8_t* ops_bg = p.ops + (bb * p.G + g) * p.ntiles * (int64_t)kOpTile;
+  const int64_t tile_beg = (int64_t)seg * p.seg_tiles;
+  const int64_t tile_end = min(p.ntiles, tile_beg + p.seg_tiles);
+  float cum = 0.0f;  // S at the tile's start, from the segment's start
+  uint32_t phase = 0;
+  bool failed = false;
+  for (int64_t tile = tile_beg; tile < tile_end; ++tile, phase ^= 1u) {
+    const int64_t t0 = tile * kQ;
+    const int ql = (int)min((int64_t)kQ, L - t0);
+    if (tid == 0) {
+      stream::expect_tx(&bars[0], (uint32_t)kOpBlock);
+      stream::bulk_g2s(smem + FX_C, ops_bg + tile * kOpTile, (uint32_t)kOpBlock, &bars[0]);
+    }
+    if (warp == 0) {
+      float dtv[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        if (4 * lane + i < ql) dtv[i] = h2f(p.dt[(bb * L + t0 + 4 * lane + i) * H + hd]);
+      float dl[4], sc[4], off, s_last;
+      tile_decay(ql, dtv, bias, p.softplus, A2, lane, dl, sc, off, s_last);
+      *reinterpret_cast<float4*>(S2 + 4 * lane) =
+          make_float4(sc[0] + off, sc[1] + off, sc[2] + off, sc[3] + off);
+      if (lane == 0) red[0] = s_last;
+    }
+    if (tid == 0) {
+      if (!tc::mbar_wait(&bars[0], phase, kWaitLimit)) {
+        flags |= SSMQ_DEV_TIMEOUT;
+        failed = true;
+      } else {
+        tc::fence_after();
+        const uint32_t id_y = tc::idesc_f16(kQ, kP, false, true);
+#pragma unroll
+        for (int k0 = 0; k0 < kN; k0 += 16)
+          tc::mma_f16(tmem, tc::kmaj_desc(s_base + FX_C, k0, kN),
+                      tc::mnmaj_desc(s_base + FX_HH, k0, kP), id_y, k0 > 0);
+        tc::mma_commit(&bars[1]);
+      }
+    }
+    if (__syncthreads_or(failed)) break;  // S of the tile published, MMA issued
+    if (!tc::mbar_wait(&bars[1], phase, kWaitLimit)) {
+      flags |= SSMQ_DEV_TIMEOUT;
+      failed = true;
+    }
+    if (__syncthreads_or(failed)) break;
+    tc::fence_after();
+    float v[16];
+    tc::tmem_ld16(tmem + t_lane + 16 * q4, v);
+    const int t = row;
+    if (t < ql) {
+      const float f = ex2_sfu(cum + S2[t]) * pow2i(eh);
+      const int64_t off = ((bb * L + t0 + t) * H + hd) * kP + 16 * q4;
+      uint4* yr = reinterpret_cast<uint4*>(p.y + off);
+      const uint4 y0 = yr[0], y1 = yr[1];
+      const uint32_t yw[8] = {y0.x, y0.y, y0.z, y0.w, y1.x, y1.y, y1.z, y1.w};
+      uint32_t zw[8];
+      if (p.z) {
+        const uint4* zr = reinterpret_cast<const uint4*>(p.z + off);
+        const uint4 z0 = __ldg(zr), z1 = __ldg(zr + 1);
+        zw[0] = z0.x; zw[1] = z0.y; zw[2] = z0.z; zw[3] = z0.w;
+        zw[4] = z1.x; zw[5] = z1.y; zw[6] = z1.z; zw[7] = z1.w;
+      }
+      uint32_t out[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const float2 yo = __half22float2(*reinterpret_cast<const __half2*>(&yw[k]));
+        float c0 = f * v[2 * k], c1 = f * v[2 * k + 1];
+        if (p.z) {
+          const float2 zf = __half22float2(*reinterpret_cast<const __half2*>(&zw[k]));
+          c0 *= silu_f(zf.x);
+          c1 *= silu_f(zf.y);
+        }
+        out[k] = pack_h2(yo.x + c0, yo.y + c1);
+      }
+      yr[0] = make_uint4(out[0], out[1], out[2], out[3]);
+      yr[1] = make_uint4(out[4], out[5], out[6], out[7]);
+    }
+    cum += red[0];
+    tc::fence_before();
+    __syncthreads();  // S and the C' buffer free for the next tile
+    tc::fence_after();
+  }
+  // a copy whose MMA was never issued lands before the CTA exits
+  if (tid == 0 && failed) tc::mbar_wait(&bars[0], phase, kWaitLimit);
+  tc::fence_before();
+  __syncthreads();
+  if (warp == 0) tc::tmem_dealloc(tmem, kFixCols);
+  flag_status(p.status, flags);
+}
+
+}  // namespace
+
+namespace {
+
+constexpr int64_t kMaxSegSlots = 256;      // segment states a workspace holds at most
+constexpr int64_t kDefaultMaxSegments = 32;  // segments per sequence when not given
+
+int64_t seg_cap(const ssmq_ssd_args& a, int64_t ntiles) {
+  if (a.max_segments == 1 || a.y_q || !a.y || ntiles < 2) return 1;
+  return min(ntiles, a.max_segments > 0 ? (int64_t)a.max_segments : kDefaultMaxSegments);
+}
+
+// segment slots the workspace reserves: r k <= min(r cap, kMaxSegSlots), r <= units
+int64_t seg_slots(const ssmq_ssd_args& a, int64_t ntiles) {
+  const int64_t cap = seg_cap(a, ntiles);
+  return cap < 2 ? 0 : min(kMaxSegSlots, a.batch * a.nheads * cap);
+}
+
+struct SegPlan {
+  int64_t full;  // whole sequences (a multiple of the SM count)
+  int64_t r;     // sequences cut into segments
+  int kseg, seg_tiles;
+};
+
+// The last SM round of sequences (r = units mod SMs, or all units when fewer
+// than the SMs) is cut into k segments each, r k <= SMs, so that round takes
+// about 1/k of a sequence's time.
+SegPlan seg_plan(const ssmq_ssd_args& a, int64_t ntiles, int sms) {
+  const int64_t units = a.batch * a.nheads;
+  const SegPlan none{units, 0, 1, (int)ntiles};
+  const int64_t cap = seg_cap(a, ntiles);
+  if (cap < 2 || sms <= 0) return none;
+  const int64_t r = units >= sms ? units % sms : units;
+  if (r == 0) return none;
+  int64_t k = min(min((int64_t)sms / r, cap), kMaxSegSlots / r);
+  if (k < 2) return none;
+  const int64_t st = (ntiles + k - 1) / k;
+  k = (ntiles + st - 1) / st;  // every segment holds at least one tile
+  if (k < 2) return none;
+  return SegPlan{units - r, r, (int)k, (int)st};
+}
+
 }  // namespace
 
 size_t ssd_workspace_bytes(const ssmq_ssd_args& a) {
   if (a.seqlen <= 0 || a.batch <= 0 || a.nheads <= 0) return 0;
   const int64_t ntiles = (a.seqlen + kQ - 1) / kQ;
-  return (size_t)(a.batch * a.ngroups * ntiles) * (size_t)kOpTile;
+  const int64_t slots = seg_slots(a, ntiles);
+  return (size_t)(a.batch * a.ngroups * ntiles) * (size_t)kOpTile +
+         (size_t)slots * (size_t)(kP * kN * 4 + 4);
 }
 
 cudaError_t launch_ssd(const ssmq_ssd_args& a, void* ws, cudaStream_t st) {
@@ -851,13 +1134,26 @@ cudaError_t launch_ssd(const ssmq_ssd_args& a, void* ws, cudaStream_t st) {
   p.status = a.status;
   p.ntiles = (a.seqlen + kQ - 1) / kQ;
   p.ops = static_cast<const uint8_t*>(ws);
+  const SegPlan sp = seg_plan(a, p.ntiles, sm_count());
+  p.full = sp.full;
+  p.kseg = sp.kseg;
+  p.seg_tiles = sp.seg_tiles;
+  const size_t ops_bytes = (size_t)(a.batch * a.ngroups * p.ntiles) * (size_t)kOpTile;
+  p.seg_state = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + ops_bytes);
+  p.seg_dec = p.seg_state + seg_slots(a, p.ntiles) * kP * kN;
   ssd_operand_kernel<<<dim3((unsigned)p.ntiles, (unsigned)(a.batch * a.ngroups)), kThreads, 0, st>>>(
       p, static_cast<uint8_t*>(ws));
   auto kern = p.y_q ? ssd_kernel<true> : ssd_kernel<false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        kSmemBytes);
   if (e != cudaSuccess) return e;
-  kern<<<(unsigned)units, kThreads, kSmemBytes, st>>>(p);
+  kern<<<(unsigned)(sp.full + sp.r * sp.kseg), kThreads, kSmemBytes, st>>>(p);
+  if (sp.r > 0) {
+    e = cudaFuncSetAttribute(ssd_fixup_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kFixSmem);
+    if (e != cudaSuccess) return e;
+    ssd_fixup_kernel<<<dim3((unsigned)(sp.kseg - 1), (unsigned)sp.r), kThreads, kFixSmem, st>>>(p);
+  }
   return cudaGetLastError();
 }
 

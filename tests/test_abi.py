@@ -154,6 +154,24 @@ def test_ssd_validation(L):
         assert S(ws=FAKE + 16, nb=need) == N.ERR_ALIGNMENT
 
 
+def test_ssd_workspace_size_rule(L):
+    """Operand blocks (64 KB per batch, group and 128-step tile), plus, when
+    sequences may be cut into segments, one fp32 (P, N) state and one decay
+    per segment slot: min(256, sequences x min(cap, tiles)) slots."""
+    W = lambda **kw: L.ssmq_ssd_workspace_size(C.byref(_ssd_args(**kw)))
+    ops = lambda b, g, L_: b * g * ((L_ + 127) // 128) * 65536
+    slot = 64 * 128 * 4 + 4
+    assert W(max_segments=1) == ops(1, 1, 512)
+    assert W() == ops(1, 1, 512) + 8 * 4 * slot                 # 8 sequences, 4 tiles
+    assert W(seqlen=100) == ops(1, 1, 100)                      # one tile: never cut
+    assert W(max_segments=3) == ops(1, 1, 512) + 8 * 3 * slot
+    assert W(seqlen=128 * 100, batch=2) == ops(2, 1, 128 * 100) + 256 * slot
+    assert W(seqlen=128 * 100, nheads=1) == ops(1, 1, 128 * 100) + 32 * slot
+    assert W(y_q=FAKE, y_group=FAKE, y_scale=FAKE, n_y_groups=1) == ops(1, 1, 512)
+    assert W(y=None) == ops(1, 1, 512)
+    assert W(seqlen=0) == 0
+
+
 def _dec_args(**kw):
     f = dict(batch=4, nheads=8, headdim=64, dstate=128, ngroups=2, state_group_size=8,
              x_format=N.X_INT8_GROUP, x=FAKE, x_group=FAKE, x_scale=FAKE, n_x_groups=2, dt=FAKE,

@@ -66,18 +66,49 @@ def test_ssd_chunk_lengths_agree(orc, chunk):
 
 
 def test_ssd_split_with_state_bit_exact():
-    """scan(L) equals scan(first 256 steps) then scan(rest, h0 = its state)."""
+    """One pass per sequence (max_segments = 1): scan(L) equals scan(first 256
+    steps) then scan(rest, h0 = its state), byte for byte."""
     p = ssd_problem(460, 2, 512, 2, 64, 128, gate=True)
-    y, hf = gpu_ssd(p)
+    y, hf = gpu_ssd(p, max_segments=1)
     a, b = dict(p), dict(p)
     for k in ("x", "dt", "z", "B", "C"):
         a[k] = np.ascontiguousarray(p[k][:, :256])
         b[k] = np.ascontiguousarray(p[k][:, 256:])
-    ya, ha = gpu_ssd(a)
+    ya, ha = gpu_ssd(a, max_segments=1)
     b["h0"] = ha
-    yb, hb = gpu_ssd(b)
+    yb, hb = gpu_ssd(b, max_segments=1)
     np.testing.assert_array_equal(np.concatenate([ya, yb], axis=1), y)
     np.testing.assert_array_equal(hb, hf)
+
+
+SEG_CASES = [
+    # (b, L, H, G, gate, h0, max_segments, units checked (None: all))
+    (1, 128 * 40 + 37, 2, 1, True, True, 0, None),    # 2 sequences, 21 segments, ragged end
+    (1, 128 * 9, 3, 1, False, True, 4, None),         # at most 4 segments: 3 of 3 tiles
+    (1, 128 * 3 + 1, 1, 1, True, True, 0, None),      # last segment a single step
+    (2, 1024, 80, 4, True, False, 0,                  # 160 sequences: whole ones and cut ones
+     [0, 1, 77, 100, 147, 148, 150, 155, 159]),
+]
+
+
+@pytest.mark.parametrize("ci", range(len(SEG_CASES)))
+def test_ssd_segments_vs_oracle(orc, ci):
+    """Sequences cut into segments (the segment start states carried by the
+    second kernel) against the oracle, and against one pass per sequence."""
+    b, L, Hh, G, gate, h0, ms, units = SEG_CASES[ci]
+    p = ssd_problem(490 + ci, b, L, Hh, 64, 128, G=G, gate=gate, h0=h0, bias=True)
+    st = status_word()
+    y, hf = gpu_ssd(p, max_segments=ms, status=st)
+    assert int(H(st)[0]) == 0
+    u = np.arange(b * Hh) if units is None else np.asarray(units, np.int64)
+    yo, ho = orc.ssd_scan(p["x"], p["dt"], p["A"], p["B"], p["C"], p["B_scale"], p["C_scale"],
+                          p["state_group_size"], units=None if units is None else u,
+                          **oracle_kwargs(p))
+    yg = y.transpose(0, 2, 1, 3).reshape(b * Hh, L, 64)[u]
+    hg = hf.reshape(b * Hh, 64, 128)[u]
+    assert_scan_close(yg, yo.reshape(yg.shape), hg, ho.reshape(hg.shape))
+    y1, h1 = gpu_ssd(p, max_segments=1)
+    assert_scan_close(y, y1, hf, h1)
 
 
 def test_ssd_delta_zero(orc):
