@@ -52,6 +52,8 @@ constexpr int kN = 128;  // state dim
 constexpr int kThreads = 512;
 constexpr uint32_t kWaitLimit = 1u << 20;  // mbarrier probes (~1 us each) before giving up
 constexpr uint32_t kTmemCols = 512;
+constexpr int kIssueWarp = 12;   // rb 0, q4 3: an all-zero block of M
+constexpr int kFactorWarp = 8;   // rb 0, q4 2: an all-zero block of M
 
 // shared-memory map (bytes)
 constexpr int OFF_C = 0;                        // C codes * w'     [t][n]  K-major   32 KB
@@ -453,15 +455,43 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_kernel(const SsdParams p) {
   const uint32_t t_lane = (uint32_t)(32 * (warp & 3)) << 16;
   const uint32_t T_CB = 0, T_YD = 128, T_YO = 192, T_ACC = 256;
 
-  // ---- tile 0: raw rows, per-step factors, state maximum
-  fetch_tile(p, smem, bb, hd, t_beg, (int)min((int64_t)kQ, t_end - t_beg), tid);
-  float dtv[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-  if (warp == 0) {
+  // Warp roles in the decay-matrix phase.  Warp (rb = warp & 3, q4) owns rows
+  // [32 rb, 32 rb + 32) and columns [32 q4, 32 q4 + 32) of M: the ten warps
+  // with q4 <= rb form M (named barrier 1); the six blocks above the
+  // diagonal are zero, written once here, and their warps take other work
+  // meanwhile: kIssueWarp issues the Y_off and state MMAs, kFactorWarp forms
+  // the next tile's per-step factors and loads the dt values of the tile
+  // after it.
+  const bool m_warp = q4 <= (warp & 3);
+  __syncthreads();  // the initial state has left OFF_M
+  if (!m_warp) {
+    const int t = row;
+    F[F_RM + q4 * kQ + t] = 0.0f;
+#pragma unroll
+    for (int grp = 0; grp < 4; ++grp)
+      *reinterpret_cast<uint4*>(smem + OFF_M + tc::kmaj_off(t, 32 * q4 + 8 * grp, kQ)) =
+          make_uint4(0u, 0u, 0u, 0u);
+  }
+  // raw dt of the tile starting at t (binary16 bits; 0 beyond the end)
+  uint16_t dtr[4] = {0, 0, 0, 0};
+  auto load_dt = [&](int64_t t) {
 #pragma unroll
     for (int i = 0; i < 4; ++i)
-      if (t_beg + 4 * lane + i < t_end) dtv[i] = h2f(p.dt[(bb * L + t_beg + 4 * lane + i) * H + hd]);
-    tile_factors(F, 0, (int)min((int64_t)kQ, t_end - t_beg), dtv, bias, p.softplus, A2, wmax,
-                 lane);
+      dtr[i] = t + 4 * lane + i < t_end ? p.dt[(bb * L + t + 4 * lane + i) * H + hd] : (uint16_t)0;
+  };
+  auto factors_from_raw = [&](int buf, int ql_) {
+    float dtv[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) dtv[i] = h2f(dtr[i]);
+    tile_factors(F, buf, ql_, dtv, bias, p.softplus, A2, wmax, lane);
+  };
+
+  // ---- tile 0: raw rows, per-step factors, state maximum
+  fetch_tile(p, smem, bb, hd, t_beg, (int)min((int64_t)kQ, t_end - t_beg), tid);
+  if (warp == kFactorWarp) {
+    load_dt(t_beg);
+    factors_from_raw(0, (int)min((int64_t)kQ, t_end - t_beg));
+    if (t_beg + kQ < t_end) load_dt(t_beg + kQ);
   }
   auto state_max = [&]() {
     float hm = 0.0f;
@@ -553,155 +583,167 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_kernel(const SsdParams p) {
     tc::fence_before();
     __syncthreads();  // (B): operands staged, raw buffer consumed
 
-    // ---- fetch the next tile while this one runs
+    // ---- fetch the next tile's raw rows while this one runs
     const bool has_next = t0 + kQ < t_end;
     if (tid == 0) s_tot += s_last;
-    if (has_next) {
-      fetch_tile(p, smem, bb, hd, t0 + kQ, (int)min((int64_t)kQ, t_end - t0 - kQ), tid);
-      if (warp == 0) {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int64_t t = t0 + kQ + 4 * lane + i;
-          dtv[i] = t < t_end ? h2f(p.dt[(bb * L + t) * H + hd]) : 0.0f;
-        }
-      }
-    }
+    if (has_next) fetch_tile(p, smem, bb, hd, t0 + kQ, (int)min((int64_t)kQ, t_end - t0 - kQ), tid);
 
-    // ---- MMA0: CB = C' B^T  (M = t, N = s, K = n); then, independent of
-    // M, MMA2 (Y_off) and MMA3 (state, hi + lo) run while the CUDA cores form M
+    // ---- MMA0 (thread 0): CB = C' B^T (M = t, N = s, K = n), first in the
+    // tensor pipe; then kIssueWarp queues MMA2 (Y_off) and MMA3 (state,
+    // hi + lo), which run while the M warps form M
     if (tid == 0) {
       tc::fence_after();
       // this tile's operand blocks have landed
       if (!tc::mbar_wait(&bars[3], phase, kWaitLimit)) {
         flags |= SSMQ_DEV_TIMEOUT;
         abort_flag = 1;
+      } else {
+        const uint32_t id = tc::idesc_f16(kQ, kQ, false, false);
+#pragma unroll
+        for (int k0 = 0; k0 < kN; k0 += 16)
+          tc::mma_f16(tmem + T_CB, tc::kmaj_desc(s_base + OFF_C, k0, kN),
+                      tc::kmaj_desc(s_base + OFF_B, k0, kN), id, k0 > 0);
+        tc::mma_commit(&bars[0]);
       }
       ops_pending = false;
-      const uint32_t id = tc::idesc_f16(kQ, kQ, false, false);
-#pragma unroll
-      for (int k0 = 0; k0 < kN; k0 += 16)
-        tc::mma_f16(tmem + T_CB, tc::kmaj_desc(s_base + OFF_C, k0, kN),
-                    tc::kmaj_desc(s_base + OFF_B, k0, kN), id, k0 > 0);
-      tc::mma_commit(&bars[0]);
-      const uint32_t id_y = tc::idesc_f16(kQ, kP, false, true);
-      const uint32_t id_s = tc::idesc_f16(kN, kP, true, true);
-#pragma unroll
-      for (int k0 = 0; k0 < kN; k0 += 16)
-        tc::mma_f16(tmem + T_YO, tc::kmaj_desc(s_base + OFF_C, k0, kN),
-                    tc::mnmaj_desc(s_base + OFF_HH, k0, kP), id_y, k0 > 0);
-#pragma unroll
-      for (int k0 = 0; k0 < kQ; k0 += 16)
-        tc::mma_f16(tmem + T_ACC, tc::mnmaj_desc(s_base + OFF_B, k0, kN),
-                    tc::mnmaj_desc(s_base + OFF_XH, k0, kP), id_s, k0 > 0);
-#pragma unroll
-      for (int k0 = 0; k0 < kQ; k0 += 16)
-        tc::mma_f16(tmem + T_ACC, tc::mnmaj_desc(s_base + OFF_B, k0, kN),
-                    tc::mnmaj_desc(s_base + OFF_XL, k0, kP), id_s, 1u);
-      tc::mma_commit(&bars[2]);
     }
-    __syncwarp();
-    if (!tc::mbar_wait(&bars[0], phase, kWaitLimit)) {
-      flags |= SSMQ_DEV_TIMEOUT;
-      abort_flag = 1;
-    }
-    tc::fence_after();
-
-    // ---- M = CB * exp(S_t - S_s) * delta_s * w_max, row-normalised, s <= t
-    // (thread: row t, columns s in [32 q4, 32 q4 + 32))
-    // Column block q4 against row block (warp & 3), both warp-uniform: above
-    // the diagonal M is zero; strictly below it exp(S_t - S_s) =
-    // exp(S_t - S_p) exp(S_p - S_s) with p the block's last step, both
-    // factors <= 1 (no overflow, underflow only of negligible terms), and the
-    // row factor is applied with the normalisation; on the diagonal block
-    // each element takes its own exponential.
-    float mv[32];
-    float rt = 1.0f;  // row factor still to apply to mv
-    {
-      const int t = row, s0 = 32 * q4, rb = warp & 3;
-      float rmax = 0.0f;
-      if (q4 <= rb) {
-        float v[32];
-        tc::tmem_ld32(tmem + t_lane + T_CB + s0, v);
-        const float st = S2[t];
-        if (q4 < rb) {
-          rt = ex2_sfu(st - S2[s0 + 31]);
-#pragma unroll
-          for (int j4 = 0; j4 < 8; ++j4) {
-            const float4 c4 = *reinterpret_cast<const float4*>(CW + s0 + 4 * j4);
-            const float cw[4] = {c4.x, c4.y, c4.z, c4.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float m = v[4 * j4 + e] * cw[e];
-              mv[4 * j4 + e] = m;
-              rmax = fmaxf(rmax, fabsf(m));
-            }
-          }
-          rmax *= rt;
-        } else if (F[F_BS + fb * 4 + q4] < 90.0f) {
-          // diagonal block, S spread below 2^90: exp(S_t - S_s) =
-          // exp(S_t - S_m) exp(S_m - S_s) with m the block's first step (both
-          // factors within 2^+-90, the products far from fp32 overflow)
-          const float sm = S2[s0];
-          rt = ex2_sfu(st - sm);
-#pragma unroll
-          for (int j4 = 0; j4 < 8; ++j4) {
-            const float4 c4 = *reinterpret_cast<const float4*>(CD + s0 + 4 * j4);
-            const float cd[4] = {c4.x, c4.y, c4.z, c4.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float m = s0 + 4 * j4 + e <= t ? v[4 * j4 + e] * cd[e] : 0.0f;
-              mv[4 * j4 + e] = m;
-              rmax = fmaxf(rmax, fabsf(m));
-            }
-          }
-          rmax *= rt;
+    if (warp == 0) {
+      __syncwarp();
+      tc::named_arrive(2, 64);  // CB issued
+    } else if (warp == kIssueWarp) {
+      tc::named_sync(2, 64);
+      if (lane == 0) {
+        tc::fence_after();
+        if (!tc::mbar_wait(&bars[3], phase, kWaitLimit)) {
+          flags |= SSMQ_DEV_TIMEOUT;
+          abort_flag = 1;
         } else {
+          const uint32_t id_y = tc::idesc_f16(kQ, kP, false, true);
+          const uint32_t id_s = tc::idesc_f16(kN, kP, true, true);
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const int s = s0 + j;
-            const float m = s <= t ? v[j] * ex2_sfu(st - S2[s]) * DW[s] * wmax : 0.0f;
-            mv[j] = m;
-            rmax = fmaxf(rmax, fabsf(m));
+          for (int k0 = 0; k0 < kN; k0 += 16)
+            tc::mma_f16(tmem + T_YO, tc::kmaj_desc(s_base + OFF_C, k0, kN),
+                        tc::mnmaj_desc(s_base + OFF_HH, k0, kP), id_y, k0 > 0);
+#pragma unroll
+          for (int k0 = 0; k0 < kQ; k0 += 16)
+            tc::mma_f16(tmem + T_ACC, tc::mnmaj_desc(s_base + OFF_B, k0, kN),
+                        tc::mnmaj_desc(s_base + OFF_XH, k0, kP), id_s, k0 > 0);
+#pragma unroll
+          for (int k0 = 0; k0 < kQ; k0 += 16)
+            tc::mma_f16(tmem + T_ACC, tc::mnmaj_desc(s_base + OFF_B, k0, kN),
+                        tc::mnmaj_desc(s_base + OFF_XL, k0, kP), id_s, 1u);
+          tc::mma_commit(&bars[2]);
+        }
+      }
+      __syncwarp();
+    } else if (warp == kFactorWarp && has_next) {
+      // the next tile's per-step factors (other buffer), then the dt values
+      // of the tile after it
+      factors_from_raw(fb ^ 1, (int)min((int64_t)kQ, t_end - t0 - kQ));
+      if (t0 + 2 * kQ < t_end) load_dt(t0 + 2 * kQ);
+    }
+
+    if (m_warp) {
+      if (!tc::mbar_wait(&bars[0], phase, kWaitLimit)) {
+        flags |= SSMQ_DEV_TIMEOUT;
+        abort_flag = 1;
+      }
+      tc::fence_after();
+      // ---- M = CB * exp(S_t - S_s) * delta_s * w_max, row-normalised, s <= t
+      // (thread: row t, columns s in [32 q4, 32 q4 + 32)).  Strictly below
+      // the diagonal exp(S_t - S_s) = exp(S_t - S_p) exp(S_p - S_s) with p
+      // the block's last step, both factors <= 1 (no overflow, underflow only
+      // of negligible terms), and the row factor is applied with the
+      // normalisation; on the diagonal block each element takes its own
+      // exponential unless the block's S spread allows one more factoring.
+      float mv[32];
+      float rt = 1.0f;  // row factor still to apply to mv
+      {
+        const int t = row, s0 = 32 * q4, rb = warp & 3;
+        float rmax = 0.0f;
+        {
+          float v[32];
+          tc::tmem_ld32(tmem + t_lane + T_CB + s0, v);
+          const float st = S2[t];
+          if (q4 < rb) {
+            rt = ex2_sfu(st - S2[s0 + 31]);
+#pragma unroll
+            for (int j4 = 0; j4 < 8; ++j4) {
+              const float4 c4 = *reinterpret_cast<const float4*>(CW + s0 + 4 * j4);
+              const float cw[4] = {c4.x, c4.y, c4.z, c4.w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const float m = v[4 * j4 + e] * cw[e];
+                mv[4 * j4 + e] = m;
+                rmax = fmaxf(rmax, fabsf(m));
+              }
+            }
+            rmax *= rt;
+          } else if (F[F_BS + fb * 4 + q4] < 90.0f) {
+            // diagonal block, S spread below 2^90: exp(S_t - S_s) =
+            // exp(S_t - S_m) exp(S_m - S_s) with m the block's first step (both
+            // factors within 2^+-90, the products far from fp32 overflow)
+            const float sm = S2[s0];
+            rt = ex2_sfu(st - sm);
+#pragma unroll
+            for (int j4 = 0; j4 < 8; ++j4) {
+              const float4 c4 = *reinterpret_cast<const float4*>(CD + s0 + 4 * j4);
+              const float cd[4] = {c4.x, c4.y, c4.z, c4.w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const float m = s0 + 4 * j4 + e <= t ? v[4 * j4 + e] * cd[e] : 0.0f;
+                mv[4 * j4 + e] = m;
+                rmax = fmaxf(rmax, fabsf(m));
+              }
+            }
+            rmax *= rt;
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const int s = s0 + j;
+              const float m = s <= t ? v[j] * ex2_sfu(st - S2[s]) * DW[s] * wmax : 0.0f;
+              mv[j] = m;
+              rmax = fmaxf(rmax, fabsf(m));
+            }
           }
         }
-      } else {
-#pragma unroll
-        for (int j = 0; j < 32; ++j) mv[j] = 0.0f;
+        F[F_RM + q4 * kQ + t] = rmax;
       }
-      F[F_RM + q4 * kQ + t] = rmax;
-    }
-    if (__syncthreads_or(abort_flag)) break;  // (C): row maxima published
-    {
-      const int t = row;
-      const float rm = fmaxf(fmaxf(F[F_RM + t], F[F_RM + kQ + t]),
-                             fmaxf(F[F_RM + 2 * kQ + t], F[F_RM + 3 * kQ + t]));
-      const int et = norm_exp(rm);
-      const float sc = pow2i(-et) * rt;
-      if (q4 == 0) F[F_RS + t] = pow2i(et);
+      tc::named_sync(1, 320);  // (C): row maxima published (the M warps)
+      {
+        const int t = row;
+        const float rm = fmaxf(fmaxf(F[F_RM + t], F[F_RM + kQ + t]),
+                               fmaxf(F[F_RM + 2 * kQ + t], F[F_RM + 3 * kQ + t]));
+        const int et = norm_exp(rm);
+        const float sc = pow2i(-et) * rt;
+        if (q4 == 0) F[F_RS + t] = pow2i(et);
 #pragma unroll
-      for (int grp = 0; grp < 4; ++grp) {
-        uint32_t o[4];
+        for (int grp = 0; grp < 4; ++grp) {
+          uint32_t o[4];
 #pragma unroll
-        for (int k = 0; k < 4; ++k) o[k] = pack_h2(mv[8 * grp + 2 * k] * sc, mv[8 * grp + 2 * k + 1] * sc);
-        *reinterpret_cast<uint4*>(smem + OFF_M + tc::kmaj_off(t, 32 * q4 + 8 * grp, kQ)) =
-            make_uint4(o[0], o[1], o[2], o[3]);
+          for (int k = 0; k < 4; ++k) o[k] = pack_h2(mv[8 * grp + 2 * k] * sc, mv[8 * grp + 2 * k + 1] * sc);
+          *reinterpret_cast<uint4*>(smem + OFF_M + tc::kmaj_off(t, 32 * q4 + 8 * grp, kQ)) =
+              make_uint4(o[0], o[1], o[2], o[3]);
+        }
       }
-    }
-    tc::fence_async_smem();
-    tc::fence_before();
-    __syncthreads();  // (D): M staged
-
-    // ---- MMA1 (Y_diag = M X)
-    if (tid == 0) {
-      tc::fence_after();
-      const uint32_t id_y = tc::idesc_f16(kQ, kP, false, true);
+      tc::fence_async_smem();
+      tc::fence_before();
+      tc::named_sync(1, 320);  // (D): M staged
+      // ---- MMA1 (Y_diag = M X)
+      if (tid == 0 && !abort_flag) {
+        tc::fence_after();
+        const uint32_t id_y = tc::idesc_f16(kQ, kP, false, true);
 #pragma unroll
-      for (int k0 = 0; k0 < kQ; k0 += 16)
-        tc::mma_f16(tmem + T_YD, tc::kmaj_desc(s_base + OFF_M, k0, kQ),
-                    tc::mnmaj_desc(s_base + OFF_X, k0, kP), id_y, k0 > 0);
-      tc::mma_commit(&bars[1]);
+        for (int k0 = 0; k0 < kQ; k0 += 16)
+          tc::mma_f16(tmem + T_YD, tc::kmaj_desc(s_base + OFF_M, k0, kQ),
+                      tc::mnmaj_desc(s_base + OFF_X, k0, kP), id_y, k0 > 0);
+        tc::mma_commit(&bars[1]);
+      }
+      __syncwarp();
+      tc::named_arrive(3, kThreads);  // row scales published to the other warps
+    } else {
+      tc::named_sync(3, kThreads);
     }
-    __syncwarp();
     if (!tc::mbar_wait(&bars[1], phase, kWaitLimit) || !tc::mbar_wait(&bars[2], phase, kWaitLimit)) {
       flags |= SSMQ_DEV_TIMEOUT;
       abort_flag = 1;
@@ -800,11 +842,7 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_kernel(const SsdParams p) {
 #pragma unroll
       for (int j = 0; j < 16; ++j) hs[j] = fmaf(decay, hs[j], f * sxv[j] * acc[j]);
     }
-    // ---- next tile: per-step factors (warp 0, other buffer), state maximum,
-    // raw rows landed
-    if (has_next && warp == 0)
-      tile_factors(F, fb ^ 1, (int)min((int64_t)kQ, t_end - t0 - kQ), dtv, bias, p.softplus, A2,
-                   wmax, lane);
+    // ---- next tile: state maximum, raw rows landed
     state_max();
     tc::cp_async_wait_all();
     tc::fence_before();
