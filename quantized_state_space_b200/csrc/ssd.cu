@@ -52,8 +52,8 @@ constexpr int kN = 128;  // state dim
 constexpr int kThreads = 512;
 constexpr uint32_t kWaitLimit = 1u << 20;  // mbarrier probes (~1 us each) before giving up
 constexpr uint32_t kTmemCols = 512;
-constexpr int kIssueWarp = 12;   // rb 0, q4 3: an all-zero block of M
-constexpr int kFactorWarp = 8;   // rb 0, q4 2: an all-zero block of M
+constexpr int kIssueWarp = 14;   // rb 2, q4 3: an all-zero block of M
+constexpr int kFactorWarp = 9;   // rb 1, q4 2: an all-zero block of M
 
 // shared-memory map (bytes)
 constexpr int OFF_C = 0;                        // C codes * w'     [t][n]  K-major   32 KB
@@ -507,6 +507,26 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_kernel(const SsdParams p) {
   __syncthreads();
   tc::fence_after();
 
+  // CB = C' B^T of a tile (M = t, N = s, K = n) into T_CB, issued by thread 0
+  // once the tile's operand blocks (copy parity par) have landed: a tile's CB
+  // is issued at the end of the previous tile and runs during the staging
+  auto issue_cb = [&](uint32_t par) {
+    if (!tc::mbar_wait(&bars[3], par, kWaitLimit)) {
+      flags |= SSMQ_DEV_TIMEOUT;
+      abort_flag = 1;
+    } else {
+      tc::fence_after();
+      const uint32_t id = tc::idesc_f16(kQ, kQ, false, false);
+#pragma unroll
+      for (int k0 = 0; k0 < kN; k0 += 16)
+        tc::mma_f16(tmem + T_CB, tc::kmaj_desc(s_base + OFF_C, k0, kN),
+                    tc::kmaj_desc(s_base + OFF_B, k0, kN), id, k0 > 0);
+      tc::mma_commit(&bars[0]);
+    }
+    ops_pending = false;
+  };
+  if (tid == 0) issue_cb(0u);
+
   uint32_t phase = 0;
   int fb = 0;  // buffer of this tile's per-step factors
   float s_tot = 0.0f;  // log2 decay over the work item (thread 0)
@@ -588,30 +608,9 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_kernel(const SsdParams p) {
     if (tid == 0) s_tot += s_last;
     if (has_next) fetch_tile(p, smem, bb, hd, t0 + kQ, (int)min((int64_t)kQ, t_end - t0 - kQ), tid);
 
-    // ---- MMA0 (thread 0): CB = C' B^T (M = t, N = s, K = n), first in the
-    // tensor pipe; then kIssueWarp queues MMA2 (Y_off) and MMA3 (state,
-    // hi + lo), which run while the M warps form M
-    if (tid == 0) {
-      tc::fence_after();
-      // this tile's operand blocks have landed
-      if (!tc::mbar_wait(&bars[3], phase, kWaitLimit)) {
-        flags |= SSMQ_DEV_TIMEOUT;
-        abort_flag = 1;
-      } else {
-        const uint32_t id = tc::idesc_f16(kQ, kQ, false, false);
-#pragma unroll
-        for (int k0 = 0; k0 < kN; k0 += 16)
-          tc::mma_f16(tmem + T_CB, tc::kmaj_desc(s_base + OFF_C, k0, kN),
-                      tc::kmaj_desc(s_base + OFF_B, k0, kN), id, k0 > 0);
-        tc::mma_commit(&bars[0]);
-      }
-      ops_pending = false;
-    }
-    if (warp == 0) {
-      __syncwarp();
-      tc::named_arrive(2, 64);  // CB issued
-    } else if (warp == kIssueWarp) {
-      tc::named_sync(2, 64);
+    // ---- CB is in the tensor pipe already; kIssueWarp queues MMA2 (Y_off)
+    // and MMA3 (state, hi + lo), which run while the M warps form M
+    if (warp == kIssueWarp) {
       if (lane == 0) {
         tc::fence_after();
         if (!tc::mbar_wait(&bars[3], phase, kWaitLimit)) {
@@ -772,7 +771,7 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_kernel(const SsdParams p) {
       const int t = row;
       if (t < ql) {
         const float rs = F[F_RS + t], es = ES[t] * pow2i(eh);
-        const int64_t yo_off = ((bb * L + t0 + t) * H + hd) * kP + 16 * q4;
+        const int64_t yo_off = ((bb * L + t0 + t) * H + hd) * kP + 16 * q4;  // z
         // x of this row as exact binary16 values from the staged MMA operand
         uint32_t xw[8];
 #pragma unroll
@@ -827,11 +826,40 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_kernel(const SsdParams p) {
           }
           out[j / 2] = pack_half2(r2[0], r2[1]);
         }
-        if (kYQ) *reinterpret_cast<uint4*>(p.y_q + yo_off) = make_uint4(qo[0], qo[1], qo[2], qo[3]);
+        // y rows through shared memory (the state operands' buffers, free
+        // once MMA3 is done): 16-byte chunks swizzled by row, no bank conflicts
+        if (kYQ)
+          *reinterpret_cast<uint4*>(smem + OFF_XL + t * kP + 16 * (q4 ^ ((t >> 1) & 3))) =
+              make_uint4(qo[0], qo[1], qo[2], qo[3]);
         if (!kYQ || p.y) {
-          uint4* yr = reinterpret_cast<uint4*>(p.y + yo_off);
-          yr[0] = make_uint4(out[0], out[1], out[2], out[3]);
-          yr[1] = make_uint4(out[4], out[5], out[6], out[7]);
+          uint8_t* yrow = smem + OFF_XH + t * (2 * kP);
+          *reinterpret_cast<uint4*>(yrow + 16 * ((2 * q4) ^ (t & 7))) =
+              make_uint4(out[0], out[1], out[2], out[3]);
+          *reinterpret_cast<uint4*>(yrow + 16 * ((2 * q4 + 1) ^ (t & 7))) =
+              make_uint4(out[4], out[5], out[6], out[7]);
+        }
+      }
+      // the four warps of this row block write its 32 rows, whole 128-byte
+      // (64-byte for int8) row segments per warp instruction
+      const int rb = warp & 3, g = 32 * q4 + lane;
+      tc::named_sync(4 + rb, 128);
+      if (!kYQ || p.y) {
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          const int k = g + 128 * i, r = 32 * rb + k / 8, c = k % 8;
+          if (r < ql) {
+            const uint4 v = *reinterpret_cast<const uint4*>(smem + OFF_XH + r * (2 * kP) +
+                                                             16 * (c ^ (r & 7)));
+            *reinterpret_cast<uint4*>(p.y + ((bb * L + t0 + r) * H + hd) * kP + 8 * c) = v;
+          }
+        }
+      }
+      if (kYQ) {
+        const int r = 32 * rb + g / 4, c = g % 4;
+        if (r < ql) {
+          const uint4 v = *reinterpret_cast<const uint4*>(smem + OFF_XL + r * kP +
+                                                           16 * (c ^ ((r >> 1) & 3)));
+          *reinterpret_cast<uint4*>(p.y_q + ((bb * L + t0 + r) * H + hd) * kP + 16 * c) = v;
         }
       }
     }
@@ -842,7 +870,8 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_kernel(const SsdParams p) {
 #pragma unroll
       for (int j = 0; j < 16; ++j) hs[j] = fmaf(decay, hs[j], f * sxv[j] * acc[j]);
     }
-    // ---- next tile: state maximum, raw rows landed
+    // ---- next tile: its CB (thread 0), state maximum, raw rows landed
+    if (tid == 0 && has_next && !abort_flag) issue_cb(phase ^ 1u);
     state_max();
     tc::cp_async_wait_all();
     tc::fence_before();
