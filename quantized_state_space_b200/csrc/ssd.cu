@@ -56,14 +56,16 @@ constexpr int kIssueWarp = 14;   // rb 2, q4 3: an all-zero block of M
 constexpr int kFactorWarp = 9;   // rb 1, q4 2: an all-zero block of M
 
 // shared-memory map (bytes)
-constexpr int OFF_C = 0;                        // C codes * w'     [t][n]  K-major   32 KB
-constexpr int OFF_B = OFF_C + kQ * kN * 2;      // B codes          [s][n]            32 KB
-constexpr int OFF_X = OFF_B + kQ * kN * 2;      // x (exact)        [s][p]  MN-major  16 KB
+// two operand buffers (tiles alternate): C' codes * w' [t][n] K-major, then
+// B codes [s][n] K-major, 32 KB each
+constexpr int OFF_OPS = 0;
+constexpr int OFF_X = OFF_OPS + 4 * kQ * kN * 2;  // x (exact)      [s][p]  MN-major  16 KB
 constexpr int OFF_XH = OFF_X + kQ * kP * 2;     // w x hi           [s][p]            16 KB
 constexpr int OFF_XL = OFF_XH + kQ * kP * 2;    // w x lo                             16 KB
 constexpr int OFF_HH = OFF_XL + kQ * kP * 2;    // state            [n][p]  MN-major  16 KB
-constexpr int OFF_M = OFF_HH + kN * kP * 2;     // M                [t][s]  K-major   32 KB
-constexpr int OFF_F = OFF_M + kQ * kQ * 2;      // fp32 scalars
+constexpr int OFF_F = OFF_HH + kN * kP * 2;    // fp32 scalars
+// the initial and final states (P x N fp32, 32 KB) pass through OFF_X..OFF_HH
+constexpr int OFF_STATE = OFF_X;
 // fp32 scalar arrays (in floats, from OFF_F).  The per-step arrays of a tile
 // are double-buffered: warp 0 fills the next tile's while the others finish
 // this one.
@@ -89,8 +91,9 @@ constexpr int F_END = F_RED + 32;
 constexpr int OFF_RAW = (OFF_F + F_END * 4 + 127) / 128 * 128;
 constexpr int OFF_RX = OFF_RAW;                 // x codes [t][p]   8 KB
 constexpr int kSmemBytes = OFF_RX + kQ * kP;
+static_assert(kSmemBytes + 1024 <= 232448, "shared memory of one CTA");
 // operand blocks written by ssd_operand_kernel, per (batch, group, tile):
-// C' then B, each in the K-major canonical layout of OFF_C / OFF_B
+// C' then B, each in the K-major canonical layout of an operand buffer
 constexpr int kOpBlock = kQ * kN * 2;           // 32 KB
 constexpr int kOpTile = 2 * kOpBlock;           // 64 KB
 
@@ -342,7 +345,7 @@ template <bool kYQ>
 __global__ void __launch_bounds__(kThreads, 1) ssd_kernel(const SsdParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ uint32_t tmem_slot;
-  __shared__ __align__(8) uint64_t bars[4];  // MMA0, MMA1, MMA2+3, operand copies
+  __shared__ __align__(8) uint64_t bars[5];  // MMA0, MMA1, MMA2+3, operand buffers 0 / 1
   __shared__ int abort_flag;
   float* F = reinterpret_cast<float*>(smem + OFF_F);
 
@@ -409,22 +412,29 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_kernel(const SsdParams p) {
     tc::mbar_init(&bars[1], 1);
     tc::mbar_init(&bars[2], 1);
     tc::mbar_init(&bars[3], 1);
+    tc::mbar_init(&bars[4], 1);
   }
   __syncthreads();
-  // the group's operand blocks of a tile (C' then B) -> OFF_C / OFF_B, one
-  // bulk copy each, completion counted in bytes on bars[3]
+  // The group's operand blocks of the work item's tile j (C' then B) go to
+  // buffer j & 1 by one bulk copy, completion counted in bytes on
+  // bars[3 + (j & 1)] (its (j >> 1)-th phase); tile j + 2 is fetched as soon
+  // as tile j's MMAs are done.
   const uint8_t* ops_bg = p.ops + (bb * p.G + g) * p.ntiles * (int64_t)kOpTile;
-  bool ops_pending = false;  // thread 0: a copy issued and not yet waited for
-  uint32_t ops_issued = 0;   // copies issued: copy i completes bars[3] phase i & 1
-  auto issue_ops = [&](int64_t tile) {
-    const uint8_t* src = ops_bg + tile * kOpTile;
-    stream::expect_tx(&bars[3], (uint32_t)kOpTile);
-    stream::bulk_g2s(smem + OFF_C, src, (uint32_t)kOpBlock, &bars[3]);
-    stream::bulk_g2s(smem + OFF_B, src + kOpBlock, (uint32_t)kOpBlock, &bars[3]);
-    ops_pending = true;
-    ++ops_issued;
+  const int64_t n_tiles = (t_end - t_beg + kQ - 1) / kQ;
+  uint32_t ops_n[2] = {0u, 0u};  // thread 0: copies issued per buffer
+  auto issue_ops = [&](int64_t j) {
+    stream::expect_tx(&bars[3 + (j & 1)], (uint32_t)kOpTile);
+    stream::bulk_g2s(smem + OFF_OPS + (j & 1) * kOpTile, ops_bg + (t_beg / kQ + j) * kOpTile,
+                     (uint32_t)kOpTile, &bars[3 + (j & 1)]);
+    ++ops_n[j & 1];
   };
-  if (tid == 0 && t_beg < t_end) issue_ops(t_beg / kQ);
+  auto ops_wait = [&](int64_t j) {
+    return tc::mbar_wait(&bars[3 + (j & 1)], (uint32_t)(j >> 1) & 1u, kWaitLimit);
+  };
+  if (tid == 0) {
+    issue_ops(0);
+    if (n_tiles > 1) issue_ops(1);
+  }
   const float wmax = block_max(sc_n * sb_n, F + F_RED, tid);
   if (tid < kN) {
     // w'_n rounded to binary16 once; the state operand factor undoes the rounding
@@ -440,7 +450,7 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_kernel(const SsdParams p) {
   // ---- initial state: thread (row = n, quarter) holds p in [16 q4, 16 q4 + 16)
   float hs[16];
   {
-    float* stage = reinterpret_cast<float*>(smem + OFF_M);  // P x N fp32 = 32 KB
+    float* stage = reinterpret_cast<float*>(smem + OFF_STATE);  // P x N fp32 = 32 KB
     if (p.h0 && seg == 0) {
       const float4* src = reinterpret_cast<const float4*>(p.h0 + u * kP * kN);
       for (int i = tid; i < kP * kN / 4; i += kThreads) reinterpret_cast<float4*>(stage)[i] = src[i];
@@ -453,7 +463,9 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_kernel(const SsdParams p) {
   const float sbr = F[F_SB + row];
   const uint32_t tmem = tmem_slot;
   const uint32_t t_lane = (uint32_t)(32 * (warp & 3)) << 16;
-  const uint32_t T_CB = 0, T_YD = 128, T_YO = 192, T_ACC = 256;
+  // tensor memory columns: CB, Y_diag, Y_off, state increments, and M as the
+  // binary16 A operand of MMA1 (row t in lane t, two steps per column)
+  const uint32_t T_CB = 0, T_YD = 128, T_YO = 192, T_ACC = 256, T_M = 320;
 
   // Warp roles in the decay-matrix phase.  Warp (rb = warp & 3, q4) owns rows
   // [32 rb, 32 rb + 32) and columns [32 q4, 32 q4 + 32) of M: the ten warps
@@ -463,14 +475,11 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_kernel(const SsdParams p) {
   // the next tile's per-step factors and loads the dt values of the tile
   // after it.
   const bool m_warp = q4 <= (warp & 3);
-  __syncthreads();  // the initial state has left OFF_M
   if (!m_warp) {
-    const int t = row;
-    F[F_RM + q4 * kQ + t] = 0.0f;
-#pragma unroll
-    for (int grp = 0; grp < 4; ++grp)
-      *reinterpret_cast<uint4*>(smem + OFF_M + tc::kmaj_off(t, 32 * q4 + 8 * grp, kQ)) =
-          make_uint4(0u, 0u, 0u, 0u);
+    F[F_RM + q4 * kQ + row] = 0.0f;
+    const uint32_t z[16] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+    tc::tmem_st16(tmem + t_lane + T_M + 16 * q4, z);
+    tc::tmem_wait_st();
   }
   // raw dt of the tile starting at t (binary16 bits; 0 beyond the end)
   uint16_t dtr[4] = {0, 0, 0, 0};
@@ -507,31 +516,33 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_kernel(const SsdParams p) {
   __syncthreads();
   tc::fence_after();
 
-  // CB = C' B^T of a tile (M = t, N = s, K = n) into T_CB, issued by thread 0
-  // once the tile's operand blocks (copy parity par) have landed: a tile's CB
-  // is issued at the end of the previous tile and runs during the staging
-  auto issue_cb = [&](uint32_t par) {
-    if (!tc::mbar_wait(&bars[3], par, kWaitLimit)) {
+  // CB = C' B^T of tile j (M = t, N = s, K = n) into T_CB, issued by thread 0
+  // once its operand blocks have landed: tile j + 1's right after tile j's
+  // MMA1, so that it runs during tile j's epilogue
+  auto issue_cb = [&](int64_t j) {
+    if (!ops_wait(j)) {
       flags |= SSMQ_DEV_TIMEOUT;
       abort_flag = 1;
-    } else {
-      tc::fence_after();
-      const uint32_t id = tc::idesc_f16(kQ, kQ, false, false);
-#pragma unroll
-      for (int k0 = 0; k0 < kN; k0 += 16)
-        tc::mma_f16(tmem + T_CB, tc::kmaj_desc(s_base + OFF_C, k0, kN),
-                    tc::kmaj_desc(s_base + OFF_B, k0, kN), id, k0 > 0);
-      tc::mma_commit(&bars[0]);
+      return;
     }
-    ops_pending = false;
+    tc::fence_after();
+    const uint32_t cb = s_base + OFF_OPS + (uint32_t)(j & 1) * kOpTile;
+    const uint32_t id = tc::idesc_f16(kQ, kQ, false, false);
+#pragma unroll
+    for (int k0 = 0; k0 < kN; k0 += 16)
+      tc::mma_f16(tmem + T_CB, tc::kmaj_desc(cb, k0, kN), tc::kmaj_desc(cb + kOpBlock, k0, kN), id,
+                  k0 > 0);
+    tc::mma_commit(&bars[0]);
   };
-  if (tid == 0) issue_cb(0u);
+  if (tid == 0) issue_cb(0);
 
   uint32_t phase = 0;
   int fb = 0;  // buffer of this tile's per-step factors
   float s_tot = 0.0f;  // log2 decay over the work item (thread 0)
   for (int64_t t0 = t_beg; t0 < t_end; t0 += kQ, phase ^= 1u, fb ^= 1) {
     const int ql = (int)min((int64_t)kQ, t_end - t0);
+    const int64_t j = (t0 - t_beg) / kQ;  // tile of the work item
+    const uint32_t cbuf = s_base + OFF_OPS + (uint32_t)(j & 1) * kOpTile;  // its C', then B
     const float* S2 = F + F_S2 + fb * kQ;
     const float* DW = F + F_DW + fb * kQ;
     const float* WX = F + F_WX + fb * kQ;
@@ -613,7 +624,7 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_kernel(const SsdParams p) {
     if (warp == kIssueWarp) {
       if (lane == 0) {
         tc::fence_after();
-        if (!tc::mbar_wait(&bars[3], phase, kWaitLimit)) {
+        if (!ops_wait(j)) {
           flags |= SSMQ_DEV_TIMEOUT;
           abort_flag = 1;
         } else {
@@ -621,15 +632,15 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_kernel(const SsdParams p) {
           const uint32_t id_s = tc::idesc_f16(kN, kP, true, true);
 #pragma unroll
           for (int k0 = 0; k0 < kN; k0 += 16)
-            tc::mma_f16(tmem + T_YO, tc::kmaj_desc(s_base + OFF_C, k0, kN),
+            tc::mma_f16(tmem + T_YO, tc::kmaj_desc(cbuf, k0, kN),
                         tc::mnmaj_desc(s_base + OFF_HH, k0, kP), id_y, k0 > 0);
 #pragma unroll
           for (int k0 = 0; k0 < kQ; k0 += 16)
-            tc::mma_f16(tmem + T_ACC, tc::mnmaj_desc(s_base + OFF_B, k0, kN),
+            tc::mma_f16(tmem + T_ACC, tc::mnmaj_desc(cbuf + kOpBlock, k0, kN),
                         tc::mnmaj_desc(s_base + OFF_XH, k0, kP), id_s, k0 > 0);
 #pragma unroll
           for (int k0 = 0; k0 < kQ; k0 += 16)
-            tc::mma_f16(tmem + T_ACC, tc::mnmaj_desc(s_base + OFF_B, k0, kN),
+            tc::mma_f16(tmem + T_ACC, tc::mnmaj_desc(cbuf + kOpBlock, k0, kN),
                         tc::mnmaj_desc(s_base + OFF_XL, k0, kP), id_s, 1u);
           tc::mma_commit(&bars[2]);
         }
@@ -716,27 +727,24 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_kernel(const SsdParams p) {
         const int et = norm_exp(rm);
         const float sc = pow2i(-et) * rt;
         if (q4 == 0) F[F_RS + t] = pow2i(et);
+        uint32_t o[16];
 #pragma unroll
-        for (int grp = 0; grp < 4; ++grp) {
-          uint32_t o[4];
-#pragma unroll
-          for (int k = 0; k < 4; ++k) o[k] = pack_h2(mv[8 * grp + 2 * k] * sc, mv[8 * grp + 2 * k + 1] * sc);
-          *reinterpret_cast<uint4*>(smem + OFF_M + tc::kmaj_off(t, 32 * q4 + 8 * grp, kQ)) =
-              make_uint4(o[0], o[1], o[2], o[3]);
-        }
+        for (int k = 0; k < 16; ++k) o[k] = pack_h2(mv[2 * k] * sc, mv[2 * k + 1] * sc);
+        tc::tmem_st16(tmem + t_lane + T_M + 16 * q4, o);
+        tc::tmem_wait_st();
       }
-      tc::fence_async_smem();
       tc::fence_before();
-      tc::named_sync(1, 320);  // (D): M staged
+      tc::named_sync(1, 320);  // (D): M in tensor memory
       // ---- MMA1 (Y_diag = M X)
       if (tid == 0 && !abort_flag) {
         tc::fence_after();
         const uint32_t id_y = tc::idesc_f16(kQ, kP, false, true);
 #pragma unroll
         for (int k0 = 0; k0 < kQ; k0 += 16)
-          tc::mma_f16(tmem + T_YD, tc::kmaj_desc(s_base + OFF_M, k0, kQ),
-                      tc::mnmaj_desc(s_base + OFF_X, k0, kP), id_y, k0 > 0);
+          tc::mma_f16_ts(tmem + T_YD, tmem + T_M + k0 / 2, tc::mnmaj_desc(s_base + OFF_X, k0, kP),
+                         id_y, k0 > 0);
         tc::mma_commit(&bars[1]);
+        if (has_next) issue_cb(j + 1);
       }
       __syncwarp();
       tc::named_arrive(3, kThreads);  // row scales published to the other warps
@@ -748,8 +756,8 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_kernel(const SsdParams p) {
       abort_flag = 1;
     }
     tc::fence_after();
-    // every MMA reading OFF_C / OFF_B is complete: bring in the next tile's
-    if (tid == 0 && has_next && !abort_flag) issue_ops(t0 / kQ + 1);
+    // every MMA reading this tile's operand buffer is complete: tile j + 2's
+    if (tid == 0 && j + 2 < n_tiles && !abort_flag) issue_ops(j + 2);
 
     // x scales of this thread's 16 columns
     float sxv[16];
@@ -870,8 +878,7 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_kernel(const SsdParams p) {
 #pragma unroll
       for (int j = 0; j < 16; ++j) hs[j] = fmaf(decay, hs[j], f * sxv[j] * acc[j]);
     }
-    // ---- next tile: its CB (thread 0), state maximum, raw rows landed
-    if (tid == 0 && has_next && !abort_flag) issue_cb(phase ^ 1u);
+    // ---- next tile: state maximum, raw rows landed
     state_max();
     tc::cp_async_wait_all();
     tc::fence_before();
@@ -881,9 +888,10 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_kernel(const SsdParams p) {
 
   tc::cp_async_wait_all();  // no copy may land after the CTA has exited (abort path)
   // a copy issued but not waited for (the loop was left early) lands first
-  if (tid == 0 && ops_pending &&
-      !tc::mbar_wait(&bars[3], (ops_issued - 1u) & 1u, kWaitLimit))
-    flags |= SSMQ_DEV_TIMEOUT;
+  if (tid == 0)
+    for (int b = 0; b < 2; ++b)
+      if (ops_n[b] && !tc::mbar_wait(&bars[3 + b], (ops_n[b] - 1u) & 1u, kWaitLimit))
+        flags |= SSMQ_DEV_TIMEOUT;
 
   // ---- final state (P, N) through shared memory for coalesced stores: the
   // sequence's h_final, or a segment's local state for the second kernel
@@ -891,7 +899,7 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_kernel(const SsdParams p) {
                         : p.seg_state + (int64_t)slot * kP * kN;
   if (slot >= 0 && tid == 0) p.seg_dec[slot] = s_tot;
   if (fin) {
-    float* stage = reinterpret_cast<float*>(smem + OFF_M);
+    float* stage = reinterpret_cast<float*>(smem + OFF_STATE);
     __syncthreads();
 #pragma unroll
     for (int j = 0; j < 16; ++j) stage[(16 * q4 + j) * kN + row] = hs[j];
