@@ -516,9 +516,10 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_kernel(const SsdParams p) {
   __syncthreads();
   tc::fence_after();
 
-  // CB = C' B^T of tile j (M = t, N = s, K = n) into T_CB, issued by thread 0
-  // once its operand blocks have landed: tile j + 1's right after tile j's
-  // MMA1, so that it runs during tile j's epilogue
+  // CB = C' B^T of tile j (M = t, N = s, K = n) into T_CB once its operand
+  // blocks have landed: tile 0's by thread 0 here, tile j + 1's by kIssueWarp
+  // once tile j's decay matrix is formed, so that it runs during tile j's
+  // epilogue
   auto issue_cb = [&](int64_t j) {
     if (!ops_wait(j)) {
       flags |= SSMQ_DEV_TIMEOUT;
@@ -744,12 +745,15 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_kernel(const SsdParams p) {
           tc::mma_f16_ts(tmem + T_YD, tmem + T_M + k0 / 2, tc::mnmaj_desc(s_base + OFF_X, k0, kP),
                          id_y, k0 > 0);
         tc::mma_commit(&bars[1]);
-        if (has_next) issue_cb(j + 1);
       }
       __syncwarp();
-      tc::named_arrive(3, kThreads);  // row scales published to the other warps
+      tc::named_arrive(3, kThreads);  // row scales published, CB read: T_CB free
     } else {
       tc::named_sync(3, kThreads);
+      // tile j + 1's CB, queued behind this tile's MMAs (it runs during the
+      // epilogue); kIssueWarp, not thread 0, waits for room in the MMA queue
+      if (warp == kIssueWarp && lane == 0 && has_next && !abort_flag) issue_cb(j + 1);
+      __syncwarp();
     }
     if (!tc::mbar_wait(&bars[1], phase, kWaitLimit) || !tc::mbar_wait(&bars[2], phase, kWaitLimit)) {
       flags |= SSMQ_DEV_TIMEOUT;
