@@ -929,8 +929,8 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_kernel(const SsdParams p) {
 // exp(S_t - S_j) C_t h_start(j) (times silu(z_t) when gated): the second
 // kernel adds it to y, rounding to binary16 once more, and forms h_final from
 // the last segment.
-constexpr int FX_C = 0;                       // C' block, K-major        32 KB
-constexpr int FX_HH = FX_C + kOpBlock;        // start state operand      16 KB
+constexpr int FX_C = 0;                       // C' blocks, K-major  [2]  64 KB
+constexpr int FX_HH = FX_C + 2 * kOpBlock;    // start state operand      16 KB
 constexpr int FX_ST = FX_HH + kN * kP * 2;    // start state fp32 (P, N)  32 KB
 constexpr int FX_S2 = FX_ST + kP * kN * 4;    // S of the tile (log2)     [128]
 constexpr int FX_HF = FX_S2 + kQ * 4;         // sC_n / w'_n              [128]
@@ -941,7 +941,7 @@ constexpr uint32_t kFixCols = 64;
 __global__ void __launch_bounds__(kThreads) ssd_fixup_kernel(const SsdParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ uint32_t tmem_slot;
-  __shared__ __align__(8) uint64_t bars[2];  // C' copy, MMA
+  __shared__ __align__(8) uint64_t bars[3];  // C' copies (two buffers), MMA
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int seg = 1 + (int)blockIdx.x;
   const int64_t slot0 = (int64_t)blockIdx.y * p.kseg;  // first segment slot of the unit
@@ -960,6 +960,22 @@ __global__ void __launch_bounds__(kThreads) ssd_fixup_kernel(const SsdParams p) 
   if (tid == 0) {
     tc::mbar_init(&bars[0], 1);
     tc::mbar_init(&bars[1], 1);
+    tc::mbar_init(&bars[2], 1);
+  }
+  const uint8_t* ops_bg = p.ops + (bb * p.G + g) * p.ntiles * (int64_t)kOpTile;
+  const int64_t tile_beg = (int64_t)seg * p.seg_tiles;
+  const int64_t tile_end = min(p.ntiles, tile_beg + p.seg_tiles);
+  // C' of the segment's tile i -> buffer i & 1 (its (i >> 1)-th copy)
+  auto issue_c = [&](int64_t i) {
+    stream::expect_tx(&bars[i & 1], (uint32_t)kOpBlock);
+    stream::bulk_g2s(smem + FX_C + (i & 1) * kOpBlock, ops_bg + (tile_beg + i) * kOpTile,
+                     (uint32_t)kOpBlock, &bars[i & 1]);
+  };
+  uint32_t copies[2] = {0u, 0u};  // thread 0: copies issued per buffer
+  __syncthreads();                // barriers initialised
+  if (tid == 0) {
+    issue_c(0);
+    ++copies[0];
   }
   // state operand factor of the group (as in ssd_kernel)
   {
@@ -976,23 +992,30 @@ __global__ void __launch_bounds__(kThreads) ssd_fixup_kernel(const SsdParams p) 
     const float* dec = p.seg_dec + slot0;
     const bool last = seg == p.kseg - 1;
     float4* st = reinterpret_cast<float4*>(smem + FX_ST);
-    for (int e = tid; e < kP * kN / 4; e += kThreads) {
-      // segment 0 ran from h0: its local state is already the true one
-      float4 h = loc[e];
-      for (int m = 1; m < seg; ++m) {
-        const float d = ex2_sfu(dec[m]);
-        const float4 l = loc[(int64_t)m * (kP * kN / 4) + e];
-        h = make_float4(fmaf(d, h.x, l.x), fmaf(d, h.y, l.y), fmaf(d, h.z, l.z),
-                        fmaf(d, h.w, l.w));
-      }
-      st[e] = h;
-      if (last && p.h_final) {
-        const float d = ex2_sfu(dec[seg]);
-        const float4 l = loc[(int64_t)seg * (kP * kN / 4) + e];
-        reinterpret_cast<float4*>(p.h_final + u * kP * kN)[e] =
-            make_float4(fmaf(d, h.x, l.x), fmaf(d, h.y, l.y), fmaf(d, h.z, l.z),
-                        fmaf(d, h.w, l.w));
-      }
+    constexpr int kE = kP * kN / 4 / kThreads;  // float4 elements per thread
+    constexpr int64_t kStride = kP * kN / 4;   // float4 per state
+    auto fma4 = [](float d, float4 h, float4 l) {
+      return make_float4(fmaf(d, h.x, l.x), fmaf(d, h.y, l.y), fmaf(d, h.z, l.z),
+                         fmaf(d, h.w, l.w));
+    };
+    // segment 0 ran from h0: its local state is already the true one
+    float4 h[kE];
+#pragma unroll
+    for (int i = 0; i < kE; ++i) h[i] = loc[tid + kThreads * i];
+#pragma unroll 2
+    for (int m = 1; m < seg; ++m) {  // kE independent loads per step
+      const float d = ex2_sfu(dec[m]);
+#pragma unroll
+      for (int i = 0; i < kE; ++i) h[i] = fma4(d, h[i], loc[m * kStride + tid + kThreads * i]);
+    }
+#pragma unroll
+    for (int i = 0; i < kE; ++i) st[tid + kThreads * i] = h[i];
+    if (last && p.h_final) {
+      const float d = ex2_sfu(dec[seg]);
+#pragma unroll
+      for (int i = 0; i < kE; ++i)
+        reinterpret_cast<float4*>(p.h_final + u * kP * kN)[tid + kThreads * i] =
+            fma4(d, h[i], loc[seg * kStride + tid + kThreads * i]);
     }
   }
   __syncthreads();
@@ -1029,46 +1052,77 @@ __global__ void __launch_bounds__(kThreads) ssd_fixup_kernel(const SsdParams p) 
   const uint32_t t_lane = (uint32_t)(32 * (warp & 3)) << 16;
   const float A2 = __ldg(p.A + hd) * kLog2e;
   const float bias = p.dt_bias ? __ldg(p.dt_bias + hd) : 0.0f;
-  const uint8_t* ops_bg = p.ops + (bb * p.G + g) * p.ntiles * (int64_t)kOpTile;
-  const int64_t tile_beg = (int64_t)seg * p.seg_tiles;
-  const int64_t tile_end = min(p.ntiles, tile_beg + p.seg_tiles);
-  float cum = 0.0f;  // S at the tile's start, from the segment's start
-  uint32_t phase = 0;
-  bool failed = false;
-  for (int64_t tile = tile_beg; tile < tile_end; ++tile, phase ^= 1u) {
-    const int64_t t0 = tile * kQ;
-    const int ql = (int)min((int64_t)kQ, L - t0);
-    if (tid == 0) {
-      stream::expect_tx(&bars[0], (uint32_t)kOpBlock);
-      stream::bulk_g2s(smem + FX_C, ops_bg + tile * kOpTile, (uint32_t)kOpBlock, &bars[0]);
-    }
-    if (warp == 0) {
-      float dtv[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+  const int64_t nt = tile_end - tile_beg;
+  // raw dt of the segment's tile i (warp 0; binary16 bits, 0 beyond the end)
+  uint16_t dtr[4] = {0, 0, 0, 0};
+  auto load_dt = [&](int64_t i) {
+    const int64_t tb = (tile_beg + i) * kQ;
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
-        if (4 * lane + i < ql) dtv[i] = h2f(p.dt[(bb * L + t0 + 4 * lane + i) * H + hd]);
-      float dl[4], sc[4], off, s_last;
-      tile_decay(ql, dtv, bias, p.softplus, A2, lane, dl, sc, off, s_last);
+    for (int k = 0; k < 4; ++k)
+      dtr[k] = tb + 4 * lane + k < L ? p.dt[(bb * L + tb + 4 * lane + k) * H + hd] : (uint16_t)0;
+  };
+  if (warp == 0) load_dt(0);
+  // this thread's y (and z) row segment of the segment's tile i, loaded a
+  // tile ahead (the rows are 10 KB apart: each load is its own transaction)
+  const int t = row;
+  uint4 yn[2], zn[2];
+  auto load_yz = [&](int64_t i) {
+    const int64_t tr = (tile_beg + i) * kQ + t;
+    yn[0] = yn[1] = zn[0] = zn[1] = make_uint4(0u, 0u, 0u, 0u);
+    if (tr < L) {
+      const uint4* yr = reinterpret_cast<const uint4*>(p.y + ((bb * L + tr) * H + hd) * kP + 16 * q4);
+      yn[0] = yr[0];
+      yn[1] = yr[1];
+      if (p.z) {
+        const uint4* zr =
+            reinterpret_cast<const uint4*>(p.z + ((bb * L + tr) * H + hd) * kP + 16 * q4);
+        zn[0] = __ldg(zr);
+        zn[1] = __ldg(zr + 1);
+      }
+    }
+  };
+  load_yz(0);
+  float cum = 0.0f;  // S at the tile's start, from the segment's start
+  bool failed = false;
+  for (int64_t i = 0; i < nt; ++i) {
+    const int64_t t0 = (tile_beg + i) * kQ;
+    const int ql = (int)min((int64_t)kQ, L - t0);
+    // the next tile's C' into the other buffer (the MMA that read it is done)
+    if (tid == 0 && i + 1 < nt) {
+      issue_c(i + 1);
+      ++copies[(i + 1) & 1];
+    }
+    const int64_t off = ((bb * L + t0 + t) * H + hd) * kP + 16 * q4;
+    const uint4 yv[2] = {yn[0], yn[1]}, zv[2] = {zn[0], zn[1]};
+    if (i + 1 < nt) load_yz(i + 1);
+    if (warp == 0) {
+      float dtv[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) dtv[k] = h2f(dtr[k]);
+      float dl[4], sc[4], so, s_last;
+      tile_decay(ql, dtv, bias, p.softplus, A2, lane, dl, sc, so, s_last);
       *reinterpret_cast<float4*>(S2 + 4 * lane) =
-          make_float4(sc[0] + off, sc[1] + off, sc[2] + off, sc[3] + off);
+          make_float4(sc[0] + so, sc[1] + so, sc[2] + so, sc[3] + so);
       if (lane == 0) red[0] = s_last;
+      if (i + 1 < nt) load_dt(i + 1);
     }
     if (tid == 0) {
-      if (!tc::mbar_wait(&bars[0], phase, kWaitLimit)) {
+      if (!tc::mbar_wait(&bars[i & 1], (uint32_t)(i >> 1) & 1u, kWaitLimit)) {
         flags |= SSMQ_DEV_TIMEOUT;
         failed = true;
       } else {
         tc::fence_after();
+        const uint32_t cb = s_base + FX_C + (uint32_t)(i & 1) * kOpBlock;
         const uint32_t id_y = tc::idesc_f16(kQ, kP, false, true);
 #pragma unroll
         for (int k0 = 0; k0 < kN; k0 += 16)
-          tc::mma_f16(tmem, tc::kmaj_desc(s_base + FX_C, k0, kN),
-                      tc::mnmaj_desc(s_base + FX_HH, k0, kP), id_y, k0 > 0);
-        tc::mma_commit(&bars[1]);
+          tc::mma_f16(tmem, tc::kmaj_desc(cb, k0, kN), tc::mnmaj_desc(s_base + FX_HH, k0, kP), id_y,
+                      k0 > 0);
+        tc::mma_commit(&bars[2]);
       }
     }
     if (__syncthreads_or(failed)) break;  // S of the tile published, MMA issued
-    if (!tc::mbar_wait(&bars[1], phase, kWaitLimit)) {
+    if (!tc::mbar_wait(&bars[2], (uint32_t)i & 1u, kWaitLimit)) {
       flags |= SSMQ_DEV_TIMEOUT;
       failed = true;
     }
@@ -1076,20 +1130,12 @@ __global__ void __launch_bounds__(kThreads) ssd_fixup_kernel(const SsdParams p) 
     tc::fence_after();
     float v[16];
     tc::tmem_ld16(tmem + t_lane + 16 * q4, v);
-    const int t = row;
     if (t < ql) {
       const float f = ex2_sfu(cum + S2[t]) * pow2i(eh);
-      const int64_t off = ((bb * L + t0 + t) * H + hd) * kP + 16 * q4;
-      uint4* yr = reinterpret_cast<uint4*>(p.y + off);
-      const uint4 y0 = yr[0], y1 = yr[1];
-      const uint32_t yw[8] = {y0.x, y0.y, y0.z, y0.w, y1.x, y1.y, y1.z, y1.w};
-      uint32_t zw[8];
-      if (p.z) {
-        const uint4* zr = reinterpret_cast<const uint4*>(p.z + off);
-        const uint4 z0 = __ldg(zr), z1 = __ldg(zr + 1);
-        zw[0] = z0.x; zw[1] = z0.y; zw[2] = z0.z; zw[3] = z0.w;
-        zw[4] = z1.x; zw[5] = z1.y; zw[6] = z1.z; zw[7] = z1.w;
-      }
+      const uint32_t yw[8] = {yv[0].x, yv[0].y, yv[0].z, yv[0].w,
+                              yv[1].x, yv[1].y, yv[1].z, yv[1].w};
+      const uint32_t zw[8] = {zv[0].x, zv[0].y, zv[0].z, zv[0].w,
+                              zv[1].x, zv[1].y, zv[1].z, zv[1].w};
       uint32_t out[8];
 #pragma unroll
       for (int k = 0; k < 8; ++k) {
@@ -1102,16 +1148,20 @@ __global__ void __launch_bounds__(kThreads) ssd_fixup_kernel(const SsdParams p) 
         }
         out[k] = pack_h2(yo.x + c0, yo.y + c1);
       }
+      uint4* yr = reinterpret_cast<uint4*>(p.y + off);
       yr[0] = make_uint4(out[0], out[1], out[2], out[3]);
       yr[1] = make_uint4(out[4], out[5], out[6], out[7]);
     }
     cum += red[0];
     tc::fence_before();
-    __syncthreads();  // S and the C' buffer free for the next tile
+    __syncthreads();  // S and tensor memory free for the next tile
     tc::fence_after();
   }
-  // a copy whose MMA was never issued lands before the CTA exits
-  if (tid == 0 && failed) tc::mbar_wait(&bars[0], phase, kWaitLimit);
+  // copies still in flight (the loop was left early) land before the CTA exits
+  if (tid == 0)
+    for (int b = 0; b < 2; ++b)
+      if (copies[b] && !tc::mbar_wait(&bars[b], (copies[b] - 1u) & 1u, kWaitLimit))
+        flags |= SSMQ_DEV_TIMEOUT;
   tc::fence_before();
   __syncthreads();
   if (warp == 0) tc::tmem_dealloc(tmem, kFixCols);
