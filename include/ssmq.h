@@ -117,6 +117,34 @@ ssmq_status ssmq_quantize_groups(const void* src, ssmq_dtype dtype,
                                  int8_t* q_out, uint32_t* status,
                                  void* stream);
 
+/*
+ * Batched static quantization: ssmq_quantize_groups with SSMQ_SCALE_STATIC
+ * for n_jobs (1..8) tensors, in one launch for all jobs of one dtype and
+ * layout class (e.g. the Mamba-1 layer's x, B and C), each job's tiles taken
+ * by its own share of the CTAs.  Results are byte-identical to one
+ * ssmq_quantize_groups call per job.  The pages have no counterpart: this is
+ * a launch-count optimisation of this library.
+ *
+ * jobs    host array of n_jobs descriptors (read during the call); each
+ *         field as for ssmq_quantize_groups (scales are inputs); the jobs'
+ *         q_out ranges must not overlap each other or any src
+ * status  device uint32 word or NULL (flags of all jobs)
+ * Errors: INVALID_ARG for n_jobs outside [1, 8] or a job that
+ * ssmq_quantize_groups would reject; ALIGNMENT likewise.
+ */
+typedef struct {
+  const void* src;
+  ssmq_dtype dtype;
+  int64_t outer, mid, inner;
+  const int32_t* group_of_mid;
+  int32_t n_groups;
+  const float* scales;
+  int8_t* q_out;
+} ssmq_quant_job;
+
+ssmq_status ssmq_quantize_groups_batch(const ssmq_quant_job* jobs, int32_t n_jobs,
+                                       uint32_t* status, void* stream);
+
 /* ------------------------------------------------------------------------ */
 /* Three-mode soft-edge codec                                                */
 /* ------------------------------------------------------------------------ */

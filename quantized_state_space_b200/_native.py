@@ -73,7 +73,13 @@ class M1DecodeArgs(C.Structure):
 
 
 # entry point -> (restype, argtypes); every name declared in include/ssmq.h
+class QuantJob(C.Structure):
+    _fields_ = [("src", _vp), ("dtype", _i32), ("outer", _i64), ("mid", _i64), ("inner", _i64),
+                ("group_of_mid", _vp), ("n_groups", _i32), ("scales", _vp), ("q_out", _vp)]
+
+
 SIGNATURES = {
+    "ssmq_quantize_groups_batch": (_i32, [C.POINTER(QuantJob), _i32, _vp, _vp]),
     "ssmq_quantize_groups": (_i32, [_vp, _i32, _i64, _i64, _i64, _vp, _i32, _i32, _vp, _vp,
                                     _vp, _vp]),
     "ssmq_softedge_encode": (_i32, [_vp, _i32, _i64, _f32, _f32, _f32, _i32, _vp, _vp, _vp]),
@@ -165,6 +171,17 @@ def ssmq_quantize_groups(src, outer, mid, inner, group_of_mid, n_groups, mode, s
     _check(lib().ssmq_quantize_groups(ptr(src), _dtype_of(src, dtype), outer, mid, inner,
                                       ptr(group_of_mid), n_groups, mode, ptr(scales), ptr(q_out),
                                       ptr(status), _stream(stream)))
+
+
+def ssmq_quantize_groups_batch(jobs, status=None, stream=None):
+    """jobs: list of dicts with the fields of ssmq_quant_job (tensors for the
+    pointer fields; dtype taken from src when absent)."""
+    arr = (QuantJob * len(jobs))()
+    for i, j in enumerate(jobs):
+        j = dict(j)
+        j.setdefault("dtype", _dtype_of(j["src"], None))
+        arr[i] = _fill(QuantJob, j)
+    _check(lib().ssmq_quantize_groups_batch(arr, len(jobs), ptr(status), _stream(stream)))
 
 
 def ssmq_softedge_encode(src, n, scale, thr_lo, thr_hi, log2_ratio, codes, status=None,

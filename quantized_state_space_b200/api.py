@@ -29,6 +29,22 @@ def quantize_groups(src, outer, mid, inner, group_of_mid, n_groups, *, scales=No
     return q, scales
 
 
+def quantize_groups_batch(jobs, *, status=None):
+    """Static int8 codes of several tensors in one launch (per dtype and
+    layout class).  jobs: sequence of (src, outer, mid, inner, group_of_mid,
+    n_groups, scales, out-or-None); returns the code tensors."""
+    outs, descs = [], []
+    for src, outer, mid, inner, gmap, n_groups, scales, out in jobs:
+        _dev_check(src, gmap, scales)
+        q = out if out is not None else torch.empty(src.shape, dtype=torch.int8,
+                                                    device=src.device)
+        outs.append(q)
+        descs.append(dict(src=src, outer=outer, mid=mid, inner=inner, group_of_mid=gmap,
+                          n_groups=n_groups, scales=scales, q_out=q))
+    N.ssmq_quantize_groups_batch(descs, status=status)
+    return outs
+
+
 def softedge_encode(src, scale, thr_lo, thr_hi, log2_ratio=2, *, out=None, status=None):
     _dev_check(src)
     codes = out if out is not None else torch.empty(src.shape, dtype=torch.uint8, device=src.device)

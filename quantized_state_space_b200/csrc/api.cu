@@ -146,6 +146,37 @@ ssmq_status ssmq_quantize_groups(const void* src, ssmq_dtype dtype, int64_t oute
                 fn);
 }
 
+ssmq_status ssmq_quantize_groups_batch(const ssmq_quant_job* jobs, int32_t n_jobs,
+                                       uint32_t* status, void* stream) {
+  const char* fn = "ssmq_quantize_groups_batch";
+  REQUIRE(jobs != nullptr, SSMQ_ERR_INVALID_ARG, "%s: jobs is NULL", fn);
+  REQUIRE(n_jobs >= 1 && n_jobs <= ssmq::kMaxQuantJobs, SSMQ_ERR_INVALID_ARG,
+          "%s: n_jobs must be in [1, %d] (got %d)", fn, ssmq::kMaxQuantJobs, (int)n_jobs);
+  ssmq::QuantJob hj[ssmq::kMaxQuantJobs];
+  for (int k = 0; k < n_jobs; ++k) {
+    const ssmq_quant_job& j = jobs[k];
+    REQUIRE(j.dtype == SSMQ_F32 || j.dtype == SSMQ_F16, SSMQ_ERR_INVALID_ARG,
+            "%s: job %d: bad dtype %d", fn, k, (int)j.dtype);
+    REQUIRE(j.outer >= 0 && j.mid >= 0 && j.inner >= 0, SSMQ_ERR_INVALID_ARG,
+            "%s: job %d: negative size", fn, k);
+    REQUIRE(j.n_groups >= 1, SSMQ_ERR_INVALID_ARG, "%s: job %d: n_groups must be >= 1", fn, k);
+    REQUIRE(j.scales != nullptr, SSMQ_ERR_INVALID_ARG, "%s: job %d: scales is NULL", fn, k);
+    const bool empty = j.outer == 0 || j.mid == 0 || j.inner == 0;
+    if (!empty) {
+      REQUIRE(j.src && j.q_out && j.group_of_mid, SSMQ_ERR_INVALID_ARG, "%s: job %d: NULL tensor",
+              fn, k);
+      REQUIRE(j.outer <= (INT64_MAX / j.mid) / j.inner, SSMQ_ERR_INVALID_ARG,
+              "%s: job %d: size overflow", fn, k);
+    }
+    REQUIRE(aligned16(j.src) && aligned16(j.q_out), SSMQ_ERR_ALIGNMENT,
+            "%s: job %d: src and q_out must be 16-byte aligned", fn, k);
+    hj[k] = ssmq::QuantJob{j.src, j.dtype == SSMQ_F16, empty ? 0 : j.outer, j.mid, j.inner,
+                           j.group_of_mid, j.n_groups, j.scales, j.q_out};
+  }
+  if (injected(fn)) return fail(SSMQ_ERR_CUDA, "%s: injected launch failure", fn);
+  return finish(ssmq::launch_quantize_batch(hj, n_jobs, status, (cudaStream_t)stream), fn);
+}
+
 ssmq_status ssmq_softedge_encode(const void* src, ssmq_dtype dtype, int64_t n, float scale,
                                  float thr_lo, float thr_hi, int32_t log2_ratio, uint8_t* codes,
                                  uint32_t* status, void* stream) {

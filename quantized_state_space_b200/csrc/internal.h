@@ -14,6 +14,19 @@ cudaError_t launch_quantize(const void* src, bool f16, int64_t outer, int64_t mi
                             bool absmax, float* scales, int8_t* q, uint32_t* status,
                             cudaStream_t st);
 
+// one static quantization of a batch (validated by the API layer)
+struct QuantJob {
+  const void* src;
+  bool f16;
+  int64_t outer, mid, inner;
+  const int32_t* gmap;
+  int32_t n_groups;
+  const float* scales;
+  int8_t* q;
+};
+constexpr int kMaxQuantJobs = 8;
+cudaError_t launch_quantize_batch(const QuantJob* jobs, int n_jobs, uint32_t* status,
+                                  cudaStream_t st);
 cudaError_t launch_softedge_encode(const void* src, bool f16, int64_t n, float scale,
                                    float lo, float hi, int log2_ratio, uint8_t* codes,
                                    uint32_t* status, cudaStream_t st);

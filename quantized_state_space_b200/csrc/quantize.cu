@@ -228,6 +228,54 @@ __global__ void __launch_bounds__(stream::kThreads)
   flag_status(status, flags);
 }
 
+// Several static quantizations in one launch (same dtype, path and index
+// width): job k owns CTAs [cta_beg, cta_end) of the grid and runs the
+// pipeline over its tensor as CTA (blockIdx.x - cta_beg) of that range.
+constexpr int kMaxJobs = kMaxQuantJobs;
+template <typename Idx>
+struct QJob {
+  const void* src;
+  Idx n, mid;
+  Geo<Idx> geo;
+  const int32_t* gmap;
+  int32_t n_groups;
+  const float* scales;
+  int8_t* q;
+  int cta_beg, cta_end;
+};
+template <typename Idx>
+struct QJobs {
+  QJob<Idx> j[kMaxJobs];
+  int n;
+};
+
+template <bool kF16, int kPath, typename Idx>
+__global__ void __launch_bounds__(stream::kThreads)
+    quant_batch_kernel(const __grid_constant__ QJobs<Idx> jobs, uint32_t* status) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  __shared__ float2 tab[kMaxTab];
+  __shared__ int ug_s[kPath == kPathCol ? kMaxU : 1];
+  int k = 0;
+  while (k + 1 < jobs.n && (int)blockIdx.x >= jobs.j[k].cta_end) ++k;
+  const QJob<Idx>& J = jobs.j[k];
+  fill_tab(J.scales, J.n_groups, tab);
+  const int* ugrp = kPath == kPathCol ? fill_ugrp(J.gmap, (uint64_t)J.mid, ug_s) : nullptr;
+  uint32_t flags = 0;
+  stream::run_part<kF16, Idx>(
+      J.src, J.n, smem, (Idx)((int)blockIdx.x - J.cta_beg), (Idx)(J.cta_end - J.cta_beg),
+      [&](const float(&x)[kVec], Idx e0) {
+        quant_vec<kF16, kPath, Idx>(x, e0, J.geo, J.gmap, J.n_groups, J.scales, tab, ugrp, J.q,
+                                    flags);
+      },
+      [&](float v, Idx e) {
+        const int g = __ldg(J.gmap + J.geo.mid_of(e));
+        const bool okg = (unsigned)g < (unsigned)J.n_groups;
+        J.q[e] = (int8_t)quant_elem(v, okg ? __ldg(J.scales + g) : 0.0f, 0.0f, okg, flags);
+      },
+      flags);
+  flag_status(status, flags);
+}
+
 // Per-group max |v| into `acc` (the scales buffer viewed as uint32 bit
 // patterns: for non-negative floats the unsigned order is the float order).
 template <bool kF16, int kPath, typename Idx>
@@ -484,6 +532,93 @@ cudaError_t launch_quantize(const void* src, bool f16, int64_t outer, int64_t mi
                                           absmax, scales, q, status, st)
              : quantize_p<false, uint64_t>(src, n, (uint64_t)mid, (uint64_t)inner, gmap, n_groups,
                                            absmax, scales, q, status, st);
+}
+
+namespace {
+
+int path_of(int64_t mid, int64_t inner) {
+  return inner % kVec == 0 ? kPathRow : (inner == 1 && mid % kVec == 0 ? kPathCol : kPathGen);
+}
+
+// one launch for jobs idx[0..m) (same dtype, path and index width); CTAs in
+// proportion to each job's tiles, one at least
+template <bool kF16, int kPath, typename Idx>
+cudaError_t batch_t(const QuantJob* jobs, const int* idx, int m, uint32_t* status,
+                    cudaStream_t st) {
+  QJobs<Idx> J{};
+  J.n = m;
+  uint64_t tiles[kMaxJobs], total = 0;
+  for (int i = 0; i < m; ++i) {
+    const QuantJob& q = jobs[idx[i]];
+    const uint64_t n = (uint64_t)q.outer * (uint64_t)q.mid * (uint64_t)q.inner;
+    tiles[i] = n / stream::kTileElems;
+    total += tiles[i];
+  }
+  const uint64_t budget = (uint64_t)sm_count() * stream::kCtasPerSm;
+  int beg = 0;
+  for (int i = 0; i < m; ++i) {
+    const QuantJob& q = jobs[idx[i]];
+    const uint64_t n = (uint64_t)q.outer * (uint64_t)q.mid * (uint64_t)q.inner;
+    uint64_t c = total ? (budget * tiles[i] + total / 2) / total : 1;
+    c = c < 1 ? 1 : (c > tiles[i] && tiles[i] > 0 ? tiles[i] : c);
+    QJob<Idx>& d = J.j[i];
+    d.src = q.src;
+    d.n = (Idx)n;
+    d.mid = (Idx)q.mid;
+    d.geo = make_geo((Idx)q.mid, (Idx)q.inner);
+    d.gmap = q.gmap;
+    d.n_groups = q.n_groups;
+    d.scales = q.scales;
+    d.q = q.q;
+    d.cta_beg = beg;
+    beg += (int)c;
+    d.cta_end = beg;
+  }
+  auto kern = quant_batch_kernel<kF16, kPath, Idx>;
+  constexpr size_t smem = (size_t)acc_smem_offset<kF16>();
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  kern<<<(unsigned)beg, stream::kThreads, smem, st>>>(J, status);
+  return cudaGetLastError();
+}
+
+template <bool kF16, typename Idx>
+cudaError_t batch_p(int path, const QuantJob* jobs, const int* idx, int m, uint32_t* status,
+                    cudaStream_t st) {
+  if (path == kPathRow) return batch_t<kF16, kPathRow, Idx>(jobs, idx, m, status, st);
+  if (path == kPathCol) return batch_t<kF16, kPathCol, Idx>(jobs, idx, m, status, st);
+  return batch_t<kF16, kPathGen, Idx>(jobs, idx, m, status, st);
+}
+
+}  // namespace
+
+cudaError_t launch_quantize_batch(const QuantJob* jobs, int n_jobs, uint32_t* status,
+                                  cudaStream_t st) {
+  // group the non-empty jobs by (dtype, path, index width): one launch each
+  bool done[kMaxJobs] = {};
+  for (int a = 0; a < n_jobs; ++a) {
+    const uint64_t na = (uint64_t)jobs[a].outer * (uint64_t)jobs[a].mid * (uint64_t)jobs[a].inner;
+    if (done[a] || na == 0) continue;
+    const int pa = path_of(jobs[a].mid, jobs[a].inner);
+    const bool wa = na + 64 >= (1ull << 32);
+    int idx[kMaxJobs], m = 0;
+    for (int b = a; b < n_jobs; ++b) {
+      const uint64_t nb =
+          (uint64_t)jobs[b].outer * (uint64_t)jobs[b].mid * (uint64_t)jobs[b].inner;
+      if (done[b] || nb == 0 || jobs[b].f16 != jobs[a].f16 ||
+          path_of(jobs[b].mid, jobs[b].inner) != pa || (nb + 64 >= (1ull << 32)) != wa)
+        continue;
+      idx[m++] = b;
+      done[b] = true;
+    }
+    const cudaError_t e =
+        wa ? (jobs[a].f16 ? batch_p<true, uint64_t>(pa, jobs, idx, m, status, st)
+                          : batch_p<false, uint64_t>(pa, jobs, idx, m, status, st))
+           : (jobs[a].f16 ? batch_p<true, uint32_t>(pa, jobs, idx, m, status, st)
+                          : batch_p<false, uint32_t>(pa, jobs, idx, m, status, st));
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
 }
 
 cudaError_t launch_group_absmax(const void* src, bool f16, int64_t outer, int64_t mid,

@@ -124,12 +124,14 @@ __device__ __forceinline__ float global1(const void* src, Idx e) {
   return static_cast<const float*>(src)[e];
 }
 
-// Runs the pipeline over src[0, n).  Every thread of the CTA (kThreads) must
-// call it.  vec(x, e0) consumes the 16 elements e0..e0+15; one(v, e) a single
-// element of the ragged end.  Returns with every copy of this CTA complete.
+// Runs the pipeline over src[0, n) as CTA c of G working on it (tile j of
+// the CTA is tile c + j G).  Every thread of the CTA (kThreads) must call it.
+// vec(x, e0) consumes the 16 elements e0..e0+15; one(v, e) a single element
+// of the ragged end.  Returns with every copy of this CTA complete.
 template <bool kF16, typename Idx, class Vec, class One>
-__device__ __forceinline__ void run(const void* __restrict__ src, Idx n, uint8_t* smem, Vec&& vec,
-                                    One&& one, uint32_t& flags) {
+__device__ __forceinline__ void run_part(const void* __restrict__ src, Idx n, uint8_t* smem,
+                                         const Idx c, const Idx G, Vec&& vec, One&& one,
+                                         uint32_t& flags) {
   constexpr int kEsz = kF16 ? 2 : 4;
   using C = Cfg<kEsz>;
   constexpr int S = C::kStages;
@@ -138,7 +140,6 @@ __device__ __forceinline__ void run(const void* __restrict__ src, Idx n, uint8_t
   volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(empty + S);
   const int tid = threadIdx.x;
   const Idx ntiles = n / (Idx)kTileElems;
-  const Idx G = (Idx)gridDim.x, c = (Idx)blockIdx.x;
   const Idx J = c < ntiles ? (ntiles - c + G - 1) / G : 0;  // full tiles of this CTA
 
   if (tid == 0) {
@@ -223,6 +224,13 @@ __device__ __forceinline__ void run(const void* __restrict__ src, Idx n, uint8_t
       if (!tc::mbar_wait(full + (int)(j % S), (uint32_t)((j / S) & 1), kWaitLimit))
         flags |= SSMQ_DEV_TIMEOUT;
   }
+}
+
+// The whole grid on src[0, n).
+template <bool kF16, typename Idx, class Vec, class One>
+__device__ __forceinline__ void run(const void* __restrict__ src, Idx n, uint8_t* smem, Vec&& vec,
+                                    One&& one, uint32_t& flags) {
+  run_part<kF16, Idx>(src, n, smem, (Idx)blockIdx.x, (Idx)gridDim.x, vec, one, flags);
 }
 
 template <int kEsz>

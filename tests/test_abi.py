@@ -154,6 +154,29 @@ def test_ssd_validation(L):
         assert S(ws=FAKE + 16, nb=need) == N.ERR_ALIGNMENT
 
 
+def test_quantize_batch_validation(L):
+    J = N.QuantJob
+    ok = dict(src=FAKE, dtype=N.F16, outer=2, mid=4, inner=16, group_of_mid=FAKE, n_groups=2,
+              scales=FAKE, q_out=FAKE)
+
+    def S(n=1, **kw):
+        arr = (J * max(n, 1))()
+        for i in range(max(n, 1)):
+            arr[i] = N._fill(J, dict(ok, **kw))
+        return L.ssmq_quantize_groups_batch(arr, n, None, None)
+
+    assert L.ssmq_quantize_groups_batch(None, 1, None, None) == N.ERR_INVALID_ARG
+    assert S(n=0) == N.ERR_INVALID_ARG
+    assert S(n=9) == N.ERR_INVALID_ARG
+    assert S(dtype=7) == N.ERR_INVALID_ARG
+    assert S(n_groups=0) == N.ERR_INVALID_ARG
+    assert S(scales=None) == N.ERR_INVALID_ARG
+    assert S(outer=-1) == N.ERR_INVALID_ARG
+    assert S(q_out=None) == N.ERR_INVALID_ARG
+    assert S(src=FAKE + 8) == N.ERR_ALIGNMENT
+    assert S(outer=1 << 40, mid=1 << 20, inner=1 << 10) == N.ERR_INVALID_ARG
+
+
 def test_ssd_workspace_size_rule(L):
     """Operand blocks (64 KB per batch, group and 128-step tile), plus, when
     sequences may be cut into segments, one fp32 (P, N) state and one decay

@@ -83,6 +83,49 @@ def test_quantize_m130m_x_full_size(orc):
     np.testing.assert_array_equal(H(qg), qo)
 
 
+def _batch_job(rng, shape, dtype, k):
+    outer, mid, inner = shape
+    k = min(k, mid)
+    gmap = rng.integers(0, k, size=mid).astype(np.int32)
+    x = (rng.standard_normal(shape) * rng.choice([0.1, 1, 20], size=shape)).astype(dtype)
+    return x, gmap, k, synth.random_scales(rng, k, 0.01, 0.2)
+
+
+def test_quantize_batch_vs_oracle_and_single_calls(orc):
+    """One batch of eight jobs (row, column and general paths, binary16 and
+    fp32, ragged, tiny and empty tensors) gives the oracle's codes and the
+    same bytes as one call per job."""
+    rng = np.random.default_rng(4242)
+    specs = [((8, 1536, 256), np.float16), ((8, 16, 256), np.float16),
+             ((8, 16, 256), np.float16), ((777, 80, 1), np.float32), ((2, 37, 1003), np.float16),
+             ((1, 1, 7), np.float16), ((0, 5, 16), np.float16), ((3, 5, 2048), np.float32)]
+    jobs, data = [], []
+    for shape, dt in specs:
+        x, gmap, k, sc = _batch_job(rng, shape, dt, 8)
+        data.append((x, gmap, k, sc))
+        jobs.append((T(x), *shape, T(gmap), k, T(sc), None))
+    st = status_word()
+    outs = api.quantize_groups_batch(jobs, status=st)
+    assert int(H(st)[0]) == 0
+    for (x, gmap, k, sc), q, (shape, _) in zip(data, outs, specs):
+        qo, _, _ = orc.quantize_groups(x, *shape, gmap, k, orc.SCALE_STATIC, sc)
+        np.testing.assert_array_equal(H(q), qo.reshape(shape))
+        single, _ = api.quantize_groups(T(x), *shape, T(gmap), k, scales=T(sc))
+        np.testing.assert_array_equal(H(q), H(single))
+
+
+def test_quantize_batch_status_and_validation():
+    x = T(np.ones(64, np.float16))
+    st = status_word()
+    api.quantize_groups_batch([(x, 1, 64, 1, T(np.full(64, 3, np.int32)), 2,
+                                T(np.ones(2, np.float32)), None)], status=st)
+    torch.cuda.synchronize()
+    assert int(H(st)[0]) & N.DEV_BAD_GROUP
+    with pytest.raises(N.SSMQError):
+        api.quantize_groups_batch([(x, 1, 64, 1, T(np.zeros(64, np.int32)), 1,
+                                    T(np.ones(1, np.float32)), None)] * 9)
+
+
 # ---- soft-edge ---------------------------------------------------------------
 
 @pytest.mark.parametrize("s,lo,hi,r", [(0.05, 0.1, 3.0, 2), (1.0 / 63, 0.02, 1.0, 2),
