@@ -553,9 +553,9 @@ def setup_softedge(torch, dev):
     def enc():
         api.softedge_encode(x, s, lo, hi, 2, out=codes)
 
-    def quant_bc():
-        api.quantize_groups(B, b, G * N, L, smap, G * N // gs, scales=bs_t, out=Bq)
-        api.quantize_groups(C, b, G * N, L, smap, G * N // gs, scales=cs_t, out=Cq)
+    def quant_bc():  # B and C in one batched launch
+        api.quantize_groups_batch([(B, b, G * N, L, smap, G * N // gs, bs_t, Bq),
+                                   (C, b, G * N, L, smap, G * N // gs, cs_t, Cq)])
 
     def scan():
         api.selective_scan(codes, dt, A, Bq, Cq, bs_t, cs_t, gs, se_scale=s, D=D, z=z, y=y,
@@ -621,10 +621,10 @@ def setup_ssd(torch, dev):
     y = torch.empty(x.shape, dtype=torch.float16, device=dev)
     hf = torch.empty((b, H, P, N), dtype=torch.float32, device=dev)
 
-    def quant():
-        api.quantize_groups(x, b * L, H * P, 1, grp_t, k, scales=xs_t, out=xq)
-        api.quantize_groups(B, b * L, G * N, 1, smap, G * N // gs, scales=bs_t, out=Bq)
-        api.quantize_groups(C, b * L, G * N, 1, smap, G * N // gs, scales=cs_t, out=Cq)
+    def quant():  # x, B and C in one batched launch
+        api.quantize_groups_batch([(x, b * L, H * P, 1, grp_t, k, xs_t, xq),
+                                   (B, b * L, G * N, 1, smap, G * N // gs, bs_t, Bq),
+                                   (C, b * L, G * N, 1, smap, G * N // gs, cs_t, Cq)])
 
     def ssd():
         api.ssd_chunk_scan(xq, dt, A, Bq, Cq, bs_t, cs_t, gs, chunk=dm["chunk"], x_group=grp_t,
