@@ -105,16 +105,19 @@ __device__ __forceinline__ uint32_t pack4(int a, int b, int c, int d) {
          ((uint32_t)(d & 0xFF) << 24);
 }
 
-// Branch-free fast route for 16 elements sharing one valid (s, rs) (the
-// argument of quant_rne_fast, in packed fp32x2 arithmetic): the code byte of
+// Branch-free fast route for 16 elements whose halves each share one valid
+// (s, rs) (the argument of quant_rne_fast, in packed fp32x2 arithmetic): the code byte of
 // each element is the low byte of m = fl32(clamp(v rs) + 1.5 2^23), which
 // holds 0x4B400000 + k for the integer k = rne(clamp(v rs)).  Two running
 // reductions replace per-element tests: the largest |y - (m - 1.5 2^23)|
 // (at least 0.5 - 2^-14 only when some element lies within 2^-14 of a tie)
 // and the sum of v * 0 (NaN exactly when some v is not finite).  Returns false
 // in either case; the caller then redoes the vector element by element.
-__device__ __forceinline__ bool quant16_fast(const float (&x)[kVec], float rs, uint4& out) {
-  const float2 r2 = make_float2(rs, rs), mg = make_float2(12582912.0f, 12582912.0f);
+__device__ __forceinline__ bool quant16_fast(const float (&x)[kVec], float rs0, float rs1,
+                                             uint4& out) {
+  // rs0 for elements 0-7, rs1 for 8-15 (two groups of 8 columns)
+  const float2 ra = make_float2(rs0, rs0), rb = make_float2(rs1, rs1);
+  const float2 mg = make_float2(12582912.0f, 12582912.0f);
   const float2 zero = make_float2(0.0f, 0.0f);
   float2 nf = zero;
   float dmax = 0.0f;
@@ -122,7 +125,7 @@ __device__ __forceinline__ bool quant16_fast(const float (&x)[kVec], float rs, u
 #pragma unroll
   for (int i = 0; i < kVec; i += 2) {
     const float2 xv = make_float2(x[i], x[i + 1]);
-    float2 y = fmul2(xv, r2);
+    float2 y = fmul2(xv, i < kVec / 2 ? ra : rb);
     y.x = fminf(fmaxf(y.x, -127.0f), 127.0f);
     y.y = fminf(fmaxf(y.y, -127.0f), 127.0f);
     const float2 m = fadd2(y, mg);
@@ -146,16 +149,19 @@ __device__ __forceinline__ void quant_vec(const float (&x)[kVec], Idx e0, const 
                                           const float* __restrict__ scales, const float2* tab,
                                           const int* ugrp, int8_t* __restrict__ q,
                                           uint32_t& flags) {
-  int gu = -1;  // one group for the whole vector, if known
+  int gu = -1, gv = -1;  // one group for each half of the vector, if known
   if (kPath == kPathRow) {
-    gu = __ldg(gmap + geo.mid_of(e0));
+    gu = gv = __ldg(gmap + geo.mid_of(e0));
   } else if (kPath == kPathCol && ugrp) {
-    gu = ugrp[geo.col_of(e0) >> 4];
+    const uint32_t u = (uint32_t)(geo.col_of(e0) >> 3);
+    gu = ugrp[u];
+    gv = ugrp[u + 1];
   }
-  if ((unsigned)gu < (unsigned)n_groups) {
-    const float2 sr = tab_get(tab, scales, gu, n_groups);
+  if ((unsigned)gu < (unsigned)n_groups && (unsigned)gv < (unsigned)n_groups) {
+    const float2 sa = tab_get(tab, scales, gu, n_groups);
+    const float2 sb = gv == gu ? sa : tab_get(tab, scales, gv, n_groups);
     uint4 o;
-    if (sr.y != 0.0f && quant16_fast(x, sr.y, o)) {
+    if (sa.y != 0.0f && sb.y != 0.0f && quant16_fast(x, sa.y, sb.y, o)) {
       *reinterpret_cast<uint4*>(q + e0) = o;
       return;
     }
@@ -163,8 +169,9 @@ __device__ __forceinline__ void quant_vec(const float (&x)[kVec], Idx e0, const 
   int r[kVec];
 #pragma unroll
   for (int i = 0; i < kVec; ++i) {
-    const int g = gu >= 0 || kPath == kPathRow
-                      ? gu
+    const int gh = i < kVec / 2 ? gu : gv;
+    const int g = gh >= 0 || kPath == kPathRow
+                      ? gh
                       : (kPath == kPathCol ? __ldg(gmap + geo.col_of(e0) + i)
                                            : __ldg(gmap + geo.mid_of(e0 + i)));
     const bool okg = (unsigned)g < (unsigned)n_groups;
@@ -186,16 +193,18 @@ __host__ __device__ constexpr int acc_smem_offset() {
   return (stream::smem_bytes<kF16 ? 2 : 4>() + 15) / 16 * 16;
 }
 
-// Column path (inner == 1, mid % 16 == 0): groups of 16 consecutive columns
-// that share one group id are marked in a per-CTA table (-1 otherwise).
-constexpr int kMaxU = 1024;
+// Column path (inner == 1, mid % 16 == 0): groups of 8 consecutive columns
+// that share one group id are marked in a per-CTA table (-1 otherwise); a
+// vector's two halves look up their own entry.
+constexpr int kMaxU = 2048;
 __device__ __forceinline__ const int* fill_ugrp(const int32_t* gmap, uint64_t mid, int* ug) {
-  const uint64_t nu = mid / kVec;
+  constexpr int kW = kVec / 2;
+  const uint64_t nu = mid / kW;
   if (nu > (uint64_t)kMaxU) return nullptr;
   for (uint64_t u = threadIdx.x; u < nu; u += blockDim.x) {
-    const int g0 = __ldg(gmap + u * kVec);
+    const int g0 = __ldg(gmap + u * kW);
     bool same = true;
-    for (int i = 1; i < kVec; ++i) same &= __ldg(gmap + u * kVec + i) == g0;
+    for (int i = 1; i < kW; ++i) same &= __ldg(gmap + u * kW + i) == g0;
     ug[u] = same ? g0 : -1;
   }
   __syncthreads();
@@ -554,13 +563,31 @@ cudaError_t batch_t(const QuantJob* jobs, const int* idx, int m, uint32_t* statu
     tiles[i] = n / stream::kTileElems;
     total += tiles[i];
   }
+  // one resident round of CTAs: floor shares (one at least), the rest to the
+  // jobs with the most tiles per CTA; never more CTAs than tiles (but one)
   const uint64_t budget = (uint64_t)sm_count() * stream::kCtasPerSm;
+  uint64_t cta[kMaxJobs], used = 0;
+  for (int i = 0; i < m; ++i) {
+    cta[i] = total ? budget * tiles[i] / total : 1;
+    if (cta[i] < 1) cta[i] = 1;
+    if (tiles[i] > 0 && cta[i] > tiles[i]) cta[i] = tiles[i];
+    used += cta[i];
+  }
+  while (used < budget) {
+    int best = -1;
+    for (int i = 0; i < m; ++i)
+      if (cta[i] < tiles[i] &&
+          (best < 0 || tiles[i] * cta[best] > tiles[best] * cta[i]))
+        best = i;
+    if (best < 0) break;
+    ++cta[best];
+    ++used;
+  }
   int beg = 0;
   for (int i = 0; i < m; ++i) {
     const QuantJob& q = jobs[idx[i]];
     const uint64_t n = (uint64_t)q.outer * (uint64_t)q.mid * (uint64_t)q.inner;
-    uint64_t c = total ? (budget * tiles[i] + total / 2) / total : 1;
-    c = c < 1 ? 1 : (c > tiles[i] && tiles[i] > 0 ? tiles[i] : c);
+    const uint64_t c = cta[i];
     QJob<Idx>& d = J.j[i];
     d.src = q.src;
     d.n = (Idx)n;

@@ -43,6 +43,23 @@ def test_quantize_absmax(orc, shape):
     np.testing.assert_array_equal(H(qg), qo)
 
 
+@pytest.mark.parametrize("dtype", [np.float16, np.float32])
+def test_quantize_column_groups_of_8(orc, dtype):
+    """Column path with 8-column groups (Mamba-2 B/C: one scale per 8
+    states) and a map whose 8-column blocks are partly mixed: each half of a
+    16-element vector takes its own scale, mixed blocks go element by element."""
+    rng = np.random.default_rng(88)
+    outer, mid = 300, 128
+    for gmap in (np.arange(mid, dtype=np.int32) // 8,
+                 np.where(np.arange(mid) % 24 < 20, np.arange(mid) // 8, 3).astype(np.int32)):
+        k = int(gmap.max()) + 1
+        x = (rng.standard_normal((outer, mid)) * 4).astype(dtype)
+        sc = synth.random_scales(rng, k, 0.01, 0.2)
+        qg, _ = api.quantize_groups(T(x), outer, mid, 1, T(gmap), k, scales=T(sc))
+        qo, _, _ = orc.quantize_groups(x, outer, mid, 1, gmap, k, orc.SCALE_STATIC, sc)
+        np.testing.assert_array_equal(H(qg), qo)
+
+
 def test_quantize_all_f16_patterns(orc):
     bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
     x = bits.view(np.float16).copy()
