@@ -88,6 +88,9 @@ SEG_CASES = [
     (1, 128 * 3 + 1, 1, 1, True, True, 0, None),      # last segment a single step
     (2, 1024, 80, 4, True, False, 0,                  # 160 sequences: whole ones and cut ones
      [0, 1, 77, 100, 147, 148, 150, 155, 159]),
+    (1, 128 * 7 + 3, 2, 1, True, True, 0, None, "softedge"),  # soft-edge x codes, cut
+    (2, 512, 74, 2, False, True, 0, [0, 73, 74, 147]),  # 148 sequences: one full round, no cut
+    (1, 128 * 6, 2, 1, True, True, 64, None),         # max_segments above the plan's cap
 ]
 
 
@@ -95,8 +98,9 @@ SEG_CASES = [
 def test_ssd_segments_vs_oracle(orc, ci):
     """Sequences cut into segments (the segment start states carried by the
     second kernel) against the oracle, and against one pass per sequence."""
-    b, L, Hh, G, gate, h0, ms, units = SEG_CASES[ci]
-    p = ssd_problem(490 + ci, b, L, Hh, 64, 128, G=G, gate=gate, h0=h0, bias=True)
+    b, L, Hh, G, gate, h0, ms, units = SEG_CASES[ci][:8]
+    fmt = SEG_CASES[ci][8] if len(SEG_CASES[ci]) > 8 else "int8"
+    p = ssd_problem(490 + ci, b, L, Hh, 64, 128, G=G, gate=gate, h0=h0, bias=True, x_format=fmt)
     st = status_word()
     y, hf = gpu_ssd(p, max_segments=ms, status=st)
     assert int(H(st)[0]) == 0
