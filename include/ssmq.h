@@ -398,11 +398,44 @@ typedef struct {
                                to 32 segments (see above); n > 1: up to n;
                                1: one pass per sequence.  The workspace size
                                depends on it, on y and on y_q. */
+  float* dec_final;         /* (b, H) fp32 output or NULL: the sequence's total
+                               log2 decay, sum_t delta_t A_h log2(e) (binary32,
+                               summed per 128-step tile in step order, the
+                               tiles in order) -- exp2 of it multiplies the
+                               state carried across the call */
 } ssmq_ssd_args;
 
 size_t ssmq_ssd_workspace_size(const ssmq_ssd_args* args);
 ssmq_status ssmq_ssd_chunk_scan_w8(const ssmq_ssd_args* args, void* workspace,
                                    size_t ws_bytes, void* stream);
+
+/*
+ * Sequence sharding: a long sequence cut into consecutive slices (one per
+ * device, say).  The pages describe no such split; it follows from the
+ * recurrence (Quamba2 abstract, the selective SSM) being linear in the state:
+ * a slice scanned from a zero state (h0 = NULL) gives y and h_final of its
+ * own inputs; the state h_carry it should have started from adds
+ * exp(S_t) C_t h_carry to y_t (S_t the decay from the slice's start through
+ * step t; gated like y) and exp(S_L) h_carry to h_final.
+ *
+ * ssmq_state_chain: h_out[u] = fold over parts q = 0 .. n_parts - 1 of
+ *   h <- exp2(dec[q][u]) h + h_end[q][u], from h = 0.  h_end: device fp32
+ *   [n_parts][units][elems], dec: device fp32 [n_parts][units] (the slices'
+ *   h_final and dec_final, in sequence order), h_out: device fp32
+ *   [units][elems].  A slice's carry-in is the chain over the slices before
+ *   it (the first slice runs with the true h0 and needs none).
+ * ssmq_ssd_carry_in: adds h_carry's contribution (above) to args->y and, when
+ *   given, args->h_final, for the inputs of args (the same arguments as the
+ *   ssmq_ssd_chunk_scan_w8 call that produced them; y must not be NULL, y_q
+ *   must be NULL; h0, dec_final and max_segments are ignored).  y is rounded
+ *   to binary16 once more.  h_carry: device fp32 (b, H, P, N).  workspace:
+ *   at least ssmq_ssd_workspace_size(args) bytes (the operand blocks are
+ *   rebuilt).
+ */
+ssmq_status ssmq_state_chain(const float* h_end, const float* dec, int32_t n_parts,
+                             int64_t units, int64_t elems, float* h_out, void* stream);
+ssmq_status ssmq_ssd_carry_in(const ssmq_ssd_args* args, const float* h_carry,
+                              void* workspace, size_t ws_bytes, void* stream);
 
 /* ------------------------------------------------------------------------ */
 /* Single-token decode state update (Mamba-2 form)                           */

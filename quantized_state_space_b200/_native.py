@@ -50,7 +50,7 @@ class SSDArgs(C.Structure):
                 ("A", _vp), ("D", _vp), ("z", _vp), ("B", _vp), ("C", _vp), ("B_scale", _vp),
                 ("C_scale", _vp), ("h0", _vp), ("y", _vp), ("h_final", _vp), ("status", _vp), ("y_q", _vp),
                 ("y_group", _vp), ("y_scale", _vp), ("n_y_groups", _i32),
-                ("max_segments", _i32)]
+                ("max_segments", _i32), ("dec_final", _vp)]
 
 
 class DecodeArgs(C.Structure):
@@ -80,6 +80,8 @@ class QuantJob(C.Structure):
 
 SIGNATURES = {
     "ssmq_quantize_groups_batch": (_i32, [C.POINTER(QuantJob), _i32, _vp, _vp]),
+    "ssmq_state_chain": (_i32, [_vp, _vp, _i32, _i64, _i64, _vp, _vp]),
+    "ssmq_ssd_carry_in": (_i32, [C.c_void_p, _vp, _vp, C.c_size_t, _vp]),
     "ssmq_quantize_groups": (_i32, [_vp, _i32, _i64, _i64, _i64, _vp, _i32, _i32, _vp, _vp,
                                     _vp, _vp]),
     "ssmq_softedge_encode": (_i32, [_vp, _i32, _i64, _f32, _f32, _f32, _i32, _vp, _vp, _vp]),
@@ -219,6 +221,17 @@ def ssmq_ssd_workspace_size(**fields):
 def ssmq_ssd_chunk_scan_w8(workspace=None, ws_bytes=0, stream=None, **fields):
     a = _fill(SSDArgs, fields)
     _check(lib().ssmq_ssd_chunk_scan_w8(C.byref(a), ptr(workspace), ws_bytes, _stream(stream)))
+
+
+def ssmq_ssd_carry_in(h_carry, workspace=None, ws_bytes=0, stream=None, **fields):
+    a = _fill(SSDArgs, fields)
+    _check(lib().ssmq_ssd_carry_in(C.addressof(a), ptr(h_carry), ptr(workspace), ws_bytes,
+                                   _stream(stream)))
+
+
+def ssmq_state_chain(h_end, dec, n_parts, units, elems, h_out, stream=None):
+    _check(lib().ssmq_state_chain(ptr(h_end), ptr(dec), n_parts, units, elems, ptr(h_out),
+                                  _stream(stream)))
 
 
 def ssmq_state_update_w8(stream=None, **fields):

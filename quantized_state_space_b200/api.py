@@ -117,36 +117,78 @@ def selective_scan(x, dt, A, B, C, B_scale, C_scale, state_group_size, *, x_grou
     return (y, h_final, y_q) if yf else (y, h_final)
 
 
-def ssd_chunk_scan(x, dt, A, B, C, B_scale, C_scale, state_group_size, *, chunk=256,
-                   x_group=None, x_scale=None, se_scale=0.0, se_log2_ratio=2, D=None, z=None,
-                   dt_bias=None, dt_softplus=True, h0=None, y=None, h_final=None,
-                   return_state=True, y_group=None, y_scale=None, y_q=None, want_y=True,
-                   max_segments=0, workspace=None, status=None):
-    """Mamba-2 SSD chunked scan.  x (b, L, H, P) int8 / soft-edge uint8;
-    dt (b, L, H) float16; B, C (b, L, G, N) int8.  Returns (y, h_final), or
-    (y, h_final, y_q) with the int8 output (y_group over the H * P channels).
-    max_segments = 1: one pass per sequence (byte-exact checkpoint / resume)."""
+def _ssd_call(x, dt, A, B, C, B_scale, C_scale, state_group_size, chunk, x_group, x_scale,
+              se_scale, se_log2_ratio, D, z, dt_bias, dt_softplus, h0, y, h_final,
+              max_segments, workspace, status, dec_final, yf):
+    """argument fields and an aligned workspace of an SSD call"""
     b, L, H, P = x.shape
     G, Nst = B.shape[2], B.shape[3]
-    _dev_check(x, dt, A, B, C, B_scale, C_scale, x_group, x_scale, D, z, dt_bias, h0)
-    y, y_q, yf = _y_fields((b, L, H, P), x.device, y_group, y_scale, y_q, want_y, y)
-    if h_final is None and return_state:
-        h_final = torch.empty((b, H, P, Nst), dtype=torch.float32, device=x.device)
     fields = dict(batch=b, seqlen=L, nheads=H, headdim=P, dstate=Nst, ngroups=G, chunk=chunk,
                   state_group_size=state_group_size,
                   **_x_fields(x, x_group, x_scale, se_scale, se_log2_ratio),
                   dt=dt, dt_bias=dt_bias, dt_softplus=int(bool(dt_softplus)), A=A, D=D, z=z,
                   B=B, C=C, B_scale=B_scale, C_scale=C_scale, h0=h0, y=y, h_final=h_final,
-                  status=status, max_segments=max_segments, **yf)
+                  status=status, max_segments=max_segments, dec_final=dec_final, **yf)
     ws = N.ssmq_ssd_workspace_size(**fields)
     if ws and workspace is None:
         workspace = torch.empty(ws + 256, dtype=torch.uint8, device=x.device)
-    wptr = None
-    if ws:
-        base = workspace.data_ptr()
-        wptr = (base + 255) // 256 * 256
+    wptr = (workspace.data_ptr() + 255) // 256 * 256 if ws else None
+    return fields, wptr, ws
+
+
+def ssd_chunk_scan(x, dt, A, B, C, B_scale, C_scale, state_group_size, *, chunk=256,
+                   x_group=None, x_scale=None, se_scale=0.0, se_log2_ratio=2, D=None, z=None,
+                   dt_bias=None, dt_softplus=True, h0=None, y=None, h_final=None,
+                   return_state=True, y_group=None, y_scale=None, y_q=None, want_y=True,
+                   max_segments=0, dec_final=None, workspace=None, status=None):
+    """Mamba-2 SSD chunked scan.  x (b, L, H, P) int8 / soft-edge uint8;
+    dt (b, L, H) float16; B, C (b, L, G, N) int8.  Returns (y, h_final), or
+    (y, h_final, y_q) with the int8 output (y_group over the H * P channels).
+    max_segments = 1: one pass per sequence (byte-exact checkpoint / resume).
+    dec_final: optional (b, H) float32 output, each sequence's total log2 decay."""
+    b, L, H, P = x.shape
+    Nst = B.shape[3]
+    _dev_check(x, dt, A, B, C, B_scale, C_scale, x_group, x_scale, D, z, dt_bias, h0, dec_final)
+    y, y_q, yf = _y_fields((b, L, H, P), x.device, y_group, y_scale, y_q, want_y, y)
+    if h_final is None and return_state:
+        h_final = torch.empty((b, H, P, Nst), dtype=torch.float32, device=x.device)
+    fields, wptr, ws = _ssd_call(x, dt, A, B, C, B_scale, C_scale, state_group_size, chunk,
+                                 x_group, x_scale, se_scale, se_log2_ratio, D, z, dt_bias,
+                                 dt_softplus, h0, y, h_final, max_segments, workspace, status,
+                                 dec_final, yf)
     N.ssmq_ssd_chunk_scan_w8(workspace=wptr, ws_bytes=ws, **fields)
     return (y, h_final, y_q) if yf else (y, h_final)
+
+
+def ssd_carry_in(x, dt, A, B, C, B_scale, C_scale, state_group_size, h_carry, y, *, chunk=256,
+                 x_group=None, x_scale=None, se_scale=0.0, se_log2_ratio=2, D=None, z=None,
+                 dt_bias=None, dt_softplus=True, h_final=None, workspace=None, status=None):
+    """Adds the contribution of the start state h_carry (b, H, P, N) to the y
+    (in place) and h_final (in place, if given) of an SSD call on the same
+    inputs that started from a zero state."""
+    _dev_check(x, dt, A, B, C, B_scale, C_scale, x_group, x_scale, D, z, dt_bias, h_carry, y,
+               h_final)
+    fields, wptr, ws = _ssd_call(x, dt, A, B, C, B_scale, C_scale, state_group_size, chunk,
+                                 x_group, x_scale, se_scale, se_log2_ratio, D, z, dt_bias,
+                                 dt_softplus, None, y, h_final, 0, workspace, status, None, {})
+    N.ssmq_ssd_carry_in(h_carry, workspace=wptr, ws_bytes=ws, **fields)
+    return y, h_final
+
+
+def state_chain(h_ends, decs):
+    """Fold of h <- exp2(dec_q) h + h_end_q over the parts q in order, from a
+    zero state.  h_ends: sequence of equal-shape float32 tensors (units...,
+    elems...) or one stacked tensor; decs likewise with one value per unit."""
+    he = torch.stack(list(h_ends)) if not torch.is_tensor(h_ends) else h_ends
+    dc = torch.stack(list(decs)) if not torch.is_tensor(decs) else decs
+    he, dc = he.contiguous(), dc.contiguous()
+    _dev_check(he, dc)
+    n_parts = he.shape[0]
+    units = dc[0].numel()
+    elems = he[0].numel() // max(units, 1)
+    out = torch.empty(he.shape[1:], dtype=torch.float32, device=he.device)
+    N.ssmq_state_chain(he, dc, n_parts, units, elems, out)
+    return out
 
 
 def state_update(state, x, dt, A, B, C, B_scale, C_scale, state_group_size, *, x_group=None,

@@ -348,9 +348,13 @@ size_t ssmq_ssd_workspace_size(const ssmq_ssd_args* a) {
   return ssmq::ssd_workspace_bytes(*a);
 }
 
-ssmq_status ssmq_ssd_chunk_scan_w8(const ssmq_ssd_args* a, void* workspace, size_t ws_bytes,
-                                   void* stream) {
-  const char* fn = "ssmq_ssd_chunk_scan_w8";
+namespace {
+
+// validation shared by the SSD scan and its carry-in; `batch` or `nheads` 0
+// returns SSMQ_OK with *skip set (nothing to launch)
+ssmq_status check_ssd(const ssmq_ssd_args* a, void* workspace, size_t ws_bytes, const char* fn,
+                      bool* skip) {
+  *skip = false;
   REQUIRE(a != nullptr, SSMQ_ERR_INVALID_ARG, "%s: args is NULL", fn);
   REQUIRE(a->batch >= 0 && a->seqlen >= 0 && a->nheads >= 0, SSMQ_ERR_INVALID_ARG,
           "%s: negative size", fn);
@@ -363,7 +367,10 @@ ssmq_status ssmq_ssd_chunk_scan_w8(const ssmq_ssd_args* a, void* workspace, size
   REQUIRE(a->state_group_size >= 1 && a->dstate % a->state_group_size == 0,
           SSMQ_ERR_INVALID_ARG, "%s: dstate must be a multiple of state_group_size", fn);
   REQUIRE(a->max_segments >= 0, SSMQ_ERR_INVALID_ARG, "%s: max_segments must be >= 0", fn);
-  if (a->batch == 0 || a->nheads == 0) return SSMQ_OK;
+  if (a->batch == 0 || a->nheads == 0) {
+    *skip = true;
+    return SSMQ_OK;
+  }
   const ssmq_status xs = check_x(a->x_format, a->x, a->x_group, a->x_scale, a->n_x_groups,
                                  a->se_log2_ratio, fn);
   if (xs != SSMQ_OK) return xs;
@@ -380,8 +387,47 @@ ssmq_status ssmq_ssd_chunk_scan_w8(const ssmq_ssd_args* a, void* workspace, size
           "%s: workspace of %zu bytes required (got %zu)", fn, need, ws_bytes);
   REQUIRE((reinterpret_cast<uintptr_t>(workspace) & 255u) == 0, SSMQ_ERR_ALIGNMENT,
           "%s: workspace must be 256-byte aligned", fn);
+  return SSMQ_OK;
+}
+
+}  // namespace
+
+ssmq_status ssmq_ssd_chunk_scan_w8(const ssmq_ssd_args* a, void* workspace, size_t ws_bytes,
+                                   void* stream) {
+  const char* fn = "ssmq_ssd_chunk_scan_w8";
+  bool skip;
+  CHECK(check_ssd(a, workspace, ws_bytes, fn, &skip));
+  if (skip) return SSMQ_OK;
   if (injected(fn)) return fail(SSMQ_ERR_CUDA, "%s: injected launch failure", fn);
   return finish(ssmq::launch_ssd(*a, workspace, (cudaStream_t)stream), fn);
+}
+
+ssmq_status ssmq_ssd_carry_in(const ssmq_ssd_args* a, const float* h_carry, void* workspace,
+                              size_t ws_bytes, void* stream) {
+  const char* fn = "ssmq_ssd_carry_in";
+  bool skip;
+  CHECK(check_ssd(a, workspace, ws_bytes, fn, &skip));
+  if (skip) return SSMQ_OK;
+  REQUIRE(a->y != nullptr && a->y_q == nullptr, SSMQ_ERR_INVALID_ARG,
+          "%s: needs the binary16 y (and no int8 y)", fn);
+  REQUIRE(h_carry != nullptr, SSMQ_ERR_INVALID_ARG, "%s: h_carry is NULL", fn);
+  REQUIRE(aligned16(h_carry), SSMQ_ERR_ALIGNMENT, "%s: h_carry must be 16-byte aligned", fn);
+  if (injected(fn)) return fail(SSMQ_ERR_CUDA, "%s: injected launch failure", fn);
+  return finish(ssmq::launch_ssd_carry_in(*a, h_carry, workspace, (cudaStream_t)stream), fn);
+}
+
+ssmq_status ssmq_state_chain(const float* h_end, const float* dec, int32_t n_parts,
+                             int64_t units, int64_t elems, float* h_out, void* stream) {
+  const char* fn = "ssmq_state_chain";
+  REQUIRE(n_parts >= 1, SSMQ_ERR_INVALID_ARG, "%s: n_parts must be >= 1", fn);
+  REQUIRE(units >= 0 && elems >= 0, SSMQ_ERR_INVALID_ARG, "%s: negative size", fn);
+  if (units == 0 || elems == 0) return SSMQ_OK;
+  REQUIRE(h_end && dec && h_out, SSMQ_ERR_INVALID_ARG, "%s: NULL tensor", fn);
+  REQUIRE(units <= INT64_MAX / elems / n_parts, SSMQ_ERR_INVALID_ARG, "%s: size overflow", fn);
+  if (injected(fn)) return fail(SSMQ_ERR_CUDA, "%s: injected launch failure", fn);
+  return finish(ssmq::launch_state_chain(h_end, dec, n_parts, units, elems, nullptr, h_out,
+                                         (cudaStream_t)stream),
+                fn);
 }
 
 ssmq_status ssmq_state_update_w8(const ssmq_decode_args* a, void* stream) {

@@ -56,5 +56,9 @@ int sm_count();
 
 size_t ssd_workspace_bytes(const ssmq_ssd_args& a);
 cudaError_t launch_ssd(const ssmq_ssd_args& a, void* ws, cudaStream_t st);
+cudaError_t launch_ssd_carry_in(const ssmq_ssd_args& a, const float* h_carry, void* ws,
+                                cudaStream_t st);
+cudaError_t launch_state_chain(const float* h_end, const float* dec, int n_parts, int64_t units,
+                               int64_t elems, const float* h_init, float* h_out, cudaStream_t st);
 
 }  // namespace ssmq

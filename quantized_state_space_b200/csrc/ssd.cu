@@ -135,6 +135,8 @@ struct SsdParams {
   int kseg, seg_tiles;
   float* seg_state;
   float* seg_dec;
+  float* dec_final;       // (b, H) total log2 decay of each sequence, or null
+  const float* h_carry;   // carry-in mode of the second kernel: (b, H, P, N)
 };
 
 // 2^e as an exact float for |e| < 126
@@ -902,6 +904,7 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_kernel(const SsdParams p) {
   float* fin = slot < 0 ? (p.h_final ? p.h_final + u * kP * kN : nullptr)
                         : p.seg_state + (int64_t)slot * kP * kN;
   if (slot >= 0 && tid == 0) p.seg_dec[slot] = s_tot;
+  if (slot < 0 && tid == 0 && p.dec_final) p.dec_final[u] = s_tot;
   if (fin) {
     float* stage = reinterpret_cast<float*>(smem + OFF_STATE);
     __syncthreads();
@@ -943,9 +946,12 @@ __global__ void __launch_bounds__(kThreads) ssd_fixup_kernel(const SsdParams p) 
   __shared__ uint32_t tmem_slot;
   __shared__ __align__(8) uint64_t bars[3];  // C' copies (two buffers), MMA
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int seg = 1 + (int)blockIdx.x;
+  // segments: CTA (seg - 1, sequence); carry-in mode (h_carry given): one CTA
+  // per sequence, its whole length, from the given start state
+  const bool carry = p.h_carry != nullptr;
+  const int seg = carry ? 0 : 1 + (int)blockIdx.x;
   const int64_t slot0 = (int64_t)blockIdx.y * p.kseg;  // first segment slot of the unit
-  const int64_t u = p.full + blockIdx.y;
+  const int64_t u = carry ? (int64_t)blockIdx.y : p.full + blockIdx.y;
   const int64_t H = p.H, L = p.L;
   const int64_t bb = u / H, hd = u % H;
   const int64_t g = hd * p.G / H;
@@ -963,8 +969,8 @@ __global__ void __launch_bounds__(kThreads) ssd_fixup_kernel(const SsdParams p) 
     tc::mbar_init(&bars[2], 1);
   }
   const uint8_t* ops_bg = p.ops + (bb * p.G + g) * p.ntiles * (int64_t)kOpTile;
-  const int64_t tile_beg = (int64_t)seg * p.seg_tiles;
-  const int64_t tile_end = min(p.ntiles, tile_beg + p.seg_tiles);
+  const int64_t tile_beg = carry ? 0 : (int64_t)seg * p.seg_tiles;
+  const int64_t tile_end = carry ? p.ntiles : min(p.ntiles, tile_beg + p.seg_tiles);
   // C' of the segment's tile i -> buffer i & 1 (its (i >> 1)-th copy)
   auto issue_c = [&](int64_t i) {
     stream::expect_tx(&bars[i & 1], (uint32_t)kOpBlock);
@@ -987,17 +993,27 @@ __global__ void __launch_bounds__(kThreads) ssd_fixup_kernel(const SsdParams p) 
     }
   }
   // h_start(seg) by the chain, elementwise; the last segment also forms h_final
-  {
+  // and the sequence's total decay.  Carry-in mode: h_start is given.
+  constexpr int kE = kP * kN / 4 / kThreads;  // float4 elements per thread
+  float4* st = reinterpret_cast<float4*>(smem + FX_ST);
+  if (carry) {
+    const float4* hc = reinterpret_cast<const float4*>(p.h_carry + u * kP * kN);
+#pragma unroll
+    for (int i = 0; i < kE; ++i) st[tid + kThreads * i] = hc[tid + kThreads * i];
+  } else {
     const float4* loc = reinterpret_cast<const float4*>(p.seg_state + slot0 * kP * kN);
     const float* dec = p.seg_dec + slot0;
     const bool last = seg == p.kseg - 1;
-    float4* st = reinterpret_cast<float4*>(smem + FX_ST);
-    constexpr int kE = kP * kN / 4 / kThreads;  // float4 elements per thread
     constexpr int64_t kStride = kP * kN / 4;   // float4 per state
     auto fma4 = [](float d, float4 h, float4 l) {
       return make_float4(fmaf(d, h.x, l.x), fmaf(d, h.y, l.y), fmaf(d, h.z, l.z),
                          fmaf(d, h.w, l.w));
     };
+    if (last && tid == 0 && p.dec_final) {
+      float tot = 0.0f;
+      for (int m = 0; m < p.kseg; ++m) tot += dec[m];
+      p.dec_final[u] = tot;
+    }
     // segment 0 ran from h0: its local state is already the true one
     float4 h[kE];
 #pragma unroll
@@ -1157,6 +1173,17 @@ __global__ void __launch_bounds__(kThreads) ssd_fixup_kernel(const SsdParams p) 
     __syncthreads();  // S and tensor memory free for the next tile
     tc::fence_after();
   }
+  // carry-in mode: h_final += exp(S over the sequence) h_carry
+  if (carry && p.h_final) {
+    const float d = ex2_sfu(cum);
+    float4* hf = reinterpret_cast<float4*>(p.h_final + u * kP * kN);
+#pragma unroll
+    for (int i = 0; i < kE; ++i) {
+      const float4 c = st[tid + kThreads * i], h = hf[tid + kThreads * i];
+      hf[tid + kThreads * i] = make_float4(fmaf(d, c.x, h.x), fmaf(d, c.y, h.y),
+                                           fmaf(d, c.z, h.z), fmaf(d, c.w, h.w));
+    }
+  }
   // copies still in flight (the loop was left early) land before the CTA exits
   if (tid == 0)
     for (int b = 0; b < 2; ++b)
@@ -1220,15 +1247,42 @@ size_t ssd_workspace_bytes(const ssmq_ssd_args& a) {
          (size_t)slots * (size_t)(kP * kN * 4 + 4);
 }
 
-cudaError_t launch_ssd(const ssmq_ssd_args& a, void* ws, cudaStream_t st) {
-  const int64_t units = a.batch * a.nheads;
-  if (units == 0) return cudaSuccess;
-  if (a.seqlen == 0) {
-    if (!a.h_final) return cudaSuccess;
-    const size_t bytes = sizeof(float) * (size_t)(units * a.headdim * a.dstate);
-    return a.h0 ? cudaMemcpyAsync(a.h_final, a.h0, bytes, cudaMemcpyDeviceToDevice, st)
-                : cudaMemsetAsync(a.h_final, 0, bytes, st);
+namespace {
+
+// h_out[u][e] = fold over parts q of h <- exp2(dec[q][u]) h + h_end[q][u][e],
+// from h = h_init[u][e] (0 when null); dec null means 0.
+__global__ void state_chain_kernel(const float* __restrict__ h_end, const float* __restrict__ dec,
+                                   int n_parts, int64_t units, int64_t elems,
+                                   const float* h_init, float* h_out) {
+  const int64_t n = units * elems;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t u = i / elems;
+    float h = h_init ? h_init[i] : 0.0f;
+    for (int q = 0; q < n_parts; ++q) {
+      const float d = dec ? ex2_sfu(__ldg(dec + (int64_t)q * units + u)) : 1.0f;
+      h = fmaf(d, h, __ldg(h_end + (int64_t)q * n + i));
+    }
+    h_out[i] = h;
   }
+}
+
+}  // namespace
+
+cudaError_t launch_state_chain(const float* h_end, const float* dec, int n_parts, int64_t units,
+                               int64_t elems, const float* h_init, float* h_out, cudaStream_t st) {
+  const int64_t n = units * elems;
+  if (n == 0) return cudaSuccess;
+  const int64_t want = (n + 255) / 256, cap = (int64_t)sm_count() * 8;
+  const int64_t blocks = want < cap ? want : cap;
+  state_chain_kernel<<<(unsigned)blocks, 256, 0, st>>>(h_end, dec, n_parts, units, elems, h_init,
+                                                       h_out);
+  return cudaGetLastError();
+}
+
+namespace {
+
+SsdParams make_params(const ssmq_ssd_args& a, void* ws) {
   SsdParams p{};
   p.L = a.seqlen;
   p.H = a.nheads;
@@ -1260,9 +1314,29 @@ cudaError_t launch_ssd(const ssmq_ssd_args& a, void* ws, cudaStream_t st) {
   p.y_scale = a.y_scale;
   p.n_y_groups = a.n_y_groups;
   p.h_final = a.h_final;
+  p.dec_final = a.dec_final;
   p.status = a.status;
   p.ntiles = (a.seqlen + kQ - 1) / kQ;
   p.ops = static_cast<const uint8_t*>(ws);
+  return p;
+}
+
+}  // namespace
+
+cudaError_t launch_ssd(const ssmq_ssd_args& a, void* ws, cudaStream_t st) {
+  const int64_t units = a.batch * a.nheads;
+  if (units == 0) return cudaSuccess;
+  if (a.seqlen == 0) {
+    if (a.dec_final) {
+      const cudaError_t e = cudaMemsetAsync(a.dec_final, 0, sizeof(float) * (size_t)units, st);
+      if (e != cudaSuccess) return e;
+    }
+    if (!a.h_final) return cudaSuccess;
+    const size_t bytes = sizeof(float) * (size_t)(units * a.headdim * a.dstate);
+    return a.h0 ? cudaMemcpyAsync(a.h_final, a.h0, bytes, cudaMemcpyDeviceToDevice, st)
+                : cudaMemsetAsync(a.h_final, 0, bytes, st);
+  }
+  SsdParams p = make_params(a, ws);
   const SegPlan sp = seg_plan(a, p.ntiles, sm_count());
   p.full = sp.full;
   p.kseg = sp.kseg;
@@ -1283,6 +1357,28 @@ cudaError_t launch_ssd(const ssmq_ssd_args& a, void* ws, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     ssd_fixup_kernel<<<dim3((unsigned)(sp.kseg - 1), (unsigned)sp.r), kThreads, kFixSmem, st>>>(p);
   }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_ssd_carry_in(const ssmq_ssd_args& a, const float* h_carry, void* ws,
+                                cudaStream_t st) {
+  const int64_t units = a.batch * a.nheads;
+  if (units == 0) return cudaSuccess;
+  if (a.seqlen == 0) {  // h_final += h_carry
+    if (!a.h_final) return cudaSuccess;
+    return launch_state_chain(h_carry, nullptr, 1, units, a.headdim * a.dstate, a.h_final,
+                              a.h_final, st);
+  }
+  SsdParams p = make_params(a, ws);
+  p.h0 = nullptr;
+  p.dec_final = nullptr;
+  p.h_carry = h_carry;
+  ssd_operand_kernel<<<dim3((unsigned)p.ntiles, (unsigned)(a.batch * a.ngroups)), kThreads, 0, st>>>(
+      p, static_cast<uint8_t*>(ws));
+  cudaError_t e = cudaFuncSetAttribute(ssd_fixup_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       kFixSmem);
+  if (e != cudaSuccess) return e;
+  ssd_fixup_kernel<<<dim3(1u, (unsigned)units), kThreads, kFixSmem, st>>>(p);
   return cudaGetLastError();
 }
 

@@ -177,6 +177,23 @@ def test_quantize_batch_validation(L):
     assert S(outer=1 << 40, mid=1 << 20, inner=1 << 10) == N.ERR_INVALID_ARG
 
 
+def test_sequence_sharding_validation(L):
+    assert L.ssmq_state_chain(FAKE, FAKE, 0, 4, 8, FAKE, None) == N.ERR_INVALID_ARG
+    assert L.ssmq_state_chain(FAKE, FAKE, 2, -1, 8, FAKE, None) == N.ERR_INVALID_ARG
+    assert L.ssmq_state_chain(None, FAKE, 2, 4, 8, FAKE, None) == N.ERR_INVALID_ARG
+    assert L.ssmq_state_chain(FAKE, FAKE, 2, 1 << 40, 1 << 30, FAKE, None) == N.ERR_INVALID_ARG
+    assert L.ssmq_state_chain(None, None, 2, 0, 8, None, None) == N.OK  # nothing to do
+    def S(hc=FAKE, **kw):
+        a = _ssd_args(**kw)  # kept alive across the call
+        return L.ssmq_ssd_carry_in(C.addressof(a), hc, FAKE, 1 << 40, None)
+
+    assert S(hc=None) == N.ERR_INVALID_ARG
+    assert S(hc=FAKE + 4) == N.ERR_ALIGNMENT
+    assert S(y=None, y_q=FAKE, y_group=FAKE, y_scale=FAKE, n_y_groups=1) == N.ERR_INVALID_ARG
+    assert S(headdim=32) == N.ERR_UNSUPPORTED
+    assert L.ssmq_ssd_carry_in(None, FAKE, FAKE, 0, None) == N.ERR_INVALID_ARG
+
+
 def test_ssd_workspace_size_rule(L):
     """Operand blocks (64 KB per batch, group and 128-step tile), plus, when
     sequences may be cut into segments, one fp32 (P, N) state and one decay

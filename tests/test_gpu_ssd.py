@@ -6,7 +6,7 @@ import numpy as np
 import pytest
 import torch
 
-from gpu_util import H, T, assert_scan_close, status_word, y_err, state_err
+from gpu_util import H, T, assert_scan_close, dev, status_word, y_err, state_err
 from problems import oracle_kwargs, ssd_problem
 from quantized_state_space_b200 import _native as N
 from quantized_state_space_b200 import api, calibrate, synth
@@ -199,3 +199,66 @@ def test_ssd_int8_y_bit_exact():
     assert y2 is None
     np.testing.assert_array_equal(H(yq2), H(yq))
     np.testing.assert_array_equal(H(hf2).view(np.uint32), H(hf).view(np.uint32))
+
+
+@pytest.mark.parametrize("cuts", [(0, 512), (0, 384, 768, 1000), (0, 127, 128, 900)])
+def test_ssd_sequence_sharded_vs_oracle(orc, cuts):
+    """Sequence sharding emulated in one process: each slice scanned from a
+    zero state (the first from h0) with its total decay, the summaries folded
+    by the state-chain kernel, each later slice's carried start state added
+    by the carry-in kernel; the concatenated y and the folded final state
+    against the oracle's unsplit scan."""
+    b, L, Hh = 2, 1100, 3
+    p = ssd_problem(940, b, L, Hh, 64, 128, G=1, gate=True, h0=True, bias=True)
+    yo, ho = oracle_ssd(orc, p)
+    bounds = list(cuts) + [L]
+    ys, h_ends, decs = [], [], []
+    for r in range(len(bounds) - 1):
+        sl = slice(bounds[r], bounds[r + 1])
+        q = dict(p)
+        for k in ("x", "dt", "z", "B", "C"):
+            q[k] = np.ascontiguousarray(p[k][:, sl])
+        args = (T(q["x"]), T(q["dt"]), T(q["A"]), T(q["B"]), T(q["C"]), T(q["B_scale"]),
+                T(q["C_scale"]), 8)
+        kw = dict(x_group=T(q["x_group"]), x_scale=T(q["x_scale"]), D=T(q["D"]), z=T(q["z"]),
+                  dt_bias=T(q["dt_bias"]))
+        dec = torch.empty((b, Hh), dtype=torch.float32, device=dev())
+        y, he = api.ssd_chunk_scan(*args, h0=T(p["h0"]) if r == 0 else None, dec_final=dec,
+                                   **kw)
+        # the total decay: sum_t delta_t A_h log2(e)
+        dt = q["dt"].astype(np.float64) + q["dt_bias"].astype(np.float64)
+        ref = (np.logaddexp(0.0, dt) * q["A"].astype(np.float64)).sum(axis=1) * np.log2(np.e)
+        np.testing.assert_allclose(H(dec), ref, rtol=2e-5, atol=1e-4)
+        if r > 0:
+            carry = api.state_chain(h_ends, decs)
+            api.ssd_carry_in(*args, carry, y, **kw)
+        ys.append(H(y).astype(np.float64))
+        h_ends.append(he)
+        decs.append(dec)
+    hf = H(api.state_chain(h_ends, decs))
+    y = np.concatenate(ys, axis=1)
+    assert_scan_close(y.transpose(0, 2, 1, 3).reshape(yo.shape), yo, hf.reshape(ho.shape), ho)
+
+
+def test_ssd_carry_in_h_final_and_dec_with_segments(orc):
+    """dec_final of sequences cut into segments (the second kernel sums the
+    segments' decays) and the carry-in's h_final update, on one call."""
+    b, L, Hh = 1, 128 * 9 + 5, 2
+    p = ssd_problem(950, b, L, Hh, 64, 128, gate=False, h0=False, bias=True)
+    args = (T(p["x"]), T(p["dt"]), T(p["A"]), T(p["B"]), T(p["C"]), T(p["B_scale"]),
+            T(p["C_scale"]), 8)
+    kw = dict(x_group=T(p["x_group"]), x_scale=T(p["x_scale"]), D=T(p["D"]),
+              dt_bias=T(p["dt_bias"]))
+    dec = torch.empty((b, Hh), dtype=torch.float32, device=dev())
+    y, hf = api.ssd_chunk_scan(*args, dec_final=dec, **kw)  # two sequences: cut
+    dt = p["dt"].astype(np.float64) + p["dt_bias"].astype(np.float64)
+    ref = (np.logaddexp(0.0, dt) * p["A"].astype(np.float64)).sum(axis=1) * np.log2(np.e)
+    np.testing.assert_allclose(H(dec), ref, rtol=2e-5, atol=1e-4)
+    rng = np.random.default_rng(951)
+    h_start = (rng.standard_normal((b, Hh, 64, 128)) * 0.1).astype(np.float32)
+    api.ssd_carry_in(*args, T(h_start), y, h_final=hf, **kw)
+    q = dict(p)
+    q["h0"] = h_start
+    yo, ho = oracle_ssd(orc, q)
+    assert_scan_close(H(y).astype(np.float64).transpose(0, 2, 1, 3).reshape(yo.shape), yo,
+                      H(hf).reshape(ho.shape), ho)

@@ -1,0 +1,112 @@
+"""Sequence sharding of the SSD scan (a slice per rank): the decomposition the
+GPU path implements, pinned on the CPU against the oracle's unsplit scan, and
+the summary exchange over gloo ranks."""
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+from problems import oracle_kwargs, ssd_problem
+
+
+def _total_log2_decay(p, sl):
+    """sum_t delta_t A_h log2(e) over the steps of slice sl, per (b, h)"""
+    dt = p["dt"][:, sl].astype(np.float64)
+    bias = 0.0 if p["dt_bias"] is None else p["dt_bias"].astype(np.float64)
+    delta = np.logaddexp(0.0, dt + bias)
+    return (delta * p["A"].astype(np.float64)).sum(axis=1) * np.log2(np.e)
+
+
+def _fold(h_ends, decs):
+    h = np.zeros_like(h_ends[0])
+    for he, d in zip(h_ends, decs):
+        h = np.exp2(d)[..., None, None] * h + he
+    return h
+
+
+def _slice(p, sl):
+    q = dict(p)
+    for k in ("x", "dt", "z", "B", "C"):
+        if q[k] is not None:
+            q[k] = np.ascontiguousarray(p[k][:, sl])
+    return q
+
+
+@pytest.mark.parametrize("cuts", [(0, 128, 300), (0, 77, 78, 200, 300)])
+def test_slices_fold_to_the_unsplit_scan(orc, cuts):
+    """Slices scanned from zero (the first from h0), folded with
+    h <- exp2(dec) h + h_end, give the unsplit final state; each slice's y
+    plus the y of its carried start state (the oracle's scan of the slice from
+    that state minus its scan from zero) is the unsplit y."""
+    b, L, H = 1, 300, 2
+    p = ssd_problem(930, b, L, H, 64, 128, gate=True, h0=True, bias=True)
+    yo, ho = orc.ssd_scan(p["x"], p["dt"], p["A"], p["B"], p["C"], p["B_scale"], p["C_scale"],
+                          8, **oracle_kwargs(p))
+    bounds = list(cuts) + [L]
+    h_ends, decs = [], []
+    for r in range(len(bounds) - 1):
+        sl = slice(bounds[r], bounds[r + 1])
+        q = _slice(p, sl)
+        if r > 0:
+            q["h0"] = None
+        kw = oracle_kwargs(q)
+        y0, he = orc.ssd_scan(q["x"], q["dt"], q["A"], q["B"], q["C"], q["B_scale"],
+                              q["C_scale"], 8, **kw)
+        if r > 0:
+            carry = _fold(h_ends, decs).reshape(b, H, 64, 128)
+            kw["h0"] = carry.astype(np.float32).astype(np.float64)
+            y1, _ = orc.ssd_scan(q["x"], q["dt"], q["A"], q["B"], q["C"], q["B_scale"],
+                                 q["C_scale"], 8, **kw)
+            kw["h0"] = np.zeros_like(kw["h0"])
+            y0z, _ = orc.ssd_scan(q["x"], q["dt"], q["A"], q["B"], q["C"], q["B_scale"],
+                                  q["C_scale"], 8, **kw)
+            y0 = y0 + (y1 - y0z)
+        np.testing.assert_allclose(y0, yo[:, sl], rtol=0, atol=2e-6 * np.abs(yo).max())
+        h_ends.append(he.reshape(b, H, 64, 128))
+        decs.append(_total_log2_decay(p, sl))
+    hf = _fold(h_ends, decs).reshape(ho.shape)
+    np.testing.assert_allclose(hf, ho, rtol=0, atol=1e-9 * np.abs(ho).max())
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=__import__("datetime").timedelta(seconds=60))
+    try:
+        from quantized_state_space_b200 import sharded
+        g = torch.Generator().manual_seed(100 + rank)
+        h_end = torch.randn(2, 3, 4, 5, generator=g)
+        dec = -torch.rand(2, 3, generator=g)
+        hs, ds = sharded.exchange(h_end, dec)
+        out[rank] = ([h.numpy() for h in hs], [d.numpy() for d in ds], h_end.numpy(),
+                     dec.numpy())
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_exchange_over_three_gloo_ranks():
+    """Every rank receives every rank's summary, in rank order."""
+    world = 3
+    port = _free_port()
+    ctx = mp.get_context("spawn")
+    with ctx.Manager() as m:
+        out = m.dict()
+        mp.start_processes(_worker, args=(world, port, out), nprocs=world, join=True,
+                           start_method="spawn")
+        res = dict(out)
+    for r in range(world):
+        hs, ds, _, _ = res[r]
+        for q in range(world):
+            np.testing.assert_array_equal(hs[q], res[q][2])
+            np.testing.assert_array_equal(ds[q], res[q][3])
