@@ -324,31 +324,16 @@ def run_ours(args):
     ms_step = ms / K
     value = weak_scaling_value(world, layer.units, K, ms)
 
-    # end to end through the public API from pinned host buffers
+    # end to end through the public API from pinned host buffers: every step
+    # uploads its inputs, quantizes and scans, and reads y back; steps are
+    # pipelined over an upload, a compute and a download stream with two
+    # device copies of the inputs and of y (step i + 1 uploads while step i
+    # computes and step i - 1 downloads)
     Ke = max(1, min(K, args.e2e_steps))
     h2d = sum(layer.host[k].numel() * layer.host[k].element_size() for k in layer.host)
-    y_host = torch.empty(layer.y.shape, dtype=torch.float16).pin_memory()
-    d2h = y_host.numel() * 2
-    for _ in range(2):
-        for kname, dst in (("x", layer.x), ("dt", layer.dt), ("z", layer.z), ("B", layer.B),
-                           ("C", layer.C)):
-            dst.copy_(layer.host[kname], non_blocking=True)
-        step()
-        y_host.copy_(layer.y, non_blocking=True)
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    a0, a1 = cuda_events(torch)
-    a0.record(stream)
-    for _ in range(Ke):
-        for kname, dst in (("x", layer.x), ("dt", layer.dt), ("z", layer.z), ("B", layer.B),
-                           ("C", layer.C)):
-            dst.copy_(layer.host[kname], non_blocking=True)
-        step()
-        y_host.copy_(layer.y, non_blocking=True)
-    a1.record(stream)
-    torch.cuda.synchronize()
-    ems = max_over_ranks(a0.elapsed_time(a1), dist if world > 1 else None, dev)
+    d2h = layer.y.numel() * 2
+    e2e_ms = e2e_pipelined(torch, layer, Ke)
+    ems = max_over_ranks(e2e_ms, dist if world > 1 else None, dev)
     e2e_value = weak_scaling_value(world, layer.units, Ke, ems)
 
     out = None
@@ -449,6 +434,72 @@ def setup_decode(torch, dev, steps=None):
                          x_scale=xs_t, D=D, y=y)
 
     return dict(b=b, H=H, P=P, N=N, G=G, S=S, step=step)
+
+
+def e2e_pipelined(torch, layer, steps):
+    """Milliseconds for `steps` end-to-end steps of the layer (upload of x,
+    dt, z, B, C from pinned host memory, quantize + scan, download of y into
+    pinned host memory), pipelined over three streams."""
+    from quantized_state_space_b200 import api
+    names = ("x", "dt", "z", "B", "C")
+    sets = [{k: getattr(layer, k) for k in names},
+            {k: torch.empty_like(getattr(layer, k)) for k in names}]
+    ys = [layer.y, torch.empty_like(layer.y)]
+    y_host = [torch.empty(layer.y.shape, dtype=torch.float16).pin_memory() for _ in range(2)]
+    up, comp, down = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    ev = lambda: torch.cuda.Event(enable_timing=False)
+    in_ready = [ev(), ev()]
+    in_free = [ev(), ev()]
+    y_ready = [ev(), ev()]
+    y_free = [ev(), ev()]
+    b, L, d, G, N, gs = layer.b, layer.L, layer.d, layer.G, layer.N, layer.gs
+
+    def run(n):
+        for i in range(n):
+            j = i % 2
+            S = sets[j]
+            with torch.cuda.stream(up):
+                if i >= 2:
+                    up.wait_event(in_free[j])
+                for k in names:
+                    S[k].copy_(layer.host[k], non_blocking=True)
+                in_ready[j].record(up)
+            with torch.cuda.stream(comp):
+                comp.wait_event(in_ready[j])
+                if i >= 2:
+                    comp.wait_event(y_free[j])
+                api.quantize_groups_batch(
+                    [(S["x"], b, d, L, layer.grp, layer.k, layer.xs, layer.xq),
+                     (S["B"], b, G * N, L, layer.smap, G * N // gs, layer.bs, layer.Bq),
+                     (S["C"], b, G * N, L, layer.smap, G * N // gs, layer.cs, layer.Cq)])
+                api.selective_scan(layer.xq, S["dt"], layer.A, layer.Bq, layer.Cq, layer.bs,
+                                   layer.cs, gs, x_group=layer.grp, x_scale=layer.xs, D=layer.D,
+                                   z=S["z"], y=ys[j], h_final=layer.hf)
+                in_free[j].record(comp)  # the scan read dt and z of this set
+                y_ready[j].record(comp)
+            with torch.cuda.stream(down):
+                down.wait_event(y_ready[j])
+                y_host[j].copy_(ys[j], non_blocking=True)
+                y_free[j].record(down)
+
+    run(2)  # warm-up
+    torch.cuda.synchronize()
+    a0, a1 = cuda_events(torch)
+    a0.record(up)
+    run(steps)
+    for s_ in (up, comp):
+        down.wait_stream(s_)
+    a1.record(down)
+    torch.cuda.synchronize()
+    # every step has the same inputs: each downloaded y equals a plain step's
+    layer.quantize()
+    layer.scan()
+    torch.cuda.synchronize()
+    ref = layer.y.cpu()
+    for yh in y_host[:min(steps, 2)]:
+        if not torch.equal(yh.view(torch.int16), ref.view(torch.int16)):
+            raise RuntimeError("pipelined end-to-end step: downloaded y differs")
+    return a0.elapsed_time(a1)
 
 
 def form_other_x_path(torch, layer):

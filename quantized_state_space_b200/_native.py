@@ -178,11 +178,10 @@ def ssmq_quantize_groups(src, outer, mid, inner, group_of_mid, n_groups, mode, s
 def ssmq_quantize_groups_batch(jobs, status=None, stream=None):
     """jobs: list of dicts with the fields of ssmq_quant_job (tensors for the
     pointer fields; dtype taken from src when absent)."""
-    arr = (QuantJob * len(jobs))()
-    for i, j in enumerate(jobs):
-        j = dict(j)
-        j.setdefault("dtype", _dtype_of(j["src"], None))
-        arr[i] = _fill(QuantJob, j)
+    arr = (QuantJob * len(jobs))(*[
+        QuantJob(ptr(j["src"]), j.get("dtype", None) or _dtype_of(j["src"], None), j["outer"],
+                 j["mid"], j["inner"], ptr(j["group_of_mid"]), j["n_groups"], ptr(j["scales"]),
+                 ptr(j["q_out"])) for j in jobs])
     _check(lib().ssmq_quantize_groups_batch(arr, len(jobs), ptr(status), _stream(stream)))
 
 
