@@ -362,6 +362,8 @@ ssmq_status ssmq_selective_scan_w8(const ssmq_scan_args* args, void* stream);
  * this off (one pass per sequence: a call on steps [0, L) equals, byte for
  * byte, a call on [0, L1) followed by one on [L1, L) with h0 = its h_final,
  * L1 a multiple of 128); so do y_q and a NULL y.
+ * seqlen = 0: h_final = h0 (or zeros) and dec_final = 0; the step tensors
+ * may then be NULL.
  * status: SSMQ_DEV_BAD_GROUP as above; SSMQ_DEV_TIMEOUT if a bounded wait for
  * the tensor core gave up (the call's outputs are then incomplete).
  */

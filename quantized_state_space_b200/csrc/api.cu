@@ -371,6 +371,11 @@ ssmq_status check_ssd(const ssmq_ssd_args* a, void* workspace, size_t ws_bytes, 
     *skip = true;
     return SSMQ_OK;
   }
+  if (a->seqlen == 0) {  // only the state passes through (h0 or zero to h_final)
+    REQUIRE(aligned16(a->h0) && aligned16(a->h_final), SSMQ_ERR_ALIGNMENT,
+            "%s: tensors must be 16-byte aligned", fn);
+    return SSMQ_OK;
+  }
   const ssmq_status xs = check_x(a->x_format, a->x, a->x_group, a->x_scale, a->n_x_groups,
                                  a->se_log2_ratio, fn);
   if (xs != SSMQ_OK) return xs;
@@ -408,7 +413,7 @@ ssmq_status ssmq_ssd_carry_in(const ssmq_ssd_args* a, const float* h_carry, void
   bool skip;
   CHECK(check_ssd(a, workspace, ws_bytes, fn, &skip));
   if (skip) return SSMQ_OK;
-  REQUIRE(a->y != nullptr && a->y_q == nullptr, SSMQ_ERR_INVALID_ARG,
+  REQUIRE((a->y != nullptr || a->seqlen == 0) && a->y_q == nullptr, SSMQ_ERR_INVALID_ARG,
           "%s: needs the binary16 y (and no int8 y)", fn);
   REQUIRE(h_carry != nullptr, SSMQ_ERR_INVALID_ARG, "%s: h_carry is NULL", fn);
   REQUIRE(aligned16(h_carry), SSMQ_ERR_ALIGNMENT, "%s: h_carry must be 16-byte aligned", fn);

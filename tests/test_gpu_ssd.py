@@ -262,3 +262,26 @@ def test_ssd_carry_in_h_final_and_dec_with_segments(orc):
     yo, ho = oracle_ssd(orc, q)
     assert_scan_close(H(y).astype(np.float64).transpose(0, 2, 1, 3).reshape(yo.shape), yo,
                       H(hf).reshape(ho.shape), ho)
+
+
+def test_state_chain_and_carry_in_edge_cases():
+    """A one-part fold is the part itself; a three-part fold matches numpy;
+    carry-in on an empty sequence adds h_carry to h_final and nothing else."""
+    rng = np.random.default_rng(960)
+    he = rng.standard_normal((3, 2, 5, 4, 8)).astype(np.float32)
+    dc = -rng.uniform(0.0, 3.0, size=(3, 2, 5)).astype(np.float32)
+    np.testing.assert_array_equal(H(api.state_chain([T(he[0])], [T(dc[0])])), he[0])
+    ref = np.zeros(he.shape[1:], np.float64)
+    for q in range(3):
+        ref = np.exp2(dc[q].astype(np.float64))[..., None, None] * ref + he[q]
+    np.testing.assert_allclose(H(api.state_chain(T(he), T(dc))), ref, rtol=1e-5, atol=1e-6)
+    p = ssd_problem(961, 1, 0, 2, 64, 128)
+    hf = (rng.standard_normal((1, 2, 64, 128)) * 0.1).astype(np.float32)
+    hc = (rng.standard_normal((1, 2, 64, 128)) * 0.1).astype(np.float32)
+    args = (T(p["x"]), T(p["dt"]), T(p["A"]), T(p["B"]), T(p["C"]), T(p["B_scale"]),
+            T(p["C_scale"]), 8)
+    y = torch.empty((1, 0, 2, 64), dtype=torch.float16, device=dev())
+    hft = T(hf)
+    api.ssd_carry_in(*args, T(hc), y, x_group=T(p["x_group"]), x_scale=T(p["x_scale"]),
+                     h_final=hft)
+    np.testing.assert_array_equal(H(hft), hf + hc)
