@@ -335,6 +335,7 @@ def run_ours(args):
     e2e_ms = e2e_pipelined(torch, layer, Ke)
     ems = max_over_ranks(e2e_ms, dist if world > 1 else None, dev)
     e2e_value = weak_scaling_value(world, layer.units, Ke, ems)
+    floor_ms = e2e_copy_floor(torch, layer, Ke) / Ke
 
     out = None
     if rank == 0:
@@ -352,7 +353,12 @@ def run_ours(args):
             "data": "synthetic (seeded numpy draws shaped like the workload; no dataset)",
             "config": dict(config_dict(layer.dm), parallelism="dp%d (independent replicas)" % world),
             "e2e": {"value": round(e2e_value, 3), "unit": UNIT, "h2d_bytes_per_step": h2d,
-                    "d2h_bytes_per_step": d2h, "steps": Ke},
+                    "d2h_bytes_per_step": d2h, "steps": Ke,
+                    "ms_per_step": round(ems / Ke, 5),
+                    "copy_floor_ms_per_step": round(floor_ms, 5),
+                    "frac_of_copy_floor": round(floor_ms / (ems / Ke), 4),
+                    "copy_floor": "the same host<->device copies without kernels, "
+                                  "uploads and the download on two streams"},
             "gpu_launches": layer.launches_per_step * K,
             "x_path": ("binary16 x quantized inside the scan (byte-identical to a separate "
                        "quantize launch followed by the int8 scan)" if layer.fused else
@@ -499,6 +505,35 @@ def e2e_pipelined(torch, layer, steps):
     for yh in y_host[:min(steps, 2)]:
         if not torch.equal(yh.view(torch.int16), ref.view(torch.int16)):
             raise RuntimeError("pipelined end-to-end step: downloaded y differs")
+    return a0.elapsed_time(a1)
+
+
+def e2e_copy_floor(torch, layer, steps):
+    """Milliseconds for `steps` steps of the end-to-end copies alone (every
+    input up, y down, on two streams as in the pipelined run, no kernels):
+    the host-link floor of an end-to-end step."""
+    names = ("x", "dt", "z", "B", "C")
+    dst = {k: torch.empty_like(getattr(layer, k)) for k in names}
+    y_host = torch.empty(layer.y.shape, dtype=torch.float16).pin_memory()
+    up, down = torch.cuda.Stream(), torch.cuda.Stream()
+
+    def run(n):
+        for _ in range(n):
+            with torch.cuda.stream(up):
+                for k in names:
+                    dst[k].copy_(layer.host[k], non_blocking=True)
+            with torch.cuda.stream(down):
+                y_host.copy_(layer.y, non_blocking=True)
+
+    run(1)
+    torch.cuda.synchronize()
+    a0, a1 = cuda_events(torch)
+    a0.record(up)
+    down.wait_stream(up)
+    run(steps)
+    down.wait_stream(up)
+    a1.record(down)
+    torch.cuda.synchronize()
     return a0.elapsed_time(a1)
 
 

@@ -73,6 +73,28 @@ def test_quantize_all_f16_patterns(orc):
         assert nf > 0 and int(H(st)[0]) & N.DEV_NONFINITE
 
 
+def test_quantize_all_f32_patterns(orc):
+    """Every binary32 bit pattern (2^32, in 16 slices of 2^28) at one scale
+    whose reciprocal is inexact: the codes equal the oracle's byte for byte,
+    including every near-tie quotient, the clamp and the non-finite inputs."""
+    s = np.array([0.7310586], np.float32)
+    n = 1 << 28
+    base = np.arange(n, dtype=np.uint32)
+    bits = np.empty(n, np.uint32)
+    sc, g0 = T(s), T(np.zeros(1, np.int32))
+    xg = torch.empty(n, dtype=torch.float32, device="cuda")
+    for k in range(16):
+        np.add(base, np.uint32(k * n), out=bits)
+        x = bits.view(np.float32)
+        xg.copy_(torch.from_numpy(x))
+        qg, _ = api.quantize_groups(xg, 1, 1, n, g0, 1, scales=sc)
+        qo, _, _ = orc.quantize_groups(x, 1, 1, n, [0], 1, orc.SCALE_STATIC, s)
+        got = H(qg)
+        if not np.array_equal(got, qo):
+            i = int(np.flatnonzero(got != qo)[0])
+            raise AssertionError("pattern 0x%08x: gpu %d oracle %d" % (int(bits[i]), got[i], qo[i]))
+
+
 def test_quantize_status_bits():
     x = T(np.ones(64, np.float16))
     st = status_word()

@@ -124,6 +124,28 @@ def test_ssd_delta_zero(orc):
     np.testing.assert_allclose(hf, p["h0"], rtol=0, atol=0)
 
 
+@pytest.mark.parametrize("max_segments", [0, 1])
+def test_ssd_head_permutation_bit_exact(max_segments):
+    """Quamba2 compute invariance for the SSD form: permuting the heads with
+    their x cluster ids, dt, z, A, D, dt_bias and h0 permutes y and the final
+    state exactly (with segments on, all 12 sequences share one SM round and
+    are cut alike)."""
+    Hh, P = 6, 64
+    p = ssd_problem(950, 2, 300, Hh, P, 128, gate=True, h0=True, bias=True)
+    perm = np.random.default_rng(2).permutation(Hh)
+    q = dict(p)
+    for k in ("x", "dt", "z"):
+        q[k] = np.ascontiguousarray(p[k][:, :, perm])
+    q["x_group"] = np.ascontiguousarray(p["x_group"].reshape(Hh, P)[perm].reshape(-1))
+    for k in ("A", "D", "dt_bias"):
+        q[k] = np.ascontiguousarray(p[k][perm])
+    q["h0"] = np.ascontiguousarray(p["h0"][:, perm])
+    y, hf = gpu_ssd(p, max_segments=max_segments)
+    yq, hq = gpu_ssd(q, max_segments=max_segments)
+    np.testing.assert_array_equal(yq, y[:, :, perm])
+    np.testing.assert_array_equal(hq, hf[:, perm])
+
+
 def test_ssd_bad_group_status():
     p = ssd_problem(480, 1, 128, 2, 64, 128)
     p["x_group"][5] = 1000
