@@ -58,7 +58,7 @@ typedef enum {
   SSMQ_OK = 0,
   SSMQ_ERR_INVALID_ARG = 1, /* null pointer, bad size, bad enum, L > H ... */
   SSMQ_ERR_ALIGNMENT = 2,   /* a base pointer violates the alignment rule */
-  SSMQ_ERR_UNSUPPORTED = 3, /* valid, but outside the shapes this build runs */
+  SSMQ_ERR_UNSUPPORTED = 3, /* valid, but outside the shapes the kernels implement */
   SSMQ_ERR_CUDA = 4,        /* a CUDA launch or runtime call failed */
   SSMQ_ERR_TIMEOUT = 5,     /* reserved: a bounded device wait gave up */
   SSMQ_ERR_NONFINITE = 6    /* reserved for host-detected non-finite scalars */

@@ -361,7 +361,7 @@ ssmq_status check_ssd(const ssmq_ssd_args* a, void* workspace, size_t ws_bytes, 
   REQUIRE(a->ngroups >= 1 && a->nheads % a->ngroups == 0, SSMQ_ERR_INVALID_ARG,
           "%s: nheads must be a multiple of ngroups >= 1", fn);
   REQUIRE(a->headdim == 64 && a->dstate == 128, SSMQ_ERR_UNSUPPORTED,
-          "%s: this build runs headdim 64, dstate 128", fn);
+          "%s: the SSD kernel runs headdim 64, dstate 128", fn);
   REQUIRE(a->chunk == 64 || a->chunk == 128 || a->chunk == 256, SSMQ_ERR_UNSUPPORTED,
           "%s: chunk must be 64, 128 or 256", fn);
   REQUIRE(a->state_group_size >= 1 && a->dstate % a->state_group_size == 0,

@@ -216,9 +216,8 @@ def test_softedge_workload_end_to_end(orc):
     _m1_end_to_end(orc, "softedge", n_units=64)
 
 
-# ---- encode then scan: binary16 x encoded inside the scan (SURVEY-next
-# producer-side fusion; Quamba-SE write-up 4.1: the range check inside
-# quantisation).  The fused call must equal the separate encoder followed by
+# ---- encode then scan: binary16 x encoded inside the scan (producer-side
+# fusion; Quamba-SE write-up 4.1: the range check inside quantisation).  The fused call must equal the separate encoder followed by
 # the code-reading scan, byte for byte, status word included.
 
 FUSED_CASES = [
