@@ -84,7 +84,7 @@ _REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_
 class ClockSampler:
     """Samples the SM clock and clock-event reasons with NVML in a thread."""
 
-    def __init__(self, torch_dev, period=0.01):
+    def __init__(self, torch_dev, period=0.002):
         self.samples, self.reasons, self.max_mhz = [], set(), None
         self.period = period
         self.ok = False
