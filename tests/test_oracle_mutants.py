@@ -40,6 +40,12 @@ MUTANTS = {
     "decode_drop_D": ("if (p->D) acc += (double)p->D[hd] * x;\n    if (p->z) acc *= orc_silu(orc_half_to_double(p->z[xi]));\n    if (o->y) o->y[k * P + pp] = acc;",
                       "if (0) acc += (double)p->D[hd] * x;\n    if (p->z) acc *= orc_silu(orc_half_to_double(p->z[xi]));\n    if (o->y) o->y[k * P + pp] = acc;"),
     "half_subnormal": ("v = ldexp((double)m, -24);", "v = ldexp((double)m, -25);"),
+    "m1_output_before_update": ("h[n] = exp(delta * (double)p->A[c * N + n]) * h[n] + delta * Bv * x;\n      acc += Cv * h[n];",
+                                "acc += Cv * h[n];\n      h[n] = exp(delta * (double)p->A[c * N + n]) * h[n] + delta * Bv * x;"),
+    "ssd_bc_scale_index": ("const int64_t si = g * spg + n / p->state_group_size;\n      Bv[n] = (double)p->B[bi] * (double)p->B_scale[si];",
+                           "const int64_t si = g * spg + n % p->state_group_size;\n      Bv[n] = (double)p->B[bi] * (double)p->B_scale[si];"),
+    "ssd_bias_dropped": ("orc_delta(orc_half_to_double(p->dt[(b * L + t) * H + hd]),\n                                   p->dt_bias ? (double)p->dt_bias[hd] : 0.0, p->dt_softplus);\n    const double dA",
+                         "orc_delta(orc_half_to_double(p->dt[(b * L + t) * H + hd]),\n                                   0.0, p->dt_softplus);\n    const double dA"),
 }
 
 

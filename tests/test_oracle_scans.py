@@ -168,6 +168,28 @@ def test_m1_lti_geometric_series(orc):
         assert _rel(hf[c], h[-1]) < 1e-12
 
 
+def test_m1_lti_materialised_convolution(orc):
+    """LTI system (constant delta, B, C) driven by a varying x: y is the causal
+    convolution of x with the materialised kernel
+    K_k = sum_n C_n exp(delta A_n)^k delta B_n, plus D x (numpy.convolve)."""
+    L, d, delta = 64, 3, 0.0625
+    p = m1_problem(4, 1, L, d, 16, gate=False, h0=False)
+    p["dt"][:] = np.float16(delta)
+    p["B"][:] = p["B"][:, :, :, :1]
+    p["C"][:] = p["C"][:, :, :, :1]
+    y, _ = _m1(orc, p, dt_softplus=False)
+    gs = p["state_group_size"]
+    x = _deq_x_m1(p)[0]
+    Bv = _deq_bc(p["B"], p["B_scale"], gs, 2)[0, 0, :, 0]
+    Cv = _deq_bc(p["C"], p["C_scale"], gs, 2)[0, 0, :, 0]
+    k = np.arange(L)[:, None]
+    for c in range(d):
+        a = np.exp(delta * p["A"][c].astype(np.float64))
+        K = (a[None, :] ** k * (delta * Bv)[None, :]) @ Cv
+        want = np.convolve(x[c], K)[:L] + p["D"][c] * x[c]
+        assert _rel(y[c], want) < 1e-12
+
+
 def test_m1_softedge_bruteforce(orc):
     """x given as soft-edge codes: the scan equals the recurrence run on the
     decoded values (decoded here through the binary32 decoder, hence the
