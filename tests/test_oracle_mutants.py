@@ -44,6 +44,12 @@ MUTANTS = {
                                 "acc += Cv * h[n];\n      h[n] = exp(delta * (double)p->A[c * N + n]) * h[n] + delta * Bv * x;"),
     "ssd_bc_scale_index": ("const int64_t si = g * spg + n / p->state_group_size;\n      Bv[n] = (double)p->B[bi] * (double)p->B_scale[si];",
                            "const int64_t si = g * spg + n % p->state_group_size;\n      Bv[n] = (double)p->B[bi] * (double)p->B_scale[si];"),
+    "softedge_ge_hi": ("else if (a > thr_hi)", "else if (a >= thr_hi)"),
+    "absmax_div_128": ("scales[g] = (float)(amax[g] / 127.0);", "scales[g] = (float)(amax[g] / 128.0);"),
+    "m1_gate_before_D": ("    if (p->D) acc += (double)p->D[c] * x;\n    if (p->z) acc *= orc_silu(orc_half_to_double(p->z[idx]));\n    if (o->y) o->y[k * L + t] = acc;",
+                         "    if (p->z) acc *= orc_silu(orc_half_to_double(p->z[idx]));\n    if (p->D) acc += (double)p->D[c] * x;\n    if (o->y) o->y[k * L + t] = acc;"),
+    "bias_after_softplus": ("  double v = dtv + bias;\n  return softplus ? orc_softplus(v) : v;",
+                            "  double v = dtv;\n  return (softplus ? orc_softplus(v) : v) + bias;"),
     "ssd_bias_dropped": ("orc_delta(orc_half_to_double(p->dt[(b * L + t) * H + hd]),\n                                   p->dt_bias ? (double)p->dt_bias[hd] : 0.0, p->dt_softplus);\n    const double dA",
                          "orc_delta(orc_half_to_double(p->dt[(b * L + t) * H + hd]),\n                                   0.0, p->dt_softplus);\n    const double dA"),
 }
