@@ -50,6 +50,11 @@ MUTANTS = {
                          "    if (p->z) acc *= orc_silu(orc_half_to_double(p->z[idx]));\n    if (p->D) acc += (double)p->D[c] * x;\n    if (o->y) o->y[k * L + t] = acc;"),
     "bias_after_softplus": ("  double v = dtv + bias;\n  return softplus ? orc_softplus(v) : v;",
                             "  double v = dtv;\n  return (softplus ? orc_softplus(v) : v) + bias;"),
+    "decode_group_index": ("  const int64_t b = u / H, hd = u % H, g = hd * G / H;\n  const int64_t spg = N / p->state_group_size;\n  const double delta = orc_delta(orc_half_to_double(p->dt[b * H + hd]),",
+                           "  const int64_t b = u / H, hd = u % H, g = hd % G;\n  const int64_t spg = N / p->state_group_size;\n  const double delta = orc_delta(orc_half_to_double(p->dt[b * H + hd]),"),
+    "percentile_signed": ("if (isfinite(f)) v[m++] = fabs((double)f);", "if (isfinite(f)) v[m++] = (double)f;"),
+    "percentile_position_n": ("const double pos = (double)(m - 1) * (q / 100.0);",
+                              "const double pos = (double)m * (q / 100.0);"),
     "ssd_bias_dropped": ("orc_delta(orc_half_to_double(p->dt[(b * L + t) * H + hd]),\n                                   p->dt_bias ? (double)p->dt_bias[hd] : 0.0, p->dt_softplus);\n    const double dA",
                          "orc_delta(orc_half_to_double(p->dt[(b * L + t) * H + hd]),\n                                   0.0, p->dt_softplus);\n    const double dA"),
 }
