@@ -16,11 +16,44 @@ def _dev_check(*ts):
             raise ValueError("tensors must be contiguous CUDA tensors")
 
 
+def _out(t, name, dtype, numel, device):
+    """A caller-supplied tensor that the call writes (or reads whole): it must
+    be contiguous, on the inputs' device, of the dtype and element count the
+    kernels use, since the library cannot see the size behind a pointer."""
+    if t is None:
+        return
+    if t.device != device or not t.is_contiguous():
+        raise ValueError("%s must be a contiguous tensor on %s" % (name, device))
+    if t.dtype != dtype or t.numel() != numel:
+        raise ValueError("%s must be %s with %d elements (got %s with %d)"
+                         % (name, dtype, numel, t.dtype, t.numel()))
+
+
+def _status(t, device):
+    """The optional device status word: 32-bit, at least one element."""
+    if t is None:
+        return
+    if t.device != device or t.element_size() != 4 or t.numel() < 1:
+        raise ValueError("status must be a 32-bit tensor of at least one element on %s" % device)
+
+
+def _workspace(t, nbytes, device):
+    """A caller-supplied workspace: uint8 bytes on the device, room for the
+    256-byte alignment of its start."""
+    if t is None or not nbytes:
+        return
+    if t.device != device or t.dtype != torch.uint8 or t.numel() < nbytes + 255:
+        raise ValueError("workspace must be a uint8 tensor of at least %d bytes on %s"
+                         % (nbytes + 255, device))
+
+
 def quantize_groups(src, outer, mid, inner, group_of_mid, n_groups, *, scales=None,
                     absmax=False, out=None, status=None):
     """int8 codes of ``src`` (float16/float32) with one scale per group.
     absmax=True computes the scales (returned); else ``scales`` are used."""
     _dev_check(src, group_of_mid, scales)
+    _out(out, "out", torch.int8, outer * mid * inner, src.device)
+    _status(status, src.device)
     q = out if out is not None else torch.empty(src.shape, dtype=torch.int8, device=src.device)
     if absmax:
         scales = torch.empty(n_groups, dtype=torch.float32, device=src.device)
@@ -36,6 +69,8 @@ def quantize_groups_batch(jobs, *, status=None):
     outs, descs = [], []
     for src, outer, mid, inner, gmap, n_groups, scales, out in jobs:
         _dev_check(src, gmap, scales)
+        _out(out, "out", torch.int8, outer * mid * inner, src.device)
+        _status(status, src.device)
         q = out if out is not None else torch.empty(src.shape, dtype=torch.int8,
                                                     device=src.device)
         outs.append(q)
@@ -47,6 +82,8 @@ def quantize_groups_batch(jobs, *, status=None):
 
 def softedge_encode(src, scale, thr_lo, thr_hi, log2_ratio=2, *, out=None, status=None):
     _dev_check(src)
+    _out(out, "out", torch.uint8, src.numel(), src.device)
+    _status(status, src.device)
     codes = out if out is not None else torch.empty(src.shape, dtype=torch.uint8, device=src.device)
     N.ssmq_softedge_encode(src, src.numel(), float(scale), float(thr_lo), float(thr_hi),
                            log2_ratio, codes, status=status)
@@ -55,6 +92,7 @@ def softedge_encode(src, scale, thr_lo, thr_hi, log2_ratio=2, *, out=None, statu
 
 def softedge_decode(codes, scale, log2_ratio=2, *, out=None):
     _dev_check(codes)
+    _out(out, "out", torch.float32, codes.numel(), codes.device)
     o = out if out is not None else torch.empty(codes.shape, dtype=torch.float32,
                                                 device=codes.device)
     N.ssmq_softedge_decode(codes, codes.numel(), float(scale), log2_ratio, o)
@@ -80,6 +118,11 @@ def _x_fields(x, x_group, x_scale, se_scale, se_log2_ratio, se_lo=None, se_hi=No
 def _y_fields(shape, device, y_group, y_scale, y_q, want_y, y):
     """Optional int8 output (static per-cluster scales) and the binary16 y."""
     f = {}
+    n = 1
+    for v in shape:
+        n *= v
+    _out(y, "y", torch.float16, n, device)
+    _out(y_q, "y_q", torch.int8, n, device)
     if y_group is not None:
         _dev_check(y_group, y_scale)
         if y_q is None:
@@ -104,6 +147,8 @@ def selective_scan(x, dt, A, B, C, B_scale, C_scale, state_group_size, *, x_grou
     b, d, L = x.shape
     G, Nst = B.shape[1], B.shape[2]
     _dev_check(x, dt, A, B, C, B_scale, C_scale, x_group, x_scale, D, z, dt_bias, h0)
+    _out(h_final, "h_final", torch.float32, b * d * Nst, x.device)
+    _status(status, x.device)
     y, y_q, yf = _y_fields((b, d, L), x.device, y_group, y_scale, y_q, want_y, y)
     if h_final is None and return_state:
         h_final = torch.empty((b, d, Nst), dtype=torch.float32, device=x.device)
@@ -130,6 +175,7 @@ def _ssd_call(x, dt, A, B, C, B_scale, C_scale, state_group_size, chunk, x_group
                   B=B, C=C, B_scale=B_scale, C_scale=C_scale, h0=h0, y=y, h_final=h_final,
                   status=status, max_segments=max_segments, dec_final=dec_final, **yf)
     ws = N.ssmq_ssd_workspace_size(**fields)
+    _workspace(workspace, ws, x.device)
     if ws and workspace is None:
         workspace = torch.empty(ws + 256, dtype=torch.uint8, device=x.device)
     wptr = (workspace.data_ptr() + 255) // 256 * 256 if ws else None
@@ -149,6 +195,9 @@ def ssd_chunk_scan(x, dt, A, B, C, B_scale, C_scale, state_group_size, *, chunk=
     b, L, H, P = x.shape
     Nst = B.shape[3]
     _dev_check(x, dt, A, B, C, B_scale, C_scale, x_group, x_scale, D, z, dt_bias, h0, dec_final)
+    _out(h_final, "h_final", torch.float32, b * H * P * Nst, x.device)
+    _out(dec_final, "dec_final", torch.float32, b * H, x.device)
+    _status(status, x.device)
     y, y_q, yf = _y_fields((b, L, H, P), x.device, y_group, y_scale, y_q, want_y, y)
     if h_final is None and return_state:
         h_final = torch.empty((b, H, P, Nst), dtype=torch.float32, device=x.device)
@@ -168,6 +217,12 @@ def ssd_carry_in(x, dt, A, B, C, B_scale, C_scale, state_group_size, h_carry, y,
     inputs that started from a zero state."""
     _dev_check(x, dt, A, B, C, B_scale, C_scale, x_group, x_scale, D, z, dt_bias, h_carry, y,
                h_final)
+    b, L, H, P = x.shape
+    Nst = B.shape[3]
+    _out(y, "y", torch.float16, b * L * H * P, x.device)
+    _out(h_carry, "h_carry", torch.float32, b * H * P * Nst, x.device)
+    _out(h_final, "h_final", torch.float32, b * H * P * Nst, x.device)
+    _status(status, x.device)
     fields, wptr, ws = _ssd_call(x, dt, A, B, C, B_scale, C_scale, state_group_size, chunk,
                                  x_group, x_scale, se_scale, se_log2_ratio, D, z, dt_bias,
                                  dt_softplus, None, y, h_final, 0, workspace, status, None, {})
@@ -199,6 +254,9 @@ def state_update(state, x, dt, A, B, C, B_scale, C_scale, state_group_size, *, x
     b, H, P, Nst = state.shape
     G = B.shape[1]
     _dev_check(state, x, dt, A, B, C, B_scale, C_scale, x_group, x_scale, D, z, dt_bias)
+    _out(state, "state", torch.float32, b * H * P * Nst, state.device)
+    _out(y, "y", torch.float16, b * H * P, state.device)
+    _status(status, state.device)
     if y is None:
         y = torch.empty((b, H, P), dtype=torch.float16, device=state.device)
     N.ssmq_state_update_w8(batch=b, nheads=H, headdim=P, dstate=Nst, ngroups=G,
@@ -218,6 +276,9 @@ def selective_state_update(state, x, dt, A, B, C, B_scale, C_scale, state_group_
     b, d, Nst = state.shape
     G = B.shape[1]
     _dev_check(state, x, dt, A, B, C, B_scale, C_scale, x_group, x_scale, D, z, dt_bias)
+    _out(state, "state", torch.float32, b * d * Nst, state.device)
+    _out(y, "y", torch.float16, b * d, state.device)
+    _status(status, state.device)
     if y is None:
         y = torch.empty((b, d), dtype=torch.float16, device=state.device)
     N.ssmq_selective_state_update_w8(batch=b, dim=d, dstate=Nst, ngroups=G,
@@ -234,6 +295,8 @@ def selective_state_update(state, x, dt, A, B, C, B_scale, C_scale, state_group_
 def group_absmax(src, outer, mid, inner, group_of_mid, n_groups, *, out=None, status=None):
     """Exact max |v| per group over the finite elements (float32[n_groups])."""
     _dev_check(src, group_of_mid)
+    _out(out, "out", torch.float32, n_groups, src.device)
+    _status(status, src.device)
     a = out if out is not None else torch.empty(n_groups, dtype=torch.float32, device=src.device)
     N.ssmq_group_absmax(src, outer, mid, inner, group_of_mid, n_groups, a, status=status)
     return a
@@ -242,6 +305,7 @@ def group_absmax(src, outer, mid, inner, group_of_mid, n_groups, *, out=None, st
 def cluster_by_absmax(absmax, k, *, status=None):
     """Sort-and-cluster on the device: (cluster id per channel int32, scales float32[k])."""
     _dev_check(absmax)
+    _status(status, absmax.device)
     n = absmax.numel()
     cl = torch.empty(n, dtype=torch.int32, device=absmax.device)
     sc = torch.empty(k, dtype=torch.float32, device=absmax.device)
@@ -251,6 +315,7 @@ def cluster_by_absmax(absmax, k, *, status=None):
 
 def _pct_workspace(device, workspace):
     nb = N.ssmq_percentile_workspace_size()
+    _workspace(workspace, nb, device)
     if workspace is None:
         workspace = torch.empty(nb + 256, dtype=torch.uint8, device=device)
     base = workspace.data_ptr()
@@ -261,6 +326,7 @@ def percentile_abs(src, q, *, out=None, workspace=None):
     """Percentiles (linear interpolation) of |src| over its finite elements."""
     _dev_check(src)
     q = [float(v) for v in (q if hasattr(q, "__len__") else [q])]
+    _out(out, "out", torch.float32, len(q), src.device)
     o = out if out is not None else torch.empty(len(q), dtype=torch.float32, device=src.device)
     wptr, nb = _pct_workspace(src.device, workspace)
     N.ssmq_percentile_abs(src, src.numel(), q, o, wptr, nb)
@@ -271,6 +337,7 @@ def softedge_calibrate(src, thresholds=None, *, q_lo=5.0, q_hi=99.9, alpha=1.0, 
     """Soft-edge parameters {scale, lo, hi} (float32[3], updated in place):
     percentiles of |src|, blended into the running values when alpha < 1."""
     _dev_check(src)
+    _out(thresholds, "thresholds", torch.float32, 3, src.device)
     thr = thresholds if thresholds is not None else torch.zeros(3, dtype=torch.float32,
                                                                   device=src.device)
     wptr, nb = _pct_workspace(src.device, workspace)

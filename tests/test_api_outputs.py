@@ -1,0 +1,122 @@
+"""The Python front end checks every tensor that a call writes (or reads
+whole) and that the caller supplies -- device, contiguity, dtype, element
+count -- since the C library sees only pointers.  Run on the CPU: the native
+calls are replaced by a recorder and the CUDA-device requirement is lifted,
+so only the front end's own checks decide."""
+import pytest
+import torch
+
+from quantized_state_space_b200 import _native as real_native
+from quantized_state_space_b200 import api
+
+
+class _Recorder:
+    def __init__(self):
+        self.calls = []
+
+    def __getattr__(self, name):
+        if name == "ssmq_ssd_workspace_size":
+            return lambda **kw: 4096
+        if name == "ssmq_percentile_workspace_size":
+            return lambda: 1024
+        if name.startswith("ssmq_"):
+            return lambda *a, **kw: self.calls.append(name)
+        return getattr(real_native, name)
+
+
+@pytest.fixture()
+def rec(monkeypatch):
+    r = _Recorder()
+    monkeypatch.setattr(api, "N", r)
+    monkeypatch.setattr(api, "_dev_check", lambda *ts: None)
+    return r
+
+
+def E(*shape, dtype=torch.float32, device="cpu"):
+    return torch.empty(shape, dtype=dtype, device=device)
+
+
+def _bad(fn, **kw):
+    with pytest.raises(ValueError):
+        fn(**kw)
+
+
+def test_quantizer_outputs(rec):
+    src, g, s = E(2, 3, 8, dtype=torch.float16), E(3, dtype=torch.int32), E(2)
+    call = lambda **kw: api.quantize_groups(src, 2, 3, 8, g, 2, scales=s, **kw)
+    call(out=E(48, dtype=torch.int8), status=E(1, dtype=torch.int32))
+    _bad(call, out=E(47, dtype=torch.int8))
+    _bad(call, out=E(48, dtype=torch.uint8))
+    _bad(call, out=E(48, dtype=torch.int8, device="meta"))
+    _bad(call, out=E(8, 6, dtype=torch.int8).t())
+    _bad(call, status=E(1, dtype=torch.int16))
+    _bad(call, status=E(0, dtype=torch.int32))
+    job = lambda out: [(src, 2, 3, 8, g, 2, s, out)]
+    api.quantize_groups_batch(job(E(48, dtype=torch.int8)))
+    _bad(lambda **kw: api.quantize_groups_batch(job(E(40, dtype=torch.int8))))
+    api.softedge_encode(src, 1.0, 0.1, 5.0, out=E(48, dtype=torch.uint8))
+    _bad(lambda: api.softedge_encode(src, 1.0, 0.1, 5.0, out=E(48, dtype=torch.int8)))
+    codes = E(48, dtype=torch.uint8)
+    api.softedge_decode(codes, 1.0, out=E(48))
+    _bad(lambda: api.softedge_decode(codes, 1.0, out=E(48, dtype=torch.float16)))
+    assert rec.calls.count("ssmq_quantize_groups") == 1
+
+
+def test_scan_outputs(rec):
+    b, d, L, G, N = 2, 8, 5, 1, 16
+    x, dt = E(b, d, L, dtype=torch.int8), E(b, d, L, dtype=torch.float16)
+    Bq = E(b, G, N, L, dtype=torch.int8)
+    args = (x, dt, E(d, N), Bq, Bq, E(4), E(4), 4)
+    kw = dict(x_group=E(d, dtype=torch.int32), x_scale=E(2))
+    api.selective_scan(*args, y=E(b, d, L, dtype=torch.float16), h_final=E(b, d, N), **kw)
+    _bad(lambda: api.selective_scan(*args, y=E(b, d, L), **kw))
+    _bad(lambda: api.selective_scan(*args, h_final=E(b, d, N - 1), **kw))
+    _bad(lambda: api.selective_scan(*args, y_group=E(d, dtype=torch.int32), y_scale=E(2),
+                                    y_q=E(b, d, L, dtype=torch.uint8), **kw))
+    dec_args = (E(b, d, dtype=torch.int8), E(b, d, dtype=torch.float16), E(d, N),
+                E(b, G, N, dtype=torch.int8), E(b, G, N, dtype=torch.int8), E(4), E(4), 4)
+    api.selective_state_update(E(b, d, N), *dec_args, y=E(b, d, dtype=torch.float16), **kw)
+    _bad(lambda: api.selective_state_update(E(b, d, N, dtype=torch.float64), *dec_args, **kw))
+    _bad(lambda: api.selective_state_update(E(b, d, N), *dec_args, y=E(b, d + 1,
+                                                                       dtype=torch.float16), **kw))
+
+
+def test_ssd_outputs(rec):
+    b, L, H, P, G, N = 1, 300, 2, 64, 1, 128
+    x, dt = E(b, L, H, P, dtype=torch.int8), E(b, L, H, dtype=torch.float16)
+    Bq = E(b, L, G, N, dtype=torch.int8)
+    args = (x, dt, E(H), Bq, Bq, E(16), E(16), 8)
+    kw = dict(x_group=E(H * P, dtype=torch.int32), x_scale=E(2))
+    y, hf, dec = E(b, L, H, P, dtype=torch.float16), E(b, H, P, N), E(b, H)
+    api.ssd_chunk_scan(*args, y=y, h_final=hf, dec_final=dec,
+                       workspace=E(4096 + 255, dtype=torch.uint8), **kw)
+    _bad(lambda: api.ssd_chunk_scan(*args, workspace=E(4096, dtype=torch.uint8), **kw))
+    _bad(lambda: api.ssd_chunk_scan(*args, workspace=E(8192), **kw))
+    _bad(lambda: api.ssd_chunk_scan(*args, dec_final=E(b, H + 1), **kw))
+    _bad(lambda: api.ssd_chunk_scan(*args, h_final=E(b, H, N, P, dtype=torch.float16), **kw))
+    api.ssd_carry_in(*args, E(b, H, P, N), y, h_final=hf, **kw)
+    _bad(lambda: api.ssd_carry_in(*args, E(b, H, P, N - 8), y, **kw))
+    _bad(lambda: api.ssd_carry_in(*args, E(b, H, P, N), E(b, L - 1, H, P, dtype=torch.float16),
+                                  **kw))
+    x0 = E(b, 0, H, P, dtype=torch.int8)  # an empty sequence: y has no elements
+    api.ssd_carry_in(x0, E(b, 0, H, dtype=torch.float16), E(H), E(b, 0, G, N, dtype=torch.int8),
+                     E(b, 0, G, N, dtype=torch.int8), E(16), E(16), 8, E(b, H, P, N),
+                     E(b, 0, H, P, dtype=torch.float16), h_final=hf, **kw)
+    st = E(2, H, P, N)
+    api.state_update(st, E(2, H, P, dtype=torch.int8), E(2, H, dtype=torch.float16), E(H),
+                     E(2, G, N, dtype=torch.int8), E(2, G, N, dtype=torch.int8), E(16), E(16), 8,
+                     y=E(2, H, P, dtype=torch.float16), **kw)
+    _bad(lambda: api.state_update(st, E(2, H, P, dtype=torch.int8), E(2, H, dtype=torch.float16),
+                                  E(H), E(2, G, N, dtype=torch.int8), E(2, G, N, dtype=torch.int8),
+                                  E(16), E(16), 8, y=E(2, H, P), **kw))
+
+
+def test_calibration_outputs(rec):
+    src = E(4, 6, dtype=torch.float16)
+    api.group_absmax(src, 1, 4, 6, E(4, dtype=torch.int32), 4, out=E(4))
+    _bad(lambda: api.group_absmax(src, 1, 4, 6, E(4, dtype=torch.int32), 4, out=E(3)))
+    api.percentile_abs(src, [5.0, 99.9], out=E(2), workspace=E(1024 + 255, dtype=torch.uint8))
+    _bad(lambda: api.percentile_abs(src, [5.0, 99.9], out=E(3)))
+    _bad(lambda: api.percentile_abs(src, 5.0, workspace=E(1024, dtype=torch.uint8)))
+    api.softedge_calibrate(src, E(3))
+    _bad(lambda: api.softedge_calibrate(src, E(3, dtype=torch.float64)))
