@@ -110,3 +110,12 @@ def test_exchange_over_three_gloo_ranks():
         for q in range(world):
             np.testing.assert_array_equal(hs[q], res[q][2])
             np.testing.assert_array_equal(ds[q], res[q][3])
+
+
+def test_sharded_call_rejects_unshared_arguments():
+    """Only the arguments that both the slice scan and its carry-in take are
+    accepted (an int8-y request, for one, has no carry-in form)."""
+    from quantized_state_space_b200 import sharded
+    with pytest.raises(TypeError, match="y_group"):
+        sharded.ssd_chunk_scan_sequence_sharded(None, None, None, None, None, None, None, 8,
+                                                y_group=None)
