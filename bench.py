@@ -206,8 +206,51 @@ class Layer:
         return self.scan_bytes() + xq + 2 * 3 * b * G * N * L
 
 
+def sfu_peak(ex2, mhz):
+    """Scan roof in G state updates/s (one exponential each): the probe's
+    measured rate, else the CUDA guide's 16 results per clock per SM."""
+    if ex2 and ex2.get("gex2_per_s"):
+        return ex2["gex2_per_s"], ("measured: ssmq_probe_ex2 in this run, %.1f G ex2/s "
+                                   "(%s per SM per clock at %s MHz); one exp per state update"
+                                   % (ex2["gex2_per_s"], ex2.get("per_sm_per_clock"),
+                                      ex2.get("sm_mhz")))
+    return SMS * MUFU_PER_CLK * mhz * 1e6 / 1e9, ("%d SMs x %d ex2/clk (SFU, CUDA guide "
+                                                  "figure) x %.0f MHz" % (SMS, MUFU_PER_CLK, mhz))
+
+
 def cuda_events(torch):
     return torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+
+def measure_ex2(torch, dev, reps=5):
+    """Rate of the special-function unit's base-2 exponential on this GPU,
+    measured with the library's own probe kernel (independent ex2 chains on
+    every SM, CUDA events, the SM clock sampled meanwhile): the compute roof
+    of the Mamba-1 scan, one exponential per state update."""
+    from quantized_state_space_b200 import _native as N
+    sink = torch.zeros(4, dtype=torch.float32, device=dev)
+    iters = 2048
+    for _ in range(3):
+        N.ssmq_probe_ex2(iters, sink)
+    torch.cuda.synchronize()
+    times = []
+    with ClockSampler(dev.index or 0, period=0.001) as clk:
+        for _ in range(reps):
+            a, b = cuda_events(torch)
+            a.record()
+            n = N.ssmq_probe_ex2(iters, sink)
+            b.record()
+            torch.cuda.synchronize()
+            times.append(a.elapsed_time(b) / 1e3)
+    t = statistics.median(times)
+    c = clk.summary()
+    mhz = c.get("sm_mhz") or None
+    rate = n / t / 1e9
+    return {"gex2_per_s": round(rate, 1), "ms_per_launch": round(t * 1e3, 4), "n_ex2": n,
+            "per_sm_per_clock": round(rate * 1e3 / (SMS * mhz), 3) if mhz else None,
+            "sm_mhz": mhz, "sm_max_mhz": c.get("sm_max_mhz"), "reasons": c.get("reasons"),
+            "method": "ssmq_probe_ex2: %d SMs x 8 CTAs x 256 threads x 8 independent ex2 "
+                      "chains, median of %d launches (CUDA events)" % (SMS, reps)}
 
 
 def cpu_baseline(layer, threads=None, max_units=None):
@@ -231,15 +274,34 @@ def cpu_baseline(layer, threads=None, max_units=None):
     ox, _, _ = O.quantize_groups(xs, bb, d, L, og, k, O.SCALE_STATIC, oxs)
     oB, _, _ = O.quantize_groups(raw["B"][:bb], bb, G * N, L, smap, G * N // gs, O.SCALE_STATIC, obs)
     oC, _, _ = O.quantize_groups(raw["C"][:bb], bb, G * N, L, smap, G * N // gs, O.SCALE_STATIC, ocs)
-    O.m1_scan(ox, raw["dt"][:bb], raw["A"], oB, oC, obs, ocs, gs, x_group=og, x_scale=oxs,
-              D=raw["D"], z=raw["z"][:bb], units=units[:bb * d], threads=threads)
+    yo, ho = O.m1_scan(ox, raw["dt"][:bb], raw["A"], oB, oC, obs, ocs, gs, x_group=og,
+                       x_scale=oxs, D=raw["D"], z=raw["z"][:bb], units=units[:bb * d],
+                       threads=threads)
     dt = time.perf_counter() - t1
     units_done = bb * d * L
+    layer.oracle_out = (bb, yo, ho)  # for the in-run parity check
     return {"value": units_done / dt / 1e9, "unit": UNIT, "cores": threads, "kind": "oracle",
             "sample": "%d of %d batch rows (%d channel rows x L %d): static quantize of "
                       "x/B/C + double-precision scan; calibration (%.1f s) untimed"
                       % (bb, b, bb * d, L, t_cal),
             "seconds": dt}
+
+
+Y_TOL, STATE_TOL = 2e-3, 1e-4  # max |y - y_ref| / max |y_ref|; final-state relative L2
+
+
+def parity(y_gpu, y_ref, h_gpu=None, h_ref=None, what=""):
+    """Errors of the GPU result against the oracle on the same inputs, with
+    the stated tolerances."""
+    y, r = np.asarray(y_gpu, np.float64), np.asarray(y_ref, np.float64)
+    out = {"y_max_err_rel": float(np.max(np.abs(y - r)) / max(np.max(np.abs(r)), 1e-30)),
+           "y_tol": Y_TOL, "sample": what}
+    if h_gpu is not None:
+        h, hr = np.asarray(h_gpu, np.float64), np.asarray(h_ref, np.float64)
+        out["state_rel_l2"] = float(np.linalg.norm(h - hr) / max(np.linalg.norm(hr), 1e-30))
+        out["state_tol"] = STATE_TOL
+    out["ok"] = out["y_max_err_rel"] <= Y_TOL and out.get("state_rel_l2", 0.0) <= STATE_TOL
+    return out
 
 
 # ---- ranks -----------------------------------------------------------------
@@ -338,12 +400,18 @@ def run_ours(args):
     floor_ms = e2e_copy_floor(torch, layer, Ke) / Ke
 
     out = None
+    ex2 = None
+    if rank == 0:
+        try:  # the SFU roof, measured on this GPU after the timed region
+            ex2 = measure_ex2(torch, dev)
+        except Exception as e:
+            ex2 = {"error": "%s: %s" % (type(e).__name__, e)}
     if rank == 0:
         scan_avg_s = statistics.mean(scan_ms) / 1e3
         clocks = clk.summary()
         mhz_max = float(clocks.get("sm_max_mhz") or pk["sm_max_mhz"])
         updates = layer.b * layer.L * layer.d * layer.N
-        peak_upd = SMS * MUFU_PER_CLK * mhz_max * 1e6 / 1e9
+        peak_upd, peak_basis = sfu_peak(ex2, mhz_max)
         achieved_upd = updates / scan_avg_s / 1e9
         scan_gbs = layer.scan_bytes() / scan_avg_s / 1e9
         out = {
@@ -368,8 +436,7 @@ def run_ours(args):
                          "unit": "Gupdates/s", "frac": round(achieved_upd / peak_upd, 4),
                          "traffic": measured_traffic("m1_scan_kernel" if not layer.fused
                                                      else "m1_scan_kernel_f16x"),
-                         "peak_basis": "%d SMs x %d ex2/clk (SFU) x %.0f MHz; one exp per "
-                                       "state update" % (SMS, MUFU_PER_CLK, mhz_max),
+                         "peak_basis": peak_basis, "sfu_probe": ex2,
                          "hbm_achieved_gbs": round(scan_gbs, 1), "hbm_peak_gbs": pk["hbm_gbs"],
                          "hbm_frac": round(scan_gbs / pk["hbm_gbs"], 4),
                          "algorithmic_bytes_per_launch": layer.scan_bytes(),
@@ -385,6 +452,13 @@ def run_ours(args):
         if world == 1 and not args.no_cpu_baseline:
             try:
                 out["cpu_baseline"] = cpu_baseline(layer)
+                # the y / h_final of the last timed step against the oracle on
+                # the baseline's sample (the same inputs every step)
+                bb, yo, ho = layer.oracle_out
+                out["parity"] = parity(
+                    layer.y[:bb].float().cpu().numpy().reshape(bb * layer.d, layer.L), yo,
+                    layer.hf[:bb].cpu().numpy().reshape(bb * layer.d, layer.N), ho,
+                    "%d (batch, channel) rows of the last timed step" % (bb * layer.d))
             except Exception as e:  # report, keep the measured line
                 out["cpu_baseline"] = {"error": "%s: %s" % (type(e).__name__, e)}
         if world == 1 and not args.no_forms:
@@ -395,7 +469,7 @@ def run_ours(args):
             if not only or "m130m_int8_y" in only:
                 out["forms"]["m130m_int8_y"] = form_int8_y(torch, layer)
             out["forms"].update(run_forms(dev, pk, out["clocks"].get("sm_max_mhz") or
-                                          pk["sm_max_mhz"], only=only, layer=layer))
+                                          pk["sm_max_mhz"], only=only, layer=layer, ex2=ex2))
         print(json.dumps(out), flush=True)
 
 
@@ -433,13 +507,12 @@ def setup_decode(torch, dev, steps=None):
                                         T(bs), T(cs))
     state = T(raw["state"])
     y = torch.empty((b, H, P), dtype=torch.float16, device=dev)
-    del raw
 
     def step(t):
         api.state_update(state, xq[t], dt[t], A, Bq[t], Cq[t], bs_t, cs_t, gs, x_group=grp_t,
                          x_scale=xs_t, D=D, y=y)
 
-    return dict(b=b, H=H, P=P, N=N, G=G, S=S, step=step)
+    return dict(b=b, H=H, P=P, N=N, G=G, S=S, gs=gs, k=k, step=step, raw=raw, state=state, y=y)
 
 
 def e2e_pipelined(torch, layer, steps):
@@ -593,6 +666,39 @@ def form_int8_y(torch, layer):
                                        "ms_per_step": round(t_s * 1e3, 4)}}
 
 
+def _units_value(units_tokens_ch, seconds):
+    return round(units_tokens_ch / seconds / 1e9, 6)
+
+
+def oracle_timing(run, single, allc, threads, what):
+    """The oracle, as it stands, timed twice on bounded samples of a form's
+    workload: `single` (n_units, tokens*channels) on one thread, `allc` on
+    all host cores.  run(n_units, threads) computes the sample and returns
+    its outputs (those of the all-core run are returned for the parity check)."""
+    t = time.perf_counter()
+    run(single[0], 1)
+    t1 = time.perf_counter() - t
+    t = time.perf_counter()
+    out = run(allc[0], threads)
+    ta = time.perf_counter() - t
+    return {"kind": "oracle", "unit": UNIT,
+            "single_thread": {"value": _units_value(single[1], t1), "seconds": round(t1, 3),
+                              "cores": 1, "sample": "%d %s" % (single[0], what)},
+            "all_cores": {"value": _units_value(allc[1], ta), "seconds": round(ta, 3),
+                          "cores": threads, "sample": "%d %s" % (allc[0], what)},
+            "value": _units_value(allc[1], ta), "cores": threads,
+            "sample": "%d %s on %d threads" % (allc[0], what, threads)}, out
+
+
+def _threaded_units(fn, units, threads):
+    """fn(units_slice) over `threads` Python threads (the oracle's C calls run
+    without the interpreter lock); returns the per-slice results in order."""
+    import concurrent.futures as cf
+    parts = [p for p in np.array_split(np.asarray(units), max(1, threads)) if p.size]
+    with cf.ThreadPoolExecutor(max_workers=len(parts)) as ex:
+        return list(ex.map(fn, parts))
+
+
 def form_decode(torch, dev, pk):
     """decode8b: 1000 chained single-token state updates."""
     c = setup_decode(torch, dev)
@@ -602,9 +708,62 @@ def form_decode(torch, dev, pk):
         for t in range(S):
             c["step"](t)
 
+    # parity: the first step from the initial state, then restore it
+    from oracle import oracle as O
+    raw = c["raw"]
+    st0 = c["state"].clone()
+    c["step"](0)
+    torch.cuda.synchronize()
+    y_gpu = c["y"].float().cpu().numpy().reshape(b * H, P)
+    st1 = c["state"].cpu().numpy().reshape(b * H, P, N)
+    c["state"].copy_(st0)
+    del st0
+    gs, k = c["gs"], c["k"]
+    head_abs = np.abs(raw["x"].astype(np.float32)).max(axis=(0, 1, 3))
+    ohc, oxs = O.cluster_by_absmax(head_abs.astype(np.float64), k)
+    ogrp = np.repeat(ohc, P).astype(np.int32)
+    omap = np.arange(G * N) // gs
+    Bf = raw["B"].reshape(S * b, G * N)
+    Cf = raw["C"].reshape(S * b, G * N)
+    _, obs, _ = O.quantize_groups(Bf, S * b, G * N, 1, omap, G * N // gs, O.SCALE_ABSMAX)
+    _, ocs, _ = O.quantize_groups(Cf, S * b, G * N, 1, omap, G * N // gs, O.SCALE_ABSMAX)
+    nst = 8  # steps in the timed oracle sample
+    ox, _, _ = O.quantize_groups(raw["x"][:nst].reshape(nst * b, H * P), nst * b, H * P, 1, ogrp,
+                                 k, O.SCALE_STATIC, oxs)
+    oB, _, _ = O.quantize_groups(Bf[:nst * b], nst * b, G * N, 1, omap, G * N // gs,
+                                 O.SCALE_STATIC, obs)
+    oC, _, _ = O.quantize_groups(Cf[:nst * b], nst * b, G * N, 1, omap, G * N // gs,
+                                 O.SCALE_STATIC, ocs)
+    ox, oB, oC = ox.reshape(nst, b, H, P), oB.reshape(nst, b, G, N), oC.reshape(nst, b, G, N)
+
+    def run(n_steps, threads):
+        units = np.arange(b * H)
+        state = raw["state"].reshape(b * H, P, N).astype(np.float64)
+
+        def part(us):
+            stp = np.ascontiguousarray(state[us])
+            ys = []
+            for t in range(n_steps):
+                ys.append(O.decode_step(stp, ox[t], raw["dt"][t], raw["A"], oB[t], oC[t], obs, ocs,
+                                        gs, x_group=ogrp, x_scale=oxs, D=raw["D"], units=us))
+            return ys[0], stp if n_steps == 1 else None
+
+        return _threaded_units(part, units, threads)
+
+    threads = O.default_threads()
+    base, _ = oracle_timing(run, (1, b * H * P), (nst, nst * b * H * P), threads,
+                            "chained steps over all %d (batch, head) states" % (b * H))
+    base["sample"] += " (of the 1000-step chain; the full chain would take ~%.0f s)" % (
+        1000 * base["all_cores"]["seconds"] / nst)
+    one = run(1, threads)
+    par = parity(y_gpu, np.concatenate([r[0] for r in one]), st1,
+                 np.concatenate([r[1] for r in one]),
+                 "step 1 of the chain, every (batch, head): y and the updated state")
+    del one
     sec = _timed(torch, chain, 2) / S
     byts = 2 * b * H * P * N * 4 + b * H * P * (1 + 2) + b * H * 2 + 2 * b * G * N
     return {"workload": "decode8b: b 64, H 128, P 64, N 128, G 8, 1000 chained steps",
+            "cpu_baseline": base, "parity": par,
             "value": round(b * H * P / sec / 1e9, 3), "unit": "Gtokens·ch/s",
             "us_per_step": round(sec * 1e6, 2),
             "roofline": {"bound": "hbm", "achieved": round(byts / sec / 1e9, 1),
@@ -629,7 +788,6 @@ def setup_softedge(torch, dev):
     smap = T(calibrate.state_group_map(G, N, gs))
     x, dt, z, B, C = (T(raw[k]) for k in ("x", "dt", "z", "B", "C"))
     A, D, bs_t, cs_t = T(raw["A"]), T(raw["D"]), T(bs), T(cs)
-    del raw
     codes = torch.empty(x.shape, dtype=torch.uint8, device=dev)
     Bq = torch.empty(B.shape, dtype=torch.int8, device=dev)
     Cq = torch.empty(C.shape, dtype=torch.int8, device=dev)
@@ -651,27 +809,61 @@ def setup_softedge(torch, dev):
         api.selective_scan(x, dt, A, Bq, Cq, bs_t, cs_t, gs, se_scale=s, se_lo=lo, se_hi=hi, D=D,
                            z=z, y=y, h_final=hf)
 
-    return dict(b=b, L=L, d=d, N=N, enc=enc, quant_bc=quant_bc, scan=scan, scan_fused=scan_fused)
+    return dict(b=b, L=L, d=d, N=N, G=G, gs=gs, enc=enc, quant_bc=quant_bc, scan=scan,
+                scan_fused=scan_fused, raw=raw, y=y, hf=hf)
 
 
-def form_softedge(torch, dev, pk, mhz):
+def softedge_oracle_check(torch, c):
+    """The oracle on sampled channel rows of the softedge workload: its own
+    thresholds (percentiles of |x| over the whole tensor) and encoder, its own
+    B / C quantizer (untimed), then the double-precision scan, timed on one
+    thread (8 rows) and on all cores (one batch row, 1536 rows); the all-core
+    sample against the GPU's y and h_final of the last scan."""
+    from oracle import oracle as O
+    raw = c["raw"]
+    b, L, d, N, G, gs = c["b"], c["L"], c["d"], c["N"], c["G"], c["gs"]
+    olo = np.float32(O.percentile_abs(raw["x"], 5.0))
+    ohi = np.float32(O.percentile_abs(raw["x"], 99.9))
+    osc = np.float32(np.float64(ohi) / 63.0)
+    ox, _ = O.softedge_encode(raw["x"][:1], osc, olo, ohi, 2)
+    gmap = np.arange(G * N) // gs
+    _, obs, _ = O.quantize_groups(raw["B"], b, G * N, L, gmap, G * N // gs, O.SCALE_ABSMAX)
+    _, ocs, _ = O.quantize_groups(raw["C"], b, G * N, L, gmap, G * N // gs, O.SCALE_ABSMAX)
+    oB, _, _ = O.quantize_groups(raw["B"][:1], 1, G * N, L, gmap, G * N // gs, O.SCALE_STATIC, obs)
+    oC, _, _ = O.quantize_groups(raw["C"][:1], 1, G * N, L, gmap, G * N // gs, O.SCALE_STATIC, ocs)
+    threads = O.default_threads()
+
+    def run(n, th):
+        return O.m1_scan(ox.reshape(1, d, L), raw["dt"][:1], raw["A"], oB.reshape(1, G, N, L),
+                         oC.reshape(1, G, N, L), obs, ocs, gs, se_scale=float(osc), D=raw["D"],
+                         z=raw["z"][:1], units=np.arange(n), threads=th)
+
+    base, (yo, ho) = oracle_timing(run, (8, 8 * L), (d, d * L), threads,
+                                   "channel rows of L %d" % L)
+    yg = c["y"][0].float().cpu().numpy()
+    hg = c["hf"][0].cpu().numpy()
+    return base, parity(yg, yo, hg, ho, "batch row 0: %d channel rows" % d)
+
+
+def form_softedge(torch, dev, pk, mhz, ex2=None):
     """softedge: encode binary16 x to soft-edge codes, quantize B/C, scan."""
     c = setup_softedge(torch, dev)
     b, L, d, N = c["b"], c["L"], c["d"], c["N"]
     enc, quant_bc, scan = c["enc"], c["quant_bc"], c["scan"]
     t_enc = _timed(torch, enc, 5)
     t_bc = _timed(torch, quant_bc, 5)
-    t_scan = _timed(torch, scan, 3)
     t_fused = _timed(torch, c["scan_fused"], 3)
+    t_scan = _timed(torch, scan, 3)  # last: its y is the one checked
+    base, par = softedge_oracle_check(torch, c)
     t = t_enc + t_bc + t_scan
     t_f = t_bc + t_fused
     n = b * L * d
     enc_bytes = n * 3
     upd = n * N
-    peak_upd = SMS * MUFU_PER_CLK * mhz * 1e6 / 1e9
+    peak_upd, _ = sfu_peak(ex2, mhz)
     return {"workload": "softedge: b 16, L 8192, d 1536, N 16; encode + scan",
             "value": round(n / t / 1e9, 3), "unit": "Gtokens·ch/s",
-            "ms_per_step": round(t * 1e3, 4),
+            "ms_per_step": round(t * 1e3, 4), "cpu_baseline": base, "parity": par,
             "x_path": "encode launch, then the scan reads the codes",
             "fused_path": {"x_path": "binary16 x soft-edge encoded inside the scan "
                                      "(byte-identical result)",
@@ -700,7 +892,6 @@ def setup_ssd(torch, dev):
     cs = calibrate.state_group_absmax_scales(raw["C"], G, N, gs, "lgn")
     x, dt, B, C = T(raw["x"]), T(raw["dt"]), T(raw["B"]), T(raw["C"])
     A, D, grp_t, xs_t, bs_t, cs_t = T(raw["A"]), T(raw["D"]), T(grp), T(xs), T(bs), T(cs)
-    del raw
     xq = torch.empty(x.shape, dtype=torch.int8, device=dev)
     Bq = torch.empty(B.shape, dtype=torch.int8, device=dev)
     Cq = torch.empty(C.shape, dtype=torch.int8, device=dev)
@@ -716,7 +907,44 @@ def setup_ssd(torch, dev):
         api.ssd_chunk_scan(xq, dt, A, Bq, Cq, bs_t, cs_t, gs, chunk=dm["chunk"], x_group=grp_t,
                            x_scale=xs_t, D=D, y=y, h_final=hf)
 
-    return dict(b=b, L=L, H=H, P=P, N=N, G=G, quant=quant, ssd=ssd)
+    return dict(b=b, L=L, H=H, P=P, N=N, G=G, gs=gs, k=k, quant=quant, ssd=ssd, raw=raw, y=y,
+                hf=hf)
+
+
+def ssd_oracle_check(torch, c):
+    """The oracle on sampled (batch, head) sequences of ssd27b: its own
+    calibration and quantizers from the raw arrays (untimed), then the
+    sequential double-precision scan, timed on one thread (one sequence) and
+    on all cores (one sequence per core); the all-core sample against the GPU's
+    y and h_final of the last timed call."""
+    from oracle import oracle as O
+    raw = c["raw"]
+    b, L, H, P, N, G, gs, k = c["b"], c["L"], c["H"], c["P"], c["N"], c["G"], c["gs"], c["k"]
+    y_gpu, hf_gpu = c["y"], c["hf"]
+    head_abs = np.abs(raw["x"].astype(np.float32)).max(axis=(0, 1, 3))
+    ohc, oxs = O.cluster_by_absmax(head_abs.astype(np.float64), k)
+    ogrp = np.repeat(ohc, P).astype(np.int32)
+    omap = np.arange(G * N) // gs
+    _, obs, _ = O.quantize_groups(raw["B"], b * L, G * N, 1, omap, G * N // gs, O.SCALE_ABSMAX)
+    _, ocs, _ = O.quantize_groups(raw["C"], b * L, G * N, 1, omap, G * N // gs, O.SCALE_ABSMAX)
+    ox, _, _ = O.quantize_groups(raw["x"], b * L, H * P, 1, ogrp, k, O.SCALE_STATIC, oxs)
+    oB, _, _ = O.quantize_groups(raw["B"], b * L, G * N, 1, omap, G * N // gs, O.SCALE_STATIC, obs)
+    oC, _, _ = O.quantize_groups(raw["C"], b * L, G * N, 1, omap, G * N // gs, O.SCALE_STATIC, ocs)
+    ox = ox.reshape(b, L, H, P)
+    oB, oC = oB.reshape(b, L, G, N), oC.reshape(b, L, G, N)
+    rng = np.random.default_rng(3)
+    threads = O.default_threads()
+    units = np.sort(rng.choice(b * H, size=min(b * H, threads), replace=False))
+
+    def run(n, th):
+        return O.ssd_scan(ox, raw["dt"], raw["A"], oB, oC, obs, ocs, gs, x_group=ogrp,
+                          x_scale=oxs, D=raw["D"], units=units[:n], threads=th)
+
+    base, (yo, ho) = oracle_timing(run, (1, L * P), (len(units), len(units) * L * P), threads,
+                                   "(batch, head) sequences of L %d x P %d" % (L, P))
+    yg = np.stack([y_gpu[u // H, :, u % H, :].float().cpu().numpy() for u in units])
+    hg = hf_gpu.reshape(b * H, P, N)[torch.as_tensor(units, device=hf_gpu.device)].cpu().numpy()
+    return base, parity(yg, yo, hg, ho, "%d sampled (batch, head) sequences" % len(units))
 
 
 def form_ssd(torch, dev, pk):
@@ -726,6 +954,7 @@ def form_ssd(torch, dev, pk):
     quant, ssd = c["quant"], c["ssd"]
     t_q = _timed(torch, quant, 5)
     t_s = _timed(torch, ssd, 5)
+    base, par = ssd_oracle_check(torch, c)
     q = 256  # the chunk length the algorithmic count refers to
     nch = L // q
     useful = (2 * q * (q + 1) // 2 * N * b * nch * G          # C B^T, causal half
@@ -737,7 +966,7 @@ def form_ssd(torch, dev, pk):
     return {"workload": "ssd27b: b 4, L 4096, H 80, P 64, N 128, G 1, chunk 256; quantize + SSD",
             "value": round(b * L * H * P / (t_q + t_s) / 1e9, 3), "unit": "Gtokens·ch/s",
             "ms_per_step": round((t_q + t_s) * 1e3, 4), "ssd_ms": round(t_s * 1e3, 4),
-            "quantize_ms": round(t_q * 1e3, 4),
+            "quantize_ms": round(t_q * 1e3, 4), "cpu_baseline": base, "parity": par,
             "roofline": {"bound": "tensor", "achieved": round(tf, 1), "peak": pk["bf16_tflops"],
                          "unit": "TFLOP/s", "frac": round(tf / pk["bf16_tflops"], 4),
                          "algorithmic_flops_per_launch": useful,
@@ -777,7 +1006,81 @@ def form_calibrate(torch, dev, pk, layer):
                                "unit": "GB/s", "frac": round(bs / t_pct / 1e9 / pk["hbm_gbs"], 4)}}
 
 
-def run_forms(dev, pk, mhz, only=None, layer=None):
+def form_tiny(torch, dev, reps=50):
+    """tiny (b 1, L 256, d 64, N 16, per-tensor absmax scales): latency of
+    one call, CUDA events around each call, median of `reps`.  The step is
+    the device-side per-tensor absmax quantize of x, B and C (scales computed
+    on the device) followed by the scan; the scan is also timed alone.  The
+    whole workload is checked against the oracle and timed on it."""
+    from oracle import oracle as O
+    from quantized_state_space_b200 import api, synth
+    dm, raw = synth.workload_inputs("tiny")
+    b, L, d, N, G, gs = (dm["batch"], dm["seqlen"], dm["dim"], dm["dstate"], dm["ngroups"],
+                         dm["state_group_size"])
+    T = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+    x, dt, B, C, A, D = (T(raw[k]) for k in ("x", "dt", "B", "C", "A", "D"))
+    g0 = torch.zeros(d, dtype=torch.int32, device=dev)
+    s0 = torch.zeros(G * N, dtype=torch.int32, device=dev)
+    xq = torch.empty(x.shape, dtype=torch.int8, device=dev)
+    Bq = torch.empty(B.shape, dtype=torch.int8, device=dev)
+    Cq = torch.empty(C.shape, dtype=torch.int8, device=dev)
+    y = torch.empty(x.shape, dtype=torch.float16, device=dev)
+    hf = torch.empty((b, d, N), dtype=torch.float32, device=dev)
+    sc = {}
+
+    def quant():
+        _, sc["x"] = api.quantize_groups(x, b, d, L, g0, 1, absmax=True, out=xq)
+        _, sc["B"] = api.quantize_groups(B, b, G * N, L, s0, 1, absmax=True, out=Bq)
+        _, sc["C"] = api.quantize_groups(C, b, G * N, L, s0, 1, absmax=True, out=Cq)
+
+    def scan():
+        api.selective_scan(xq, dt, A, Bq, Cq, sc["B"], sc["C"], gs, x_group=g0, x_scale=sc["x"],
+                           D=D, y=y, h_final=hf)
+
+    def step():
+        quant()
+        scan()
+
+    def lat(fn):
+        for _ in range(5):
+            fn()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(reps):
+            a, e = cuda_events(torch)
+            a.record()
+            fn()
+            e.record()
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(e) * 1e3)
+        return round(statistics.median(ts), 2)
+
+    t_step, t_scan = lat(step), lat(scan)
+    ox, oxs, _ = O.quantize_groups(raw["x"], b, d, L, np.zeros(d, np.int32), 1, O.SCALE_ABSMAX)
+    gm = np.zeros(G * N, np.int32)
+    oB, obs, _ = O.quantize_groups(raw["B"], b, G * N, L, gm, 1, O.SCALE_ABSMAX)
+    oC, ocs, _ = O.quantize_groups(raw["C"], b, G * N, L, gm, 1, O.SCALE_ABSMAX)
+
+    def run(n, th):
+        return O.m1_scan(ox, raw["dt"], raw["A"], oB, oC, obs, ocs, gs,
+                         x_group=np.zeros(d, np.int32), x_scale=oxs, D=raw["D"],
+                         units=np.arange(n), threads=th)
+
+    base, (yo, ho) = oracle_timing(run, (b * d, b * d * L), (b * d, b * d * L),
+                                   O.default_threads(), "channel rows of L %d (the whole "
+                                   "workload)" % L)
+    par = parity(y.float().cpu().numpy().reshape(b * d, L), yo,
+                 hf.cpu().numpy().reshape(b * d, N), ho, "the whole workload")
+    return {"workload": "tiny: b 1, L 256, d 64, N 16, per-tensor absmax scales; latency",
+            "step_us": t_step, "scan_us": t_scan,
+            "step": "device absmax quantize of x, B, C (3 calls, 12 launches incl. memsets) "
+                    "+ scan", "statistic": "median of %d calls, CUDA events per call" % reps,
+            "value": round(b * L * d / (t_step / 1e6) / 1e9, 4), "unit": UNIT,
+            "roofline": "launch-latency bound (98.6 KB, 262 k state updates): not meaningful",
+            "cpu_baseline": base, "parity": par}
+
+
+def run_forms(dev, pk, mhz, only=None, layer=None, ex2=None):
     import torch
     out = {}
     if layer is not None and (not only or "calibrate" in only):
@@ -788,7 +1091,8 @@ def run_forms(dev, pk, mhz, only=None, layer=None):
         torch.cuda.empty_cache()
     for name, fn in (("ssd27b", lambda: form_ssd(torch, dev, pk)),
                      ("decode8b", lambda: form_decode(torch, dev, pk)),
-                     ("softedge", lambda: form_softedge(torch, dev, pk, mhz))):
+                     ("softedge", lambda: form_softedge(torch, dev, pk, mhz, ex2)),
+                     ("tiny", lambda: form_tiny(torch, dev))):
         if only and name not in only:
             continue
         try:
@@ -850,6 +1154,10 @@ def run_kernel(args):
     torch.cuda.set_device(dev)
     from quantized_state_space_b200 import api
     name = args.kernel
+    if name == "ex2":
+        print(json.dumps(dict(kernel="ex2_rate_kernel (SFU exp2 throughput probe)",
+                              **measure_ex2(torch, dev))), flush=True)
+        return
     if name in ("scan", "scan-int8", "quantize"):
         lay = Layer(dev, 0, fused=name == "scan")
         lay.quantize()
@@ -895,13 +1203,13 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-forms", action="store_true")
     ap.add_argument("--forms", default="", help="comma list of m130m_other_x_path,m130m_int8_y,calibrate,ssd27b,decode8b,"
-                         "softedge")
+                         "softedge,tiny")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--fused", action="store_true",
                     help="headline step with binary16 x encoded inside the scan (byte-identical "
                          "result; default: x quantized by its own launch, the faster path here)")
     ap.add_argument("--kernel", choices=["scan", "scan-int8", "quantize", "ssd", "encode",
-                                         "softedge-scan", "decode"],
+                                         "softedge-scan", "decode", "ex2"],
                     help="profiling aid: run only this kernel on its workload")
     args = ap.parse_args()
     if args.kernel:

@@ -68,7 +68,13 @@ typedef enum {
 #define SSMQ_DEV_NONFINITE 1u /* a non-finite input element was met (coded 0) */
 #define SSMQ_DEV_BAD_GROUP 2u /* a device group id was out of range (coded 0) */
 #define SSMQ_DEV_BAD_SCALE 4u /* a device scale was negative / non-finite */
-#define SSMQ_DEV_TIMEOUT 8u   /* a bounded wait for the tensor core gave up */
+#define SSMQ_DEV_TIMEOUT 8u   /* a bounded device wait (tensor core, bulk copy) gave up;
+                                 the call's outputs are then incomplete.  Every such
+                                 wait probes at most ~2^20 times (about a second).
+                                 For tests of this path, the environment variable
+                                 SSMQ_WAIT_LIMIT=<probes> (read at each call) lowers
+                                 the limit of ssmq_quantize_groups' pipeline waits;
+                                 0 makes them give up at once. */
 
 typedef enum { SSMQ_F32 = 0, SSMQ_F16 = 1 } ssmq_dtype;
 typedef enum { SSMQ_SCALE_STATIC = 0, SSMQ_SCALE_ABSMAX = 1 } ssmq_scale_mode;
@@ -227,14 +233,26 @@ ssmq_status ssmq_softedge_calibrate(const void* src, ssmq_dtype dtype, int64_t n
                                     void* workspace, size_t ws_bytes, void* stream);
 
 /*
- * Allocation-free variants of the two percentile calls: the same computation
- * and results, with the library's own scratch instead of a caller workspace --
- * a static device array (one per device, found with cudaGetSymbolAddress for
- * the current device).  Nothing is allocated or freed.  Calls that use the
- * scratch of one device must not overlap (issue them on one stream, or
- * synchronise between them).  SSMQ_ERR_UNSUPPORTED if the scratch a call
- * needs exceeds the static array.  The pages have no counterpart: this is a
- * deployment convenience of this library, not part of the method.
+ * Allocation-free variants of the two percentile calls, for callers that may
+ * not allocate device memory: code running while a CUDA graph is captured,
+ * or a serving loop whose memory is fixed at start-up, cannot call cudaMalloc
+ * or an allocator for the workspace.  Same computation and results as the
+ * workspace forms; the scratch is the library's own file-scope device array
+ * of about 136 KB (ssmq_percentile_workspace_size() bytes), which every GPU
+ * that loads the library holds until the process exits.  Nothing is
+ * allocated or freed.
+ *   - The calls run on the current device (like every entry point): src,
+ *     out / thresholds and stream must belong to it.
+ *   - The first call on a device, with that device current, looks up the
+ *     device address of that device's copy of the array (cudaGetSymbolAddress)
+ *     and keeps it; make that first call before any stream capture.
+ *   - All calls on one device share the array and it keeps the last call's
+ *     contents (each call clears what it needs).  Calls that overlap on the
+ *     GPU race: issue them on one stream, or synchronise between them.
+ *   - SSMQ_ERR_UNSUPPORTED if a call needs more scratch than the array holds;
+ *     SSMQ_ERR_CUDA if the address lookup fails.
+ * The pages have no counterpart: this is a deployment convenience of this
+ * library, not part of the method.
  */
 ssmq_status ssmq_percentile_abs_noalloc(const void* src, ssmq_dtype dtype, int64_t n,
                                         const double* q, int32_t nq, float* out, void* stream);
@@ -537,6 +555,19 @@ ssmq_status ssmq_selective_state_update_w8(const ssmq_m1_decode_args* args, void
 const char* ssmq_last_error(void);
 /* Library ABI version (major * 10000 + minor * 100 + patch). */
 int32_t ssmq_version(void);
+
+/*
+ * Throughput probe of the special-function unit's base-2 exponential, the
+ * compute roof of the Mamba-1 scan (one exp(delta A) per state update; the
+ * Quamba2 abstract's Mamba1 recurrence, whose decay the pages leave to the
+ * hardware).  Launches sms * 8 CTAs of 256 threads; every thread evaluates
+ * iters * 8 independent ex2.approx.ftz.f32 and nothing else that the unit
+ * executes.  *n_ex2 (host) receives the number of exponentials; the caller
+ * times the launch on `stream` (rate = *n_ex2 / time).  sink: device fp32[1],
+ * not written.  Not part of the method.
+ * Errors: INVALID_ARG for iters < 1 or NULL sink / n_ex2.
+ */
+ssmq_status ssmq_probe_ex2(int32_t iters, float* sink, int64_t* n_ex2, void* stream);
 
 #ifdef __cplusplus
 }

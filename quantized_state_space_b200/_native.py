@@ -102,6 +102,7 @@ SIGNATURES = {
                                            _vp]),
     "ssmq_softedge_calibrate_noalloc": (_i32, [_vp, _i32, _i64, C.c_double, C.c_double, _f32,
                                                _vp, _vp]),
+    "ssmq_probe_ex2": (_i32, [_i32, _vp, C.POINTER(C.c_int64), _vp]),
     "ssmq_last_error": (C.c_char_p, []),
     "ssmq_version": (_i32, []),
 }
@@ -166,6 +167,13 @@ def ssmq_last_error():
 
 def ssmq_version():
     return lib().ssmq_version()
+
+
+def ssmq_probe_ex2(iters, sink, stream=None):
+    """Launches the exp2 throughput probe; returns the number of exponentials."""
+    n = C.c_int64(0)
+    _check(lib().ssmq_probe_ex2(int(iters), ptr(sink), C.byref(n), _stream(stream)))
+    return int(n.value)
 
 
 def ssmq_quantize_groups(src, outer, mid, inner, group_of_mid, n_groups, mode, scales, q_out,

@@ -5,6 +5,8 @@ PyTorch's job) and calls one C-ABI entry point through ``_native``; every step
 of the computation runs in the CUDA library.  Layouts and semantics are those
 of include/ssmq.h.
 """
+import contextlib
+
 import torch
 
 from . import _native as N
@@ -29,6 +31,33 @@ def _out(t, name, dtype, numel, device):
                          % (name, dtype, numel, t.dtype, t.numel()))
 
 
+def _in(t, name, dtypes, numel, device):
+    """A caller-supplied tensor that the call reads: on the call's device,
+    contiguous, of one of ``dtypes`` and with the element count the kernels
+    read (the library reads that many elements behind the pointer)."""
+    if t is None:
+        return
+    if not isinstance(dtypes, tuple):
+        dtypes = (dtypes,)
+    if t.device != device or not t.is_contiguous():
+        raise ValueError("%s must be a contiguous tensor on %s" % (name, device))
+    if t.dtype not in dtypes or (numel is not None and t.numel() != numel):
+        raise ValueError("%s must be %s with %s elements (got %s with %d)"
+                         % (name, "/".join(str(d) for d in dtypes),
+                            "any number of" if numel is None else numel, t.dtype, t.numel()))
+
+
+def _on(device):
+    """Launches go to the device that holds the tensors (and its current
+    stream), whatever device is current in the caller."""
+    if device.type == "cuda":
+        return torch.cuda.device(device)
+    return contextlib.nullcontext()
+
+
+_FP = (torch.float16, torch.float32)
+
+
 def _status(t, device):
     """The optional device status word: 32-bit, at least one element."""
     if t is None:
@@ -47,18 +76,51 @@ def _workspace(t, nbytes, device):
                          % (nbytes + 255, device))
 
 
+def _x_in(x, x_group, x_scale, channels, device, codes_only=False):
+    """x and its cluster map: int8 codes, soft-edge uint8 codes, or (Mamba-1
+    scan only) binary16 activations; the cluster map has one int32 entry per
+    channel and the scale table at least one fp32 entry."""
+    _in(x, "x", (torch.int8, torch.uint8) if codes_only else
+        (torch.int8, torch.uint8, torch.float16), None, device)
+    if x.dtype != torch.uint8:
+        _in(x_group, "x_group", torch.int32, channels, device)
+        _in(x_scale, "x_scale", torch.float32, None, device)
+        if x_group is None or x_scale is None or x_scale.numel() < 1:
+            raise ValueError("x_group and a non-empty x_scale are required for int8 / binary16 x")
+
+
+def _bc_in(B, C, B_scale, C_scale, numel, n_scales, device):
+    _in(B, "B", torch.int8, numel, device)
+    _in(C, "C", torch.int8, numel, device)
+    _in(B_scale, "B_scale", torch.float32, n_scales, device)
+    _in(C_scale, "C_scale", torch.float32, n_scales, device)
+
+
+def _n_scales(G, Nst, state_group_size):
+    if state_group_size < 1 or Nst % state_group_size:
+        raise ValueError("dstate must be a multiple of state_group_size >= 1")
+    return G * Nst // state_group_size
+
+
 def quantize_groups(src, outer, mid, inner, group_of_mid, n_groups, *, scales=None,
                     absmax=False, out=None, status=None):
     """int8 codes of ``src`` (float16/float32) with one scale per group.
     absmax=True computes the scales (returned); else ``scales`` are used."""
     _dev_check(src, group_of_mid, scales)
-    _out(out, "out", torch.int8, outer * mid * inner, src.device)
-    _status(status, src.device)
-    q = out if out is not None else torch.empty(src.shape, dtype=torch.int8, device=src.device)
-    if absmax:
-        scales = torch.empty(n_groups, dtype=torch.float32, device=src.device)
-    N.ssmq_quantize_groups(src, outer, mid, inner, group_of_mid, n_groups,
-                           N.SCALE_ABSMAX if absmax else N.SCALE_STATIC, scales, q, status=status)
+    dv = src.device
+    _in(src, "src", _FP, outer * mid * inner, dv)
+    _in(group_of_mid, "group_of_mid", torch.int32, mid, dv)
+    if not absmax:
+        _in(scales, "scales", torch.float32, n_groups, dv)
+    _out(out, "out", torch.int8, outer * mid * inner, dv)
+    _status(status, dv)
+    with _on(dv):
+        q = out if out is not None else torch.empty(src.shape, dtype=torch.int8, device=dv)
+        if absmax:
+            scales = torch.empty(n_groups, dtype=torch.float32, device=dv)
+        N.ssmq_quantize_groups(src, outer, mid, inner, group_of_mid, n_groups,
+                               N.SCALE_ABSMAX if absmax else N.SCALE_STATIC, scales, q,
+                               status=status)
     return q, scales
 
 
@@ -67,35 +129,47 @@ def quantize_groups_batch(jobs, *, status=None):
     layout class).  jobs: sequence of (src, outer, mid, inner, group_of_mid,
     n_groups, scales, out-or-None); returns the code tensors."""
     outs, descs = [], []
+    jobs = list(jobs)
+    if not jobs:
+        raise ValueError("at least one job")
+    dv = jobs[0][0].device
     for src, outer, mid, inner, gmap, n_groups, scales, out in jobs:
         _dev_check(src, gmap, scales)
-        _out(out, "out", torch.int8, outer * mid * inner, src.device)
-        _status(status, src.device)
-        q = out if out is not None else torch.empty(src.shape, dtype=torch.int8,
-                                                    device=src.device)
+        _in(src, "src", _FP, outer * mid * inner, dv)
+        _in(gmap, "group_of_mid", torch.int32, mid, dv)
+        _in(scales, "scales", torch.float32, n_groups, dv)
+        _out(out, "out", torch.int8, outer * mid * inner, dv)
+        _status(status, dv)
+        q = out if out is not None else torch.empty(src.shape, dtype=torch.int8, device=dv)
         outs.append(q)
         descs.append(dict(src=src, outer=outer, mid=mid, inner=inner, group_of_mid=gmap,
                           n_groups=n_groups, scales=scales, q_out=q))
-    N.ssmq_quantize_groups_batch(descs, status=status)
+    with _on(dv):
+        N.ssmq_quantize_groups_batch(descs, status=status)
     return outs
 
 
 def softedge_encode(src, scale, thr_lo, thr_hi, log2_ratio=2, *, out=None, status=None):
     _dev_check(src)
+    _in(src, "src", _FP, None, src.device)
     _out(out, "out", torch.uint8, src.numel(), src.device)
     _status(status, src.device)
-    codes = out if out is not None else torch.empty(src.shape, dtype=torch.uint8, device=src.device)
-    N.ssmq_softedge_encode(src, src.numel(), float(scale), float(thr_lo), float(thr_hi),
-                           log2_ratio, codes, status=status)
+    with _on(src.device):
+        codes = out if out is not None else torch.empty(src.shape, dtype=torch.uint8,
+                                                        device=src.device)
+        N.ssmq_softedge_encode(src, src.numel(), float(scale), float(thr_lo), float(thr_hi),
+                               log2_ratio, codes, status=status)
     return codes
 
 
 def softedge_decode(codes, scale, log2_ratio=2, *, out=None):
     _dev_check(codes)
+    _in(codes, "codes", torch.uint8, None, codes.device)
     _out(out, "out", torch.float32, codes.numel(), codes.device)
-    o = out if out is not None else torch.empty(codes.shape, dtype=torch.float32,
-                                                device=codes.device)
-    N.ssmq_softedge_decode(codes, codes.numel(), float(scale), log2_ratio, o)
+    with _on(codes.device):
+        o = out if out is not None else torch.empty(codes.shape, dtype=torch.float32,
+                                                    device=codes.device)
+        N.ssmq_softedge_decode(codes, codes.numel(), float(scale), log2_ratio, o)
     return o
 
 
@@ -115,7 +189,7 @@ def _x_fields(x, x_group, x_scale, se_scale, se_log2_ratio, se_lo=None, se_hi=No
                 n_x_groups=int(x_scale.numel()), se_log2_ratio=se_log2_ratio)
 
 
-def _y_fields(shape, device, y_group, y_scale, y_q, want_y, y):
+def _y_fields(shape, device, y_group, y_scale, y_q, want_y, y, channels):
     """Optional int8 output (static per-cluster scales) and the binary16 y."""
     f = {}
     n = 1
@@ -125,6 +199,10 @@ def _y_fields(shape, device, y_group, y_scale, y_q, want_y, y):
     _out(y_q, "y_q", torch.int8, n, device)
     if y_group is not None:
         _dev_check(y_group, y_scale)
+        _in(y_group, "y_group", torch.int32, channels, device)
+        _in(y_scale, "y_scale", torch.float32, None, device)
+        if y_scale is None or y_scale.numel() < 1:
+            raise ValueError("y_group needs a non-empty y_scale")
         if y_q is None:
             y_q = torch.empty(shape, dtype=torch.int8, device=device)
         f = dict(y_q=y_q, y_group=y_group, y_scale=y_scale, n_y_groups=int(y_scale.numel()))
@@ -147,19 +225,43 @@ def selective_scan(x, dt, A, B, C, B_scale, C_scale, state_group_size, *, x_grou
     b, d, L = x.shape
     G, Nst = B.shape[1], B.shape[2]
     _dev_check(x, dt, A, B, C, B_scale, C_scale, x_group, x_scale, D, z, dt_bias, h0)
-    _out(h_final, "h_final", torch.float32, b * d * Nst, x.device)
-    _status(status, x.device)
-    y, y_q, yf = _y_fields((b, d, L), x.device, y_group, y_scale, y_q, want_y, y)
-    if h_final is None and return_state:
-        h_final = torch.empty((b, d, Nst), dtype=torch.float32, device=x.device)
-    N.ssmq_selective_scan_w8(batch=b, seqlen=L, dim=d, dstate=Nst, ngroups=G,
-                             state_group_size=state_group_size,
-                             **_x_fields(x, x_group, x_scale, se_scale, se_log2_ratio, se_lo,
-                                         se_hi),
-                             dt=dt, dt_bias=dt_bias, dt_softplus=int(bool(dt_softplus)), A=A,
-                             D=D, z=z, B=B, C=C, B_scale=B_scale, C_scale=C_scale, h0=h0, y=y,
-                             h_final=h_final, status=status, **yf)
+    dv = x.device
+    _x_in(x, x_group, x_scale, d, dv)
+    _in(dt, "dt", torch.float16, b * d * L, dv)
+    _in(z, "z", torch.float16, b * d * L, dv)
+    _in(A, "A", torch.float32, d * Nst, dv)
+    _in(D, "D", torch.float32, d, dv)
+    _in(dt_bias, "dt_bias", torch.float32, d, dv)
+    _bc_in(B, C, B_scale, C_scale, b * G * Nst * L, _n_scales(G, Nst, state_group_size), dv)
+    _in(h0, "h0", torch.float32, b * d * Nst, dv)
+    _out(h_final, "h_final", torch.float32, b * d * Nst, dv)
+    _status(status, dv)
+    with _on(dv):
+        y, y_q, yf = _y_fields((b, d, L), dv, y_group, y_scale, y_q, want_y, y, d)
+        if h_final is None and return_state:
+            h_final = torch.empty((b, d, Nst), dtype=torch.float32, device=dv)
+        N.ssmq_selective_scan_w8(batch=b, seqlen=L, dim=d, dstate=Nst, ngroups=G,
+                                 state_group_size=state_group_size,
+                                 **_x_fields(x, x_group, x_scale, se_scale, se_log2_ratio, se_lo,
+                                             se_hi),
+                                 dt=dt, dt_bias=dt_bias, dt_softplus=int(bool(dt_softplus)), A=A,
+                                 D=D, z=z, B=B, C=C, B_scale=B_scale, C_scale=C_scale, h0=h0,
+                                 y=y, h_final=h_final, status=status, **yf)
     return (y, h_final, y_q) if yf else (y, h_final)
+
+
+def _ssd_inputs(x, dt, A, B, C, B_scale, C_scale, state_group_size, x_group, x_scale, D, z,
+                dt_bias, h0):
+    b, L, H, P = x.shape
+    G, Nst = B.shape[2], B.shape[3]
+    dv = x.device
+    _x_in(x, x_group, x_scale, H * P, dv, codes_only=True)
+    _in(dt, "dt", torch.float16, b * L * H, dv)
+    _in(z, "z", torch.float16, b * L * H * P, dv)
+    for t, name in ((A, "A"), (D, "D"), (dt_bias, "dt_bias")):
+        _in(t, name, torch.float32, H, dv)
+    _bc_in(B, C, B_scale, C_scale, b * L * G * Nst, _n_scales(G, Nst, state_group_size), dv)
+    _in(h0, "h0", torch.float32, b * H * P * Nst, dv)
 
 
 def _ssd_call(x, dt, A, B, C, B_scale, C_scale, state_group_size, chunk, x_group, x_scale,
@@ -195,17 +297,21 @@ def ssd_chunk_scan(x, dt, A, B, C, B_scale, C_scale, state_group_size, *, chunk=
     b, L, H, P = x.shape
     Nst = B.shape[3]
     _dev_check(x, dt, A, B, C, B_scale, C_scale, x_group, x_scale, D, z, dt_bias, h0, dec_final)
-    _out(h_final, "h_final", torch.float32, b * H * P * Nst, x.device)
-    _out(dec_final, "dec_final", torch.float32, b * H, x.device)
-    _status(status, x.device)
-    y, y_q, yf = _y_fields((b, L, H, P), x.device, y_group, y_scale, y_q, want_y, y)
-    if h_final is None and return_state:
-        h_final = torch.empty((b, H, P, Nst), dtype=torch.float32, device=x.device)
-    fields, wptr, ws = _ssd_call(x, dt, A, B, C, B_scale, C_scale, state_group_size, chunk,
-                                 x_group, x_scale, se_scale, se_log2_ratio, D, z, dt_bias,
-                                 dt_softplus, h0, y, h_final, max_segments, workspace, status,
-                                 dec_final, yf)
-    N.ssmq_ssd_chunk_scan_w8(workspace=wptr, ws_bytes=ws, **fields)
+    dv = x.device
+    _ssd_inputs(x, dt, A, B, C, B_scale, C_scale, state_group_size, x_group, x_scale, D, z,
+                dt_bias, h0)
+    _out(h_final, "h_final", torch.float32, b * H * P * Nst, dv)
+    _out(dec_final, "dec_final", torch.float32, b * H, dv)
+    _status(status, dv)
+    with _on(dv):
+        y, y_q, yf = _y_fields((b, L, H, P), dv, y_group, y_scale, y_q, want_y, y, H * P)
+        if h_final is None and return_state:
+            h_final = torch.empty((b, H, P, Nst), dtype=torch.float32, device=dv)
+        fields, wptr, ws = _ssd_call(x, dt, A, B, C, B_scale, C_scale, state_group_size, chunk,
+                                     x_group, x_scale, se_scale, se_log2_ratio, D, z, dt_bias,
+                                     dt_softplus, h0, y, h_final, max_segments, workspace,
+                                     status, dec_final, yf)
+        N.ssmq_ssd_chunk_scan_w8(workspace=wptr, ws_bytes=ws, **fields)
     return (y, h_final, y_q) if yf else (y, h_final)
 
 
@@ -219,14 +325,19 @@ def ssd_carry_in(x, dt, A, B, C, B_scale, C_scale, state_group_size, h_carry, y,
                h_final)
     b, L, H, P = x.shape
     Nst = B.shape[3]
-    _out(y, "y", torch.float16, b * L * H * P, x.device)
-    _out(h_carry, "h_carry", torch.float32, b * H * P * Nst, x.device)
-    _out(h_final, "h_final", torch.float32, b * H * P * Nst, x.device)
-    _status(status, x.device)
-    fields, wptr, ws = _ssd_call(x, dt, A, B, C, B_scale, C_scale, state_group_size, chunk,
-                                 x_group, x_scale, se_scale, se_log2_ratio, D, z, dt_bias,
-                                 dt_softplus, None, y, h_final, 0, workspace, status, None, {})
-    N.ssmq_ssd_carry_in(h_carry, workspace=wptr, ws_bytes=ws, **fields)
+    dv = x.device
+    _ssd_inputs(x, dt, A, B, C, B_scale, C_scale, state_group_size, x_group, x_scale, D, z,
+                dt_bias, None)
+    _out(y, "y", torch.float16, b * L * H * P, dv)
+    _out(h_carry, "h_carry", torch.float32, b * H * P * Nst, dv)
+    _out(h_final, "h_final", torch.float32, b * H * P * Nst, dv)
+    _status(status, dv)
+    with _on(dv):
+        fields, wptr, ws = _ssd_call(x, dt, A, B, C, B_scale, C_scale, state_group_size, chunk,
+                                     x_group, x_scale, se_scale, se_log2_ratio, D, z, dt_bias,
+                                     dt_softplus, None, y, h_final, 0, workspace, status, None,
+                                     {})
+        N.ssmq_ssd_carry_in(h_carry, workspace=wptr, ws_bytes=ws, **fields)
     return y, h_final
 
 
@@ -241,8 +352,11 @@ def state_chain(h_ends, decs):
     n_parts = he.shape[0]
     units = dc[0].numel()
     elems = he[0].numel() // max(units, 1)
-    out = torch.empty(he.shape[1:], dtype=torch.float32, device=he.device)
-    N.ssmq_state_chain(he, dc, n_parts, units, elems, out)
+    _in(he, "h_ends", torch.float32, n_parts * units * elems, he.device)
+    _in(dc, "decs", torch.float32, n_parts * units, he.device)
+    with _on(he.device):
+        out = torch.empty(he.shape[1:], dtype=torch.float32, device=he.device)
+        N.ssmq_state_chain(he, dc, n_parts, units, elems, out)
     return out
 
 
@@ -254,17 +368,26 @@ def state_update(state, x, dt, A, B, C, B_scale, C_scale, state_group_size, *, x
     b, H, P, Nst = state.shape
     G = B.shape[1]
     _dev_check(state, x, dt, A, B, C, B_scale, C_scale, x_group, x_scale, D, z, dt_bias)
-    _out(state, "state", torch.float32, b * H * P * Nst, state.device)
-    _out(y, "y", torch.float16, b * H * P, state.device)
-    _status(status, state.device)
-    if y is None:
-        y = torch.empty((b, H, P), dtype=torch.float16, device=state.device)
-    N.ssmq_state_update_w8(batch=b, nheads=H, headdim=P, dstate=Nst, ngroups=G,
-                           state_group_size=state_group_size,
-                           **_x_fields(x, x_group, x_scale, se_scale, se_log2_ratio),
-                           dt=dt, dt_bias=dt_bias, dt_softplus=int(bool(dt_softplus)), A=A, D=D,
-                           z=z, B=B, C=C, B_scale=B_scale, C_scale=C_scale, state=state, y=y,
-                           status=status)
+    dv = state.device
+    _x_in(x, x_group, x_scale, H * P, dv, codes_only=True)
+    _in(x, "x", (torch.int8, torch.uint8), b * H * P, dv)
+    _in(dt, "dt", torch.float16, b * H, dv)
+    _in(z, "z", torch.float16, b * H * P, dv)
+    for t, name in ((A, "A"), (D, "D"), (dt_bias, "dt_bias")):
+        _in(t, name, torch.float32, H, dv)
+    _bc_in(B, C, B_scale, C_scale, b * G * Nst, _n_scales(G, Nst, state_group_size), dv)
+    _out(state, "state", torch.float32, b * H * P * Nst, dv)
+    _out(y, "y", torch.float16, b * H * P, dv)
+    _status(status, dv)
+    with _on(dv):
+        if y is None:
+            y = torch.empty((b, H, P), dtype=torch.float16, device=dv)
+        N.ssmq_state_update_w8(batch=b, nheads=H, headdim=P, dstate=Nst, ngroups=G,
+                               state_group_size=state_group_size,
+                               **_x_fields(x, x_group, x_scale, se_scale, se_log2_ratio),
+                               dt=dt, dt_bias=dt_bias, dt_softplus=int(bool(dt_softplus)), A=A,
+                               D=D, z=z, B=B, C=C, B_scale=B_scale, C_scale=C_scale,
+                               state=state, y=y, status=status)
     return y
 
 
@@ -276,17 +399,29 @@ def selective_state_update(state, x, dt, A, B, C, B_scale, C_scale, state_group_
     b, d, Nst = state.shape
     G = B.shape[1]
     _dev_check(state, x, dt, A, B, C, B_scale, C_scale, x_group, x_scale, D, z, dt_bias)
-    _out(state, "state", torch.float32, b * d * Nst, state.device)
-    _out(y, "y", torch.float16, b * d, state.device)
-    _status(status, state.device)
-    if y is None:
-        y = torch.empty((b, d), dtype=torch.float16, device=state.device)
-    N.ssmq_selective_state_update_w8(batch=b, dim=d, dstate=Nst, ngroups=G,
-                                     state_group_size=state_group_size,
-                                     **_x_fields(x, x_group, x_scale, se_scale, se_log2_ratio),
-                                     dt=dt, dt_bias=dt_bias, dt_softplus=int(bool(dt_softplus)),
-                                     A=A, D=D, z=z, B=B, C=C, B_scale=B_scale, C_scale=C_scale,
-                                     state=state, y=y, status=status)
+    dv = state.device
+    _x_in(x, x_group, x_scale, d, dv, codes_only=True)
+    _in(x, "x", (torch.int8, torch.uint8), b * d, dv)
+    _in(dt, "dt", torch.float16, b * d, dv)
+    _in(z, "z", torch.float16, b * d, dv)
+    _in(A, "A", torch.float32, d * Nst, dv)
+    _in(D, "D", torch.float32, d, dv)
+    _in(dt_bias, "dt_bias", torch.float32, d, dv)
+    _bc_in(B, C, B_scale, C_scale, b * G * Nst, _n_scales(G, Nst, state_group_size), dv)
+    _out(state, "state", torch.float32, b * d * Nst, dv)
+    _out(y, "y", torch.float16, b * d, dv)
+    _status(status, dv)
+    with _on(dv):
+        if y is None:
+            y = torch.empty((b, d), dtype=torch.float16, device=dv)
+        N.ssmq_selective_state_update_w8(batch=b, dim=d, dstate=Nst, ngroups=G,
+                                         state_group_size=state_group_size,
+                                         **_x_fields(x, x_group, x_scale, se_scale,
+                                                     se_log2_ratio),
+                                         dt=dt, dt_bias=dt_bias,
+                                         dt_softplus=int(bool(dt_softplus)), A=A, D=D, z=z, B=B,
+                                         C=C, B_scale=B_scale, C_scale=C_scale, state=state, y=y,
+                                         status=status)
     return y
 
 
@@ -295,21 +430,27 @@ def selective_state_update(state, x, dt, A, B, C, B_scale, C_scale, state_group_
 def group_absmax(src, outer, mid, inner, group_of_mid, n_groups, *, out=None, status=None):
     """Exact max |v| per group over the finite elements (float32[n_groups])."""
     _dev_check(src, group_of_mid)
-    _out(out, "out", torch.float32, n_groups, src.device)
-    _status(status, src.device)
-    a = out if out is not None else torch.empty(n_groups, dtype=torch.float32, device=src.device)
-    N.ssmq_group_absmax(src, outer, mid, inner, group_of_mid, n_groups, a, status=status)
+    dv = src.device
+    _in(src, "src", _FP, outer * mid * inner, dv)
+    _in(group_of_mid, "group_of_mid", torch.int32, mid, dv)
+    _out(out, "out", torch.float32, n_groups, dv)
+    _status(status, dv)
+    with _on(dv):
+        a = out if out is not None else torch.empty(n_groups, dtype=torch.float32, device=dv)
+        N.ssmq_group_absmax(src, outer, mid, inner, group_of_mid, n_groups, a, status=status)
     return a
 
 
 def cluster_by_absmax(absmax, k, *, status=None):
     """Sort-and-cluster on the device: (cluster id per channel int32, scales float32[k])."""
     _dev_check(absmax)
+    _in(absmax, "absmax", torch.float32, None, absmax.device)
     _status(status, absmax.device)
     n = absmax.numel()
-    cl = torch.empty(n, dtype=torch.int32, device=absmax.device)
-    sc = torch.empty(k, dtype=torch.float32, device=absmax.device)
-    N.ssmq_cluster_by_absmax(absmax, n, k, cl, sc, status=status)
+    with _on(absmax.device):
+        cl = torch.empty(n, dtype=torch.int32, device=absmax.device)
+        sc = torch.empty(k, dtype=torch.float32, device=absmax.device)
+        N.ssmq_cluster_by_absmax(absmax, n, k, cl, sc, status=status)
     return cl, sc
 
 
@@ -322,14 +463,21 @@ def _pct_workspace(device, workspace):
     return (base + 255) // 256 * 256, nb
 
 
+def _qlist(q):
+    return [float(v) for v in (q if hasattr(q, "__len__") else [q])]
+
+
 def percentile_abs(src, q, *, out=None, workspace=None):
     """Percentiles (linear interpolation) of |src| over its finite elements."""
     _dev_check(src)
-    q = [float(v) for v in (q if hasattr(q, "__len__") else [q])]
+    _in(src, "src", _FP, None, src.device)
+    q = _qlist(q)
     _out(out, "out", torch.float32, len(q), src.device)
-    o = out if out is not None else torch.empty(len(q), dtype=torch.float32, device=src.device)
-    wptr, nb = _pct_workspace(src.device, workspace)
-    N.ssmq_percentile_abs(src, src.numel(), q, o, wptr, nb)
+    with _on(src.device):
+        o = out if out is not None else torch.empty(len(q), dtype=torch.float32,
+                                                    device=src.device)
+        wptr, nb = _pct_workspace(src.device, workspace)
+        N.ssmq_percentile_abs(src, src.numel(), q, o, wptr, nb)
     return o
 
 
@@ -337,9 +485,40 @@ def softedge_calibrate(src, thresholds=None, *, q_lo=5.0, q_hi=99.9, alpha=1.0, 
     """Soft-edge parameters {scale, lo, hi} (float32[3], updated in place):
     percentiles of |src|, blended into the running values when alpha < 1."""
     _dev_check(src)
+    _in(src, "src", _FP, None, src.device)
     _out(thresholds, "thresholds", torch.float32, 3, src.device)
-    thr = thresholds if thresholds is not None else torch.zeros(3, dtype=torch.float32,
-                                                                  device=src.device)
-    wptr, nb = _pct_workspace(src.device, workspace)
-    N.ssmq_softedge_calibrate(src, src.numel(), q_lo, q_hi, alpha, thr, wptr, nb)
+    with _on(src.device):
+        thr = thresholds if thresholds is not None else torch.zeros(3, dtype=torch.float32,
+                                                                      device=src.device)
+        wptr, nb = _pct_workspace(src.device, workspace)
+        N.ssmq_softedge_calibrate(src, src.numel(), q_lo, q_hi, alpha, thr, wptr, nb)
     return thr
+
+
+# Allocation-free forms: the library's own static device scratch replaces the
+# workspace, so a caller that may not allocate device memory (a CUDA graph
+# being captured, an allocator-free serving loop) can still calibrate.  The
+# out / thresholds tensors are the caller's.  Calls on one device share the
+# scratch: do not let two overlap on the GPU.
+
+def percentile_abs_noalloc(src, q, out):
+    """percentile_abs into the caller's ``out`` (float32[len(q)]), with the
+    library's static scratch; nothing is allocated."""
+    _dev_check(src, out)
+    _in(src, "src", _FP, None, src.device)
+    q = _qlist(q)
+    _out(out, "out", torch.float32, len(q), src.device)
+    with _on(src.device):
+        N.ssmq_percentile_abs_noalloc(src, src.numel(), q, out)
+    return out
+
+
+def softedge_calibrate_noalloc(src, thresholds, *, q_lo=5.0, q_hi=99.9, alpha=1.0):
+    """softedge_calibrate on the caller's ``thresholds`` (float32[3], in
+    place), with the library's static scratch; nothing is allocated."""
+    _dev_check(src, thresholds)
+    _in(src, "src", _FP, None, src.device)
+    _out(thresholds, "thresholds", torch.float32, 3, src.device)
+    with _on(src.device):
+        N.ssmq_softedge_calibrate_noalloc(src, src.numel(), q_lo, q_hi, alpha, thresholds)
+    return thresholds

@@ -6,6 +6,8 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "../../include/ssmq.h"
 #include "internal.h"
 
@@ -20,6 +22,15 @@ ssmq_status fail(ssmq_status s, const char* fmt, ...) {
   va_end(ap);
   return s;
 }
+
+// One NVTX range per entry-point call (named after the entry point), seen by
+// profilers as the host-side span of the call; a no-op without a tool.
+struct Range {
+  explicit Range(const char* name) { nvtxRangePushA(name); }
+  ~Range() { nvtxRangePop(); }
+  Range(const Range&) = delete;
+  Range& operator=(const Range&) = delete;
+};
 
 bool aligned16(const void* p) { return p == nullptr || (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -124,6 +135,7 @@ ssmq_status ssmq_quantize_groups(const void* src, ssmq_dtype dtype, int64_t oute
                                  ssmq_scale_mode mode, float* scales, int8_t* q_out,
                                  uint32_t* status, void* stream) {
   const char* fn = "ssmq_quantize_groups";
+  Range nvtx_range(fn);
   REQUIRE(dtype == SSMQ_F32 || dtype == SSMQ_F16, SSMQ_ERR_INVALID_ARG, "%s: bad dtype %d", fn,
           (int)dtype);
   REQUIRE(mode == SSMQ_SCALE_STATIC || mode == SSMQ_SCALE_ABSMAX, SSMQ_ERR_INVALID_ARG,
@@ -149,6 +161,7 @@ ssmq_status ssmq_quantize_groups(const void* src, ssmq_dtype dtype, int64_t oute
 ssmq_status ssmq_quantize_groups_batch(const ssmq_quant_job* jobs, int32_t n_jobs,
                                        uint32_t* status, void* stream) {
   const char* fn = "ssmq_quantize_groups_batch";
+  Range nvtx_range(fn);
   REQUIRE(jobs != nullptr, SSMQ_ERR_INVALID_ARG, "%s: jobs is NULL", fn);
   REQUIRE(n_jobs >= 1 && n_jobs <= ssmq::kMaxQuantJobs, SSMQ_ERR_INVALID_ARG,
           "%s: n_jobs must be in [1, %d] (got %d)", fn, ssmq::kMaxQuantJobs, (int)n_jobs);
@@ -181,6 +194,7 @@ ssmq_status ssmq_softedge_encode(const void* src, ssmq_dtype dtype, int64_t n, f
                                  float thr_lo, float thr_hi, int32_t log2_ratio, uint8_t* codes,
                                  uint32_t* status, void* stream) {
   const char* fn = "ssmq_softedge_encode";
+  Range nvtx_range(fn);
   REQUIRE(dtype == SSMQ_F32 || dtype == SSMQ_F16, SSMQ_ERR_INVALID_ARG, "%s: bad dtype", fn);
   REQUIRE(n >= 0, SSMQ_ERR_INVALID_ARG, "%s: negative size", fn);
   REQUIRE(thr_lo <= thr_hi, SSMQ_ERR_INVALID_ARG,
@@ -199,6 +213,7 @@ ssmq_status ssmq_group_absmax(const void* src, ssmq_dtype dtype, int64_t outer, 
                               int64_t inner, const int32_t* group_of_mid, int32_t n_groups,
                               float* absmax, uint32_t* status, void* stream) {
   const char* fn = "ssmq_group_absmax";
+  Range nvtx_range(fn);
   REQUIRE(dtype == SSMQ_F32 || dtype == SSMQ_F16, SSMQ_ERR_INVALID_ARG, "%s: bad dtype %d", fn,
           (int)dtype);
   REQUIRE(outer >= 0 && mid >= 0 && inner >= 0, SSMQ_ERR_INVALID_ARG, "%s: negative size", fn);
@@ -216,6 +231,7 @@ ssmq_status ssmq_group_absmax(const void* src, ssmq_dtype dtype, int64_t outer, 
 ssmq_status ssmq_cluster_by_absmax(const float* absmax, int64_t n, int32_t k, int32_t* cluster_of,
                                    float* scales, uint32_t* status, void* stream) {
   const char* fn = "ssmq_cluster_by_absmax";
+  Range nvtx_range(fn);
   REQUIRE(n >= 1 && k >= 1 && k <= n, SSMQ_ERR_INVALID_ARG, "%s: need 1 <= k <= n", fn);
   REQUIRE(n <= 65536, SSMQ_ERR_UNSUPPORTED, "%s: n > 65536 channels", fn);
   REQUIRE(absmax && cluster_of && scales, SSMQ_ERR_INVALID_ARG, "%s: NULL tensor", fn);
@@ -225,6 +241,16 @@ ssmq_status ssmq_cluster_by_absmax(const float* absmax, int64_t n, int32_t k, in
                 fn);
 }
 
+ssmq_status ssmq_probe_ex2(int32_t iters, float* sink, int64_t* n_ex2, void* stream) {
+  const char* fn = "ssmq_probe_ex2";
+  Range nvtx_range(fn);
+  REQUIRE(iters >= 1 && sink && n_ex2, SSMQ_ERR_INVALID_ARG,
+          "%s: iters >= 1, sink and n_ex2 required", fn);
+  REQUIRE(aligned16(sink), SSMQ_ERR_ALIGNMENT, "%s: sink must be 16-byte aligned", fn);
+  if (injected(fn)) return fail(SSMQ_ERR_CUDA, "%s: injected launch failure", fn);
+  return finish(ssmq::launch_probe_ex2(iters, sink, n_ex2, (cudaStream_t)stream), fn);
+}
+
 size_t ssmq_percentile_workspace_size(void) { return ssmq::percentile_workspace_bytes(); }
 
 
@@ -232,6 +258,7 @@ ssmq_status ssmq_percentile_abs(const void* src, ssmq_dtype dtype, int64_t n, co
                                 int32_t nq, float* out, void* workspace, size_t ws_bytes,
                                 void* stream) {
   const char* fn = "ssmq_percentile_abs";
+  Range nvtx_range(fn);
   CHECK(check_src(src, dtype, n, fn));
   CHECK(check_pct_q(q, nq, out, fn));
   CHECK(check_ws(workspace, ws_bytes, fn));
@@ -245,6 +272,7 @@ ssmq_status ssmq_softedge_calibrate(const void* src, ssmq_dtype dtype, int64_t n
                                     double q_hi, float alpha, float* thresholds, void* workspace,
                                     size_t ws_bytes, void* stream) {
   const char* fn = "ssmq_softedge_calibrate";
+  Range nvtx_range(fn);
   CHECK(check_src(src, dtype, n, fn));
   CHECK(check_se_cal(q_lo, q_hi, alpha, thresholds, fn));
   CHECK(check_ws(workspace, ws_bytes, fn));
@@ -272,6 +300,7 @@ ssmq_status static_scratch(void** ws, const char* fn) {
 ssmq_status ssmq_percentile_abs_noalloc(const void* src, ssmq_dtype dtype, int64_t n,
                                         const double* q, int32_t nq, float* out, void* stream) {
   const char* fn = "ssmq_percentile_abs_noalloc";
+  Range nvtx_range(fn);
   CHECK(check_src(src, dtype, n, fn));  // argument errors before any device call
   CHECK(check_pct_q(q, nq, out, fn));
   void* ws = nullptr;
@@ -284,6 +313,7 @@ ssmq_status ssmq_softedge_calibrate_noalloc(const void* src, ssmq_dtype dtype, i
                                             double q_lo, double q_hi, float alpha,
                                             float* thresholds, void* stream) {
   const char* fn = "ssmq_softedge_calibrate_noalloc";
+  Range nvtx_range(fn);
   CHECK(check_src(src, dtype, n, fn));
   CHECK(check_se_cal(q_lo, q_hi, alpha, thresholds, fn));
   void* ws = nullptr;
@@ -295,6 +325,7 @@ ssmq_status ssmq_softedge_calibrate_noalloc(const void* src, ssmq_dtype dtype, i
 ssmq_status ssmq_softedge_decode(const uint8_t* codes, int64_t n, float scale, int32_t log2_ratio,
                                  float* out, void* stream) {
   const char* fn = "ssmq_softedge_decode";
+  Range nvtx_range(fn);
   REQUIRE(n >= 0, SSMQ_ERR_INVALID_ARG, "%s: negative size", fn);
   REQUIRE(log2_ratio >= 0 && log2_ratio <= 8, SSMQ_ERR_INVALID_ARG,
           "%s: log2_ratio must be in [0, 8]", fn);
@@ -308,6 +339,7 @@ ssmq_status ssmq_softedge_decode(const uint8_t* codes, int64_t n, float scale, i
 
 ssmq_status ssmq_selective_scan_w8(const ssmq_scan_args* a, void* stream) {
   const char* fn = "ssmq_selective_scan_w8";
+  Range nvtx_range(fn);
   REQUIRE(a != nullptr, SSMQ_ERR_INVALID_ARG, "%s: args is NULL", fn);
   REQUIRE(a->batch >= 0 && a->seqlen >= 0 && a->dim >= 0, SSMQ_ERR_INVALID_ARG,
           "%s: negative size", fn);
@@ -400,6 +432,7 @@ ssmq_status check_ssd(const ssmq_ssd_args* a, void* workspace, size_t ws_bytes, 
 ssmq_status ssmq_ssd_chunk_scan_w8(const ssmq_ssd_args* a, void* workspace, size_t ws_bytes,
                                    void* stream) {
   const char* fn = "ssmq_ssd_chunk_scan_w8";
+  Range nvtx_range(fn);
   bool skip;
   CHECK(check_ssd(a, workspace, ws_bytes, fn, &skip));
   if (skip) return SSMQ_OK;
@@ -410,6 +443,7 @@ ssmq_status ssmq_ssd_chunk_scan_w8(const ssmq_ssd_args* a, void* workspace, size
 ssmq_status ssmq_ssd_carry_in(const ssmq_ssd_args* a, const float* h_carry, void* workspace,
                               size_t ws_bytes, void* stream) {
   const char* fn = "ssmq_ssd_carry_in";
+  Range nvtx_range(fn);
   bool skip;
   CHECK(check_ssd(a, workspace, ws_bytes, fn, &skip));
   if (skip) return SSMQ_OK;
@@ -424,6 +458,7 @@ ssmq_status ssmq_ssd_carry_in(const ssmq_ssd_args* a, const float* h_carry, void
 ssmq_status ssmq_state_chain(const float* h_end, const float* dec, int32_t n_parts,
                              int64_t units, int64_t elems, float* h_out, void* stream) {
   const char* fn = "ssmq_state_chain";
+  Range nvtx_range(fn);
   REQUIRE(n_parts >= 1, SSMQ_ERR_INVALID_ARG, "%s: n_parts must be >= 1", fn);
   REQUIRE(units >= 0 && elems >= 0, SSMQ_ERR_INVALID_ARG, "%s: negative size", fn);
   if (units == 0 || elems == 0) return SSMQ_OK;
@@ -437,6 +472,7 @@ ssmq_status ssmq_state_chain(const float* h_end, const float* dec, int32_t n_par
 
 ssmq_status ssmq_state_update_w8(const ssmq_decode_args* a, void* stream) {
   const char* fn = "ssmq_state_update_w8";
+  Range nvtx_range(fn);
   REQUIRE(a != nullptr, SSMQ_ERR_INVALID_ARG, "%s: args is NULL", fn);
   REQUIRE(a->batch >= 0 && a->nheads >= 0 && a->headdim >= 0, SSMQ_ERR_INVALID_ARG,
           "%s: negative size", fn);
@@ -462,6 +498,7 @@ ssmq_status ssmq_state_update_w8(const ssmq_decode_args* a, void* stream) {
 
 ssmq_status ssmq_selective_state_update_w8(const ssmq_m1_decode_args* a, void* stream) {
   const char* fn = "ssmq_selective_state_update_w8";
+  Range nvtx_range(fn);
   REQUIRE(a != nullptr, SSMQ_ERR_INVALID_ARG, "%s: args is NULL", fn);
   REQUIRE(a->batch >= 0 && a->dim >= 0, SSMQ_ERR_INVALID_ARG, "%s: negative size", fn);
   REQUIRE(a->ngroups >= 1 && a->dim % a->ngroups == 0, SSMQ_ERR_INVALID_ARG,

@@ -14,6 +14,8 @@
 //                         one 15-bit histogram pass for binary16 input (the
 //                         bins are the values), three passes (15 + 8 + 8 bits)
 //                         for fp32; the interpolation is done in double.
+#include <atomic>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -298,12 +300,25 @@ __device__ __align__(256) uint8_t g_pct_scratch[kPctWsBytes];
 
 }  // namespace
 
+// Device address of each device's copy of the array, resolved by the first
+// call made while that device is current (a host-side stand-in is all the
+// symbol name gives host code).  Racing first calls store the same value.
+static constexpr int kMaxDevices = 64;
+static std::atomic<void*> g_scratch_addr[kMaxDevices];
+
 void* percentile_static_scratch(size_t need, cudaError_t* err) {
   *err = cudaSuccess;
   if (need > kPctWsBytes) return nullptr;  // caller reports the size mismatch
-  void* p = nullptr;
+  int dev = -1;
+  *err = cudaGetDevice(&dev);
+  if (*err != cudaSuccess) return nullptr;
+  const bool cached = dev >= 0 && dev < kMaxDevices;
+  void* p = cached ? g_scratch_addr[dev].load(std::memory_order_acquire) : nullptr;
+  if (p) return p;
   *err = cudaGetSymbolAddress(&p, g_pct_scratch);  // the current device's copy
-  return *err == cudaSuccess ? p : nullptr;
+  if (*err != cudaSuccess) return nullptr;
+  if (cached) g_scratch_addr[dev].store(p, std::memory_order_release);
+  return p;
 }
 
 // workspace: the histograms and control block, then 256 bytes for the

@@ -51,6 +51,9 @@ cudaError_t launch_percentile_abs(const void* src, bool f16, int64_t n, const do
                                   float* out, float* thr, float alpha, void* workspace,
                                   cudaStream_t st);
 
+// diagnostics: base-2 exponentials on the special-function unit
+cudaError_t launch_probe_ex2(int iters, float* sink, int64_t* n_ex2, cudaStream_t st);
+
 // streaming multiprocessors of the current device
 int sm_count();
 

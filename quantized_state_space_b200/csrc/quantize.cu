@@ -216,7 +216,7 @@ __global__ void __launch_bounds__(stream::kThreads)
     quant_static_kernel(const void* __restrict__ src, Idx n, Idx mid, const Geo<Idx> geo,
                         const int32_t* __restrict__ gmap, int32_t n_groups,
                         const float* __restrict__ scales, int8_t* __restrict__ q,
-                        uint32_t* status) {
+                        uint32_t* status, uint32_t wait_limit) {
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ float2 tab[kMaxTab];
   __shared__ int ug_s[kPath == kPathCol ? kMaxU : 1];
@@ -233,7 +233,7 @@ __global__ void __launch_bounds__(stream::kThreads)
         const bool okg = (unsigned)g < (unsigned)n_groups;
         q[e] = (int8_t)quant_elem(v, okg ? __ldg(scales + g) : 0.0f, 0.0f, okg, flags);
       },
-      flags);
+      flags, wait_limit);
   flag_status(status, flags);
 }
 
@@ -394,7 +394,7 @@ cudaError_t quantize_t(const void* src, Idx n, Idx mid, Idx inner, const int32_t
   }
   if (n > 0)
     e = launch_stream(quant_static_kernel<kF16, kPath, Idx>, (uint64_t)n, pipe, st, src, n, mid,
-                      geo, gmap, n_groups, (const float*)scales, q, status);
+                      geo, gmap, n_groups, (const float*)scales, q, status, stream::wait_limit());
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

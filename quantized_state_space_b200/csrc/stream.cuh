@@ -13,6 +13,8 @@
 // the CTA that would own it.
 #pragma once
 
+#include <stdlib.h>
+
 #include "common.cuh"
 #include "tc.cuh"
 
@@ -131,7 +133,7 @@ __device__ __forceinline__ float global1(const void* src, Idx e) {
 template <bool kF16, typename Idx, class Vec, class One>
 __device__ __forceinline__ void run_part(const void* __restrict__ src, Idx n, uint8_t* smem,
                                          const Idx c, const Idx G, Vec&& vec, One&& one,
-                                         uint32_t& flags) {
+                                         uint32_t& flags, uint32_t limit = kWaitLimit) {
   constexpr int kEsz = kF16 ? 2 : 4;
   using C = Cfg<kEsz>;
   constexpr int S = C::kStages;
@@ -160,7 +162,7 @@ __device__ __forceinline__ void run_part(const void* __restrict__ src, Idx n, ui
         if (j >= (Idx)S) {
           const uint32_t par = (uint32_t)((j / S - 1) & 1);
           bool ok = false;
-          for (uint32_t i = 0; i < kWaitLimit && !ok; ++i) {
+          for (uint32_t i = 0; i < limit && !ok; ++i) {
             ok = tc::mbar_try(empty + s, par);
             if (!ok && *abort_flag) break;
           }
@@ -186,7 +188,7 @@ __device__ __forceinline__ void run_part(const void* __restrict__ src, Idx n, ui
       const int s = (int)(j % S);
       const uint32_t par = (uint32_t)((j / S) & 1);
       bool ok = false;
-      for (uint32_t i = 0; i < kWaitLimit && !ok; ++i) {
+      for (uint32_t i = 0; i < limit && !ok; ++i) {
         ok = tc::mbar_try(full + s, par);
         if (!ok && *abort_flag) break;
       }
@@ -229,8 +231,22 @@ __device__ __forceinline__ void run_part(const void* __restrict__ src, Idx n, ui
 // The whole grid on src[0, n).
 template <bool kF16, typename Idx, class Vec, class One>
 __device__ __forceinline__ void run(const void* __restrict__ src, Idx n, uint8_t* smem, Vec&& vec,
-                                    One&& one, uint32_t& flags) {
-  run_part<kF16, Idx>(src, n, smem, (Idx)blockIdx.x, (Idx)gridDim.x, vec, one, flags);
+                                    One&& one, uint32_t& flags, uint32_t limit = kWaitLimit) {
+  run_part<kF16, Idx>(src, n, smem, (Idx)blockIdx.x, (Idx)gridDim.x, vec, one, flags, limit);
+}
+
+// Probes before a pipeline wait (a consumer waiting for a tile, the producer
+// for a free stage) gives up: kWaitLimit, unless the environment variable
+// SSMQ_WAIT_LIMIT asks for fewer -- the tests of the timeout path set 0, so
+// that every such wait gives up at once, SSMQ_DEV_TIMEOUT is raised and the
+// CTAs return.  The drain of copies already in flight always keeps the full
+// limit, so no copy lands after its CTA has exited.
+inline uint32_t wait_limit() {
+  const char* v = getenv("SSMQ_WAIT_LIMIT");
+  if (!v || !*v) return kWaitLimit;
+  char* end = nullptr;
+  const unsigned long x = strtoul(v, &end, 10);
+  return (end && *end == '\0' && x < kWaitLimit) ? (uint32_t)x : kWaitLimit;
 }
 
 template <int kEsz>

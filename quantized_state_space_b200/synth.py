@@ -97,7 +97,7 @@ def m1_inputs(batch, seqlen, dim, dstate, ngroups=1, *, gate=True, seed=0, index
     else:
         A = a_log_uniform(rng, (d, N))
     D = _normal(rng, (d,))
-    outlier_channels = None
+    outlier_channels = spike_positions = None
     if outlier_frac > 0:
         n_out = int(round(outlier_frac * d))
         outlier_channels = np.sort(rng.choice(d, size=n_out, replace=False))
@@ -108,11 +108,12 @@ def m1_inputs(batch, seqlen, dim, dstate, ngroups=1, *, gate=True, seed=0, index
         fac = rng.uniform(spike_range[0], spike_range[1], size=n_sp).astype(np.float32)
         flat = x.reshape(-1)
         flat[pos] *= fac
+        spike_positions = np.sort(pos)
     dt_bias = _normal(rng, (d,), std=0.1) if with_bias else None
     h0 = _normal(rng, (b, d, N), std=0.1) if with_h0 else None
     return dict(x=_f16(x), dt=_f16(dt), z=None if z is None else _f16(z), B=_f16(B),
                 C=_f16(Cm), A=A, D=D, dt_bias=dt_bias, h0=h0,
-                outlier_channels=outlier_channels)
+                outlier_channels=outlier_channels, spike_positions=spike_positions)
 
 
 def ssd_inputs(batch, seqlen, nheads, headdim, dstate, ngroups=1, *, gate=False, seed=0,

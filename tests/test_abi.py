@@ -252,6 +252,15 @@ def test_version(L):
     assert N.ssmq_version() >= 100
 
 
+def test_probe_validation(L):
+    n = C.c_int64(-1)
+    assert L.ssmq_probe_ex2(0, FAKE, C.byref(n), None) == N.ERR_INVALID_ARG
+    assert L.ssmq_probe_ex2(16, None, C.byref(n), None) == N.ERR_INVALID_ARG
+    assert L.ssmq_probe_ex2(16, FAKE, None, None) == N.ERR_INVALID_ARG
+    assert L.ssmq_probe_ex2(16, FAKE + 4, C.byref(n), None) == N.ERR_ALIGNMENT
+    assert n.value == -1  # nothing written on a rejected call
+
+
 def test_m1_decode_validation(L):
     f = dict(batch=4, dim=32, dstate=16, ngroups=1, state_group_size=4, x_format=N.X_INT8_GROUP,
              x=FAKE, x_group=FAKE, x_scale=FAKE, n_x_groups=2, dt=FAKE, A=FAKE, B=FAKE, C=FAKE,

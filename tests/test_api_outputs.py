@@ -1,6 +1,6 @@
-"""The Python front end checks every tensor that a call writes (or reads
-whole) and that the caller supplies -- device, contiguity, dtype, element
-count -- since the C library sees only pointers.  Run on the CPU: the native
+"""The Python front end checks every tensor that the caller supplies to a
+call, read or written -- device, contiguity, dtype, element count -- since
+the C library sees only pointers.  Run on the CPU: the native
 calls are replaced by a recorder and the CUDA-device requirement is lifted,
 so only the front end's own checks decide."""
 import pytest
@@ -120,3 +120,92 @@ def test_calibration_outputs(rec):
     _bad(lambda: api.percentile_abs(src, 5.0, workspace=E(1024, dtype=torch.uint8)))
     api.softedge_calibrate(src, E(3))
     _bad(lambda: api.softedge_calibrate(src, E(3, dtype=torch.float64)))
+
+
+def test_scan_inputs(rec):
+    """Every tensor a call reads is checked too: a short or mistyped input,
+    or one on another device, would be read past its end or across devices."""
+    b, d, L, G, N = 2, 8, 5, 1, 16
+    good = dict(x=E(b, d, L, dtype=torch.int8), dt=E(b, d, L, dtype=torch.float16), A=E(d, N),
+                B=E(b, G, N, L, dtype=torch.int8), C=E(b, G, N, L, dtype=torch.int8),
+                B_scale=E(4), C_scale=E(4))
+    kw = dict(x_group=E(d, dtype=torch.int32), x_scale=E(2), z=E(b, d, L, dtype=torch.float16),
+              h0=E(b, d, N), D=E(d), dt_bias=E(d))
+
+    def call(**over):
+        a = dict(good, **{k: v for k, v in over.items() if k in good})
+        k2 = dict(kw, **{k: v for k, v in over.items() if k not in good})
+        return api.selective_scan(a["x"], a["dt"], a["A"], a["B"], a["C"], a["B_scale"],
+                                  a["C_scale"], 4, **k2)
+
+    call()
+    for bad in (dict(h0=E(b, d, N - 1)), dict(h0=E(b, d, N, dtype=torch.float16)),
+                dict(dt=E(b, d, L - 1, dtype=torch.float16)), dict(dt=E(b, d, L)),
+                dict(z=E(b, d, L - 1, dtype=torch.float16)),
+                dict(C=E(b, G, N, L - 1, dtype=torch.int8)), dict(B=E(b, G, N, L, dtype=torch.uint8)),
+                dict(C_scale=E(3)), dict(B_scale=E(4, dtype=torch.float64)),
+                dict(A=E(d, N - 1)), dict(D=E(d + 1)), dict(dt_bias=E(d - 1)),
+                dict(x_group=E(d - 1, dtype=torch.int32)), dict(x_group=E(d, dtype=torch.int64)),
+                dict(x=E(b, d, L, dtype=torch.float32)),
+                dict(h0=E(b, d, N, device="meta")), dict(A=E(d, N, device="meta"))):
+        _bad(call, **bad)
+    assert rec.calls.count("ssmq_selective_scan_w8") == 1
+
+
+def test_ssd_and_decode_inputs(rec):
+    b, L, H, P, G, N = 1, 300, 2, 64, 1, 128
+    x, dt = E(b, L, H, P, dtype=torch.int8), E(b, L, H, dtype=torch.float16)
+    Bq = E(b, L, G, N, dtype=torch.int8)
+    kw = dict(x_group=E(H * P, dtype=torch.int32), x_scale=E(2))
+    api.ssd_chunk_scan(x, dt, E(H), Bq, Bq, E(16), E(16), 8, h0=E(b, H, P, N), **kw)
+    _bad(lambda: api.ssd_chunk_scan(x, dt, E(H), Bq, Bq, E(16), E(16), 8, h0=E(b, H, P, N - 1),
+                                    **kw))
+    _bad(lambda: api.ssd_chunk_scan(x, E(b, L - 1, H, dtype=torch.float16), E(H), Bq, Bq, E(16),
+                                    E(16), 8, **kw))
+    _bad(lambda: api.ssd_chunk_scan(x, dt, E(H), Bq, E(b, L, G, N - 1, dtype=torch.int8), E(16),
+                                    E(16), 8, **kw))
+    _bad(lambda: api.ssd_chunk_scan(x, dt, E(H), Bq, Bq, E(16), E(15), 8, **kw))
+    _bad(lambda: api.ssd_chunk_scan(x, dt, E(H), Bq, Bq, E(16), E(16), 8,
+                                    z=E(b, L, H, P - 1, dtype=torch.float16), **kw))
+    _bad(lambda: api.ssd_chunk_scan(x, dt, E(H, device="meta"), Bq, Bq, E(16), E(16), 8, **kw))
+    _bad(lambda: api.ssd_chunk_scan(x.to(torch.float16), dt, E(H), Bq, Bq, E(16), E(16), 8, **kw))
+    st = E(2, H, P, N)
+    dargs = lambda xx, dtt, BB: (st, xx, dtt, E(H), BB, BB, E(16), E(16), 8)
+    good = (E(2, H, P, dtype=torch.int8), E(2, H, dtype=torch.float16),
+            E(2, G, N, dtype=torch.int8))
+    api.state_update(*dargs(*good), **kw)
+    _bad(lambda: api.state_update(*dargs(E(2, H, P - 1, dtype=torch.int8), *good[1:]), **kw))
+    _bad(lambda: api.state_update(*dargs(good[0], E(2, H + 1, dtype=torch.float16), good[2]),
+                                  **kw))
+    _bad(lambda: api.state_update(*dargs(*good[:2], E(2, G, N - 8, dtype=torch.int8)), **kw))
+
+
+def test_quantizer_and_calibration_inputs(rec):
+    src, g, s = E(2, 3, 8, dtype=torch.float16), E(3, dtype=torch.int32), E(2)
+    _bad(lambda: api.quantize_groups(src, 2, 3, 8, E(2, dtype=torch.int32), 2, scales=s))
+    _bad(lambda: api.quantize_groups(src, 2, 3, 8, g, 2, scales=E(1)))
+    _bad(lambda: api.quantize_groups(src, 2, 3, 9, g, 2, scales=s))
+    _bad(lambda: api.quantize_groups(E(48, dtype=torch.int8), 2, 3, 8, g, 2, scales=s))
+    _bad(lambda: api.quantize_groups_batch([(src, 2, 3, 8, g, 2, E(2, device="meta"), None)]))
+    _bad(lambda: api.softedge_encode(E(8, dtype=torch.float64), 1.0, 0.1, 5.0))
+    _bad(lambda: api.softedge_decode(E(8, dtype=torch.int8), 1.0))
+    _bad(lambda: api.group_absmax(src, 1, 6, 8, g, 3))
+    _bad(lambda: api.cluster_by_absmax(E(4, dtype=torch.float16), 2))
+    _bad(lambda: api.percentile_abs(E(4, dtype=torch.int8), [5.0]))
+
+
+def test_noalloc_wrappers(rec):
+    """The allocation-free calls check their tensors like the others and
+    allocate nothing themselves (the recorder sees exactly one native call)."""
+    src = E(100, dtype=torch.float16)
+    out = E(2)
+    assert api.percentile_abs_noalloc(src, [5.0, 99.9], out) is out
+    _bad(lambda: api.percentile_abs_noalloc(src, [5.0, 99.9], E(3)))
+    _bad(lambda: api.percentile_abs_noalloc(src, [5.0], E(1, dtype=torch.float16)))
+    _bad(lambda: api.percentile_abs_noalloc(src, [5.0], E(1, device="meta")))
+    _bad(lambda: api.percentile_abs_noalloc(E(100, dtype=torch.int32), [5.0], E(1)))
+    thr = E(3)
+    assert api.softedge_calibrate_noalloc(src, thr, alpha=0.1) is thr
+    _bad(lambda: api.softedge_calibrate_noalloc(src, E(2)))
+    _bad(lambda: api.softedge_calibrate_noalloc(src, E(3, device="meta")))
+    assert rec.calls == ["ssmq_percentile_abs_noalloc", "ssmq_softedge_calibrate_noalloc"]

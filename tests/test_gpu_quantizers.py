@@ -108,6 +108,32 @@ def test_quantize_status_bits():
     assert int(H(st)[0]) & N.DEV_BAD_SCALE and not H(q).any()
 
 
+def test_pipeline_wait_gives_up(orc, monkeypatch):
+    """Failure detection on the GPU without a fault: with SSMQ_WAIT_LIMIT=0
+    every wait of the quantizer's bulk-copy pipeline gives up at once.  The
+    kernel must still return (after draining the copies it issued), the call
+    reports SSMQ_DEV_TIMEOUT in the status word, and the context stays usable:
+    the next call, with the normal limit, gives the oracle's codes."""
+    rng = np.random.default_rng(11)
+    b, d, L = 4, 96, 4096  # many tiles per CTA
+    x = rng.standard_normal((b, d, L)).astype(np.float16)
+    grp = rng.integers(0, 4, size=d).astype(np.int32)
+    sc = synth.random_scales(rng, 4, 0.01, 0.05)
+    xt, gt, st_ = T(x), T(grp), T(sc)
+    st = status_word()
+    monkeypatch.setenv("SSMQ_WAIT_LIMIT", "0")
+    api.quantize_groups(xt, b, d, L, gt, 4, scales=st_, status=st)
+    torch.cuda.synchronize()
+    assert int(H(st)[0]) & N.DEV_TIMEOUT
+    monkeypatch.delenv("SSMQ_WAIT_LIMIT")
+    st.zero_()
+    q, _ = api.quantize_groups(xt, b, d, L, gt, 4, scales=st_, status=st)
+    torch.cuda.synchronize()
+    assert int(H(st)[0]) == 0
+    qo, _, _ = orc.quantize_groups(x, b, d, L, grp, 4, orc.SCALE_STATIC, sc)
+    np.testing.assert_array_equal(H(q), qo)
+
+
 def test_quantize_m130m_x_full_size(orc):
     """Full-size Mamba-130M-shaped x with its sort-and-cluster scales."""
     _, raw = synth.workload_inputs("m130m")

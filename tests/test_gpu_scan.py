@@ -7,7 +7,7 @@ import numpy as np
 import pytest
 import torch
 
-from gpu_util import H, T, assert_scan_close, dev, status_word
+from gpu_util import Y_TOL, H, T, assert_scan_close, dev, status_word, y_err
 from problems import m1_problem, oracle_kwargs
 from quantized_state_space_b200 import _native as N
 from quantized_state_space_b200 import api, calibrate, synth
@@ -201,7 +201,23 @@ def _m1_end_to_end(orc, name, n_units=96):
     yg = H(y).reshape(b * d, L)[units].astype(np.float64)
     hg = H(hf).reshape(b * d, Nst)[units]
     # the tolerance is relative to max |y_ref| over the sampled channels
-    return assert_scan_close(yg, yo, hg, ho)
+    e = assert_scan_close(yg, yo, hg, ho)
+    # A few huge values set that max: the m130m outlier channels (x50 at
+    # every step) and the softedge spikes (x100..1000 at single elements).
+    # The same bound must also hold for the ordinary channels / positions
+    # against their own max |y_ref|, or an error of several percent of a
+    # typical |y| could pass.
+    keep = np.ones(yo.shape, dtype=bool)
+    if raw.get("outlier_channels") is not None:
+        keep &= ~np.isin(units % d, raw["outlier_channels"])[:, None]
+    if raw.get("spike_positions") is not None:
+        flat = units[:, None] * L + np.arange(L)[None, :]  # (b, d, L) element index
+        keep &= ~np.isin(flat, raw["spike_positions"])
+    if not keep.all():
+        assert keep.any()
+        e2 = y_err(yg[keep], yo[keep])
+        assert e2 <= Y_TOL, "ordinary channels / positions: y error %.3g > %.1g" % (e2, Y_TOL)
+    return e
 
 
 def test_tiny_workload_end_to_end(orc):
