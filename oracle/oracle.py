@@ -91,6 +91,12 @@ def lib():
         L.orc_cluster_by_absmax.argtypes = [_vp, _i64, _i32, _vp, _vp]
         L.orc_percentile_abs.restype = C.c_double
         L.orc_percentile_abs.argtypes = [_vp, _i32, _i64, C.c_double]
+        L.orc_exp_f32_n.restype = None
+        L.orc_exp_f32_n.argtypes = [_vp, _i64, _vp]
+        L.orc_silu_f32_n.restype = None
+        L.orc_silu_f32_n.argtypes = [_vp, _i64, _vp]
+        L.orc_conv_silu.restype = _i64
+        L.orc_conv_silu.argtypes = [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _i32, _vp, _vp]
         L.orc_softedge_thresholds.restype = None
         L.orc_softedge_thresholds.argtypes = [_vp, _i32, _i64, C.c_double, C.c_double,
                                               C.c_double, _vp]
@@ -384,3 +390,40 @@ def softedge_thresholds(src, q_lo, q_hi, alpha, previous=(0.0, 0.0, 0.0)):
     thr = np.asarray(previous, dtype=np.float32).copy()
     lib().orc_softedge_thresholds(_p(s), is16, s.size, q_lo, q_hi, alpha, _p(thr))
     return thr
+
+
+# ---- causal depthwise convolution + SiLU (the producer of the scan input) --
+
+def exp_f32(v):
+    """The oracle's binary32 e^v (Cody-Waite reduction + Taylor polynomial)."""
+    v = np.ascontiguousarray(v, dtype=np.float32)
+    out = np.empty_like(v)
+    lib().orc_exp_f32_n(_p(v), v.size, _p(out))
+    return out
+
+
+def silu_f32(a):
+    """The oracle's binary32 silu(a) = a * fl32(1 / fl32(1 + e^-a))."""
+    a = np.ascontiguousarray(a, dtype=np.float32)
+    out = np.empty_like(a)
+    lib().orc_silu_f32_n(_p(a), a.size, _p(out))
+    return out
+
+
+def conv_silu(x, weight, bias=None, x_prev=None):
+    """u = silu(causal depthwise conv(x)) in binary32 for x (b, d, L)
+    float16, weight (d, W) float32, bias (d,) or None, x_prev (b, d, W-1)
+    float16 or None.  Returns (u float32 (b, d, L), the next call's conv
+    state float16 (b, d, W-1), number of non-finite u)."""
+    x = np.ascontiguousarray(x, dtype=np.float16)
+    b, d, L = x.shape
+    w = np.ascontiguousarray(weight, dtype=np.float32)
+    W = w.shape[1]
+    bias = _c(bias, np.float32)
+    x_prev = _c(x_prev, np.float16)
+    u = np.empty((b, d, L), np.float32)
+    st = np.empty((b, d, W - 1), np.float16)
+    r = lib().orc_conv_silu(_p(x), _p(x_prev), _p(w), _p(bias), b, d, L, W, _p(u), _p(st))
+    if r < 0:
+        raise ValueError("orc_conv_silu: invalid arguments")
+    return u, st, int(r)

@@ -735,3 +735,121 @@ void orc_softedge_thresholds(const void* src, int32_t src_is_f16, int64_t n, dou
   thr[2] = hi;
   thr[0] = (float)((double)hi / 63.0);
 }
+
+/* ------------------------------------------------------------------------ */
+/* causal depthwise convolution + SiLU: the producer of the scan input       */
+/* ------------------------------------------------------------------------ */
+/* In the Mamba-1 block the scan input x is the output of a short causal
+ * depthwise convolution along time followed by SiLU; [SE] 4.1 puts the range
+ * check (the quantizer or the soft-edge encoder) where that activation is
+ * produced.  The quantizer's code is decided in binary32 (the quantizer's
+ * own rule), so the value it is given is defined as a binary32 evaluation,
+ * step by step, with IEEE operations only (fused multiply-add, add, multiply,
+ * correctly rounded reciprocal) -- reproducible to the bit by any IEEE
+ * implementation.  The tests pin every step against double-precision
+ * mathematics. */
+
+/* 2^k as an exact binary32 number, -126 <= k <= 127. */
+static float orc_pow2f(int k) {
+  union {
+    uint32_t u;
+    float f;
+  } b;
+  b.u = (uint32_t)(k + 127) << 23;
+  return b.f;
+}
+
+/* e^v in binary32 by Cody and Waite's argument reduction (published method):
+ *   k = round-half-even(fl32(v * log2 e))
+ *   r = (v - k LN2_HI) - k LN2_LO, two fused multiply-adds, with
+ *       LN2_HI = 0.693145751953125 (16 significant bits: k LN2_HI is exact)
+ *       and LN2_LO = fl32(ln 2 - LN2_HI), so |r| <= ln2 / 2 + tiny
+ *   p = sum_{n<=7} r^n / n!  (Taylor series, Horner form, fused multiply-adds,
+ *       coefficients fl32(1 / n!); the truncation is below 5e-9 relative)
+ *   e^v = p * 2^k  (one rounding; subnormal results rounded as IEEE does)
+ * Range of this definition: v > 88 gives +inf, v < -87 gives 0, NaN stays
+ * NaN. */
+float orc_exp_f32(float v) {
+  if (v != v) return v;
+  if (v > 88.0f) return INFINITY;
+  if (v < -87.0f) return 0.0f;
+  const float log2e = 1.44269504088896340736f;
+  const float ln2_hi = 0.693145751953125f;
+  const float ln2_lo = (float)(0.69314718055994530942 - 0.693145751953125);
+  const float kf = nearbyintf(v * log2e);
+  float r = fmaf(-kf, ln2_hi, v);
+  r = fmaf(-kf, ln2_lo, r);
+  float p = (float)(1.0 / 5040.0);
+  p = fmaf(p, r, (float)(1.0 / 720.0));
+  p = fmaf(p, r, (float)(1.0 / 120.0));
+  p = fmaf(p, r, (float)(1.0 / 24.0));
+  p = fmaf(p, r, (float)(1.0 / 6.0));
+  p = fmaf(p, r, 0.5f);
+  p = fmaf(p, r, 1.0f);
+  p = fmaf(p, r, 1.0f);
+  return p * orc_pow2f((int)kf);
+}
+
+/* silu(a) = a sigmoid(a) = a / (1 + e^-a), in binary32:
+ *   e = orc_exp_f32(-a); den = fl32(1 + e); r = fl32(1 / den); u = fl32(a r). */
+float orc_silu_f32(float a) {
+  const float e = orc_exp_f32(-a);
+  const float den = 1.0f + e;
+  const float r = 1.0f / den;
+  return a * r;
+}
+
+void orc_exp_f32_n(const float* v, int64_t n, float* out) {
+  for (int64_t i = 0; i < n; ++i) out[i] = orc_exp_f32(v[i]);
+}
+
+void orc_silu_f32_n(const float* a, int64_t n, float* out) {
+  for (int64_t i = 0; i < n; ++i) out[i] = orc_silu_f32(a[i]);
+}
+
+/* The scan input of channel c at step t, for x (b, d, L) binary16:
+ *   a = fl32 chain: a = bias_c (0 without bias); for tap k = 0 .. W-1:
+ *       a = fma(w[c][k], x[t - (W - 1) + k], a)   (oldest tap first)
+ *   u = orc_silu_f32(a)
+ * Steps before t = 0 read the conv state x_prev (b, d, W-1: the W-1 inputs
+ * before the call, oldest first), or zero without one.  x_prev_out (if not
+ * NULL) receives the W-1 most recent inputs, the state of the next call.
+ * Returns the number of non-finite u, or -1 on invalid arguments. */
+int64_t orc_conv_silu(const uint16_t* x, const uint16_t* x_prev, const float* weight,
+                      const float* bias, int64_t batch, int64_t dim, int64_t seqlen,
+                      int32_t width, float* u, uint16_t* x_prev_out) {
+  if (batch < 0 || dim < 0 || seqlen < 0 || width < 1 || width > 4) return -1;
+  const int64_t W = width, S = width - 1;
+  int64_t nonfinite = 0;
+  for (int64_t b = 0; b < batch; ++b)
+    for (int64_t c = 0; c < dim; ++c) {
+      const uint16_t* xr = x + (b * dim + c) * seqlen;
+      const uint16_t* pr = x_prev ? x_prev + (b * dim + c) * S : NULL;
+      for (int64_t t = 0; t < seqlen; ++t) {
+        float a = bias ? bias[c] : 0.0f;
+        for (int64_t k = 0; k < W; ++k) {
+          const int64_t s = t - (W - 1) + k;
+          float xv = 0.0f;
+          if (s >= 0)
+            xv = (float)orc_half_to_double(xr[s]);
+          else if (pr)
+            xv = (float)orc_half_to_double(pr[S + s]);
+          a = fmaf(weight[c * W + k], xv, a);
+        }
+        const float v = orc_silu_f32(a);
+        if (!isfinite(v)) ++nonfinite;
+        u[(b * dim + c) * seqlen + t] = v;
+      }
+      if (x_prev_out)
+        for (int64_t j = 0; j < S; ++j) {
+          const int64_t s = seqlen - S + j; /* time of state slot j */
+          uint16_t h = 0;
+          if (s >= 0)
+            h = xr[s];
+          else if (pr)
+            h = pr[S + s];
+          x_prev_out[(b * dim + c) * S + j] = h;
+        }
+    }
+  return nonfinite;
+}

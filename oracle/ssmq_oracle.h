@@ -172,6 +172,20 @@ double orc_percentile_abs(const void* src, int32_t src_is_f16, int64_t n,
 void orc_softedge_thresholds(const void* src, int32_t src_is_f16, int64_t n, double q_lo,
                              double q_hi, double alpha, float* thr);
 
+
+/* ---- causal depthwise convolution + SiLU (producer of the scan input) ---
+ * binary32 evaluation defined step by step in ssmq_oracle.c; x (b, d, L)
+ * binary16 bits, weight (d, W) fp32, bias fp32[d] or NULL, x_prev (b, d, W-1)
+ * binary16 or NULL (zeros), u (b, d, L) fp32 out, x_prev_out (b, d, W-1) or
+ * NULL.  Returns the number of non-finite u, -1 on invalid arguments. */
+float orc_exp_f32(float v);
+float orc_silu_f32(float a);
+void orc_exp_f32_n(const float* v, int64_t n, float* out);
+void orc_silu_f32_n(const float* a, int64_t n, float* out);
+int64_t orc_conv_silu(const uint16_t* x, const uint16_t* x_prev, const float* weight,
+                      const float* bias, int64_t batch, int64_t dim, int64_t seqlen,
+                      int32_t width, float* u, uint16_t* x_prev_out);
+
 #ifdef __cplusplus
 }
 #endif

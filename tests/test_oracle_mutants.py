@@ -10,7 +10,7 @@ import pytest
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 SRC = os.path.join(ROOT, "oracle", "ssmq_oracle.c")
 PINS = ["tests/test_oracle_quantizers.py", "tests/test_oracle_scans.py",
-        "tests/test_calibration.py"]
+        "tests/test_calibration.py", "tests/test_oracle_conv.py"]
 
 MUTANTS = {
     "m1_drop_Dx": ("if (p->D) acc += (double)p->D[c] * x;\n    if (p->z) acc *= orc_silu(orc_half_to_double(p->z[idx]));\n    if (o->y) o->y[k * L + t] = acc;",
@@ -55,6 +55,17 @@ MUTANTS = {
     "percentile_signed": ("if (isfinite(f)) v[m++] = fabs((double)f);", "if (isfinite(f)) v[m++] = (double)f;"),
     "percentile_position_n": ("const double pos = (double)(m - 1) * (q / 100.0);",
                               "const double pos = (double)m * (q / 100.0);"),
+    "conv_taps_reversed": ("a = fmaf(weight[c * W + k], xv, a);",
+                           "a = fmaf(weight[c * W + (W - 1 - k)], xv, a);"),
+    "conv_bias_dropped": ("float a = bias ? bias[c] : 0.0f;", "float a = 0.0f;"),
+    "conv_state_order": ("xv = (float)orc_half_to_double(pr[S + s]);",
+                         "xv = (float)orc_half_to_double(pr[-s - 1]);"),
+    "conv_state_out_shift": ("const int64_t s = seqlen - S + j; /* time of state slot j */",
+                             "const int64_t s = seqlen - S + j - 1; /* time of state slot j */"),
+    "exp_taylor_coefficient": ("p = fmaf(p, r, (float)(1.0 / 120.0));",
+                               "p = fmaf(p, r, (float)(1.0 / 100.0));"),
+    "exp_ln2_lo_dropped": ("r = fmaf(-kf, ln2_lo, r);", "r = fmaf(-kf, 0.0f, r);"),
+    "silu_f32_sign": ("const float e = orc_exp_f32(-a);", "const float e = orc_exp_f32(a);"),
     "ssd_bias_dropped": ("orc_delta(orc_half_to_double(p->dt[(b * L + t) * H + hd]),\n                                   p->dt_bias ? (double)p->dt_bias[hd] : 0.0, p->dt_softplus);\n    const double dA",
                          "orc_delta(orc_half_to_double(p->dt[(b * L + t) * H + hd]),\n                                   0.0, p->dt_softplus);\n    const double dA"),
 }
