@@ -1056,6 +1056,21 @@ def form_tiny(torch, dev, reps=50):
         return round(statistics.median(ts), 2)
 
     t_step, t_scan = lat(step), lat(scan)
+    # the same step captured once in a CUDA graph and replayed: the device-side
+    # latency without the host's per-launch cost
+    try:
+        g = torch.cuda.CUDAGraph()
+        s_ = torch.cuda.Stream()
+        s_.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s_):
+            step()
+            torch.cuda.synchronize()
+            with torch.cuda.graph(g, stream=s_):
+                step()
+        torch.cuda.current_stream().wait_stream(s_)
+        t_graph = lat(g.replay)
+    except Exception as e:  # report, keep the eager numbers
+        t_graph = "%s: %s" % (type(e).__name__, e)
     ox, oxs, _ = O.quantize_groups(raw["x"], b, d, L, np.zeros(d, np.int32), 1, O.SCALE_ABSMAX)
     gm = np.zeros(G * N, np.int32)
     oB, obs, _ = O.quantize_groups(raw["B"], b, G * N, L, gm, 1, O.SCALE_ABSMAX)
@@ -1072,7 +1087,7 @@ def form_tiny(torch, dev, reps=50):
     par = parity(y.float().cpu().numpy().reshape(b * d, L), yo,
                  hf.cpu().numpy().reshape(b * d, N), ho, "the whole workload")
     return {"workload": "tiny: b 1, L 256, d 64, N 16, per-tensor absmax scales; latency",
-            "step_us": t_step, "scan_us": t_scan,
+            "step_us": t_step, "scan_us": t_scan, "step_graph_replay_us": t_graph,
             "step": "device absmax quantize of x, B, C (3 calls, 12 launches incl. memsets) "
                     "+ scan", "statistic": "median of %d calls, CUDA events per call" % reps,
             "value": round(b * L * d / (t_step / 1e6) / 1e9, 4), "unit": UNIT,
@@ -1080,9 +1095,41 @@ def form_tiny(torch, dev, reps=50):
             "cpu_baseline": base, "parity": par}
 
 
+def form_conv(torch, dev, pk, layer):
+    """Producer-side fusion: causal depthwise conv (W 4) + SiLU + the group
+    quantizer on the m130m-shaped conv input (binary16, 8 x 1536 x 2048, the
+    layer's x standing in for the in_proj output), int8 codes straight out.
+    Algorithmic bytes: 2 in + 1 out per element (weights negligible)."""
+    from quantized_state_space_b200 import api
+    b, d, L = layer.b, layer.d, layer.L
+    rng = np.random.default_rng(12)
+    w = torch.from_numpy(rng.uniform(-0.5, 0.5, size=(d, 4)).astype(np.float32)).to(dev)
+    bs = torch.from_numpy(rng.uniform(-0.2, 0.2, size=d).astype(np.float32)).to(dev)
+    codes = torch.empty((b, d, L), dtype=torch.int8, device=dev)
+
+    def conv():
+        api.conv_silu_quantize(layer.x, w, bias=bs, x_group=layer.grp, x_scale=layer.xs,
+                               codes=codes)
+
+    t = _timed(torch, conv, 20)
+    byts = b * d * L * 3 + d * 4 * 5
+    return {"workload": "m130m conv input (8 x 1536 x 2048 binary16) -> causal conv W 4 + "
+                        "SiLU + int8 group codes (8 clusters), one launch",
+            "ms": round(t * 1e3, 4), "value": round(b * d * L / t / 1e9, 3), "unit": UNIT,
+            "roofline": {"bound": "hbm", "achieved": round(byts / t / 1e9, 1),
+                         "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": round(byts / t / 1e9 / pk["hbm_gbs"], 4),
+                         "algorithmic_bytes_per_launch": byts}}
+
+
 def run_forms(dev, pk, mhz, only=None, layer=None, ex2=None):
     import torch
     out = {}
+    if layer is not None and (not only or "conv" in only):
+        try:
+            out["conv"] = form_conv(torch, dev, pk, layer)
+        except Exception as e:
+            out["conv"] = {"error": "%s: %s" % (type(e).__name__, e)}
     if layer is not None and (not only or "calibrate" in only):
         try:
             out["calibrate"] = form_calibrate(torch, dev, pk, layer)
@@ -1202,8 +1249,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-forms", action="store_true")
-    ap.add_argument("--forms", default="", help="comma list of m130m_other_x_path,m130m_int8_y,calibrate,ssd27b,decode8b,"
-                         "softedge,tiny")
+    ap.add_argument("--forms", default="", help="comma list of m130m_other_x_path,m130m_int8_y,conv,calibrate,ssd27b,"
+                         "decode8b,softedge,tiny")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--fused", action="store_true",
                     help="headline step with binary16 x encoded inside the scan (byte-identical "

@@ -261,6 +261,70 @@ ssmq_status ssmq_softedge_calibrate_noalloc(const void* src, ssmq_dtype dtype, i
                                             float* thresholds, void* stream);
 
 /* ------------------------------------------------------------------------ */
+/* Producer of the scan input: causal conv + SiLU + quantize, fused           */
+/* ------------------------------------------------------------------------ */
+/*
+ * Passage: Quamba-SE write-up 4.1 (the range check is inserted into the
+ * quantization where the activation is produced, inside a custom CUDA
+ * kernel) and Quamba2 abstract / method step 3 (x quantized per
+ * sorted-and-clustered channel group).  In the Mamba-1 block the scan input x
+ * is the output of a short causal depthwise convolution along time followed
+ * by SiLU; this call computes it and writes its 8-bit codes directly (no
+ * binary16 x through HBM).
+ *
+ * The value coded is a binary32 evaluation, step by step (reproducible to the
+ * bit by any IEEE implementation):
+ *   a = bias[c] (0 without bias); a = fma(weight[c][k], x[t - (W-1) + k], a)
+ *       for k = 0 .. W-1 (oldest tap first; steps before 0 read x_prev)
+ *   e = exp32(-a): k = round-half-even(fl32(v * log2 e));
+ *       r = fma(-k, LN2_LO, fma(-k, LN2_HI, v)) with LN2_HI = 0.693145751953125,
+ *       LN2_LO = fl32(ln 2 - LN2_HI); p = sum_{n<=7} r^n / n! in Horner form
+ *       (fused multiply-adds, coefficients fl32(fl64(1 / n!))); e = fl32(p 2^k);
+ *       v > 88 gives +inf, v < -87 gives 0
+ *   u = fl32(a * fl32(1 / fl32(1 + e)))
+ * then u is coded as ssmq_quantize_groups (SCALE_STATIC, binary32 source,
+ * group x_group[c]) or ssmq_softedge_encode would code it.
+ *
+ * Layouts (b, d, L, W):
+ *   x        (b, d, L) binary16: the convolution's input (the in_proj output)
+ *   weight   fp32 (d, W), W in 1..4;  bias fp32[d] or NULL
+ *   x_prev   (b, d, W-1) binary16: the W-1 inputs before step 0, oldest first
+ *            (the conv state of a previous call), or NULL for zeros
+ *   codes    (b, d, L) int8 (out_format INT8_GROUP: x_group int32[d], x_scale
+ *            fp32[n_x_groups]) or uint8 soft-edge codes (SOFTEDGE: se_scale,
+ *            se_lo, se_hi, se_log2_ratio as ssmq_softedge_encode)
+ *   u        (b, d, L) fp32 out (the values coded) or NULL
+ *   x_prev_out (b, d, W-1) binary16 out or NULL: the W-1 most recent inputs,
+ *            the x_prev of the next call (a call on steps [0, L1) followed by
+ *            one on [L1, L) with that state gives the unsplit call's bytes);
+ *            must not overlap x_prev
+ * status: NONFINITE (non-finite u, coded 0), BAD_GROUP, BAD_SCALE as the
+ * quantizer.  Errors: INVALID_ARG (NULL tensors, W outside 1..4, bad
+ * out_format, se_lo > se_hi, overlapping states), ALIGNMENT (x, codes, u not
+ * 16-byte aligned).  Rows of L % 16 == 0 steps take the vectorised kernel.
+ */
+typedef struct {
+  int64_t batch, seqlen, dim;
+  int32_t width;
+  const uint16_t* x;
+  const float* weight;
+  const float* bias;
+  const uint16_t* x_prev;
+  int32_t out_format;       /* SSMQ_X_INT8_GROUP or SSMQ_X_SOFTEDGE */
+  const int32_t* x_group;
+  const float* x_scale;
+  int32_t n_x_groups;
+  float se_scale, se_lo, se_hi;
+  int32_t se_log2_ratio;
+  void* codes;
+  float* u;
+  uint16_t* x_prev_out;
+  uint32_t* status;
+} ssmq_conv_args;
+
+ssmq_status ssmq_conv_silu_quantize(const ssmq_conv_args* args, void* stream);
+
+/* ------------------------------------------------------------------------ */
 /* Mamba-1 diagonal selective scan                                           */
 /* ------------------------------------------------------------------------ */
 /*

@@ -72,6 +72,14 @@ class M1DecodeArgs(C.Structure):
                 ("C_scale", _vp), ("state", _vp), ("y", _vp), ("status", _vp)]
 
 
+class ConvArgs(C.Structure):
+    _fields_ = [("batch", _i64), ("seqlen", _i64), ("dim", _i64), ("width", _i32), ("x", _vp),
+                ("weight", _vp), ("bias", _vp), ("x_prev", _vp), ("out_format", _i32),
+                ("x_group", _vp), ("x_scale", _vp), ("n_x_groups", _i32), ("se_scale", _f32),
+                ("se_lo", _f32), ("se_hi", _f32), ("se_log2_ratio", _i32), ("codes", _vp),
+                ("u", _vp), ("x_prev_out", _vp), ("status", _vp)]
+
+
 # entry point -> (restype, argtypes); every name declared in include/ssmq.h
 class QuantJob(C.Structure):
     _fields_ = [("src", _vp), ("dtype", _i32), ("outer", _i64), ("mid", _i64), ("inner", _i64),
@@ -87,6 +95,7 @@ SIGNATURES = {
     "ssmq_softedge_encode": (_i32, [_vp, _i32, _i64, _f32, _f32, _f32, _i32, _vp, _vp, _vp]),
     "ssmq_softedge_decode": (_i32, [_vp, _i64, _f32, _i32, _vp, _vp]),
     "ssmq_selective_scan_w8": (_i32, [C.POINTER(ScanArgs), _vp]),
+    "ssmq_conv_silu_quantize": (_i32, [C.POINTER(ConvArgs), _vp]),
     "ssmq_ssd_workspace_size": (C.c_size_t, [C.POINTER(SSDArgs)]),
     "ssmq_ssd_chunk_scan_w8": (_i32, [C.POINTER(SSDArgs), _vp, C.c_size_t, _vp]),
     "ssmq_state_update_w8": (_i32, [C.POINTER(DecodeArgs), _vp]),
@@ -219,6 +228,12 @@ def ssmq_selective_scan_w8(stream=None, **fields):
     """Fields of ssmq_scan_args as keywords (tensors for pointer fields)."""
     a = _fill(ScanArgs, fields)
     _check(lib().ssmq_selective_scan_w8(C.byref(a), _stream(stream)))
+
+
+def ssmq_conv_silu_quantize(stream=None, **fields):
+    """Fields of ssmq_conv_args as keywords (tensors for pointer fields)."""
+    a = _fill(ConvArgs, fields)
+    _check(lib().ssmq_conv_silu_quantize(C.byref(a), _stream(stream)))
 
 
 def ssmq_ssd_workspace_size(**fields):

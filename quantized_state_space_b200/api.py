@@ -76,13 +76,14 @@ def _workspace(t, nbytes, device):
                          % (nbytes + 255, device))
 
 
-def _x_in(x, x_group, x_scale, channels, device, codes_only=False):
+def _x_in(x, x_group, x_scale, channels, device, codes_only=False, se_lo=None):
     """x and its cluster map: int8 codes, soft-edge uint8 codes, or (Mamba-1
-    scan only) binary16 activations; the cluster map has one int32 entry per
-    channel and the scale table at least one fp32 entry."""
+    scan only) binary16 activations, soft-edge encoded when thresholds are
+    given; int8 codes and group-quantized binary16 x need the cluster map (one
+    int32 entry per channel) and a scale table of at least one fp32 entry."""
     _in(x, "x", (torch.int8, torch.uint8) if codes_only else
         (torch.int8, torch.uint8, torch.float16), None, device)
-    if x.dtype != torch.uint8:
+    if x.dtype == torch.int8 or (x.dtype == torch.float16 and se_lo is None):
         _in(x_group, "x_group", torch.int32, channels, device)
         _in(x_scale, "x_scale", torch.float32, None, device)
         if x_group is None or x_scale is None or x_scale.numel() < 1:
@@ -226,7 +227,7 @@ def selective_scan(x, dt, A, B, C, B_scale, C_scale, state_group_size, *, x_grou
     G, Nst = B.shape[1], B.shape[2]
     _dev_check(x, dt, A, B, C, B_scale, C_scale, x_group, x_scale, D, z, dt_bias, h0)
     dv = x.device
-    _x_in(x, x_group, x_scale, d, dv)
+    _x_in(x, x_group, x_scale, d, dv, se_lo=se_lo)
     _in(dt, "dt", torch.float16, b * d * L, dv)
     _in(z, "z", torch.float16, b * d * L, dv)
     _in(A, "A", torch.float32, d * Nst, dv)
@@ -248,6 +249,60 @@ def selective_scan(x, dt, A, B, C, B_scale, C_scale, state_group_size, *, x_grou
                                  D=D, z=z, B=B, C=C, B_scale=B_scale, C_scale=C_scale, h0=h0,
                                  y=y, h_final=h_final, status=status, **yf)
     return (y, h_final, y_q) if yf else (y, h_final)
+
+
+def conv_silu_quantize(x, weight, *, bias=None, x_prev=None, x_group=None, x_scale=None,
+                       se_scale=None, se_lo=None, se_hi=None, se_log2_ratio=2, codes=None,
+                       want_u=False, u=None, x_prev_out=None, want_state=False, status=None):
+    """The scan input's codes straight from the convolution's input: causal
+    depthwise conv (weight (d, W), W <= 4; bias (d,); conv state x_prev
+    (b, d, W-1)) + SiLU + the group quantizer (x_group / x_scale: int8
+    codes) or the soft-edge encoder (se_scale / se_lo / se_hi: uint8 codes).
+    x (b, d, L) float16.  Returns codes, plus u (float32 values coded) when
+    want_u, plus the next call's state (b, d, W-1) float16 when want_state."""
+    _dev_check(x, weight, bias, x_prev, x_group, x_scale)
+    b, d, L = x.shape
+    dv = x.device
+    W = weight.shape[-1] if weight.dim() == 2 else 0
+    _in(x, "x", torch.float16, b * d * L, dv)
+    _in(weight, "weight", torch.float32, d * W, dv)
+    _in(bias, "bias", torch.float32, d, dv)
+    _in(x_prev, "x_prev", torch.float16, b * d * max(W - 1, 0), dv)
+    soft = se_scale is not None
+    if soft:
+        cdt = torch.uint8
+        fmt = dict(out_format=N.X_SOFTEDGE, se_scale=float(se_scale), se_lo=float(se_lo),
+                   se_hi=float(se_hi), se_log2_ratio=se_log2_ratio)
+    else:
+        _in(x_group, "x_group", torch.int32, d, dv)
+        _in(x_scale, "x_scale", torch.float32, None, dv)
+        if x_group is None or x_scale is None or x_scale.numel() < 1:
+            raise ValueError("x_group and a non-empty x_scale, or the soft-edge parameters, "
+                             "are required")
+        cdt = torch.int8
+        fmt = dict(out_format=N.X_INT8_GROUP, x_group=x_group, x_scale=x_scale,
+                   n_x_groups=int(x_scale.numel()))
+    _out(codes, "codes", cdt, b * d * L, dv)
+    _out(u, "u", torch.float32, b * d * L, dv)
+    _out(x_prev_out, "x_prev_out", torch.float16, b * d * max(W - 1, 0), dv)
+    _status(status, dv)
+    with _on(dv):
+        if codes is None:
+            codes = torch.empty((b, d, L), dtype=cdt, device=dv)
+        if want_u and u is None:
+            u = torch.empty((b, d, L), dtype=torch.float32, device=dv)
+        if want_state and x_prev_out is None:
+            x_prev_out = torch.empty((b, d, max(W - 1, 0)), dtype=torch.float16, device=dv)
+        N.ssmq_conv_silu_quantize(batch=b, seqlen=L, dim=d, width=W, x=x, weight=weight,
+                                  bias=bias, x_prev=x_prev, codes=codes,
+                                  u=u if want_u or u is not None else None,
+                                  x_prev_out=x_prev_out, status=status, **fmt)
+    out = (codes,)
+    if want_u:
+        out += (u,)
+    if want_state:
+        out += (x_prev_out,)
+    return out if len(out) > 1 else codes
 
 
 def _ssd_inputs(x, dt, A, B, C, B_scale, C_scale, state_group_size, x_group, x_scale, D, z,

@@ -337,6 +337,41 @@ ssmq_status ssmq_softedge_decode(const uint8_t* codes, int64_t n, float scale, i
                 fn);
 }
 
+ssmq_status ssmq_conv_silu_quantize(const ssmq_conv_args* a, void* stream) {
+  const char* fn = "ssmq_conv_silu_quantize";
+  Range nvtx_range(fn);
+  REQUIRE(a != nullptr, SSMQ_ERR_INVALID_ARG, "%s: args is NULL", fn);
+  REQUIRE(a->batch >= 0 && a->seqlen >= 0 && a->dim >= 0, SSMQ_ERR_INVALID_ARG,
+          "%s: negative size", fn);
+  REQUIRE(a->width >= 1 && a->width <= 4, SSMQ_ERR_INVALID_ARG, "%s: width %d not in 1..4", fn,
+          (int)a->width);
+  REQUIRE(a->out_format == SSMQ_X_INT8_GROUP || a->out_format == SSMQ_X_SOFTEDGE,
+          SSMQ_ERR_INVALID_ARG, "%s: out_format must be INT8_GROUP or SOFTEDGE", fn);
+  if (a->out_format == SSMQ_X_INT8_GROUP) {
+    REQUIRE(a->x_group && a->x_scale && a->n_x_groups >= 1, SSMQ_ERR_INVALID_ARG,
+            "%s: x_group, x_scale and n_x_groups >= 1 required", fn);
+  } else {
+    REQUIRE(a->se_lo <= a->se_hi, SSMQ_ERR_INVALID_ARG, "%s: se_lo > se_hi", fn);
+    REQUIRE(a->se_log2_ratio >= 0 && a->se_log2_ratio <= 8, SSMQ_ERR_INVALID_ARG,
+            "%s: se_log2_ratio must be in [0, 8]", fn);
+  }
+  const int64_t n = a->batch * a->dim * a->seqlen;
+  const int64_t ns = a->batch * a->dim * (a->width - 1);
+  if (n > 0) REQUIRE(a->x && a->weight && a->codes, SSMQ_ERR_INVALID_ARG, "%s: NULL tensor", fn);
+  if (a->x_prev_out && a->x_prev && ns > 0) {
+    const uintptr_t p0 = (uintptr_t)a->x_prev, p1 = (uintptr_t)a->x_prev_out;
+    const uintptr_t nb = (uintptr_t)ns * sizeof(uint16_t);
+    REQUIRE(p0 + nb <= p1 || p1 + nb <= p0, SSMQ_ERR_INVALID_ARG,
+            "%s: x_prev_out overlaps x_prev", fn);
+  }
+  if (a->x_prev_out && ns > 0 && a->seqlen > 0)
+    REQUIRE(a->x != nullptr, SSMQ_ERR_INVALID_ARG, "%s: x is NULL", fn);
+  REQUIRE(aligned16(a->x) && aligned16(a->codes) && aligned16(a->u), SSMQ_ERR_ALIGNMENT,
+          "%s: x, codes and u must be 16-byte aligned", fn);
+  if (injected(fn)) return fail(SSMQ_ERR_CUDA, "%s: injected launch failure", fn);
+  return finish(ssmq::launch_conv_silu_quantize(*a, (cudaStream_t)stream), fn);
+}
+
 ssmq_status ssmq_selective_scan_w8(const ssmq_scan_args* a, void* stream) {
   const char* fn = "ssmq_selective_scan_w8";
   Range nvtx_range(fn);

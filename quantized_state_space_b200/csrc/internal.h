@@ -34,6 +34,7 @@ cudaError_t launch_softedge_decode(const uint8_t* codes, int64_t n, float scale,
                                    int log2_ratio, float* out, cudaStream_t st);
 
 cudaError_t launch_selective_scan(const ssmq_scan_args& a, cudaStream_t st);
+cudaError_t launch_conv_silu_quantize(const ssmq_conv_args& a, cudaStream_t st);
 
 cudaError_t launch_state_update(const ssmq_decode_args& a, cudaStream_t st);
 cudaError_t launch_m1_state_update(const ssmq_m1_decode_args& a, cudaStream_t st);

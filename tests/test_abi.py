@@ -40,7 +40,8 @@ def test_exports_every_declared_symbol(L):
 
 
 STRUCTS = ((N.ScanArgs, "ssmq_scan_args"), (N.SSDArgs, "ssmq_ssd_args"),
-           (N.DecodeArgs, "ssmq_decode_args"), (N.M1DecodeArgs, "ssmq_m1_decode_args"))
+           (N.DecodeArgs, "ssmq_decode_args"), (N.M1DecodeArgs, "ssmq_m1_decode_args"),
+           (N.ConvArgs, "ssmq_conv_args"))
 
 
 def test_struct_layout_matches_header(tmp_path):
@@ -301,3 +302,34 @@ def test_calibration_validation(L):
     assert S(5.0, 99.9, 0.0) == N.ERR_INVALID_ARG
     assert S(5.0, 99.9, 1.5) == N.ERR_INVALID_ARG
     assert S(99.9, 5.0, 0.1) == N.ERR_INVALID_ARG
+
+
+def _conv_args(**kw):
+    a = N.ConvArgs(batch=2, seqlen=32, dim=8, width=4, x=FAKE, weight=FAKE, bias=None,
+                   x_prev=None, out_format=N.X_INT8_GROUP, x_group=FAKE, x_scale=FAKE,
+                   n_x_groups=2, se_scale=1.0, se_lo=0.1, se_hi=5.0, se_log2_ratio=2,
+                   codes=FAKE, u=None, x_prev_out=None, status=None)
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a
+
+
+def test_conv_validation(L):
+    S = lambda **kw: L.ssmq_conv_silu_quantize(C.byref(_conv_args(**kw)), None)
+    assert L.ssmq_conv_silu_quantize(None, None) == N.ERR_INVALID_ARG
+    assert S(width=0) == N.ERR_INVALID_ARG
+    assert S(width=5) == N.ERR_INVALID_ARG
+    assert S(seqlen=-1) == N.ERR_INVALID_ARG
+    assert S(out_format=N.X_F16_GROUP) == N.ERR_INVALID_ARG
+    assert S(x_group=None) == N.ERR_INVALID_ARG
+    assert S(n_x_groups=0) == N.ERR_INVALID_ARG
+    assert S(out_format=N.X_SOFTEDGE, se_lo=6.0, se_hi=5.0) == N.ERR_INVALID_ARG
+    assert S(out_format=N.X_SOFTEDGE, se_log2_ratio=9) == N.ERR_INVALID_ARG
+    assert S(x=None) == N.ERR_INVALID_ARG
+    assert S(codes=None) == N.ERR_INVALID_ARG
+    assert S(x=FAKE + 2) == N.ERR_ALIGNMENT
+    assert S(u=FAKE + 8) == N.ERR_ALIGNMENT
+    # the two conv states may not overlap (2 * 8 * 3 binary16 = 96 bytes each)
+    assert S(x_prev=FAKE, x_prev_out=FAKE + 64) == N.ERR_INVALID_ARG
+    assert S(batch=0, x=None, codes=None, x_prev=FAKE, x_prev_out=FAKE + 96,
+             x_group=None) == N.ERR_INVALID_ARG  # group map still required

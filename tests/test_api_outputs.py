@@ -139,6 +139,10 @@ def test_scan_inputs(rec):
                                   a["C_scale"], 4, **k2)
 
     call()
+    # binary16 x soft-edge encoded in the scan: no cluster map needed
+    call(x=E(b, d, L, dtype=torch.float16), x_group=None, x_scale=None, se_scale=1.0,
+         se_lo=0.1, se_hi=5.0)
+    _bad(call, x=E(b, d, L, dtype=torch.float16), x_group=None, x_scale=None)
     for bad in (dict(h0=E(b, d, N - 1)), dict(h0=E(b, d, N, dtype=torch.float16)),
                 dict(dt=E(b, d, L - 1, dtype=torch.float16)), dict(dt=E(b, d, L)),
                 dict(z=E(b, d, L - 1, dtype=torch.float16)),
@@ -149,7 +153,7 @@ def test_scan_inputs(rec):
                 dict(x=E(b, d, L, dtype=torch.float32)),
                 dict(h0=E(b, d, N, device="meta")), dict(A=E(d, N, device="meta"))):
         _bad(call, **bad)
-    assert rec.calls.count("ssmq_selective_scan_w8") == 1
+    assert rec.calls.count("ssmq_selective_scan_w8") == 2
 
 
 def test_ssd_and_decode_inputs(rec):
