@@ -1205,7 +1205,15 @@ def run_kernel(args):
         print(json.dumps(dict(kernel="ex2_rate_kernel (SFU exp2 throughput probe)",
                               **measure_ex2(torch, dev))), flush=True)
         return
-    if name in ("scan", "scan-int8", "quantize"):
+    if name == "conv":
+        lay = Layer(dev, 0)
+        rng = np.random.default_rng(12)
+        w = torch.from_numpy(rng.uniform(-0.5, 0.5, size=(lay.d, 4)).astype(np.float32)).to(dev)
+        bs = torch.from_numpy(rng.uniform(-0.2, 0.2, size=lay.d).astype(np.float32)).to(dev)
+        fn = (lambda: api.conv_silu_quantize(lay.x, w, bias=bs, x_group=lay.grp,
+                                             x_scale=lay.xs, codes=lay.xq))
+        label = "m130m conv input: causal conv + SiLU + int8 group codes"
+    elif name in ("scan", "scan-int8", "quantize"):
         lay = Layer(dev, 0, fused=name == "scan")
         lay.quantize()
         fn = lay.scan if name != "quantize" else (
@@ -1256,7 +1264,7 @@ def main():
                     help="headline step with binary16 x encoded inside the scan (byte-identical "
                          "result; default: x quantized by its own launch, the faster path here)")
     ap.add_argument("--kernel", choices=["scan", "scan-int8", "quantize", "ssd", "encode",
-                                         "softedge-scan", "decode", "ex2"],
+                                         "softedge-scan", "decode", "ex2", "conv"],
                     help="profiling aid: run only this kernel on its workload")
     args = ap.parse_args()
     if args.kernel:

@@ -427,6 +427,54 @@ __global__ void __launch_bounds__(stream::kThreads)
   flag_status(status, flags);
 }
 
+// binary16 input: the code of every one of the 65536 bit patterns is
+// computed once per CTA, exactly as se_encode1 defines it, into a 64 KB
+// shared-memory table (by the consumers, while the producer's first copies
+// are in flight); each element is then one table load.  A non-finite element
+// (exponent bits all ones) is found per 32-bit pair: (w & 0x7C007C00) +
+// 0x04000400 sets bit 15 of a half exactly when that half's exponent field
+// is 0x1F.  Two CTAs per SM (64 KB table + 48 KB of stages each).
+constexpr int kLutBytes = 65536;
+constexpr int kLutCtasPerSm = 2;
+
+template <typename Idx>
+__global__ void __launch_bounds__(stream::kThreads, kLutCtasPerSm)
+    se_encode_lut_kernel(const uint16_t* __restrict__ src, Idx n, float lo, float hi, SeSteps st,
+                         uint8_t* __restrict__ codes, uint32_t* status) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  uint8_t* lut = smem;
+  uint32_t flags = 0;
+  auto build = [&]() {
+    uint32_t dummy = 0;
+    for (int i = threadIdx.x; i < kLutBytes / 4; i += stream::kConsumers) {
+      uint32_t w = 0;
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        w |= se_encode1(h2f((uint16_t)(4 * i + k)), lo, hi, st, dummy) << (8 * k);
+      reinterpret_cast<uint32_t*>(lut)[i] = w;
+    }
+  };
+  uint32_t nf = 0;  // bit 15 / 31 set by a non-finite half
+  auto vec = [&](const uint32_t(&w)[8], Idx e0) {
+    uint32_t o[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const uint32_t a = w[2 * k], b = w[2 * k + 1];
+      nf |= ((a & 0x7C007C00u) + 0x04000400u) | ((b & 0x7C007C00u) + 0x04000400u);
+      const uint32_t c0 = lut[a & 0xFFFFu], c1 = lut[a >> 16];
+      const uint32_t c2 = lut[b & 0xFFFFu], c3 = lut[b >> 16];
+      o[k] = __byte_perm(__byte_perm(c0, c1, 0x0040), __byte_perm(c2, c3, 0x0040), 0x5410);
+    }
+    *reinterpret_cast<uint4*>(codes + e0) = make_uint4(o[0], o[1], o[2], o[3]);
+  };
+  auto one = [&](float v, Idx e) { codes[e] = (uint8_t)se_encode1(v, lo, hi, st, flags); };
+  stream::run_part<true, Idx, decltype(vec)&, decltype(one)&, decltype(build)&, true>(
+      src, n, smem + kLutBytes, (Idx)blockIdx.x, (Idx)gridDim.x, vec, one, flags,
+      stream::kWaitLimit, build);
+  if (nf & 0x80008000u) flags |= SSMQ_DEV_NONFINITE;
+  flag_status(status, flags);
+}
+
 template <typename Idx>
 __global__ void __launch_bounds__(kThreads)
     se_decode_kernel(const uint8_t* __restrict__ codes, Idx n, SeSteps st, float* __restrict__ out) {
@@ -591,19 +639,35 @@ cudaError_t launch_softedge_encode(const void* src, bool f16, int64_t n, float s
                                    cudaStream_t st) {
   if (n == 0) return cudaSuccess;
   const SeSteps steps = se_steps(scale, log2_ratio);
-  const size_t smem = (size_t)acc_smem_offset<true>(), smem32 = (size_t)acc_smem_offset<false>();
+  const size_t smem32 = (size_t)acc_smem_offset<false>();
+  if (f16) {
+    // the table kernel: 64 KB of codes + the pipeline's stages per CTA
+    const size_t smem_lut = kLutBytes + (size_t)acc_smem_offset<true>();
+    const uint64_t tiles = ((uint64_t)n + stream::kTileElems - 1) / stream::kTileElems;
+    uint64_t grid = (uint64_t)sm_count() * kLutCtasPerSm;
+    if (grid > tiles) grid = tiles ? tiles : 1;
+    auto go = [&](auto kern, auto nn) {
+      cudaError_t e =
+          cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_lut);
+      if (e != cudaSuccess) return e;
+      // two 113 KB CTAs per SM need the whole shared-memory carveout
+      e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+      if (e != cudaSuccess) return e;
+      kern<<<(unsigned)grid, stream::kThreads, smem_lut, st>>>(
+          static_cast<const uint16_t*>(src), nn, lo, hi, steps, codes, status);
+      return cudaGetLastError();
+    };
+    if ((uint64_t)n + 64 < (1ull << 32)) return go(se_encode_lut_kernel<uint32_t>, (uint32_t)n);
+    return go(se_encode_lut_kernel<uint64_t>, (uint64_t)n);
+  }
   if ((uint64_t)n + 64 < (1ull << 32)) {
     const uint32_t n32 = (uint32_t)n;
-    return f16 ? launch_stream(se_encode_kernel<true, uint32_t>, (uint64_t)n, smem, st, src, n32,
-                               lo, hi, steps, codes, status)
-               : launch_stream(se_encode_kernel<false, uint32_t>, (uint64_t)n, smem32, st, src,
-                               n32, lo, hi, steps, codes, status);
+    return launch_stream(se_encode_kernel<false, uint32_t>, (uint64_t)n, smem32, st, src, n32, lo,
+                         hi, steps, codes, status);
   }
   const uint64_t n64 = (uint64_t)n;
-  return f16 ? launch_stream(se_encode_kernel<true, uint64_t>, n64, smem, st, src, n64, lo, hi,
-                             steps, codes, status)
-             : launch_stream(se_encode_kernel<false, uint64_t>, n64, smem32, st, src, n64, lo, hi,
-                             steps, codes, status);
+  return launch_stream(se_encode_kernel<false, uint64_t>, n64, smem32, st, src, n64, lo, hi,
+                       steps, codes, status);
 }
 
 cudaError_t launch_softedge_decode(const uint8_t* codes, int64_t n, float scale, int log2_ratio,

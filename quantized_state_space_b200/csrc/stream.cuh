@@ -95,6 +95,18 @@ __device__ __forceinline__ void smem16(const uint8_t* tile, int tid, float (&v)[
   }
 }
 
+// Thread `tid`'s 16 binary16 elements of a tile as 8 words of raw bits
+// (element 2 i in the low half of w[i]), same bank-conflict-free order as
+// smem16.
+__device__ __forceinline__ void smem16_bits(const uint8_t* tile, int tid, uint32_t (&w)[8]) {
+  const uint4* p = reinterpret_cast<const uint4*>(tile) + 2 * tid;
+  const int f = (tid >> 2) & 1;
+  const uint4 a = p[f], b = p[f ^ 1];
+  const uint4 lo = f ? b : a, hi = f ? a : b;
+  w[0] = lo.x; w[1] = lo.y; w[2] = lo.z; w[3] = lo.w;
+  w[4] = hi.x; w[5] = hi.y; w[6] = hi.z; w[7] = hi.w;
+}
+
 template <bool kF16, typename Idx>
 __device__ __forceinline__ void global16(const void* src, Idx e0, float (&v)[kVec]) {
   if (kF16) {
@@ -126,14 +138,25 @@ __device__ __forceinline__ float global1(const void* src, Idx e) {
   return static_cast<const float*>(src)[e];
 }
 
+struct NoPrologue {
+  __device__ __forceinline__ void operator()() const {}
+};
+
 // Runs the pipeline over src[0, n) as CTA c of G working on it (tile j of
 // the CTA is tile c + j G).  Every thread of the CTA (kThreads) must call it.
 // vec(x, e0) consumes the 16 elements e0..e0+15; one(v, e) a single element
-// of the ragged end.  Returns with every copy of this CTA complete.
-template <bool kF16, typename Idx, class Vec, class One>
+// of the ragged end.  prologue() runs on the consumer threads before their
+// first tile, while the producer's first copies are in flight, and is
+// followed by a barrier of the consumers.  Returns with every copy of this
+// CTA complete.
+// kBits (binary16 sources only): vec receives the raw bits, vec(const
+// uint32_t (&w)[8], e0), instead of fp32 values.
+template <bool kF16, typename Idx, class Vec, class One, class Pro = NoPrologue,
+          bool kBits = false>
 __device__ __forceinline__ void run_part(const void* __restrict__ src, Idx n, uint8_t* smem,
                                          const Idx c, const Idx G, Vec&& vec, One&& one,
-                                         uint32_t& flags, uint32_t limit = kWaitLimit) {
+                                         uint32_t& flags, uint32_t limit = kWaitLimit,
+                                         Pro&& prologue = Pro()) {
   constexpr int kEsz = kF16 ? 2 : 4;
   using C = Cfg<kEsz>;
   constexpr int S = C::kStages;
@@ -183,6 +206,8 @@ __device__ __forceinline__ void run_part(const void* __restrict__ src, Idx n, ui
     __syncwarp();
   } else {
     // ---- consumers
+    prologue();
+    tc::named_sync(1, kConsumers);
     const int lane = tid & 31;
     for (Idx j = 0; j < J; ++j) {
       const int s = (int)(j % S);
@@ -198,10 +223,17 @@ __device__ __forceinline__ void run_part(const void* __restrict__ src, Idx n, ui
         *abort_flag = 1u;
         break;
       }
-      float x[kVec];
-      smem16<kF16>(smem + s * C::kTileBytes, tid, x);
       const Idx tile = c + j * G;
-      vec(x, tile * (Idx)kTileElems + (Idx)tid * kVec);
+      if constexpr (kBits) {
+        static_assert(kF16, "raw bits are binary16 only");
+        uint32_t w[8];
+        smem16_bits(smem + s * C::kTileBytes, tid, w);
+        vec(w, tile * (Idx)kTileElems + (Idx)tid * kVec);
+      } else {
+        float x[kVec];
+        smem16<kF16>(smem + s * C::kTileBytes, tid, x);
+        vec(x, tile * (Idx)kTileElems + (Idx)tid * kVec);
+      }
       __syncwarp();
       if (lane == 0) arrive(empty + s);
     }
@@ -209,9 +241,16 @@ __device__ __forceinline__ void run_part(const void* __restrict__ src, Idx n, ui
     if (ntiles % G == c && !*abort_flag) {
       for (Idx e0 = ntiles * (Idx)kTileElems + (Idx)tid * kVec; e0 < n; e0 += (Idx)kConsumers * kVec) {
         if (e0 + kVec <= n) {
-          float x[kVec];
-          global16<kF16, Idx>(src, e0, x);
-          vec(x, e0);
+          if constexpr (kBits) {
+            const uint4* p = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(src) + e0);
+            const uint4 a = __ldg(p), b = __ldg(p + 1);
+            const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+            vec(w, e0);
+          } else {
+            float x[kVec];
+            global16<kF16, Idx>(src, e0, x);
+            vec(x, e0);
+          }
         } else {
           for (Idx e = e0; e < n; ++e) one(global1<kF16, Idx>(src, e), e);
         }
