@@ -38,6 +38,9 @@
 // The chunk length of the interface only fixes where the decomposition
 // restarts; the result is the recurrence's for any length, so the kernel uses
 // 128-step tiles for every accepted chunk length.
+#include <stdlib.h>
+#include <string.h>
+
 #include "common.cuh"
 #include "internal.h"
 #include "stream.cuh"
@@ -1195,6 +1198,8 @@ __global__ void __launch_bounds__(kThreads) ssd_fixup_kernel(const SsdParams p) 
   flag_status(p.status, flags);
 }
 
+#include "ssd_pipe.cuh"
+
 }  // namespace
 
 namespace {
@@ -1346,11 +1351,23 @@ cudaError_t launch_ssd(const ssmq_ssd_args& a, void* ws, cudaStream_t st) {
   p.seg_dec = p.seg_state + seg_slots(a, p.ntiles) * kP * kN;
   ssd_operand_kernel<<<dim3((unsigned)p.ntiles, (unsigned)(a.batch * a.ngroups)), kThreads, 0, st>>>(
       p, static_cast<uint8_t*>(ws));
-  auto kern = p.y_q ? ssd_kernel<true> : ssd_kernel<false>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       kSmemBytes);
-  if (e != cudaSuccess) return e;
-  kern<<<(unsigned)(sp.full + sp.r * sp.kseg), kThreads, kSmemBytes, st>>>(p);
+  // binary16 y: the pipelined kernel; int8 y (and SSMQ_SSD_KERNEL=classic, a
+  // diagnostic switch for comparing the two): the single-schedule kernel
+  const char* kv = getenv("SSMQ_SSD_KERNEL");
+  const bool classic = p.y_q || (kv && strcmp(kv, "classic") == 0);
+  const unsigned grid = (unsigned)(sp.full + sp.r * sp.kseg);
+  cudaError_t e;
+  if (classic) {
+    auto kern = p.y_q ? ssd_kernel<true> : ssd_kernel<false>;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    if (e != cudaSuccess) return e;
+    kern<<<grid, kThreads, kSmemBytes, st>>>(p);
+  } else {
+    e = cudaFuncSetAttribute(ssd_pipe_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             pipe::kPSmem);
+    if (e != cudaSuccess) return e;
+    ssd_pipe_kernel<<<grid, pipe::kPThreads, pipe::kPSmem, st>>>(p);
+  }
   if (sp.r > 0) {
     e = cudaFuncSetAttribute(ssd_fixup_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              kFixSmem);

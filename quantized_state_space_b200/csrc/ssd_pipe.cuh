@@ -1,0 +1,803 @@
+// Pipelined SSD kernel (binary16 y): included inside ssd.cu's anonymous
+// namespace, after ssd_kernel, whose decomposition, operand layouts and
+// arithmetic it keeps operation for operation (so its y and final state equal
+// ssd_kernel's bit for bit).  What changes is the schedule.
+//
+// The recurrence couples 128-step tiles only through the fp32 state:
+//   h_j = exp(S_last) h_{j-1} + ACC_j,   Y_off_j = C'_j h_{j-1}.
+// Everything else of tile j (CB_j, the decay-weighted M_j, Y_diag_j = M_j X_j,
+// the state increment ACC_j = B_j^T (w X)_j and the staging of x_j) does not
+// depend on the state, so it can run a tile ahead.  The CTA is split into
+// warp roles that work on different tiles at once and hand tiles to each
+// other through mbarriers; the tensor core, driven by one thread, runs
+// ACC_j, YD_j, YO_j and CB_{j+1} back to back while the CUDA cores form
+// M_{j+1}, stage x_{j+1}, update the state and write y_j.
+//
+//   warps 0-3   M role: M_j from CB_j (TMEM) -> TMEM (A operand of YD_j);
+//               thread = row t (warp w reads TMEM lanes 32 w ..), column
+//               blocks 0 .. w (the causal ones), two passes per row (row max,
+//               then the normalised binary16 values)
+//   warps 4-7   Y role: y_j from YD_j, YO_j (thread = row t), rows staged in
+//               shared memory, stored as whole 128-byte row segments
+//   warps 8-11  S role: the state h (thread = row n, all 64 p in registers),
+//               its maximum, the binary16 operand HH_{j+1} of YO_{j+1}
+//   warp 12     per-step factors of each tile (delta, S, w, the decay
+//               factors) and the operand-block copies
+//   warps 13-14 stage x_j (exact, and w x as binary16 high / residual parts)
+//               from the raw codes, fetched a tile ahead with cp.async
+//   warp 15     lane 0 issues every MMA
+// Every wait is bounded; a wait that gives up raises SSMQ_DEV_TIMEOUT and
+// the shared abort word, which ends every role's loop; the CTA then waits
+// (bounded) for its copies and MMAs in flight before it frees TMEM and exits.
+
+namespace pipe {
+
+constexpr int kPThreads = 512;
+// shared memory (bytes, dynamic)
+constexpr int P_OPS = 0;                      // 2 x 64 KB operand blocks (C', B) of tiles
+constexpr int P_X = P_OPS + 2 * kOpTile;      // x exact        [s][p] MN-major  16 KB
+constexpr int P_XH = P_X + kQ * kP * 2;       // w x high                        16 KB
+constexpr int P_XL = P_XH + kQ * kP * 2;      // w x residual                    16 KB
+constexpr int P_HH = P_XL + kQ * kP * 2;      // state operand  [n][p] MN-major  16 KB
+constexpr int P_YS = P_HH + kN * kP * 2;      // y rows of a tile (binary16)     16 KB
+constexpr int P_RX = P_YS + kQ * kP * 2;      // raw x codes    [t][p]            8 KB
+constexpr int P_F = P_RX + kQ * kP;           // fp32 scalars below
+// the final state (P x N fp32, 32 KB) passes through P_XH .. P_XL at the end
+// per-tile factor buffers (two, tile j in j & 1), floats
+constexpr int FB_S2 = 0;          // S_t log2(e) within the tile    [128]
+constexpr int FB_DW = 128;        // delta_s                        [128]
+constexpr int FB_WX = 256;        // w_s = exp2(S_last - S_s) delta_s
+constexpr int FB_ES = 384;        // exp2(S_t)
+constexpr int FB_CW = 512;        // exp2(S_p(s) - S_s) delta_s w_max, p(s) = s | 31
+constexpr int FB_CD = 640;        // exp2(S_m(s) - S_s) delta_s w_max, m(s) = s & ~31
+constexpr int FB_BS = 768;        // S spread per 32-step block     [4]
+constexpr int FB_WM = 772;        // max w_s of the tile
+constexpr int FB_SL = 773;        // S_last
+constexpr int FB_SIZE = 776;
+constexpr int G_FB = 0;                       // 2 factor buffers
+constexpr int G_RS = G_FB + 2 * FB_SIZE;      // row scale 2^e_t of M_j  [2][128]
+constexpr int G_EH = G_RS + 2 * kQ;           // state normalisation exponent of HH_j [2] (int)
+constexpr int G_HF = G_EH + 4;                // sC_n / w'_n              [128]
+constexpr int G_SB = G_HF + kN;               // sB_n                     [128]
+constexpr int G_SX = G_SB + kN;               // x scale per p            [64]
+constexpr int G_RED = G_SX + kP;              // reductions               [32]
+constexpr int G_END = G_RED + 32;
+constexpr int kPSmem = P_F + G_END * 4;
+static_assert(kPSmem + 1024 <= 232448, "shared memory of one CTA");
+static_assert(P_XL + kQ * kP * 2 - P_XH >= kP * kN * 4, "final state staging");
+
+// TMEM columns
+constexpr uint32_t T_CB = 0, T_M = 128, T_YD = 192, T_YO = 256, T_ACC = 320;
+
+// mbarriers (static shared memory), index
+enum {
+  B_OPS0 = 0, B_OPS1,   // operand block of a tile landed (bytes)
+  B_CB,                 // CB_j complete (tcgen05.commit)
+  B_ACC,                // ACC_j complete
+  B_YD,                 // YD_j complete (and every earlier MMA)
+  B_YO,                 // YO_j complete
+  B_M,                  // M_j in TMEM (4 M warps)
+  B_STAGE,              // X_j, XH_j, XL_j staged (2 staging warps)
+  B_HH,                 // HH_j staged (4 S warps)
+  B_YFREE,              // Y role done reading YD_j, YO_j (4 Y warps)
+  B_ACCFREE,            // S role done reading ACC_j (4 S warps)
+  B_FAC0, B_FAC1,       // factors of a tile ready (factor warp)
+  B_FFREE0, B_FFREE1,   // factor buffer free again (14 consumer warps)
+  B_RS0, B_RS1,         // row scales of M_j written (4 M warps), buffer j & 1
+  B_EH0, B_EH1,         // e_h of HH_j written (one S thread), buffer j & 1
+  B_OPSF0, B_OPSF1,     // every MMA reading operand buffer j & 1 complete
+  B_FINAL,              // every MMA complete (end)
+  kNumBars
+};
+// A wait for phase k of an mbarrier is only correct while phase k + 1 has not
+// completed (the parity would alias); every wait below is gated that way: the
+// barrier's next phase needs something the waiting role does after the wait.
+constexpr uint32_t kFacConsumers = 14;  // M 4 + Y 4 + S 4 + staging 2
+
+// Probes at most `limit` times, giving up early when another role aborted.
+__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity,
+                                         const volatile int* abort_flag) {
+  for (uint32_t i = 0; i < kWaitLimit; ++i) {
+    if (tc::mbar_try(bar, parity)) return true;
+    if (*abort_flag) return false;
+  }
+  return false;
+}
+
+__device__ __forceinline__ void bar_arrive(uint64_t* bar) { stream::arrive(bar); }
+
+// AND of `pred` over the `n` threads of named barrier `id` (all of them take
+// part, so a role's warps leave a loop together and never leave one another
+// waiting at a named barrier)
+__device__ __forceinline__ bool named_and(uint32_t id, uint32_t n, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
+      "barrier.red.and.pred q, %2, %3, p;\n\tselp.u32 %0, 1, 0, q;\n\t}\n"
+      : "=r"(r)
+      : "r"((uint32_t)pred), "r"(id), "r"(n)
+      : "memory");
+  return r != 0;
+}
+
+}  // namespace pipe
+
+__global__ void __launch_bounds__(pipe::kPThreads, 1) ssd_pipe_kernel(const SsdParams p) {
+  using namespace pipe;
+  extern __shared__ __align__(128) uint8_t smem[];
+  __shared__ uint32_t tmem_slot;
+  __shared__ __align__(8) uint64_t bars[kNumBars];
+  __shared__ int abort_flag;
+  float* F = reinterpret_cast<float*>(smem + P_F);
+  volatile int* abort_v = &abort_flag;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  // work item: a whole (batch, head) sequence, or segment seg of one
+  int64_t u, t_beg = 0, t_end = p.L;
+  int seg = 0, slot = -1;
+  if ((int64_t)blockIdx.x < p.full) {
+    u = blockIdx.x;
+  } else {
+    const int64_t idx = (int64_t)blockIdx.x - p.full;
+    u = p.full + idx / p.kseg;
+    seg = (int)(idx % p.kseg);
+    slot = (int)idx;
+    t_beg = (int64_t)seg * p.seg_tiles * kQ;
+    t_end = min(p.L, t_beg + (int64_t)p.seg_tiles * kQ);
+  }
+  const int64_t H = p.H, L = p.L;
+  const int64_t bb = u / H, hd = u % H;
+  const int64_t g = hd * p.G / H;
+  const int nt = (int)((t_end - t_beg + kQ - 1) / kQ);
+  const uint32_t s_base = tc::smem_u32(smem);
+  uint32_t flags = 0;
+  auto fail = [&]() {
+    flags |= SSMQ_DEV_TIMEOUT;
+    *abort_v = 1;
+  };
+
+  // ---- per-CTA constants (as ssd_kernel)
+  float sc_n = 0.0f, sb_n = 0.0f;
+  if (tid < kN) {
+    const int si = (int)g * (kN / p.gs) + tid / p.gs;
+    sc_n = __ldg(p.C_scale + si);
+    sb_n = __ldg(p.B_scale + si);
+    F[G_SB + tid] = sb_n;
+  }
+  if (tid < kP) {
+    float sx = p.se.s[0];
+    if (p.xfmt == SSMQ_X_INT8_GROUP) {
+      const int xg = __ldg(p.x_group + hd * kP + tid);
+      if ((unsigned)xg < (unsigned)p.n_x_groups) {
+        sx = __ldg(p.x_scale + xg);
+      } else {
+        sx = 0.0f;
+        flags |= SSMQ_DEV_BAD_GROUP;
+      }
+    }
+    F[G_SX + tid] = sx;
+  }
+  if (tid == 0) abort_flag = 0;
+  if (warp == 0) tc::tmem_alloc(&tmem_slot, 512);
+  if (tid == 0) {
+    tc::mbar_init(&bars[B_OPS0], 1);
+    tc::mbar_init(&bars[B_OPS1], 1);
+    tc::mbar_init(&bars[B_CB], 1);
+    tc::mbar_init(&bars[B_ACC], 1);
+    tc::mbar_init(&bars[B_YD], 1);
+    tc::mbar_init(&bars[B_YO], 1);
+    tc::mbar_init(&bars[B_M], 4);
+    tc::mbar_init(&bars[B_STAGE], 2);
+    tc::mbar_init(&bars[B_HH], 4);
+    tc::mbar_init(&bars[B_YFREE], 4);
+    tc::mbar_init(&bars[B_ACCFREE], 4);
+    tc::mbar_init(&bars[B_FAC0], 1);
+    tc::mbar_init(&bars[B_FAC1], 1);
+    tc::mbar_init(&bars[B_FFREE0], kFacConsumers);
+    tc::mbar_init(&bars[B_FFREE1], kFacConsumers);
+    tc::mbar_init(&bars[B_RS0], 4);
+    tc::mbar_init(&bars[B_RS1], 4);
+    tc::mbar_init(&bars[B_EH0], 1);
+    tc::mbar_init(&bars[B_EH1], 1);
+    tc::mbar_init(&bars[B_OPSF0], 1);
+    tc::mbar_init(&bars[B_OPSF1], 1);
+    tc::mbar_init(&bars[B_FINAL], 1);
+  }
+  __syncthreads();
+  const float wmax = block_max(sc_n * sb_n, F + G_RED, tid);
+  if (tid < kN) {
+    const __half wh = __float2half_rn(wmax > 0.0f ? sc_n * sb_n / wmax : 0.0f);
+    const float whf = __half2float(wh);
+    F[G_HF + tid] = whf > 0.0f ? sc_n / whf : 0.0f;
+  }
+  const float A2 = __ldg(p.A + hd) * kLog2e;
+  const float bias = p.dt_bias ? __ldg(p.dt_bias + hd) : 0.0f;
+  const float Dh = p.D ? __ldg(p.D + hd) : 0.0f;
+  const uint8_t* ops_bg = p.ops + (bb * p.G + g) * p.ntiles * (int64_t)kOpTile;
+  const int64_t tile0 = t_beg / kQ;
+  const uint32_t tmem = tmem_slot;
+  // operand block of tile j -> buffer j & 1 (the (j >> 1)-th copy into it)
+  auto issue_ops = [&](int j) {
+    stream::expect_tx(&bars[B_OPS0 + (j & 1)], (uint32_t)kOpTile);
+    stream::bulk_g2s(smem + P_OPS + (j & 1) * kOpTile, ops_bg + (tile0 + j) * kOpTile,
+                     (uint32_t)kOpTile, &bars[B_OPS0 + (j & 1)]);
+  };
+  int ops_issued = 0;  // warp 12 lane 0
+  tc::fence_before();
+  __syncthreads();  // constants and the TMEM address published
+  tc::fence_after();
+
+  if (warp < 4) {
+    // =================================================================== M
+    const int q = warp, t = 32 * q + lane;
+    const uint32_t t_lane = (uint32_t)(32 * q) << 16;
+    {  // column blocks above the diagonal stay zero
+      const uint32_t z[16] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+      for (int cb = q + 1; cb < 4; ++cb) tc::tmem_st16(tmem + t_lane + T_M + 16 * cb, z);
+      tc::tmem_wait_st();
+    }
+    for (int j = 0; j < nt; ++j) {
+      const int fb = j & 1;
+      const float* FB = F + G_FB + fb * FB_SIZE;
+      const bool ok = wait_bar(&bars[B_FAC0 + fb], (uint32_t)(j >> 1) & 1u, abort_v) &&
+                      wait_bar(&bars[B_CB], (uint32_t)j & 1u, abort_v) &&
+                      (j == 0 || wait_bar(&bars[B_YD], (uint32_t)(j - 1) & 1u, abort_v));
+      if (!__all_sync(0xffffffffu, ok)) {  // the warp leaves together (.sync.aligned loads)
+        fail();
+        break;
+      }
+      tc::fence_after();
+      const float st = FB[FB_S2 + t];
+      const float* S2 = FB + FB_S2;
+      const float* CW = FB + FB_CW;
+      const float* CD = FB + FB_CD;
+      const float* DW = FB + FB_DW;
+      // per block: the row factor rt and its max (pass 1), exactly as
+      // ssd_kernel's block (rb = q, q4 = cb) forms them
+      float rt[4], bmax[4];
+      int mode[4];  // 0 below the diagonal, 1 diagonal factored, 2 diagonal per element
+#pragma unroll
+      for (int cb = 0; cb < 4; ++cb) {
+        rt[cb] = 1.0f;
+        bmax[cb] = 0.0f;
+        mode[cb] = 0;
+        if (cb > q) continue;
+        const int s0 = 32 * cb;
+        if (cb < q) {
+          rt[cb] = ex2_sfu(st - S2[s0 + 31]);
+        } else if (FB[FB_BS + cb] < 90.0f) {
+          rt[cb] = ex2_sfu(st - S2[s0]);
+          mode[cb] = 1;
+        } else {
+          mode[cb] = 2;
+        }
+      }
+      auto block_vals = [&](int cb, float (&mv)[32]) {
+        float v[32];
+        tc::tmem_ld32(tmem + t_lane + T_CB + 32 * cb, v);
+        const int s0 = 32 * cb;
+        if (mode[cb] == 0) {
+#pragma unroll
+          for (int j4 = 0; j4 < 8; ++j4) {
+            const float4 c4 = *reinterpret_cast<const float4*>(CW + s0 + 4 * j4);
+            mv[4 * j4] = v[4 * j4] * c4.x;
+            mv[4 * j4 + 1] = v[4 * j4 + 1] * c4.y;
+            mv[4 * j4 + 2] = v[4 * j4 + 2] * c4.z;
+            mv[4 * j4 + 3] = v[4 * j4 + 3] * c4.w;
+          }
+        } else if (mode[cb] == 1) {
+#pragma unroll
+          for (int j4 = 0; j4 < 8; ++j4) {
+            const float4 c4 = *reinterpret_cast<const float4*>(CD + s0 + 4 * j4);
+            const float cd[4] = {c4.x, c4.y, c4.z, c4.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              mv[4 * j4 + e] = s0 + 4 * j4 + e <= t ? v[4 * j4 + e] * cd[e] : 0.0f;
+          }
+        } else {
+#pragma unroll
+          for (int jj = 0; jj < 32; ++jj) {
+            const int s = s0 + jj;
+            mv[jj] = s <= t ? v[jj] * ex2_sfu(st - S2[s]) * DW[s] * wmax : 0.0f;
+          }
+        }
+      };
+      // pass 1: block maxima
+      float rm = 0.0f;
+#pragma unroll
+      for (int cb = 0; cb < 4; ++cb) {
+        if (cb > q) break;
+        float mv[32];
+        block_vals(cb, mv);
+        float mx = 0.0f;
+#pragma unroll
+        for (int jj = 0; jj < 32; ++jj) mx = fmaxf(mx, fabsf(mv[jj]));
+        bmax[cb] = mode[cb] == 2 ? mx : mx * rt[cb];
+        rm = fmaxf(rm, bmax[cb]);
+      }
+      const int et = norm_exp(rm);
+      // pass 2: the normalised binary16 values
+#pragma unroll
+      for (int cb = 0; cb < 4; ++cb) {
+        if (cb > q) break;
+        float mv[32];
+        block_vals(cb, mv);
+        const float sc = pow2i(-et) * rt[cb];
+        uint32_t o[16];
+#pragma unroll
+        for (int k = 0; k < 16; ++k) o[k] = pack_h2(mv[2 * k] * sc, mv[2 * k + 1] * sc);
+        tc::tmem_st16(tmem + t_lane + T_M + 16 * cb, o);
+      }
+      F[G_RS + fb * kQ + t] = pow2i(et);
+      tc::tmem_wait_st();
+      tc::fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        bar_arrive(&bars[B_M]);
+        bar_arrive(&bars[B_RS0 + fb]);
+        bar_arrive(&bars[B_FFREE0 + fb]);
+      }
+    }
+  } else if (warp < 8) {
+    // =================================================================== Y
+    const int q = warp - 4, t = 32 * q + lane;
+    const uint32_t t_lane = (uint32_t)(32 * q) << 16;
+    for (int j = 0; j < nt; ++j) {
+      const int fb = j & 1;
+      const float* FB = F + G_FB + fb * FB_SIZE;
+      const int64_t t0 = t_beg + (int64_t)j * kQ;
+      const int ql = (int)min((int64_t)kQ, t_end - t0);
+      // this row's x codes (64 bytes, an L2 hit: the staging fetched them) and z
+      uint32_t xwv[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) xwv[i] = 0u;
+      const int64_t row_off = ((bb * L + t0 + t) * H + hd) * kP;
+      if (t < ql) {
+        const uint4* xs = reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(p.x) + row_off);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const uint4 v = __ldg(xs + i);
+          xwv[4 * i] = v.x;
+          xwv[4 * i + 1] = v.y;
+          xwv[4 * i + 2] = v.z;
+          xwv[4 * i + 3] = v.w;
+        }
+      }
+      bool ok = wait_bar(&bars[B_FAC0 + fb], (uint32_t)(j >> 1) & 1u, abort_v) &&
+                wait_bar(&bars[B_RS0 + fb], (uint32_t)(j >> 1) & 1u, abort_v) &&
+                wait_bar(&bars[B_EH0 + fb], (uint32_t)(j >> 1) & 1u, abort_v) &&
+                wait_bar(&bars[B_YD], (uint32_t)j & 1u, abort_v) &&
+                wait_bar(&bars[B_YO], (uint32_t)j & 1u, abort_v);
+      if (!named_and(1, 128, ok)) {
+        fail();
+        break;
+      }
+      tc::fence_after();
+      const float rs = F[G_RS + fb * kQ + t];
+      const int eh = reinterpret_cast<const int*>(F + G_EH)[fb];
+      const float es = FB[FB_ES + t] * pow2i(eh);
+      uint8_t* yrow = smem + P_YS + t * (2 * kP);
+#pragma unroll
+      for (int qq = 0; qq < 4; ++qq) {  // columns 16 qq .. 16 qq + 15
+        float yd[16], yo[16];
+        tc::tmem_ld16(tmem + t_lane + T_YD + 16 * qq, yd);
+        tc::tmem_ld16(tmem + t_lane + T_YO + 16 * qq, yo);
+        uint32_t zw[8];
+        if (p.z && t < ql) {
+          const uint4* zr = reinterpret_cast<const uint4*>(p.z + row_off + 16 * qq);
+          const uint4 z0 = __ldg(zr), z1 = __ldg(zr + 1);
+          zw[0] = z0.x; zw[1] = z0.y; zw[2] = z0.z; zw[3] = z0.w;
+          zw[4] = z1.x; zw[5] = z1.y; zw[6] = z1.z; zw[7] = z1.w;
+        }
+        uint32_t out[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const int pj = 16 * qq + 2 * k;  // column of the pair
+          const uint32_t xw = xwv[pj >> 2];
+          const float x0 = x_exact((xw >> (8 * (pj & 3))) & 0xFFu, p.xfmt, p.se_shift);
+          const float x1 = x_exact((xw >> (8 * ((pj + 1) & 3))) & 0xFFu, p.xfmt, p.se_shift);
+          const float2 sx = *reinterpret_cast<const float2*>(F + G_SX + pj);
+          float r2[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const float xv = e ? x1 : x0;
+            float yv = fmaf(e ? sx.y : sx.x, fmaf(Dh, xv, yd[2 * k + e] * rs), es * yo[2 * k + e]);
+            if (p.z) {
+              const float2 zf = __half22float2(*reinterpret_cast<const __half2*>(&zw[k]));
+              yv *= silu_f(e ? zf.y : zf.x);
+            }
+            r2[e] = yv;
+          }
+          out[k] = pack_half2(r2[0], r2[1]);
+        }
+        // swizzled 16-byte chunks (chunk c of row t at c ^ (t & 7))
+#pragma unroll
+        for (int c = 0; c < 2; ++c)
+          *reinterpret_cast<uint4*>(yrow + 16 * ((2 * qq + c) ^ (t & 7))) =
+              make_uint4(out[4 * c], out[4 * c + 1], out[4 * c + 2], out[4 * c + 3]);
+      }
+      tc::fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        bar_arrive(&bars[B_YFREE]);
+        bar_arrive(&bars[B_FFREE0 + fb]);
+      }
+      tc::named_sync(1, 128);  // the tile's y rows staged
+      // store: 128 threads, whole 128-byte row segments (8 threads per row)
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int k = 128 * i + 32 * q + lane, r = k >> 3, c = k & 7;
+        if (r < ql) {
+          const uint4 v = *reinterpret_cast<const uint4*>(smem + P_YS + r * (2 * kP) +
+                                                           16 * (c ^ (r & 7)));
+          *reinterpret_cast<uint4*>(p.y + ((bb * L + t0 + r) * H + hd) * kP + 8 * c) = v;
+        }
+      }
+      tc::named_sync(1, 128);  // staging buffer free for the next tile
+    }
+  } else if (warp < 12) {
+    // =================================================================== S
+    const int q = warp - 8, n = 32 * q + lane;
+    const uint32_t t_lane = (uint32_t)(32 * q) << 16;
+    const float hfac = F[G_HF + n];
+    const float sbr = F[G_SB + n];
+    float hs[64];
+#pragma unroll
+    for (int i = 0; i < 64; ++i)
+      hs[i] = (p.h0 && seg == 0) ? __ldg(p.h0 + u * kP * kN + (int64_t)i * kN + n) : 0.0f;
+    float s_tot = 0.0f;
+    // exponent e_h of the state operand: the maximum of |h sC/w'| over the
+    // whole state (the S warps), as ssd_kernel's state_max
+    auto state_exp = [&]() {
+      float hm = 0.0f;
+#pragma unroll
+      for (int i = 0; i < 64; ++i) hm = fmaxf(hm, fabsf(hs[i] * hfac));
+#pragma unroll
+      for (int o = 16; o >= 1; o >>= 1) hm = fmaxf(hm, __shfl_xor_sync(0xffffffffu, hm, o));
+      if (lane == 0) F[G_RED + 8 + q] = hm;
+      tc::named_sync(2, 128);
+      const float m = fmaxf(fmaxf(F[G_RED + 8], F[G_RED + 9]), fmaxf(F[G_RED + 10], F[G_RED + 11]));
+      tc::named_sync(2, 128);  // partials read before the next round writes them
+      return norm_exp(m);
+    };
+    // HH = h sC_n / w'_n 2^-e_h, binary16, [n][p] MN-major
+    auto stage_hh = [&](int eh) {
+      const float f = hfac * pow2i(-eh);
+#pragma unroll
+      for (int grp = 0; grp < 8; ++grp) {
+        uint32_t oh[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) oh[k] = pack_h2(hs[8 * grp + 2 * k] * f, hs[8 * grp + 2 * k + 1] * f);
+        *reinterpret_cast<uint4*>(smem + P_HH + tc::mnmaj_off(8 * grp, n, kP)) =
+            make_uint4(oh[0], oh[1], oh[2], oh[3]);
+      }
+      tc::fence_async_smem();
+      __syncwarp();
+    };
+    {
+      const int eh = state_exp();
+      if (n == 0) {
+        reinterpret_cast<int*>(F + G_EH)[0] = eh;
+        bar_arrive(&bars[B_EH0]);
+      }
+      stage_hh(eh);
+      if (lane == 0) bar_arrive(&bars[B_HH]);
+    }
+    for (int j = 0; j < nt; ++j) {
+      const int fb = j & 1;
+      const float* FB = F + G_FB + fb * FB_SIZE;
+      const bool ok = wait_bar(&bars[B_FAC0 + fb], (uint32_t)(j >> 1) & 1u, abort_v) &&
+                      wait_bar(&bars[B_ACC], (uint32_t)j & 1u, abort_v);
+      if (!named_and(2, 128, ok)) {
+        fail();
+        break;
+      }
+      tc::fence_after();
+      const float s_last = FB[FB_SL];
+      const int ex = norm_exp(FB[FB_WM] * p.x_bound);
+      const float decay = ex2_sfu(s_last);
+      const float f = sbr * pow2i(ex);
+#pragma unroll
+      for (int qq = 0; qq < 4; ++qq) {
+        float acc[16];
+        tc::tmem_ld16(tmem + t_lane + T_ACC + 16 * qq, acc);
+#pragma unroll
+        for (int i4 = 0; i4 < 4; ++i4) {
+          const float4 sx4 = *reinterpret_cast<const float4*>(F + G_SX + 16 * qq + 4 * i4);
+          const float sx[4] = {sx4.x, sx4.y, sx4.z, sx4.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int i = 16 * qq + 4 * i4 + e;
+            hs[i] = fmaf(decay, hs[i], f * sx[e] * acc[4 * i4 + e]);
+          }
+        }
+      }
+      if (n == 0) s_tot += s_last;
+      tc::fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        bar_arrive(&bars[B_ACCFREE]);
+        bar_arrive(&bars[B_FFREE0 + fb]);
+      }
+      if (j + 1 < nt) {
+        const int eh = state_exp();
+        const bool ok2 = wait_bar(&bars[B_YO], (uint32_t)j & 1u, abort_v);  // HH_j read by YO_j
+        if (!named_and(2, 128, ok2)) {
+          fail();
+          break;
+        }
+        if (n == 0) {
+          reinterpret_cast<int*>(F + G_EH)[(j + 1) & 1] = eh;
+          bar_arrive(&bars[B_EH0 + ((j + 1) & 1)]);
+        }
+        stage_hh(eh);
+        if (lane == 0) bar_arrive(&bars[B_HH]);
+      }
+    }
+    // every MMA is complete (the MMA thread waited for all of them) before
+    // the state staging area (XH, XL) is written
+    if (!wait_bar(&bars[B_FINAL], 0u, abort_v)) fail();
+    float* fin = slot < 0 ? (p.h_final ? p.h_final + u * kP * kN : nullptr)
+                          : p.seg_state + (int64_t)slot * kP * kN;
+    if (slot >= 0 && n == 0) p.seg_dec[slot] = s_tot;
+    if (slot < 0 && n == 0 && p.dec_final) p.dec_final[u] = s_tot;
+    if (fin) {
+      float* stage = reinterpret_cast<float*>(smem + P_XH);
+#pragma unroll
+      for (int i = 0; i < 64; ++i) stage[i * kN + n] = hs[i];
+      tc::named_sync(2, 128);
+      float4* dst = reinterpret_cast<float4*>(fin);
+      for (int i = 32 * q + lane; i < kP * kN / 4; i += 128) dst[i] = reinterpret_cast<float4*>(stage)[i];
+    }
+  } else if (warp == 12) {
+    // =========================================================== factors
+    uint16_t dtr[4] = {0, 0, 0, 0};
+    auto load_dt = [&](int j) {
+      const int64_t tt = t_beg + (int64_t)j * kQ;
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        dtr[i] = tt + 4 * lane + i < t_end ? p.dt[(bb * L + tt + 4 * lane + i) * H + hd] : (uint16_t)0;
+    };
+    if (lane == 0) {
+      issue_ops(0);
+      ++ops_issued;
+      if (nt > 1) {
+        issue_ops(1);
+        ++ops_issued;
+      }
+    }
+    load_dt(0);
+    for (int j = 0; j < nt; ++j) {
+      const int fb = j & 1;
+      const bool ok = j < 2 || wait_bar(&bars[B_FFREE0 + fb], (uint32_t)((j - 2) >> 1) & 1u, abort_v);
+      if (!__all_sync(0xffffffffu, ok)) {  // the warp leaves together (full-mask shuffles)
+        fail();
+        break;
+      }
+      const int ql = (int)min((int64_t)kQ, t_end - t_beg - (int64_t)j * kQ);
+      float dtv[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) dtv[i] = h2f(dtr[i]);
+      float* FBw = F + G_FB + fb * FB_SIZE;
+      // the same values as tile_factors (ssd_kernel), in this buffer layout
+      {
+        float dl[4], sc[4], off, s_last;
+        tile_decay(ql, dtv, bias, p.softplus, A2, lane, dl, sc, off, s_last);
+        float wmx = 0.0f;
+        const float s_blk = __shfl_sync(0xffffffffu, sc[3] + off, lane | 7);
+        const float s_beg = __shfl_sync(0xffffffffu, sc[0] + off, lane & ~7);
+        float smax = fmaxf(fmaxf(sc[0], sc[1]), fmaxf(sc[2], sc[3])) + off;
+        float smin = fminf(fminf(sc[0], sc[1]), fminf(sc[2], sc[3])) + off;
+#pragma unroll
+        for (int o = 4; o >= 1; o >>= 1) {
+          smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, o));
+          smin = fminf(smin, __shfl_xor_sync(0xffffffffu, smin, o));
+        }
+        if ((lane & 7) == 0) FBw[FB_BS + (lane >> 3)] = smax - smin;
+        float4 s2v, dwv, wxv, esv, cwv, cdv;
+        float* o4[6] = {&s2v.x, &dwv.x, &wxv.x, &esv.x, &cwv.x, &cdv.x};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float s2 = sc[i] + off;
+          const float w = ex2_sfu(s_last - s2) * dl[i];
+          o4[0][i] = s2;
+          o4[1][i] = dl[i];
+          o4[2][i] = w;
+          o4[3][i] = ex2_sfu(s2);
+          o4[4][i] = ex2_sfu(s_blk - s2) * dl[i] * wmax;
+          o4[5][i] = ex2_sfu(s_beg - s2) * dl[i] * wmax;
+          wmx = fmaxf(wmx, w);
+        }
+        *reinterpret_cast<float4*>(FBw + FB_S2 + 4 * lane) = s2v;
+        *reinterpret_cast<float4*>(FBw + FB_DW + 4 * lane) = dwv;
+        *reinterpret_cast<float4*>(FBw + FB_WX + 4 * lane) = wxv;
+        *reinterpret_cast<float4*>(FBw + FB_ES + 4 * lane) = esv;
+        *reinterpret_cast<float4*>(FBw + FB_CW + 4 * lane) = cwv;
+        *reinterpret_cast<float4*>(FBw + FB_CD + 4 * lane) = cdv;
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) wmx = fmaxf(wmx, __shfl_xor_sync(0xffffffffu, wmx, o));
+        if (lane == 0) {
+          FBw[FB_WM] = wmx;
+          FBw[FB_SL] = s_last;
+        }
+      }
+      __syncwarp();
+      if (lane == 0) bar_arrive(&bars[B_FAC0 + fb]);
+      if (j + 1 < nt) load_dt(j + 1);
+      // operand block of tile j + 1 into the buffer tile j - 1 used, once
+      // YO_{j-1} (the last MMA reading it) is complete
+      if (lane == 0 && j >= 1 && j + 1 < nt) {
+        if (!wait_bar(&bars[B_OPSF0 + ((j - 1) & 1)], (uint32_t)((j - 1) >> 1) & 1u, abort_v)) {
+          fail();
+        } else {
+          issue_ops(j + 1);
+          ++ops_issued;
+        }
+      }
+      if (__shfl_sync(0xffffffffu, *abort_v, 0)) break;
+    }
+    // copies issued land before the CTA may exit (the last two at most)
+    if (lane == 0)
+      for (int j = max(0, ops_issued - 2); j < ops_issued; ++j)
+        if (!tc::mbar_wait(&bars[B_OPS0 + (j & 1)], (uint32_t)(j >> 1) & 1u, kWaitLimit))
+          flags |= SSMQ_DEV_TIMEOUT;
+  } else if (warp < 15) {
+    // ============================================================ staging
+    const int sw = warp - 13, st_tid = 32 * sw + lane;  // 64 threads
+    // cp.async the raw x codes of tile j into RX (rows at or beyond the end
+    // are not fetched; the staging zeroes them)
+    auto fetch = [&](int j) {
+      const int64_t tt = t_beg + (int64_t)j * kQ;
+      const int ql = (int)min((int64_t)kQ, t_end - tt);
+      for (int w = st_tid; w < kQ * (kP / 16); w += 64) {
+        const int r = w >> 2, c = w & 3;
+        if (r >= ql) continue;
+        const int64_t xo = ((bb * L + tt + r) * H + hd) * kP + 16 * c;
+        tc::cp_async16(smem + P_RX + r * kP + 16 * (c ^ (r & 3)),
+                       static_cast<const uint8_t*>(p.x) + xo);
+      }
+      tc::cp_async_commit();
+    };
+    fetch(0);
+    for (int j = 0; j < nt; ++j) {
+      const int fb = j & 1;
+      const float* FB = F + G_FB + fb * FB_SIZE;
+      const int ql = (int)min((int64_t)kQ, t_end - t_beg - (int64_t)j * kQ);
+      const bool ok = wait_bar(&bars[B_FAC0 + fb], (uint32_t)(j >> 1) & 1u, abort_v) &&
+                      (j == 0 || wait_bar(&bars[B_YD], (uint32_t)(j - 1) & 1u, abort_v));
+      tc::cp_async_wait_all();
+      if (!named_and(3, 64, ok)) {  // also: the raw rows of tile j landed (both warps' copies)
+        fail();
+        break;
+      }
+      const int ex = norm_exp(FB[FB_WM] * p.x_bound);
+      const float xsc = pow2i(-ex);
+      // item (s, part): row s, p in [16 part, 16 part + 16): 512 items
+      for (int it = st_tid; it < kQ * 4; it += 64) {
+        const int s = it >> 2, part = it & 3;
+        const bool ok = s < ql;
+        const uint4 xq = ok ? *reinterpret_cast<const uint4*>(smem + P_RX + s * kP +
+                                                              16 * (part ^ (s & 3)))
+                            : make_uint4(0, 0, 0, 0);
+        const float ws = FB[FB_WX + s] * xsc;
+#pragma unroll
+        for (int grp = 0; grp < 2; ++grp) {
+          const uint32_t w0 = grp ? xq.z : xq.x, w1 = grp ? xq.w : xq.y;
+          float xv[8];
+          uint32_t ox[4], oh[4], ol[4];
+          if (p.xfmt == SSMQ_X_INT8_GROUP) {
+            const uint32_t x0 = w0 ^ 0x80808080u, x1 = w1 ^ 0x80808080u;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              xv[k] = s8_to_f32(x0, k);
+              xv[4 + k] = s8_to_f32(x1, k);
+            }
+            ox[0] = h2_bits(s8x2_to_h2(x0, 0, 1));
+            ox[1] = h2_bits(s8x2_to_h2(x0, 2, 3));
+            ox[2] = h2_bits(s8x2_to_h2(x1, 0, 1));
+            ox[3] = h2_bits(s8x2_to_h2(x1, 2, 3));
+          } else {
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              xv[k] = x_exact((w0 >> (8 * k)) & 0xFFu, p.xfmt, p.se_shift);
+              xv[4 + k] = x_exact((w1 >> (8 * k)) & 0xFFu, p.xfmt, p.se_shift);
+            }
+#pragma unroll
+            for (int k = 0; k < 4; ++k) ox[k] = pack_h2(xv[2 * k], xv[2 * k + 1]);
+          }
+#pragma unroll
+          for (int k = 0; k < 4; ++k) split_h2(ws * xv[2 * k], ws * xv[2 * k + 1], oh[k], ol[k]);
+          const uint32_t off = tc::mnmaj_off(16 * part + 8 * grp, s, kP);
+          *reinterpret_cast<uint4*>(smem + P_X + off) = make_uint4(ox[0], ox[1], ox[2], ox[3]);
+          *reinterpret_cast<uint4*>(smem + P_XH + off) = make_uint4(oh[0], oh[1], oh[2], oh[3]);
+          *reinterpret_cast<uint4*>(smem + P_XL + off) = make_uint4(ol[0], ol[1], ol[2], ol[3]);
+        }
+      }
+      tc::fence_async_smem();
+      tc::named_sync(3, 64);  // operands staged, raw rows consumed
+      if (lane == 0) {
+        bar_arrive(&bars[B_STAGE]);
+        bar_arrive(&bars[B_FFREE0 + fb]);
+      }
+      if (j + 1 < nt) fetch(j + 1);
+    }
+    tc::cp_async_wait_all();  // no copy lands after the CTA has exited
+  } else {
+    // ================================================================ MMA
+    if (lane == 0) {
+      const uint32_t id_cb = tc::idesc_f16(kQ, kQ, false, false);
+      const uint32_t id_y = tc::idesc_f16(kQ, kP, false, true);
+      const uint32_t id_s = tc::idesc_f16(kN, kP, true, true);
+      bool ok = wait_bar(&bars[B_OPS0], 0u, abort_v);
+      if (ok) {
+        tc::fence_after();
+        const uint32_t cb = s_base + P_OPS;
+#pragma unroll
+        for (int k0 = 0; k0 < kN; k0 += 16)
+          tc::mma_f16(tmem + T_CB, tc::kmaj_desc(cb, k0, kN), tc::kmaj_desc(cb + kOpBlock, k0, kN),
+                      id_cb, k0 > 0);
+        tc::mma_commit(&bars[B_CB]);
+      }
+      for (int j = 0; ok && j < nt; ++j) {
+        const uint32_t cbuf = s_base + P_OPS + (uint32_t)(j & 1) * kOpTile;
+        // ACC_j = B_j^T (w X)_j, high and residual parts
+        ok = wait_bar(&bars[B_STAGE], (uint32_t)j & 1u, abort_v) &&
+             (j == 0 || wait_bar(&bars[B_ACCFREE], (uint32_t)(j - 1) & 1u, abort_v));
+        if (!ok) break;
+        tc::fence_after();
+#pragma unroll
+        for (int k0 = 0; k0 < kQ; k0 += 16)
+          tc::mma_f16(tmem + T_ACC, tc::mnmaj_desc(cbuf + kOpBlock, k0, kN),
+                      tc::mnmaj_desc(s_base + P_XH, k0, kP), id_s, k0 > 0);
+#pragma unroll
+        for (int k0 = 0; k0 < kQ; k0 += 16)
+          tc::mma_f16(tmem + T_ACC, tc::mnmaj_desc(cbuf + kOpBlock, k0, kN),
+                      tc::mnmaj_desc(s_base + P_XL, k0, kP), id_s, 1u);
+        tc::mma_commit(&bars[B_ACC]);
+        // YD_j = M_j X_j
+        ok = wait_bar(&bars[B_M], (uint32_t)j & 1u, abort_v) &&
+             (j == 0 || wait_bar(&bars[B_YFREE], (uint32_t)(j - 1) & 1u, abort_v));
+        if (!ok) break;
+        tc::fence_after();
+#pragma unroll
+        for (int k0 = 0; k0 < kQ; k0 += 16)
+          tc::mma_f16_ts(tmem + T_YD, tmem + T_M + k0 / 2, tc::mnmaj_desc(s_base + P_X, k0, kP),
+                         id_y, k0 > 0);
+        tc::mma_commit(&bars[B_YD]);
+        // YO_j = C'_j HH_j
+        ok = wait_bar(&bars[B_HH], (uint32_t)j & 1u, abort_v);
+        if (!ok) break;
+        tc::fence_after();
+#pragma unroll
+        for (int k0 = 0; k0 < kN; k0 += 16)
+          tc::mma_f16(tmem + T_YO, tc::kmaj_desc(cbuf, k0, kN),
+                      tc::mnmaj_desc(s_base + P_HH, k0, kP), id_y, k0 > 0);
+        tc::mma_commit(&bars[B_YO]);
+        tc::mma_commit(&bars[B_OPSF0 + (j & 1)]);  // operand buffer j & 1 read completely
+        // CB_{j+1} (M_j has read CB_j: the wait on B_M above)
+        if (j + 1 < nt) {
+          ok = wait_bar(&bars[B_OPS0 + ((j + 1) & 1)], (uint32_t)((j + 1) >> 1) & 1u, abort_v);
+          if (!ok) break;
+          tc::fence_after();
+          const uint32_t nb = s_base + P_OPS + (uint32_t)((j + 1) & 1) * kOpTile;
+#pragma unroll
+          for (int k0 = 0; k0 < kN; k0 += 16)
+            tc::mma_f16(tmem + T_CB, tc::kmaj_desc(nb, k0, kN),
+                        tc::kmaj_desc(nb + kOpBlock, k0, kN), id_cb, k0 > 0);
+          tc::mma_commit(&bars[B_CB]);
+        }
+      }
+      if (!ok) fail();
+      // every MMA issued is complete before TMEM is freed (and before the S
+      // role reuses XH / XL for the final state)
+      tc::mma_commit(&bars[B_FINAL]);
+      if (!tc::mbar_wait(&bars[B_FINAL], 0u, kWaitLimit)) fail();
+    }
+    __syncwarp();
+  }
+
+  tc::fence_before();
+  __syncthreads();
+  if (warp == 0) tc::tmem_dealloc(tmem, 512);
+  flag_status(p.status, flags);
+}

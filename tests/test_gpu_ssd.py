@@ -307,3 +307,40 @@ def test_state_chain_and_carry_in_edge_cases():
     api.ssd_carry_in(*args, T(hc), y, x_group=T(p["x_group"]), x_scale=T(p["x_scale"]),
                      h_final=hft)
     np.testing.assert_array_equal(H(hft), hf + hc)
+
+
+# ---- the pipelined kernel against the single-schedule kernel ---------------
+# The binary16-y path runs a kernel whose warp roles work on different tiles
+# at once; it keeps the other kernel's arithmetic operation for operation, so
+# the two give the same bits (SSMQ_SSD_KERNEL=classic selects the other one).
+
+PIPE_CASES = [
+    # (b, L, H, G, gs, gate, h0, bias, fmt, dt_mean, max_segments)
+    (1, 128, 2, 1, 8, False, False, False, "int8", -4.0, 1),
+    (2, 300, 3, 1, 8, True, True, True, "int8", -4.0, 0),
+    (1, 1, 2, 1, 8, False, True, False, "int8", -4.0, 0),
+    (2, 512, 4, 4, 16, True, False, True, "int8", -2.0, 0),
+    (1, 384, 2, 1, 8, True, True, False, "softedge", -4.0, 0),
+    (1, 1000, 2, 1, 8, False, False, False, "int8", -5.0, 1),
+    (2, 2048, 5, 1, 8, False, True, True, "int8", -4.0, 0),   # segments of the last round
+    (1, 640, 2, 2, 8, False, False, False, "int8", 0.5, 1),   # very strong decay: per-element branch
+]
+
+
+@pytest.mark.parametrize("ci", range(len(PIPE_CASES)))
+def test_ssd_pipelined_equals_single_schedule(ci, monkeypatch):
+    b, L, Hh, G, gs, gate, h0, bias, fmt, dtm, ms = PIPE_CASES[ci]
+    p = ssd_problem(470 + ci, b, L, Hh, 64, 128, G=G, gs=gs, gate=gate, h0=h0, bias=bias,
+                    x_format=fmt, dt_mean=dtm)
+    dec_a = torch.zeros((b, Hh), dtype=torch.float32, device=dev())
+    dec_b = torch.zeros((b, Hh), dtype=torch.float32, device=dev())
+    st_a, st_b = status_word(), status_word()
+    ya, ha = gpu_ssd(p, max_segments=ms, dec_final=dec_a, status=st_a)
+    monkeypatch.setenv("SSMQ_SSD_KERNEL", "classic")
+    yb, hb = gpu_ssd(p, max_segments=ms, dec_final=dec_b, status=st_b)
+    torch.cuda.synchronize()
+    assert int(H(st_a)[0]) == 0 and int(H(st_b)[0]) == 0
+    np.testing.assert_array_equal(ya.astype(np.float16).view(np.uint16),
+                                  yb.astype(np.float16).view(np.uint16))
+    np.testing.assert_array_equal(ha.view(np.uint32), hb.view(np.uint32))
+    np.testing.assert_array_equal(H(dec_a).view(np.uint32), H(dec_b).view(np.uint32))
