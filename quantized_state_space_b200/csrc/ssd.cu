@@ -1363,10 +1363,12 @@ cudaError_t launch_ssd(const ssmq_ssd_args& a, void* ws, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     kern<<<grid, kThreads, kSmemBytes, st>>>(p);
   } else {
-    e = cudaFuncSetAttribute(ssd_pipe_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             pipe::kPSmem);
+    const bool se = p.xfmt == SSMQ_X_SOFTEDGE, gz = p.z != nullptr;
+    auto kern = se ? (gz ? ssd_pipe_kernel<true, true> : ssd_pipe_kernel<true, false>)
+                   : (gz ? ssd_pipe_kernel<false, true> : ssd_pipe_kernel<false, false>);
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, pipe::kPSmem);
     if (e != cudaSuccess) return e;
-    ssd_pipe_kernel<<<grid, pipe::kPThreads, pipe::kPSmem, st>>>(p);
+    kern<<<grid, pipe::kPThreads, pipe::kPSmem, st>>>(p);
   }
   if (sp.r > 0) {
     e = cudaFuncSetAttribute(ssd_fixup_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,

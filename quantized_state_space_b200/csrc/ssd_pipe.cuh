@@ -122,8 +122,14 @@ __device__ __forceinline__ bool named_and(uint32_t id, uint32_t n, bool pred) {
 
 }  // namespace pipe
 
+// kSE: x as soft-edge codes (else int8 codes); kZ: gated output.  The
+// specialisations keep each role's code small: the roles run different code
+// at the same time, so every instruction of a hot loop competes for the
+// instruction cache.
+template <bool kSE, bool kZ>
 __global__ void __launch_bounds__(pipe::kPThreads, 1) ssd_pipe_kernel(const SsdParams p) {
   using namespace pipe;
+  constexpr int kXF = kSE ? SSMQ_X_SOFTEDGE : SSMQ_X_INT8_GROUP;
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ uint32_t tmem_slot;
   __shared__ __align__(8) uint64_t bars[kNumBars];
@@ -252,81 +258,69 @@ __global__ void __launch_bounds__(pipe::kPThreads, 1) ssd_pipe_kernel(const SsdP
       const float* CW = FB + FB_CW;
       const float* CD = FB + FB_CD;
       const float* DW = FB + FB_DW;
-      // per block: the row factor rt and its max (pass 1), exactly as
-      // ssd_kernel's block (rb = q, q4 = cb) forms them
-      float rt[4], bmax[4];
-      int mode[4];  // 0 below the diagonal, 1 diagonal factored, 2 diagonal per element
-#pragma unroll
-      for (int cb = 0; cb < 4; ++cb) {
-        rt[cb] = 1.0f;
-        bmax[cb] = 0.0f;
-        mode[cb] = 0;
-        if (cb > q) continue;
-        const int s0 = 32 * cb;
+      // block cb's row factor and mode (0 below the diagonal, 1 diagonal
+      // factored, 2 diagonal per element), exactly as ssd_kernel's blocks
+      auto block_mode = [&](int cb, float& rt) {
+        rt = 1.0f;
         if (cb < q) {
-          rt[cb] = ex2_sfu(st - S2[s0 + 31]);
-        } else if (FB[FB_BS + cb] < 90.0f) {
-          rt[cb] = ex2_sfu(st - S2[s0]);
-          mode[cb] = 1;
-        } else {
-          mode[cb] = 2;
+          rt = ex2_sfu(st - S2[32 * cb + 31]);
+          return 0;
         }
-      }
-      auto block_vals = [&](int cb, float (&mv)[32]) {
-        float v[32];
-        tc::tmem_ld32(tmem + t_lane + T_CB + 32 * cb, v);
+        if (FB[FB_BS + cb] < 90.0f) {
+          rt = ex2_sfu(st - S2[32 * cb]);
+          return 1;
+        }
+        return 2;
+      };
+      auto block_vals = [&](int cb, int mode, float (&mv)[32]) {
+        tc::tmem_ld32(tmem + t_lane + T_CB + 32 * cb, mv);
         const int s0 = 32 * cb;
-        if (mode[cb] == 0) {
+        if (mode != 2) {
+          const float* fac = (mode == 0 ? CW : CD) + s0;
 #pragma unroll
           for (int j4 = 0; j4 < 8; ++j4) {
-            const float4 c4 = *reinterpret_cast<const float4*>(CW + s0 + 4 * j4);
-            mv[4 * j4] = v[4 * j4] * c4.x;
-            mv[4 * j4 + 1] = v[4 * j4 + 1] * c4.y;
-            mv[4 * j4 + 2] = v[4 * j4 + 2] * c4.z;
-            mv[4 * j4 + 3] = v[4 * j4 + 3] * c4.w;
+            const float4 c4 = *reinterpret_cast<const float4*>(fac + 4 * j4);
+            mv[4 * j4] *= c4.x;
+            mv[4 * j4 + 1] *= c4.y;
+            mv[4 * j4 + 2] *= c4.z;
+            mv[4 * j4 + 3] *= c4.w;
           }
-        } else if (mode[cb] == 1) {
+          if (mode == 1) {
 #pragma unroll
-          for (int j4 = 0; j4 < 8; ++j4) {
-            const float4 c4 = *reinterpret_cast<const float4*>(CD + s0 + 4 * j4);
-            const float cd[4] = {c4.x, c4.y, c4.z, c4.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e)
-              mv[4 * j4 + e] = s0 + 4 * j4 + e <= t ? v[4 * j4 + e] * cd[e] : 0.0f;
+            for (int jj = 0; jj < 32; ++jj)
+              if (s0 + jj > t) mv[jj] = 0.0f;
           }
         } else {
 #pragma unroll
           for (int jj = 0; jj < 32; ++jj) {
             const int s = s0 + jj;
-            mv[jj] = s <= t ? v[jj] * ex2_sfu(st - S2[s]) * DW[s] * wmax : 0.0f;
+            mv[jj] = s <= t ? mv[jj] * ex2_sfu(st - S2[s]) * DW[s] * wmax : 0.0f;
           }
         }
       };
-      // pass 1: block maxima
+      // pass 0: the row maximum over the blocks; pass 1: the normalised
+      // binary16 values (one loop body for both, to keep the code small)
       float rm = 0.0f;
+      int et = 0;
+#pragma unroll 1
+      for (int it = 0; it < 2 * (q + 1); ++it) {
+        const int pass = it > q, cb = pass ? it - q - 1 : it;
+        if (it == q + 1) et = norm_exp(rm);
+        float rt, mv[32];
+        const int mode = block_mode(cb, rt);
+        block_vals(cb, mode, mv);
+        if (!pass) {
+          float mx = 0.0f;
 #pragma unroll
-      for (int cb = 0; cb < 4; ++cb) {
-        if (cb > q) break;
-        float mv[32];
-        block_vals(cb, mv);
-        float mx = 0.0f;
+          for (int jj = 0; jj < 32; ++jj) mx = fmaxf(mx, fabsf(mv[jj]));
+          rm = fmaxf(rm, mode == 2 ? mx : mx * rt);
+        } else {
+          const float sc = pow2i(-et) * rt;
+          uint32_t o[16];
 #pragma unroll
-        for (int jj = 0; jj < 32; ++jj) mx = fmaxf(mx, fabsf(mv[jj]));
-        bmax[cb] = mode[cb] == 2 ? mx : mx * rt[cb];
-        rm = fmaxf(rm, bmax[cb]);
-      }
-      const int et = norm_exp(rm);
-      // pass 2: the normalised binary16 values
-#pragma unroll
-      for (int cb = 0; cb < 4; ++cb) {
-        if (cb > q) break;
-        float mv[32];
-        block_vals(cb, mv);
-        const float sc = pow2i(-et) * rt[cb];
-        uint32_t o[16];
-#pragma unroll
-        for (int k = 0; k < 16; ++k) o[k] = pack_h2(mv[2 * k] * sc, mv[2 * k + 1] * sc);
-        tc::tmem_st16(tmem + t_lane + T_M + 16 * cb, o);
+          for (int k = 0; k < 16; ++k) o[k] = pack_h2(mv[2 * k] * sc, mv[2 * k + 1] * sc);
+          tc::tmem_st16(tmem + t_lane + T_M + 16 * cb, o);
+        }
       }
       F[G_RS + fb * kQ + t] = pow2i(et);
       tc::tmem_wait_st();
@@ -347,22 +341,22 @@ __global__ void __launch_bounds__(pipe::kPThreads, 1) ssd_pipe_kernel(const SsdP
       const float* FB = F + G_FB + fb * FB_SIZE;
       const int64_t t0 = t_beg + (int64_t)j * kQ;
       const int ql = (int)min((int64_t)kQ, t_end - t0);
-      // this row's x codes (64 bytes, an L2 hit: the staging fetched them) and z
-      uint32_t xwv[16];
-#pragma unroll
-      for (int i = 0; i < 16; ++i) xwv[i] = 0u;
       const int64_t row_off = ((bb * L + t0 + t) * H + hd) * kP;
-      if (t < ql) {
-        const uint4* xs = reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(p.x) + row_off);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const uint4 v = __ldg(xs + i);
-          xwv[4 * i] = v.x;
-          xwv[4 * i + 1] = v.y;
-          xwv[4 * i + 2] = v.z;
-          xwv[4 * i + 3] = v.w;
+      const uint8_t* xrow = static_cast<const uint8_t*>(p.x) + row_off;
+      // this row's x codes (an L2 hit: the staging fetched them a tile ago)
+      // and z, one 16-column quarter ahead of their use
+      uint4 xq = make_uint4(0u, 0u, 0u, 0u), z0 = xq, z1 = xq;
+      auto load_q = [&](int qq, uint4& xv, uint4& za, uint4& zb) {
+        if (t < ql) {
+          xv = __ldg(reinterpret_cast<const uint4*>(xrow + 16 * qq));
+          if (kZ) {
+            const uint4* zr = reinterpret_cast<const uint4*>(p.z + row_off + 16 * qq);
+            za = __ldg(zr);
+            zb = __ldg(zr + 1);
+          }
         }
-      }
+      };
+      load_q(0, xq, z0, z1);
       bool ok = wait_bar(&bars[B_FAC0 + fb], (uint32_t)(j >> 1) & 1u, abort_v) &&
                 wait_bar(&bars[B_RS0 + fb], (uint32_t)(j >> 1) & 1u, abort_v) &&
                 wait_bar(&bars[B_EH0 + fb], (uint32_t)(j >> 1) & 1u, abort_v) &&
@@ -377,32 +371,29 @@ __global__ void __launch_bounds__(pipe::kPThreads, 1) ssd_pipe_kernel(const SsdP
       const int eh = reinterpret_cast<const int*>(F + G_EH)[fb];
       const float es = FB[FB_ES + t] * pow2i(eh);
       uint8_t* yrow = smem + P_YS + t * (2 * kP);
-#pragma unroll
+#pragma unroll 1
       for (int qq = 0; qq < 4; ++qq) {  // columns 16 qq .. 16 qq + 15
+        uint4 xn = make_uint4(0u, 0u, 0u, 0u), zn0 = xn, zn1 = xn;
+        if (qq < 3) load_q(qq + 1, xn, zn0, zn1);
         float yd[16], yo[16];
         tc::tmem_ld16(tmem + t_lane + T_YD + 16 * qq, yd);
         tc::tmem_ld16(tmem + t_lane + T_YO + 16 * qq, yo);
-        uint32_t zw[8];
-        if (p.z && t < ql) {
-          const uint4* zr = reinterpret_cast<const uint4*>(p.z + row_off + 16 * qq);
-          const uint4 z0 = __ldg(zr), z1 = __ldg(zr + 1);
-          zw[0] = z0.x; zw[1] = z0.y; zw[2] = z0.z; zw[3] = z0.w;
-          zw[4] = z1.x; zw[5] = z1.y; zw[6] = z1.z; zw[7] = z1.w;
-        }
+        const uint32_t xw[4] = {xq.x, xq.y, xq.z, xq.w};
+        const uint32_t zw[8] = {z0.x, z0.y, z0.z, z0.w, z1.x, z1.y, z1.z, z1.w};
+        const float* sxq = F + G_SX + 16 * qq;
         uint32_t out[8];
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
-          const int pj = 16 * qq + 2 * k;  // column of the pair
-          const uint32_t xw = xwv[pj >> 2];
-          const float x0 = x_exact((xw >> (8 * (pj & 3))) & 0xFFu, p.xfmt, p.se_shift);
-          const float x1 = x_exact((xw >> (8 * ((pj + 1) & 3))) & 0xFFu, p.xfmt, p.se_shift);
-          const float2 sx = *reinterpret_cast<const float2*>(F + G_SX + pj);
+          const uint32_t w = xw[k >> 1];
+          const float x0 = x_exact((w >> (16 * (k & 1))) & 0xFFu, kXF, p.se_shift);
+          const float x1 = x_exact((w >> (16 * (k & 1) + 8)) & 0xFFu, kXF, p.se_shift);
+          const float2 sx = *reinterpret_cast<const float2*>(sxq + 2 * k);
           float r2[2];
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
             const float xv = e ? x1 : x0;
             float yv = fmaf(e ? sx.y : sx.x, fmaf(Dh, xv, yd[2 * k + e] * rs), es * yo[2 * k + e]);
-            if (p.z) {
+            if (kZ) {
               const float2 zf = __half22float2(*reinterpret_cast<const __half2*>(&zw[k]));
               yv *= silu_f(e ? zf.y : zf.x);
             }
@@ -411,10 +402,13 @@ __global__ void __launch_bounds__(pipe::kPThreads, 1) ssd_pipe_kernel(const SsdP
           out[k] = pack_half2(r2[0], r2[1]);
         }
         // swizzled 16-byte chunks (chunk c of row t at c ^ (t & 7))
-#pragma unroll
-        for (int c = 0; c < 2; ++c)
-          *reinterpret_cast<uint4*>(yrow + 16 * ((2 * qq + c) ^ (t & 7))) =
-              make_uint4(out[4 * c], out[4 * c + 1], out[4 * c + 2], out[4 * c + 3]);
+        *reinterpret_cast<uint4*>(yrow + 16 * ((2 * qq) ^ (t & 7))) =
+            make_uint4(out[0], out[1], out[2], out[3]);
+        *reinterpret_cast<uint4*>(yrow + 16 * ((2 * qq + 1) ^ (t & 7))) =
+            make_uint4(out[4], out[5], out[6], out[7]);
+        xq = xn;
+        z0 = zn0;
+        z1 = zn1;
       }
       tc::fence_before();
       __syncwarp();
@@ -685,7 +679,7 @@ __global__ void __launch_bounds__(pipe::kPThreads, 1) ssd_pipe_kernel(const SsdP
           const uint32_t w0 = grp ? xq.z : xq.x, w1 = grp ? xq.w : xq.y;
           float xv[8];
           uint32_t ox[4], oh[4], ol[4];
-          if (p.xfmt == SSMQ_X_INT8_GROUP) {
+          if (!kSE) {
             const uint32_t x0 = w0 ^ 0x80808080u, x1 = w1 ^ 0x80808080u;
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
@@ -699,8 +693,8 @@ __global__ void __launch_bounds__(pipe::kPThreads, 1) ssd_pipe_kernel(const SsdP
           } else {
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
-              xv[k] = x_exact((w0 >> (8 * k)) & 0xFFu, p.xfmt, p.se_shift);
-              xv[4 + k] = x_exact((w1 >> (8 * k)) & 0xFFu, p.xfmt, p.se_shift);
+              xv[k] = x_exact((w0 >> (8 * k)) & 0xFFu, kXF, p.se_shift);
+              xv[4 + k] = x_exact((w1 >> (8 * k)) & 0xFFu, kXF, p.se_shift);
             }
 #pragma unroll
             for (int k = 0; k < 4; ++k) ox[k] = pack_h2(xv[2 * k], xv[2 * k + 1]);
