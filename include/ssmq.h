@@ -448,6 +448,9 @@ ssmq_status ssmq_selective_scan_w8(const ssmq_scan_args* args, void* stream);
  * may then be NULL.
  * status: SSMQ_DEV_BAD_GROUP as above; SSMQ_DEV_TIMEOUT if a bounded wait for
  * the tensor core gave up (the call's outputs are then incomplete).
+ * The environment variable SSMQ_SSD_KERNEL=pipelined (read at each call)
+ * selects, for binary16 y, an alternative kernel whose warp roles work on
+ * different tiles at once; it gives the same bytes.
  */
 typedef struct {
   int64_t batch, seqlen, nheads, headdim, dstate, ngroups;

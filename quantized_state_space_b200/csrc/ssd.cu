@@ -1351,10 +1351,12 @@ cudaError_t launch_ssd(const ssmq_ssd_args& a, void* ws, cudaStream_t st) {
   p.seg_dec = p.seg_state + seg_slots(a, p.ntiles) * kP * kN;
   ssd_operand_kernel<<<dim3((unsigned)p.ntiles, (unsigned)(a.batch * a.ngroups)), kThreads, 0, st>>>(
       p, static_cast<uint8_t*>(ws));
-  // binary16 y: the pipelined kernel; int8 y (and SSMQ_SSD_KERNEL=classic, a
-  // diagnostic switch for comparing the two): the single-schedule kernel
+  // The single-schedule kernel by default; SSMQ_SSD_KERNEL=pipelined selects
+  // the warp-role kernel for binary16 y (same bytes; slower on the 2.7B-shaped
+  // workload so far: its roles run different code at once and each role has
+  // one warp per scheduler, so instruction fetch and latency bound it)
   const char* kv = getenv("SSMQ_SSD_KERNEL");
-  const bool classic = p.y_q || (kv && strcmp(kv, "classic") == 0);
+  const bool classic = p.y_q || !(kv && strcmp(kv, "pipelined") == 0);
   const unsigned grid = (unsigned)(sp.full + sp.r * sp.kseg);
   cudaError_t e;
   if (classic) {

@@ -13,35 +13,39 @@
 // ACC_j, YD_j, YO_j and CB_{j+1} back to back while the CUDA cores form
 // M_{j+1}, stage x_{j+1}, update the state and write y_j.
 //
-//   warps 0-3   M role: M_j from CB_j (TMEM) -> TMEM (A operand of YD_j);
-//               thread = row t (warp w reads TMEM lanes 32 w ..), column
-//               blocks 0 .. w (the causal ones), two passes per row (row max,
+// Warp w reads TMEM lanes 32 (w % 4) .. (its lane quarter q = w % 4):
+//   warps 0-7   M role: M_j from CB_j (TMEM) -> TMEM (A operand of YD_j);
+//               thread = row t; the causal 32-column blocks 0 .. q of a row
+//               are split between warps q and q + 4 (at most two each), two
+//               passes (the row maximum, exchanged through shared memory,
 //               then the normalised binary16 values)
-//   warps 4-7   Y role: y_j from YD_j, YO_j (thread = row t), rows staged in
-//               shared memory, stored as whole 128-byte row segments
-//   warps 8-11  S role: the state h (thread = row n, all 64 p in registers),
-//               its maximum, the binary16 operand HH_{j+1} of YO_{j+1}
-//   warp 12     per-step factors of each tile (delta, S, w, the decay
+//   warps 8-11  Y role: y_j from YD_j, YO_j (thread = row t), each thread
+//               writing its row's 128 bytes
+//   warps 12-19 S role: the state h (thread = row n and 32 of the 64 p in
+//               registers), its maximum, the binary16 operand HH_{j+1}; and,
+//               right after the state update (when ACC_j has freed the w x
+//               buffers), the x operands of tile j + 1 (exact, double-
+//               buffered, and w x as binary16 high / residual parts) from the
+//               raw codes loaded before the wait
+//   warp 20     per-step factors of each tile (delta, S, w, the decay
 //               factors) and the operand-block copies
-//   warps 13-14 stage x_j (exact, and w x as binary16 high / residual parts)
-//               from the raw codes, fetched a tile ahead with cp.async
-//   warp 15     lane 0 issues every MMA
+//   warp 21     lane 0 issues every MMA: CB_{j+1} as soon as M_j has read
+//               CB_j, then ACC_j, YD_j, YO_j
 // Every wait is bounded; a wait that gives up raises SSMQ_DEV_TIMEOUT and
 // the shared abort word, which ends every role's loop; the CTA then waits
 // (bounded) for its copies and MMAs in flight before it frees TMEM and exits.
 
 namespace pipe {
 
-constexpr int kPThreads = 512;
+constexpr int kPThreads = 704;
+constexpr int W_Y = 8, W_S = 12, W_FAC = 20, W_MMA = 21;
 // shared memory (bytes, dynamic)
 constexpr int P_OPS = 0;                      // 2 x 64 KB operand blocks (C', B) of tiles
-constexpr int P_X = P_OPS + 2 * kOpTile;      // x exact        [s][p] MN-major  16 KB
-constexpr int P_XH = P_X + kQ * kP * 2;       // w x high                        16 KB
+constexpr int P_X = P_OPS + 2 * kOpTile;      // x exact [s][p] MN-major, 2 x 16 KB (tile j in j & 1)
+constexpr int P_XH = P_X + 2 * kQ * kP * 2;   // w x high                        16 KB
 constexpr int P_XL = P_XH + kQ * kP * 2;      // w x residual                    16 KB
 constexpr int P_HH = P_XL + kQ * kP * 2;      // state operand  [n][p] MN-major  16 KB
-constexpr int P_YS = P_HH + kN * kP * 2;      // y rows of a tile (binary16)     16 KB
-constexpr int P_RX = P_YS + kQ * kP * 2;      // raw x codes    [t][p]            8 KB
-constexpr int P_F = P_RX + kQ * kP;           // fp32 scalars below
+constexpr int P_F = P_HH + kN * kP * 2;       // fp32 scalars below
 // the final state (P x N fp32, 32 KB) passes through P_XH .. P_XL at the end
 // per-tile factor buffers (two, tile j in j & 1), floats
 constexpr int FB_S2 = 0;          // S_t log2(e) within the tile    [128]
@@ -61,7 +65,8 @@ constexpr int G_HF = G_EH + 4;                // sC_n / w'_n              [128]
 constexpr int G_SB = G_HF + kN;               // sB_n                     [128]
 constexpr int G_SX = G_SB + kN;               // x scale per p            [64]
 constexpr int G_RED = G_SX + kP;              // reductions               [32]
-constexpr int G_END = G_RED + 32;
+constexpr int G_RMX = G_RED + 32;             // M row maxima of the two warps of a quarter [2][128]
+constexpr int G_END = G_RMX + 2 * kQ;
 constexpr int kPSmem = P_F + G_END * 4;
 static_assert(kPSmem + 1024 <= 232448, "shared memory of one CTA");
 static_assert(P_XL + kQ * kP * 2 - P_XH >= kP * kN * 4, "final state staging");
@@ -76,23 +81,24 @@ enum {
   B_ACC,                // ACC_j complete
   B_YD,                 // YD_j complete (and every earlier MMA)
   B_YO,                 // YO_j complete
-  B_M,                  // M_j in TMEM (4 M warps)
-  B_STAGE,              // X_j, XH_j, XL_j staged (2 staging warps)
-  B_HH,                 // HH_j staged (4 S warps)
+  B_M,                  // M_j in TMEM (8 M warps)
+  B_STAGE,              // X_j, XH_j, XL_j staged (8 S warps)
+  B_HH,                 // HH_j staged (8 S warps)
   B_YFREE,              // Y role done reading YD_j, YO_j (4 Y warps)
-  B_ACCFREE,            // S role done reading ACC_j (4 S warps)
+  B_ACCFREE,            // S role done reading ACC_j (8 S warps)
   B_FAC0, B_FAC1,       // factors of a tile ready (factor warp)
-  B_FFREE0, B_FFREE1,   // factor buffer free again (14 consumer warps)
-  B_RS0, B_RS1,         // row scales of M_j written (4 M warps), buffer j & 1
+  B_FFREE0, B_FFREE1,   // factor buffer free again (20 consumer warps)
+  B_RS0, B_RS1,         // row scales of M_j written (8 M warps), buffer j & 1
   B_EH0, B_EH1,         // e_h of HH_j written (one S thread), buffer j & 1
   B_OPSF0, B_OPSF1,     // every MMA reading operand buffer j & 1 complete
+  B_XF0, B_XF1,         // YD of the tile in x buffer j & 1 complete
   B_FINAL,              // every MMA complete (end)
   kNumBars
 };
 // A wait for phase k of an mbarrier is only correct while phase k + 1 has not
 // completed (the parity would alias); every wait below is gated that way: the
 // barrier's next phase needs something the waiting role does after the wait.
-constexpr uint32_t kFacConsumers = 14;  // M 4 + Y 4 + S 4 + staging 2
+constexpr uint32_t kFacConsumers = 20;  // M 8 + Y 4 + S 8
 
 // Probes at most `limit` times, giving up early when another role aborted.
 __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity,
@@ -192,21 +198,23 @@ __global__ void __launch_bounds__(pipe::kPThreads, 1) ssd_pipe_kernel(const SsdP
     tc::mbar_init(&bars[B_ACC], 1);
     tc::mbar_init(&bars[B_YD], 1);
     tc::mbar_init(&bars[B_YO], 1);
-    tc::mbar_init(&bars[B_M], 4);
-    tc::mbar_init(&bars[B_STAGE], 2);
-    tc::mbar_init(&bars[B_HH], 4);
+    tc::mbar_init(&bars[B_M], 8);
+    tc::mbar_init(&bars[B_STAGE], 8);
+    tc::mbar_init(&bars[B_HH], 8);
     tc::mbar_init(&bars[B_YFREE], 4);
-    tc::mbar_init(&bars[B_ACCFREE], 4);
+    tc::mbar_init(&bars[B_ACCFREE], 8);
     tc::mbar_init(&bars[B_FAC0], 1);
     tc::mbar_init(&bars[B_FAC1], 1);
     tc::mbar_init(&bars[B_FFREE0], kFacConsumers);
     tc::mbar_init(&bars[B_FFREE1], kFacConsumers);
-    tc::mbar_init(&bars[B_RS0], 4);
-    tc::mbar_init(&bars[B_RS1], 4);
+    tc::mbar_init(&bars[B_RS0], 8);
+    tc::mbar_init(&bars[B_RS1], 8);
     tc::mbar_init(&bars[B_EH0], 1);
     tc::mbar_init(&bars[B_EH1], 1);
     tc::mbar_init(&bars[B_OPSF0], 1);
     tc::mbar_init(&bars[B_OPSF1], 1);
+    tc::mbar_init(&bars[B_XF0], 1);
+    tc::mbar_init(&bars[B_XF1], 1);
     tc::mbar_init(&bars[B_FINAL], 1);
   }
   __syncthreads();
@@ -233,11 +241,14 @@ __global__ void __launch_bounds__(pipe::kPThreads, 1) ssd_pipe_kernel(const SsdP
   __syncthreads();  // constants and the TMEM address published
   tc::fence_after();
 
-  if (warp < 4) {
+  if (warp < W_Y) {
     // =================================================================== M
-    const int q = warp, t = 32 * q + lane;
+    const int q = warp & 3, half = warp >> 2, t = 32 * q + lane;
     const uint32_t t_lane = (uint32_t)(32 * q) << 16;
-    {  // column blocks above the diagonal stay zero
+    // this warp's blocks [cb0, cb1) of the causal blocks 0 .. q
+    const int nb0 = (q + 2) >> 1;
+    const int cb0 = half ? nb0 : 0, cb1 = half ? q + 1 : nb0;
+    if (half == 0) {  // column blocks above the diagonal stay zero
       const uint32_t z[16] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
       for (int cb = q + 1; cb < 4; ++cb) tc::tmem_st16(tmem + t_lane + T_M + 16 * cb, z);
       tc::tmem_wait_st();
@@ -246,9 +257,8 @@ __global__ void __launch_bounds__(pipe::kPThreads, 1) ssd_pipe_kernel(const SsdP
       const int fb = j & 1;
       const float* FB = F + G_FB + fb * FB_SIZE;
       const bool ok = wait_bar(&bars[B_FAC0 + fb], (uint32_t)(j >> 1) & 1u, abort_v) &&
-                      wait_bar(&bars[B_CB], (uint32_t)j & 1u, abort_v) &&
-                      (j == 0 || wait_bar(&bars[B_YD], (uint32_t)(j - 1) & 1u, abort_v));
-      if (!__all_sync(0xffffffffu, ok)) {  // the warp leaves together (.sync.aligned loads)
+                      wait_bar(&bars[B_CB], (uint32_t)j & 1u, abort_v);
+      if (!named_and(4, 256, ok)) {  // the M warps leave together
         fail();
         break;
       }
@@ -298,14 +308,30 @@ __global__ void __launch_bounds__(pipe::kPThreads, 1) ssd_pipe_kernel(const SsdP
           }
         }
       };
-      // pass 0: the row maximum over the blocks; pass 1: the normalised
-      // binary16 values (one loop body for both, to keep the code small)
+      // pass 0: this warp's blocks' maximum, combined with the other warp of
+      // the quarter through shared memory; pass 1: the normalised binary16
+      // values (one loop body for both, to keep the code small)
       float rm = 0.0f;
       int et = 0;
+      bool stop = false;  // uniform over the M warps (a named-barrier result)
+      const int nbw = cb1 - cb0;
 #pragma unroll 1
-      for (int it = 0; it < 2 * (q + 1); ++it) {
-        const int pass = it > q, cb = pass ? it - q - 1 : it;
-        if (it == q + 1) et = norm_exp(rm);
+      for (int it = 0; it < 2 * nbw + 1; ++it) {
+        if (it == nbw) {
+          F[G_RMX + half * kQ + t] = rm;
+          tc::named_sync(4, 256);
+          rm = fmaxf(F[G_RMX + t], F[G_RMX + kQ + t]);
+          et = norm_exp(rm);
+          // M_{j-1} has been read by YD_{j-1} before M_j is written
+          const bool ok2 = j == 0 || wait_bar(&bars[B_YD], (uint32_t)(j - 1) & 1u, abort_v);
+          if (!named_and(4, 256, ok2)) {  // also: the maxima are read before they are rewritten
+            fail();
+            stop = true;
+            break;
+          }
+          continue;
+        }
+        const int pass = it > nbw, cb = cb0 + (pass ? it - nbw - 1 : it);
         float rt, mv[32];
         const int mode = block_mode(cb, rt);
         block_vals(cb, mode, mv);
@@ -322,7 +348,8 @@ __global__ void __launch_bounds__(pipe::kPThreads, 1) ssd_pipe_kernel(const SsdP
           tc::tmem_st16(tmem + t_lane + T_M + 16 * cb, o);
         }
       }
-      F[G_RS + fb * kQ + t] = pow2i(et);
+      if (stop) break;
+      if (half == 0) F[G_RS + fb * kQ + t] = pow2i(et);
       tc::tmem_wait_st();
       tc::fence_before();
       __syncwarp();
@@ -332,9 +359,9 @@ __global__ void __launch_bounds__(pipe::kPThreads, 1) ssd_pipe_kernel(const SsdP
         bar_arrive(&bars[B_FFREE0 + fb]);
       }
     }
-  } else if (warp < 8) {
+  } else if (warp < W_S) {
     // =================================================================== Y
-    const int q = warp - 4, t = 32 * q + lane;
+    const int q = warp - W_Y, t = 32 * q + lane;
     const uint32_t t_lane = (uint32_t)(32 * q) << 16;
     for (int j = 0; j < nt; ++j) {
       const int fb = j & 1;
@@ -370,7 +397,7 @@ __global__ void __launch_bounds__(pipe::kPThreads, 1) ssd_pipe_kernel(const SsdP
       const float rs = F[G_RS + fb * kQ + t];
       const int eh = reinterpret_cast<const int*>(F + G_EH)[fb];
       const float es = FB[FB_ES + t] * pow2i(eh);
-      uint8_t* yrow = smem + P_YS + t * (2 * kP);
+      uint16_t* ydst = p.y + row_off;
 #pragma unroll 1
       for (int qq = 0; qq < 4; ++qq) {  // columns 16 qq .. 16 qq + 15
         uint4 xn = make_uint4(0u, 0u, 0u, 0u), zn0 = xn, zn1 = xn;
@@ -401,11 +428,11 @@ __global__ void __launch_bounds__(pipe::kPThreads, 1) ssd_pipe_kernel(const SsdP
           }
           out[k] = pack_half2(r2[0], r2[1]);
         }
-        // swizzled 16-byte chunks (chunk c of row t at c ^ (t & 7))
-        *reinterpret_cast<uint4*>(yrow + 16 * ((2 * qq) ^ (t & 7))) =
-            make_uint4(out[0], out[1], out[2], out[3]);
-        *reinterpret_cast<uint4*>(yrow + 16 * ((2 * qq + 1) ^ (t & 7))) =
-            make_uint4(out[4], out[5], out[6], out[7]);
+        if (t < ql) {
+          uint4* yq = reinterpret_cast<uint4*>(ydst + 16 * qq);
+          yq[0] = make_uint4(out[0], out[1], out[2], out[3]);
+          yq[1] = make_uint4(out[4], out[5], out[6], out[7]);
+        }
         xq = xn;
         z0 = zn0;
         z1 = zn1;
@@ -416,73 +443,133 @@ __global__ void __launch_bounds__(pipe::kPThreads, 1) ssd_pipe_kernel(const SsdP
         bar_arrive(&bars[B_YFREE]);
         bar_arrive(&bars[B_FFREE0 + fb]);
       }
-      tc::named_sync(1, 128);  // the tile's y rows staged
-      // store: 128 threads, whole 128-byte row segments (8 threads per row)
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int k = 128 * i + 32 * q + lane, r = k >> 3, c = k & 7;
-        if (r < ql) {
-          const uint4 v = *reinterpret_cast<const uint4*>(smem + P_YS + r * (2 * kP) +
-                                                           16 * (c ^ (r & 7)));
-          *reinterpret_cast<uint4*>(p.y + ((bb * L + t0 + r) * H + hd) * kP + 8 * c) = v;
-        }
-      }
-      tc::named_sync(1, 128);  // staging buffer free for the next tile
     }
-  } else if (warp < 12) {
+  } else if (warp < W_FAC) {
     // =================================================================== S
-    const int q = warp - 8, n = 32 * q + lane;
+    const int sw = warp - W_S, q = sw & 3, half = sw >> 2, n = 32 * q + lane;
+    const int p0 = 32 * half;  // this thread's columns p0 .. p0 + 31
     const uint32_t t_lane = (uint32_t)(32 * q) << 16;
     const float hfac = F[G_HF + n];
     const float sbr = F[G_SB + n];
-    float hs[64];
+    float hs[32];
 #pragma unroll
-    for (int i = 0; i < 64; ++i)
-      hs[i] = (p.h0 && seg == 0) ? __ldg(p.h0 + u * kP * kN + (int64_t)i * kN + n) : 0.0f;
+    for (int i = 0; i < 32; ++i)
+      hs[i] = (p.h0 && seg == 0) ? __ldg(p.h0 + u * kP * kN + (int64_t)(p0 + i) * kN + n) : 0.0f;
+    // x operands of tile jj (exact into x buffer jj & 1, w x high / residual)
+    // from raw codes xr[2] (items st_tid, st_tid + 256: row s, p in [16 part,
+    // 16 part + 16)), with tile jj's per-step factors
+    const int st_tid = 32 * sw + lane;
+    auto load_x = [&](int jj, uint4 (&xr)[2]) {
+      const int64_t tt = t_beg + (int64_t)jj * kQ;
+      const int ql = (int)min((int64_t)kQ, t_end - tt);
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const int it = st_tid + 256 * i, s_ = it >> 2, part = it & 3;
+        xr[i] = s_ < ql ? __ldg(reinterpret_cast<const uint4*>(
+                              static_cast<const uint8_t*>(p.x) +
+                              ((bb * L + tt + s_) * H + hd) * kP + 16 * part))
+                        : make_uint4(0u, 0u, 0u, 0u);
+      }
+    };
+    auto stage_x = [&](int jj, const uint4 (&xr)[2]) {
+      const float* FBs = F + G_FB + (jj & 1) * FB_SIZE;
+      const int ex = norm_exp(FBs[FB_WM] * p.x_bound);
+      const float xsc = pow2i(-ex);
+      const uint32_t xb = P_X + (uint32_t)(jj & 1) * (kQ * kP * 2);
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const int it = st_tid + 256 * i, s_ = it >> 2, part = it & 3;
+        const float ws = FBs[FB_WX + s_] * xsc;
+#pragma unroll
+        for (int grp = 0; grp < 2; ++grp) {
+          const uint32_t w0 = grp ? xr[i].z : xr[i].x, w1 = grp ? xr[i].w : xr[i].y;
+          float xv[8];
+          uint32_t ox[4], oh[4], ol[4];
+          if (!kSE) {
+            const uint32_t x0 = w0 ^ 0x80808080u, x1 = w1 ^ 0x80808080u;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              xv[k] = s8_to_f32(x0, k);
+              xv[4 + k] = s8_to_f32(x1, k);
+            }
+            ox[0] = h2_bits(s8x2_to_h2(x0, 0, 1));
+            ox[1] = h2_bits(s8x2_to_h2(x0, 2, 3));
+            ox[2] = h2_bits(s8x2_to_h2(x1, 0, 1));
+            ox[3] = h2_bits(s8x2_to_h2(x1, 2, 3));
+          } else {
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              xv[k] = x_exact((w0 >> (8 * k)) & 0xFFu, kXF, p.se_shift);
+              xv[4 + k] = x_exact((w1 >> (8 * k)) & 0xFFu, kXF, p.se_shift);
+            }
+#pragma unroll
+            for (int k = 0; k < 4; ++k) ox[k] = pack_h2(xv[2 * k], xv[2 * k + 1]);
+          }
+#pragma unroll
+          for (int k = 0; k < 4; ++k) split_h2(ws * xv[2 * k], ws * xv[2 * k + 1], oh[k], ol[k]);
+          const uint32_t off = tc::mnmaj_off(16 * part + 8 * grp, s_, kP);
+          *reinterpret_cast<uint4*>(smem + xb + off) = make_uint4(ox[0], ox[1], ox[2], ox[3]);
+          *reinterpret_cast<uint4*>(smem + P_XH + off) = make_uint4(oh[0], oh[1], oh[2], oh[3]);
+          *reinterpret_cast<uint4*>(smem + P_XL + off) = make_uint4(ol[0], ol[1], ol[2], ol[3]);
+        }
+      }
+      tc::fence_async_smem();
+      __syncwarp();
+      if (lane == 0) bar_arrive(&bars[B_STAGE]);
+    };
     float s_tot = 0.0f;
     // exponent e_h of the state operand: the maximum of |h sC/w'| over the
     // whole state (the S warps), as ssd_kernel's state_max
     auto state_exp = [&]() {
       float hm = 0.0f;
 #pragma unroll
-      for (int i = 0; i < 64; ++i) hm = fmaxf(hm, fabsf(hs[i] * hfac));
+      for (int i = 0; i < 32; ++i) hm = fmaxf(hm, fabsf(hs[i] * hfac));
 #pragma unroll
       for (int o = 16; o >= 1; o >>= 1) hm = fmaxf(hm, __shfl_xor_sync(0xffffffffu, hm, o));
-      if (lane == 0) F[G_RED + 8 + q] = hm;
-      tc::named_sync(2, 128);
-      const float m = fmaxf(fmaxf(F[G_RED + 8], F[G_RED + 9]), fmaxf(F[G_RED + 10], F[G_RED + 11]));
-      tc::named_sync(2, 128);  // partials read before the next round writes them
+      if (lane == 0) F[G_RED + 8 + sw] = hm;
+      tc::named_sync(2, 256);
+      float m = F[G_RED + 8];
+#pragma unroll
+      for (int i = 1; i < 8; ++i) m = fmaxf(m, F[G_RED + 8 + i]);
+      tc::named_sync(2, 256);  // partials read before the next round writes them
       return norm_exp(m);
     };
     // HH = h sC_n / w'_n 2^-e_h, binary16, [n][p] MN-major
     auto stage_hh = [&](int eh) {
       const float f = hfac * pow2i(-eh);
 #pragma unroll
-      for (int grp = 0; grp < 8; ++grp) {
+      for (int grp = 0; grp < 4; ++grp) {
         uint32_t oh[4];
 #pragma unroll
         for (int k = 0; k < 4; ++k) oh[k] = pack_h2(hs[8 * grp + 2 * k] * f, hs[8 * grp + 2 * k + 1] * f);
-        *reinterpret_cast<uint4*>(smem + P_HH + tc::mnmaj_off(8 * grp, n, kP)) =
+        *reinterpret_cast<uint4*>(smem + P_HH + tc::mnmaj_off(p0 + 8 * grp, n, kP)) =
             make_uint4(oh[0], oh[1], oh[2], oh[3]);
       }
       tc::fence_async_smem();
       __syncwarp();
     };
-    {
+    uint4 xr[2];
+    load_x(0, xr);
+    bool started = named_and(2, 256, wait_bar(&bars[B_FAC0], 0u, abort_v));
+    if (started) {
+      stage_x(0, xr);
+      if (nt > 1) load_x(1, xr);
       const int eh = state_exp();
-      if (n == 0) {
+      if (n == 0 && half == 0) {
         reinterpret_cast<int*>(F + G_EH)[0] = eh;
         bar_arrive(&bars[B_EH0]);
       }
       stage_hh(eh);
       if (lane == 0) bar_arrive(&bars[B_HH]);
+    } else {
+      fail();
     }
-    for (int j = 0; j < nt; ++j) {
+    for (int j = 0; started && j < nt; ++j) {
       const int fb = j & 1;
       const float* FB = F + G_FB + fb * FB_SIZE;
       const bool ok = wait_bar(&bars[B_FAC0 + fb], (uint32_t)(j >> 1) & 1u, abort_v) &&
                       wait_bar(&bars[B_ACC], (uint32_t)j & 1u, abort_v);
-      if (!named_and(2, 128, ok)) {
+      if (!named_and(2, 256, ok)) {
         fail();
         break;
       }
@@ -492,12 +579,12 @@ __global__ void __launch_bounds__(pipe::kPThreads, 1) ssd_pipe_kernel(const SsdP
       const float decay = ex2_sfu(s_last);
       const float f = sbr * pow2i(ex);
 #pragma unroll
-      for (int qq = 0; qq < 4; ++qq) {
+      for (int qq = 0; qq < 2; ++qq) {
         float acc[16];
-        tc::tmem_ld16(tmem + t_lane + T_ACC + 16 * qq, acc);
+        tc::tmem_ld16(tmem + t_lane + T_ACC + p0 + 16 * qq, acc);
 #pragma unroll
         for (int i4 = 0; i4 < 4; ++i4) {
-          const float4 sx4 = *reinterpret_cast<const float4*>(F + G_SX + 16 * qq + 4 * i4);
+          const float4 sx4 = *reinterpret_cast<const float4*>(F + G_SX + p0 + 16 * qq + 4 * i4);
           const float sx[4] = {sx4.x, sx4.y, sx4.z, sx4.w};
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
@@ -506,7 +593,7 @@ __global__ void __launch_bounds__(pipe::kPThreads, 1) ssd_pipe_kernel(const SsdP
           }
         }
       }
-      if (n == 0) s_tot += s_last;
+      if (n == 0 && half == 0) s_tot += s_last;
       tc::fence_before();
       __syncwarp();
       if (lane == 0) {
@@ -514,13 +601,24 @@ __global__ void __launch_bounds__(pipe::kPThreads, 1) ssd_pipe_kernel(const SsdP
         bar_arrive(&bars[B_FFREE0 + fb]);
       }
       if (j + 1 < nt) {
-        const int eh = state_exp();
-        const bool ok2 = wait_bar(&bars[B_YO], (uint32_t)j & 1u, abort_v);  // HH_j read by YO_j
-        if (!named_and(2, 128, ok2)) {
+        // x operands of tile j + 1: its factors, and x buffer (j + 1) & 1 read
+        // by YD_{j-1} (w x was read by ACC_j, complete)
+        const bool ok1 = wait_bar(&bars[B_FAC0 + (fb ^ 1)], (uint32_t)((j + 1) >> 1) & 1u, abort_v) &&
+                         (j < 1 || wait_bar(&bars[B_XF0 + (fb ^ 1)], (uint32_t)((j - 1) >> 1) & 1u,
+                                            abort_v));
+        if (!named_and(2, 256, ok1)) {
           fail();
           break;
         }
-        if (n == 0) {
+        stage_x(j + 1, xr);
+        if (j + 2 < nt) load_x(j + 2, xr);
+        const int eh = state_exp();
+        const bool ok2 = wait_bar(&bars[B_YO], (uint32_t)j & 1u, abort_v);  // HH_j read by YO_j
+        if (!named_and(2, 256, ok2)) {
+          fail();
+          break;
+        }
+        if (n == 0 && half == 0) {
           reinterpret_cast<int*>(F + G_EH)[(j + 1) & 1] = eh;
           bar_arrive(&bars[B_EH0 + ((j + 1) & 1)]);
         }
@@ -533,17 +631,17 @@ __global__ void __launch_bounds__(pipe::kPThreads, 1) ssd_pipe_kernel(const SsdP
     if (!wait_bar(&bars[B_FINAL], 0u, abort_v)) fail();
     float* fin = slot < 0 ? (p.h_final ? p.h_final + u * kP * kN : nullptr)
                           : p.seg_state + (int64_t)slot * kP * kN;
-    if (slot >= 0 && n == 0) p.seg_dec[slot] = s_tot;
-    if (slot < 0 && n == 0 && p.dec_final) p.dec_final[u] = s_tot;
+    if (slot >= 0 && n == 0 && half == 0) p.seg_dec[slot] = s_tot;
+    if (slot < 0 && n == 0 && half == 0 && p.dec_final) p.dec_final[u] = s_tot;
     if (fin) {
       float* stage = reinterpret_cast<float*>(smem + P_XH);
 #pragma unroll
-      for (int i = 0; i < 64; ++i) stage[i * kN + n] = hs[i];
-      tc::named_sync(2, 128);
+      for (int i = 0; i < 32; ++i) stage[(p0 + i) * kN + n] = hs[i];
+      tc::named_sync(2, 256);
       float4* dst = reinterpret_cast<float4*>(fin);
-      for (int i = 32 * q + lane; i < kP * kN / 4; i += 128) dst[i] = reinterpret_cast<float4*>(stage)[i];
+      for (int i = 32 * sw + lane; i < kP * kN / 4; i += 256) dst[i] = reinterpret_cast<float4*>(stage)[i];
     }
-  } else if (warp == 12) {
+  } else if (warp == W_FAC) {
     // =========================================================== factors
     uint16_t dtr[4] = {0, 0, 0, 0};
     auto load_dt = [&](int j) {
@@ -635,87 +733,6 @@ __global__ void __launch_bounds__(pipe::kPThreads, 1) ssd_pipe_kernel(const SsdP
       for (int j = max(0, ops_issued - 2); j < ops_issued; ++j)
         if (!tc::mbar_wait(&bars[B_OPS0 + (j & 1)], (uint32_t)(j >> 1) & 1u, kWaitLimit))
           flags |= SSMQ_DEV_TIMEOUT;
-  } else if (warp < 15) {
-    // ============================================================ staging
-    const int sw = warp - 13, st_tid = 32 * sw + lane;  // 64 threads
-    // cp.async the raw x codes of tile j into RX (rows at or beyond the end
-    // are not fetched; the staging zeroes them)
-    auto fetch = [&](int j) {
-      const int64_t tt = t_beg + (int64_t)j * kQ;
-      const int ql = (int)min((int64_t)kQ, t_end - tt);
-      for (int w = st_tid; w < kQ * (kP / 16); w += 64) {
-        const int r = w >> 2, c = w & 3;
-        if (r >= ql) continue;
-        const int64_t xo = ((bb * L + tt + r) * H + hd) * kP + 16 * c;
-        tc::cp_async16(smem + P_RX + r * kP + 16 * (c ^ (r & 3)),
-                       static_cast<const uint8_t*>(p.x) + xo);
-      }
-      tc::cp_async_commit();
-    };
-    fetch(0);
-    for (int j = 0; j < nt; ++j) {
-      const int fb = j & 1;
-      const float* FB = F + G_FB + fb * FB_SIZE;
-      const int ql = (int)min((int64_t)kQ, t_end - t_beg - (int64_t)j * kQ);
-      const bool ok = wait_bar(&bars[B_FAC0 + fb], (uint32_t)(j >> 1) & 1u, abort_v) &&
-                      (j == 0 || wait_bar(&bars[B_YD], (uint32_t)(j - 1) & 1u, abort_v));
-      tc::cp_async_wait_all();
-      if (!named_and(3, 64, ok)) {  // also: the raw rows of tile j landed (both warps' copies)
-        fail();
-        break;
-      }
-      const int ex = norm_exp(FB[FB_WM] * p.x_bound);
-      const float xsc = pow2i(-ex);
-      // item (s, part): row s, p in [16 part, 16 part + 16): 512 items
-      for (int it = st_tid; it < kQ * 4; it += 64) {
-        const int s = it >> 2, part = it & 3;
-        const bool ok = s < ql;
-        const uint4 xq = ok ? *reinterpret_cast<const uint4*>(smem + P_RX + s * kP +
-                                                              16 * (part ^ (s & 3)))
-                            : make_uint4(0, 0, 0, 0);
-        const float ws = FB[FB_WX + s] * xsc;
-#pragma unroll
-        for (int grp = 0; grp < 2; ++grp) {
-          const uint32_t w0 = grp ? xq.z : xq.x, w1 = grp ? xq.w : xq.y;
-          float xv[8];
-          uint32_t ox[4], oh[4], ol[4];
-          if (!kSE) {
-            const uint32_t x0 = w0 ^ 0x80808080u, x1 = w1 ^ 0x80808080u;
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              xv[k] = s8_to_f32(x0, k);
-              xv[4 + k] = s8_to_f32(x1, k);
-            }
-            ox[0] = h2_bits(s8x2_to_h2(x0, 0, 1));
-            ox[1] = h2_bits(s8x2_to_h2(x0, 2, 3));
-            ox[2] = h2_bits(s8x2_to_h2(x1, 0, 1));
-            ox[3] = h2_bits(s8x2_to_h2(x1, 2, 3));
-          } else {
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              xv[k] = x_exact((w0 >> (8 * k)) & 0xFFu, kXF, p.se_shift);
-              xv[4 + k] = x_exact((w1 >> (8 * k)) & 0xFFu, kXF, p.se_shift);
-            }
-#pragma unroll
-            for (int k = 0; k < 4; ++k) ox[k] = pack_h2(xv[2 * k], xv[2 * k + 1]);
-          }
-#pragma unroll
-          for (int k = 0; k < 4; ++k) split_h2(ws * xv[2 * k], ws * xv[2 * k + 1], oh[k], ol[k]);
-          const uint32_t off = tc::mnmaj_off(16 * part + 8 * grp, s, kP);
-          *reinterpret_cast<uint4*>(smem + P_X + off) = make_uint4(ox[0], ox[1], ox[2], ox[3]);
-          *reinterpret_cast<uint4*>(smem + P_XH + off) = make_uint4(oh[0], oh[1], oh[2], oh[3]);
-          *reinterpret_cast<uint4*>(smem + P_XL + off) = make_uint4(ol[0], ol[1], ol[2], ol[3]);
-        }
-      }
-      tc::fence_async_smem();
-      tc::named_sync(3, 64);  // operands staged, raw rows consumed
-      if (lane == 0) {
-        bar_arrive(&bars[B_STAGE]);
-        bar_arrive(&bars[B_FFREE0 + fb]);
-      }
-      if (j + 1 < nt) fetch(j + 1);
-    }
-    tc::cp_async_wait_all();  // no copy lands after the CTA has exited
   } else {
     // ================================================================ MMA
     if (lane == 0) {
@@ -734,6 +751,20 @@ __global__ void __launch_bounds__(pipe::kPThreads, 1) ssd_pipe_kernel(const SsdP
       }
       for (int j = 0; ok && j < nt; ++j) {
         const uint32_t cbuf = s_base + P_OPS + (uint32_t)(j & 1) * kOpTile;
+        // CB_{j+1}, as soon as M_j has read CB_j
+        ok = wait_bar(&bars[B_M], (uint32_t)j & 1u, abort_v);
+        if (!ok) break;
+        if (j + 1 < nt) {
+          ok = wait_bar(&bars[B_OPS0 + ((j + 1) & 1)], (uint32_t)((j + 1) >> 1) & 1u, abort_v);
+          if (!ok) break;
+          tc::fence_after();
+          const uint32_t nb = s_base + P_OPS + (uint32_t)((j + 1) & 1) * kOpTile;
+#pragma unroll
+          for (int k0 = 0; k0 < kN; k0 += 16)
+            tc::mma_f16(tmem + T_CB, tc::kmaj_desc(nb, k0, kN),
+                        tc::kmaj_desc(nb + kOpBlock, k0, kN), id_cb, k0 > 0);
+          tc::mma_commit(&bars[B_CB]);
+        }
         // ACC_j = B_j^T (w X)_j, high and residual parts
         ok = wait_bar(&bars[B_STAGE], (uint32_t)j & 1u, abort_v) &&
              (j == 0 || wait_bar(&bars[B_ACCFREE], (uint32_t)(j - 1) & 1u, abort_v));
@@ -749,15 +780,16 @@ __global__ void __launch_bounds__(pipe::kPThreads, 1) ssd_pipe_kernel(const SsdP
                       tc::mnmaj_desc(s_base + P_XL, k0, kP), id_s, 1u);
         tc::mma_commit(&bars[B_ACC]);
         // YD_j = M_j X_j
-        ok = wait_bar(&bars[B_M], (uint32_t)j & 1u, abort_v) &&
-             (j == 0 || wait_bar(&bars[B_YFREE], (uint32_t)(j - 1) & 1u, abort_v));
+        ok = j == 0 || wait_bar(&bars[B_YFREE], (uint32_t)(j - 1) & 1u, abort_v);
         if (!ok) break;
         tc::fence_after();
+        const uint32_t xbuf = s_base + P_X + (uint32_t)(j & 1) * (kQ * kP * 2);
 #pragma unroll
         for (int k0 = 0; k0 < kQ; k0 += 16)
-          tc::mma_f16_ts(tmem + T_YD, tmem + T_M + k0 / 2, tc::mnmaj_desc(s_base + P_X, k0, kP),
-                         id_y, k0 > 0);
+          tc::mma_f16_ts(tmem + T_YD, tmem + T_M + k0 / 2, tc::mnmaj_desc(xbuf, k0, kP), id_y,
+                         k0 > 0);
         tc::mma_commit(&bars[B_YD]);
+        tc::mma_commit(&bars[B_XF0 + (j & 1)]);  // x buffer j & 1 read completely
         // YO_j = C'_j HH_j
         ok = wait_bar(&bars[B_HH], (uint32_t)j & 1u, abort_v);
         if (!ok) break;
@@ -768,18 +800,6 @@ __global__ void __launch_bounds__(pipe::kPThreads, 1) ssd_pipe_kernel(const SsdP
                       tc::mnmaj_desc(s_base + P_HH, k0, kP), id_y, k0 > 0);
         tc::mma_commit(&bars[B_YO]);
         tc::mma_commit(&bars[B_OPSF0 + (j & 1)]);  // operand buffer j & 1 read completely
-        // CB_{j+1} (M_j has read CB_j: the wait on B_M above)
-        if (j + 1 < nt) {
-          ok = wait_bar(&bars[B_OPS0 + ((j + 1) & 1)], (uint32_t)((j + 1) >> 1) & 1u, abort_v);
-          if (!ok) break;
-          tc::fence_after();
-          const uint32_t nb = s_base + P_OPS + (uint32_t)((j + 1) & 1) * kOpTile;
-#pragma unroll
-          for (int k0 = 0; k0 < kN; k0 += 16)
-            tc::mma_f16(tmem + T_CB, tc::kmaj_desc(nb, k0, kN),
-                        tc::kmaj_desc(nb + kOpBlock, k0, kN), id_cb, k0 > 0);
-          tc::mma_commit(&bars[B_CB]);
-        }
       }
       if (!ok) fail();
       // every MMA issued is complete before TMEM is freed (and before the S

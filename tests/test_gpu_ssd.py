@@ -310,9 +310,9 @@ def test_state_chain_and_carry_in_edge_cases():
 
 
 # ---- the pipelined kernel against the single-schedule kernel ---------------
-# The binary16-y path runs a kernel whose warp roles work on different tiles
-# at once; it keeps the other kernel's arithmetic operation for operation, so
-# the two give the same bits (SSMQ_SSD_KERNEL=classic selects the other one).
+# SSMQ_SSD_KERNEL=pipelined selects, for binary16 y, a kernel whose warp roles
+# work on different tiles at once; it keeps the default kernel's arithmetic
+# operation for operation, so the two give the same bits.
 
 PIPE_CASES = [
     # (b, L, H, G, gs, gate, h0, bias, fmt, dt_mean, max_segments)
@@ -335,8 +335,9 @@ def test_ssd_pipelined_equals_single_schedule(ci, monkeypatch):
     dec_a = torch.zeros((b, Hh), dtype=torch.float32, device=dev())
     dec_b = torch.zeros((b, Hh), dtype=torch.float32, device=dev())
     st_a, st_b = status_word(), status_word()
+    monkeypatch.setenv("SSMQ_SSD_KERNEL", "pipelined")
     ya, ha = gpu_ssd(p, max_segments=ms, dec_final=dec_a, status=st_a)
-    monkeypatch.setenv("SSMQ_SSD_KERNEL", "classic")
+    monkeypatch.delenv("SSMQ_SSD_KERNEL")
     yb, hb = gpu_ssd(p, max_segments=ms, dec_final=dec_b, status=st_b)
     torch.cuda.synchronize()
     assert int(H(st_a)[0]) == 0 and int(H(st_b)[0]) == 0
