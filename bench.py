@@ -443,6 +443,14 @@ def run_ours(args):
                          "scan_ms_per_launch": round(scan_avg_s * 1e3, 5),
                          "peaks_source": pk["source"]},
             "step_hbm_gbs": round(layer.step_bytes() / (ms_step / 1e3) / 1e9, 1),
+            "quantize_leg": {"kernel": "quant_batch_kernel (x, B, C in one launch)",
+                             "algorithmic_bytes_per_launch": layer.step_bytes() - layer.scan_bytes(),
+                             "ms_per_launch": round(ms_step - scan_avg_s * 1e3, 5),
+                             "hbm_frac": round((layer.step_bytes() - layer.scan_bytes()) /
+                                               ((ms_step - scan_avg_s * 1e3) / 1e3) / 1e9 /
+                                               pk["hbm_gbs"], 4),
+                             "traffic": measured_traffic("quant_batch_kernel"),
+                             "note": "time = step minus the scan's CUDA-event time"},
             "clocks": clocks,
         }
     if world > 1:
@@ -871,7 +879,9 @@ def form_softedge(torch, dev, pk, mhz, ex2=None):
                            "scan_ms": round(t_fused * 1e3, 4)},
             "encode": {"ms": round(t_enc * 1e3, 4), "bound": "hbm",
                        "achieved": round(enc_bytes / t_enc / 1e9, 1), "peak": pk["hbm_gbs"],
-                       "unit": "GB/s", "frac": round(enc_bytes / t_enc / 1e9 / pk["hbm_gbs"], 4)},
+                       "unit": "GB/s", "frac": round(enc_bytes / t_enc / 1e9 / pk["hbm_gbs"], 4),
+                       "kernel": "se_encode_lut_kernel", "algorithmic_bytes_per_launch": enc_bytes,
+                       "traffic": measured_traffic("se_encode_lut_kernel")},
             "scan": {"ms": round(t_scan * 1e3, 4), "bound": "alu",
                      "achieved": round(upd / t_scan / 1e9, 1), "peak": round(peak_upd, 1),
                      "unit": "Gupdates/s", "frac": round(upd / t_scan / 1e9 / peak_upd, 4)}}
@@ -1119,7 +1129,8 @@ def form_conv(torch, dev, pk, layer):
             "roofline": {"bound": "hbm", "achieved": round(byts / t / 1e9, 1),
                          "peak": pk["hbm_gbs"], "unit": "GB/s",
                          "frac": round(byts / t / 1e9 / pk["hbm_gbs"], 4),
-                         "algorithmic_bytes_per_launch": byts}}
+                         "algorithmic_bytes_per_launch": byts,
+                         "traffic": measured_traffic("conv_vec_kernel")}}
 
 
 def run_forms(dev, pk, mhz, only=None, layer=None, ex2=None):
@@ -1213,15 +1224,16 @@ def run_kernel(args):
         fn = (lambda: api.conv_silu_quantize(lay.x, w, bias=bs, x_group=lay.grp,
                                              x_scale=lay.xs, codes=lay.xq))
         label = "m130m conv input: causal conv + SiLU + int8 group codes"
-    elif name in ("scan", "scan-int8", "quantize"):
+    elif name in ("scan", "scan-int8", "quantize", "quantize-batch"):
         lay = Layer(dev, 0, fused=name == "scan")
         lay.quantize()
-        fn = lay.scan if name != "quantize" else (
-            lambda: api.quantize_groups(lay.x, lay.b, lay.d, lay.L, lay.grp, lay.k,
-                                        scales=lay.xs, out=lay.xq))
+        fn = {"scan": lay.scan, "scan-int8": lay.scan, "quantize-batch": lay.quantize,
+              "quantize": (lambda: api.quantize_groups(lay.x, lay.b, lay.d, lay.L, lay.grp, lay.k,
+                                                       scales=lay.xs, out=lay.xq))}[name]
         label = "m130m " + {"scan": "selective scan, binary16 x encoded in the scan",
                             "scan-int8": "selective scan of int8 x codes",
-                            "quantize": "x quantize (static scales)"}[name]
+                            "quantize": "x quantize (static scales)",
+                            "quantize-batch": "x, B, C quantize in one launch"}[name]
     elif name == "ssd":
         c = setup_ssd(torch, dev)
         c["quant"]()
@@ -1263,8 +1275,9 @@ def main():
     ap.add_argument("--fused", action="store_true",
                     help="headline step with binary16 x encoded inside the scan (byte-identical "
                          "result; default: x quantized by its own launch, the faster path here)")
-    ap.add_argument("--kernel", choices=["scan", "scan-int8", "quantize", "ssd", "encode",
-                                         "softedge-scan", "decode", "ex2", "conv"],
+    ap.add_argument("--kernel", choices=["scan", "scan-int8", "quantize", "quantize-batch",
+                                         "ssd", "encode", "softedge-scan", "decode", "ex2",
+                                         "conv"],
                     help="profiling aid: run only this kernel on its workload")
     args = ap.parse_args()
     if args.kernel:

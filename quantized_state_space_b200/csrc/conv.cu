@@ -22,8 +22,8 @@
 // Layout (b, d, L), channel rows contiguous in time.  A thread takes 16
 // consecutive steps of one row (two 16-byte loads) plus the 3 inputs before
 // them (one 8-byte load, an L1/L2 hit: they belong to the neighbouring
-// thread's vector) and keeps the next vector's loads in flight while it
-// computes.  The conv taps and the exponential run as packed fp32x2
+// thread's vector); four CTAs of eight warps per SM hide the load latency.
+// The conv taps and the exponential run as packed fp32x2
 // operations (each lane a correctly rounded fma / add / multiply, so the
 // packing changes no bit); the IEEE reciprocal is per element.  Vectors with
 // an |a| above 87 (or a NaN) take the scalar route, which handles the range
@@ -181,7 +181,7 @@ struct Raw16 {
 
 // Vector path: rows of L % 16 == 0 steps; vector v covers steps 16 (v % (L /
 // 16)) .. + 15 of row v / (L / 16).
-__global__ void __launch_bounds__(kConvThreads) conv_vec_kernel(const ConvParams p) {
+__global__ void __launch_bounds__(kConvThreads, kConvCtasPerSm) conv_vec_kernel(const ConvParams p) {
   const int64_t vpr = p.L / 16;  // vectors per row
   const int64_t nvec = p.b * p.d * vpr;
   const int64_t stride = (int64_t)gridDim.x * kConvThreads;
@@ -207,12 +207,9 @@ __global__ void __launch_bounds__(kConvThreads) conv_vec_kernel(const ConvParams
     }
   };
 
-  int64_t v = (int64_t)blockIdx.x * kConvThreads + threadIdx.x;
-  Raw16 cur;
-  if (v < nvec) load(v, cur);
-  for (; v < nvec; v += stride) {
-    Raw16 nxt;
-    if (v + stride < nvec) load(v + stride, nxt);  // in flight while this one computes
+  for (int64_t v = (int64_t)blockIdx.x * kConvThreads + threadIdx.x; v < nvec; v += stride) {
+    Raw16 cur;
+    load(v, cur);
     const int64_t row = v / vpr, t0 = (v % vpr) * 16;
     const int64_t c = row % p.d;
     // xs[0..19]: steps t0 - 4 .. t0 + 15 (wd: the same as binary16 pairs)
@@ -294,7 +291,6 @@ __global__ void __launch_bounds__(kConvThreads) conv_vec_kernel(const ConvParams
       for (int i = 17; i < 20; ++i)  // slot j = i - (20 - S) for i >= 20 - S
         if (i >= 20 - S) p.x_prev_out[row * S + i - (20 - S)] = (uint16_t)(wd[i / 2] >> (16 * (i & 1)));
     }
-    cur = nxt;
   }
   flag_status(p.status, flags);
 }
