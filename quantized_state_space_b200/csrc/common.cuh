@@ -140,14 +140,21 @@ __device__ __forceinline__ void se_split(uint32_t c, int& q, int& mode) {
 
 // Step sizes of the three soft-edge modes: {scale, scale / 2^r, scale * 2^r},
 // each one binary32 product.
-// rs[] are the correctly rounded reciprocals of s[] when s[] is a normal
-// number with a finite reciprocal, else 0 (which selects the exact division).
+// rs[] are the correctly rounded reciprocals of s[] when s[] is at least
+// 2^-100 with a normal reciprocal, else 0 (which selects the exact division).
+// fm[] are the quotient multipliers of the modes, {1, 2^r, 2^-r}: whenever
+// rs[] are all usable, s[1] = s[0] / 2^r and s[2] = s[0] 2^r exactly, so
+// fl32(v / s[m]) = fl32(v / s[0]) fm[m] up to underflow of tiny quotients.
 struct SeSteps {
   float s[3];
   float rs[3];
+  float fm[3];
 };
+// The bound 2^-100 keeps the residual of the packed routes' division
+// correction (quant_fast.cuh) exact: for a quotient of magnitude at least
+// 1/4 the residual is a multiple of 2^-149.
 __host__ __device__ inline bool usable_recip(float s, float r) {
-  return s >= 1.17549435e-38f && r > 0.0f && r <= 3.40282347e+38f && r >= 1.17549435e-38f;
+  return s >= 0x1p-100f && r > 0.0f && r <= 3.40282347e+38f && r >= 1.17549435e-38f;
 }
 __host__ inline SeSteps se_steps(float scale, int log2_ratio) {
   SeSteps st;
@@ -155,6 +162,9 @@ __host__ inline SeSteps se_steps(float scale, int log2_ratio) {
   st.s[0] = scale;
   st.s[1] = scale * (1.0f / f);
   st.s[2] = scale * f;
+  st.fm[0] = 1.0f;
+  st.fm[1] = f;
+  st.fm[2] = 1.0f / f;
   for (int i = 0; i < 3; ++i) {
     const float r = 1.0f / st.s[i];
     st.rs[i] = usable_recip(st.s[i], r) ? r : 0.0f;

@@ -136,7 +136,7 @@ __device__ __forceinline__ uint4 encode16(const ConvParams& p, const float (&u)[
                                           float rs, bool okg, uint32_t& flags) {
   uint4 o;
   if (p.fmt == SSMQ_X_INT8_GROUP) {
-    if (okg && rs != 0.0f && quant16_fast(u, rs, rs, o)) return o;
+    if (okg && rs != 0.0f && quant16_fast(u, make_float2(s, rs), make_float2(s, rs), o)) return o;
     int r[kQVec];
 #pragma unroll
     for (int i = 0; i < kQVec; ++i) r[i] = quant_elem(u[i], s, rs, okg, flags);

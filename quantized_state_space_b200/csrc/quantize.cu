@@ -121,7 +121,7 @@ __device__ __forceinline__ void quant_vec(const float (&x)[kVec], Idx e0, const 
     const float2 sa = tab_get(tab, scales, gu, n_groups);
     const float2 sb = gv == gu ? sa : tab_get(tab, scales, gv, n_groups);
     uint4 o;
-    if (sa.y != 0.0f && sb.y != 0.0f && quant16_fast(x, sa.y, sb.y, o)) {
+    if (sa.y != 0.0f && sb.y != 0.0f && quant16_fast(x, sa, sb, o)) {
       *reinterpret_cast<uint4*>(q + e0) = o;
       return;
     }
