@@ -112,12 +112,25 @@ struct Raw {
   int8_t C[kN][kT];
 };
 
-template <int kN, int kCH, typename XT>
+// Rows of per-lane partial sums kept in shared memory: the binary16 x with
+// group codes combines the channel's lanes in its store phase (measured
+// faster there: 0.257 against 0.274 ms on the Mamba-130M layer); the other
+// formats reduce with shuffles, which keeps their shared memory (and the
+// number of resident CTAs of large grids) as it was.
+__host__ __device__ constexpr int part_rows(int xfmt, int lpc) {
+  return xfmt == SSMQ_X_F16_GROUP ? lpc : 1;
+}
+
+template <int kN, int kCH, int kPR, typename XT>
 struct M1Smem {
   Raw<kN, kCH, XT> raw[kRawBufs];
   __align__(16) float2 dd[kCH][kT + 2];   // (delta, delta x) of the chunk being scanned
   __align__(16) float bc[2][2][kT][kN];   // [buffer][B, C][t][n], dequantised
-  __align__(16) float y[kCH][kSeg + 4];   // C . h of the current segment
+  // C . h of the current segment's steps: kPR = 1 row of sums (lanes
+  // combined by shuffles), or kPR = LPC rows of each lane's partial sums over
+  // its states (combined by the store phase); row stride kSeg + 4 keeps the
+  // 16-byte stores and loads of a warp free of bank conflicts
+  __align__(16) float part[kCH][kPR][kSeg + 4];
   float scale[2][kN];                     // B, C scale of each state
 };
 
@@ -202,8 +215,10 @@ __global__ void __launch_bounds__(kCH*(kN / kSPL)) m1_scan_kernel(const M1Params
   constexpr int NT = kCH * LPC;
   constexpr int SPS = kSeg / LPC;   // steps per lane per segment (stores, staging)
   static_assert(LPC >= 1 && LPC <= 16 && kSeg % LPC == 0, "lanes per channel");
+  // how the LPC lanes of a channel combine their partial C . h
+  constexpr int PR = part_rows(kXFmt, LPC);
   extern __shared__ __align__(16) uint8_t smem_bytes[];
-  M1Smem<kN, kCH, XT>& S = *reinterpret_cast<M1Smem<kN, kCH, XT>*>(smem_bytes);
+  M1Smem<kN, kCH, PR, XT>& S = *reinterpret_cast<M1Smem<kN, kCH, PR, XT>*>(smem_bytes);
 
   const int tid = threadIdx.x;
   const int64_t bb = blockIdx.y;
@@ -362,10 +377,19 @@ __global__ void __launch_bounds__(kCH*(kN / kSPL)) m1_scan_kernel(const M1Params
     uint32_t xw[(XB + 3) / 4], zw[(2 * SPS + 3) / 4];
     lds_words<XB>(&r.x[lc][tb], xw);
     if (p.z) lds_words<2 * SPS>(&r.z[lc][tb], zw);
+    // C . h of these steps (the sum of the channel's PR rows)
+    float ch[SPS];
+#pragma unroll
+    for (int l = 0; l < PR; ++l) {
+      uint32_t o[SPS];
+      lds_words<4 * SPS>(&S.part[lc][l][lj * SPS], o);
+#pragma unroll
+      for (int i = 0; i < SPS; ++i) ch[i] = l ? ch[i] + __uint_as_float(o[i]) : __uint_as_float(o[i]);
+    }
     float yv[SPS];
 #pragma unroll
     for (int i = 0; i < SPS; ++i) {
-      float v = fmaf(Dc, x_value(xw, i), S.y[lc][lj * SPS + i]);
+      float v = fmaf(Dc, x_value(xw, i), ch[i]);
       if (p.z) v *= silu_f(h2f((uint16_t)(zw[i >> 1] >> (16 * (i & 1)))));
       yv[i] = v;
     }
@@ -465,11 +489,13 @@ __global__ void __launch_bounds__(kCH*(kN / kSPL)) m1_scan_kernel(const M1Params
 
 #pragma unroll
     for (int s = 0; s < kSegs; ++s) {
-      // ---- scan segment s: kSeg / LPC groups of LPC steps; after each group
-      // lane lj holds y of step (group start + lj)
+      // ---- scan segment s: kSeg / LPC groups of LPC steps; each lane's
+      // partial C . h of every step goes to the store phase, combined over the
+      // channel's lanes by a shuffle reduce-scatter after each group (PR = 1)
+      // or through shared memory (PR = LPC)
+      float part[kSeg];
 #pragma unroll
       for (int tg = 0; tg < kSeg / LPC; ++tg) {
-        float part[LPC];
 #pragma unroll
         for (int kk = 0; kk < LPC; ++kk) {
           const int t = s * kSeg + tg * LPC + kk;
@@ -495,10 +521,17 @@ __global__ void __launch_bounds__(kCH*(kN / kSPL)) m1_scan_kernel(const M1Params
             hp[i] = ffma2(e, hp[i], fmul2(dxv, bq[i]));
             q = i == 0 ? fmul2(cq[i], hp[i]) : ffma2(cq[i], hp[i], q);
           }
-          part[kk] = q.x + q.y;
+          part[tg * LPC + kk] = q.x + q.y;
         }
-        S.y[lc][tg * LPC + lj] = reduce_scatter<LPC>(part, lj);
+        if constexpr (PR == 1)
+          S.part[lc][0][tg * LPC + lj] =
+              reduce_scatter<LPC>(*reinterpret_cast<float(*)[LPC]>(&part[tg * LPC]), lj);
       }
+      if constexpr (PR > 1)
+#pragma unroll
+        for (int i = 0; i < kSeg / 4; ++i)
+          reinterpret_cast<float4*>(&S.part[lc][lj][0])[i] =
+              make_float4(part[4 * i], part[4 * i + 1], part[4 * i + 2], part[4 * i + 3]);
       __syncwarp();
       store_seg(rcur, s, t0, tl);
       if (has_next) {
@@ -525,7 +558,11 @@ cudaError_t launch_m1(const M1Params& prm, int xfmt, int64_t batch, cudaStream_t
   const dim3 grid((unsigned)(p.n_ctile * p.G), (unsigned)batch);
   const dim3 block(kCH * (kN / kSPL));
   const bool f16 = xfmt == SSMQ_X_F16_GROUP || xfmt == SSMQ_X_F16_SOFTEDGE;
-  const size_t smem = f16 ? sizeof(M1Smem<kN, kCH, uint16_t>) : sizeof(M1Smem<kN, kCH, uint8_t>);
+  constexpr int LPC = kN / kSPL;
+  const size_t smem =
+      xfmt == SSMQ_X_F16_GROUP
+          ? sizeof(M1Smem<kN, kCH, part_rows(SSMQ_X_F16_GROUP, LPC), uint16_t>)
+          : (f16 ? sizeof(M1Smem<kN, kCH, 1, uint16_t>) : sizeof(M1Smem<kN, kCH, 1, uint8_t>));
   auto pick = [&](auto yq) {
     constexpr bool Q = decltype(yq)::value;
     return xfmt == SSMQ_X_SOFTEDGE       ? m1_scan_kernel<kN, kCH, kSPL, SSMQ_X_SOFTEDGE, Q>
