@@ -377,19 +377,32 @@ __global__ void __launch_bounds__(kCH*(kN / kSPL)) m1_scan_kernel(const M1Params
     uint32_t xw[(XB + 3) / 4], zw[(2 * SPS + 3) / 4];
     lds_words<XB>(&r.x[lc][tb], xw);
     if (p.z) lds_words<2 * SPS>(&r.z[lc][tb], zw);
-    // C . h of these steps (the sum of the channel's PR rows)
-    float ch[SPS];
+    // C . h of these steps: the channel's PR rows summed in the order of the
+    // shuffle reduce-scatter (pairs l, l + PR / 2 first, then halving the
+    // stride), so both forms give the same bits
+    float ch[PR > 1 ? SPS : 1];
+    if constexpr (PR > 1) {
+      uint32_t o[PR][SPS];
 #pragma unroll
-    for (int l = 0; l < PR; ++l) {
-      uint32_t o[SPS];
-      lds_words<4 * SPS>(&S.part[lc][l][lj * SPS], o);
+      for (int l = 0; l < PR; ++l) lds_words<4 * SPS>(&S.part[lc][l][lj * SPS], o[l]);
 #pragma unroll
-      for (int i = 0; i < SPS; ++i) ch[i] = l ? ch[i] + __uint_as_float(o[i]) : __uint_as_float(o[i]);
+      for (int st = PR / 2; st >= 1; st /= 2)
+#pragma unroll
+        for (int l = 0; l < st; ++l)
+#pragma unroll
+          for (int i = 0; i < SPS; ++i)
+            o[l][i] = __float_as_uint(__uint_as_float(o[l][i]) + __uint_as_float(o[l + st][i]));
+#pragma unroll
+      for (int i = 0; i < SPS; ++i) ch[i] = __uint_as_float(o[0][i]);
     }
     float yv[SPS];
 #pragma unroll
     for (int i = 0; i < SPS; ++i) {
-      float v = fmaf(Dc, x_value(xw, i), ch[i]);
+      float v;
+      if constexpr (PR > 1)
+        v = fmaf(Dc, x_value(xw, i), ch[i]);
+      else
+        v = fmaf(Dc, x_value(xw, i), S.part[lc][0][lj * SPS + i]);
       if (p.z) v *= silu_f(h2f((uint16_t)(zw[i >> 1] >> (16 * (i & 1)))));
       yv[i] = v;
     }
@@ -493,9 +506,10 @@ __global__ void __launch_bounds__(kCH*(kN / kSPL)) m1_scan_kernel(const M1Params
       // partial C . h of every step goes to the store phase, combined over the
       // channel's lanes by a shuffle reduce-scatter after each group (PR = 1)
       // or through shared memory (PR = LPC)
-      float part[kSeg];
+      float seg[PR > 1 ? kSeg : 1];
 #pragma unroll
       for (int tg = 0; tg < kSeg / LPC; ++tg) {
+        float part[LPC];
 #pragma unroll
         for (int kk = 0; kk < LPC; ++kk) {
           const int t = s * kSeg + tg * LPC + kk;
@@ -521,17 +535,16 @@ __global__ void __launch_bounds__(kCH*(kN / kSPL)) m1_scan_kernel(const M1Params
             hp[i] = ffma2(e, hp[i], fmul2(dxv, bq[i]));
             q = i == 0 ? fmul2(cq[i], hp[i]) : ffma2(cq[i], hp[i], q);
           }
-          part[tg * LPC + kk] = q.x + q.y;
+          part[kk] = q.x + q.y;
+          if constexpr (PR > 1) seg[tg * LPC + kk] = part[kk];
         }
-        if constexpr (PR == 1)
-          S.part[lc][0][tg * LPC + lj] =
-              reduce_scatter<LPC>(*reinterpret_cast<float(*)[LPC]>(&part[tg * LPC]), lj);
+        if constexpr (PR == 1) S.part[lc][0][tg * LPC + lj] = reduce_scatter<LPC>(part, lj);
       }
       if constexpr (PR > 1)
 #pragma unroll
         for (int i = 0; i < kSeg / 4; ++i)
           reinterpret_cast<float4*>(&S.part[lc][lj][0])[i] =
-              make_float4(part[4 * i], part[4 * i + 1], part[4 * i + 2], part[4 * i + 3]);
+              make_float4(seg[4 * i], seg[4 * i + 1], seg[4 * i + 2], seg[4 * i + 3]);
       __syncwarp();
       store_seg(rcur, s, t0, tl);
       if (has_next) {
