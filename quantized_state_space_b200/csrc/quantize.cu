@@ -444,14 +444,29 @@ __global__ void __launch_bounds__(stream::kThreads, kLutCtasPerSm)
   extern __shared__ __align__(128) uint8_t smem[];
   uint8_t* lut = smem;
   uint32_t flags = 0;
+  // the table, 16 patterns per step by the packed route (se16_fast); a run
+  // holding a non-finite pattern, or any run when the steps do not allow the
+  // packed route, by se_encode1 element by element (its flags discarded: a
+  // pattern in the table need not occur in the data)
+  const bool fast_ok = st.rs[0] != 0.0f && st.rs[1] != 0.0f && st.rs[2] != 0.0f;
   auto build = [&]() {
     uint32_t dummy = 0;
-    for (int i = threadIdx.x; i < kLutBytes / 4; i += stream::kConsumers) {
-      uint32_t w = 0;
+    for (int i = threadIdx.x; i < kLutBytes / kQVec; i += stream::kConsumers) {
+      float x[kQVec];
 #pragma unroll
-      for (int k = 0; k < 4; ++k)
-        w |= se_encode1(h2f((uint16_t)(4 * i + k)), lo, hi, st, dummy) << (8 * k);
-      reinterpret_cast<uint32_t*>(lut)[i] = w;
+      for (int k = 0; k < kQVec; ++k) x[k] = h2f((uint16_t)(kQVec * i + k));
+      uint4 o;
+      if (!(fast_ok && se16_fast(x, lo, hi, st, o))) {
+        uint32_t w[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          w[k] = se_encode1(x[4 * k], lo, hi, st, dummy) |
+                 (se_encode1(x[4 * k + 1], lo, hi, st, dummy) << 8) |
+                 (se_encode1(x[4 * k + 2], lo, hi, st, dummy) << 16) |
+                 (se_encode1(x[4 * k + 3], lo, hi, st, dummy) << 24);
+        o = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+      reinterpret_cast<uint4*>(lut)[i] = o;
     }
   };
   uint32_t nf = 0;  // bit 15 / 31 set by a non-finite half
