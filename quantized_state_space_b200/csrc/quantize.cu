@@ -435,6 +435,17 @@ __global__ void __launch_bounds__(stream::kThreads)
 // 0x04000400 sets bit 15 of a half exactly when that half's exponent field
 // is 0x1F.  Two CTAs per SM (64 KB table + 48 KB of stages each).
 constexpr int kLutBytes = 65536;
+
+// Four soft-edge codes with their payloads negated, byte by byte: a standard
+// code (bit 7 clear) holds q mod 128 and becomes (128 - b) mod 128; a small
+// or large code keeps its two mode bits and its 6-bit payload p becomes
+// (64 - p) mod 64.  The per-byte differences never borrow across bytes.
+__device__ __forceinline__ uint32_t neg_codes4(uint32_t w) {
+  const uint32_t std = (0x80808080u - (w & 0x7F7F7F7Fu)) & 0x7F7F7F7Fu;
+  const uint32_t spec = ((0x40404040u - (w & 0x3F3F3F3Fu)) & 0x3F3F3F3Fu) | (w & 0xC0C0C0C0u);
+  const uint32_t sm = ((w & 0x80808080u) >> 7) * 0xFFu;  // 0xFF in each small / large byte
+  return (std & ~sm) | (spec & sm);
+}
 constexpr int kLutCtasPerSm = 2;
 
 template <typename Idx>
@@ -444,14 +455,17 @@ __global__ void __launch_bounds__(stream::kThreads, kLutCtasPerSm)
   extern __shared__ __align__(128) uint8_t smem[];
   uint8_t* lut = smem;
   uint32_t flags = 0;
-  // the table, 16 patterns per step by the packed route (se16_fast); a run
-  // holding a non-finite pattern, or any run when the steps do not allow the
-  // packed route, by se_encode1 element by element (its flags discarded: a
-  // pattern in the table need not occur in the data)
+  // the table: the codes of the non-negative patterns 16 at a time by the
+  // packed route (se16_fast); a run holding a non-finite pattern, or any run
+  // when the steps do not allow the packed route, by se_encode1 element by
+  // element (its flags discarded: a pattern in the table need not occur in
+  // the data).  The negative patterns take the negated payloads
+  // (neg_codes4): the mode depends on |v| only and the rounding and the
+  // clamp are odd functions, so code(-v) carries -q in the same mode.
   const bool fast_ok = st.rs[0] != 0.0f && st.rs[1] != 0.0f && st.rs[2] != 0.0f;
   auto build = [&]() {
     uint32_t dummy = 0;
-    for (int i = threadIdx.x; i < kLutBytes / kQVec; i += stream::kConsumers) {
+    for (int i = threadIdx.x; i < kLutBytes / 2 / kQVec; i += stream::kConsumers) {
       float x[kQVec];
 #pragma unroll
       for (int k = 0; k < kQVec; ++k) x[k] = h2f((uint16_t)(kQVec * i + k));
@@ -467,6 +481,8 @@ __global__ void __launch_bounds__(stream::kThreads, kLutCtasPerSm)
         o = make_uint4(w[0], w[1], w[2], w[3]);
       }
       reinterpret_cast<uint4*>(lut)[i] = o;
+      reinterpret_cast<uint4*>(lut + kLutBytes / 2)[i] =
+          make_uint4(neg_codes4(o.x), neg_codes4(o.y), neg_codes4(o.z), neg_codes4(o.w));
     }
   };
   uint32_t nf = 0;  // bit 15 / 31 set by a non-finite half
