@@ -86,15 +86,16 @@ inline Geo<uint32_t> make_geo(uint32_t mid, uint32_t inner) {
 }
 inline Geo<uint64_t> make_geo(uint64_t mid, uint64_t inner) { return Geo<uint64_t>{inner, mid}; }
 
-// Per-CTA table of (scale, reciprocal) for small group counts.
+// Per-CTA table of (scale, reciprocal) for small group counts, filled by
+// the consumer threads in the pipeline's prologue (the producer's first
+// copies are already in flight; the prologue ends with a consumer barrier).
 constexpr int kMaxTab = 256;
 __device__ __forceinline__ void fill_tab(const float* scales, int32_t n_groups, float2* tab) {
-  for (int g = threadIdx.x; g < n_groups && g < kMaxTab; g += blockDim.x) {
+  for (int g = threadIdx.x; g < n_groups && g < kMaxTab; g += stream::kConsumers) {
     const float s = scales[g];
     const float r = __frcp_rn(s);
     tab[g] = make_float2(s, usable_recip(s, r) ? r : 0.0f);
   }
-  __syncthreads();
 }
 __device__ __forceinline__ float2 tab_get(const float2* tab, const float* scales, int g,
                                           int32_t n_groups) {
@@ -155,20 +156,22 @@ __host__ __device__ constexpr int acc_smem_offset() {
 
 // Column path (inner == 1, mid % 16 == 0): groups of 8 consecutive columns
 // that share one group id are marked in a per-CTA table (-1 otherwise); a
-// vector's two halves look up their own entry.
+// vector's two halves look up their own entry.  ugrp_of says whether the
+// table is used; fill_ugrp fills it in the prologue, like fill_tab.
 constexpr int kMaxU = 2048;
-__device__ __forceinline__ const int* fill_ugrp(const int32_t* gmap, uint64_t mid, int* ug) {
+__device__ __forceinline__ const int* ugrp_of(uint64_t mid, int* ug) {
+  return mid / (kVec / 2) > (uint64_t)kMaxU ? nullptr : ug;
+}
+__device__ __forceinline__ void fill_ugrp(const int32_t* gmap, uint64_t mid, int* ug) {
   constexpr int kW = kVec / 2;
   const uint64_t nu = mid / kW;
-  if (nu > (uint64_t)kMaxU) return nullptr;
-  for (uint64_t u = threadIdx.x; u < nu; u += blockDim.x) {
+  if (nu > (uint64_t)kMaxU) return;
+  for (uint64_t u = threadIdx.x; u < nu; u += stream::kConsumers) {
     const int g0 = __ldg(gmap + u * kW);
     bool same = true;
     for (int i = 1; i < kW; ++i) same &= __ldg(gmap + u * kW + i) == g0;
     ug[u] = same ? g0 : -1;
   }
-  __syncthreads();
-  return ug;
 }
 
 template <bool kF16, int kPath, typename Idx>
@@ -180,20 +183,22 @@ __global__ void __launch_bounds__(stream::kThreads)
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ float2 tab[kMaxTab];
   __shared__ int ug_s[kPath == kPathCol ? kMaxU : 1];
-  fill_tab(scales, n_groups, tab);
-  const int* ugrp = kPath == kPathCol ? fill_ugrp(gmap, (uint64_t)mid, ug_s) : nullptr;
+  const int* ugrp = kPath == kPathCol ? ugrp_of((uint64_t)mid, ug_s) : nullptr;
   uint32_t flags = 0;
-  stream::run<kF16, Idx>(
-      src, n, smem,
-      [&](const float(&x)[kVec], Idx e0) {
-        quant_vec<kF16, kPath, Idx>(x, e0, geo, gmap, n_groups, scales, tab, ugrp, q, flags);
-      },
-      [&](float v, Idx e) {
-        const int g = __ldg(gmap + geo.mid_of(e));
-        const bool okg = (unsigned)g < (unsigned)n_groups;
-        q[e] = (int8_t)quant_elem(v, okg ? __ldg(scales + g) : 0.0f, 0.0f, okg, flags);
-      },
-      flags, wait_limit);
+  auto vec = [&](const float(&x)[kVec], Idx e0) {
+    quant_vec<kF16, kPath, Idx>(x, e0, geo, gmap, n_groups, scales, tab, ugrp, q, flags);
+  };
+  auto one = [&](float v, Idx e) {
+    const int g = __ldg(gmap + geo.mid_of(e));
+    const bool okg = (unsigned)g < (unsigned)n_groups;
+    q[e] = (int8_t)quant_elem(v, okg ? __ldg(scales + g) : 0.0f, 0.0f, okg, flags);
+  };
+  auto pro = [&]() {
+    fill_tab(scales, n_groups, tab);
+    if (kPath == kPathCol) fill_ugrp(gmap, (uint64_t)mid, ug_s);
+  };
+  stream::run_part<kF16, Idx, decltype(vec)&, decltype(one)&, decltype(pro)&>(
+      src, n, smem, (Idx)blockIdx.x, (Idx)gridDim.x, vec, one, flags, wait_limit, pro);
   flag_status(status, flags);
 }
 
@@ -227,21 +232,24 @@ __global__ void __launch_bounds__(stream::kThreads)
   int k = 0;
   while (k + 1 < jobs.n && (int)blockIdx.x >= jobs.j[k].cta_end) ++k;
   const QJob<Idx>& J = jobs.j[k];
-  fill_tab(J.scales, J.n_groups, tab);
-  const int* ugrp = kPath == kPathCol ? fill_ugrp(J.gmap, (uint64_t)J.mid, ug_s) : nullptr;
+  const int* ugrp = kPath == kPathCol ? ugrp_of((uint64_t)J.mid, ug_s) : nullptr;
   uint32_t flags = 0;
-  stream::run_part<kF16, Idx>(
-      J.src, J.n, smem, (Idx)((int)blockIdx.x - J.cta_beg), (Idx)(J.cta_end - J.cta_beg),
-      [&](const float(&x)[kVec], Idx e0) {
-        quant_vec<kF16, kPath, Idx>(x, e0, J.geo, J.gmap, J.n_groups, J.scales, tab, ugrp, J.q,
-                                    flags);
-      },
-      [&](float v, Idx e) {
-        const int g = __ldg(J.gmap + J.geo.mid_of(e));
-        const bool okg = (unsigned)g < (unsigned)J.n_groups;
-        J.q[e] = (int8_t)quant_elem(v, okg ? __ldg(J.scales + g) : 0.0f, 0.0f, okg, flags);
-      },
-      flags);
+  auto vec = [&](const float(&x)[kVec], Idx e0) {
+    quant_vec<kF16, kPath, Idx>(x, e0, J.geo, J.gmap, J.n_groups, J.scales, tab, ugrp, J.q,
+                                flags);
+  };
+  auto one = [&](float v, Idx e) {
+    const int g = __ldg(J.gmap + J.geo.mid_of(e));
+    const bool okg = (unsigned)g < (unsigned)J.n_groups;
+    J.q[e] = (int8_t)quant_elem(v, okg ? __ldg(J.scales + g) : 0.0f, 0.0f, okg, flags);
+  };
+  auto pro = [&]() {
+    fill_tab(J.scales, J.n_groups, tab);
+    if (kPath == kPathCol) fill_ugrp(J.gmap, (uint64_t)J.mid, ug_s);
+  };
+  stream::run_part<kF16, Idx, decltype(vec)&, decltype(one)&, decltype(pro)&>(
+      J.src, J.n, smem, (Idx)((int)blockIdx.x - J.cta_beg), (Idx)(J.cta_end - J.cta_beg), vec,
+      one, flags, stream::kWaitLimit, pro);
   flag_status(status, flags);
 }
 
