@@ -159,8 +159,10 @@ class Layer:
         smap = calibrate.state_group_map(self.G, self.N, self.gs)
         self.raw = raw
         T = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev)
-        self.host = {k: torch.from_numpy(raw[k]).pin_memory() for k in ("x", "dt", "z", "B", "C")}
-        self.x, self.dt, self.z, self.B, self.C = (T(raw[k]) for k in ("x", "dt", "z", "B", "C"))
+        self.host = {k: torch.from_numpy(raw[k]).pin_memory() for k in ("x", "dt", "z", "B", "C")
+                     if raw.get(k) is not None}
+        self.x, self.dt, self.z, self.B, self.C = (None if raw.get(k) is None else T(raw[k])
+                                                   for k in ("x", "dt", "z", "B", "C"))
         self.A, self.D = T(raw["A"]), T(raw["D"])
         self.grp, self.xs, self.bs, self.cs, self.smap = T(grp), T(xs), T(bs), T(cs), T(smap)
         self.xq = torch.empty(self.x.shape, dtype=torch.int8, device=dev)
@@ -186,11 +188,11 @@ class Layer:
             jobs.insert(0, (self.x, b, d, L, self.grp, self.k, self.xs, self.xq))
         api.quantize_groups_batch(jobs)
 
-    def scan(self):
+    def scan(self, time_segments=1):
         from quantized_state_space_b200 import api
         api.selective_scan(self.x if self.fused else self.xq, self.dt, self.A, self.Bq, self.Cq,
                            self.bs, self.cs, self.gs, x_group=self.grp, x_scale=self.xs, D=self.D,
-                           z=self.z, y=self.y, h_final=self.hf)
+                           z=self.z, y=self.y, h_final=self.hf, time_segments=time_segments)
 
     def scan_bytes(self):
         """Algorithmic HBM bytes of one scan launch."""
@@ -1225,12 +1227,16 @@ def run_kernel(args):
                                              x_scale=lay.xs, codes=lay.xq))
         label = "m130m conv input: causal conv + SiLU + int8 group codes"
     elif name in ("scan", "scan-int8", "quantize", "quantize-batch"):
+        global WORKLOAD
+        WORKLOAD = args.workload
         lay = Layer(dev, 0, fused=name == "scan")
         lay.quantize()
-        fn = {"scan": lay.scan, "scan-int8": lay.scan, "quantize-batch": lay.quantize,
+        k = args.time_segments
+        fn = {"scan": lambda: lay.scan(k), "scan-int8": lambda: lay.scan(k),
+              "quantize-batch": lay.quantize,
               "quantize": (lambda: api.quantize_groups(lay.x, lay.b, lay.d, lay.L, lay.grp, lay.k,
                                                        scales=lay.xs, out=lay.xq))}[name]
-        label = "m130m " + {"scan": "selective scan, binary16 x encoded in the scan",
+        label = args.workload + " " + {"scan": "selective scan, binary16 x encoded in the scan",
                             "scan-int8": "selective scan of int8 x codes",
                             "quantize": "x quantize (static scales)",
                             "quantize-batch": "x, B, C quantize in one launch"}[name]
@@ -1279,6 +1285,11 @@ def main():
                                          "ssd", "encode", "softedge-scan", "decode", "ex2",
                                          "conv"],
                     help="profiling aid: run only this kernel on its workload")
+    ap.add_argument("--workload", choices=["m130m", "tiny", "softedge"], default="m130m",
+                    help="with --kernel scan / scan-int8 / quantize / quantize-batch: the "
+                         "Mamba-1 workload")
+    ap.add_argument("--time-segments", type=int, default=1,
+                    help="with --kernel scan / scan-int8: time segments of the scan call")
     args = ap.parse_args()
     if args.kernel:
         run_kernel(args)

@@ -366,6 +366,22 @@ ssmq_status ssmq_conv_silu_quantize(const ssmq_conv_args* args, void* stream);
  * Supported: N in {4, 8, 16, 32, 64}; d % G == 0; any L >= 0.
  * status: device word or NULL (SSMQ_DEV_BAD_GROUP for x_group / y_group ids
  * out of range, which then read scale 0; the quantizer's bits for y_q).
+ * time_segments: 0 or 1 scans each (batch, channel) row in one pass.  k > 1
+ *   cuts L into k segments of whole 32-step chunks that run in parallel
+ *   (segment 0 from h0, the others from a zero state), then a carry-in kernel
+ *   adds to each later step the term of the state carried into its segment,
+ *   (sum_n C_tn exp(A_n S_t) h_in,n) silu(z_t), S_t the sum of delta over the
+ *   segment up to t, and forms h_final: the recurrence is linear in the
+ *   state, so the result is the one-pass result up to rounding (y of the
+ *   later segments is rounded to binary16 twice).  It multiplies the rows in
+ *   flight by k, for shapes with too few (batch, channel) rows to fill the
+ *   GPU.  The effective count is ssmq_scan_time_segments(args): 1 when y is
+ *   NULL, y_q is given, L < 64 or batch * k > 65535.
+ * workspace / workspace_bytes: with an effective count k > 1, caller-owned
+ *   device memory of at least ssmq_scan_workspace_size(args) bytes (16-byte
+ *   aligned, contents need not be initialised; it receives every segment's
+ *   local final state, k * b * d * N fp32); unused otherwise.  Errors:
+ *   INVALID_ARG when it is NULL or too small, ALIGNMENT when misaligned.
  */
 typedef struct {
   int64_t batch, seqlen, dim, dstate, ngroups;
@@ -397,9 +413,18 @@ typedef struct {
   const int32_t* y_group;   /* [d] output cluster of each channel (with y_q) */
   const float* y_scale;     /* [n_y_groups] static output scales (with y_q) */
   int32_t n_y_groups;
+  int32_t time_segments;    /* see above; 0 or 1: one pass */
+  void* workspace;          /* with time segments (see above) */
+  size_t workspace_bytes;
 } ssmq_scan_args;
 
 ssmq_status ssmq_selective_scan_w8(const ssmq_scan_args* args, void* stream);
+
+/* Effective number of time segments of a scan call (>= 1; 0 for NULL args). */
+int32_t ssmq_scan_time_segments(const ssmq_scan_args* args);
+
+/* Workspace bytes a scan call needs (0 without time segments or for NULL args). */
+size_t ssmq_scan_workspace_size(const ssmq_scan_args* args);
 
 /* ------------------------------------------------------------------------ */
 /* Mamba-2 SSD chunked scan                                                  */

@@ -38,7 +38,8 @@ class ScanArgs(C.Structure):
                 ("dt_softplus", _i32), ("A", _vp), ("D", _vp), ("z", _vp), ("B", _vp),
                 ("C", _vp), ("B_scale", _vp), ("C_scale", _vp), ("h0", _vp), ("y", _vp),
                 ("h_final", _vp), ("status", _vp), ("se_lo", _f32), ("se_hi", _f32),
-                ("y_q", _vp), ("y_group", _vp), ("y_scale", _vp), ("n_y_groups", _i32)]
+                ("y_q", _vp), ("y_group", _vp), ("y_scale", _vp), ("n_y_groups", _i32),
+                ("time_segments", _i32), ("workspace", _vp), ("workspace_bytes", C.c_size_t)]
 
 
 class SSDArgs(C.Structure):
@@ -95,6 +96,8 @@ SIGNATURES = {
     "ssmq_softedge_encode": (_i32, [_vp, _i32, _i64, _f32, _f32, _f32, _i32, _vp, _vp, _vp]),
     "ssmq_softedge_decode": (_i32, [_vp, _i64, _f32, _i32, _vp, _vp]),
     "ssmq_selective_scan_w8": (_i32, [C.POINTER(ScanArgs), _vp]),
+    "ssmq_scan_time_segments": (_i32, [C.POINTER(ScanArgs)]),
+    "ssmq_scan_workspace_size": (C.c_size_t, [C.POINTER(ScanArgs)]),
     "ssmq_conv_silu_quantize": (_i32, [C.POINTER(ConvArgs), _vp]),
     "ssmq_ssd_workspace_size": (C.c_size_t, [C.POINTER(SSDArgs)]),
     "ssmq_ssd_chunk_scan_w8": (_i32, [C.POINTER(SSDArgs), _vp, C.c_size_t, _vp]),
@@ -228,6 +231,14 @@ def ssmq_selective_scan_w8(stream=None, **fields):
     """Fields of ssmq_scan_args as keywords (tensors for pointer fields)."""
     a = _fill(ScanArgs, fields)
     _check(lib().ssmq_selective_scan_w8(C.byref(a), _stream(stream)))
+
+
+def ssmq_scan_time_segments(**fields):
+    return int(lib().ssmq_scan_time_segments(C.byref(_fill(ScanArgs, fields))))
+
+
+def ssmq_scan_workspace_size(**fields):
+    return int(lib().ssmq_scan_workspace_size(C.byref(_fill(ScanArgs, fields))))
 
 
 def ssmq_conv_silu_quantize(stream=None, **fields):

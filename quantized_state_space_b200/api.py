@@ -216,13 +216,15 @@ def selective_scan(x, dt, A, B, C, B_scale, C_scale, state_group_size, *, x_grou
                    x_scale=None, se_scale=0.0, se_log2_ratio=2, se_lo=None, se_hi=None, D=None,
                    z=None, dt_bias=None, dt_softplus=True, h0=None, y=None, h_final=None,
                    return_state=True, y_group=None, y_scale=None, y_q=None, want_y=True,
-                   status=None):
+                   time_segments=1, workspace=None, status=None):
     """Mamba-1 W8A8 selective scan.  x (b, d, L) int8 codes, soft-edge uint8
     codes, or float16 activations that the kernel encodes itself (with
     x_group / x_scale, or with se_scale / se_lo / se_hi); dt, z (b, d, L)
     float16; B, C (b, G, N, L) int8.  Returns (y, h_final), or (y, h_final,
     y_q) when y_group / y_scale ask for the int8 output (y is None when
-    want_y is False)."""
+    want_y is False).  time_segments > 1 cuts L into that many segments
+    scanned in parallel plus a carry-in pass (include/ssmq.h); the workspace
+    it needs (uint8 bytes on the device) is allocated when not given."""
     b, d, L = x.shape
     G, Nst = B.shape[1], B.shape[2]
     _dev_check(x, dt, A, B, C, B_scale, C_scale, x_group, x_scale, D, z, dt_bias, h0)
@@ -241,13 +243,18 @@ def selective_scan(x, dt, A, B, C, B_scale, C_scale, state_group_size, *, x_grou
         y, y_q, yf = _y_fields((b, d, L), dv, y_group, y_scale, y_q, want_y, y, d)
         if h_final is None and return_state:
             h_final = torch.empty((b, d, Nst), dtype=torch.float32, device=dv)
-        N.ssmq_selective_scan_w8(batch=b, seqlen=L, dim=d, dstate=Nst, ngroups=G,
-                                 state_group_size=state_group_size,
-                                 **_x_fields(x, x_group, x_scale, se_scale, se_log2_ratio, se_lo,
-                                             se_hi),
-                                 dt=dt, dt_bias=dt_bias, dt_softplus=int(bool(dt_softplus)), A=A,
-                                 D=D, z=z, B=B, C=C, B_scale=B_scale, C_scale=C_scale, h0=h0,
-                                 y=y, h_final=h_final, status=status, **yf)
+        fields = dict(batch=b, seqlen=L, dim=d, dstate=Nst, ngroups=G,
+                      state_group_size=state_group_size,
+                      **_x_fields(x, x_group, x_scale, se_scale, se_log2_ratio, se_lo, se_hi),
+                      dt=dt, dt_bias=dt_bias, dt_softplus=int(bool(dt_softplus)), A=A, D=D, z=z,
+                      B=B, C=C, B_scale=B_scale, C_scale=C_scale, h0=h0, y=y, h_final=h_final,
+                      status=status, time_segments=int(time_segments), **yf)
+        ws = N.ssmq_scan_workspace_size(**fields)
+        _workspace(workspace, ws, dv)
+        if ws and workspace is None:
+            workspace = torch.empty(ws + 256, dtype=torch.uint8, device=dv)
+        wptr = (workspace.data_ptr() + 255) // 256 * 256 if ws else None
+        N.ssmq_selective_scan_w8(workspace=wptr, workspace_bytes=ws, **fields)
     return (y, h_final, y_q) if yf else (y, h_final)
 
 

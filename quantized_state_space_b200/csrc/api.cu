@@ -405,9 +405,30 @@ ssmq_status ssmq_selective_scan_w8(const ssmq_scan_args* a, void* stream) {
             "%s: a required tensor (dt, A, B, C, B_scale, C_scale, y or y_q) is NULL", fn);
     const ssmq_status ys = check_yq(a->y_q, a->y_group, a->y_scale, a->n_y_groups, fn);
     if (ys != SSMQ_OK) return ys;
+    if (ssmq_scan_time_segments(a) > 1) {
+      const size_t need = ssmq_scan_workspace_size(a);
+      REQUIRE(a->workspace && a->workspace_bytes >= need, SSMQ_ERR_INVALID_ARG,
+              "%s: %d time segments need a workspace of %zu bytes", fn,
+              (int)ssmq_scan_time_segments(a), need);
+      REQUIRE(aligned16(a->workspace), SSMQ_ERR_ALIGNMENT,
+              "%s: workspace must be 16-byte aligned", fn);
+    }
   }
   if (injected(fn)) return fail(SSMQ_ERR_CUDA, "%s: injected launch failure", fn);
   return finish(ssmq::launch_selective_scan(*a, (cudaStream_t)stream), fn);
+}
+
+int32_t ssmq_scan_time_segments(const ssmq_scan_args* a) {
+  if (!a) return 0;
+  int64_t seg_len = 0;
+  return (int32_t)ssmq::scan_time_segments(*a, &seg_len);
+}
+
+size_t ssmq_scan_workspace_size(const ssmq_scan_args* a) {
+  if (!a) return 0;
+  const int64_t k = ssmq_scan_time_segments(a);
+  if (k <= 1 || a->batch <= 0 || a->dim <= 0 || a->dstate <= 0) return 0;
+  return (size_t)k * (size_t)a->batch * (size_t)a->dim * (size_t)a->dstate * sizeof(float);
 }
 
 size_t ssmq_ssd_workspace_size(const ssmq_ssd_args* a) {

@@ -33,6 +33,9 @@ cudaError_t launch_softedge_encode(const void* src, bool f16, int64_t n, float s
 cudaError_t launch_softedge_decode(const uint8_t* codes, int64_t n, float scale,
                                    int log2_ratio, float* out, cudaStream_t st);
 
+// Time segments of a Mamba-1 scan call (1: one pass per row) and their
+// length in steps (whole 32-step chunks).
+int scan_time_segments(const ssmq_scan_args& a, int64_t* seg_len);
 cudaError_t launch_selective_scan(const ssmq_scan_args& a, cudaStream_t st);
 cudaError_t launch_conv_silu_quantize(const ssmq_conv_args& a, cudaStream_t st);
 

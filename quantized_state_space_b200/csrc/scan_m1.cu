@@ -73,6 +73,14 @@ struct M1Params {
   uint32_t* status;
   int n_ctile;
   int vec_ok;
+  // time segments: CTA row blockIdx.y = bb * nseg + seg scans steps
+  // [seg * seg_len, min(L, (seg + 1) * seg_len)) of batch row bb, segment 0
+  // from h0 and the others from a zero state; with nseg > 1 every segment's
+  // local final state goes to seg_state[((seg * b + bb) * d + c) * N + n]
+  // (the carry-in kernel adds the carried terms and writes h_final)
+  int nseg;
+  int64_t seg_len;
+  float* seg_state;
 };
 
 // ---- cp.async (16-byte, L2-only) -------------------------------------------
@@ -221,8 +229,10 @@ __global__ void __launch_bounds__(kCH*(kN / kSPL)) m1_scan_kernel(const M1Params
   M1Smem<kN, kCH, PR, XT>& S = *reinterpret_cast<M1Smem<kN, kCH, PR, XT>*>(smem_bytes);
 
   const int tid = threadIdx.x;
-  const int64_t bb = blockIdx.y;
+  const int64_t bb = blockIdx.y / p.nseg;
+  const int seg = (int)(blockIdx.y % p.nseg);
   const int64_t d = p.d, L = p.L;
+  const int64_t t_beg = (int64_t)seg * p.seg_len, t_end = min(L, t_beg + p.seg_len);
   const int dg = (int)(d / p.G);
   const int g = blockIdx.x / p.n_ctile;
   const int c0 = g * dg + (blockIdx.x % p.n_ctile) * kCH;
@@ -241,7 +251,7 @@ __global__ void __launch_bounds__(kCH*(kN / kSPL)) m1_scan_kernel(const M1Params
     const int n = lj * kSPL + 2 * i;
     ap[i] = lvalid ? make_float2(__ldg(p.A + lch * kN + n) * kLog2e, __ldg(p.A + lch * kN + n + 1) * kLog2e)
                    : make_float2(0.0f, 0.0f);
-    hp[i] = (lvalid && p.h0) ? make_float2(__ldg(p.h0 + (bb * d + lch) * kN + n),
+    hp[i] = (lvalid && p.h0 && seg == 0) ? make_float2(__ldg(p.h0 + (bb * d + lch) * kN + n),
                                            __ldg(p.h0 + (bb * d + lch) * kN + n + 1))
                              : make_float2(0.0f, 0.0f);
   }
@@ -465,15 +475,16 @@ __global__ void __launch_bounds__(kCH*(kN / kSPL)) m1_scan_kernel(const M1Params
     }
   };
 
-  const int nchunks = (int)((L + kT - 1) / kT);
-  auto chunk_len = [&](int k) { return (int)min((int64_t)kT, L - (int64_t)k * kT); };
+  const int nchunks = (int)((t_end - t_beg + kT - 1) / kT);
+  auto chunk_len = [&](int k) { return (int)min((int64_t)kT, t_end - t_beg - (int64_t)k * kT); };
 
   // prologue: raw bytes of chunks 0 and 1, chunk 0 staged
-  fetch_chunk<kN, kCH, XT>(p, S.raw[0], bb, g, c0, nc, 0, chunk_len(0), tid, NT);
+  fetch_chunk<kN, kCH, XT>(p, S.raw[0], bb, g, c0, nc, t_beg, chunk_len(0), tid, NT);
   cp_async_commit();
   cp_async_wait_all();
   __syncthreads();
-  if (nchunks > 1) fetch_chunk<kN, kCH, XT>(p, S.raw[1], bb, g, c0, nc, kT, chunk_len(1), tid, NT);
+  if (nchunks > 1)
+    fetch_chunk<kN, kCH, XT>(p, S.raw[1], bb, g, c0, nc, t_beg + kT, chunk_len(1), tid, NT);
   cp_async_commit();
 #pragma unroll
   for (int s = 0; s < kSegs; ++s) {
@@ -482,7 +493,7 @@ __global__ void __launch_bounds__(kCH*(kN / kSPL)) m1_scan_kernel(const M1Params
   }
 
   for (int k = 0; k < nchunks; ++k) {
-    const int64_t t0 = (int64_t)k * kT;
+    const int64_t t0 = t_beg + (int64_t)k * kT;
     const int tl = chunk_len(k);
     const bool has_next = k + 1 < nchunks;
     const int tl_next = has_next ? chunk_len(k + 1) : 0;
@@ -556,11 +567,93 @@ __global__ void __launch_bounds__(kCH*(kN / kSPL)) m1_scan_kernel(const M1Params
     }
   }
 
-  if (lvalid && p.h_final)
+  float* hout = p.nseg > 1 ? p.seg_state + (int64_t)seg * p.b * d * kN : p.h_final;
+  if (lvalid && hout)
 #pragma unroll
     for (int i = 0; i < NP; ++i)
-      *reinterpret_cast<float2*>(p.h_final + (bb * d + lch) * kN + lj * kSPL + 2 * i) = hp[i];
+      *reinterpret_cast<float2*>(hout + (bb * d + lch) * kN + lj * kSPL + 2 * i) = hp[i];
   flag_status(p.status, flags);
+}
+
+// ---- carry-in of the time segments ------------------------------------------
+// The recurrence is linear in the state: for a step t of segment j >= 1 the
+// true state is the segment's local one (scanned from zero) plus
+// exp(A S_t) h_in(j), S_t the sum of delta over the segment's steps up to and
+// including t, where h_in(1) is segment 0's final state (it started from h0)
+// and h_in(j + 1) = exp(A S_end(j)) h_in(j) + h_local_end(j).  So y_t gains
+// (sum_n C_tn sC_n exp(A_n S_t) h_in,n) times silu(z_t), rounded to binary16
+// once more, and h_final = h_in(nseg).  One warp per (batch, channel) row
+// walks the later segments in order with its lanes over 32 consecutive
+// steps: delta per lane, S_t by an inclusive warp scan plus the total of the
+// earlier blocks; the per-state exponentials are independent across steps,
+// so the work is parallel over (row, step) and needs no sequential pass.
+constexpr int kCarryWarps = 8;
+
+__device__ __forceinline__ float s8f(int8_t v) {
+  // exact int8 -> fp32 without the conversion unit: 2^23 + (v + 128) - (2^23 + 128)
+  return __int_as_float(0x4B000000 | ((uint32_t)(uint8_t)v ^ 0x80u)) - 8388736.0f;
+}
+
+template <int kN>
+__global__ void __launch_bounds__(32 * kCarryWarps) m1_carry_kernel(const M1Params p) {
+  __shared__ float sh_a[kCarryWarps][kN];  // A_cn log2(e)
+  __shared__ float sh_w[kCarryWarps][kN];  // sC_n h_in,n of the current segment
+  __shared__ float sh_h[kCarryWarps][kN];  // h_in,n
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t d = p.d, L = p.L;
+  const int64_t row = (int64_t)blockIdx.x * kCarryWarps + warp;  // bb * d + c
+  if (row >= p.b * d) return;  // whole warps only
+  const int64_t bb = row / d, c = row % d;
+  const int g = (int)(c / (d / p.G));
+  const int spg = kN / p.gs;
+  const float bias = p.dt_bias ? __ldg(p.dt_bias + c) : 0.0f;
+  float* A2 = sh_a[warp];
+  float* W = sh_w[warp];
+  float* Hs = sh_h[warp];
+  for (int n = lane; n < kN; n += 32) {
+    A2[n] = __ldg(p.A + c * kN + n) * kLog2e;
+    Hs[n] = p.seg_state[row * kN + n];  // segment 0's final state
+  }
+  const int8_t* Crow = p.C + (bb * p.G + g) * kN * L;  // C of state n, step t: Crow[n L + t]
+  for (int seg = 1; seg < p.nseg; ++seg) {
+    const int64_t t_beg = (int64_t)seg * p.seg_len, t_end = min(L, t_beg + p.seg_len);
+    __syncwarp();
+    for (int n = lane; n < kN; n += 32) W[n] = __ldg(p.C_scale + g * spg + n / p.gs) * Hs[n];
+    __syncwarp();
+    float s_run = 0.0f;  // delta summed over the segment's earlier blocks
+    for (int64_t t0 = t_beg; t0 < t_end; t0 += 32) {
+      const int64_t t = t0 + lane;
+      const bool ok = t < t_end;
+      float delta = 0.0f;
+      if (ok) {
+        const float dv = h2f(p.dt[row * L + t]) + bias;
+        delta = p.softplus ? softplus_f(dv) : dv;
+      }
+      float sc = delta;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const float v = __shfl_up_sync(0xffffffffu, sc, o);
+        if (lane >= o) sc += v;
+      }
+      const float S = s_run + sc;
+      s_run += __shfl_sync(0xffffffffu, sc, 31);
+      if (ok) {
+        float corr = 0.0f;
+#pragma unroll
+        for (int n = 0; n < kN; ++n)
+          corr = fmaf(s8f(Crow[n * L + t]) * W[n], ex2_sfu(A2[n] * S), corr);
+        const float gate = p.z ? silu_f(h2f(p.z[row * L + t])) : 1.0f;
+        uint16_t* yp = p.y + row * L + t;
+        *yp = f2h(fmaf(corr, gate, h2f(*yp)));
+      }
+    }
+    __syncwarp();
+    const float* hl = p.seg_state + ((int64_t)seg * p.b * d + row) * kN;
+    for (int n = lane; n < kN; n += 32) Hs[n] = fmaf(ex2_sfu(A2[n] * s_run), Hs[n], hl[n]);
+  }
+  __syncwarp();
+  if (p.h_final)
+    for (int n = lane; n < kN; n += 32) p.h_final[row * kN + n] = Hs[n];
 }
 
 template <int kN, int kCH, int kSPL>
@@ -568,7 +661,7 @@ cudaError_t launch_m1(const M1Params& prm, int xfmt, int64_t batch, cudaStream_t
   M1Params p = prm;
   const int dg = (int)(p.d / p.G);
   p.n_ctile = (dg + kCH - 1) / kCH;
-  const dim3 grid((unsigned)(p.n_ctile * p.G), (unsigned)batch);
+  const dim3 grid((unsigned)(p.n_ctile * p.G), (unsigned)(batch * p.nseg));
   const dim3 block(kCH * (kN / kSPL));
   const bool f16 = xfmt == SSMQ_X_F16_GROUP || xfmt == SSMQ_X_F16_SOFTEDGE;
   constexpr int LPC = kN / kSPL;
@@ -587,14 +680,32 @@ cudaError_t launch_m1(const M1Params& prm, int xfmt, int64_t batch, cudaStream_t
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   kern<<<grid, block, smem, st>>>(p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess || p.nseg <= 1) return e;
+  const int64_t rows = p.b * p.d;
+  m1_carry_kernel<kN><<<(unsigned)((rows + kCarryWarps - 1) / kCarryWarps), 32 * kCarryWarps, 0,
+                        st>>>(p);
   return cudaGetLastError();
 }
 
 }  // namespace
 
+int scan_time_segments(const ssmq_scan_args& a, int64_t* seg_len) {
+  *seg_len = a.seqlen;
+  int64_t k = a.time_segments;
+  if (k <= 1 || a.y == nullptr || a.y_q != nullptr || a.seqlen < 2 * kT) return 1;
+  const int64_t sl = ((a.seqlen + k - 1) / k + kT - 1) / kT * kT;  // whole chunks
+  k = (a.seqlen + sl - 1) / sl;
+  if (k <= 1 || a.batch * k > 65535) return 1;
+  *seg_len = sl;
+  return (int)k;
+}
+
 cudaError_t launch_selective_scan(const ssmq_scan_args& a, cudaStream_t st) {
   if (a.batch == 0 || a.dim == 0) return cudaSuccess;
   M1Params p{};
+  p.nseg = scan_time_segments(a, &p.seg_len);
+  p.seg_state = static_cast<float*>(a.workspace);
   p.b = a.batch;
   p.L = a.seqlen;
   p.d = a.dim;

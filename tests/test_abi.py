@@ -131,6 +131,38 @@ def test_scan_validation(L):
     assert L.ssmq_selective_scan_w8(None, None) == N.ERR_INVALID_ARG
 
 
+def test_scan_time_segments_rule(L):
+    """Segments of whole 32-step chunks; one pass without binary16 y, with
+    int8 y, below 64 steps or beyond 65535 (batch x segments) rows; the
+    workspace holds every segment's fp32 (d, N) state per batch row."""
+    K = lambda **kw: L.ssmq_scan_time_segments(C.byref(_scan_args(**kw)))
+    W = lambda **kw: L.ssmq_scan_workspace_size(C.byref(_scan_args(**kw)))
+    a = dict(batch=2, seqlen=2048, dim=64, dstate=16)
+    assert K(**a) == 1 and W(**a) == 0
+    assert K(time_segments=0, **a) == 1
+    assert K(time_segments=2, **a) == 2 and W(time_segments=2, **a) == 2 * 2 * 64 * 16 * 4
+    assert K(time_segments=4, **a) == 4
+    assert K(time_segments=3, batch=2, seqlen=100, dim=64, dstate=16) == 2  # 34 -> 64 steps
+    assert K(time_segments=8, batch=2, seqlen=64, dim=64, dstate=16) == 2   # whole chunks
+    assert K(time_segments=2, batch=2, seqlen=63, dim=64, dstate=16) == 1
+    assert K(time_segments=2, y=None, y_q=FAKE, y_group=FAKE, y_scale=FAKE, n_y_groups=1,
+             **a) == 1
+    assert K(time_segments=2, batch=40000, seqlen=2048, dim=64, dstate=16) == 1
+    assert L.ssmq_scan_time_segments(None) == 0 and L.ssmq_scan_workspace_size(None) == 0
+
+
+def test_scan_time_segments_validation(L):
+    S = lambda **kw: L.ssmq_selective_scan_w8(C.byref(_scan_args(**kw)), None)
+    a = dict(time_segments=2, seqlen=2048)
+    nb = L.ssmq_scan_workspace_size(C.byref(_scan_args(**a)))
+    assert nb > 0
+    assert S(**a) == N.ERR_INVALID_ARG                                   # no workspace
+    assert S(workspace=FAKE, workspace_bytes=nb - 4, **a) == N.ERR_INVALID_ARG
+    assert S(workspace=FAKE + 8, workspace_bytes=nb, **a) == N.ERR_ALIGNMENT
+    # one pass: the workspace is not looked at
+    assert S(batch=0, **a) == N.OK
+
+
 def _ssd_args(**kw):
     f = dict(batch=1, seqlen=512, nheads=8, headdim=64, dstate=128, ngroups=1, chunk=256,
              state_group_size=8, x_format=N.X_INT8_GROUP, x=FAKE, x_group=FAKE, x_scale=FAKE,

@@ -137,9 +137,75 @@ def test_scan_checkpoint_split_bit_exact():
     np.testing.assert_array_equal(hb, hf)
 
 
+# ---- time segments: L cut into k segments scanned in parallel (later ones
+# from a zero state) plus the carry-in pass; the recurrence is linear in the
+# state, so the result is the one-pass result up to rounding
+
+SEG_CASES = [
+    # (b, L, d, N, G, gs, gate, h0, bias, fmt, k)
+    (2, 200, 40, 16, 1, 4, True, False, False, "int8", 2),    # ragged L: short last segment
+    (3, 512, 48, 16, 2, 4, True, True, True, "int8", 4),      # G = 2, h0, bias
+    (2, 300, 32, 8, 1, 4, False, True, True, "int8", 3),
+    (2, 256, 32, 32, 1, 8, True, True, False, "int8", 2),
+    (1, 200, 24, 64, 1, 16, True, False, True, "int8", 3),
+    (2, 384, 48, 16, 1, 4, True, True, False, "softedge", 3),
+    (2, 96, 64, 4, 1, 2, True, True, False, "int8", 2),
+    (1, 2048, 16, 16, 1, 4, True, True, True, "int8", 8),     # eight 256-step segments
+]
+
+
+@pytest.mark.parametrize("ci", range(len(SEG_CASES)))
+def test_scan_time_segments_vs_oracle(orc, ci):
+    b, L, d, N_, G, gs, gate, h0, bias, fmt, k = SEG_CASES[ci]
+    p = m1_problem(400 + ci, b, L, d, N_, G=G, gs=gs, gate=gate, h0=h0, bias=bias,
+                   x_format=fmt)
+    y, hf = gpu_scan(p, time_segments=k)
+    yo, ho = oracle_scan(orc, p)
+    assert_scan_close(y, yo.reshape(y.shape), hf, ho.reshape(hf.shape))
+    # and close to the one-pass kernel (y of later segments rounded twice)
+    y1, h1 = gpu_scan(p)
+    assert y_err(y, y1) <= 2 * 2.0 ** -11
+    assert np.linalg.norm(hf - h1) <= 1e-5 * np.linalg.norm(h1)
+
+
+def test_scan_time_segments_fused_encode_bit_exact():
+    """Binary16 x encoded in the scan with time segments equals the separate
+    quantizer followed by the code-reading scan with the same segments."""
+    b, L, d, N_ = 2, 320, 48, 16
+    p = m1_problem(450, b, L, d, N_, gate=True, h0=True)
+    rng = np.random.default_rng(451)
+    xf = _f16_activations(rng, (b, d, L))
+    grp, xs = T(p["x_group"]), T(p["x_scale"])
+    codes, _ = api.quantize_groups(T(xf), b, d, L, grp, int(xs.numel()), scales=xs)
+    args = (T(p["dt"]), T(p["A"]), T(p["B"]), T(p["C"]), T(p["B_scale"]), T(p["C_scale"]), 4)
+    kw = dict(x_group=grp, x_scale=xs, D=T(p["D"]), z=T(p["z"]), h0=T(p["h0"]), time_segments=3)
+    y1, h1 = api.selective_scan(codes, *args, **kw)
+    y2, h2 = api.selective_scan(T(xf), *args, **kw)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(H(y2).view(np.uint16), H(y1).view(np.uint16))
+    np.testing.assert_array_equal(H(h2).view(np.uint32), H(h1).view(np.uint32))
+
+
+def test_scan_time_segments_off_with_int8_y():
+    """With the int8 y output the call keeps one pass: the bytes equal the
+    call without segments."""
+    p = m1_problem(460, 2, 256, 32, 16, gate=True, h0=True)
+    yg = T(np.arange(32, dtype=np.int32) % 2)
+    ys = T(np.array([0.02, 0.05], np.float32))
+    args = (T(p["x"]), T(p["dt"]), T(p["A"]), T(p["B"]), T(p["C"]), T(p["B_scale"]),
+            T(p["C_scale"]), 4)
+    kw = dict(x_group=T(p["x_group"]), x_scale=T(p["x_scale"]), D=T(p["D"]), z=T(p["z"]),
+              h0=T(p["h0"]), y_group=yg, y_scale=ys)
+    a = api.selective_scan(*args, **kw)
+    c = api.selective_scan(*args, time_segments=4, **kw)
+    torch.cuda.synchronize()
+    for u, v in zip(a, c):
+        np.testing.assert_array_equal(H(u), H(v))
+
+
 # ---- full-size workloads, end to end from raw activations ------------------
 
-def _m1_end_to_end(orc, name, n_units=96):
+def _m1_end_to_end(orc, name, n_units=96, time_segments=1):
     dm, raw = synth.workload_inputs(name)
     b, L, d, Nst, G, gs = dm["batch"], dm["seqlen"], dm["dim"], dm["dstate"], dm["ngroups"], \
         dm["state_group_size"]
@@ -164,7 +230,7 @@ def _m1_end_to_end(orc, name, n_units=96):
             xq, _ = api.quantize_groups(T(raw["x"]), b, d, L, T(grp), k, scales=T(xs))
             xkw = dict(x_group=T(grp), x_scale=T(xs))
     y, hf = api.selective_scan(xq, T(raw["dt"]), T(raw["A"]), Bq, Cq, T(bs), T(cs), gs,
-                               D=T(raw["D"]), z=T(raw["z"]), **xkw)
+                               D=T(raw["D"]), z=T(raw["z"]), time_segments=time_segments, **xkw)
     torch.cuda.synchronize()
     # oracle: its own calibration and quantizers from the same raw arrays; the
     # B/C scale index of row (g, n) is (g N + n) / gs in the ABI's layout
@@ -230,6 +296,11 @@ def test_m130m_workload_end_to_end(orc):
 
 def test_softedge_workload_end_to_end(orc):
     _m1_end_to_end(orc, "softedge", n_units=64)
+
+
+@pytest.mark.parametrize("k", [2, 4])
+def test_m130m_workload_time_segments(orc, k):
+    _m1_end_to_end(orc, "m130m", time_segments=k)
 
 
 # ---- encode then scan: binary16 x encoded inside the scan (producer-side
