@@ -382,6 +382,11 @@ ssmq_status ssmq_conv_silu_quantize(const ssmq_conv_args* args, void* stream);
  *   aligned, contents need not be initialised; it receives every segment's
  *   local final state, k * b * d * N fp32); unused otherwise.  Errors:
  *   INVALID_ARG when it is NULL or too small, ALIGNMENT when misaligned.
+ * dec_final: fp32 (b, d, N) output or NULL: the log2 decay of the call's
+ *   steps, A_cn log2(e) sum_t delta_t per (batch, channel, state), which
+ *   chains the slices of a sequence cut over several calls or ranks
+ *   (ssmq_state_chain with units b * d * N, elems 1).  A call with dec_final
+ *   keeps one pass (no time segments).
  */
 typedef struct {
   int64_t batch, seqlen, dim, dstate, ngroups;
@@ -416,6 +421,7 @@ typedef struct {
   int32_t time_segments;    /* see above; 0 or 1: one pass */
   void* workspace;          /* with time segments (see above) */
   size_t workspace_bytes;
+  float* dec_final;         /* (b, d, N) log2 decays of the call, or NULL */
 } ssmq_scan_args;
 
 ssmq_status ssmq_selective_scan_w8(const ssmq_scan_args* args, void* stream);
@@ -425,6 +431,24 @@ int32_t ssmq_scan_time_segments(const ssmq_scan_args* args);
 
 /* Workspace bytes a scan call needs (0 without time segments or for NULL args). */
 size_t ssmq_scan_workspace_size(const ssmq_scan_args* args);
+
+/*
+ * ssmq_selective_scan_carry_in: a slice of a sequence (the steps of args)
+ * was scanned from a zero state while the true state entering it is h_carry
+ * (fp32 (b, d, N), device): adds the carried term to every step,
+ * y_t += (sum_n C_tn sC_n exp(A_cn S_ct) h_carry,cn) silu(z_t), S_ct the sum
+ * of delta over the slice up to t (y rounded to binary16 once more), and,
+ * when args->h_final is given, turns the slice's final state into the true
+ * one: h_final = exp(A S_c,L) h_carry + h_final.  args are those of the
+ * slice's ssmq_selective_scan_w8 call (y required; y_q, h0, dec_final,
+ * time_segments and workspace are ignored; x is not read).  With the slices'
+ * h_final and dec_final chained by ssmq_state_chain this gives the unsplit
+ * scan up to rounding (Mamba-1 sequence sharding).  Errors: INVALID_ARG for
+ * NULL args / y / h_carry / dt / A / C / C_scale, UNSUPPORTED dstate,
+ * ALIGNMENT for misaligned tensors.
+ */
+ssmq_status ssmq_selective_scan_carry_in(const ssmq_scan_args* args, const float* h_carry,
+                                         void* stream);
 
 /* ------------------------------------------------------------------------ */
 /* Mamba-2 SSD chunked scan                                                  */

@@ -39,7 +39,8 @@ class ScanArgs(C.Structure):
                 ("C", _vp), ("B_scale", _vp), ("C_scale", _vp), ("h0", _vp), ("y", _vp),
                 ("h_final", _vp), ("status", _vp), ("se_lo", _f32), ("se_hi", _f32),
                 ("y_q", _vp), ("y_group", _vp), ("y_scale", _vp), ("n_y_groups", _i32),
-                ("time_segments", _i32), ("workspace", _vp), ("workspace_bytes", C.c_size_t)]
+                ("time_segments", _i32), ("workspace", _vp), ("workspace_bytes", C.c_size_t),
+                ("dec_final", _vp)]
 
 
 class SSDArgs(C.Structure):
@@ -97,6 +98,7 @@ SIGNATURES = {
     "ssmq_softedge_decode": (_i32, [_vp, _i64, _f32, _i32, _vp, _vp]),
     "ssmq_selective_scan_w8": (_i32, [C.POINTER(ScanArgs), _vp]),
     "ssmq_scan_time_segments": (_i32, [C.POINTER(ScanArgs)]),
+    "ssmq_selective_scan_carry_in": (_i32, [C.POINTER(ScanArgs), _vp, _vp]),
     "ssmq_scan_workspace_size": (C.c_size_t, [C.POINTER(ScanArgs)]),
     "ssmq_conv_silu_quantize": (_i32, [C.POINTER(ConvArgs), _vp]),
     "ssmq_ssd_workspace_size": (C.c_size_t, [C.POINTER(SSDArgs)]),
@@ -231,6 +233,12 @@ def ssmq_selective_scan_w8(stream=None, **fields):
     """Fields of ssmq_scan_args as keywords (tensors for pointer fields)."""
     a = _fill(ScanArgs, fields)
     _check(lib().ssmq_selective_scan_w8(C.byref(a), _stream(stream)))
+
+
+def ssmq_selective_scan_carry_in(h_carry, stream=None, **fields):
+    """Fields of ssmq_scan_args as keywords; h_carry the carried state."""
+    a = _fill(ScanArgs, fields)
+    _check(lib().ssmq_selective_scan_carry_in(C.byref(a), ptr(h_carry), _stream(stream)))
 
 
 def ssmq_scan_time_segments(**fields):

@@ -216,7 +216,7 @@ def selective_scan(x, dt, A, B, C, B_scale, C_scale, state_group_size, *, x_grou
                    x_scale=None, se_scale=0.0, se_log2_ratio=2, se_lo=None, se_hi=None, D=None,
                    z=None, dt_bias=None, dt_softplus=True, h0=None, y=None, h_final=None,
                    return_state=True, y_group=None, y_scale=None, y_q=None, want_y=True,
-                   time_segments=1, workspace=None, status=None):
+                   time_segments=1, workspace=None, dec_final=None, status=None):
     """Mamba-1 W8A8 selective scan.  x (b, d, L) int8 codes, soft-edge uint8
     codes, or float16 activations that the kernel encodes itself (with
     x_group / x_scale, or with se_scale / se_lo / se_hi); dt, z (b, d, L)
@@ -224,7 +224,9 @@ def selective_scan(x, dt, A, B, C, B_scale, C_scale, state_group_size, *, x_grou
     y_q) when y_group / y_scale ask for the int8 output (y is None when
     want_y is False).  time_segments > 1 cuts L into that many segments
     scanned in parallel plus a carry-in pass (include/ssmq.h); the workspace
-    it needs (uint8 bytes on the device) is allocated when not given."""
+    it needs (uint8 bytes on the device) is allocated when not given.
+    dec_final (b, d, N) float32, when given, receives the call's log2 decays
+    A log2(e) sum_t delta_t (for chaining slices of a sequence)."""
     b, d, L = x.shape
     G, Nst = B.shape[1], B.shape[2]
     _dev_check(x, dt, A, B, C, B_scale, C_scale, x_group, x_scale, D, z, dt_bias, h0)
@@ -238,6 +240,7 @@ def selective_scan(x, dt, A, B, C, B_scale, C_scale, state_group_size, *, x_grou
     _bc_in(B, C, B_scale, C_scale, b * G * Nst * L, _n_scales(G, Nst, state_group_size), dv)
     _in(h0, "h0", torch.float32, b * d * Nst, dv)
     _out(h_final, "h_final", torch.float32, b * d * Nst, dv)
+    _out(dec_final, "dec_final", torch.float32, b * d * Nst, dv)
     _status(status, dv)
     with _on(dv):
         y, y_q, yf = _y_fields((b, d, L), dv, y_group, y_scale, y_q, want_y, y, d)
@@ -248,7 +251,8 @@ def selective_scan(x, dt, A, B, C, B_scale, C_scale, state_group_size, *, x_grou
                       **_x_fields(x, x_group, x_scale, se_scale, se_log2_ratio, se_lo, se_hi),
                       dt=dt, dt_bias=dt_bias, dt_softplus=int(bool(dt_softplus)), A=A, D=D, z=z,
                       B=B, C=C, B_scale=B_scale, C_scale=C_scale, h0=h0, y=y, h_final=h_final,
-                      status=status, time_segments=int(time_segments), **yf)
+                      status=status, time_segments=int(time_segments), dec_final=dec_final,
+                      **yf)
         ws = N.ssmq_scan_workspace_size(**fields)
         _workspace(workspace, ws, dv)
         if ws and workspace is None:
@@ -256,6 +260,35 @@ def selective_scan(x, dt, A, B, C, B_scale, C_scale, state_group_size, *, x_grou
         wptr = (workspace.data_ptr() + 255) // 256 * 256 if ws else None
         N.ssmq_selective_scan_w8(workspace=wptr, workspace_bytes=ws, **fields)
     return (y, h_final, y_q) if yf else (y, h_final)
+
+
+def selective_scan_carry_in(x, dt, A, B, C, B_scale, C_scale, state_group_size, h_carry, y, *,
+                            D=None, z=None, dt_bias=None, dt_softplus=True, h_final=None,
+                            status=None):
+    """Adds the contribution of the start state h_carry (b, d, N) to the y
+    (in place) and h_final (in place, if given) of a Mamba-1 scan call on the
+    same inputs that started from a zero state.  x gives the shapes only."""
+    _dev_check(x, dt, A, B, C, B_scale, C_scale, D, z, dt_bias, h_carry, y, h_final)
+    b, d, L = x.shape
+    G, Nst = B.shape[1], B.shape[2]
+    dv = x.device
+    _in(dt, "dt", torch.float16, b * d * L, dv)
+    _in(z, "z", torch.float16, b * d * L, dv)
+    _in(A, "A", torch.float32, d * Nst, dv)
+    _in(D, "D", torch.float32, d, dv)
+    _in(dt_bias, "dt_bias", torch.float32, d, dv)
+    _bc_in(B, C, B_scale, C_scale, b * G * Nst * L, _n_scales(G, Nst, state_group_size), dv)
+    _out(y, "y", torch.float16, b * d * L, dv)
+    _out(h_carry, "h_carry", torch.float32, b * d * Nst, dv)
+    _out(h_final, "h_final", torch.float32, b * d * Nst, dv)
+    _status(status, dv)
+    with _on(dv):
+        N.ssmq_selective_scan_carry_in(h_carry, batch=b, seqlen=L, dim=d, dstate=Nst, ngroups=G,
+                                       state_group_size=state_group_size, dt=dt,
+                                       dt_bias=dt_bias, dt_softplus=int(bool(dt_softplus)), A=A,
+                                       D=D, z=z, B=B, C=C, B_scale=B_scale, C_scale=C_scale, y=y,
+                                       h_final=h_final, status=status)
+    return y, h_final
 
 
 def conv_silu_quantize(x, weight, *, bias=None, x_prev=None, x_group=None, x_scale=None,

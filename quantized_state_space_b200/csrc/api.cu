@@ -389,7 +389,7 @@ ssmq_status ssmq_selective_scan_w8(const ssmq_scan_args* a, void* stream) {
   if (a->batch == 0 || a->dim == 0) return SSMQ_OK;
   REQUIRE(aligned16(a->x) && aligned16(a->dt) && aligned16(a->z) && aligned16(a->B) &&
               aligned16(a->C) && aligned16(a->y) && aligned16(a->h0) && aligned16(a->h_final) &&
-              aligned16(a->A),
+              aligned16(a->A) && aligned16(a->dec_final),
           SSMQ_ERR_ALIGNMENT, "%s: tensors must be 16-byte aligned", fn);
   REQUIRE(a->batch <= 65535, SSMQ_ERR_UNSUPPORTED, "%s: batch > 65535", fn);
   if (a->seqlen > 0) {
@@ -416,6 +416,33 @@ ssmq_status ssmq_selective_scan_w8(const ssmq_scan_args* a, void* stream) {
   }
   if (injected(fn)) return fail(SSMQ_ERR_CUDA, "%s: injected launch failure", fn);
   return finish(ssmq::launch_selective_scan(*a, (cudaStream_t)stream), fn);
+}
+
+ssmq_status ssmq_selective_scan_carry_in(const ssmq_scan_args* a, const float* h_carry,
+                                         void* stream) {
+  const char* fn = "ssmq_selective_scan_carry_in";
+  Range nvtx_range(fn);
+  REQUIRE(a != nullptr, SSMQ_ERR_INVALID_ARG, "%s: args is NULL", fn);
+  REQUIRE(a->batch >= 0 && a->seqlen >= 0 && a->dim >= 0, SSMQ_ERR_INVALID_ARG,
+          "%s: negative size", fn);
+  REQUIRE(a->ngroups >= 1 && a->dim % a->ngroups == 0, SSMQ_ERR_INVALID_ARG,
+          "%s: dim must be a multiple of ngroups >= 1", fn);
+  REQUIRE(a->dstate == 4 || a->dstate == 8 || a->dstate == 16 || a->dstate == 32 ||
+              a->dstate == 64,
+          SSMQ_ERR_UNSUPPORTED, "%s: dstate %lld not in {4, 8, 16, 32, 64}", fn,
+          (long long)a->dstate);
+  REQUIRE(a->state_group_size >= 1 && a->dstate % a->state_group_size == 0,
+          SSMQ_ERR_INVALID_ARG, "%s: dstate must be a multiple of state_group_size", fn);
+  if (a->batch == 0 || a->dim == 0) return SSMQ_OK;
+  REQUIRE(h_carry != nullptr, SSMQ_ERR_INVALID_ARG, "%s: h_carry is NULL", fn);
+  if (a->seqlen > 0)
+    REQUIRE(a->y && a->dt && a->A && a->C && a->C_scale, SSMQ_ERR_INVALID_ARG,
+            "%s: a required tensor (y, dt, A, C, C_scale) is NULL", fn);
+  REQUIRE(aligned16(a->dt) && aligned16(a->z) && aligned16(a->C) && aligned16(a->y) &&
+              aligned16(a->h_final) && aligned16(a->A) && aligned16(h_carry),
+          SSMQ_ERR_ALIGNMENT, "%s: tensors must be 16-byte aligned", fn);
+  if (injected(fn)) return fail(SSMQ_ERR_CUDA, "%s: injected launch failure", fn);
+  return finish(ssmq::launch_selective_scan_carry_in(*a, h_carry, (cudaStream_t)stream), fn);
 }
 
 int32_t ssmq_scan_time_segments(const ssmq_scan_args* a) {

@@ -37,6 +37,8 @@ cudaError_t launch_softedge_decode(const uint8_t* codes, int64_t n, float scale,
 // length in steps (whole 32-step chunks).
 int scan_time_segments(const ssmq_scan_args& a, int64_t* seg_len);
 cudaError_t launch_selective_scan(const ssmq_scan_args& a, cudaStream_t st);
+cudaError_t launch_selective_scan_carry_in(const ssmq_scan_args& a, const float* h_carry,
+                                           cudaStream_t st);
 cudaError_t launch_conv_silu_quantize(const ssmq_conv_args& a, cudaStream_t st);
 
 cudaError_t launch_state_update(const ssmq_decode_args& a, cudaStream_t st);

@@ -81,6 +81,13 @@ struct M1Params {
   int nseg;
   int64_t seg_len;
   float* seg_state;
+  // one-pass calls: the log2 decay of the call's steps per (b, c, n),
+  // A_cn log2(e) sum_t delta_t (for chaining sequence slices), or NULL
+  float* dec_final;
+  // carry-in kernel: the state carried into segment carry_from (NULL: segment
+  // 0's final state in seg_state); segments carry_from .. nseg - 1 corrected
+  const float* h_carry;
+  int carry_from;
 };
 
 // ---- cp.async (16-byte, L2-only) -------------------------------------------
@@ -338,6 +345,7 @@ __global__ void __launch_bounds__(kCH*(kN / kSPL)) m1_scan_kernel(const M1Params
   };
 
   constexpr int XB = SPS * (int)sizeof(XT);  // x bytes of a lane's run
+  float dsum = 0.0f;  // delta summed over this lane's staged steps (dec_final)
   auto stage_dd = [&](RawT& r, int s, int tl) {
     const int tb = s * kSeg + lj * SPS;
     uint32_t xw[(XB + 3) / 4], dw[(2 * SPS + 3) / 4];
@@ -359,6 +367,7 @@ __global__ void __launch_bounds__(kCH*(kN / kSPL)) m1_scan_kernel(const M1Params
       const float dv = h2f((uint16_t)(dw[i >> 1] >> (16 * (i & 1)))) + bias;
       float delta = p.softplus ? softplus_f(dv) : dv;
       if (!lvalid || tb + i >= tl) delta = 0.0f;
+      dsum += delta;
       S.dd[lc][tb + i] = make_float2(delta, delta * x_value(xw, i));
     }
   };
@@ -572,6 +581,16 @@ __global__ void __launch_bounds__(kCH*(kN / kSPL)) m1_scan_kernel(const M1Params
 #pragma unroll
     for (int i = 0; i < NP; ++i)
       *reinterpret_cast<float2*>(hout + (bb * d + lch) * kN + lj * kSPL + 2 * i) = hp[i];
+  if (p.dec_final) {
+    // the channel's delta total over its LPC lanes (consecutive lanes)
+#pragma unroll
+    for (int o = 1; o < LPC; o <<= 1) dsum += __shfl_xor_sync(0xffffffffu, dsum, o);
+    if (lvalid)
+#pragma unroll
+      for (int i = 0; i < NP; ++i)
+        *reinterpret_cast<float2*>(p.dec_final + (bb * d + lch) * kN + lj * kSPL + 2 * i) =
+            make_float2(ap[i].x * dsum, ap[i].y * dsum);
+  }
   flag_status(p.status, flags);
 }
 
@@ -612,10 +631,11 @@ __global__ void __launch_bounds__(32 * kCarryWarps) m1_carry_kernel(const M1Para
   float* Hs = sh_h[warp];
   for (int n = lane; n < kN; n += 32) {
     A2[n] = __ldg(p.A + c * kN + n) * kLog2e;
-    Hs[n] = p.seg_state[row * kN + n];  // segment 0's final state
+    // the state entering segment carry_from: given, or segment 0's final state
+    Hs[n] = p.h_carry ? __ldg(p.h_carry + row * kN + n) : p.seg_state[row * kN + n];
   }
   const int8_t* Crow = p.C + (bb * p.G + g) * kN * L;  // C of state n, step t: Crow[n L + t]
-  for (int seg = 1; seg < p.nseg; ++seg) {
+  for (int seg = p.carry_from; seg < p.nseg; ++seg) {
     const int64_t t_beg = (int64_t)seg * p.seg_len, t_end = min(L, t_beg + p.seg_len);
     __syncwarp();
     for (int n = lane; n < kN; n += 32) W[n] = __ldg(p.C_scale + g * spg + n / p.gs) * Hs[n];
@@ -648,12 +668,24 @@ __global__ void __launch_bounds__(32 * kCarryWarps) m1_carry_kernel(const M1Para
       }
     }
     __syncwarp();
-    const float* hl = p.seg_state + ((int64_t)seg * p.b * d + row) * kN;
-    for (int n = lane; n < kN; n += 32) Hs[n] = fmaf(ex2_sfu(A2[n] * s_run), Hs[n], hl[n]);
+    // the segment's local final state: its workspace slot, or, for a carry
+    // into a whole call, the h_final that call wrote
+    const float* hl = p.nseg > 1 ? p.seg_state + ((int64_t)seg * p.b * d + row) * kN
+                                 : (p.h_final ? p.h_final + row * kN : nullptr);
+    for (int n = lane; n < kN; n += 32)
+      Hs[n] = fmaf(ex2_sfu(A2[n] * s_run), Hs[n], hl ? hl[n] : 0.0f);
   }
   __syncwarp();
   if (p.h_final)
     for (int n = lane; n < kN; n += 32) p.h_final[row * kN + n] = Hs[n];
+}
+
+template <int kN>
+cudaError_t launch_carry(const M1Params& p, cudaStream_t st) {
+  const int64_t rows = p.b * p.d;
+  m1_carry_kernel<kN><<<(unsigned)((rows + kCarryWarps - 1) / kCarryWarps), 32 * kCarryWarps, 0,
+                        st>>>(p);
+  return cudaGetLastError();
 }
 
 template <int kN, int kCH, int kSPL>
@@ -682,10 +714,7 @@ cudaError_t launch_m1(const M1Params& prm, int xfmt, int64_t batch, cudaStream_t
   kern<<<grid, block, smem, st>>>(p);
   e = cudaGetLastError();
   if (e != cudaSuccess || p.nseg <= 1) return e;
-  const int64_t rows = p.b * p.d;
-  m1_carry_kernel<kN><<<(unsigned)((rows + kCarryWarps - 1) / kCarryWarps), 32 * kCarryWarps, 0,
-                        st>>>(p);
-  return cudaGetLastError();
+  return launch_carry<kN>(p, st);
 }
 
 }  // namespace
@@ -693,7 +722,9 @@ cudaError_t launch_m1(const M1Params& prm, int xfmt, int64_t batch, cudaStream_t
 int scan_time_segments(const ssmq_scan_args& a, int64_t* seg_len) {
   *seg_len = a.seqlen;
   int64_t k = a.time_segments;
-  if (k <= 1 || a.y == nullptr || a.y_q != nullptr || a.seqlen < 2 * kT) return 1;
+  if (k <= 1 || a.y == nullptr || a.y_q != nullptr || a.dec_final != nullptr ||
+      a.seqlen < 2 * kT)
+    return 1;
   const int64_t sl = ((a.seqlen + k - 1) / k + kT - 1) / kT * kT;  // whole chunks
   k = (a.seqlen + sl - 1) / sl;
   if (k <= 1 || a.batch * k > 65535) return 1;
@@ -701,11 +732,9 @@ int scan_time_segments(const ssmq_scan_args& a, int64_t* seg_len) {
   return (int)k;
 }
 
-cudaError_t launch_selective_scan(const ssmq_scan_args& a, cudaStream_t st) {
-  if (a.batch == 0 || a.dim == 0) return cudaSuccess;
+namespace {
+M1Params m1_params(const ssmq_scan_args& a) {
   M1Params p{};
-  p.nseg = scan_time_segments(a, &p.seg_len);
-  p.seg_state = static_cast<float*>(a.workspace);
   p.b = a.batch;
   p.L = a.seqlen;
   p.d = a.dim;
@@ -737,6 +766,17 @@ cudaError_t launch_selective_scan(const ssmq_scan_args& a, cudaStream_t st) {
   p.h_final = a.h_final;
   p.status = a.status;
   p.vec_ok = (a.seqlen % 16 == 0) ? 1 : 0;
+  p.dec_final = a.dec_final;
+  return p;
+}
+}  // namespace
+
+cudaError_t launch_selective_scan(const ssmq_scan_args& a, cudaStream_t st) {
+  if (a.batch == 0 || a.dim == 0) return cudaSuccess;
+  M1Params p = m1_params(a);
+  p.nseg = scan_time_segments(a, &p.seg_len);
+  p.seg_state = static_cast<float*>(a.workspace);
+  p.carry_from = 1;
   if (a.seqlen == 0) {
     // nothing to scan: the final state is the initial state
     if (a.h_final) {
@@ -744,6 +784,9 @@ cudaError_t launch_selective_scan(const ssmq_scan_args& a, cudaStream_t st) {
       return a.h0 ? cudaMemcpyAsync(a.h_final, a.h0, bytes, cudaMemcpyDeviceToDevice, st)
                   : cudaMemsetAsync(a.h_final, 0, bytes, st);
     }
+    if (a.dec_final)
+      return cudaMemsetAsync(a.dec_final, 0, sizeof(float) * (size_t)(a.batch * a.dim * a.dstate),
+                             st);
     return cudaSuccess;
   }
   switch (a.dstate) {
@@ -752,6 +795,35 @@ cudaError_t launch_selective_scan(const ssmq_scan_args& a, cudaStream_t st) {
     case 16: return launch_m1<16, 16, 4>(p, a.x_format, a.batch, st);
     case 32: return launch_m1<32, 16, 4>(p, a.x_format, a.batch, st);
     case 64: return launch_m1<64, 8, 4>(p, a.x_format, a.batch, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace ssmq
+
+namespace ssmq {
+
+cudaError_t launch_selective_scan_carry_in(const ssmq_scan_args& a, const float* h_carry,
+                                           cudaStream_t st) {
+  if (a.batch == 0 || a.dim == 0 || a.seqlen == 0) {
+    // no steps: the final state is the carried state
+    if (a.batch == 0 || a.dim == 0 || !a.h_final) return cudaSuccess;
+    return cudaMemcpyAsync(a.h_final, h_carry,
+                           sizeof(float) * (size_t)(a.batch * a.dim * a.dstate),
+                           cudaMemcpyDeviceToDevice, st);
+  }
+  M1Params p = m1_params(a);
+  p.nseg = 1;
+  p.seg_len = a.seqlen;
+  p.carry_from = 0;
+  p.h_carry = h_carry;
+  p.dec_final = nullptr;
+  switch (a.dstate) {
+    case 4: return launch_carry<4>(p, st);
+    case 8: return launch_carry<8>(p, st);
+    case 16: return launch_carry<16>(p, st);
+    case 32: return launch_carry<32>(p, st);
+    case 64: return launch_carry<64>(p, st);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -163,6 +163,20 @@ def test_scan_time_segments_validation(L):
     assert S(batch=0, **a) == N.OK
 
 
+def test_scan_carry_in_validation(L):
+    K = lambda h=FAKE, **kw: L.ssmq_selective_scan_carry_in(C.byref(_scan_args(**kw)), h, None)
+    assert K(h=None) == N.ERR_INVALID_ARG
+    assert K(dstate=12) == N.ERR_UNSUPPORTED
+    assert K(y=None) == N.ERR_INVALID_ARG
+    assert K(C_scale=None) == N.ERR_INVALID_ARG
+    assert K(h=FAKE + 4) == N.ERR_ALIGNMENT
+    assert K(batch=0, h=None) == N.OK
+    assert L.ssmq_selective_scan_carry_in(None, FAKE, None) == N.ERR_INVALID_ARG
+    # a call with log2 decays keeps one pass
+    assert L.ssmq_scan_time_segments(C.byref(_scan_args(time_segments=4, seqlen=2048,
+                                                        dec_final=FAKE))) == 1
+
+
 def _ssd_args(**kw):
     f = dict(batch=1, seqlen=512, nheads=8, headdim=64, dstate=128, ngroups=1, chunk=256,
              state_group_size=8, x_format=N.X_INT8_GROUP, x=FAKE, x_group=FAKE, x_scale=FAKE,

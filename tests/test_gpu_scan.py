@@ -203,6 +203,49 @@ def test_scan_time_segments_off_with_int8_y():
         np.testing.assert_array_equal(H(u), H(v))
 
 
+@pytest.mark.parametrize("cuts", [(0, 512), (0, 300, 301, 700)])
+def test_m1_sequence_sharded_vs_oracle(orc, cuts):
+    """Mamba-1 sequence sharding emulated in one process: each slice scanned
+    from a zero state (the first from h0) with its per-(channel, state) log2
+    decays, the summaries folded by the state-chain kernel, each later
+    slice's carried start state added by the carry-in kernel; the
+    concatenated y and the folded final state against the oracle's unsplit
+    scan."""
+    b, L, d, N_ = 2, 1000, 48, 16
+    p = m1_problem(470, b, L, d, N_, gate=True, h0=True, bias=True)
+    yo, ho = oracle_scan(orc, p)
+    bounds = list(cuts) + [L]
+    ys, h_ends, decs = [], [], []
+    for r in range(len(bounds) - 1):
+        sl = slice(bounds[r], bounds[r + 1])
+        q = dict(p)
+        for k in ("x", "dt", "z", "B", "C"):
+            q[k] = np.ascontiguousarray(p[k][..., sl])
+        args = (T(q["x"]), T(q["dt"]), T(q["A"]), T(q["B"]), T(q["C"]), T(q["B_scale"]),
+                T(q["C_scale"]), p["state_group_size"])
+        kw = dict(D=T(q["D"]), z=T(q["z"]), dt_bias=T(q["dt_bias"]))
+        dec = torch.empty((b, d, N_), dtype=torch.float32, device=dev())
+        y, he = api.selective_scan(*args, x_group=T(q["x_group"]), x_scale=T(q["x_scale"]),
+                                   h0=T(p["h0"]) if r == 0 else None, dec_final=dec, **kw)
+        # the log2 decays: A_cn log2(e) sum_t delta_t
+        dv = q["dt"].astype(np.float64) + q["dt_bias"].astype(np.float64)[None, :, None]
+        ref = (np.logaddexp(0.0, dv).sum(axis=2)[:, :, None] * q["A"].astype(np.float64)[None]
+               * np.log2(np.e))
+        np.testing.assert_allclose(H(dec), ref, rtol=2e-5, atol=1e-4)
+        if r > 0:
+            carry = api.state_chain(h_ends, decs)
+            he_true = he.clone()  # the chain below folds the slices' local states
+            api.selective_scan_carry_in(*args, carry, y, h_final=he_true, **kw)
+        ys.append(H(y).astype(np.float64))
+        h_ends.append(he)
+        decs.append(dec)
+    hf = H(api.state_chain(h_ends, decs))
+    # the last carry-in's h_final: the same state as the fold of every slice
+    np.testing.assert_allclose(H(he_true), hf, rtol=0, atol=1e-5 * np.abs(hf).max())
+    y = np.concatenate(ys, axis=-1)
+    assert_scan_close(y, yo.reshape(y.shape), hf, ho.reshape(hf.shape))
+
+
 # ---- full-size workloads, end to end from raw activations ------------------
 
 def _m1_end_to_end(orc, name, n_units=96, time_segments=1):

@@ -119,3 +119,60 @@ def test_sharded_call_rejects_unshared_arguments():
     with pytest.raises(TypeError, match="y_group"):
         sharded.ssd_chunk_scan_sequence_sharded(None, None, None, None, None, None, None, 8,
                                                 y_group=None)
+
+
+def test_m1_sharded_call_rejects_unshared_arguments():
+    """The Mamba-1 slice call takes the scan's x / gate / delta arguments; an
+    int8-y request or a time split has no sharded form."""
+    from quantized_state_space_b200 import sharded
+    for bad in ("y_group", "time_segments"):
+        with pytest.raises(TypeError, match=bad):
+            sharded.selective_scan_sequence_sharded(None, None, None, None, None, None, None, 4,
+                                                    **{bad: None})
+
+
+def _m1_fold(h_ends, decs):
+    h = np.zeros_like(h_ends[0])
+    for he, d in zip(h_ends, decs):
+        h = np.exp2(d) * h + he
+    return h
+
+
+@pytest.mark.parametrize("cuts", [(0, 100, 250), (0, 1, 2, 180)])
+def test_m1_slices_fold_to_the_unsplit_scan(orc, cuts):
+    """Mamba-1: slices scanned from zero (the first from h0), folded with
+    h <- exp2(dec) h + h_end, dec = A_cn log2(e) sum_t delta_t per (b, c, n),
+    give the unsplit final state; each slice's y plus the y of its carried
+    start state is the unsplit y."""
+    from problems import m1_problem
+    b, L, d, N_ = 2, 300, 16, 8
+    p = m1_problem(935, b, L, d, N_, gate=True, h0=True, bias=True)
+    sc = lambda q, **kw: orc.m1_scan(q["x"], q["dt"], q["A"], q["B"], q["C"], q["B_scale"],
+                                     q["C_scale"], q["state_group_size"], **kw)
+    yo, ho = sc(p, **oracle_kwargs(p))
+    bounds = list(cuts) + [L]
+    h_ends, decs = [], []
+    for r in range(len(bounds) - 1):
+        sl = slice(bounds[r], bounds[r + 1])
+        q = dict(p)
+        for k in ("x", "dt", "z", "B", "C"):
+            q[k] = np.ascontiguousarray(p[k][..., sl])
+        if r > 0:
+            q["h0"] = None
+        kw = oracle_kwargs(q)
+        y0, he = sc(q, **kw)
+        if r > 0:
+            carry = _m1_fold(h_ends, decs)
+            kw["h0"] = carry.astype(np.float32).astype(np.float64)
+            y1, _ = sc(q, **kw)
+            kw["h0"] = np.zeros_like(kw["h0"])
+            y0z, _ = sc(q, **kw)
+            y0 = y0 + (y1 - y0z)
+        np.testing.assert_allclose(y0.reshape(b, d, -1), yo.reshape(b, d, L)[..., sl], rtol=0,
+                                   atol=2e-6 * np.abs(yo).max())
+        h_ends.append(he.reshape(b, d, N_))
+        dv = q["dt"].astype(np.float64) + p["dt_bias"].astype(np.float64)[None, :, None]
+        decs.append(np.logaddexp(0.0, dv).sum(axis=2)[:, :, None]
+                    * p["A"].astype(np.float64)[None] * np.log2(np.e))
+    hf = _m1_fold(h_ends, decs)
+    np.testing.assert_allclose(hf, ho.reshape(hf.shape), rtol=0, atol=1e-9 * np.abs(ho).max())
