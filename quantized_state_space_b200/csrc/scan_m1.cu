@@ -219,7 +219,9 @@ __device__ __forceinline__ void fetch_chunk(const M1Params& p, Raw<kN, kCH, XT>&
   }
 }
 
-template <int kN, int kCH, int kSPL, int kXFmt, bool kYQ>
+// kSplit: the call has time segments or asks for dec_final (a separate
+// instantiation keeps the one-pass kernel's code as it was)
+template <int kN, int kCH, int kSPL, int kXFmt, bool kYQ, bool kSplit>
 __global__ void __launch_bounds__(kCH*(kN / kSPL)) m1_scan_kernel(const M1Params p) {
   static_assert(kSPL == 2 || kSPL == 4, "2 or 4 states per thread");
   constexpr bool kXF16 = kXFmt == SSMQ_X_F16_GROUP || kXFmt == SSMQ_X_F16_SOFTEDGE;
@@ -236,10 +238,11 @@ __global__ void __launch_bounds__(kCH*(kN / kSPL)) m1_scan_kernel(const M1Params
   M1Smem<kN, kCH, PR, XT>& S = *reinterpret_cast<M1Smem<kN, kCH, PR, XT>*>(smem_bytes);
 
   const int tid = threadIdx.x;
-  const int64_t bb = blockIdx.y / p.nseg;
-  const int seg = (int)(blockIdx.y % p.nseg);
+  const int64_t bb = kSplit ? blockIdx.y / p.nseg : blockIdx.y;
+  const int seg = kSplit ? (int)(blockIdx.y % p.nseg) : 0;
   const int64_t d = p.d, L = p.L;
-  const int64_t t_beg = (int64_t)seg * p.seg_len, t_end = min(L, t_beg + p.seg_len);
+  const int64_t t_beg = kSplit ? (int64_t)seg * p.seg_len : 0;
+  const int64_t t_end = kSplit ? min(L, t_beg + p.seg_len) : L;
   const int dg = (int)(d / p.G);
   const int g = blockIdx.x / p.n_ctile;
   const int c0 = g * dg + (blockIdx.x % p.n_ctile) * kCH;
@@ -367,7 +370,7 @@ __global__ void __launch_bounds__(kCH*(kN / kSPL)) m1_scan_kernel(const M1Params
       const float dv = h2f((uint16_t)(dw[i >> 1] >> (16 * (i & 1)))) + bias;
       float delta = p.softplus ? softplus_f(dv) : dv;
       if (!lvalid || tb + i >= tl) delta = 0.0f;
-      dsum += delta;
+      if constexpr (kSplit) dsum += delta;
       S.dd[lc][tb + i] = make_float2(delta, delta * x_value(xw, i));
     }
   };
@@ -576,12 +579,12 @@ __global__ void __launch_bounds__(kCH*(kN / kSPL)) m1_scan_kernel(const M1Params
     }
   }
 
-  float* hout = p.nseg > 1 ? p.seg_state + (int64_t)seg * p.b * d * kN : p.h_final;
+  float* hout = kSplit && p.nseg > 1 ? p.seg_state + (int64_t)seg * p.b * d * kN : p.h_final;
   if (lvalid && hout)
 #pragma unroll
     for (int i = 0; i < NP; ++i)
       *reinterpret_cast<float2*>(hout + (bb * d + lch) * kN + lj * kSPL + 2 * i) = hp[i];
-  if (p.dec_final) {
+  if (kSplit && p.dec_final) {
     // the channel's delta total over its LPC lanes (consecutive lanes)
 #pragma unroll
     for (int o = 1; o < LPC; o <<= 1) dsum += __shfl_xor_sync(0xffffffffu, dsum, o);
@@ -701,14 +704,19 @@ cudaError_t launch_m1(const M1Params& prm, int xfmt, int64_t batch, cudaStream_t
       xfmt == SSMQ_X_F16_GROUP
           ? sizeof(M1Smem<kN, kCH, part_rows(SSMQ_X_F16_GROUP, LPC), uint16_t>)
           : (f16 ? sizeof(M1Smem<kN, kCH, 1, uint16_t>) : sizeof(M1Smem<kN, kCH, 1, uint8_t>));
-  auto pick = [&](auto yq) {
-    constexpr bool Q = decltype(yq)::value;
-    return xfmt == SSMQ_X_SOFTEDGE       ? m1_scan_kernel<kN, kCH, kSPL, SSMQ_X_SOFTEDGE, Q>
-           : xfmt == SSMQ_X_F16_GROUP    ? m1_scan_kernel<kN, kCH, kSPL, SSMQ_X_F16_GROUP, Q>
-           : xfmt == SSMQ_X_F16_SOFTEDGE ? m1_scan_kernel<kN, kCH, kSPL, SSMQ_X_F16_SOFTEDGE, Q>
-                                         : m1_scan_kernel<kN, kCH, kSPL, SSMQ_X_INT8_GROUP, Q>;
+  auto pick = [&](auto yq, auto split) {
+    constexpr bool Q = decltype(yq)::value, S = decltype(split)::value;
+    return xfmt == SSMQ_X_SOFTEDGE       ? m1_scan_kernel<kN, kCH, kSPL, SSMQ_X_SOFTEDGE, Q, S>
+           : xfmt == SSMQ_X_F16_GROUP    ? m1_scan_kernel<kN, kCH, kSPL, SSMQ_X_F16_GROUP, Q, S>
+           : xfmt == SSMQ_X_F16_SOFTEDGE ? m1_scan_kernel<kN, kCH, kSPL, SSMQ_X_F16_SOFTEDGE, Q, S>
+                                         : m1_scan_kernel<kN, kCH, kSPL, SSMQ_X_INT8_GROUP, Q, S>;
   };
-  auto kern = p.y_q ? pick(std::true_type{}) : pick(std::false_type{});
+  // time segments need binary16 y without y_q; dec_final may come with y_q
+  const bool split = p.nseg > 1 || p.dec_final != nullptr;
+  auto kern = p.y_q ? (split ? pick(std::true_type{}, std::true_type{})
+                             : pick(std::true_type{}, std::false_type{}))
+                    : (split ? pick(std::false_type{}, std::true_type{})
+                             : pick(std::false_type{}, std::false_type{}));
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   kern<<<grid, block, smem, st>>>(p);
