@@ -218,13 +218,18 @@ def ssmq_softedge_decode(codes, n, scale, log2_ratio, out, stream=None):
                                       _stream(stream)))
 
 
+_FIELD_TYPES = {}
+
+
 def _fill(struct_cls, fields):
+    types = _FIELD_TYPES.get(struct_cls)
+    if types is None:
+        types = _FIELD_TYPES[struct_cls] = dict(struct_cls._fields_)
     a = struct_cls()
-    names = {f[0] for f in struct_cls._fields_}
     for k, v in fields.items():
-        if k not in names:
+        ftype = types.get(k)
+        if ftype is None:
             raise TypeError("unknown field %r for %s" % (k, struct_cls.__name__))
-        ftype = dict(struct_cls._fields_)[k]
         setattr(a, k, ptr(v) if ftype is _vp else v)
     return a
 

@@ -253,7 +253,8 @@ def selective_scan(x, dt, A, B, C, B_scale, C_scale, state_group_size, *, x_grou
                       B=B, C=C, B_scale=B_scale, C_scale=C_scale, h0=h0, y=y, h_final=h_final,
                       status=status, time_segments=int(time_segments), dec_final=dec_final,
                       **yf)
-        ws = N.ssmq_scan_workspace_size(**fields)
+        # (one pass needs no workspace: no size query on that path)
+        ws = N.ssmq_scan_workspace_size(**fields) if int(time_segments) > 1 else 0
         _workspace(workspace, ws, dv)
         if ws and workspace is None:
             workspace = torch.empty(ws + 256, dtype=torch.uint8, device=dv)
