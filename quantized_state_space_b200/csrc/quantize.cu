@@ -287,13 +287,55 @@ __global__ void __launch_bounds__(stream::kThreads)
       cur_m = max(cur_m, a);
     }
   };
+  auto one = [&](float v, Idx e) { push(__ldg(gmap + geo.mid_of(e)), v); };
+  if constexpr (kPath == kPathRow && kF16) {
+    // a vector's 16 elements share one group: the largest magnitude pattern
+    // of the vector by packed 16-bit maxima (for non-negative binary16 the
+    // pattern order is the value order); a vector holding a non-finite
+    // element (exponent bits all ones, found per pair as in the encoder)
+    // takes the per-element definition
+    auto vec = [&](const uint32_t(&w)[8], Idx e0) {
+      const int g = __ldg(gmap + geo.mid_of(e0));
+      uint32_t m = 0u, nf = 0u;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        nf |= (w[i] & 0x7C007C00u) + 0x04000400u;
+        m = __vmaxu2(m, w[i] & 0x7FFF7FFFu);
+      }
+      if (nf & 0x80008000u) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          push(g, h2f((uint16_t)(w[i] & 0xFFFFu)));
+          push(g, h2f((uint16_t)(w[i] >> 16)));
+        }
+        return;
+      }
+      push(g, h2f((uint16_t)max(m & 0xFFFFu, m >> 16)));
+    };
+    stream::run_part<true, Idx, decltype(vec)&, decltype(one)&, stream::NoPrologue, true>(
+        src, n, smem, (Idx)blockIdx.x, (Idx)gridDim.x, vec, one, flags);
+  } else {
   stream::run<kF16, Idx>(
       src, n, smem,
       [&](const float(&x)[kVec], Idx e0) {
         if (kPath == kPathRow) {
+          // binary32: the largest magnitude bit pattern of the vector, or the
+          // per-element definition when an element is not finite
           const int g = __ldg(gmap + geo.mid_of(e0));
+          uint32_t m = 0u;
+          bool nfv = false;
 #pragma unroll
-          for (int i = 0; i < kVec; ++i) push(g, x[i]);
+          for (int i = 0; i < kVec; ++i) {
+            const uint32_t a = __float_as_uint(x[i]) & 0x7FFFFFFFu;
+            nfv |= a >= 0x7F800000u;
+            m = max(m, a);
+          }
+          if (nfv) {
+#pragma unroll
+            for (int i = 0; i < kVec; ++i) push(g, x[i]);
+          } else {
+            push(g, __uint_as_float(m));
+          }
         } else if (kPath == kPathCol) {
           const Idx m0 = geo.col_of(e0);
 #pragma unroll
@@ -303,7 +345,8 @@ __global__ void __launch_bounds__(stream::kThreads)
           for (int i = 0; i < kVec; ++i) push(__ldg(gmap + geo.mid_of(e0 + i)), x[i]);
         }
       },
-      [&](float v, Idx e) { push(__ldg(gmap + geo.mid_of(e)), v); }, flags);
+      one, flags);
+  }
   if (cur_g >= 0 && cur_m) atomicMax(tgt + cur_g, cur_m);
   if (use_smem) {
     __syncthreads();
