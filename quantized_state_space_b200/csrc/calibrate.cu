@@ -117,7 +117,31 @@ __global__ void __launch_bounds__(kHistThreads)
   const int nt = 2 * ws->ctrl.nq;
   __syncthreads();
   const int64_t stride = (int64_t)gridDim.x * kHistThreads;
-  for (int64_t i = (int64_t)blockIdx.x * kHistThreads + threadIdx.x; i < n; i += stride) {
+  int64_t i0 = 0;  // first element of the scalar loop below
+  if (kLevel == 0 && (reinterpret_cast<uintptr_t>(src) & 15u) == 0) {
+    // 16-byte loads (8 binary16 or 4 binary32 elements), then one shared
+    // atomic per finite element; the scalar loop takes the remainder
+    constexpr int kPer = kF16 ? 8 : 4;
+    const int64_t nv = n / kPer;
+    const uint4* v4 = static_cast<const uint4*>(src);
+    for (int64_t v = (int64_t)blockIdx.x * kHistThreads + threadIdx.x; v < nv; v += stride) {
+      const uint4 q = __ldg(v4 + v);
+      const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        if (kF16) {
+          const uint32_t lo = w[k] & 0x7FFFu, hi = (w[k] >> 16) & 0x7FFFu;
+          if (lo < 0x7C00u) atomicAdd(&sh[lo], 1u);
+          if (hi < 0x7C00u) atomicAdd(&sh[hi], 1u);
+        } else {
+          const uint32_t m = w[k] & 0x7FFFFFFFu;
+          if (m < 0x7F800000u) atomicAdd(&sh[m >> 16], 1u);
+        }
+      }
+    }
+    i0 = nv * kPer;
+  }
+  for (int64_t i = i0 + (int64_t)blockIdx.x * kHistThreads + threadIdx.x; i < n; i += stride) {
     bool fin;
     const uint32_t m = mag_bits<kF16>(src, i, fin);
     if (!fin) continue;
