@@ -644,12 +644,33 @@ __global__ void __launch_bounds__(32 * kCarryWarps) m1_carry_kernel(const M1Para
     for (int n = lane; n < kN; n += 32) W[n] = __ldg(p.C_scale + g * spg + n / p.gs) * Hs[n];
     __syncwarp();
     float s_run = 0.0f;  // delta summed over the segment's earlier blocks
+    // the block's operands are loaded one block ahead (the walk over the
+    // blocks is sequential only through s_run)
+    constexpr int kPC = kN <= 16 ? kN : 1;  // C codes held ahead (small N)
+    uint16_t dt_n = 0, z_n = 0, y_n = 0;
+    int8_t c_n[kPC];
+    auto load = [&](int64_t t0) {
+      const int64_t t = t0 + lane;
+      if (t < t_end) {
+        dt_n = p.dt[row * L + t];
+        z_n = p.z ? p.z[row * L + t] : (uint16_t)0;
+        y_n = p.y[row * L + t];
+#pragma unroll
+        for (int n = 0; n < kPC; ++n) c_n[n] = Crow[n * L + t];
+      }
+    };
+    load(t_beg);
     for (int64_t t0 = t_beg; t0 < t_end; t0 += 32) {
       const int64_t t = t0 + lane;
       const bool ok = t < t_end;
+      const uint16_t dt_c = dt_n, z_c = z_n, y_c = y_n;
+      int8_t c_c[kPC];
+#pragma unroll
+      for (int n = 0; n < kPC; ++n) c_c[n] = c_n[n];
+      if (t0 + 32 < t_end) load(t0 + 32);
       float delta = 0.0f;
       if (ok) {
-        const float dv = h2f(p.dt[row * L + t]) + bias;
+        const float dv = h2f(dt_c) + bias;
         delta = p.softplus ? softplus_f(dv) : dv;
       }
       float sc = delta;
@@ -664,10 +685,10 @@ __global__ void __launch_bounds__(32 * kCarryWarps) m1_carry_kernel(const M1Para
         float corr = 0.0f;
 #pragma unroll
         for (int n = 0; n < kN; ++n)
-          corr = fmaf(s8f(Crow[n * L + t]) * W[n], ex2_sfu(A2[n] * S), corr);
-        const float gate = p.z ? silu_f(h2f(p.z[row * L + t])) : 1.0f;
-        uint16_t* yp = p.y + row * L + t;
-        *yp = f2h(fmaf(corr, gate, h2f(*yp)));
+          corr = fmaf(s8f(kN <= 16 ? c_c[n < kPC ? n : 0] : Crow[n * L + t]) * W[n],
+                      ex2_sfu(A2[n] * S), corr);
+        const float gate = p.z ? silu_f(h2f(z_c)) : 1.0f;
+        p.y[row * L + t] = f2h(fmaf(corr, gate, h2f(y_c)));
       }
     }
     __syncwarp();
