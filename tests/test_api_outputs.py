@@ -19,6 +19,8 @@ class _Recorder:
             return lambda **kw: 4096
         if name == "ssmq_percentile_workspace_size":
             return lambda: 1024
+        if name == "ssmq_scan_workspace_size":
+            return lambda **kw: 512 if kw.get("time_segments", 1) > 1 else 0
         if name.startswith("ssmq_"):
             return lambda *a, **kw: self.calls.append(name)
         return getattr(real_native, name)
@@ -213,3 +215,34 @@ def test_noalloc_wrappers(rec):
     _bad(lambda: api.softedge_calibrate_noalloc(src, E(2)))
     _bad(lambda: api.softedge_calibrate_noalloc(src, E(3, device="meta")))
     assert rec.calls == ["ssmq_percentile_abs_noalloc", "ssmq_softedge_calibrate_noalloc"]
+
+
+def test_scan_time_segments_and_carry_in_checks(rec):
+    """Time segments: the workspace is sized by the library's query only for
+    a split call and checked when supplied; dec_final and the carry-in's
+    tensors are checked like every other tensor."""
+    b, d, L, G, N = 2, 8, 64, 1, 16
+    x, dt = E(b, d, L, dtype=torch.int8), E(b, d, L, dtype=torch.float16)
+    Bq = E(b, G, N, L, dtype=torch.int8)
+    args = (x, dt, E(d, N), Bq, Bq, E(4), E(4), 4)
+    kw = dict(x_group=E(d, dtype=torch.int32), x_scale=E(2))
+    api.selective_scan(*args, time_segments=2, **kw)
+    api.selective_scan(*args, time_segments=2, workspace=E(512 + 255, dtype=torch.uint8), **kw)
+    _bad(lambda: api.selective_scan(*args, time_segments=2,
+                                    workspace=E(512, dtype=torch.uint8), **kw))
+    _bad(lambda: api.selective_scan(*args, time_segments=2,
+                                    workspace=E(1024, dtype=torch.int8), **kw))
+    api.selective_scan(*args, dec_final=E(b, d, N), **kw)
+    _bad(lambda: api.selective_scan(*args, dec_final=E(b, d), **kw))
+    _bad(lambda: api.selective_scan(*args, dec_final=E(b, d, N, dtype=torch.float16), **kw))
+    y = E(b, d, L, dtype=torch.float16)
+    carry = lambda **k: api.selective_scan_carry_in(*args, k.pop("h", E(b, d, N)),
+                                                    k.pop("y", y), **k)
+    carry()
+    carry(h_final=E(b, d, N), D=E(d), z=E(b, d, L, dtype=torch.float16), dt_bias=E(d))
+    _bad(lambda: carry(h=E(b, d, N - 1)))
+    _bad(lambda: carry(y=E(b, d, L)))
+    _bad(lambda: carry(h_final=E(b, d)))
+    _bad(lambda: carry(z=E(b, d, L - 1, dtype=torch.float16)))
+    assert rec.calls.count("ssmq_selective_scan_carry_in") == 2
+    assert rec.calls.count("ssmq_selective_scan_w8") == 3
