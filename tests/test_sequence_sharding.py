@@ -176,3 +176,94 @@ def test_m1_slices_fold_to_the_unsplit_scan(orc, cuts):
                     * p["A"].astype(np.float64)[None] * np.log2(np.e))
     hf = _m1_fold(h_ends, decs)
     np.testing.assert_allclose(hf, ho.reshape(hf.shape), rtol=0, atol=1e-9 * np.abs(ho).max())
+
+
+class _OracleKernels:
+    """Stand-ins for the library calls of the Mamba-1 sharded path, computed
+    by the oracle in float64 on the host (the orchestration under test is the
+    rank logic: who starts from h0, which summaries are folded, where the
+    carry-in goes)."""
+
+    def __init__(self, O, gs, kw):
+        self.O, self.gs, self.kw = O, gs, kw
+
+    def _scan(self, x, dt, A, B, C, Bs, Cs, h0):
+        kw = dict(self.kw)
+        kw["h0"] = None if h0 is None else h0.numpy().astype(np.float64)
+        y, h = self.O.m1_scan(x.numpy(), dt.numpy(), A.numpy(), B.numpy(), C.numpy(),
+                              Bs.numpy(), Cs.numpy(), self.gs, **kw)
+        b, d, L = x.shape
+        return torch.from_numpy(y.reshape(b, d, L)), torch.from_numpy(h.reshape(b, d, -1))
+
+    def selective_scan(self, x, dt, A, B, C, Bs, Cs, gs, h0=None, dec_final=None, **_):
+        y, h = self._scan(x, dt, A, B, C, Bs, Cs, h0)
+        dv = dt.numpy().astype(np.float64) + self.kw["dt_bias"][None, :, None]
+        dec = (np.logaddexp(0.0, dv).sum(axis=2)[:, :, None] * A.numpy().astype(np.float64)[None]
+               * np.log2(np.e))
+        dec_final.copy_(torch.from_numpy(dec))
+        return y, h
+
+    @staticmethod
+    def state_chain(hs, ds):
+        h = torch.zeros_like(hs[0])
+        for he, d in zip(hs, ds):
+            h = torch.exp2(d) * h + he
+        return h
+
+    def selective_scan_carry_in(self, x, dt, A, B, C, Bs, Cs, gs, h_carry, y, **_):
+        y1, _ = self._scan(x, dt, A, B, C, Bs, Cs, h_carry)
+        y0, _ = self._scan(x, dt, A, B, C, Bs, Cs, None)
+        y += y1 - y0
+
+
+def _m1_sharded_worker(rank, world, port, out, cuts):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=__import__("datetime").timedelta(seconds=60))
+    try:
+        from oracle import oracle as O
+        from problems import m1_problem
+        from quantized_state_space_b200 import sharded
+        p = m1_problem(960, 2, 200, 8, 8, gate=True, h0=True, bias=True)
+        kw = dict(D=p["D"], z=None, dt_bias=p["dt_bias"], x_group=p["x_group"],
+                  x_scale=p["x_scale"])
+        sl = slice(cuts[rank], cuts[rank + 1])
+        q = {k: (np.ascontiguousarray(p[k][..., sl]) if k in ("x", "dt", "z", "B", "C") else p[k])
+             for k in p}
+        kw["z"] = q["z"].astype(np.float64)
+        sharded.api = _OracleKernels(O, p["state_group_size"], kw)
+        T = lambda a: torch.from_numpy(np.ascontiguousarray(a))
+        y, hf = sharded.selective_scan_sequence_sharded(
+            T(q["x"]), T(q["dt"]), T(q["A"]), T(q["B"]), T(q["C"]), T(q["B_scale"]),
+            T(q["C_scale"]), p["state_group_size"], h0=T(p["h0"]))
+        out[rank] = (y.numpy(), hf.numpy())
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("cuts", [(0, 90, 200), (0, 50, 51, 200)])
+def test_m1_sharded_orchestration_over_gloo_ranks(orc, cuts):
+    """The Mamba-1 sequence-sharded call on 2 and 3 gloo ranks, the library
+    calls stood in for by the oracle: the slices' y concatenated and every
+    rank's final state against the oracle's unsplit scan."""
+    world = len(cuts) - 1
+    port = _free_port()
+    ctx = mp.get_context("spawn")
+    with ctx.Manager() as m:
+        out = m.dict()
+        mp.start_processes(_m1_sharded_worker, args=(world, port, out, cuts), nprocs=world,
+                           join=True, start_method="spawn")
+        res = dict(out)
+    from problems import m1_problem
+    p = m1_problem(960, 2, 200, 8, 8, gate=True, h0=True, bias=True)
+    kw = oracle_kwargs(p)
+    yo, ho = orc.m1_scan(p["x"], p["dt"], p["A"], p["B"], p["C"], p["B_scale"], p["C_scale"],
+                         p["state_group_size"], **kw)
+    # the exchanged log2 decays are fp32 (as the library's): 1e-6 of the
+    # largest value; a wrong start state or fold order is off by O(1)
+    y = np.concatenate([res[r][0] for r in range(world)], axis=-1)
+    np.testing.assert_allclose(y, yo.reshape(y.shape), rtol=0, atol=1e-6 * np.abs(yo).max())
+    for r in range(world):
+        np.testing.assert_allclose(res[r][1], ho.reshape(res[r][1].shape), rtol=0,
+                                   atol=1e-6 * np.abs(ho).max())
