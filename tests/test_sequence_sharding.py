@@ -267,3 +267,87 @@ def test_m1_sharded_orchestration_over_gloo_ranks(orc, cuts):
     for r in range(world):
         np.testing.assert_allclose(res[r][1], ho.reshape(res[r][1].shape), rtol=0,
                                    atol=1e-6 * np.abs(ho).max())
+
+
+class _OracleSsdKernels:
+    """The SSD sharded path's library calls, stood in for by the oracle."""
+
+    def __init__(self, O, gs, kw):
+        self.O, self.gs, self.kw = O, gs, kw
+
+    def _scan(self, x, dt, A, B, C, Bs, Cs, h0):
+        kw = dict(self.kw)
+        kw["h0"] = None if h0 is None else h0.numpy().astype(np.float64)
+        y, h = self.O.ssd_scan(x.numpy(), dt.numpy(), A.numpy(), B.numpy(), C.numpy(),
+                               Bs.numpy(), Cs.numpy(), self.gs, **kw)
+        b, L, H, P = x.shape  # the oracle's y is (b H, L, P)
+        y = np.ascontiguousarray(y.reshape(b, H, L, P).transpose(0, 2, 1, 3))
+        return torch.from_numpy(y), torch.from_numpy(h.reshape(b, H, P, -1))
+
+    def ssd_chunk_scan(self, x, dt, A, B, C, Bs, Cs, gs, h0=None, dec_final=None, **_):
+        y, h = self._scan(x, dt, A, B, C, Bs, Cs, h0)
+        dv = dt.numpy().astype(np.float64) + self.kw["dt_bias"][None, None, :]
+        dec = np.logaddexp(0.0, dv).sum(axis=1) * A.numpy().astype(np.float64) * np.log2(np.e)
+        dec_final.copy_(torch.from_numpy(dec))
+        return y, h
+
+    state_chain = staticmethod(lambda hs, ds: _fold_t(hs, ds))
+
+    def ssd_carry_in(self, x, dt, A, B, C, Bs, Cs, gs, h_carry, y, **_):
+        y1, _ = self._scan(x, dt, A, B, C, Bs, Cs, h_carry)
+        y0, _ = self._scan(x, dt, A, B, C, Bs, Cs, None)
+        y += y1 - y0
+
+
+def _fold_t(hs, ds):
+    h = torch.zeros_like(hs[0])
+    for he, d in zip(hs, ds):
+        h = torch.exp2(d).reshape(d.shape + (1,) * (he.dim() - d.dim())) * h + he
+    return h
+
+
+def _ssd_sharded_worker(rank, world, port, out, cuts):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=__import__("datetime").timedelta(seconds=60))
+    try:
+        from oracle import oracle as O
+        from quantized_state_space_b200 import sharded
+        p = ssd_problem(965, 1, 300, 2, 64, 128, gate=False, h0=True, bias=True)
+        kw = oracle_kwargs(p)
+        kw.pop("h0")
+        sl = slice(cuts[rank], cuts[rank + 1])
+        q = {k: (np.ascontiguousarray(p[k][:, sl]) if k in ("x", "dt", "B", "C") else p[k])
+             for k in p}
+        sharded.api = _OracleSsdKernels(O, 8, kw)
+        T = lambda a: torch.from_numpy(np.ascontiguousarray(a))
+        y, hf = sharded.ssd_chunk_scan_sequence_sharded(
+            T(q["x"]), T(q["dt"]), T(q["A"]), T(q["B"]), T(q["C"]), T(q["B_scale"]),
+            T(q["C_scale"]), 8, h0=T(p["h0"]))
+        out[rank] = (y.numpy(), hf.numpy())
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_ssd_sharded_orchestration_over_gloo_ranks(orc):
+    """The SSD sequence-sharded call on 3 gloo ranks, the library calls stood
+    in for by the oracle, against the oracle's unsplit scan."""
+    cuts = (0, 77, 201, 300)
+    world = len(cuts) - 1
+    port = _free_port()
+    ctx = mp.get_context("spawn")
+    with ctx.Manager() as m:
+        out = m.dict()
+        mp.start_processes(_ssd_sharded_worker, args=(world, port, out, cuts), nprocs=world,
+                           join=True, start_method="spawn")
+        res = dict(out)
+    p = ssd_problem(965, 1, 300, 2, 64, 128, gate=False, h0=True, bias=True)
+    yo, ho = orc.ssd_scan(p["x"], p["dt"], p["A"], p["B"], p["C"], p["B_scale"], p["C_scale"],
+                          8, **oracle_kwargs(p))
+    y = np.concatenate([res[r][0] for r in range(world)], axis=1)
+    yo = yo.reshape(1, 2, 300, 64).transpose(0, 2, 1, 3)  # (b H, L, P) -> (b, L, H, P)
+    np.testing.assert_allclose(y, yo, rtol=0, atol=1e-6 * np.abs(yo).max())
+    for r in range(world):
+        np.testing.assert_allclose(res[r][1], ho.reshape(res[r][1].shape), rtol=0,
+                                   atol=1e-6 * np.abs(ho).max())
